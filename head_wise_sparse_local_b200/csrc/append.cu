@@ -1,0 +1,123 @@
+// rtp_append_kv: RoPE'd key, value and 16-d pre-RoPE indexer key per token.
+//
+// One warp per (sequence, token, KV head) row.  Lane l owns the RoPE pairs
+// (k, k + D/2) for k in [l*PP, (l+1)*PP), PP = D/64, so the rotation needs no
+// shuffle.  Retrieval heads also project the pre-RoPE key through W_k^(r)
+// ("pre-RoPE low-dimensional projection", atlas.scime.ai summary, "Approach"):
+// each lane forms partial dot products over its dims and a butterfly reduction
+// gives every lane the same 16 sums.
+#include "common.cuh"
+#include "internal.h"
+
+namespace rtp {
+namespace {
+
+struct AppendArgs {
+  int B, T, Hkv, D, Lmax, R;
+  float rope_base;
+  const void* k_pre;
+  const void* v_in;
+  const int* start_pos;
+  const float* w_k;
+  void* k;
+  void* v;
+  void* kidx;
+  int* status;
+  int ret_rank[kMaxRetrieval];
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
+  constexpr int PP = D / 64;  // pairs per lane
+  constexpr int H = D / 2;
+  const int lane = threadIdx.x & 31;
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const long long n_rows = (long long)a.B * a.T * a.Hkv;
+  if (row >= n_rows) return;
+  const int h = int(row % a.Hkv);
+  const int t = int((row / a.Hkv) % a.T);
+  const int b = int(row / ((long long)a.Hkv * a.T));
+  const int pos = a.start_pos[b] + t;
+  if (pos < 0 || pos >= a.Lmax) {
+    if (lane == 0) atomicOr(a.status, RTP_DEV_POSITION);
+    return;
+  }
+  const T* kp = static_cast<const T*>(a.k_pre) + row * D;
+  const T* vp = static_cast<const T*>(a.v_in) + row * D;
+  const size_t dst = (((size_t)b * a.Hkv + h) * a.Lmax + pos) * D;
+  T* ko = static_cast<T*>(a.k) + dst;
+  T* vo = static_cast<T*>(a.v) + dst;
+
+  float x1[PP], x2[PP];
+#pragma unroll
+  for (int i = 0; i < PP; ++i) {
+    const int k = lane * PP + i;
+    x1[i] = to_f32(kp[k]);
+    x2[i] = to_f32(kp[k + H]);
+    vo[k] = vp[k];
+    vo[k + H] = vp[k + H];
+  }
+#pragma unroll
+  for (int i = 0; i < PP; ++i) {
+    const int k = lane * PP + i;
+    float c, s;
+    rope_cos_sin(pos, k, D, a.rope_base, c, s);
+    ko[k] = from_f32<T>(x1[i] * c - x2[i] * s);
+    ko[k + H] = from_f32<T>(x2[i] * c + x1[i] * s);
+  }
+
+  const int r = a.ret_rank[h];
+  if (r < 0) return;
+  const float* w = a.w_k + (size_t)r * kIdxDim * D;
+  float acc[kIdxDim];
+#pragma unroll
+  for (int i = 0; i < kIdxDim; ++i) {
+    float sacc = 0.f;
+#pragma unroll
+    for (int p = 0; p < PP; ++p) {
+      const int k = lane * PP + p;
+      sacc = fmaf(__ldg(w + i * D + k), x1[p], sacc);
+      sacc = fmaf(__ldg(w + i * D + k + H), x2[p], sacc);
+    }
+    acc[i] = sacc;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+    for (int i = 0; i < kIdxDim; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+  }
+  T* ki = static_cast<T*>(a.kidx) + (((size_t)b * a.R + r) * a.Lmax + pos) * kIdxDim;
+#pragma unroll
+  for (int i = 0; i < kIdxDim; ++i)
+    if (lane == i) ki[i] = from_f32<T>(acc[i]);
+}
+
+}  // namespace
+
+int launch_append(const Shape& sh, const rtp_cache* cache, const void* k_pre, const void* v_in,
+                  const int* start_pos, int T, const float* w_k, cudaStream_t st) {
+  AppendArgs a;
+  a.B = sh.B; a.T = T; a.Hkv = sh.Hkv; a.D = sh.D; a.Lmax = sh.Lmax; a.R = sh.R;
+  a.rope_base = sh.rope_base;
+  a.k_pre = k_pre; a.v_in = v_in; a.start_pos = start_pos; a.w_k = w_k;
+  a.k = cache->k; a.v = cache->v; a.kidx = cache->kidx; a.status = cache->status;
+  for (int i = 0; i < kMaxRetrieval; ++i) a.ret_rank[i] = sh.ret_rank[i];
+  const long long rows = (long long)sh.B * T * sh.Hkv;
+  if (rows == 0) return RTP_OK;
+  const unsigned grid = (unsigned)((rows + 7) / 8);
+  if (sh.dtype == RTP_BF16) {
+    if (sh.D == 128) append_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(a);
+    else append_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(a);
+  } else {
+    if (sh.D == 128) append_kernel<float, 128><<<grid, 256, 0, st>>>(a);
+    else append_kernel<float, 64><<<grid, 256, 0, st>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error(std::string("append launch: ") + cudaGetErrorString(e));
+    return RTP_ERR_CUDA;
+  }
+  return RTP_OK;
+}
+
+}  // namespace rtp

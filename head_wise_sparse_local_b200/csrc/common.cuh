@@ -1,0 +1,188 @@
+// Device helpers shared by the layer's kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math_constants.h>
+#include <stdint.h>
+
+#include "rtp.h"
+
+namespace rtp {
+
+constexpr int kIdxDim = 16;        // indexer width (abstract, observation (2))
+constexpr float kIdxScale = 0.25f; // 1/sqrt(16)
+constexpr int kMaxRetrieval = 64;
+
+// ---------------------------------------------------------------------------
+// element IO
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+__device__ __forceinline__ float to_f32(float x) { return x; }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+  return __float2bfloat16_rn(x);
+}
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+
+// Load N contiguous elements (N * sizeof(T) a multiple of 16 bytes, 16-byte
+// aligned) and widen to fp32.
+template <typename T, int N>
+__device__ __forceinline__ void load_row(const T* __restrict__ p, float (&out)[N]) {
+  static_assert((N * sizeof(T)) % 16 == 0, "row slice must be whole 16-byte vectors");
+  constexpr int kVec = (N * sizeof(T)) / 16;
+  const uint4* v = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < kVec; ++i) {
+    uint4 u = __ldg(v + i);
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float2 f = __bfloat1622float2(h[k]);
+        out[i * 8 + 2 * k] = f.x;
+        out[i * 8 + 2 * k + 1] = f.y;
+      }
+    } else {
+      out[i * 4 + 0] = __uint_as_float(u.x);
+      out[i * 4 + 1] = __uint_as_float(u.y);
+      out[i * 4 + 2] = __uint_as_float(u.z);
+      out[i * 4 + 3] = __uint_as_float(u.w);
+    }
+  }
+}
+
+// Raw 16-byte vector loads of N elements (kept packed, for software pipelining).
+template <typename T, int N>
+struct RawRow {
+  static constexpr int kVec = (N * sizeof(T)) / 16;
+  uint4 v[kVec];
+  __device__ __forceinline__ void load(const T* __restrict__ p) {
+    const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+    for (int i = 0; i < kVec; ++i) v[i] = __ldg(q + i);
+  }
+  __device__ __forceinline__ float get(int i) const {  // i must be a compile-time index after unrolling
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(v);
+      return __bfloat162float(h[i]);
+    } else {
+      const float* f = reinterpret_cast<const float*>(v);
+      return f[i];
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------
+// score ordering for top-p
+// ---------------------------------------------------------------------------
+// Order-preserving 32-bit key of a (non-NaN, canonical-zero) fp32 score:
+// key(a) < key(b)  <=>  a < b.
+__device__ __forceinline__ uint32_t score_key(float s) {
+  uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_score(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// First-level histogram bucket of a score: 2048 buckets, monotone
+// non-decreasing in s.  Per sign: 16 octaves |s| in [2^-6, 2^10) with 64
+// sub-buckets each; smaller magnitudes share the innermost bucket and larger
+// ones the outermost.
+constexpr int kNumBuckets = 2048;
+constexpr int kBucketELo = 121;  // biased exponent of 2^-6
+__device__ __forceinline__ int score_bucket(float s) {
+  const uint32_t u = __float_as_uint(s);
+  const uint32_t mag = u & 0x7fffffffu;
+  const int e = int(mag >> 23);
+  int t;
+  if (e < kBucketELo) t = 0;
+  else if (e > kBucketELo + 15) t = 1023;
+  else t = (e - kBucketELo) * 64 + int((mag >> 17) & 63u);
+  return (u >> 31) ? 1023 - t : 1024 + t;
+}
+
+// Softmax mass of a score relative to the maximum, in 2^-40 fixed point.
+// exp(s - m) is in (0, 1]; integer sums are exact and order independent, so
+// every kernel that accumulates these weights agrees bit for bit.
+__device__ __forceinline__ unsigned long long mass_fx(float s, float m) {
+  const float w = expf(s - m);
+  return __float2ull_rn(w * 1099511627776.0f);
+}
+
+// ---------------------------------------------------------------------------
+// reductions
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Inclusive warp scan of u64.
+__device__ __forceinline__ unsigned long long warp_incl_scan_u64(unsigned long long v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    unsigned long long n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+__device__ __forceinline__ unsigned warp_incl_scan_u32(unsigned v) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    unsigned n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  return v;
+}
+
+// Exclusive block scan (u64 and u32 together) for blockDim.x == kThreads.
+// `sm` needs 2 * (kThreads / 32) slots of each type.
+template <int kThreads>
+__device__ __forceinline__ void block_excl_scan2(unsigned long long a, unsigned c,
+                                                 unsigned long long& a_ex, unsigned& c_ex,
+                                                 unsigned long long& a_tot, unsigned& c_tot,
+                                                 unsigned long long* sm_a, unsigned* sm_c) {
+  constexpr int kWarps = kThreads / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned long long ai = warp_incl_scan_u64(a);
+  unsigned ci = warp_incl_scan_u32(c);
+  if (lane == 31) { sm_a[warp] = ai; sm_c[warp] = ci; }
+  __syncthreads();
+  unsigned long long wa = 0, ta = 0;
+  unsigned wc = 0, tc = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    if (w < warp) { wa += sm_a[w]; wc += sm_c[w]; }
+    ta += sm_a[w];
+    tc += sm_c[w];
+  }
+  a_ex = wa + ai - a;
+  c_ex = wc + ci - c;
+  a_tot = ta;
+  c_tot = tc;
+  __syncthreads();
+}
+
+// RoPE angle: pos * base^(-2k/D), reduced to [-pi, pi] in fp64 before the
+// fp32 sincos so that positions up to 2^23 keep full fp32 accuracy.
+__device__ __forceinline__ void rope_cos_sin(int pos, int k, int D, float base, float& c,
+                                             float& s) {
+  const double inv = pow((double)base, -2.0 * (double)k / (double)D);
+  const double th = (double)pos * inv;
+  const double two_pi = 6.283185307179586476925286766559;
+  const double r = th - two_pi * rint(th / two_pi);
+  sincosf((float)r, &s, &c);
+}
+
+}  // namespace rtp

@@ -1,0 +1,204 @@
+/*
+ * rtp.h -- C ABI of the B200 (sm_100a) head-wise sparse attention layer.
+ *
+ * The layer is the one described for RTPurbo in "Full Attention Strikes Back:
+ * Transferring Full Attention into Sparse within Hundred Training Steps"
+ * (arXiv 2605.16928): only a few KV heads ("retrieval heads") keep the whole
+ * context; the others ("local heads") attend to attention sinks plus a sliding
+ * window (atlas.scime.ai summary, "Approach").  Retrieval heads choose tokens
+ * with a 16-dimensional pre-RoPE indexer (abstract, observation (2)) and keep
+ * a query-dependent top-p set instead of a fixed top-k (abstract, observation
+ * (3); atlas "Approach": "query-adaptive top-p threshold"), then run exact
+ * attention over the kept rows.
+ *
+ * Conventions for every entry point
+ *   - Pointers are DEVICE pointers unless the comment says "host".  The caller
+ *     owns all memory; the library never allocates, frees or keeps a pointer
+ *     after the call returns.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All device work is enqueued on it; nothing synchronises.
+ *   - The return value is an rtp_status.  Errors that the host can see (null
+ *     pointers, bad shapes, small workspace, a failed launch) return at once
+ *     with nothing enqueued and a message in rtp_last_error().
+ *   - Errors only the device can see (a sequence length or a position outside
+ *     the cache) never trap: the kernels skip the offending sequence/row and
+ *     OR an RTP_DEV_* bit into *cache->status, which the caller reads back
+ *     when it wants (it is never cleared by the library).
+ *   - Layouts are dense row-major in the order written, e.g. K [B][Hkv][Lmax][D]
+ *     means element (b, h, j, d) sits at ((b*Hkv + h)*Lmax + j)*D + d.
+ *   - Element type of q, k, v, out and of the caches is cfg->dtype (bf16 or
+ *     fp32); the indexer projections are always fp32; accumulation is fp32.
+ */
+#ifndef RTP_H_
+#define RTP_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Host-visible status codes. */
+typedef enum rtp_status {
+  RTP_OK = 0,
+  RTP_ERR_INVALID = 1,   /* null pointer or scalar argument out of range */
+  RTP_ERR_SHAPE = 2,     /* unsupported head_dim / group size / sizes */
+  RTP_ERR_DTYPE = 3,     /* dtype not RTP_BF16 or RTP_FP32 */
+  RTP_ERR_WORKSPACE = 4, /* workspace NULL, too small or not 256-byte aligned */
+  RTP_ERR_CUDA = 5       /* a CUDA runtime call or kernel launch failed */
+} rtp_status;
+
+/* Device-side status bits OR-ed into *cache->status. */
+#define RTP_DEV_SEQ_LEN  0x1  /* decode: seq_len[b] < 1 or > max_seq_len; sequence b skipped */
+#define RTP_DEV_POSITION 0x2  /* append/prefill: a position outside [0, max_ctx); rows skipped */
+
+typedef enum rtp_dtype { RTP_BF16 = 0, RTP_FP32 = 1 } rtp_dtype;
+
+/* One attention layer.
+ *   batch         B, sequences per call
+ *   n_q_heads     Hq;  n_kv_heads Hkv;  G = Hq / Hkv query heads share a KV head
+ *                 (GQA; q head hq reads KV head hq / G).  Supported G: 1, 2, 4, 8.
+ *   head_dim      D: 64 or 128
+ *   idx_dim       indexer width; must be 16 (abstract, observation (2))
+ *   max_ctx       Lmax, cache capacity per sequence (positions [0, Lmax));
+ *                 at most 2^23
+ *   n_sink        S >= 0: positions [0, S) are always attended (sinks)
+ *   window        W >= 1: the last W positions up to and including the query
+ *                 position are always attended (sliding window)
+ *   top_p         p in (0, 1]: retrieval heads keep the smallest set of tokens
+ *                 whose indexer softmax mass reaches p (>= p), ties to the lower
+ *                 token index; p = 1 keeps every token
+ *   rope_base     rotary base (10000 for Qwen3); rotate-half convention
+ *   retrieval_mask bit h set => KV head h is a retrieval head.  Retrieval
+ *                 heads are ranked r = 0..R-1 in increasing h; R <= 64
+ *   dtype         rtp_dtype of q, k, v, out and the caches
+ */
+typedef struct rtp_layer_cfg {
+  int batch;
+  int n_q_heads;
+  int n_kv_heads;
+  int head_dim;
+  int idx_dim;
+  int max_ctx;
+  int n_sink;
+  int window;
+  float top_p;
+  float rope_base;
+  uint64_t retrieval_mask;
+  int dtype;
+} rtp_layer_cfg;
+
+/* The layer's cache (device memory owned by the caller; sizes from
+ * rtp_cache_bytes):
+ *   k       [B][Hkv][Lmax][D]  keys after RoPE at their own position
+ *   v       [B][Hkv][Lmax][D]  values
+ *   kidx    [B][R][Lmax][16]   16-d indexer keys k~ = W_k k_pre, one row per
+ *                              token for each retrieval KV head (pre-RoPE)
+ *   status  one int of device-side error bits (see RTP_DEV_*), zeroed by the
+ *           caller before first use
+ */
+typedef struct rtp_cache {
+  void* k;
+  void* v;
+  void* kidx;
+  int* status;
+} rtp_cache;
+
+/* Host.  Bytes of each cache buffer for cfg.  Any output pointer may be NULL. */
+int rtp_cache_bytes(const rtp_layer_cfg* cfg, size_t* k_bytes, size_t* v_bytes,
+                    size_t* kidx_bytes);
+
+/* Host.  Scratch bytes rtp_decode_attn needs for cfg (any max_seq_len <= max_ctx). */
+int rtp_decode_workspace_bytes(const rtp_layer_cfg* cfg, size_t* bytes);
+
+/* Host.  Scratch bytes rtp_prefill_attn needs for cfg and chunk length T. */
+int rtp_prefill_workspace_bytes(const rtp_layer_cfg* cfg, int T, size_t* bytes);
+
+/* Append T tokens per sequence to the cache.
+ *
+ * For every sequence b, token t and KV head h, at position pos = start_pos[b] + t:
+ *   k[b][h][pos] = RoPE(k_pre[b][t][h], pos)            (stored in dtype)
+ *   v[b][h][pos] = v_in[b][t][h]
+ *   kidx[b][r][pos] = W_k^(r) k_pre[b][t][h]              (retrieval head h of rank r;
+ *                                                         fp32 accumulation, stored in dtype)
+ * The indexer key is taken BEFORE RoPE, as the pages' "pre-RoPE" projection
+ * says (atlas.scime.ai summary, "Approach" and its one-line summary).
+ *
+ *   k_pre, v_in  [B][T][Hkv][D] dtype, device
+ *   start_pos    [B] int32, device
+ *   w_k          [R][16][D] fp32, device (may be NULL when R = 0)
+ * Rows with pos outside [0, max_ctx) are skipped and set RTP_DEV_POSITION.
+ */
+int rtp_append_kv(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* k_pre,
+                  const void* v_in, const int* start_pos, int T, const float* w_k,
+                  void* stream);
+
+/* One decode step: the query of sequence b sits at position seq_len[b] - 1 (the
+ * token just appended with rtp_append_kv) and sees positions [0, seq_len[b]).
+ *
+ * Local KV heads: exact attention over sinks [0, S) and window
+ * [seq_len-W, seq_len) (atlas.scime.ai summary, "Approach").
+ * Retrieval KV heads, for each of their G query heads separately:
+ *   q~ = W_q^(r) q_pre (fp32), s_j = q~ . kidx_j / 4 for every cached j,
+ *   P = softmax(s); keep the smallest set, ordered by (P desc, j asc), whose
+ *   mass reaches top_p (abstract, observations (2)-(3)); attend exactly over
+ *   that set united with the sinks and the window.
+ * Attention: softmax(RoPE(q, pos) . k_j / sqrt(D)) over the attended rows.
+ *
+ *   q_pre        [B][Hq][D] dtype, device, pre-RoPE queries
+ *   seq_len      [B] int32, device, 1 <= seq_len[b] <= max_seq_len
+ *   max_seq_len  host int, an upper bound on seq_len (sizes the grid);
+ *                0 means cfg->max_ctx
+ *   w_q          [R][16][D] fp32, device
+ *   out          [B][Hq][D] dtype, device
+ *   sel_bitmask  optional (NULL to skip) [B][R*G][ceil(max_ctx/32)] uint32: bit
+ *                j of head (b, r*G+g) is set iff token j is in that query head's
+ *                top-p set (before the sinks/window union).  Words covering
+ *                positions >= max_seq_len are not written.
+ *   sel_count    optional [B][R*G] int32: size of each top-p set
+ *   workspace    >= rtp_decode_workspace_bytes, 256-byte aligned, device; its
+ *                contents need no initialisation and are clobbered
+ * A sequence with an invalid seq_len is skipped (its out rows untouched) and
+ * sets RTP_DEV_SEQ_LEN.
+ */
+int rtp_decode_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
+                    const int* seq_len, int max_seq_len, const float* w_q, void* out,
+                    uint32_t* sel_bitmask, int* sel_count, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/* One causal prefill chunk: query row t of sequence b sits at position
+ * i = start_pos[b] + t and sees positions [0, i].  The chunk's keys and values
+ * must already be in the cache (rtp_append_kv with the same start_pos and T).
+ * Per row the layer computes exactly what rtp_decode_attn computes for a
+ * query at position i (top-p over the indexer scores of [0, i] for retrieval
+ * query heads; sinks and window [i-W+1, i] for every head).
+ *
+ *   q_pre        [B][T][Hq][D] dtype, device
+ *   start_pos    [B] int32, device; start_pos[b] + T <= max_ctx
+ *   w_q          [R][16][D] fp32, device
+ *   out          [B][T][Hq][D] dtype, device
+ *   sel_tau      optional [B][R*G][T] float: score of the last kept token of the
+ *                row's top-p set (+inf-free; p = 1 gives -inf)
+ *   sel_jcut     optional [B][R*G][T] int32: tokens with score == sel_tau are kept
+ *                iff their index <= sel_jcut (so membership is
+ *                s_j > tau || (s_j == tau && j <= jcut))
+ *   sel_count    optional [B][R*G][T] int32: size of the row's top-p set
+ *   workspace    >= rtp_prefill_workspace_bytes(cfg, T), 256-byte aligned
+ */
+int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
+                     const int* start_pos, int T, const float* w_q, void* out, float* sel_tau,
+                     int* sel_jcut, int* sel_count, void* workspace, size_t workspace_bytes,
+                     void* stream);
+
+/* Host.  Message for the last non-OK return on this thread ("" if none). */
+const char* rtp_last_error(void);
+
+/* Host.  Library version string. */
+const char* rtp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RTP_H_ */
