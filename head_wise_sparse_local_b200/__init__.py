@@ -17,14 +17,15 @@ from typing import Optional, Sequence
 import torch
 
 from . import _abi
-from ._abi import (EXPORTS, RTP_BF16, RTP_DEV_POSITION, RTP_DEV_SEQ_LEN, RTP_FP32, RtpError,
-                   rtp_cache, rtp_layer_cfg)
+from ._abi import (EXPORTS, RTP_BF16, RTP_DEV_POSITION, RTP_DEV_SEQ_LEN, RTP_FP32, STAGES,
+                   RtpError, rtp_cache, rtp_layer_cfg)
 
 _lib = _abi.load()
 
 __all__ = ["Layer", "RtpError", "rtp_layer_cfg", "rtp_cache", "rtp_cache_bytes",
            "rtp_decode_workspace_bytes", "rtp_prefill_workspace_bytes", "rtp_append_kv",
-           "rtp_decode_attn", "rtp_prefill_attn", "rtp_last_error", "rtp_version", "make_cfg",
+           "rtp_decode_attn", "rtp_prefill_attn", "rtp_trace_stage", "rtp_last_error",
+           "rtp_version", "make_cfg", "STAGES",
            "library_path", "EXPORTS", "RTP_BF16", "RTP_FP32", "RTP_DEV_SEQ_LEN",
            "RTP_DEV_POSITION"]
 
@@ -71,6 +72,20 @@ def rtp_version() -> str:
 
 def rtp_last_error() -> str:
     return _lib.rtp_last_error().decode()
+
+
+def rtp_trace_stage(stage, start_event=None, stop_event=None) -> None:
+    """Arm CUDA events (torch.cuda.Event with timing) around the next launch of a stage."""
+    sid = STAGES[stage] if isinstance(stage, str) else int(stage)
+    handles = []
+    for ev in (start_event, stop_event):
+        if ev is None:
+            handles.append(None)
+            continue
+        if not ev.cuda_event:  # torch creates its events lazily, at the first record
+            ev.record()
+        handles.append(ev.cuda_event)
+    _abi.check(_lib.rtp_trace_stage(sid, handles[0], handles[1]))
 
 
 def rtp_cache_bytes(cfg: rtp_layer_cfg):

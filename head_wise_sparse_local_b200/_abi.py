@@ -24,7 +24,11 @@ STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_INVALID", 2: "RTP_ERR_SHAPE", 3: "RTP_E
 
 # Every entry point declared in include/rtp.h.
 EXPORTS = ("rtp_cache_bytes", "rtp_decode_workspace_bytes", "rtp_prefill_workspace_bytes",
-           "rtp_append_kv", "rtp_decode_attn", "rtp_prefill_attn", "rtp_last_error", "rtp_version")
+           "rtp_append_kv", "rtp_decode_attn", "rtp_prefill_attn", "rtp_trace_stage",
+           "rtp_last_error", "rtp_version")
+
+STAGES = {"append": 0, "decode_score": 1, "decode_hist": 2, "decode_select": 3, "decode_attn": 4,
+          "prefill_index": 5, "prefill_attn": 6}
 
 
 class rtp_layer_cfg(ctypes.Structure):
@@ -55,7 +59,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     if _lib is not None:
         return _lib
     if not os.path.exists(path):
-        raise ImportError(f"{path} is missing: build it with `python -m head_wise_sparse_local_b200.build`")
+        raise ImportError(f"{path} is missing: build it with `python head_wise_sparse_local_b200/build.py`")
     lib = ctypes.CDLL(path)
     P = ctypes.POINTER
     vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
@@ -66,6 +70,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rtp_append_kv.argtypes = [cfgp, cachep, vp, vp, vp, i32, vp, vp]
     lib.rtp_decode_attn.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
     lib.rtp_prefill_attn.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.rtp_trace_stage.argtypes = [i32, vp, vp]
     for name in EXPORTS:
         getattr(lib, name).restype = ctypes.c_char_p if name in ("rtp_last_error", "rtp_version") \
             else ctypes.c_int

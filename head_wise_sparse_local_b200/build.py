@@ -1,6 +1,8 @@
 """Build librtp.so in-tree with nvcc for sm_100a (B200).
 
-    python -m head_wise_sparse_local_b200.build [--force] [--jobs N]
+    python head_wise_sparse_local_b200/build.py [--force] [--jobs N] [-v]
+
+(Run it as a script: importing the package itself loads librtp.so.)
 
 Each csrc/*.cu compiles to an object under _build/ (skipped when newer than
 its sources), then one shared library is linked next to this file.

@@ -105,6 +105,7 @@ int launch_append(const Shape& sh, const rtp_cache* cache, const void* k_pre, co
   const long long rows = (long long)sh.B * T * sh.Hkv;
   if (rows == 0) return RTP_OK;
   const unsigned grid = (unsigned)((rows + 7) / 8);
+  trace_begin(RTP_STAGE_APPEND, st);
   if (sh.dtype == RTP_BF16) {
     if (sh.D == 128) append_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(a);
     else append_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(a);
@@ -112,6 +113,7 @@ int launch_append(const Shape& sh, const rtp_cache* cache, const void* k_pre, co
     if (sh.D == 128) append_kernel<float, 128><<<grid, 256, 0, st>>>(a);
     else append_kernel<float, 64><<<grid, 256, 0, st>>>(a);
   }
+  trace_end(RTP_STAGE_APPEND, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("append launch: ") + cudaGetErrorString(e));

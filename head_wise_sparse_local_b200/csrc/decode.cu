@@ -823,15 +823,22 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   const int n_sel_tiles = (Lh + kSelTile - 1) / kSelTile;
   if (sh.R > 0) {
     const dim3 gs(nch_score, sh.B * sh.R);
+    trace_begin(RTP_STAGE_DECODE_SCORE, st);
     if (sh.dtype == RTP_BF16) launch_score_g<__nv_bfloat16>(a, gs, st);
     else launch_score_g<float>(a, gs, st);
+    trace_end(RTP_STAGE_DECODE_SCORE, st);
     const dim3 gh(nch_sel, sh.B * sh.NR);
+    trace_begin(RTP_STAGE_DECODE_HIST, st);
     hist_kernel<<<gh, kThreads, 0, st>>>(a);
+    trace_end(RTP_STAGE_DECODE_HIST, st);
+    trace_begin(RTP_STAGE_DECODE_SELECT, st);
     collect_kernel<<<gh, kThreads, 0, st>>>(a);
+    trace_end(RTP_STAGE_DECODE_SELECT, st);
   } else {
     cudaMemsetAsync(a.ctl, 0, (size_t)a.n_ctl * sizeof(unsigned), st);
   }
   const dim3 ga(lay.n_sw_tiles + (sh.R > 0 ? n_sel_tiles : 0), sh.B * sh.Hkv);
+  trace_begin(RTP_STAGE_DECODE_ATTN, st);
   if (sh.dtype == RTP_BF16) {
     if (sh.D == 128) launch_attn_g<__nv_bfloat16, 128>(a, ga, st);
     else launch_attn_g<__nv_bfloat16, 64>(a, ga, st);
@@ -839,6 +846,7 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
     if (sh.D == 128) launch_attn_g<float, 128>(a, ga, st);
     else launch_attn_g<float, 64>(a, ga, st);
   }
+  trace_end(RTP_STAGE_DECODE_ATTN, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("decode launch: ") + cudaGetErrorString(e));

@@ -13,6 +13,11 @@ namespace rtp {
 
 void set_error(const std::string& msg);
 
+// One-shot launch tracing (rtp_trace_stage): record the armed start event
+// before, and the stop event after, a stage's kernel launch on `st`.
+void trace_begin(int stage, cudaStream_t st);
+void trace_end(int stage, cudaStream_t st);
+
 struct Shape {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W;
   float top_p, rope_base;

@@ -13,6 +13,26 @@ static thread_local std::string g_last_error;
 
 void set_error(const std::string& msg) { g_last_error = msg; }
 
+struct TraceSlot {
+  cudaEvent_t start = nullptr, stop = nullptr;
+  bool started = false;
+};
+static thread_local TraceSlot g_trace[RTP_STAGE_COUNT];
+
+void trace_begin(int stage, cudaStream_t st) {
+  TraceSlot& t = g_trace[stage];
+  if (!t.start || t.started) return;
+  cudaEventRecord(t.start, st);
+  t.started = true;
+}
+
+void trace_end(int stage, cudaStream_t st) {
+  TraceSlot& t = g_trace[stage];
+  if (!t.started) return;
+  cudaEventRecord(t.stop, st);
+  t = TraceSlot();
+}
+
 static int fail(int code, const std::string& msg) {
   set_error(msg);
   return code;
@@ -91,6 +111,17 @@ extern "C" {
 const char* rtp_last_error(void) { return g_last_error.c_str(); }
 
 const char* rtp_version(void) { return "rtp 0.1 sm_100a"; }
+
+int rtp_trace_stage(int stage, void* start_event, void* stop_event) {
+  if (stage < 0 || stage >= RTP_STAGE_COUNT) return fail(RTP_ERR_INVALID, "unknown stage");
+  TraceSlot& t = g_trace[stage];
+  t = TraceSlot();
+  if (start_event && stop_event) {
+    t.start = static_cast<cudaEvent_t>(start_event);
+    t.stop = static_cast<cudaEvent_t>(stop_event);
+  }
+  return RTP_OK;
+}
 
 int rtp_cache_bytes(const rtp_layer_cfg* cfg, size_t* k_bytes, size_t* v_bytes,
                     size_t* kidx_bytes) {

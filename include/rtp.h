@@ -191,6 +191,28 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
                      int* sel_jcut, int* sel_count, void* workspace, size_t workspace_bytes,
                      void* stream);
 
+/* Kernel stages, for rtp_trace_stage. */
+typedef enum rtp_stage {
+  RTP_STAGE_APPEND = 0,         /* rtp_append_kv: RoPE + cache + indexer-key store */
+  RTP_STAGE_DECODE_SCORE = 1,   /* decode: indexer scores over the 16-d key cache */
+  RTP_STAGE_DECODE_HIST = 2,    /* decode: softmax-mass histogram + boundary bucket */
+  RTP_STAGE_DECODE_SELECT = 3,  /* decode: boundary candidates + exact threshold */
+  RTP_STAGE_DECODE_ATTN = 4,    /* decode: gathered attention + log-sum-exp merge */
+  RTP_STAGE_PREFILL_INDEX = 5,  /* prefill: indexer score/threshold passes */
+  RTP_STAGE_PREFILL_ATTN = 6,   /* prefill: masked causal attention */
+  RTP_STAGE_COUNT = 7
+} rtp_stage;
+
+/* Host.  Optional instrumentation (no work is skipped or added).  Arms a
+ * one-shot trace: the next kernel of `stage` launched by an rtp_* call on this
+ * host thread is bracketed by cudaEventRecord(start_event) and
+ * cudaEventRecord(stop_event) on its launch stream.  Events are cudaEvent_t
+ * passed as void*, created and owned by the caller (with timing enabled to
+ * read cudaEventElapsedTime).  A stage launched several times by one call
+ * (none today) records around its first launch.  NULL events disarm the stage.
+ * Returns RTP_ERR_INVALID for an unknown stage. */
+int rtp_trace_stage(int stage, void* start_event, void* stop_event);
+
 /* Host.  Message for the last non-OK return on this thread ("" if none). */
 const char* rtp_last_error(void);
 
