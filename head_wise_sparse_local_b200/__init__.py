@@ -17,14 +17,15 @@ from typing import Optional, Sequence
 import torch
 
 from . import _abi
-from ._abi import (EXPORTS, RTP_BF16, RTP_DEV_POSITION, RTP_DEV_SEQ_LEN, RTP_FP32, STAGES,
-                   RtpError, rtp_cache, rtp_layer_cfg)
+from ._abi import (EXPORTS, RTP_BF16, RTP_DEV_POSITION, RTP_DEV_SEQ_LEN, RTP_FP32,
+                   RTP_NOALLOC_SCRATCH_BYTES, STAGES, RtpError, rtp_cache, rtp_layer_cfg)
 
 _lib = _abi.load()
 
 __all__ = ["Layer", "RtpError", "rtp_layer_cfg", "rtp_cache", "rtp_cache_bytes",
            "rtp_decode_workspace_bytes", "rtp_prefill_workspace_bytes", "rtp_append_kv",
-           "rtp_decode_attn", "rtp_prefill_attn", "rtp_trace_stage", "rtp_last_error",
+           "rtp_decode_attn", "rtp_decode_attn_noalloc", "rtp_prefill_attn", "rtp_trace_stage",
+           "rtp_last_error", "RTP_NOALLOC_SCRATCH_BYTES",
            "rtp_version", "make_cfg", "STAGES",
            "library_path", "EXPORTS", "RTP_BF16", "RTP_FP32", "RTP_DEV_SEQ_LEN",
            "RTP_DEV_POSITION"]
@@ -117,6 +118,14 @@ def rtp_decode_attn(cfg, cache, q_pre, seq_len, max_seq_len, w_q, out, sel_bitma
                                     _ptr(seq_len), int(max_seq_len), _ptr(w_q), _ptr(out),
                                     _ptr(sel_bitmask), _ptr(sel_count), _ptr(workspace),
                                     int(workspace_bytes), _stream(stream)))
+
+
+def rtp_decode_attn_noalloc(cfg, cache, q_pre, seq_len, max_seq_len, w_q, out, sel_bitmask=None,
+                            sel_count=None, stream=None) -> None:
+    """rtp_decode_attn with the library's fixed device scratch instead of a workspace."""
+    _abi.check(_lib.rtp_decode_attn_noalloc(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q_pre),
+                                            _ptr(seq_len), int(max_seq_len), _ptr(w_q), _ptr(out),
+                                            _ptr(sel_bitmask), _ptr(sel_count), _stream(stream)))
 
 
 def rtp_prefill_attn(cfg, cache, q_pre, start_pos, T, w_q, out, sel_tau=None, sel_jcut=None,

@@ -18,13 +18,15 @@ RTP_DEV_SEQ_LEN = 0x1
 RTP_DEV_POSITION = 0x2
 RTP_BF16 = 0
 RTP_FP32 = 1
+RTP_NOALLOC_SCRATCH_BYTES = 32 << 20
 
 STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_INVALID", 2: "RTP_ERR_SHAPE", 3: "RTP_ERR_DTYPE",
                 4: "RTP_ERR_WORKSPACE", 5: "RTP_ERR_CUDA"}
 
 # Every entry point declared in include/rtp.h.
 EXPORTS = ("rtp_cache_bytes", "rtp_decode_workspace_bytes", "rtp_prefill_workspace_bytes",
-           "rtp_append_kv", "rtp_decode_attn", "rtp_prefill_attn", "rtp_trace_stage",
+           "rtp_append_kv", "rtp_decode_attn", "rtp_decode_attn_noalloc", "rtp_prefill_attn",
+           "rtp_trace_stage",
            "rtp_last_error", "rtp_version")
 
 STAGES = {"append": 0, "decode_score": 1, "decode_hist": 2, "decode_select": 3, "decode_attn": 4,
@@ -71,6 +73,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rtp_decode_attn.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
     lib.rtp_prefill_attn.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.rtp_trace_stage.argtypes = [i32, vp, vp]
+    lib.rtp_decode_attn_noalloc.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp]
     for name in EXPORTS:
         getattr(lib, name).restype = ctypes.c_char_p if name in ("rtp_last_error", "rtp_version") \
             else ctypes.c_int

@@ -167,6 +167,34 @@ int rtp_decode_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void
                     uint32_t* sel_bitmask, int* sel_count, void* workspace,
                     size_t workspace_bytes, void* stream);
 
+/* Size of the fixed device scratch array behind rtp_decode_attn_noalloc. */
+#define RTP_NOALLOC_SCRATCH_BYTES (32u << 20)
+
+/* rtp_decode_attn without a caller workspace, for callers that cannot
+ * allocate device memory: plug-ins inside a host framework that owns the
+ * device memory pool, latency-critical callers that cannot accept
+ * cudaMalloc's implicit synchronisation, plain C callers holding only their
+ * input and output buffers.  (The paper has no counterpart; this is an
+ * interface convenience.)
+ *
+ * Arguments, results and errors are those of rtp_decode_attn minus
+ * `workspace`/`workspace_bytes`: the scratch lives in one library-owned
+ * device array of RTP_NOALLOC_SCRATCH_BYTES (32 MiB), reserved on every GPU
+ * that loads the library until the process exits.  The call allocates
+ * nothing.
+ *   - Configurations needing more scratch than that (rtp_decode_workspace_bytes
+ *     > RTP_NOALLOC_SCRATCH_BYTES) return RTP_ERR_WORKSPACE, nothing enqueued.
+ *   - All calls share the array and it keeps the last call's contents; the
+ *     kernels clear what must start at zero.  Calls whose device work
+ *     overlaps (several streams or threads) race on it: serialise them.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current and caches it; make that first call before any
+ *     stream capture.
+ */
+int rtp_decode_attn_noalloc(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
+                            const int* seq_len, int max_seq_len, const float* w_q, void* out,
+                            uint32_t* sel_bitmask, int* sel_count, void* stream);
+
 /* One causal prefill chunk: query row t of sequence b sits at position
  * i = start_pos[b] + t and sees positions [0, i].  The chunk's keys and values
  * must already be in the cache (rtp_append_kv with the same start_pos and T).
