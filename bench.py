@@ -161,11 +161,13 @@ def algorithmic_bytes(shape, seq_len, kept_outside_sw_rows) -> dict:
     idx = sum(R * int(L) * 16 * es for L in seq_len)
     sw_rows = sum(Hkv * (min(shape.n_sink, int(L)) + int(L) - max(min(shape.n_sink, int(L)), int(L) - shape.window))
                   for L in seq_len)
-    kv = (sw_rows + int(kept_outside_sw_rows)) * 2 * D * es
+    sw = sw_rows * 2 * D * es
+    kept = int(kept_outside_sw_rows) * 2 * D * es
     B = len(seq_len)
     append = B * Hkv * D * es * 2 * 2 + B * R * 16 * es  # read k,v; write K,V; write kidx
     qo = B * Hq * D * es * 2
-    return {"score": idx, "attn": kv + qo, "append": append, "total": idx + kv + qo + append}
+    return {"score": idx, "sw": sw, "kept": kept, "qo": qo, "append": append,
+            "total": idx + sw + kept + qo + append}
 
 
 def kept_rows_outside_sw(shape, seq_len, bitmask: torch.Tensor) -> int:
@@ -319,8 +321,8 @@ def run_ours(args, dist: Dist) -> dict:
         raise RuntimeError(f"device status {status} during the timed steps")
 
     # per-kernel CUDA-event timing (same steps, eager launches behind a pre-roll)
-    stages = ["append", "decode_score", "decode_hist", "decode_select", "decode_attn"] if R else \
-        ["append", "decode_attn"]
+    stages = ["append", "decode_stream", "decode_select", "decode_gather"] if R else \
+        ["append", "decode_stream", "decode_gather"]
     n_k = args.kernel_steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_k)]
     torch.cuda.synchronize()
@@ -372,8 +374,8 @@ def run_ours(args, dist: Dist) -> dict:
 
     # roofline of the dominant kernel
     dominant = max(kern_us, key=lambda s: kern_us[s])
-    kbytes = {"append": nbytes["append"], "decode_score": nbytes["score"], "decode_hist": 0,
-              "decode_select": 0, "decode_attn": nbytes["attn"]}
+    kbytes = {"append": nbytes["append"], "decode_stream": nbytes["score"] + nbytes["sw"],
+              "decode_select": 0, "decode_gather": nbytes["kept"] + nbytes["qo"]}
     peaks = {}
     if os.path.exists(PEAKS_PATH):
         peaks = json.load(open(PEAKS_PATH))
@@ -391,7 +393,7 @@ def run_ours(args, dist: Dist) -> dict:
         e2e={"value": e2e_s * 1e6 / (n_e * B * dist.world), "unit": "µs/token",
              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e},
         clocks=(clocks.summary(t_wall0, t_wall1) if clocks else None),
-        gpu_launches=K * (5 if R else 2), l2=l2, inp=inp, Lh=Lh,
+        gpu_launches=K * (4 if R else 3), l2=l2, inp=inp, Lh=Lh,
     )
 
 

@@ -1,59 +1,61 @@
 // rtp_decode_attn: one decode step of the head-wise sparse attention layer.
 //
-// Pipeline (all on the caller's stream, scratch in the caller's workspace):
-//   1. score_kernel   streams the 16-d indexer-key cache once (two 16-byte
-//                     loads per token), forms s_j = q~ . k~_j / 4 for the G
-//                     query heads of a retrieval KV head, stores the fp32
-//                     scores and a per-chunk maximum.
-//   2. hist_kernel    softmax mass of every score, exp(s - max) in 2^-40 fixed
-//                     point, into a 2048-bucket histogram ordered by score;
-//                     the last CTA of a head finds the bucket where the
-//                     cumulative mass (highest scores first) reaches
-//                     ceil(p * Z).
-//   3. collect_kernel gathers the scores that fall into that bucket; the last
-//                     CTA of a head resolves the exact threshold score tau by
-//                     8-bit radix passes over the candidates and, when only
-//                     some tokens tied at tau fit, the index j_cut of the last
-//                     one kept (ties go to the lower index).
-//   4. attn_kernel    exact attention.  Sink/window tiles cover every KV head;
-//                     selected-row tiles scan a retrieval head's context and
-//                     attend the kept rows outside sinks/window.  Each CTA
-//                     writes (max, sum, unnormalised o) per query head; the
-//                     last CTA of a KV head merges them (log-sum-exp) into out.
+// Three kernels on the caller's stream, chained with programmatic dependent
+// launch (each waits on griddepcontrol before touching its predecessor's
+// results), scratch in the caller's workspace:
+//
+//   stream_kernel  two kinds of CTA in one grid, both HBM streams:
+//                  * score CTAs read the 16-d indexer-key cache once (two
+//                    16-byte loads per token for bf16) and write the fp32
+//                    scores s_j = q~ . k~_j / 4 of the G query heads of a
+//                    retrieval KV head plus a per-chunk maximum;
+//                  * sink/window CTAs run exact attention over the sinks and
+//                    the window of every KV head (these rows do not depend on
+//                    the selection) and write one partial (m, l, o) per tile.
+//   select_kernel  one thread-block cluster per (sequence, retrieval q head).
+//                  The softmax mass exp(s - max) of every score, in 2^-36
+//                  fixed point (integer sums: exact and order independent),
+//                  goes into a 2048-bucket histogram ordered by score; the
+//                  cluster merges it through distributed shared memory, finds
+//                  the bucket where the mass of the highest scores reaches
+//                  ceil(p * Z), gathers that bucket's scores in the leader CTA,
+//                  and the leader resolves the exact threshold score tau and,
+//                  for ties at tau, the last kept index j_cut.  The top-p set
+//                  is written as a bitmask.
+//   gather_kernel  for retrieval KV heads: the union over the G query heads
+//                  of the kept rows outside sinks/window, read from the
+//                  bitmask, attended exactly; the last CTA of each KV head
+//                  merges every partial of that head (log-sum-exp) into out.
+//                  Local KV heads only merge their sink/window partials.
+//
 // Top-p follows the abstract's observation (3) and the atlas.scime.ai summary
-// ("query-adaptive top-p threshold"); sinks + window follow the same summary's
+// ("query-adaptive top-p threshold"); sinks + window follow that summary's
 // "Approach"; the 16-d pre-RoPE indexer follows observation (2).
 #include <climits>
+#include <type_traits>
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 #include "internal.h"
+
+namespace cg = cooperative_groups;
 
 namespace rtp {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kScoreChunk = 1024;  // tokens per score CTA
-constexpr int kSelChunk = 4096;    // tokens per histogram / collect CTA
-constexpr int kSwTile = 128;       // sink/window rows per attention CTA
-constexpr int kSelTile = 2048;     // context rows scanned per selected-row CTA
-constexpr int kCandSmem = 4096;    // candidates staged in shared memory for the solve
-
-enum : int { kModeThresh = 0, kModeAll = 1, kModeSkip = 2 };
-
-struct DecodeHead {
-  unsigned long long target;  // ceil(p * Z), 2^-40 units
-  unsigned long long above;   // mass of the buckets above the boundary bucket
-  float m;                    // maximum score
-  float tau;                  // score of the last kept token
-  int bucket;                 // boundary bucket
-  int mode;
-  int jcut;                   // tokens with score == tau kept iff index <= jcut
-  unsigned cnt_above;         // tokens in the buckets above the boundary
-  int pad[2];
-};
+constexpr int kWarps = kThreads / 32;
+constexpr int kScoreChunk = 1024;   // tokens per score CTA (4 per thread)
+constexpr int kSwTile = 256;        // sink/window rows per attention CTA (32 per warp)
+constexpr int kGatherTile = 8192;   // context tokens scanned per gather CTA (256 mask words)
+constexpr int kSelThreads = 512;
+constexpr int kCandSmem = 4096;     // candidates the leader stages in shared memory
+constexpr int kBruteMax = kSelThreads;  // exact solve by pairwise ranks up to this many candidates
 
 struct DecodeArgs {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W, max_seq_len, words;
+  int lstride;      // row stride of the score scratch (Lmax rounded up to 32)
   float top_p, rope_base;
   const void* q_pre;
   const float* w_q;
@@ -63,33 +65,28 @@ struct DecodeArgs {
   const void* kidx;
   int* status;
   const int* seq_len;
-  uint32_t* sel_bitmask;
-  int* sel_count;
-  float* logits;
-  float* cmax;
-  unsigned long long* hmass;
-  unsigned* hcnt;
-  DecodeHead* heads;
-  unsigned* ctl;  // [tick_hist NRt][tick_coll NRt][ncand NRt][tick_attn B*Hkv]
-  uint2* cand;
-  float* pm;
+  uint32_t* mask;   // [B][NR][words] top-p bitmask (caller's sel_bitmask or scratch)
+  int* sel_count;   // optional [B][NR]
+  float* logits;    // [B][NR][lstride]
+  float* cmax;      // [B][NR][nch_score_max]
+  float* pm;        // [B][Hkv][n_parts_max][G]
   float* pl;
-  float* po;
-  int n_ctl, nch_score_max, n_sw_tiles, n_tiles_max;
+  float* po;        // [B][Hkv][n_parts_max][G][D]
+  unsigned* ctl;    // [B*Hkv] gather tickets
+  uint2* cand;      // [B][NR][lstride] boundary-bucket candidates (key, index)
+  int n_ctl, nch_score_max, n_sw_tiles, n_parts_max, n_score_ctas, n_sw_ctas;
   int ret_head[kMaxRetrieval];
   int ret_rank[kMaxRetrieval];
 };
 
-__device__ __forceinline__ unsigned* tick_hist(const DecodeArgs& a) { return a.ctl; }
-__device__ __forceinline__ unsigned* tick_coll(const DecodeArgs& a) { return a.ctl + a.B * a.NR; }
-__device__ __forceinline__ unsigned* ncand(const DecodeArgs& a) { return a.ctl + 2 * a.B * a.NR; }
-__device__ __forceinline__ unsigned* tick_attn(const DecodeArgs& a) { return a.ctl + 3 * a.B * a.NR; }
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 __device__ __forceinline__ bool seq_ok(int L, const DecodeArgs& a) {
   return L >= 1 && L <= a.max_seq_len;
 }
 
-// Block-wide max for kThreads threads.
+template <int kN>
 __device__ __forceinline__ float block_max(float v, float* sm) {
   v = warp_max(v);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -98,8 +95,20 @@ __device__ __forceinline__ float block_max(float v, float* sm) {
   __syncthreads();
   float r = sm[0];
 #pragma unroll
-  for (int w = 1; w < kThreads / 32; ++w) r = fmaxf(r, sm[w]);
+  for (int w = 1; w < kN / 32; ++w) r = fmaxf(r, sm[w]);
   return r;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
 }
 
 // "Last CTA of the group" ticket: every CTA of the group calls this once.
@@ -116,226 +125,402 @@ __device__ __forceinline__ bool take_ticket(unsigned* counter, unsigned n, int* 
   return last;
 }
 
-// ---------------------------------------------------------------------------
-// 1. indexer scores
-// ---------------------------------------------------------------------------
-template <typename T, int G>
-__global__ void __launch_bounds__(kThreads) score_kernel(DecodeArgs a) {
-  const int chunk = blockIdx.x;
-  const int b = blockIdx.y / a.R, r = blockIdx.y % a.R;
-  const int tid = threadIdx.x;
-  {  // zero this call's histograms and control words (read by later kernels)
-    const size_t cta = (size_t)blockIdx.y * gridDim.x + chunk;
-    const size_t n_cta = (size_t)gridDim.x * gridDim.y;
-    const size_t n_hist = (size_t)a.B * a.NR * kNumBuckets;
-    for (size_t i = cta * kThreads + tid; i < n_hist; i += n_cta * kThreads) {
-      a.hmass[i] = 0ull;
-      a.hcnt[i] = 0u;
-    }
-    if (cta == 0)
-      for (int i = tid; i < a.n_ctl; i += kThreads) a.ctl[i] = 0u;
-  }
-  const int L = a.seq_len[b];
-  if (!seq_ok(L, a)) {
-    if (chunk == 0 && r == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
-    return;
-  }
-  const int j0 = chunk * kScoreChunk;
-  if (j0 >= L) return;
-  const int h = a.ret_head[r];
-
-  __shared__ float s_q[G][kIdxDim];
-  __shared__ float s_red[kThreads / 32];
-  if (tid < G * kIdxDim) {
-    const int g = tid / kIdxDim, i = tid % kIdxDim;
-    const float* w = a.w_q + ((size_t)r * kIdxDim + i) * a.D;
-    const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * G + g) * a.D;
-    float acc = 0.f;
-    for (int d = 0; d < a.D; ++d) acc = fmaf(__ldg(w + d), to_f32(q[d]), acc);
-    s_q[g][i] = acc;
-  }
-  __syncthreads();
-  float qr[G][kIdxDim];
-#pragma unroll
-  for (int g = 0; g < G; ++g)
-#pragma unroll
-    for (int i = 0; i < kIdxDim; ++i) qr[g][i] = s_q[g][i];
-
-  const T* kidx = static_cast<const T*>(a.kidx) + ((size_t)b * a.R + r) * a.Lmax * kIdxDim;
-  float* lg = a.logits + ((size_t)b * a.NR + (size_t)r * G) * a.Lmax;
-  float mx[G];
-#pragma unroll
-  for (int g = 0; g < G; ++g) mx[g] = -CUDART_INF_F;
-  const int j1 = min(L, j0 + kScoreChunk);
-#pragma unroll 4
-  for (int j = j0 + tid; j < j1; j += kThreads) {
-    float kv[kIdxDim];
-    load_row<T, kIdxDim>(kidx + (size_t)j * kIdxDim, kv);
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float s = 0.f;
-#pragma unroll
-      for (int i = 0; i < kIdxDim; ++i) s = fmaf(qr[g][i], kv[i], s);
-      s = s * kIdxScale + 0.0f;  // exact scaling; +0 turns -0 into +0
-      lg[(size_t)g * a.Lmax + j] = s;
-      mx[g] = fmaxf(mx[g], s);
-    }
-  }
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float m = block_max(mx[g], s_red);
-    if (tid == 0) a.cmax[((size_t)b * a.NR + r * G + g) * a.nch_score_max + chunk] = m;
+// RoPE'd query of the G heads of KV head h at position pos, scaled by
+// log2(e)/sqrt(D), into shared memory [G][D].
+template <typename T, int D, int G>
+__device__ void rope_query(const DecodeArgs& a, int b, int h, int pos, float* s_q) {
+  const float qscale = 1.4426950408889634f * rsqrtf((float)D);
+  for (int i = threadIdx.x; i < G * (D / 2); i += blockDim.x) {
+    const int g = i / (D / 2), k = i % (D / 2);
+    const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * G + g) * D;
+    const float x1 = to_f32(q[k]), x2 = to_f32(q[k + D / 2]);
+    float c, s;
+    rope_cos_sin(pos, k, D, a.rope_base, c, s);
+    s_q[g * D + k] = (x1 * c - x2 * s) * qscale;
+    s_q[g * D + k + D / 2] = (x2 * c + x1 * s) * qscale;
   }
 }
 
 // ---------------------------------------------------------------------------
-// 2. mass histogram + boundary bucket
+// warp-level attention over tiles of 32 rows
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads) hist_kernel(DecodeArgs a) {
-  const int chunk = blockIdx.x;
-  const int bh = blockIdx.y;
-  const int b = bh / a.NR;
-  const int tid = threadIdx.x;
-  __shared__ unsigned long long s_mass[kNumBuckets];
-  __shared__ unsigned s_cnt[kNumBuckets];
-  __shared__ float s_red[kThreads / 32];
-  __shared__ unsigned long long s_sa[kThreads / 32];
-  __shared__ unsigned s_sc[kThreads / 32];
-  __shared__ int s_flag;
+// load(): lane i requests row i's whole key and, for every live row of the
+// tile, its own D/32 value dims, so a tile costs one memory round trip.
+// compute(): lane-per-row dot products against the G queries (broadcast from
+// shared memory), the tile's softmax per head with one exp2 per (row, head),
+// and P V with the row weights broadcast by shuffle.
+template <typename T, int D, int G>
+struct WarpAttn {
+  static constexpr int DL = D / 32;             // output dims per lane
+  static constexpr int KV = D * sizeof(T) / 16; // 16-byte vectors per key row
+  static constexpr int VB = DL * sizeof(T);     // value bytes per lane per row
+  using VRaw = typename std::conditional<VB == 16, uint4,
+               typename std::conditional<VB == 8, uint2,
+               typename std::conditional<VB == 4, unsigned, unsigned short>::type>::type>::type;
+  float m[G], l[G], o[G][DL];
+  uint4 kraw[KV];
+  VRaw vraw[32];
+  int row;
+  unsigned msk, live;
 
-  const int L = a.seq_len[b];
-  const bool valid = seq_ok(L, a);
-  const bool keep_all = a.top_p >= 1.0f;
-  float m = -CUDART_INF_F;
-  unsigned long long* gm = a.hmass + (size_t)bh * kNumBuckets;
-  unsigned* gc = a.hcnt + (size_t)bh * kNumBuckets;
-  if (valid && !keep_all) {
-    const int nch = (L + kScoreChunk - 1) / kScoreChunk;
-    const float* cm = a.cmax + (size_t)bh * a.nch_score_max;
-    for (int c = tid; c < nch; c += kThreads) m = fmaxf(m, cm[c]);
-    m = block_max(m, s_red);
-    const int j0 = chunk * kSelChunk;
-    if (j0 < L) {
-      for (int i = tid; i < kNumBuckets; i += kThreads) { s_mass[i] = 0ull; s_cnt[i] = 0u; }
-      __syncthreads();
-      const float* lg = a.logits + (size_t)bh * a.Lmax;
-      const int j1 = min(L, j0 + kSelChunk);
-      for (int j = j0 + tid; j < j1; j += kThreads) {
-        const float s = lg[j];
-        const int bk = score_bucket(s);
-        atomicAdd(&s_mass[bk], mass_fx(s, m));
-        atomicAdd(&s_cnt[bk], 1u);
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      m[g] = -CUDART_INF_F;
+      l[g] = 0.f;
+#pragma unroll
+      for (int d = 0; d < DL; ++d) o[g][d] = 0.f;
+    }
+  }
+
+  // row_: this lane's row (ignored when msk_ == 0); msk_: head bits.
+  __device__ __forceinline__ void load(const T* __restrict__ kb, const T* __restrict__ vb, int row_,
+                                       unsigned msk_) {
+    const int lane = threadIdx.x & 31;
+    row = msk_ ? row_ : 0;
+    msk = msk_;
+    live = __ballot_sync(0xffffffffu, msk_ != 0u);
+    const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)row * D);
+#pragma unroll
+    for (int i = 0; i < KV; ++i) kraw[i] = msk ? __ldg(kr + i) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      const int rr = __shfl_sync(0xffffffffu, row, r);
+      if ((live >> r) & 1u) vraw[r] = __ldg(reinterpret_cast<const VRaw*>(vb + (size_t)rr * D + lane * DL));
+      else vraw[r] = VRaw();
+    }
+  }
+
+  __device__ __forceinline__ void compute(const float* __restrict__ s_q) {
+    float s[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) s[g] = 0.f;
+    constexpr int E = 16 / sizeof(T);
+#pragma unroll
+    for (int i = 0; i < KV; ++i) {
+      float kf[E];
+      if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kraw[i]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h2[q]);
+          kf[2 * q] = f.x;
+          kf[2 * q + 1] = f.y;
+        }
+      } else {
+        kf[0] = __uint_as_float(kraw[i].x); kf[1] = __uint_as_float(kraw[i].y);
+        kf[2] = __uint_as_float(kraw[i].z); kf[3] = __uint_as_float(kraw[i].w);
       }
-      __syncthreads();
-      for (int i = tid; i < kNumBuckets; i += kThreads) {
-        if (s_cnt[i]) {
-          atomicAdd(&gm[i], s_mass[i]);
-          atomicAdd(&gc[i], s_cnt[i]);
+#pragma unroll
+      for (int e = 0; e < E; e += 4) {
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float4 qv = *reinterpret_cast<const float4*>(s_q + g * D + i * E + e);
+          s[g] = fmaf(qv.x, kf[e], s[g]);
+          s[g] = fmaf(qv.y, kf[e + 1], s[g]);
+          s[g] = fmaf(qv.z, kf[e + 2], s[g]);
+          s[g] = fmaf(qv.w, kf[e + 3], s[g]);
         }
       }
     }
+    float p[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const bool on = (msk >> g) & 1u;
+      const float sv = on ? s[g] : -CUDART_INF_F;
+      const float tm = warp_max(sv);
+      const float mn = fmaxf(m[g], tm);
+      if (mn == -CUDART_INF_F) {  // nothing kept for this head yet (warp-uniform)
+        p[g] = 0.f;
+        continue;
+      }
+      const float al = exp2f(m[g] - mn);
+      p[g] = on ? exp2f(sv - mn) : 0.f;
+      l[g] = l[g] * al + p[g];
+#pragma unroll
+      for (int d = 0; d < DL; ++d) o[g][d] *= al;
+      m[g] = mn;
+    }
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      if (!((live >> r) & 1u)) continue;  // warp-uniform
+      float vv[DL];
+      const T* vt = reinterpret_cast<const T*>(&vraw[r]);
+#pragma unroll
+      for (int d = 0; d < DL; ++d) vv[d] = to_f32(vt[d]);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float pr = __shfl_sync(0xffffffffu, p[g], r);
+#pragma unroll
+        for (int d = 0; d < DL; ++d) o[g][d] = fmaf(pr, vv[d], o[g][d]);
+      }
+    }
   }
-  if (!take_ticket(&tick_hist(a)[bh], gridDim.x, &s_flag)) return;
+};
 
-  DecodeHead* hd = a.heads + bh;
-  if (!valid) {
-    if (tid == 0) hd->mode = kModeSkip;
-    return;
-  }
-  if (keep_all) {
-    if (tid == 0) {
-      hd->mode = kModeAll;
-      if (a.sel_count) a.sel_count[bh] = L;
-    }
-    return;
-  }
-  // Thread t owns buckets NB-1-8t-k, k = 0..7 (highest scores first).
-  constexpr int kPer = kNumBuckets / kThreads;
-  unsigned long long ms[kPer];
-  unsigned cs[kPer];
-  unsigned long long my_m = 0ull;
-  unsigned my_c = 0u;
+// Merge the warps' WarpAttn states of a CTA and write one partial (m, l, o)
+// per query head at slot `part`.
+template <int D, int G, typename WA>
+__device__ void write_partial(const DecodeArgs& a, WA& wa, size_t part, float* s_o, float* s_ml) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int bk = kNumBuckets - 1 - (tid * kPer + k);
-    ms[k] = __ldcg(gm + bk);
-    cs[k] = __ldcg(gc + bk);
-    my_m += ms[k];
-    my_c += cs[k];
-  }
-  unsigned long long ex_m, tot_m;
-  unsigned ex_c, tot_c;
-  block_excl_scan2<kThreads>(my_m, my_c, ex_m, ex_c, tot_m, tot_c, s_sa, s_sc);
-  const double pz = (double)a.top_p * (double)tot_m;
-  unsigned long long target = (unsigned long long)ceil(pz);
-  if (target > tot_m) target = tot_m;
-  if (target < 1ull) target = 1ull;
-  __shared__ unsigned long long s_above;
-  __shared__ unsigned s_cabove;
-  __shared__ int s_bucket;
-  if (tid == 0) s_bucket = -1;
-  __syncthreads();
-  unsigned long long cum = ex_m;
-  unsigned cumc = ex_c;
+  for (int g = 0; g < G; ++g) {
+    const float lw = warp_sum(wa.l[g]);
 #pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    if (cum < target && cum + ms[k] >= target) {  // exactly one (thread, k) crosses
-      s_above = cum;
-      s_cabove = cumc;
-      s_bucket = kNumBuckets - 1 - (tid * kPer + k);
+    for (int d = 0; d < WA::DL; ++d) s_o[(warp * G + g) * D + lane * WA::DL + d] = wa.o[g][d];
+    if (lane == 0) {
+      s_ml[(warp * G + g) * 2] = wa.m[g];
+      s_ml[(warp * G + g) * 2 + 1] = lw;
     }
-    cum += ms[k];
-    cumc += cs[k];
   }
   __syncthreads();
-  if (tid == 0) {
-    if (s_bucket < 0) {  // unreachable for target <= Z; keep every token rather than guess
-      hd->mode = kModeAll;
-      if (a.sel_count) a.sel_count[bh] = L;
-    } else {
-      hd->target = target;
-      hd->above = s_above;
-      hd->cnt_above = s_cabove;
-      hd->bucket = s_bucket;
-      hd->m = m;
-      hd->mode = kModeThresh;
+  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
+    const int g = i / D, d = i % D;
+    float mn = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mn = fmaxf(mn, s_ml[(w * G + g) * 2]);
+    float acc = 0.f, den = 0.f;
+    if (mn != -CUDART_INF_F) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = s_ml[(w * G + g) * 2];
+        if (mw == -CUDART_INF_F) continue;
+        const float sc = exp2f(mw - mn);
+        acc = fmaf(s_o[(w * G + g) * D + d], sc, acc);
+        den = fmaf(s_ml[(w * G + g) * 2 + 1], sc, den);
+      }
+    }
+    a.po[(part * G + g) * D + d] = acc;
+    if (d == 0) {
+      a.pm[part * G + g] = mn;
+      a.pl[part * G + g] = den;
     }
   }
 }
 
 // ---------------------------------------------------------------------------
-// 3. candidates of the boundary bucket + exact threshold
+// 1. stream kernel: indexer scores + sink/window attention
 // ---------------------------------------------------------------------------
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads) stream_kernel(DecodeArgs a) {
+  griddep_wait();
+  griddep_launch();
+  __shared__ __align__(16) float s_q[G * D];
+  __shared__ __align__(16) float s_o[kWarps * G * D];
+  __shared__ float s_ml[kWarps * G * 2];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (blockIdx.x == 0) {  // zero this call's counters (read by later kernels)
+    for (int i = tid; i < a.n_ctl; i += kThreads) a.ctl[i] = 0u;
+    if (a.sel_count)
+      for (int i = tid; i < a.B * a.NR; i += kThreads) a.sel_count[i] = 0;
+  }
+  if ((int)blockIdx.x < a.n_score_ctas) {
+    // ---- indexer scores ----
+    const int nch = a.n_score_ctas / (a.B * a.R);
+    const int chunk = blockIdx.x % nch;
+    const int br = blockIdx.x / nch;
+    const int b = br / a.R, r = br % a.R;
+    const int L = a.seq_len[b];
+    if (!seq_ok(L, a)) {
+      if (chunk == 0 && r == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
+      return;
+    }
+    const int j0 = chunk * kScoreChunk;
+    if (j0 >= L) return;
+    const int j1 = min(L, j0 + kScoreChunk);
+    const int h = a.ret_head[r];
+    // issue this thread's indexer-key loads first (they stay in flight while q~ is formed)
+    constexpr int TPT = kScoreChunk / kThreads;
+    constexpr int NV = kIdxDim * sizeof(T) / 16;
+    const uint4* kidx = reinterpret_cast<const uint4*>(static_cast<const T*>(a.kidx) +
+                                                       ((size_t)b * a.R + r) * a.Lmax * kIdxDim);
+    uint4 kr[TPT][NV];
+#pragma unroll
+    for (int t = 0; t < TPT; ++t) {
+      const int j = j0 + t * kThreads + tid;
+#pragma unroll
+      for (int v = 0; v < NV; ++v) kr[t][v] = (j < j1) ? __ldg(kidx + (size_t)j * NV + v) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // q~ = W_q q_pre: four threads per output, a quarter of the dims each
+    float* s_qi = s_q;  // [G][16]
+    for (int o4 = tid; o4 < G * kIdxDim * 4; o4 += kThreads) {
+      const int o = o4 >> 2, qd = o4 & 3;
+      const int g = o / kIdxDim, i = o % kIdxDim;
+      constexpr int DQ = D / 4;
+      const float4* w = reinterpret_cast<const float4*>(a.w_q + ((size_t)r * kIdxDim + i) * D + qd * DQ);
+      const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * G + g) * D + qd * DQ;
+      float wv[DQ], qv[DQ];
+#pragma unroll
+      for (int k = 0; k < DQ / 4; ++k) {
+        const float4 f = __ldg(w + k);
+        wv[4 * k] = f.x; wv[4 * k + 1] = f.y; wv[4 * k + 2] = f.z; wv[4 * k + 3] = f.w;
+      }
+      load_row<T, DQ>(q, qv);
+      float acc = 0.f;
+#pragma unroll
+      for (int k = 0; k < DQ; ++k) acc = fmaf(wv[k], qv[k], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (qd == 0) s_qi[g * kIdxDim + i] = acc;
+    }
+    __syncthreads();
+    float qr[G][kIdxDim];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int i = 0; i < kIdxDim; ++i) qr[g][i] = s_qi[g * kIdxDim + i];
+    float* lg = a.logits + ((size_t)b * a.NR + (size_t)r * G) * a.lstride;
+    float mx[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) mx[g] = -CUDART_INF_F;
+#pragma unroll
+    for (int t = 0; t < TPT; ++t) {
+      const int j = j0 + t * kThreads + tid;
+      if (j >= j1) continue;
+      float kv[kIdxDim];
+      if constexpr (sizeof(T) == 2) {
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kr[t][v]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float2 f = __bfloat1622float2(h2[q]);
+            kv[v * 8 + 2 * q] = f.x;
+            kv[v * 8 + 2 * q + 1] = f.y;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int v = 0; v < NV; ++v) {
+          kv[v * 4 + 0] = __uint_as_float(kr[t][v].x); kv[v * 4 + 1] = __uint_as_float(kr[t][v].y);
+          kv[v * 4 + 2] = __uint_as_float(kr[t][v].z); kv[v * 4 + 3] = __uint_as_float(kr[t][v].w);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float s = 0.f;
+#pragma unroll
+        for (int i = 0; i < kIdxDim; ++i) s = fmaf(qr[g][i], kv[i], s);
+        s = s * kIdxScale + 0.0f;  // exact scaling; +0 turns -0 into +0
+        lg[(size_t)g * a.lstride + j] = s;
+        mx[g] = fmaxf(mx[g], s);
+      }
+    }
+    // one block reduction for the G chunk maxima
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float v = warp_max(mx[g]);
+      if (lane == 0) s_ml[warp * G + g] = v;
+    }
+    __syncthreads();
+    if (tid < G) {
+      float v = s_ml[tid];
+#pragma unroll
+      for (int w = 1; w < kWarps; ++w) v = fmaxf(v, s_ml[w * G + tid]);
+      a.cmax[((size_t)b * a.NR + r * G + tid) * a.nch_score_max + chunk] = v;
+    }
+    return;
+  }
+  // ---- sink/window attention ----
+  const int idx = blockIdx.x - a.n_score_ctas;
+  const int tile = idx % a.n_sw_tiles;
+  const int bkv = idx / a.n_sw_tiles;
+  const int b = bkv / a.Hkv, h = bkv % a.Hkv;
+  const int L = a.seq_len[b];
+  if (!seq_ok(L, a)) {
+    if (tile == 0 && h == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
+    return;
+  }
+  const int s_cnt = min(a.S, L);
+  const int sw0 = max(s_cnt, L - a.W);
+  const int n_sw = s_cnt + (L - sw0);
+  const int e = tile * kSwTile + threadIdx.x;  // one row per thread, 32 per warp
+  const bool ok = e < n_sw;
+  const int row = ok ? (e < s_cnt ? e : sw0 + (e - s_cnt)) : 0;
+  WarpAttn<T, D, G> wa;
+  wa.init();
+  const T* kb = static_cast<const T*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+  const T* vb = static_cast<const T*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+  wa.load(kb, vb, row, ok ? ((1u << G) - 1u) : 0u);  // in flight during RoPE
+  rope_query<T, D, G>(a, b, h, L - 1, s_q);
+  __syncthreads();
+  wa.compute(s_q);
+  write_partial<D, G>(a, wa, (size_t)bkv * a.n_parts_max + tile, s_o, s_ml);
+}
+
+// ---------------------------------------------------------------------------
+// 2. select kernel (cluster per head): exact top-p threshold + bitmask
+// ---------------------------------------------------------------------------
+template <int CS>
+struct SelShared {
+  unsigned long long slice[CS];   // per-rank slice totals of the approximate histogram
+  unsigned long long zpart[CS];   // [0]: mass above the boundary bucket (broadcast)
+  int bucket;                     // boundary bucket (broadcast)
+  float tau;                      // final threshold (broadcast)
+  int jcut;
+  unsigned n_cand;                // leader: candidates reserved
+  float red[kSelThreads / 32];
+  unsigned long long scan_a[kSelThreads / 32];
+  unsigned scan_c[kSelThreads / 32];
+};
+
+// Softmax mass exp(s - max) in 2^-36 fixed point.  Integer sums of these are
+// exact and order independent, so the histogram and the exact solve agree bit
+// for bit.  The selection accumulates it per bucket as two 18-bit halves with
+// 32-bit shared atomics (native and robust to contention); a score whose mass
+// rounds to zero adds nothing and is skipped.
+__device__ __forceinline__ unsigned long long mass_fx36(float s, float m) {
+  return __float2ull_rn(expf(s - m) * 68719476736.0f);  // 2^36
+}
+
 struct DigitResult {
   int digit;
-  unsigned long long above;  // mass (or count) of the digits ranked before `digit`
+  unsigned long long above;
   unsigned cnt_above;
   unsigned cnt_digit;
 };
 
-// One 8-bit radix step over items[0, n).  kMass: items matching (x & mask) ==
-// prefix are weighted by their softmax mass and digits are ranked from high to
-// low (highest scores first).  !kMass: items with x == key_eq are counted and
-// their index digits (y) ranked from low to high (lowest index first).  Finds
-// the first digit at which the running total reaches `need`.
+// Items for the exact solve: a list of (order key, index), or the scores
+// [0, n) of one head themselves (every score is an item).
+struct Items {
+  const uint2* list;
+  const float* scores;
+  int bucket;  // scan mode: only scores of this bucket are items
+  __device__ __forceinline__ bool get(int i, uint2& e) const {
+    if (list) {
+      e = list[i];
+      return true;
+    }
+    const float s = scores[i];
+    e = make_uint2(score_key(s), (unsigned)i);
+    return score_bucket(s) == bucket;
+  }
+};
+
+// One 8-bit radix step.  kMass: items with (key & mask) == prefix, weighted by
+// their softmax mass, digits ranked high to low.  !kMass: items with key ==
+// key_eq counted, index digits ranked low to high.  Finds the first digit at
+// which the running total reaches `need`.
 template <bool kMass>
-__device__ DigitResult radix_step(const uint2* items, int n, uint32_t prefix, uint32_t mask,
+__device__ DigitResult radix_step(const Items& it, int n, uint32_t prefix, uint32_t mask,
                                   uint32_t key_eq, int shift, float m, unsigned long long need,
                                   unsigned long long* h_m, unsigned* h_c, DigitResult* s_res) {
   const int tid = threadIdx.x;
-  for (int i = tid; i < 256; i += kThreads) { h_m[i] = 0ull; h_c[i] = 0u; }
+  for (int i = tid; i < 256; i += blockDim.x) { h_m[i] = 0ull; h_c[i] = 0u; }
+  if (tid == 0) *s_res = DigitResult{0, 0ull, 0u, 0u};
   __syncthreads();
-  for (int i = tid; i < n; i += kThreads) {
-    const uint2 it = items[i];
+  for (int i = tid; i < n; i += blockDim.x) {
+    uint2 e;
+    if (!it.get(i, e)) continue;
     if constexpr (kMass) {
-      if ((it.x & mask) == prefix) {
-        const int dg = (it.x >> shift) & 255;
-        atomicAdd(&h_m[dg], mass_fx(key_score(it.x), m));
+      if ((e.x & mask) == prefix) {
+        const int dg = (e.x >> shift) & 255;
+        atomicAdd(&h_m[dg], mass_fx36(key_score(e.x), m));
         atomicAdd(&h_c[dg], 1u);
       }
     } else {
-      if (it.x == key_eq && (it.y & mask) == prefix) {
-        const int dg = (it.y >> shift) & 255;
+      if (e.x == key_eq && (e.y & mask) == prefix) {
+        const int dg = (e.y >> shift) & 255;
         atomicAdd(&h_m[dg], 1ull);
         atomicAdd(&h_c[dg], 1u);
       }
@@ -378,387 +563,584 @@ __device__ DigitResult radix_step(const uint2* items, int n, uint32_t prefix, ui
   return res;
 }
 
-__global__ void __launch_bounds__(kThreads) collect_kernel(DecodeArgs a) {
-  const int chunk = blockIdx.x;
-  const int bh = blockIdx.y;
-  const int b = bh / a.NR;
-  const int tid = threadIdx.x, lane = tid & 31;
-  __shared__ int s_flag;
-  __shared__ __align__(16) uint2 s_cand[kCandSmem];
-  __shared__ unsigned long long h_m[256];
-  __shared__ unsigned h_c[256];
-  __shared__ DigitResult s_res;
-  __shared__ uint32_t s_kmin[kThreads / 32], s_kmax[kThreads / 32];
-
-  const int L = a.seq_len[b];
-  const bool valid = seq_ok(L, a);
-  DecodeHead* hd = a.heads + bh;
-  const int mode = valid ? hd->mode : kModeSkip;
-  uint2* cand = a.cand + (size_t)bh * a.Lmax;
-  if (mode == kModeThresh) {
-    const int bucket = hd->bucket;
-    const float* lg = a.logits + (size_t)bh * a.Lmax;
-    const int j0 = chunk * kSelChunk;
-    const int j1 = min(L, j0 + kSelChunk);
-    for (int jb = j0; jb < j1; jb += kThreads) {
-      const int j = jb + tid;
-      float s = 0.f;
-      bool in = false;
-      if (j < j1) {
-        s = lg[j];
-        in = score_bucket(s) == bucket;
-      }
-      const unsigned bal = __ballot_sync(0xffffffffu, in);
-      if (bal) {
-        unsigned base = 0;
-        if (lane == 0) base = atomicAdd(&ncand(a)[bh], (unsigned)__popc(bal));
-        base = __shfl_sync(0xffffffffu, base, 0);
-        if (in) cand[base + __popc(bal & ((1u << lane) - 1u))] = make_uint2(score_key(s), (unsigned)j);
-      }
-    }
-  }
-  if (!take_ticket(&tick_coll(a)[bh], gridDim.x, &s_flag)) return;
-  if (mode != kModeThresh) return;
-
-  // ---- exact threshold among the candidates (this CTA only) ----
-  const int n = (int)__ldcg(&ncand(a)[bh]);
-  const float m = hd->m;
-  const unsigned long long need0 = hd->target - hd->above;
-  const uint2* items = cand;
-  if (n <= kCandSmem) {
-    for (int i = tid; i < n; i += kThreads) s_cand[i] = __ldcg(cand + i);
-    __syncthreads();
-    items = s_cand;
-  }
+// Exact tau / j_cut among n items whose mass must supply `need` (one CTA).
+// Order: key descending, index ascending.  The kept set is the shortest prefix
+// whose mass reaches `need`.
+__device__ void solve_radix(const Items& it, int n, float m, unsigned long long need,
+                            unsigned long long* h_m, unsigned* h_c, DigitResult* s_res,
+                            uint32_t* s_kr, float& tau, int& jcut) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = blockDim.x >> 5;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for (int i = tid; i < n; i += kThreads) {
-    const uint32_t k = items[i].x;
-    kmin = min(kmin, k);
-    kmax = max(kmax, k);
+  int cnt = 0;
+  for (int i = tid; i < n; i += blockDim.x) {
+    uint2 e;
+    if (!it.get(i, e)) continue;
+    kmin = min(kmin, e.x);
+    kmax = max(kmax, e.x);
+    ++cnt;
   }
+  cnt = warp_sum_i(cnt);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     kmin = min(kmin, __shfl_xor_sync(0xffffffffu, kmin, o));
     kmax = max(kmax, __shfl_xor_sync(0xffffffffu, kmax, o));
   }
-  if (lane == 0) { s_kmin[tid >> 5] = kmin; s_kmax[tid >> 5] = kmax; }
+  if (lane == 0) { s_kr[warp] = kmin; s_kr[32 + warp] = kmax; s_kr[64 + warp] = (uint32_t)cnt; }
   __syncthreads();
-  kmin = s_kmin[0];
-  kmax = s_kmax[0];
-#pragma unroll
-  for (int w = 1; w < kThreads / 32; ++w) { kmin = min(kmin, s_kmin[w]); kmax = max(kmax, s_kmax[w]); }
+  kmin = s_kr[0];
+  kmax = s_kr[32];
+  unsigned n_items = s_kr[64];
+  for (int w = 1; w < nw; ++w) {
+    kmin = min(kmin, s_kr[w]);
+    kmax = max(kmax, s_kr[32 + w]);
+    n_items += s_kr[64 + w];
+  }
+  __syncthreads();
 
   uint32_t prefix = kmin, mask = 0xffffffffu;
-  unsigned long long need = need0;
-  unsigned cnt_above_in = 0u;
-  unsigned cnt_eq = (unsigned)n;
+  unsigned cnt_eq = 0u;
   const uint32_t diff = kmin ^ kmax;
   if (diff != 0u) {
     const int hb = 31 - __clz(diff);
     mask = (hb == 31) ? 0u : ~((2u << hb) - 1u);
     prefix = kmin & mask;
     for (int shift = (hb / 8) * 8; shift >= 0; shift -= 8) {
-      const DigitResult d = radix_step<true>(items, n, prefix, mask, 0u, shift, m, need, h_m, h_c, &s_res);
+      const DigitResult d = radix_step<true>(it, n, prefix, mask, 0u, shift, m, need, h_m, h_c, s_res);
       need -= d.above;
-      cnt_above_in += d.cnt_above;
       cnt_eq = d.cnt_digit;
       prefix |= (uint32_t)d.digit << shift;
       mask |= 0xffu << shift;
     }
+  } else {
+    cnt_eq = n_items;  // every item has the same key
   }
   const uint32_t tau_key = prefix;
-  const unsigned long long w_tau = mass_fx(key_score(tau_key), m);
+  const unsigned long long w_tau = mass_fx36(key_score(tau_key), m);
   unsigned long long kk = (w_tau > 0ull) ? (need + w_tau - 1ull) / w_tau : (unsigned long long)cnt_eq;
   if (kk < 1ull) kk = 1ull;
   if (kk > cnt_eq) kk = cnt_eq;
-  int jcut = INT_MAX;
+  int jc = INT_MAX;
   if (kk < cnt_eq) {  // only the first kk tied tokens (by index) are kept
     uint32_t ip = 0u, im = 0u;
     unsigned long long want = kk;
     for (int shift = 16; shift >= 0; shift -= 8) {
-      const DigitResult d = radix_step<false>(items, n, ip, im, tau_key, shift, 0.f, want, h_m, h_c, &s_res);
+      const DigitResult d = radix_step<false>(it, n, ip, im, tau_key, shift, 0.f, want, h_m, h_c, s_res);
       want -= d.above;
       ip |= (uint32_t)d.digit << shift;
       im |= 0xffu << shift;
     }
-    jcut = (int)ip;
+    jc = (int)ip;
   }
-  if (tid == 0) {
-    hd->tau = key_score(tau_key);
-    hd->jcut = jcut;
-    if (a.sel_count) a.sel_count[bh] = (int)(hd->cnt_above + cnt_above_in + (unsigned)kk);
+  tau = key_score(tau_key);
+  jcut = jc;
+}
+
+// Exact tau / j_cut for n <= blockDim.x list items: item i is kept iff the
+// mass of the items ordered before it is below `need`.
+__device__ void solve_brute(const uint2* items, int n, float m, unsigned long long need,
+                            unsigned long long* s_w, uint32_t* s_min, int* s_jmax, float& tau,
+                            int& jcut) {
+  const int tid = threadIdx.x;
+  uint2 me = make_uint2(0u, 0u);
+  if (tid < n) {
+    me = items[tid];
+    s_w[tid] = mass_fx36(key_score(me.x), m);
+  }
+  if (tid == 0) { *s_min = 0xffffffffu; *s_jmax = -1; }
+  __syncthreads();
+  bool kept = false;
+  if (tid < n) {
+    unsigned long long before = 0ull;
+    for (int j = 0; j < n; ++j) {
+      const uint2 o = items[j];
+      if (o.x > me.x || (o.x == me.x && o.y < me.y)) before += s_w[j];
+    }
+    kept = before < need;
+    if (kept) atomicMin(s_min, me.x);
+  }
+  __syncthreads();
+  const uint32_t tk = *s_min;
+  if (kept && me.x == tk) atomicMax(s_jmax, (int)me.y);
+  __syncthreads();
+  tau = key_score(tk);
+  jcut = *s_jmax;
+}
+
+template <int CS>
+struct SelCfg {
+  static constexpr int kLgCap = 131072 / CS;  // scores cached in shared memory per CTA
+  static constexpr size_t kSmem = (size_t)kLgCap * sizeof(float) +
+                                  kNumBuckets * (2 * sizeof(unsigned) + sizeof(unsigned long long)) +
+                                  kBruteMax * sizeof(unsigned long long) + sizeof(SelShared<CS>);
+};
+static_assert(kNumBuckets * (2 * sizeof(unsigned) + sizeof(unsigned long long)) >= kCandSmem * sizeof(uint2),
+              "the leader stages candidates in the histogram's bytes");
+
+// Every kFold scores the 18-bit halves of the histogram are folded into the
+// 64-bit bins, so no 32-bit sum can overflow.
+constexpr int kFold = 8192;
+
+template <int CS>
+__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads) select_kernel(DecodeArgs a) {
+  griddep_wait();
+  griddep_launch();
+  constexpr int kLgCap = SelCfg<CS>::kLgCap;
+  cg::cluster_group cl = cg::this_cluster();
+  const int rank = (int)cl.block_rank();
+  const int bh = blockIdx.y;
+  const int b = bh / a.NR;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  extern __shared__ __align__(16) unsigned char dsm[];
+  float* s_lg = reinterpret_cast<float*>(dsm);                                           // kLgCap
+  unsigned* s_hi = reinterpret_cast<unsigned*>(s_lg + kLgCap);                           // 2048
+  unsigned* s_lo = s_hi + kNumBuckets;                                                   // 2048
+  unsigned long long* s_h = reinterpret_cast<unsigned long long*>(s_lo + kNumBuckets);   // 2048
+  uint2* s_cand = reinterpret_cast<uint2*>(s_hi);  // leader, after the histogram is dead
+  unsigned long long* s_w = reinterpret_cast<unsigned long long*>(s_h + kNumBuckets);    // kBruteMax
+  SelShared<CS>* sh = reinterpret_cast<SelShared<CS>*>(s_w + kBruteMax);
+  __shared__ unsigned long long r_hm[256];
+  __shared__ unsigned r_hc[256];
+  __shared__ DigitResult s_dres;
+  __shared__ uint32_t s_kr[96];
+  __shared__ uint32_t s_min;
+  __shared__ int s_jmax;
+
+  const int L = a.seq_len[b];
+  if (!seq_ok(L, a)) return;  // uniform over the cluster; the stream kernel flagged it
+  const int per = (((L + CS - 1) / CS) + 31) & ~31;
+  const int j0 = min(L, rank * per);
+  const int j1 = min(L, j0 + per);
+  uint32_t* mask = a.mask + (size_t)bh * a.words;
+  const float* lg_g = a.logits + (size_t)bh * a.lstride;
+
+  if (a.top_p >= 1.0f) {  // keep every token
+    for (int w = (j0 >> 5) + tid; w < ((j1 + 31) >> 5); w += kSelThreads) {
+      const int nb = min(32, L - w * 32);
+      mask[w] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
+    }
+    if (rank == 0 && tid == 0 && a.sel_count) a.sel_count[bh] = L;
+    return;
+  }
+
+  // maximum score (per-chunk maxima of the stream kernel)
+  float m = -CUDART_INF_F;
+  {
+    const int nch = (L + kScoreChunk - 1) / kScoreChunk;
+    const float* cm = a.cmax + (size_t)bh * a.nch_score_max;
+    for (int c = tid; c < nch; c += kSelThreads) m = fmaxf(m, cm[c]);
+    m = block_max<kSelThreads>(m, sh->red);
+  }
+  // Scores are staged in shared memory kLgCap at a time with 16-byte loads
+  // issued together (rows are 16-byte aligned, j0 a multiple of 32); when the
+  // whole range fits, it is staged once and reused by every pass.
+  const bool cached = (j1 - j0) <= kLgCap;
+  auto stage = [&](int c0, int c1) {
+    const float4* src = reinterpret_cast<const float4*>(lg_g + c0);
+    float4* dst = reinterpret_cast<float4*>(s_lg);
+    const int nv = (c1 - c0 + 3) >> 2;
+#pragma unroll 8
+    for (int i = tid; i < nv; i += kSelThreads) dst[i] = __ldcg(src + i);
+  };
+  for (int i = tid; i < kNumBuckets; i += kSelThreads) { s_hi[i] = 0u; s_lo[i] = 0u; s_h[i] = 0ull; }
+  if (rank == 0 && tid == 0) sh->n_cand = 0u;
+  for (int c0 = j0; c0 < j1; c0 += kLgCap) {
+    const int c1 = min(j1, c0 + kLgCap);
+    __syncthreads();
+    stage(c0, c1);
+    __syncthreads();
+    for (int f0 = c0; f0 < c1; f0 += kFold) {
+      const int f1 = min(c1, f0 + kFold);
+      for (int j = f0 + tid; j < f1; j += kSelThreads) {
+        const float sv = s_lg[j - c0];
+        const unsigned long long w = sv > m - 25.0f ? mass_fx36(sv, m) : 0ull;  // e^-25 < 2^-36
+        if (w) {
+          const int bk = score_bucket(sv);
+          atomicAdd(&s_hi[bk], (unsigned)(w >> 18));
+          atomicAdd(&s_lo[bk], (unsigned)(w & 0x3ffffu));
+        }
+      }
+      __syncthreads();
+      for (int i = tid; i < kNumBuckets; i += kSelThreads) {  // fold into the 64-bit bins
+        s_h[i] += ((unsigned long long)s_hi[i] << 18) + s_lo[i];
+        s_hi[i] = 0u;
+        s_lo[i] = 0u;
+      }
+      __syncthreads();
+    }
+  }
+  cl.sync();  // (1) every rank's exact histogram is complete
+
+  // reduce this rank's slice of buckets over the cluster; broadcast its total
+  constexpr int NS = kNumBuckets / CS;
+  {
+    unsigned long long sm_ = 0ull;
+    if (tid < NS) {
+      const int bk = rank * NS + tid;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) sm_ += *cl.map_shared_rank(s_h + bk, q);
+      r_hm[tid] = sm_;
+    }
+    unsigned long long ex_m, tot_m;
+    unsigned ex_c, tot_c;
+    block_excl_scan2<kSelThreads>(sm_, 0u, ex_m, ex_c, tot_m, tot_c, sh->scan_a, sh->scan_c);
+    if (tid < CS) cl.map_shared_rank(sh, tid)->slice[rank] = tot_m;
+  }
+  cl.sync();  // (2) slice totals everywhere
+
+  unsigned long long target;
+  {  // exact boundary bucket: highest buckets live in the highest rank's slice
+    unsigned long long Z = 0ull;
+    for (int q = 0; q < CS; ++q) Z += sh->slice[q];
+    target = (unsigned long long)ceil((double)a.top_p * (double)Z);
+    if (target > Z) target = Z;
+    if (target < 1ull) target = 1ull;
+    int kslice = 0;
+    unsigned long long above_slice = 0ull;
+    for (int q = CS - 1; q >= 0; --q) {
+      if (above_slice + sh->slice[q] >= target) { kslice = q; break; }
+      above_slice += sh->slice[q];
+    }
+    if (rank == kslice && warp == 0) {
+      constexpr int PL = NS / 32;
+      unsigned long long w8[PL];
+      unsigned long long sw = 0ull;
+#pragma unroll
+      for (int k = 0; k < PL; ++k) {
+        w8[k] = r_hm[NS - 1 - (lane * PL + k)];
+        sw += w8[k];
+      }
+      const unsigned long long incl = warp_incl_scan_u64(sw);
+      unsigned long long cum = above_slice + incl - sw;
+      int found = -1;
+      unsigned long long fab = 0ull;
+#pragma unroll
+      for (int k = 0; k < PL; ++k) {
+        if (found < 0 && cum < target && cum + w8[k] >= target) {
+          found = rank * NS + NS - 1 - (lane * PL + k);
+          fab = cum;
+        }
+        cum += w8[k];
+      }
+      const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+      const int src = who ? __ffs(who) - 1 : 0;
+      found = who ? __shfl_sync(0xffffffffu, found, src) : -1;
+      fab = __shfl_sync(0xffffffffu, fab, src);
+      if (lane < CS) {
+        SelShared<CS>* rem = cl.map_shared_rank(sh, lane);
+        rem->bucket = found;
+        rem->zpart[0] = fab;  // mass above the boundary bucket
+      }
+    }
+  }
+  cl.sync();  // (3) boundary bucket everywhere
+
+  const int bucket = sh->bucket;
+  const unsigned long long above = sh->zpart[0];
+  uint2* gcand = a.cand + (size_t)bh * a.lstride;
+  if (bucket >= 0) {  // candidates of the boundary bucket -> scratch (order does not matter)
+    SelShared<CS>* lead = cl.map_shared_rank(sh, 0);
+    for (int c0 = j0; c0 < j1; c0 += kLgCap) {
+      const int c1 = min(j1, c0 + kLgCap);
+      if (!cached) {
+        __syncthreads();
+        stage(c0, c1);
+        __syncthreads();
+      }
+      for (int jb = c0; jb < c1; jb += kSelThreads) {
+        const int j = jb + tid;
+        float sv = 0.f;
+        bool in = false;
+        if (j < c1) {
+          sv = s_lg[j - c0];
+          in = score_bucket(sv) == bucket && sv > m - 25.0f && mass_fx36(sv, m) != 0ull;
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, in);
+        if (bal) {
+          unsigned base = 0u;
+          if (lane == 0) base = atomicAdd(&lead->n_cand, (unsigned)__popc(bal));
+          base = __shfl_sync(0xffffffffu, base, 0);
+          const unsigned slot = base + __popc(bal & ((1u << lane) - 1u));
+          if (in) gcand[slot] = make_uint2(score_key(sv), (unsigned)j);
+        }
+      }
+    }
+  }
+  __threadfence();
+  cl.sync();  // (4) candidates complete
+
+  if (rank == 0) {
+    float tau = -CUDART_INF_F;  // no boundary (unreachable): keep every token
+    int jcut = INT_MAX;
+    if (bucket >= 0) {
+      const int n = (int)sh->n_cand;
+      const unsigned long long need = target - above;
+      const uint2* items = gcand;
+      if (n <= kCandSmem) {  // stage them where the histogram was
+        for (int i = tid; i < n; i += kSelThreads) s_cand[i] = __ldcg(gcand + i);
+        __syncthreads();
+        items = s_cand;
+      }
+      if (n <= kBruteMax)
+        solve_brute(items, n, m, need, s_w, &s_min, &s_jmax, tau, jcut);
+      else
+        solve_radix(Items{items, nullptr, bucket}, n, m, need, r_hm, r_hc, &s_dres, s_kr, tau, jcut);
+    }
+    if (tid < CS) {
+      SelShared<CS>* rem = cl.map_shared_rank(sh, tid);
+      rem->tau = tau;
+      rem->jcut = jcut;
+    }
+  }
+  cl.sync();  // (5) final threshold everywhere (no DSMEM access after this)
+
+  const float tau = sh->tau;
+  const int jcut = sh->jcut;
+  int cnt = 0;
+  for (int c0 = j0; c0 < j1; c0 += kLgCap) {
+    const int c1 = min(j1, c0 + kLgCap);
+    if (!cached) {
+      __syncthreads();
+      stage(c0, c1);
+      __syncthreads();
+    }
+    for (int jb = c0; jb < c1; jb += kSelThreads) {
+      const int j = jb + tid;
+      bool in = false;
+      if (j < c1) {
+        const float sv = s_lg[j - c0];
+        in = sv > tau || (sv == tau && j <= jcut);
+      }
+      const unsigned word = __ballot_sync(0xffffffffu, in);
+      if (lane == 0 && jb + warp * 32 < c1) mask[(jb >> 5) + warp] = word;
+      cnt += in ? 1 : 0;
+    }
+  }
+  if (a.sel_count) {
+    cnt = warp_sum_i(cnt);
+    if (lane == 0 && cnt) atomicAdd(&a.sel_count[bh], cnt);
   }
 }
 
 // ---------------------------------------------------------------------------
-// 4. attention over sinks/window and kept rows, then the log-sum-exp merge
+// 3. gather kernel: kept rows outside sinks/window + log-sum-exp merge
 // ---------------------------------------------------------------------------
-template <int D, int G>
-struct AttnCfg {
-  static constexpr int kLpr = (G == 8 && D == 128) ? 16 : 8;  // lanes per row
-  static constexpr int kDpl = D / kLpr;                       // dims per lane
-  static constexpr int kGroups = kThreads / kLpr;             // rows in flight per CTA
-};
-
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) attn_kernel(DecodeArgs a) {
-  using C = AttnCfg<D, G>;
-  constexpr int LPR = C::kLpr, DPL = C::kDpl, NGRP = C::kGroups;
-  constexpr int kWarps = kThreads / 32;
+__global__ void __launch_bounds__(kThreads) gather_kernel(DecodeArgs a) {
+  griddep_wait();
+  griddep_launch();
+  // The row list and the warp-merge buffer are never live at the same time.
+  constexpr size_t kRowBytes = (size_t)kGatherTile * (sizeof(int) + 1);
+  constexpr size_t kMergeBytes = (size_t)kWarps * G * D * sizeof(float);
+  __shared__ __align__(16) unsigned char s_buf[kRowBytes > kMergeBytes ? kRowBytes : kMergeBytes];
+  __shared__ __align__(16) float s_q[G * D];
+  __shared__ float s_ml[kWarps * G * 2];
+  __shared__ unsigned s_wcnt[kWarps];
+  __shared__ int s_flag;
+  int* s_row = reinterpret_cast<int*>(s_buf);
+  unsigned char* s_msk = s_buf + (size_t)kGatherTile * sizeof(int);
+  float* s_o = reinterpret_cast<float*>(s_buf);
   const int tile = blockIdx.x;
   const int bkv = blockIdx.y;
   const int b = bkv / a.Hkv, h = bkv % a.Hkv;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int r = a.ret_rank[h];
-  const bool sel_tile = tile >= a.n_sw_tiles;
-
-  __shared__ float s_q[G][D];
-  __shared__ int s_row[kSelTile];
-  __shared__ unsigned char s_msk[kSelTile];
-  __shared__ int s_wcnt[kWarps];
-  __shared__ float s_o[kWarps][G][D];
-  __shared__ float s_m[kWarps][G], s_l[kWarps][G];
-  __shared__ int s_flag;
-
   const int L = a.seq_len[b];
-  const bool valid = seq_ok(L, a);
-  const int s_cnt = valid ? min(a.S, L) : 0;
-  const int sw0 = valid ? max(s_cnt, L - a.W) : 0;
-  const bool active = valid && (!sel_tile || r >= 0);
-  const size_t part0 = (size_t)bkv * a.n_tiles_max + tile;
-
-  if (!valid && tile == 0 && h == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
-
-  if (active) {
-    // RoPE'd query at position L-1, pre-scaled by log2(e)/sqrt(D)
-    const float qscale = 1.4426950408889634f * rsqrtf((float)D);
-    for (int i = tid; i < G * (D / 2); i += kThreads) {
-      const int g = i / (D / 2), k = i % (D / 2);
-      const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * G + g) * D;
-      const float x1 = to_f32(q[k]), x2 = to_f32(q[k + D / 2]);
-      float c, s;
-      rope_cos_sin(L - 1, k, D, a.rope_base, c, s);
-      s_q[g][k] = (x1 * c - x2 * s) * qscale;
-      s_q[g][k + D / 2] = (x2 * c + x1 * s) * qscale;
-    }
+  if (!seq_ok(L, a)) return;
+  const size_t pbase = (size_t)bkv * a.n_parts_max;
+  int n_parts = a.n_sw_tiles;
+  if (r >= 0) {
+    const int s_cnt = min(a.S, L);
+    const int sw0 = max(s_cnt, L - a.W);
+    const int jt0 = tile * kGatherTile;
     int n_rows = 0;
-    int e0 = 0;
-    if (!sel_tile) {
-      const int n_sw = s_cnt + (L - sw0);
-      e0 = tile * kSwTile;
-      n_rows = max(0, min(kSwTile, n_sw - e0));
-    } else {
-      // scan [j0, j0 + kSelTile) for kept rows; record bitmask / list
-      const int j0 = (tile - a.n_sw_tiles) * kSelTile;
-      float tau[G];
-      int jcut[G], mode[G];
+    if (jt0 < L) {
+      // union of the G heads' kept rows in [jt0, jt0 + kGatherTile), outside sinks/window
+      unsigned wg[G];
+      unsigned uni = 0u;
+      const int w = (jt0 >> 5) + tid;  // one 32-token word per thread
+      const int jw = w * 32;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const DecodeHead* hd = a.heads + (size_t)b * a.NR + r * G + g;
-        mode[g] = hd->mode;
-        tau[g] = hd->tau;
-        jcut[g] = hd->jcut;
-      }
-      const float* lg = a.logits + ((size_t)b * a.NR + (size_t)r * G) * a.Lmax;
-      int base = 0;
-      for (int it = 0; it < kSelTile; it += kThreads) {
-        const int j = j0 + it + tid;
-        unsigned msk = 0u;
+      for (int g = 0; g < G; ++g) wg[g] = 0u;
+      if (jw < L) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          bool in = false;
-          if (j < L) {
-            if (mode[g] == kModeAll) in = true;
-            else {
-              const float s = lg[(size_t)g * a.Lmax + j];
-              in = s > tau[g] || (s == tau[g] && j <= jcut[g]);
-            }
-          }
-          const unsigned word = __ballot_sync(0xffffffffu, in);
-          if (a.sel_bitmask && lane == 0 && (j >> 5) < a.words && j0 + it < a.max_seq_len)
-            a.sel_bitmask[((size_t)b * a.NR + r * G + g) * a.words + (j >> 5)] = word;
-          msk |= (in ? 1u : 0u) << g;
+          wg[g] = a.mask[((size_t)b * a.NR + r * G + g) * a.words + w];
+          uni |= wg[g];
         }
-        const bool att = msk != 0u && j >= s_cnt && j < sw0;
-        const unsigned bal = __ballot_sync(0xffffffffu, att);
-        if (lane == 0) s_wcnt[warp] = __popc(bal);
-        __syncthreads();
-        int off = base;
-        int tot = 0;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          if (w < warp) off += s_wcnt[w];
-          tot += s_wcnt[w];
+        // keep positions in [s_cnt, sw0): drop sinks, window and positions >= L
+        const int lo = max(0, s_cnt - jw), hi = min(32, sw0 - jw);
+        if (hi <= lo) uni = 0u;
+        else {
+          const unsigned keep_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+          const unsigned keep_lo = lo <= 0 ? 0xffffffffu : ~((1u << lo) - 1u);
+          uni &= keep_hi & keep_lo;
         }
-        if (att) {
-          const int p = off + __popc(bal & ((1u << lane) - 1u));
-          s_row[p] = j;
-          s_msk[p] = (unsigned char)msk;
-        }
-        base += tot;
-        __syncthreads();
       }
-      n_rows = base;
+      const unsigned cntw = __popc(uni);
+      unsigned incl = cntw;  // block exclusive scan of cntw, in index order
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned n2 = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n2;
+      }
+      if (lane == 31) s_wcnt[warp] = incl;
+      __syncthreads();
+      unsigned off = incl - cntw;
+      unsigned tot = 0u;
+#pragma unroll
+      for (int q = 0; q < kWarps; ++q) {
+        if (q < warp) off += s_wcnt[q];
+        tot += s_wcnt[q];
+      }
+      unsigned bits = uni;
+      while (bits) {
+        const int k = __ffs(bits) - 1;
+        bits &= bits - 1u;
+        unsigned msk = 0u;
+#pragma unroll
+        for (int g = 0; g < G; ++g) msk |= ((wg[g] >> k) & 1u) << g;
+        s_row[off] = jw + k;
+        s_msk[off] = (unsigned char)msk;
+        ++off;
+      }
+      n_rows = (int)tot;
+      __syncthreads();
     }
-    __syncthreads();
-
-    // ---- rows: LPR lanes per row, DPL dims per lane ----
-    const int grp = tid / LPR, sub = tid % LPR;
-    float qv[G][DPL];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int d = 0; d < DPL; ++d) qv[g][d] = s_q[g][sub * DPL + d];
-    float mrun[G], lrun[G], o[G][DPL];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      mrun[g] = -CUDART_INF_F;
-      lrun[g] = 0.f;
-#pragma unroll
-      for (int d = 0; d < DPL; ++d) o[g][d] = 0.f;
-    }
-    const T* kbase = static_cast<const T*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D + sub * DPL;
-    const T* vbase = static_cast<const T*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D + sub * DPL;
-    // Every lane runs the same trip count (the shuffles below name the whole
-    // warp); rows past n_rows are masked out.
-    const int n_iter = (n_rows + NGRP - 1) / NGRP;
-    for (int itr = 0; itr < n_iter; ++itr) {
-      const int e = itr * NGRP + grp;
-      int row = 0;
-      unsigned msk = 0u;
-      if (e < n_rows) {
-        if (!sel_tile) {
-          const int idx = e0 + e;
-          row = idx < s_cnt ? idx : sw0 + (idx - s_cnt);
-          msk = (1u << G) - 1u;
-        } else {
-          row = s_row[e];
-          msk = s_msk[e];
+    if (n_rows > 0) {
+      WarpAttn<T, D, G> wa;
+      wa.init();
+      const T* kb = static_cast<const T*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+      const T* vb = static_cast<const T*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+      const int n_it = (n_rows + kThreads - 1) / kThreads;  // same trip count in every warp
+      {
+        const int e = warp * 32 + lane;
+        const bool ok = e < n_rows;
+        wa.load(kb, vb, ok ? s_row[e] : 0, ok ? (unsigned)s_msk[e] : 0u);  // in flight during RoPE
+      }
+      rope_query<T, D, G>(a, b, h, L - 1, s_q);
+      __syncthreads();
+      for (int it = 0; it < n_it; ++it) {
+        if (it > 0) {
+          const int e = it * kThreads + warp * 32 + lane;
+          const bool ok = e < n_rows;
+          wa.load(kb, vb, ok ? s_row[e] : 0, ok ? (unsigned)s_msk[e] : 0u);
         }
+        wa.compute(s_q);
       }
-      RawRow<T, DPL> kr, vr;
-      kr.load(kbase + (size_t)row * D);  // row 0 always exists (L >= 1)
-      vr.load(vbase + (size_t)row * D);
-      float sc[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float acc = 0.f;
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) acc = fmaf(qv[g][d], kr.get(d), acc);
-        sc[g] = acc;
-      }
-#pragma unroll
-      for (int off = 1; off < LPR; off <<= 1)
-#pragma unroll
-        for (int g = 0; g < G; ++g) sc[g] += __shfl_xor_sync(0xffffffffu, sc[g], off);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        if ((msk >> g) & 1u) {
-          const float mn = fmaxf(mrun[g], sc[g]);
-          const float al = exp2f(mrun[g] - mn);
-          const float p = exp2f(sc[g] - mn);
-          lrun[g] = lrun[g] * al + p;
-#pragma unroll
-          for (int d = 0; d < DPL; ++d) o[g][d] = fmaf(p, vr.get(d), o[g][d] * al);
-          mrun[g] = mn;
-        }
-      }
+      __syncthreads();  // the row list is dead; its bytes become the merge buffer
+      write_partial<D, G>(a, wa, pbase + a.n_sw_tiles + tile, s_o, s_ml);
+    } else if (tid < G) {
+      a.pm[(pbase + a.n_sw_tiles + tile) * G + tid] = -CUDART_INF_F;
+      a.pl[(pbase + a.n_sw_tiles + tile) * G + tid] = 0.f;
     }
-    // merge the row groups of a warp (lanes differing in bits >= log2(LPR))
-#pragma unroll
-    for (int off = LPR; off < 32; off <<= 1) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float mo = __shfl_xor_sync(0xffffffffu, mrun[g], off);
-        const float lo = __shfl_xor_sync(0xffffffffu, lrun[g], off);
-        const float mn = fmaxf(mrun[g], mo);
-        const float al = (mn == -CUDART_INF_F) ? 0.f : exp2f(mrun[g] - mn);
-        const float be = (mn == -CUDART_INF_F) ? 0.f : exp2f(mo - mn);
-        lrun[g] = lrun[g] * al + lo * be;
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) {
-          const float oo = __shfl_xor_sync(0xffffffffu, o[g][d], off);
-          o[g][d] = o[g][d] * al + oo * be;
-        }
-        mrun[g] = mn;
-      }
-    }
-    if (lane < LPR) {
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-#pragma unroll
-        for (int d = 0; d < DPL; ++d) s_o[warp][g][lane * DPL + d] = o[g][d];
-        if (lane == 0) { s_m[warp][g] = mrun[g]; s_l[warp][g] = lrun[g]; }
-      }
-    }
-    __syncthreads();
-    for (int i = tid; i < G * D; i += kThreads) {
-      const int g = i / D, d = i % D;
-      float mn = -CUDART_INF_F;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) mn = fmaxf(mn, s_m[w][g]);
-      float acc = 0.f, den = 0.f;
-      if (mn != -CUDART_INF_F) {
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          const float sc = exp2f(s_m[w][g] - mn);
-          acc = fmaf(s_o[w][g][d], sc, acc);
-          den = fmaf(s_l[w][g], sc, den);
-        }
-      }
-      a.po[(part0 * G + g) * D + d] = acc;
-      if (d == 0) {
-        a.pm[part0 * G + g] = mn;
-        a.pl[part0 * G + g] = den;
-      }
+    if (!take_ticket(&a.ctl[bkv], gridDim.x, &s_flag)) return;
+    n_parts = a.n_sw_tiles + gridDim.x;
+  } else if (tile != 0) {
+    return;  // local KV heads: tile 0 merges the sink/window partials
+  }
+  // ---- merge all partials of this KV head ----
+  float* s_pm = s_o;  // [n_parts][G] (reuse)
+  float* s_pl = s_o + a.n_parts_max * G;
+  __syncthreads();
+  for (int i = tid; i < n_parts * G; i += kThreads) {
+    s_pm[i] = __ldcg(a.pm + pbase * G + i);
+    s_pl[i] = __ldcg(a.pl + pbase * G + i);
+  }
+  __syncthreads();
+  if (tid < G) {  // per-part weights exp2(m_t - max) (0 for empty parts)
+    float mn = -CUDART_INF_F;
+    for (int t = 0; t < n_parts; ++t) mn = fmaxf(mn, s_pm[t * G + tid]);
+    for (int t = 0; t < n_parts; ++t) {
+      const float pmv = s_pm[t * G + tid];
+      s_pm[t * G + tid] = (pmv == -CUDART_INF_F) ? 0.f : exp2f(pmv - mn);
     }
   }
-
-  if (!take_ticket(&tick_attn(a)[bkv], gridDim.x, &s_flag)) return;
-  if (!valid) return;
-  // ---- merge the tiles of this KV head into out ----
-  const int n_parts = (r >= 0) ? (int)gridDim.x : a.n_sw_tiles;
-  const size_t pbase = (size_t)bkv * a.n_tiles_max;
+  __syncthreads();
   for (int i = tid; i < G * D; i += kThreads) {
     const int g = i / D, d = i % D;
-    float mn = -CUDART_INF_F;
-    for (int t = 0; t < n_parts; ++t) mn = fmaxf(mn, __ldcg(a.pm + (pbase + t) * G + g));
     float acc = 0.f, den = 0.f;
+#pragma unroll 8
     for (int t = 0; t < n_parts; ++t) {
-      const float pmv = __ldcg(a.pm + (pbase + t) * G + g);
-      if (pmv == -CUDART_INF_F) continue;
-      const float sc = exp2f(pmv - mn);
-      acc = fmaf(__ldcg(a.po + ((pbase + t) * G + g) * D + d), sc, acc);
-      den = fmaf(__ldcg(a.pl + (pbase + t) * G + g), sc, den);
+      const float sc = s_pm[t * G + g];
+      const float pv = __ldcg(a.po + ((pbase + t) * G + g) * D + d);  // stale if sc == 0
+      acc = sc > 0.f ? fmaf(pv, sc, acc) : acc;
+      den = fmaf(s_pl[t * G + g], sc, den);
     }
     T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + h * G + g) * D + d;
     *out = from_f32<T>(acc / den);
   }
 }
 
-template <typename T, int G>
-void launch_score(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  score_kernel<T, G><<<grid, kThreads, 0, st>>>(a);
+// ---------------------------------------------------------------------------
+// launch helpers
+// ---------------------------------------------------------------------------
+cudaError_t launch_pdl(void (*k)(DecodeArgs), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       const DecodeArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, a);
+}
+
+template <typename T, int D, int G>
+cudaError_t launch_dg(const DecodeArgs& a, int kind, dim3 grid, cudaStream_t st) {
+  if (kind == 0) return launch_pdl(stream_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
+  return launch_pdl(gather_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
 }
 
 template <typename T, int D>
-void launch_attn_g(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
+cudaError_t launch_d(const DecodeArgs& a, int kind, dim3 grid, cudaStream_t st) {
   switch (a.G) {
-    case 1: attn_kernel<T, D, 1><<<grid, kThreads, 0, st>>>(a); break;
-    case 2: attn_kernel<T, D, 2><<<grid, kThreads, 0, st>>>(a); break;
-    case 4: attn_kernel<T, D, 4><<<grid, kThreads, 0, st>>>(a); break;
-    default: attn_kernel<T, D, 8><<<grid, kThreads, 0, st>>>(a); break;
+    case 1: return launch_dg<T, D, 1>(a, kind, grid, st);
+    case 2: return launch_dg<T, D, 2>(a, kind, grid, st);
+    case 4: return launch_dg<T, D, 4>(a, kind, grid, st);
+    default: return launch_dg<T, D, 8>(a, kind, grid, st);
   }
 }
 
-template <typename T>
-void launch_score_g(const DecodeArgs& a, dim3 grid, cudaStream_t st) {
-  switch (a.G) {
-    case 1: launch_score<T, 1>(a, grid, st); break;
-    case 2: launch_score<T, 2>(a, grid, st); break;
-    case 4: launch_score<T, 4>(a, grid, st); break;
-    default: launch_score<T, 8>(a, grid, st); break;
-  }
+cudaError_t launch_kind(const Shape& sh, const DecodeArgs& a, int kind, dim3 grid, cudaStream_t st) {
+  if (sh.dtype == RTP_BF16)
+    return sh.D == 128 ? launch_d<__nv_bfloat16, 128>(a, kind, grid, st)
+                       : launch_d<__nv_bfloat16, 64>(a, kind, grid, st);
+  return sh.D == 128 ? launch_d<float, 128>(a, kind, grid, st) : launch_d<float, 64>(a, kind, grid, st);
+}
+
+// Cluster size of the select kernel on each device: 16 CTAs where the device
+// can co-schedule several such clusters with the kernel's shared memory, else 8.
+int select_cluster_size() {
+  static int s_cs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
+  if (s_cs[dev]) return s_cs[dev];
+  cudaFuncSetAttribute(select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<8>::kSmem);
+  cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<16>::kSmem);
+  cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  int cs = 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(16, 1);
+  cfg.blockDim = dim3(kSelThreads);
+  cfg.dynamicSmemBytes = SelCfg<16>::kSmem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 16;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n_clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&n_clusters, select_kernel<16>, &cfg) == cudaSuccess && n_clusters >= 4)
+    cs = 16;
+  cudaGetLastError();  // clear a refused query
+  s_cs[dev] = cs;
+  return cs;
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -769,19 +1151,21 @@ DecodeLayout decode_layout(const Shape& sh) {
   DecodeLayout l;
   const size_t NRt = (size_t)sh.B * sh.NR;
   l.nch_score_max = (sh.Lmax + kScoreChunk - 1) / kScoreChunk;
-  l.nch_sel_max = (sh.Lmax + kSelChunk - 1) / kSelChunk;
+  l.nch_sel_max = (sh.Lmax + kGatherTile - 1) / kGatherTile;
   l.n_sw_tiles = (sh.S + sh.W + kSwTile - 1) / kSwTile;
-  l.n_sel_tiles_max = (sh.Lmax + kSelTile - 1) / kSelTile;
+  l.n_sel_tiles_max = (sh.Lmax + kGatherTile - 1) / kGatherTile;
   l.n_tiles_max = l.n_sw_tiles + (sh.R > 0 ? l.n_sel_tiles_max : 0);
-  l.n_ctl = (int)(3 * NRt + (size_t)sh.B * sh.Hkv);
+  l.n_ctl = (int)((size_t)sh.B * sh.Hkv);
+  const size_t words = (size_t)(sh.Lmax + 31) / 32;
+  const size_t lstride = ((size_t)sh.Lmax + 31) & ~size_t(31);
   size_t off = 0;
-  l.logits = off; off = align256(off + NRt * sh.Lmax * sizeof(float));
+  l.logits = off; off = align256(off + NRt * lstride * sizeof(float));
   l.cmax = off;   off = align256(off + NRt * l.nch_score_max * sizeof(float));
-  l.hmass = off;  off = align256(off + NRt * kNumBuckets * sizeof(unsigned long long));
-  l.hcnt = off;   off = align256(off + NRt * kNumBuckets * sizeof(unsigned));
-  l.heads = off;  off = align256(off + NRt * sizeof(DecodeHead));
+  l.hmass = off;  off = align256(off + NRt * words * sizeof(uint32_t));  // scratch bitmask
+  l.hcnt = off;
+  l.heads = off;
   l.ctl = off;    off = align256(off + (size_t)l.n_ctl * sizeof(unsigned));
-  l.cand = off;   off = align256(off + NRt * sh.Lmax * sizeof(uint2));
+  l.cand = off;   off = align256(off + NRt * lstride * sizeof(uint2));
   const size_t nparts = (size_t)sh.B * sh.Hkv * l.n_tiles_max * sh.G;
   l.pm = off;     off = align256(off + nparts * sizeof(float));
   l.pl = off;     off = align256(off + nparts * sizeof(float));
@@ -798,56 +1182,49 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   a.Lmax = sh.Lmax; a.S = sh.S; a.W = sh.W;
   a.max_seq_len = max_seq_len > 0 ? max_seq_len : sh.Lmax;
   a.words = (sh.Lmax + 31) / 32;
+  a.lstride = (sh.Lmax + 31) & ~31;
   a.top_p = sh.top_p; a.rope_base = sh.rope_base;
   a.q_pre = q_pre; a.w_q = w_q; a.out = out;
   a.k = cache->k; a.v = cache->v; a.kidx = cache->kidx; a.status = cache->status;
-  a.seq_len = seq_len; a.sel_bitmask = sel_bitmask; a.sel_count = sel_count;
+  a.seq_len = seq_len; a.sel_count = sel_count;
   char* w = static_cast<char*>(ws);
   a.logits = reinterpret_cast<float*>(w + lay.logits);
   a.cmax = reinterpret_cast<float*>(w + lay.cmax);
-  a.hmass = reinterpret_cast<unsigned long long*>(w + lay.hmass);
-  a.hcnt = reinterpret_cast<unsigned*>(w + lay.hcnt);
-  a.heads = reinterpret_cast<DecodeHead*>(w + lay.heads);
+  a.mask = sel_bitmask ? sel_bitmask : reinterpret_cast<uint32_t*>(w + lay.hmass);
   a.ctl = reinterpret_cast<unsigned*>(w + lay.ctl);
   a.cand = reinterpret_cast<uint2*>(w + lay.cand);
   a.pm = reinterpret_cast<float*>(w + lay.pm);
   a.pl = reinterpret_cast<float*>(w + lay.pl);
   a.po = reinterpret_cast<float*>(w + lay.po);
   a.n_ctl = lay.n_ctl; a.nch_score_max = lay.nch_score_max; a.n_sw_tiles = lay.n_sw_tiles;
-  a.n_tiles_max = lay.n_tiles_max;
+  a.n_parts_max = lay.n_tiles_max;
   for (int i = 0; i < kMaxRetrieval; ++i) { a.ret_head[i] = sh.ret_head[i]; a.ret_rank[i] = sh.ret_rank[i]; }
 
   const int Lh = a.max_seq_len;
   const int nch_score = (Lh + kScoreChunk - 1) / kScoreChunk;
-  const int nch_sel = (Lh + kSelChunk - 1) / kSelChunk;
-  const int n_sel_tiles = (Lh + kSelTile - 1) / kSelTile;
-  if (sh.R > 0) {
-    const dim3 gs(nch_score, sh.B * sh.R);
-    trace_begin(RTP_STAGE_DECODE_SCORE, st);
-    if (sh.dtype == RTP_BF16) launch_score_g<__nv_bfloat16>(a, gs, st);
-    else launch_score_g<float>(a, gs, st);
-    trace_end(RTP_STAGE_DECODE_SCORE, st);
-    const dim3 gh(nch_sel, sh.B * sh.NR);
-    trace_begin(RTP_STAGE_DECODE_HIST, st);
-    hist_kernel<<<gh, kThreads, 0, st>>>(a);
-    trace_end(RTP_STAGE_DECODE_HIST, st);
+  const int n_gtiles = (Lh + kGatherTile - 1) / kGatherTile;
+  a.n_score_ctas = sh.R > 0 ? sh.B * sh.R * nch_score : 0;
+  a.n_sw_ctas = sh.B * sh.Hkv * lay.n_sw_tiles;
+  const int cs = sh.R > 0 ? select_cluster_size() : 8;
+
+  cudaError_t e;
+  trace_begin(RTP_STAGE_DECODE_STREAM, st);
+  e = launch_kind(sh, a, 0, dim3(a.n_score_ctas + a.n_sw_ctas), st);
+  trace_end(RTP_STAGE_DECODE_STREAM, st);
+  if (e == cudaSuccess && sh.R > 0) {
     trace_begin(RTP_STAGE_DECODE_SELECT, st);
-    collect_kernel<<<gh, kThreads, 0, st>>>(a);
+    if (cs == 16)
+      e = launch_pdl(select_kernel<16>, dim3(16, sh.B * sh.NR), dim3(kSelThreads), SelCfg<16>::kSmem, st, a);
+    else
+      e = launch_pdl(select_kernel<8>, dim3(8, sh.B * sh.NR), dim3(kSelThreads), SelCfg<8>::kSmem, st, a);
     trace_end(RTP_STAGE_DECODE_SELECT, st);
-  } else {
-    cudaMemsetAsync(a.ctl, 0, (size_t)a.n_ctl * sizeof(unsigned), st);
   }
-  const dim3 ga(lay.n_sw_tiles + (sh.R > 0 ? n_sel_tiles : 0), sh.B * sh.Hkv);
-  trace_begin(RTP_STAGE_DECODE_ATTN, st);
-  if (sh.dtype == RTP_BF16) {
-    if (sh.D == 128) launch_attn_g<__nv_bfloat16, 128>(a, ga, st);
-    else launch_attn_g<__nv_bfloat16, 64>(a, ga, st);
-  } else {
-    if (sh.D == 128) launch_attn_g<float, 128>(a, ga, st);
-    else launch_attn_g<float, 64>(a, ga, st);
+  if (e == cudaSuccess) {
+    trace_begin(RTP_STAGE_DECODE_GATHER, st);
+    e = launch_kind(sh, a, 1, dim3(sh.R > 0 ? n_gtiles : 1, sh.B * sh.Hkv), st);
+    trace_end(RTP_STAGE_DECODE_GATHER, st);
   }
-  trace_end(RTP_STAGE_DECODE_ATTN, st);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("decode launch: ") + cudaGetErrorString(e));
     return RTP_ERR_CUDA;

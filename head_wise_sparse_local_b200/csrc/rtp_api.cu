@@ -180,6 +180,8 @@ int rtp_decode_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void
   if (sh.R > 0 && !w_q) return fail(RTP_ERR_INVALID, "w_q is NULL with retrieval heads");
   if (max_seq_len < 0 || max_seq_len > sh.Lmax)
     return fail(RTP_ERR_SHAPE, "max_seq_len must be in [0, max_ctx]");
+  if (!aligned16(q_pre) || (w_q && !aligned16(w_q)))
+    return fail(RTP_ERR_INVALID, "q_pre and w_q must be 16-byte aligned");
   const DecodeLayout lay = decode_layout(sh);
   if (!workspace) return fail(RTP_ERR_WORKSPACE, "workspace is NULL");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
@@ -201,6 +203,8 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
   if (T < 1 || T > sh.Lmax) return fail(RTP_ERR_SHAPE, "T must be in [1, max_ctx]");
   if (!q_pre || !start_pos || !out) return fail(RTP_ERR_INVALID, "q_pre/start_pos/out is NULL");
   if (sh.R > 0 && !w_q) return fail(RTP_ERR_INVALID, "w_q is NULL with retrieval heads");
+  if (!aligned16(q_pre) || (w_q && !aligned16(w_q)))
+    return fail(RTP_ERR_INVALID, "q_pre and w_q must be 16-byte aligned");
   const PrefillLayout lay = prefill_layout(sh, T);
   if (!workspace) return fail(RTP_ERR_WORKSPACE, "workspace is NULL");
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)

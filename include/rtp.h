@@ -24,6 +24,8 @@
  *     the cache) never trap: the kernels skip the offending sequence/row and
  *     OR an RTP_DEV_* bit into *cache->status, which the caller reads back
  *     when it wants (it is never cleared by the library).
+ *   - Device buffers must be 16-byte aligned (torch and cudaMalloc allocations
+ *     are); a misaligned pointer returns RTP_ERR_INVALID.
  *   - Layouts are dense row-major in the order written, e.g. K [B][Hkv][Lmax][D]
  *     means element (b, h, j, d) sits at ((b*Hkv + h)*Lmax + j)*D + d.
  *   - Element type of q, k, v, out and of the caches is cfg->dtype (bf16 or
@@ -222,13 +224,12 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
 /* Kernel stages, for rtp_trace_stage. */
 typedef enum rtp_stage {
   RTP_STAGE_APPEND = 0,         /* rtp_append_kv: RoPE + cache + indexer-key store */
-  RTP_STAGE_DECODE_SCORE = 1,   /* decode: indexer scores over the 16-d key cache */
-  RTP_STAGE_DECODE_HIST = 2,    /* decode: softmax-mass histogram + boundary bucket */
-  RTP_STAGE_DECODE_SELECT = 3,  /* decode: boundary candidates + exact threshold */
-  RTP_STAGE_DECODE_ATTN = 4,    /* decode: gathered attention + log-sum-exp merge */
-  RTP_STAGE_PREFILL_INDEX = 5,  /* prefill: indexer score/threshold passes */
-  RTP_STAGE_PREFILL_ATTN = 6,   /* prefill: masked causal attention */
-  RTP_STAGE_COUNT = 7
+  RTP_STAGE_DECODE_STREAM = 1,  /* decode: indexer scores + sink/window attention */
+  RTP_STAGE_DECODE_SELECT = 2,  /* decode: exact top-p threshold + selection bitmask */
+  RTP_STAGE_DECODE_GATHER = 3,  /* decode: kept-row attention + log-sum-exp merge */
+  RTP_STAGE_PREFILL_INDEX = 4,  /* prefill: indexer score/threshold passes */
+  RTP_STAGE_PREFILL_ATTN = 5,   /* prefill: masked causal attention */
+  RTP_STAGE_COUNT = 6
 } rtp_stage;
 
 /* Host.  Optional instrumentation (no work is skipped or added).  Arms a

@@ -145,3 +145,39 @@ def test_decode_1m_full_size():
     inp = make_decode_inputs(workload("decode_1m_bf16"))
     st = check_decode_parity(inp)
     assert st["exact"] >= st["heads"] - 1
+
+
+@pytest.mark.parametrize("n_tied,p", [(300, 0.5), (2000, 0.3), (2000, 0.9)])
+def test_decode_large_tie_blocks(n_tied, p):
+    """Many identical indexer keys near the boundary: exercises the exact solve
+    over small and large candidate sets (pairwise ranks / radix passes)."""
+    inp = _small(ctx=12000, needles=8)
+    sh = inp["shape"]
+    h = sh.retrieval[1]
+    src = int(inp["needles"][0][1][1])  # a needle aimed at q head h*G + 1
+    inp["k_pre"][0, 200:200 + n_tied, h] = inp["k_pre"][0, src, h]
+    g = run_gpu_decode(inp, top_p=p)
+    oc = oracle_cache_from_inputs(inp)
+    oc.shape = sh.replace(top_p=p)
+    hq = h * sh.group + 1
+    _, topp_o, _ = oracle.decode(oc, inp["q_pre"], inp["seq_len"], inp["w_q"], heads=[hq])
+    gset = bitmask_to_sets(g["bitmask"][0], [12000] * (sh.n_retrieval * sh.group))[sh.group + 1]
+    assert np.array_equal(gset, topp_o[(0, hq)]), (len(gset), len(topp_o[(0, hq)]))
+
+
+@pytest.mark.parametrize("p", [0.5, 0.77])
+def test_decode_all_scores_equal(p):
+    """Every indexer key identical: one bucket holds all 20000 scores (more than
+    the leader's candidate buffer), so the exact solve scans every score; the
+    kept set is the first ceil(p * L) tokens."""
+    inp = _small(ctx=20000, needles=0)
+    sh = inp["shape"]
+    for h in sh.retrieval:
+        inp["k_pre"][0, :, h] = inp["k_pre"][0, 0, h]
+    g = run_gpu_decode(inp, top_p=p)
+    L = 20000
+    want = int(np.ceil(p * L - 1e-9))
+    sets = bitmask_to_sets(g["bitmask"][0], [L] * (sh.n_retrieval * sh.group))
+    for s in sets:
+        assert np.array_equal(s, np.arange(want)), (len(s), want)
+    check_decode_parity(inp, top_p=p)
