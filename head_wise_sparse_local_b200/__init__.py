@@ -128,12 +128,14 @@ def rtp_decode_attn_noalloc(cfg, cache, q_pre, seq_len, max_seq_len, w_q, out, s
                                             _ptr(sel_bitmask), _ptr(sel_count), _stream(stream)))
 
 
-def rtp_prefill_attn(cfg, cache, q_pre, start_pos, T, w_q, out, sel_tau=None, sel_jcut=None,
-                     sel_count=None, workspace=None, workspace_bytes=0, stream=None) -> None:
+def rtp_prefill_attn(cfg, cache, q_pre, start_pos, T, w_q, out, sel_bitmask=None, sel_tau=None,
+                     sel_jcut=None, sel_count=None, workspace=None, workspace_bytes=0,
+                     stream=None) -> None:
     _abi.check(_lib.rtp_prefill_attn(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q_pre),
-                                     _ptr(start_pos), int(T), _ptr(w_q), _ptr(out), _ptr(sel_tau),
-                                     _ptr(sel_jcut), _ptr(sel_count), _ptr(workspace),
-                                     int(workspace_bytes), _stream(stream)))
+                                     _ptr(start_pos), int(T), _ptr(w_q), _ptr(out),
+                                     _ptr(sel_bitmask), _ptr(sel_tau), _ptr(sel_jcut),
+                                     _ptr(sel_count), _ptr(workspace), int(workspace_bytes),
+                                     _stream(stream)))
 
 
 class Layer:
@@ -174,12 +176,12 @@ class Layer:
         rtp_decode_attn(self.cfg, self.cache, q_pre, seq_len, max_seq_len, w_q, out, sel_bitmask,
                         sel_count, self.ws_decode, self.ws_decode_bytes, stream)
 
-    def prefill(self, q_pre, start_pos, w_q, out, sel_tau=None, sel_jcut=None, sel_count=None,
-                stream=None) -> None:
+    def prefill(self, q_pre, start_pos, w_q, out, sel_bitmask=None, sel_tau=None, sel_jcut=None,
+                sel_count=None, stream=None) -> None:
         T = q_pre.shape[1]
         self.reserve_prefill(T)
-        rtp_prefill_attn(self.cfg, self.cache, q_pre, start_pos, T, w_q, out, sel_tau, sel_jcut,
-                         sel_count, self.ws_prefill, self.ws_prefill_bytes, stream)
+        rtp_prefill_attn(self.cfg, self.cache, q_pre, start_pos, T, w_q, out, sel_bitmask, sel_tau,
+                         sel_jcut, sel_count, self.ws_prefill, self.ws_prefill_bytes, stream)
 
     def device_status(self) -> int:
         return int(self.status.item())

@@ -71,7 +71,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rtp_prefill_workspace_bytes.argtypes = [cfgp, i32, P(sz)]
     lib.rtp_append_kv.argtypes = [cfgp, cachep, vp, vp, vp, i32, vp, vp]
     lib.rtp_decode_attn.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
-    lib.rtp_prefill_attn.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.rtp_prefill_attn.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.rtp_trace_stage.argtypes = [i32, vp, vp]
     lib.rtp_decode_attn_noalloc.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp]
     for name in EXPORTS:

@@ -50,7 +50,7 @@ struct PrefillLayout {
 };
 PrefillLayout prefill_layout(const Shape& sh, int T);
 int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* start_pos,
-                   int T, const float* w_q, void* out, float* sel_tau, int* sel_jcut,
-                   int* sel_count, void* ws, const PrefillLayout& lay, cudaStream_t st);
+                   int T, const float* w_q, void* out, uint32_t* sel_bitmask, float* sel_tau,
+                   int* sel_jcut, int* sel_count, void* ws, const PrefillLayout& lay, cudaStream_t st);
 
 }  // namespace rtp

@@ -1,24 +1,746 @@
-// rtp_prefill_attn: causal prefill chunk (work in progress).
+// rtp_prefill_attn: one causal prefill chunk of the head-wise sparse attention
+// layer.  Every query row does what a decode step at its position does
+// (atlas.scime.ai summary, "Approach"; abstract, observations (2)-(3)).
+//
+//   select_rows_kernel  retrieval query heads only.  One warp per query row,
+//       8 rows per CTA sharing the 16-d indexer-key tiles staged in shared
+//       memory.  Scores use the same fp32 FMA sequence as the decode path,
+//       so a row's selection equals the decode selection at that position.
+//       The exact top-p threshold is found by splitting the score interval
+//       that contains the boundary 8 ways per pass, with the softmax mass
+//       exp(s - max) of every score in 2^-36 fixed point (exact integer sums
+//       in registers), until at most kCand tokens remain; a warp-level exact
+//       solve finishes (ties to the lower index).  The row's top-p set is
+//       written as a bitmask.
+//   attn_rows_kernel  tensor-core (mma.sync m16n8k16 bf16, fp32 accumulate)
+//       flash attention over 64-row query tiles and 64-key tiles, masked by
+//       causality, sinks, the window and (retrieval heads) the bitmask; key
+//       tiles holding nothing a row keeps are skipped.
+#include <climits>
+
 #include "common.cuh"
 #include "internal.h"
 
 namespace rtp {
+namespace {
+
+constexpr int kSelRows = 8;       // query rows (warps) per selection CTA
+constexpr int kKeyTile = 256;     // indexer keys staged per step
+constexpr int kCand = 256;        // tokens the exact solve takes per row
+constexpr int kBQ = 64;           // attention: query rows per CTA (16 per warp)
+constexpr int kBK = 64;           // attention: keys per tile
+
+struct PrefillArgs {
+  int B, Hq, Hkv, G, D, R, NR, Lmax, S, W, T, words;
+  float top_p, rope_base;
+  const void* q_pre;
+  const float* w_q;
+  void* out;
+  const void* k;
+  const void* v;
+  const void* kidx;
+  int* status;
+  const int* start_pos;
+  float* sel_tau;
+  int* sel_jcut;
+  int* sel_count;
+  uint32_t* mask;  // [B][NR][T][words] top-p bitmask per query row
+  int ret_head[kMaxRetrieval];
+  int ret_rank[kMaxRetrieval];
+};
+
+__device__ __forceinline__ unsigned long long mass36(float s, float m) {
+  return __float2ull_rn(expf(s - m) * 68719476736.0f);  // 2^36
+}
+__device__ __forceinline__ unsigned long long wsum64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ unsigned wsum32(unsigned v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float wmaxf(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ unsigned wminu(unsigned v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ unsigned wmaxu(unsigned v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// What a row's warp does with each of its scores in one pass over its keys.
+enum : int {
+  kOpMax = 0,    // row maximum
+  kOpSplit = 1,  // mass/count of the 8 sub-intervals of the current interval
+  kOpRange = 2,  // min/max order key inside the current interval
+  kOpCand = 3,   // collect the current interval's tokens for the exact solve
+  kOpTies = 4,   // count tied tokens with index <= probe (index bisection)
+  kOpEmit = 5,   // write the top-p bitmask
+  kOpDone = 6
+};
+
+// Per-row selection state (kept identical in every lane of the row's warp).
+struct RowSel {
+  float m;                   // row maximum score
+  unsigned long long need;   // mass still needed inside the current interval
+  unsigned cnt_above;        // tokens ordered before the current interval
+  unsigned cnt_in;           // tokens inside the current interval
+  // current interval: d = m - s in [dlo, dhi) (dhi < 0: no upper bound) and
+  // order key in [klo, khi]
+  float dlo, dhi;
+  unsigned klo, khi;
+  bool by_key;               // split on order keys (d can no longer be split)
+  bool first;                // first split: also sums the total mass Z
+  float th[7];               // thresholds of the 8 sub-intervals (d or key as float bits)
+  unsigned kth[7];
+  // ties: all remaining tokens share one key; keep the first `need_ties` by index
+  unsigned tie_key, need_ties, tie_lo, tie_hi;
+  float tau;
+  int jcut;
+  unsigned count;
+  int op;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kSelRows * 32) select_rows_kernel(PrefillArgs a) {
+  __shared__ __align__(16) __nv_bfloat16 s_k[kKeyTile * kIdxDim];
+  __shared__ uint2 s_cand[kSelRows][kCand];
+  __shared__ unsigned long long s_cw[kSelRows][kCand];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.y;
+  const int b = bh / a.NR, hh = bh % a.NR;
+  const int r = hh / a.G, g = hh % a.G;
+  const int h = a.ret_head[r];
+  const int t = blockIdx.x * kSelRows + warp;
+  const int start = a.start_pos[b];
+  if (start < 0 || start + a.T > a.Lmax) {
+    if (threadIdx.x == 0 && blockIdx.x == 0 && hh == 0) atomicOr(a.status, RTP_DEV_POSITION);
+    return;  // uniform over the CTA
+  }
+  const bool row_ok = t < a.T;
+  const int i = start + t;  // query position; keys [0, i]
+  const int i_last = start + min(a.T, (int)(blockIdx.x + 1) * kSelRows) - 1;
+
+  // q~ = W_q q_pre with the decode path's association: four quarter sums of
+  // D/4 dims each, then butterfly adds.
+  float qi[kIdxDim];
+  {
+    constexpr int DQ = D / 4;
+    float part[2];
+#pragma unroll
+    for (int it = 0; it < 2; ++it) {
+      const int task = it * 32 + lane;  // 16 outputs x 4 quarters
+      const int o = task >> 2, qd = task & 3;
+      float acc = 0.f;
+      if (row_ok) {
+        const float4* w = reinterpret_cast<const float4*>(a.w_q + ((size_t)r * kIdxDim + o) * D + qd * DQ);
+        const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q_pre) +
+                                 (((size_t)b * a.T + t) * a.Hq + h * a.G + g) * D + qd * DQ;
+        float wv[DQ], qv[DQ];
+#pragma unroll
+        for (int k = 0; k < DQ / 4; ++k) {
+          const float4 f = __ldg(w + k);
+          wv[4 * k] = f.x; wv[4 * k + 1] = f.y; wv[4 * k + 2] = f.z; wv[4 * k + 3] = f.w;
+        }
+        load_row<__nv_bfloat16, DQ>(q, qv);
+#pragma unroll
+        for (int k = 0; k < DQ; ++k) acc = fmaf(wv[k], qv[k], acc);
+      }
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      part[it] = acc;
+    }
+#pragma unroll
+    for (int o = 0; o < kIdxDim; ++o) qi[o] = __shfl_sync(0xffffffffu, part[o >> 3], (o & 7) * 4);
+  }
+
+  RowSel rs;
+  rs.op = row_ok ? kOpMax : kOpDone;
+  rs.m = -CUDART_INF_F;
+  rs.first = false;
+  const __nv_bfloat16* kidx = static_cast<const __nv_bfloat16*>(a.kidx) + ((size_t)b * a.R + r) * a.Lmax * kIdxDim;
+  uint32_t* mrow = a.mask + (((size_t)b * a.NR + hh) * a.T + (row_ok ? t : 0)) * a.words;
+
+  // pass accumulators
+  unsigned long long pm[8];
+  unsigned pc[8];
+  float fmx;
+  unsigned kmn, kmx, n_cand, tie_cnt;
+  unsigned long long zsum;
+
+  for (int pass = 0; pass < 200; ++pass) {
+    const int op = rs.op;
+    // reset accumulators
+#pragma unroll
+    for (int q = 0; q < 8; ++q) { pm[q] = 0ull; pc[q] = 0u; }
+    fmx = -CUDART_INF_F;
+    kmn = 0xffffffffu;
+    kmx = 0u;
+    n_cand = 0u;
+    tie_cnt = 0u;
+    zsum = 0ull;
+    const bool first_split = (op == kOpSplit) && rs.first;
+    for (int kt = 0; kt <= i_last; kt += kKeyTile) {
+      __syncthreads();
+      {  // stage keys [kt, kt + kKeyTile) (only up to i_last)
+        const int n = min(kKeyTile, i_last + 1 - kt);
+        const uint4* src = reinterpret_cast<const uint4*>(kidx + (size_t)kt * kIdxDim);
+        uint4* dst = reinterpret_cast<uint4*>(s_k);
+        for (int v = threadIdx.x; v < n * 2; v += kSelRows * 32) dst[v] = __ldg(src + v);
+      }
+      __syncthreads();
+      if (op == kOpDone || kt > i) continue;  // uniform per warp
+#pragma unroll 2
+      for (int u = 0; u < kKeyTile / 32; ++u) {
+        const int j = kt + u * 32 + lane;
+        const bool on = j <= i;
+        float s = 0.f;
+        if (on) {
+          float kv[kIdxDim];
+          {  // shared-memory row (plain loads: this is not global memory)
+            const uint4* kp = reinterpret_cast<const uint4*>(s_k + (size_t)(u * 32 + lane) * kIdxDim);
+#pragma unroll
+            for (int v = 0; v < 2; ++v) {
+              const uint4 raw = kp[v];
+              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                const float2 f = __bfloat1622float2(h2[q]);
+                kv[v * 8 + 2 * q] = f.x;
+                kv[v * 8 + 2 * q + 1] = f.y;
+              }
+            }
+          }
+#pragma unroll
+          for (int q = 0; q < kIdxDim; ++q) s = fmaf(qi[q], kv[q], s);
+          s = s * kIdxScale + 0.0f;
+        }
+        const unsigned key = score_key(s);
+        if (op == kOpMax) {
+          if (on) fmx = fmaxf(fmx, s);
+        } else if (op == kOpEmit) {
+          const bool in = on && (s > rs.tau || (s == rs.tau && j <= rs.jcut));
+          const unsigned wd = __ballot_sync(0xffffffffu, in);
+          if (lane == 0 && kt + u * 32 <= i) mrow[(kt >> 5) + u] = wd;
+        } else if (on) {
+          const float d = rs.m - s;
+          const unsigned long long w = mass36(s, rs.m);
+          if (first_split) zsum += w;
+          const bool inside = d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi;
+          if (inside) {
+            if (op == kOpSplit) {
+              int q = 0;
+              if (!rs.by_key) {
+#pragma unroll
+                for (int e = 0; e < 7; ++e) q += (d >= rs.th[e]) ? 1 : 0;
+              } else {
+#pragma unroll
+                for (int e = 0; e < 7; ++e) q += (key < rs.kth[e]) ? 1 : 0;
+              }
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                if (q == e) { pm[e] += w; pc[e] += 1u; }
+              }
+            } else if (op == kOpRange) {
+              kmn = min(kmn, key);
+              kmx = max(kmx, key);
+            } else if (op == kOpTies) {
+              if (key == rs.tie_key && (unsigned)j <= rs.tie_hi) tie_cnt += 1u;
+            }
+          }
+        }
+        if (op == kOpCand) {
+          bool inside = false;
+          if (on) {
+            const float d = rs.m - s;
+            inside = d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi;
+          }
+          const unsigned bal = __ballot_sync(0xffffffffu, inside);
+          const unsigned slot = n_cand + __popc(bal & ((1u << lane) - 1u));
+          if (inside && slot < (unsigned)kCand) {
+            s_cand[warp][slot] = make_uint2(key, (unsigned)j);
+            s_cw[warp][slot] = mass36(s, rs.m);
+          }
+          n_cand += __popc(bal);
+        }
+      }
+    }
+    // ---- reduce this pass and choose the next step (warp-uniform) ----
+    if (op == kOpDone) {
+      // nothing
+    } else if (op == kOpMax) {
+      rs.m = wmaxf(fmx);
+      rs.op = kOpSplit;
+      rs.dlo = 0.f;
+      rs.dhi = -1.f;
+      rs.klo = 0u;
+      rs.khi = 0xffffffffu;
+      rs.by_key = false;
+      rs.first = true;
+      rs.cnt_above = 0u;
+      rs.need = 0ull;
+      // first split: fixed d edges (scores within 0.5, 1, 2, 3, 4.5, 7, 12 of the max)
+      const float edges[7] = {0.5f, 1.f, 2.f, 3.f, 4.5f, 7.f, 12.f};
+#pragma unroll
+      for (int e = 0; e < 7; ++e) rs.th[e] = edges[e];
+      if (a.top_p >= 1.0f) {  // keep everything
+        rs.tau = -CUDART_INF_F;
+        rs.jcut = INT_MAX;
+        rs.count = (unsigned)(i + 1);
+        rs.op = kOpEmit;
+      }
+    } else if (op == kOpSplit) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { pm[e] = wsum64(pm[e]); pc[e] = wsum32(pc[e]); }
+      if (first_split) {
+        const unsigned long long Z = wsum64(zsum);
+        unsigned long long target = (unsigned long long)ceil((double)a.top_p * (double)Z);
+        if (target > Z) target = Z;
+        if (target < 1ull) target = 1ull;
+        rs.need = target;
+        rs.cnt_in = (unsigned)(i + 1);
+        rs.first = false;
+      }
+      // sub-intervals are ordered from the highest scores (e = 0) down
+      unsigned long long cum = 0ull;
+      unsigned cc = 0u;
+      int sel = 7;
+      for (int e = 0; e < 8; ++e) {
+        if (cum + pm[e] >= rs.need) { sel = e; break; }
+        cum += pm[e];
+        cc += pc[e];
+      }
+      rs.need -= cum;
+      rs.cnt_above += cc;
+      const unsigned before = rs.cnt_in;
+      rs.cnt_in = pc[sel];
+      if (!rs.by_key) {
+        const float lo = sel == 0 ? rs.dlo : rs.th[sel - 1];
+        const float hi = sel == 7 ? rs.dhi : rs.th[sel];
+        rs.dlo = lo;
+        rs.dhi = hi;
+      } else {
+        // key sub-intervals: e = 0 holds the highest keys
+        const unsigned hi = sel == 0 ? rs.khi : rs.kth[sel - 1] - 1u;
+        const unsigned lo = sel == 7 ? rs.klo : rs.kth[sel];
+        rs.klo = lo;
+        rs.khi = hi;
+      }
+      if (rs.cnt_in <= (unsigned)kCand) {
+        rs.op = kOpCand;
+      } else {
+        // next split: d thresholds while they still separate, else order keys
+        bool split_d = !rs.by_key && rs.dhi >= 0.f && rs.cnt_in < before;
+        if (!rs.by_key && rs.dhi < 0.f) {  // open interval: bound it first
+          rs.op = kOpRange;
+        } else if (split_d) {
+          const float step = (rs.dhi - rs.dlo) * 0.125f;
+#pragma unroll
+          for (int e = 0; e < 7; ++e) rs.th[e] = fminf(rs.dlo + step * (float)(e + 1), rs.dhi);
+          rs.op = (rs.th[0] > rs.dlo && rs.th[6] < rs.dhi) ? kOpSplit : kOpRange;
+        } else {
+          rs.op = kOpRange;
+        }
+      }
+    } else if (op == kOpRange) {
+      kmn = wminu(kmn);
+      kmx = wmaxu(kmx);
+      rs.klo = max(rs.klo, kmn);
+      rs.khi = min(rs.khi, kmx);
+      rs.by_key = true;
+      if (rs.klo == rs.khi) {  // exact ties: keep the first ceil(need / w) by index
+        const unsigned long long w = mass36(key_score(rs.klo), rs.m);
+        unsigned long long kk = w ? (rs.need + w - 1ull) / w : (unsigned long long)rs.cnt_in;
+        if (kk < 1ull) kk = 1ull;
+        if (kk > rs.cnt_in) kk = rs.cnt_in;
+        rs.tie_key = rs.klo;
+        rs.need_ties = (unsigned)kk;
+        rs.tau = key_score(rs.klo);
+        rs.count = rs.cnt_above + (unsigned)kk;
+        if (kk == rs.cnt_in) {
+          rs.jcut = INT_MAX;
+          rs.op = kOpEmit;
+        } else {
+          rs.tie_lo = 0u;
+          rs.tie_hi = (unsigned)i;
+          rs.op = kOpTies;
+          // first probe
+          rs.tie_hi = (rs.tie_lo + (unsigned)i) / 2u;
+          rs.kth[0] = (unsigned)i;  // upper end of the bisection range
+        }
+      } else {
+        const unsigned long long span = (unsigned long long)rs.khi - rs.klo + 1ull;
+#pragma unroll
+        for (int e = 0; e < 7; ++e)  // kth[e]: first key of the (e+1)-th interval from the top
+          rs.kth[e] = (unsigned)(rs.khi + 1ull - (span * (unsigned long long)(e + 1) + 7ull) / 8ull);
+        rs.op = kOpSplit;
+      }
+    } else if (op == kOpTies) {
+      // bisection on the index: smallest probe with count(ties <= probe) >= need_ties
+      tie_cnt = wsum32(tie_cnt);
+      unsigned lo = rs.tie_lo, hi = rs.kth[0];
+      if (tie_cnt >= rs.need_ties) hi = rs.tie_hi;
+      else lo = rs.tie_hi + 1u;
+      rs.tie_lo = lo;
+      rs.kth[0] = hi;
+      if (lo >= hi) {
+        rs.jcut = (int)lo;
+        rs.op = kOpEmit;
+      } else {
+        rs.tie_hi = (lo + hi) / 2u;
+      }
+    } else if (op == kOpCand) {
+      // exact solve: candidate c is kept iff the mass ordered before it is < need
+      const int n = (int)min(n_cand, (unsigned)kCand);
+      unsigned kept_n = 0u, tkey = 0xffffffffu;
+      __syncwarp();
+      for (int c = lane; c < n; c += 32) {
+        const uint2 me = s_cand[warp][c];
+        unsigned long long before = 0ull;
+        for (int o = 0; o < n; ++o) {
+          const uint2 ot = s_cand[warp][o];
+          if (ot.x > me.x || (ot.x == me.x && ot.y < me.y)) before += s_cw[warp][o];
+        }
+        if (before < rs.need) {
+          ++kept_n;
+          tkey = min(tkey, me.x);
+        }
+      }
+      kept_n = wsum32(kept_n);
+      tkey = wminu(tkey);
+      int jc = -1;
+      for (int c = lane; c < n; c += 32) {
+        const uint2 me = s_cand[warp][c];
+        if (me.x != tkey) continue;
+        unsigned long long before = 0ull;
+        for (int o = 0; o < n; ++o) {
+          const uint2 ot = s_cand[warp][o];
+          if (ot.x > me.x || (ot.x == me.x && ot.y < me.y)) before += s_cw[warp][o];
+        }
+        if (before < rs.need) jc = max(jc, (int)me.y);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) jc = max(jc, __shfl_xor_sync(0xffffffffu, jc, o));
+      __syncwarp();
+      rs.tau = key_score(tkey);
+      rs.jcut = jc;
+      rs.count = rs.cnt_above + kept_n;
+      rs.op = kOpEmit;
+    } else if (op == kOpEmit) {
+      // last word(s) past i inside the row stay as written (bits > i are zero)
+      if (lane == 0) {
+        if (a.sel_tau) a.sel_tau[((size_t)b * a.NR + hh) * a.T + t] = rs.tau;
+        if (a.sel_jcut) a.sel_jcut[((size_t)b * a.NR + hh) * a.T + t] = rs.jcut;
+        if (a.sel_count) a.sel_count[((size_t)b * a.NR + hh) * a.T + t] = (int)rs.count;
+      }
+      rs.op = kOpDone;
+    }
+    if (!__syncthreads_or(rs.op != kOpDone)) break;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// masked causal attention on tensor cores
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(unsigned& r0, unsigned& r1, unsigned& r2, unsigned& r3, const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x2(unsigned& r0, unsigned& r1, const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x2_t(unsigned& r0, unsigned& r1, const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(a));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
+                                         unsigned b0, unsigned b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ unsigned pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const unsigned*>(&v);
+}
+
+template <int D>
+struct AttnSmem {
+  static constexpr int kStride = D + 8;  // bf16 elements per shared row (pad: no ldmatrix conflicts)
+  static constexpr size_t kBytes = (size_t)(kBQ + 2 * kBK) * kStride * sizeof(__nv_bfloat16);
+};
+
+template <int D>
+__global__ void __launch_bounds__(128) attn_rows_kernel(PrefillArgs a) {
+  constexpr int ST = AttnSmem<D>::kStride;
+  constexpr int KS = D / 16;  // k-steps of Q K^T
+  constexpr int NO = D / 8;   // n8 tiles of the output
+  extern __shared__ __align__(16) unsigned char smem[];
+  __nv_bfloat16* s_q = reinterpret_cast<__nv_bfloat16*>(smem);
+  __nv_bfloat16* s_k = s_q + kBQ * ST;
+  __nv_bfloat16* s_v = s_k + kBK * ST;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int bq = blockIdx.y;
+  const int b = bq / a.Hq, hq = bq % a.Hq;
+  const int h = hq / a.G, g = hq % a.G;
+  const int r = a.ret_rank[h];
+  const int start = a.start_pos[b];
+  if (start < 0 || start + a.T > a.Lmax) return;  // flagged by the selection kernel / host
+  const int t0 = blockIdx.x * kBQ;
+  const int hh = r >= 0 ? r * a.G + g : 0;
+
+  // ---- Q tile: RoPE at each row's position, scaled by log2(e)/sqrt(D), bf16 ----
+  const float qscale = 1.4426950408889634f * rsqrtf((float)D);
+  for (int e = threadIdx.x; e < kBQ * (D / 2); e += blockDim.x) {
+    const int rr = e / (D / 2), kk = e % (D / 2);
+    const int t = t0 + rr;
+    float y1 = 0.f, y2 = 0.f;
+    if (t < a.T) {
+      const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q_pre) + (((size_t)b * a.T + t) * a.Hq + hq) * D;
+      const float x1 = __bfloat162float(q[kk]), x2 = __bfloat162float(q[kk + D / 2]);
+      float c, sn;
+      rope_cos_sin(start + t, kk, D, a.rope_base, c, sn);
+      y1 = (x1 * c - x2 * sn) * qscale;
+      y2 = (x2 * c + x1 * sn) * qscale;
+    }
+    s_q[rr * ST + kk] = __float2bfloat16_rn(y1);
+    s_q[rr * ST + kk + D / 2] = __float2bfloat16_rn(y2);
+  }
+  __syncthreads();
+  // Q fragments of this warp's 16 rows stay in registers
+  unsigned qa[KS][4];
+#pragma unroll
+  for (int ks = 0; ks < KS; ++ks) {
+    const int row = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+    const int col = ks * 16 + (lane >> 4) * 8;
+    ldsm_x4(qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], s_q + row * ST + col);
+  }
+
+  // rows of this thread: warp*16 + gq and + 8
+  int ti[2], pi[2], wlo[2];
+  bool rv[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    ti[x] = t0 + warp * 16 + gq + 8 * x;
+    rv[x] = ti[x] < a.T;
+    pi[x] = start + ti[x];
+    wlo[x] = pi[x] - a.W + 1;  // window: keys >= wlo
+  }
+  const int t_last = min(a.T, t0 + kBQ) - 1;
+  const int i_max = start + t_last;
+  const int i_min = start + t0;
+  const uint32_t* mrow[2];
+#pragma unroll
+  for (int x = 0; x < 2; ++x)
+    mrow[x] = a.mask + (((size_t)b * a.NR + hh) * a.T + (rv[x] ? ti[x] : 0)) * a.words;
+
+  float o[NO][4];
+#pragma unroll
+  for (int n = 0; n < NO; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  float mrun[2] = {-CUDART_INF_F, -CUDART_INF_F}, lrun[2] = {0.f, 0.f};
+
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+
+  for (int kt = 0; kt <= i_max; kt += kBK) {
+    // does any row of the tile keep a key of this tile?
+    const bool sink_tile = kt < a.S;
+    const bool win_tile = kt + kBK - 1 >= i_min - a.W + 1;
+    unsigned mw[2][2] = {{0u, 0u}, {0u, 0u}};
+    bool any = false;
+    if (r >= 0) {
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        if (!rv[x]) continue;
+#pragma unroll
+        for (int y = 0; y < 2; ++y) {
+          const int wd = (kt >> 5) + y;
+          if (wd * 32 <= pi[x]) mw[x][y] = __ldg(mrow[x] + wd);
+          any |= mw[x][y] != 0u;
+        }
+      }
+    }
+    if (!__syncthreads_or(any || sink_tile || win_tile)) continue;
+    // stage K and V tiles
+    for (int e = threadIdx.x; e < kBK * (D / 8); e += blockDim.x) {
+      const int kr = e / (D / 8), c8 = e % (D / 8);
+      const int j = kt + kr;
+      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
+      if (j <= i_max) {
+        kv = __ldg(reinterpret_cast<const uint4*>(kg + (size_t)j * D) + c8);
+        vv = __ldg(reinterpret_cast<const uint4*>(vg + (size_t)j * D) + c8);
+      }
+      *reinterpret_cast<uint4*>(s_k + kr * ST + c8 * 8) = kv;
+      *reinterpret_cast<uint4*>(s_v + kr * ST + c8 * 8) = vv;
+    }
+    __syncthreads();
+    // S = Q K^T for this warp's 16 rows x 64 keys
+    float sc[kBK / 8][4];
+#pragma unroll
+    for (int n = 0; n < kBK / 8; ++n) {
+      sc[n][0] = sc[n][1] = sc[n][2] = sc[n][3] = 0.f;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        unsigned b0, b1;
+        const int krow = n * 8 + (lane & 7);
+        const int kcol = ks * 16 + ((lane >> 3) & 1) * 8;
+        ldsm_x2(b0, b1, s_k + krow * ST + kcol);
+        mma_bf16(sc[n], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], b0, b1);
+      }
+    }
+    // mask + tile maximum per row
+    float tmax[2] = {-CUDART_INF_F, -CUDART_INF_F};
+#pragma unroll
+    for (int n = 0; n < kBK / 8; ++n) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int x = c >> 1;
+        const int jj = n * 8 + 2 * tq + (c & 1);
+        const int j = kt + jj;
+        bool ok = rv[x] && j <= pi[x] && (j < a.S || j >= wlo[x]);
+        if (!ok && r >= 0 && rv[x] && j <= pi[x]) ok = (mw[x][jj >> 5] >> (jj & 31)) & 1u;
+        sc[n][c] = ok ? sc[n][c] : -CUDART_INF_F;
+        tmax[x] = fmaxf(tmax[x], sc[n][c]);
+      }
+    }
+    float alpha[2];
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      tmax[x] = fmaxf(tmax[x], __shfl_xor_sync(0xffffffffu, tmax[x], 1));
+      tmax[x] = fmaxf(tmax[x], __shfl_xor_sync(0xffffffffu, tmax[x], 2));
+      const float mn = fmaxf(mrun[x], tmax[x]);
+      alpha[x] = (mn == -CUDART_INF_F) ? 1.f : exp2f(mrun[x] - mn);
+      mrun[x] = mn;
+    }
+    float lsum[2] = {0.f, 0.f};
+#pragma unroll
+    for (int n = 0; n < kBK / 8; ++n) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int x = c >> 1;
+        const float p = (sc[n][c] == -CUDART_INF_F) ? 0.f : exp2f(sc[n][c] - mrun[x]);
+        sc[n][c] = p;
+        lsum[x] += p;
+      }
+    }
+#pragma unroll
+    for (int x = 0; x < 2; ++x) lrun[x] = lrun[x] * alpha[x] + lsum[x];
+#pragma unroll
+    for (int n = 0; n < NO; ++n) {
+      o[n][0] *= alpha[0];
+      o[n][1] *= alpha[0];
+      o[n][2] *= alpha[1];
+      o[n][3] *= alpha[1];
+    }
+    // O += P V
+#pragma unroll
+    for (int kc = 0; kc < kBK / 16; ++kc) {
+      const unsigned pa0 = pack_bf16(sc[2 * kc][0], sc[2 * kc][1]);
+      const unsigned pa1 = pack_bf16(sc[2 * kc][2], sc[2 * kc][3]);
+      const unsigned pa2 = pack_bf16(sc[2 * kc + 1][0], sc[2 * kc + 1][1]);
+      const unsigned pa3 = pack_bf16(sc[2 * kc + 1][2], sc[2 * kc + 1][3]);
+#pragma unroll
+      for (int n = 0; n < NO; ++n) {
+        unsigned b0, b1;
+        const int vrow = kc * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+        ldsm_x2_t(b0, b1, s_v + vrow * ST + n * 8);
+        mma_bf16(o[n], pa0, pa1, pa2, pa3, b0, b1);
+      }
+    }
+    __syncthreads();
+  }
+  // ---- epilogue ----
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    lrun[x] += __shfl_xor_sync(0xffffffffu, lrun[x], 1);
+    lrun[x] += __shfl_xor_sync(0xffffffffu, lrun[x], 2);
+  }
+#pragma unroll
+  for (int x = 0; x < 2; ++x) {
+    if (!rv[x]) continue;
+    const float inv = 1.f / lrun[x];
+    __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.T + ti[x]) * a.Hq + hq) * D;
+#pragma unroll
+    for (int n = 0; n < NO; ++n) {
+      const __nv_bfloat162 v2 = __floats2bfloat162_rn(o[n][2 * x] * inv, o[n][2 * x + 1] * inv);
+      *reinterpret_cast<__nv_bfloat162*>(orow + n * 8 + 2 * tq) = v2;
+    }
+  }
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+}  // namespace
 
 PrefillLayout prefill_layout(const Shape& sh, int T) {
   PrefillLayout l;
-  (void)sh;
-  (void)T;
-  l.total = 256;
+  const size_t words = (size_t)(sh.Lmax + 31) / 32;
+  l.total = align256((size_t)sh.B * sh.NR * T * words * sizeof(uint32_t)) + 256;
   return l;
 }
 
 int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* start_pos,
-                   int T, const float* w_q, void* out, float* sel_tau, int* sel_jcut,
-                   int* sel_count, void* ws, const PrefillLayout& lay, cudaStream_t st) {
-  (void)sh; (void)cache; (void)q_pre; (void)start_pos; (void)T; (void)w_q; (void)out;
-  (void)sel_tau; (void)sel_jcut; (void)sel_count; (void)ws; (void)lay; (void)st;
-  set_error("rtp_prefill_attn: not built yet");
-  return RTP_ERR_SHAPE;
+                   int T, const float* w_q, void* out, uint32_t* sel_bitmask, float* sel_tau,
+                   int* sel_jcut, int* sel_count, void* ws, const PrefillLayout& lay, cudaStream_t st) {
+  (void)lay;
+  if (sh.dtype != RTP_BF16) {
+    set_error("rtp_prefill_attn: the prefill path computes in bf16 (dtype must be RTP_BF16)");
+    return RTP_ERR_DTYPE;
+  }
+  PrefillArgs a;
+  a.B = sh.B; a.Hq = sh.Hq; a.Hkv = sh.Hkv; a.G = sh.G; a.D = sh.D; a.R = sh.R; a.NR = sh.NR;
+  a.Lmax = sh.Lmax; a.S = sh.S; a.W = sh.W; a.T = T; a.words = (sh.Lmax + 31) / 32;
+  a.top_p = sh.top_p; a.rope_base = sh.rope_base;
+  a.q_pre = q_pre; a.w_q = w_q; a.out = out;
+  a.k = cache->k; a.v = cache->v; a.kidx = cache->kidx; a.status = cache->status;
+  a.start_pos = start_pos;
+  a.sel_tau = sel_tau; a.sel_jcut = sel_jcut; a.sel_count = sel_count;
+  a.mask = sel_bitmask ? sel_bitmask : static_cast<uint32_t*>(ws);
+  for (int i = 0; i < kMaxRetrieval; ++i) { a.ret_head[i] = sh.ret_head[i]; a.ret_rank[i] = sh.ret_rank[i]; }
+
+  static bool s_attr[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !s_attr[dev]) {
+    cudaFuncSetAttribute(attn_rows_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)AttnSmem<128>::kBytes);
+    cudaFuncSetAttribute(attn_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)AttnSmem<64>::kBytes);
+    s_attr[dev] = true;
+  }
+  if (sh.R > 0) {
+    const dim3 gs((T + kSelRows - 1) / kSelRows, sh.B * sh.NR);
+    trace_begin(RTP_STAGE_PREFILL_INDEX, st);
+    if (sh.D == 128) select_rows_kernel<128><<<gs, kSelRows * 32, 0, st>>>(a);
+    else select_rows_kernel<64><<<gs, kSelRows * 32, 0, st>>>(a);
+    trace_end(RTP_STAGE_PREFILL_INDEX, st);
+  }
+  const dim3 ga((T + kBQ - 1) / kBQ, sh.B * sh.Hq);
+  trace_begin(RTP_STAGE_PREFILL_ATTN, st);
+  if (sh.D == 128) attn_rows_kernel<128><<<ga, 128, AttnSmem<128>::kBytes, st>>>(a);
+  else attn_rows_kernel<64><<<ga, 128, AttnSmem<64>::kBytes, st>>>(a);
+  trace_end(RTP_STAGE_PREFILL_ATTN, st);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    set_error(std::string("prefill launch: ") + cudaGetErrorString(e));
+    return RTP_ERR_CUDA;
+  }
+  return RTP_OK;
 }
 
 }  // namespace rtp

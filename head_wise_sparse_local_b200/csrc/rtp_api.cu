@@ -193,9 +193,9 @@ int rtp_decode_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void
 }
 
 int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
-                     const int* start_pos, int T, const float* w_q, void* out, float* sel_tau,
-                     int* sel_jcut, int* sel_count, void* workspace, size_t workspace_bytes,
-                     void* stream) {
+                     const int* start_pos, int T, const float* w_q, void* out,
+                     uint32_t* sel_bitmask, float* sel_tau, int* sel_jcut, int* sel_count,
+                     void* workspace, size_t workspace_bytes, void* stream) {
   Shape sh;
   int rc = make_shape(cfg, &sh);
   if (rc != RTP_OK) return rc;
@@ -211,8 +211,8 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
     return fail(RTP_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   if (workspace_bytes < lay.total)
     return fail(RTP_ERR_WORKSPACE, "workspace smaller than rtp_prefill_workspace_bytes");
-  return launch_prefill(sh, cache, q_pre, start_pos, T, w_q, out, sel_tau, sel_jcut, sel_count,
-                        workspace, lay, (cudaStream_t)stream);
+  return launch_prefill(sh, cache, q_pre, start_pos, T, w_q, out, sel_bitmask, sel_tau, sel_jcut,
+                        sel_count, workspace, lay, (cudaStream_t)stream);
 }
 
 }  // extern "C"

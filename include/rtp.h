@@ -202,14 +202,22 @@ int rtp_decode_attn_noalloc(const rtp_layer_cfg* cfg, const rtp_cache* cache, co
  * must already be in the cache (rtp_append_kv with the same start_pos and T).
  * Per row the layer computes exactly what rtp_decode_attn computes for a
  * query at position i (top-p over the indexer scores of [0, i] for retrieval
- * query heads; sinks and window [i-W+1, i] for every head).
+ * query heads; sinks and window [i-W+1, i] for every head); the indexer
+ * scores use the same fp32 arithmetic as rtp_decode_attn, so a row's top-p
+ * set equals the decode step's at that position.  The attention itself runs
+ * on tensor cores in bf16 with fp32 accumulation (atlas.scime.ai summary,
+ * "Approach"; abstract, observations (2)-(3)).  cfg->dtype must be RTP_BF16.
  *
- *   q_pre        [B][T][Hq][D] dtype, device
- *   start_pos    [B] int32, device; start_pos[b] + T <= max_ctx
+ *   q_pre        [B][T][Hq][D] bf16, device
+ *   start_pos    [B] int32, device; 0 <= start_pos[b] and start_pos[b] + T <= max_ctx
+ *                (else the sequence is skipped and RTP_DEV_POSITION is set)
  *   w_q          [R][16][D] fp32, device
- *   out          [B][T][Hq][D] dtype, device
- *   sel_tau      optional [B][R*G][T] float: score of the last kept token of the
- *                row's top-p set (+inf-free; p = 1 gives -inf)
+ *   out          [B][T][Hq][D] bf16, device
+ *   sel_bitmask  optional [B][R*G][T][ceil(max_ctx/32)] uint32: row (b, r*G+g, t)
+ *                has bit j set iff token j is in that row's top-p set; words
+ *                past position i of the row are not written
+ *   sel_tau      optional [B][R*G][T] float: score of the last kept token
+ *                (-inf when p = 1 keeps every token)
  *   sel_jcut     optional [B][R*G][T] int32: tokens with score == sel_tau are kept
  *                iff their index <= sel_jcut (so membership is
  *                s_j > tau || (s_j == tau && j <= jcut))
@@ -217,9 +225,9 @@ int rtp_decode_attn_noalloc(const rtp_layer_cfg* cfg, const rtp_cache* cache, co
  *   workspace    >= rtp_prefill_workspace_bytes(cfg, T), 256-byte aligned
  */
 int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
-                     const int* start_pos, int T, const float* w_q, void* out, float* sel_tau,
-                     int* sel_jcut, int* sel_count, void* workspace, size_t workspace_bytes,
-                     void* stream);
+                     const int* start_pos, int T, const float* w_q, void* out,
+                     uint32_t* sel_bitmask, float* sel_tau, int* sel_jcut, int* sel_count,
+                     void* workspace, size_t workspace_bytes, void* stream);
 
 /* Kernel stages, for rtp_trace_stage. */
 typedef enum rtp_stage {
@@ -227,7 +235,7 @@ typedef enum rtp_stage {
   RTP_STAGE_DECODE_STREAM = 1,  /* decode: indexer scores + sink/window attention */
   RTP_STAGE_DECODE_SELECT = 2,  /* decode: exact top-p threshold + selection bitmask */
   RTP_STAGE_DECODE_GATHER = 3,  /* decode: kept-row attention + log-sum-exp merge */
-  RTP_STAGE_PREFILL_INDEX = 4,  /* prefill: indexer score/threshold passes */
+  RTP_STAGE_PREFILL_INDEX = 4,  /* prefill: per-row exact top-p selection */
   RTP_STAGE_PREFILL_ATTN = 5,   /* prefill: masked causal attention */
   RTP_STAGE_COUNT = 6
 } rtp_stage;

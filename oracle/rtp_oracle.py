@@ -282,12 +282,14 @@ def decode(cache: OracleCache, q_pre, seq_len, w_q, top_p: Optional[float] = Non
 
 
 def prefill(cache: OracleCache, q_pre, start_pos, w_q, rows: Optional[Sequence[int]] = None,
-            top_p: Optional[float] = None, heads: Optional[Iterable[int]] = None):
+            top_p: Optional[float] = None, heads: Optional[Iterable[int]] = None,
+            rows_override: Optional[Dict] = None):
     """Causal prefill chunk: query row t of sequence b sits at position
     start_pos[b] + t and sees [0, start_pos[b] + t].
 
     q_pre [B, T, Hq, D].  Returns out {(b, t): [Hq, D]}, topp {(b, t, hq): kept
     indices} for retrieval heads, over the requested rows (default: all).
+    `rows_override` {(b, t, hq): rows} replaces the attended rows of a query.
     """
     sh = cache.shape
     p = sh.top_p if top_p is None else top_p
@@ -300,7 +302,10 @@ def prefill(cache: OracleCache, q_pre, start_pos, w_q, rows: Optional[Sequence[i
             i = int(start_pos[b]) + int(t)
             o_bt = np.zeros((sh.n_q_heads, sh.head_dim))
             for hq in hs:
-                o, tp, _ = _row(cache, b, hq, i, q_pre[b, t, hq], w_q, p)
+                ov = None
+                if rows_override is not None and (b, int(t), hq) in rows_override:
+                    ov = {(b, hq): rows_override[(b, int(t), hq)]}
+                o, tp, _ = _row(cache, b, hq, i, q_pre[b, t, hq], w_q, p, ov)
                 o_bt[hq] = o
                 if tp is not None:
                     topp[(b, int(t), hq)] = tp

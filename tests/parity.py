@@ -142,3 +142,84 @@ def check_decode_parity(inp, top_p=None, oc=None):
     assert np.all(err <= lim), f"output mismatch: max err {err.max():.3e}, worst ratio {worst:.3f}"
     return dict(heads=n_heads, exact=n_exact, diff_tokens=n_diff_tok, worst_ratio=worst,
                 max_abs_err=float(err.max()), counts=g["count"])
+
+
+def run_gpu_prefill(inp, top_p=None):
+    """Append the context and the chunk, then run one prefill over the chunk.
+
+    Returns out [B, T, Hq, D] float64, bitmask [B, NR, T, words], count [B, NR, T]."""
+    from head_wise_sparse_local_b200 import Layer
+    sh = inp["shape"]
+    if top_p is not None:
+        sh = sh.replace(top_p=top_p)
+    dev = torch.device("cuda")
+    Lmax = inp["max_ctx"]
+    T = inp["T"]
+    lay = Layer(sh, Lmax, device=dev, prefill_T=T)
+    start = torch.from_numpy(inp["start_pos"]).to(dev)
+    n_ctx = int(inp["start_pos"].max()) + T
+    lay.append(inp["k_pre"][:, :n_ctx].contiguous().to(dev), inp["v"][:, :n_ctx].contiguous().to(dev),
+               torch.zeros(sh.batch, dtype=torch.int32, device=dev), inp["w_k"].to(dev))
+    q = inp["q_pre"].to(dev)
+    out = torch.empty((sh.batch, T, sh.n_q_heads, sh.head_dim), dtype=sh.torch_dtype, device=dev)
+    NR = max(sh.n_retrieval * sh.group, 1)
+    words = (Lmax + 31) // 32
+    bm = torch.zeros((sh.batch, NR, T, words), dtype=torch.int32, device=dev)
+    cnt = torch.full((sh.batch, NR, T), -1, dtype=torch.int32, device=dev)
+    tau = torch.zeros((sh.batch, NR, T), dtype=torch.float32, device=dev)
+    jcut = torch.zeros((sh.batch, NR, T), dtype=torch.int32, device=dev)
+    lay.prefill(q, start, inp["w_q"].to(dev), out, sel_bitmask=bm, sel_tau=tau, sel_jcut=jcut,
+                sel_count=cnt)
+    torch.cuda.synchronize()
+    return dict(out=out.double().cpu().numpy(), bitmask=bm, count=cnt.cpu().numpy(),
+                tau=tau.cpu().numpy(), jcut=jcut.cpu().numpy(), status=lay.device_status(),
+                layer=lay, shape=sh)
+
+
+def check_prefill_parity(inp, rows=None, top_p=None, g=None):
+    """Selection sets (per row, per retrieval q head) and outputs of the GPU
+    prefill against the oracle, over `rows` (default: every row)."""
+    sh = inp["shape"] if top_p is None else inp["shape"].replace(top_p=top_p)
+    g = g or run_gpu_prefill(inp, top_p)
+    assert g["status"] == 0, f"device status {g['status']}"
+    T = inp["T"]
+    rows = list(range(T)) if rows is None else list(rows)
+    oc = OracleCache(sh, inp["max_ctx"])
+    n_ctx = inp["start_pos"] + T
+    oc.append_in_place(inp["k_pre"], inp["v"], n_ctx, inp["w_k"])
+    out_o, topp_o = oracle.prefill(oc, inp["q_pre"], inp["start_pos"], inp["w_q"], rows=rows)
+    G = sh.group
+    bm = g["bitmask"].cpu().numpy().view(np.uint32)
+    override = {}
+    n_exact = n_heads = 0
+    for b in range(sh.batch):
+        for t in rows:
+            i = int(inp["start_pos"][b]) + t
+            for r, h in enumerate(sh.retrieval):
+                for gg in range(G):
+                    hq = h * G + gg
+                    rg = r * G + gg
+                    bits = np.unpackbits(bm[b, rg, t].view(np.uint8), bitorder="little")[: i + 1]
+                    gset = np.nonzero(bits)[0]
+                    assert g["count"][b, rg, t] == len(gset), (b, t, hq, g["count"][b, rg, t], len(gset))
+                    qi = oracle.indexer_project(inp["q_pre"][b, t, hq], inp["w_q"][r])
+                    s = oracle.indexer_scores(qi, oc.indexer_keys(b, r, i + 1))
+                    exact, _ = compare_selection(s, sh.top_p, gset, topp_o[(b, t, hq)])
+                    n_heads += 1
+                    n_exact += int(exact)
+                    if not exact:
+                        override[(b, t, hq)] = np.union1d(gset, oracle.sink_window_set(i, sh.n_sink, sh.window))
+    if override:
+        out_o, _ = oracle.prefill(oc, inp["q_pre"], inp["start_pos"], inp["w_q"], rows=rows,
+                                  rows_override=override)
+    atol, rtol = TOL[sh.dtype]
+    worst = 0.0
+    for b in range(sh.batch):
+        for t in rows:
+            ref = out_o[(b, t)]
+            got = g["out"][b, t]
+            err = np.abs(got - ref)
+            lim = atol + rtol * np.abs(ref)
+            worst = max(worst, float((err / lim).max()))
+            assert np.all(err <= lim), (b, t, float(err.max()), np.unravel_index(np.argmax(err / lim), err.shape))
+    return dict(heads=n_heads, exact=n_exact, worst_ratio=worst, g=g)

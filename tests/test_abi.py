@@ -109,3 +109,12 @@ def test_null_pointers_rejected_before_launch(rtp):
     with pytest.raises(rtp.RtpError) as e:
         rtp.rtp_prefill_attn(c, cache, fake, fake, 0, fake, fake, workspace=fake, stream=0)
     assert e.value.code == 2
+    with pytest.raises(rtp.RtpError) as e:  # prefill workspace too small
+        rtp.rtp_prefill_attn(c, cache, fake, fake, 16, fake, fake, workspace=fake,
+                             workspace_bytes=256, stream=0)
+    assert e.value.code == 4
+    cf = _cfg(rtp, dtype="fp32")
+    with pytest.raises(rtp.RtpError) as e:  # prefill computes in bf16 only
+        rtp.rtp_prefill_attn(cf, cache, fake, fake, 16, fake, fake, workspace=fake,
+                             workspace_bytes=1 << 40, stream=0)
+    assert e.value.code == 3
