@@ -1,17 +1,12 @@
 // rtp_decode_attn: one decode step of the head-wise sparse attention layer.
 //
-// Three kernels on the caller's stream, chained with programmatic dependent
-// launch (each waits on griddepcontrol before touching its predecessor's
-// results), scratch in the caller's workspace:
+// Four kernels on the caller's stream, chained with programmatic dependent
+// launch, scratch in the caller's workspace:
 //
-//   stream_kernel  two kinds of CTA in one grid, both HBM streams:
-//                  * score CTAs read the 16-d indexer-key cache once (two
-//                    16-byte loads per token for bf16) and write the fp32
-//                    scores s_j = q~ . k~_j / 4 of the G query heads of a
-//                    retrieval KV head plus a per-chunk maximum;
-//                  * sink/window CTAs run exact attention over the sinks and
-//                    the window of every KV head (these rows do not depend on
-//                    the selection) and write one partial (m, l, o) per tile.
+//   score_kernel   reads the 16-d indexer-key cache once (two 16-byte loads
+//                  per token for bf16) and writes the fp32 scores
+//                  s_j = q~ . k~_j / 4 of the G query heads of a retrieval KV
+//                  head plus a per-chunk maximum.
 //   select_kernel  one thread-block cluster per (sequence, retrieval q head).
 //                  The softmax mass exp(s - max) of every score, in 2^-36
 //                  fixed point (integer sums: exact and order independent),
@@ -22,6 +17,9 @@
 //                  and the leader resolves the exact threshold score tau and,
 //                  for ties at tau, the last kept index j_cut.  The top-p set
 //                  is written as a bitmask.
+//   sw_kernel      exact attention over the sinks and the window of every KV
+//                  head; launched after the select kernel without waiting for
+//                  it, so this HBM stream overlaps the selection.
 //   gather_kernel  for retrieval KV heads: the union over the G query heads
 //                  of the kept rows outside sinks/window, read from the
 //                  bitmask, attended exactly; the last CTA of each KV head
@@ -73,6 +71,7 @@ struct DecodeArgs {
   float* pl;
   float* po;        // [B][Hkv][n_parts_max][G][D]
   unsigned* ctl;    // [B*Hkv] gather tickets
+  float* qrope;     // [B][Hkv][G][D] RoPE'd, pre-scaled queries (written by the stream kernel)
   uint2* cand;      // [B][NR][lstride] boundary-bucket candidates (key, index)
   int n_ctl, nch_score_max, n_sw_tiles, n_parts_max, n_score_ctas, n_sw_ctas;
   int ret_head[kMaxRetrieval];
@@ -159,7 +158,7 @@ struct WarpAttn {
                typename std::conditional<VB == 4, unsigned, unsigned short>::type>::type>::type;
   float m[G], l[G], o[G][DL];
   uint4 kraw[KV];
-  VRaw vraw[32];
+  const T* vb;
   int row;
   unsigned msk, live;
 
@@ -173,28 +172,24 @@ struct WarpAttn {
     }
   }
 
-  // row_: this lane's row (ignored when msk_ == 0); msk_: head bits.
-  __device__ __forceinline__ void load(const T* __restrict__ kb, const T* __restrict__ vb, int row_,
+  // row_: this lane's row (ignored when msk_ == 0); msk_: head bits.  Issues
+  // the key loads; the value loads are issued inside compute(), after the
+  // scores, so keys and values are never live in registers together.
+  __device__ __forceinline__ void load(const T* __restrict__ kb, const T* __restrict__ vb_, int row_,
                                        unsigned msk_) {
-    const int lane = threadIdx.x & 31;
     row = msk_ ? row_ : 0;
     msk = msk_;
+    vb = vb_;
     live = __ballot_sync(0xffffffffu, msk_ != 0u);
     const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)row * D);
 #pragma unroll
-    for (int i = 0; i < KV; ++i) kraw[i] = msk ? __ldg(kr + i) : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      const int rr = __shfl_sync(0xffffffffu, row, r);
-      if ((live >> r) & 1u) vraw[r] = __ldg(reinterpret_cast<const VRaw*>(vb + (size_t)rr * D + lane * DL));
-      else vraw[r] = VRaw();
-    }
+    for (int i = 0; i < KV; ++i) kraw[i] = msk ? __ldcg(kr + i) : make_uint4(0u, 0u, 0u, 0u);
   }
 
   __device__ __forceinline__ void compute(const float* __restrict__ s_q) {
-    float s[G];
+    float s4[G][4];  // four independent partial sums per head
 #pragma unroll
-    for (int g = 0; g < G; ++g) s[g] = 0.f;
+    for (int g = 0; g < G; ++g) s4[g][0] = s4[g][1] = s4[g][2] = s4[g][3] = 0.f;
     constexpr int E = 16 / sizeof(T);
 #pragma unroll
     for (int i = 0; i < KV; ++i) {
@@ -216,13 +211,17 @@ struct WarpAttn {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
           const float4 qv = *reinterpret_cast<const float4*>(s_q + g * D + i * E + e);
-          s[g] = fmaf(qv.x, kf[e], s[g]);
-          s[g] = fmaf(qv.y, kf[e + 1], s[g]);
-          s[g] = fmaf(qv.z, kf[e + 2], s[g]);
-          s[g] = fmaf(qv.w, kf[e + 3], s[g]);
+          float* acc = s4[g];
+          acc[0] = fmaf(qv.x, kf[e], acc[0]);
+          acc[1] = fmaf(qv.y, kf[e + 1], acc[1]);
+          acc[2] = fmaf(qv.z, kf[e + 2], acc[2]);
+          acc[3] = fmaf(qv.w, kf[e + 3], acc[3]);
         }
       }
     }
+    float s[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) s[g] = (s4[g][0] + s4[g][1]) + (s4[g][2] + s4[g][3]);
     float p[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -241,18 +240,33 @@ struct WarpAttn {
       for (int d = 0; d < DL; ++d) o[g][d] *= al;
       m[g] = mn;
     }
+    // value slices of the tile's live rows (lane owns dims [lane*DL, lane*DL + DL)),
+    // 16 rows at a time
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-    for (int r = 0; r < 32; ++r) {
-      if (!((live >> r) & 1u)) continue;  // warp-uniform
-      float vv[DL];
-      const T* vt = reinterpret_cast<const T*>(&vraw[r]);
+    for (int half = 0; half < 2; ++half) {
+      VRaw vraw[16];
 #pragma unroll
-      for (int d = 0; d < DL; ++d) vv[d] = to_f32(vt[d]);
+      for (int r = 0; r < 16; ++r) {
+        const int rr = __shfl_sync(0xffffffffu, row, half * 16 + r);
+        if ((live >> (half * 16 + r)) & 1u)
+          vraw[r] = __ldcg(reinterpret_cast<const VRaw*>(vb + (size_t)rr * D + lane * DL));
+        else
+          vraw[r] = VRaw();
+      }
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float pr = __shfl_sync(0xffffffffu, p[g], r);
+      for (int r = 0; r < 16; ++r) {
+        if (!((live >> (half * 16 + r)) & 1u)) continue;  // warp-uniform
+        float vv[DL];
+        const T* vt = reinterpret_cast<const T*>(&vraw[r]);
 #pragma unroll
-        for (int d = 0; d < DL; ++d) o[g][d] = fmaf(pr, vv[d], o[g][d]);
+        for (int d = 0; d < DL; ++d) vv[d] = to_f32(vt[d]);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float pr = __shfl_sync(0xffffffffu, p[g], half * 16 + r);
+#pragma unroll
+          for (int d = 0; d < DL; ++d) o[g][d] = fmaf(pr, vv[d], o[g][d]);
+        }
       }
     }
   }
@@ -299,22 +313,21 @@ __device__ void write_partial(const DecodeArgs& a, WA& wa, size_t part, float* s
 }
 
 // ---------------------------------------------------------------------------
-// 1. stream kernel: indexer scores + sink/window attention
+// 1. score kernel: indexer scores (+ this call's counters zeroed)
 // ---------------------------------------------------------------------------
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) stream_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads) score_kernel(DecodeArgs a) {
   griddep_wait();
   griddep_launch();
-  __shared__ __align__(16) float s_q[G * D];
-  __shared__ __align__(16) float s_o[kWarps * G * D];
-  __shared__ float s_ml[kWarps * G * 2];
+  __shared__ __align__(16) float s_q[G * kIdxDim];
+  __shared__ float s_ml[kWarps * G];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (blockIdx.x == 0) {  // zero this call's counters (read by later kernels)
     for (int i = tid; i < a.n_ctl; i += kThreads) a.ctl[i] = 0u;
     if (a.sel_count)
       for (int i = tid; i < a.B * a.NR; i += kThreads) a.sel_count[i] = 0;
   }
-  if ((int)blockIdx.x < a.n_score_ctas) {
+  {
     // ---- indexer scores ----
     const int nch = a.n_score_ctas / (a.B * a.R);
     const int chunk = blockIdx.x % nch;
@@ -421,14 +434,31 @@ __global__ void __launch_bounds__(kThreads) stream_kernel(DecodeArgs a) {
     }
     return;
   }
-  // ---- sink/window attention ----
-  const int idx = blockIdx.x - a.n_score_ctas;
+}
+
+// ---------------------------------------------------------------------------
+// 2b. sink/window kernel: exact attention over the sinks and the window of
+// every KV head.  These rows do not depend on the selection, so this kernel is
+// launched after the select kernel without waiting for it: it runs while the
+// selection runs and waits for the select kernel only before it exits (so its
+// completion implies the selection's).  Everything it reads was finished by
+// rtp_append_kv before the select kernel could start; it reads through L2.
+// ---------------------------------------------------------------------------
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads, 2) sw_kernel(DecodeArgs a) {
+  griddep_launch();
+  __shared__ __align__(16) float s_q[G * D];
+  __shared__ __align__(16) float s_o[kWarps * G * D];
+  __shared__ float s_ml[kWarps * G * 2];
+  const int tid = threadIdx.x;
+  const int idx = blockIdx.x;
   const int tile = idx % a.n_sw_tiles;
   const int bkv = idx / a.n_sw_tiles;
   const int b = bkv / a.Hkv, h = bkv % a.Hkv;
   const int L = a.seq_len[b];
   if (!seq_ok(L, a)) {
     if (tile == 0 && h == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
+    griddep_wait();
     return;
   }
   const int s_cnt = min(a.S, L);
@@ -444,12 +474,15 @@ __global__ void __launch_bounds__(kThreads) stream_kernel(DecodeArgs a) {
   wa.load(kb, vb, row, ok ? ((1u << G) - 1u) : 0u);  // in flight during RoPE
   rope_query<T, D, G>(a, b, h, L - 1, s_q);
   __syncthreads();
+  if (tile == 0)  // the gather kernel reuses this KV head's RoPE'd queries
+    for (int e2 = tid; e2 < G * D; e2 += kThreads) a.qrope[(size_t)bkv * G * D + e2] = s_q[e2];
   wa.compute(s_q);
   write_partial<D, G>(a, wa, (size_t)bkv * a.n_parts_max + tile, s_o, s_ml);
+  griddep_wait();  // complete only after the selection has
 }
 
 // ---------------------------------------------------------------------------
-// 2. select kernel (cluster per head): exact top-p threshold + bitmask
+// 2a. select kernel (cluster per head): exact top-p threshold + bitmask
 // ---------------------------------------------------------------------------
 template <int CS>
 struct SelShared {
@@ -471,6 +504,16 @@ struct SelShared {
 // rounds to zero adds nothing and is skipped.
 __device__ __forceinline__ unsigned long long mass_fx36(float s, float m) {
   return __float2ull_rn(expf(s - m) * 68719476736.0f);  // 2^36
+}
+// The same integer as two 32-bit halves, hi * 2^18 + lo, computed in fp32
+// without a 64-bit conversion: x = e^(s-m) 2^36 is exact (power-of-two
+// scale); hi = floor(x / 2^18) and x - hi 2^18 are exact; rounding the
+// remainder gives rint(x) - hi 2^18 because hi 2^18 is an even integer.
+__device__ __forceinline__ void mass_split36(float s, float m, unsigned& hi, unsigned& lo) {
+  const float x = expf(s - m) * 68719476736.0f;
+  const float hf = floorf(x * 3.814697265625e-06f);  // 2^-18
+  hi = (unsigned)hf;
+  lo = __float2uint_rn(fmaf(hf, -262144.0f, x));
 }
 
 struct DigitResult {
@@ -751,13 +794,24 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads) select
     __syncthreads();
     for (int f0 = c0; f0 < c1; f0 += kFold) {
       const int f1 = min(c1, f0 + kFold);
-      for (int j = f0 + tid; j < f1; j += kSelThreads) {
-        const float sv = s_lg[j - c0];
-        const unsigned long long w = sv > m - 25.0f ? mass_fx36(sv, m) : 0ull;  // e^-25 < 2^-36
-        if (w) {
-          const int bk = score_bucket(sv);
-          atomicAdd(&s_hi[bk], (unsigned)(w >> 18));
-          atomicAdd(&s_lo[bk], (unsigned)(w & 0x3ffffu));
+      for (int j = f0 + tid; j < f1; j += 4 * kSelThreads) {  // 4 independent scores per step
+        float sv[4];
+        bool on[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int jj = j + u * kSelThreads;
+          on[u] = jj < f1;
+          sv[u] = on[u] ? s_lg[jj - c0] : -CUDART_INF_F;
+          on[u] = on[u] && sv[u] > m - 25.0f;  // e^-25 < 2^-36: adds nothing
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (!on[u]) continue;
+          unsigned hi, lo;
+          mass_split36(sv[u], m, hi, lo);
+          const int bk = score_bucket(sv[u]);
+          if (hi) atomicAdd(&s_hi[bk], hi);
+          if (lo) atomicAdd(&s_lo[bk], lo);
         }
       }
       __syncthreads();
@@ -847,21 +901,29 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads) select
         stage(c0, c1);
         __syncthreads();
       }
-      for (int jb = c0; jb < c1; jb += kSelThreads) {
-        const int j = jb + tid;
-        float sv = 0.f;
-        bool in = false;
-        if (j < c1) {
-          sv = s_lg[j - c0];
-          in = score_bucket(sv) == bucket && sv > m - 25.0f && mass_fx36(sv, m) != 0ull;
+      for (int jb = c0; jb < c1; jb += 4 * kSelThreads) {
+        float sv[4];
+        bool in[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = jb + u * kSelThreads + tid;
+          in[u] = false;
+          sv[u] = 0.f;
+          if (j < c1) {
+            sv[u] = s_lg[j - c0];
+            in[u] = score_bucket(sv[u]) == bucket && sv[u] > m - 25.0f && mass_fx36(sv[u], m) != 0ull;
+          }
         }
-        const unsigned bal = __ballot_sync(0xffffffffu, in);
-        if (bal) {
-          unsigned base = 0u;
-          if (lane == 0) base = atomicAdd(&lead->n_cand, (unsigned)__popc(bal));
-          base = __shfl_sync(0xffffffffu, base, 0);
-          const unsigned slot = base + __popc(bal & ((1u << lane) - 1u));
-          if (in) gcand[slot] = make_uint2(score_key(sv), (unsigned)j);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const unsigned bal = __ballot_sync(0xffffffffu, in[u]);
+          if (bal) {
+            unsigned base = 0u;
+            if (lane == 0) base = atomicAdd(&lead->n_cand, (unsigned)__popc(bal));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            const unsigned slot = base + __popc(bal & ((1u << lane) - 1u));
+            if (in[u]) gcand[slot] = make_uint2(score_key(sv[u]), (unsigned)(jb + u * kSelThreads + tid));
+          }
         }
       }
     }
@@ -904,16 +966,24 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads) select
       stage(c0, c1);
       __syncthreads();
     }
-    for (int jb = c0; jb < c1; jb += kSelThreads) {
-      const int j = jb + tid;
-      bool in = false;
-      if (j < c1) {
-        const float sv = s_lg[j - c0];
-        in = sv > tau || (sv == tau && j <= jcut);
+    for (int jb = c0; jb < c1; jb += 4 * kSelThreads) {
+      bool in[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = jb + u * kSelThreads + tid;
+        in[u] = false;
+        if (j < c1) {
+          const float sv = s_lg[j - c0];
+          in[u] = sv > tau || (sv == tau && j <= jcut);
+        }
       }
-      const unsigned word = __ballot_sync(0xffffffffu, in);
-      if (lane == 0 && jb + warp * 32 < c1) mask[(jb >> 5) + warp] = word;
-      cnt += in ? 1 : 0;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const unsigned word = __ballot_sync(0xffffffffu, in[u]);
+        const int jw = jb + u * kSelThreads + warp * 32;
+        if (lane == 0 && jw < c1) mask[jw >> 5] = word;
+        cnt += in[u] ? 1 : 0;
+      }
     }
   }
   if (a.sel_count) {
@@ -1016,9 +1086,9 @@ __global__ void __launch_bounds__(kThreads) gather_kernel(DecodeArgs a) {
       {
         const int e = warp * 32 + lane;
         const bool ok = e < n_rows;
-        wa.load(kb, vb, ok ? s_row[e] : 0, ok ? (unsigned)s_msk[e] : 0u);  // in flight during RoPE
+        wa.load(kb, vb, ok ? s_row[e] : 0, ok ? (unsigned)s_msk[e] : 0u);
       }
-      rope_query<T, D, G>(a, b, h, L - 1, s_q);
+      for (int e2 = tid; e2 < G * D; e2 += kThreads) s_q[e2] = __ldcg(a.qrope + (size_t)bkv * G * D + e2);
       __syncthreads();
       for (int it = 0; it < n_it; ++it) {
         if (it > 0) {
@@ -1092,7 +1162,8 @@ cudaError_t launch_pdl(void (*k)(DecodeArgs), dim3 grid, dim3 block, size_t smem
 
 template <typename T, int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int kind, dim3 grid, cudaStream_t st) {
-  if (kind == 0) return launch_pdl(stream_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
+  if (kind == 0) return launch_pdl(score_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
+  if (kind == 2) return launch_pdl(sw_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
   return launch_pdl(gather_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
 }
 
@@ -1113,34 +1184,37 @@ cudaError_t launch_kind(const Shape& sh, const DecodeArgs& a, int kind, dim3 gri
   return sh.D == 128 ? launch_d<float, 128>(a, kind, grid, st) : launch_d<float, 64>(a, kind, grid, st);
 }
 
-// Cluster size of the select kernel on each device: 16 CTAs where the device
-// can co-schedule several such clusters with the kernel's shared memory, else 8.
-int select_cluster_size() {
-  static int s_cs[64] = {};
+// Cluster size of the select kernel: 16 CTAs when the device can keep all of
+// this call's clusters resident at once, else 8 (its clusters always fit in
+// fewer SMs per GPC); one wave of clusters keeps the kernel as short as one
+// cluster's work.
+int select_cluster_size(int n_clusters_needed) {
+  static int s_max16[64] = {};
+  static bool s_done[64] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  if (s_cs[dev]) return s_cs[dev];
-  cudaFuncSetAttribute(select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<8>::kSmem);
-  cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<16>::kSmem);
-  cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-  int cs = 8;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(16, 1);
-  cfg.blockDim = dim3(kSelThreads);
-  cfg.dynamicSmemBytes = SelCfg<16>::kSmem;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 16;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n_clusters = 0;
-  if (cudaOccupancyMaxActiveClusters(&n_clusters, select_kernel<16>, &cfg) == cudaSuccess && n_clusters >= 4)
-    cs = 16;
-  cudaGetLastError();  // clear a refused query
-  s_cs[dev] = cs;
-  return cs;
+  if (!s_done[dev]) {
+    cudaFuncSetAttribute(select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<8>::kSmem);
+    cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<16>::kSmem);
+    cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(16, 1);
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = SelCfg<16>::kSmem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 16;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, select_kernel<16>, &cfg) != cudaSuccess) n = 0;
+    cudaGetLastError();  // clear a refused query
+    s_max16[dev] = n;
+    s_done[dev] = true;
+  }
+  return (s_max16[dev] >= n_clusters_needed) ? 16 : 8;
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -1163,9 +1237,9 @@ DecodeLayout decode_layout(const Shape& sh) {
   l.cmax = off;   off = align256(off + NRt * l.nch_score_max * sizeof(float));
   l.hmass = off;  off = align256(off + NRt * words * sizeof(uint32_t));  // scratch bitmask
   l.hcnt = off;
-  l.heads = off;
   l.ctl = off;    off = align256(off + (size_t)l.n_ctl * sizeof(unsigned));
   l.cand = off;   off = align256(off + NRt * lstride * sizeof(uint2));
+  l.heads = off;  off = align256(off + (size_t)sh.B * sh.Hkv * sh.G * sh.D * sizeof(float));  // RoPE'd queries
   const size_t nparts = (size_t)sh.B * sh.Hkv * l.n_tiles_max * sh.G;
   l.pm = off;     off = align256(off + nparts * sizeof(float));
   l.pl = off;     off = align256(off + nparts * sizeof(float));
@@ -1193,6 +1267,7 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   a.mask = sel_bitmask ? sel_bitmask : reinterpret_cast<uint32_t*>(w + lay.hmass);
   a.ctl = reinterpret_cast<unsigned*>(w + lay.ctl);
   a.cand = reinterpret_cast<uint2*>(w + lay.cand);
+  a.qrope = reinterpret_cast<float*>(w + lay.heads);
   a.pm = reinterpret_cast<float*>(w + lay.pm);
   a.pl = reinterpret_cast<float*>(w + lay.pl);
   a.po = reinterpret_cast<float*>(w + lay.po);
@@ -1205,19 +1280,28 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   const int n_gtiles = (Lh + kGatherTile - 1) / kGatherTile;
   a.n_score_ctas = sh.R > 0 ? sh.B * sh.R * nch_score : 0;
   a.n_sw_ctas = sh.B * sh.Hkv * lay.n_sw_tiles;
-  const int cs = sh.R > 0 ? select_cluster_size() : 8;
+  const int cs = sh.R > 0 ? select_cluster_size(sh.B * sh.NR) : 8;
 
-  cudaError_t e;
-  trace_begin(RTP_STAGE_DECODE_STREAM, st);
-  e = launch_kind(sh, a, 0, dim3(a.n_score_ctas + a.n_sw_ctas), st);
-  trace_end(RTP_STAGE_DECODE_STREAM, st);
-  if (e == cudaSuccess && sh.R > 0) {
-    trace_begin(RTP_STAGE_DECODE_SELECT, st);
-    if (cs == 16)
-      e = launch_pdl(select_kernel<16>, dim3(16, sh.B * sh.NR), dim3(kSelThreads), SelCfg<16>::kSmem, st, a);
-    else
-      e = launch_pdl(select_kernel<8>, dim3(8, sh.B * sh.NR), dim3(kSelThreads), SelCfg<8>::kSmem, st, a);
-    trace_end(RTP_STAGE_DECODE_SELECT, st);
+  cudaError_t e = cudaSuccess;
+  if (sh.R > 0) {
+    trace_begin(RTP_STAGE_DECODE_STREAM, st);
+    e = launch_kind(sh, a, 0, dim3(a.n_score_ctas), st);
+    trace_end(RTP_STAGE_DECODE_STREAM, st);
+    if (e == cudaSuccess) {
+      trace_begin(RTP_STAGE_DECODE_SELECT, st);
+      if (cs == 16)
+        e = launch_pdl(select_kernel<16>, dim3(16, sh.B * sh.NR), dim3(kSelThreads), SelCfg<16>::kSmem, st, a);
+      else
+        e = launch_pdl(select_kernel<8>, dim3(8, sh.B * sh.NR), dim3(kSelThreads), SelCfg<8>::kSmem, st, a);
+      trace_end(RTP_STAGE_DECODE_SELECT, st);
+    }
+  } else {
+    cudaMemsetAsync(a.ctl, 0, (size_t)a.n_ctl * sizeof(unsigned), st);
+  }
+  if (e == cudaSuccess) {
+    trace_begin(RTP_STAGE_DECODE_SINKWIN, st);
+    e = launch_kind(sh, a, 2, dim3(a.n_sw_ctas), st);
+    trace_end(RTP_STAGE_DECODE_SINKWIN, st);
   }
   if (e == cudaSuccess) {
     trace_begin(RTP_STAGE_DECODE_GATHER, st);
