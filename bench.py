@@ -321,8 +321,7 @@ def run_ours(args, dist: Dist) -> dict:
         raise RuntimeError(f"device status {status} during the timed steps")
 
     # per-kernel CUDA-event timing (same steps, eager launches behind a pre-roll)
-    stages = ["append", "decode_score", "decode_select", "decode_sinkwin", "decode_gather"] if R else \
-        ["append", "decode_sinkwin", "decode_gather"]
+    stages = ["append", "decode_score", "decode_select", "decode_local"] if R else ["append", "decode_local"]
     n_k = args.kernel_steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_k)]
     torch.cuda.synchronize()
@@ -374,8 +373,8 @@ def run_ours(args, dist: Dist) -> dict:
 
     # roofline of the dominant kernel
     dominant = max(kern_us, key=lambda s: kern_us[s])
-    kbytes = {"append": nbytes["append"], "decode_score": nbytes["score"], "decode_sinkwin": nbytes["sw"],
-              "decode_select": 0, "decode_gather": nbytes["kept"] + nbytes["qo"]}
+    kbytes = {"append": nbytes["append"], "decode_score": nbytes["score"], "decode_select": nbytes["kept"],
+              "decode_local": nbytes["sw"] + nbytes["qo"]}
     peaks = {}
     if os.path.exists(PEAKS_PATH):
         peaks = json.load(open(PEAKS_PATH))
@@ -393,7 +392,7 @@ def run_ours(args, dist: Dist) -> dict:
         e2e={"value": e2e_s * 1e6 / (n_e * B * dist.world), "unit": "µs/token",
              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e},
         clocks=(clocks.summary(t_wall0, t_wall1) if clocks else None),
-        gpu_launches=K * (5 if R else 3), l2=l2, inp=inp, Lh=Lh,
+        gpu_launches=K * (4 if R else 2), l2=l2, inp=inp, Lh=Lh,
     )
 
 

@@ -24,10 +24,15 @@ struct AppendArgs {
   void* kidx;
   int* status;
   int ret_rank[kMaxRetrieval];
+  double inv_freq[64];
 };
 
 template <typename T, int D>
 __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
+  // The inputs (k_pre, v, start_pos, W_k) are read and the rotated key and the
+  // indexer key formed before waiting for the previous kernel on the stream;
+  // only the cache stores wait (a decode step still running may read the cache).
+  griddep_launch();
   constexpr int PP = D / 64;  // pairs per lane
   constexpr int H = D / 2;
   const int lane = threadIdx.x & 31;
@@ -44,52 +49,64 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   }
   const T* kp = static_cast<const T*>(a.k_pre) + row * D;
   const T* vp = static_cast<const T*>(a.v_in) + row * D;
-  const size_t dst = (((size_t)b * a.Hkv + h) * a.Lmax + pos) * D;
-  T* ko = static_cast<T*>(a.k) + dst;
-  T* vo = static_cast<T*>(a.v) + dst;
-
   float x1[PP], x2[PP];
+  T v1[PP], v2[PP];
 #pragma unroll
   for (int i = 0; i < PP; ++i) {
     const int k = lane * PP + i;
     x1[i] = to_f32(kp[k]);
     x2[i] = to_f32(kp[k + H]);
-    vo[k] = vp[k];
-    vo[k + H] = vp[k + H];
+    v1[i] = vp[k];
+    v2[i] = vp[k + H];
   }
+  T y1[PP], y2[PP];
 #pragma unroll
   for (int i = 0; i < PP; ++i) {
     const int k = lane * PP + i;
     float c, s;
-    rope_cos_sin(pos, k, D, a.rope_base, c, s);
-    ko[k] = from_f32<T>(x1[i] * c - x2[i] * s);
-    ko[k + H] = from_f32<T>(x2[i] * c + x1[i] * s);
+    rope_cos_sin(pos, a.inv_freq[k], c, s);
+    y1[i] = from_f32<T>(x1[i] * c - x2[i] * s);
+    y2[i] = from_f32<T>(x2[i] * c + x1[i] * s);
   }
-
   const int r = a.ret_rank[h];
-  if (r < 0) return;
-  const float* w = a.w_k + (size_t)r * kIdxDim * D;
   float acc[kIdxDim];
+  if (r >= 0) {  // warp-uniform
+    const float* w = a.w_k + (size_t)r * kIdxDim * D;
 #pragma unroll
-  for (int i = 0; i < kIdxDim; ++i) {
-    float sacc = 0.f;
+    for (int i = 0; i < kIdxDim; ++i) {
+      float sacc = 0.f;
 #pragma unroll
-    for (int p = 0; p < PP; ++p) {
-      const int k = lane * PP + p;
-      sacc = fmaf(__ldg(w + i * D + k), x1[p], sacc);
-      sacc = fmaf(__ldg(w + i * D + k + H), x2[p], sacc);
+      for (int p = 0; p < PP; ++p) {
+        const int k = lane * PP + p;
+        sacc = fmaf(__ldg(w + i * D + k), x1[p], sacc);
+        sacc = fmaf(__ldg(w + i * D + k + H), x2[p], sacc);
+      }
+      acc[i] = sacc;
     }
-    acc[i] = sacc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+#pragma unroll
+      for (int i = 0; i < kIdxDim; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+    }
   }
+  griddep_wait();
+  const size_t dst = (((size_t)b * a.Hkv + h) * a.Lmax + pos) * D;
+  T* ko = static_cast<T*>(a.k) + dst;
+  T* vo = static_cast<T*>(a.v) + dst;
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-#pragma unroll
-    for (int i = 0; i < kIdxDim; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+  for (int i = 0; i < PP; ++i) {
+    const int k = lane * PP + i;
+    ko[k] = y1[i];
+    ko[k + H] = y2[i];
+    vo[k] = v1[i];
+    vo[k + H] = v2[i];
   }
-  T* ki = static_cast<T*>(a.kidx) + (((size_t)b * a.R + r) * a.Lmax + pos) * kIdxDim;
+  if (r >= 0) {
+    T* ki = static_cast<T*>(a.kidx) + (((size_t)b * a.R + r) * a.Lmax + pos) * kIdxDim;
 #pragma unroll
-  for (int i = 0; i < kIdxDim; ++i)
-    if (lane == i) ki[i] = from_f32<T>(acc[i]);
+    for (int i = 0; i < kIdxDim; ++i)
+      if (lane == i) ki[i] = from_f32<T>(acc[i]);
+  }
 }
 
 }  // namespace
@@ -102,19 +119,21 @@ int launch_append(const Shape& sh, const rtp_cache* cache, const void* k_pre, co
   a.k_pre = k_pre; a.v_in = v_in; a.start_pos = start_pos; a.w_k = w_k;
   a.k = cache->k; a.v = cache->v; a.kidx = cache->kidx; a.status = cache->status;
   for (int i = 0; i < kMaxRetrieval; ++i) a.ret_rank[i] = sh.ret_rank[i];
+  for (int i = 0; i < 64; ++i) a.inv_freq[i] = sh.inv_freq[i];
   const long long rows = (long long)sh.B * T * sh.Hkv;
   if (rows == 0) return RTP_OK;
   const unsigned grid = (unsigned)((rows + 7) / 8);
   trace_begin(RTP_STAGE_APPEND, st);
+  cudaError_t e;
   if (sh.dtype == RTP_BF16) {
-    if (sh.D == 128) append_kernel<__nv_bfloat16, 128><<<grid, 256, 0, st>>>(a);
-    else append_kernel<__nv_bfloat16, 64><<<grid, 256, 0, st>>>(a);
+    if (sh.D == 128) e = launch_pdl(append_kernel<__nv_bfloat16, 128>, dim3(grid), dim3(256), 0, st, a);
+    else e = launch_pdl(append_kernel<__nv_bfloat16, 64>, dim3(grid), dim3(256), 0, st, a);
   } else {
-    if (sh.D == 128) append_kernel<float, 128><<<grid, 256, 0, st>>>(a);
-    else append_kernel<float, 64><<<grid, 256, 0, st>>>(a);
+    if (sh.D == 128) e = launch_pdl(append_kernel<float, 128>, dim3(grid), dim3(256), 0, st, a);
+    else e = launch_pdl(append_kernel<float, 64>, dim3(grid), dim3(256), 0, st, a);
   }
   trace_end(RTP_STAGE_APPEND, st);
-  cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("append launch: ") + cudaGetErrorString(e));
     return RTP_ERR_CUDA;

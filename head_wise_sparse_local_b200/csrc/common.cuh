@@ -174,15 +174,37 @@ __device__ __forceinline__ void block_excl_scan2(unsigned long long a, unsigned 
   __syncthreads();
 }
 
-// RoPE angle: pos * base^(-2k/D), reduced to [-pi, pi] in fp64 before the
-// fp32 sincos so that positions up to 2^23 keep full fp32 accuracy.
-__device__ __forceinline__ void rope_cos_sin(int pos, int k, int D, float base, float& c,
-                                             float& s) {
-  const double inv = pow((double)base, -2.0 * (double)k / (double)D);
-  const double th = (double)pos * inv;
+// RoPE angle pos * inv_freq (inv_freq = base^(-2k/D), computed in fp64 on the
+// host), reduced to [-pi, pi] in fp64 before the fp32 sincos so that positions
+// up to 2^23 keep full fp32 accuracy.
+__device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float& c, float& s) {
+  const double th = (double)pos * inv_freq;
   const double two_pi = 6.283185307179586476925286766559;
   const double r = th - two_pi * rint(th / two_pi);
   sincosf((float)r, &s, &c);
+}
+
+// Programmatic dependent launch: a kernel launched with launch_pdl may start
+// while its predecessor on the stream is still running.  griddep_wait() blocks
+// until the predecessor grid has completed and its memory is visible;
+// griddep_launch() lets the successor grid start launching.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+template <typename Args>
+inline cudaError_t launch_pdl(void (*k)(Args), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              const Args& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k, a);
 }
 
 }  // namespace rtp

@@ -1,6 +1,6 @@
 // rtp_decode_attn: one decode step of the head-wise sparse attention layer.
 //
-// Four kernels on the caller's stream, chained with programmatic dependent
+// Three kernels on the caller's stream, chained with programmatic dependent
 // launch, scratch in the caller's workspace:
 //
 //   score_kernel   reads the 16-d indexer-key cache once (two 16-byte loads
@@ -15,16 +15,16 @@
 //                  the bucket where the mass of the highest scores reaches
 //                  ceil(p * Z), gathers that bucket's scores in the leader CTA,
 //                  and the leader resolves the exact threshold score tau and,
-//                  for ties at tau, the last kept index j_cut.  The top-p set
-//                  is written as a bitmask.
+//                  for ties at tau, the last kept index j_cut.  Every CTA then
+//                  writes its share of the top-p bitmask and attends, for its
+//                  query head, the kept rows of its share that lie outside
+//                  the sinks and the window (one partial per CTA).
 //   sw_kernel      exact attention over the sinks and the window of every KV
-//                  head; launched after the select kernel without waiting for
-//                  it, so this HBM stream overlaps the selection.
-//   gather_kernel  for retrieval KV heads: the union over the G query heads
-//                  of the kept rows outside sinks/window, read from the
-//                  bitmask, attended exactly; the last CTA of each KV head
-//                  merges every partial of that head (log-sum-exp) into out.
-//                  Local KV heads only merge their sink/window partials.
+//                  head.  It is launched after the select kernel and does not
+//                  wait for it until its own partial is written, so this HBM
+//                  stream overlaps the selection; then the last CTA of each KV
+//                  head merges every partial of that head (log-sum-exp) into
+//                  the output.
 //
 // Top-p follows the abstract's observation (3) and the atlas.scime.ai summary
 // ("query-adaptive top-p threshold"); sinks + window follow that summary's
@@ -44,12 +44,17 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kScoreChunk = 1024;   // tokens per score CTA (4 per thread)
 constexpr int kSwTile = 256;        // sink/window rows per attention CTA (32 per warp)
-constexpr int kGatherTile = 8192;   // context tokens scanned per gather CTA (256 mask words)
 constexpr int kSelThreads = 512;
-constexpr int kCandSmem = 4096;     // candidates the leader stages in shared memory
+constexpr int kSelWarps = kSelThreads / 32;
+constexpr int kMaxCS = 16;          // largest select cluster
+constexpr int kLgCap = 8192;        // scores a select CTA holds in shared memory
+constexpr int kCandSmem = 4096;     // candidates the leader holds in shared memory
 constexpr int kBruteMax = kSelThreads;  // exact solve by pairwise ranks up to this many candidates
+constexpr int kGroup = 4;           // kept rows a warp attends per memory round trip
+
+// Tokens per score CTA: eight (bf16) or four (fp32) 16-d keys per thread.
+__host__ __device__ constexpr int score_chunk(int esize) { return kThreads * (esize == 2 ? 8 : 4); }
 
 struct DecodeArgs {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W, max_seq_len, words;
@@ -67,19 +72,18 @@ struct DecodeArgs {
   int* sel_count;   // optional [B][NR]
   float* logits;    // [B][NR][lstride]
   float* cmax;      // [B][NR][nch_score_max]
-  float* pm;        // [B][Hkv][n_parts_max][G]
+  float* pm;        // [B][Hkv][n_parts_max][G]: sink/window tiles, then select CTAs
   float* pl;
   float* po;        // [B][Hkv][n_parts_max][G][D]
-  unsigned* ctl;    // [B*Hkv] gather tickets
-  float* qrope;     // [B][Hkv][G][D] RoPE'd, pre-scaled queries (written by the stream kernel)
-  uint2* cand;      // [B][NR][lstride] boundary-bucket candidates (key, index)
-  int n_ctl, nch_score_max, n_sw_tiles, n_parts_max, n_score_ctas, n_sw_ctas;
+  unsigned* ctl;    // [B*Hkv] merge tickets
+  int* rank_cnt;    // [B][NR][kMaxCS] kept tokens per select CTA
+  uint2* cand;      // [B][NR][lstride] boundary-bucket candidates past kCandSmem
+  int n_ctl, nch_score_max, n_sw_tiles, n_parts_max, n_score_ctas, n_sw_ctas, sel_cs;
   int ret_head[kMaxRetrieval];
   int ret_rank[kMaxRetrieval];
+  double inv_freq[64];  // RoPE frequencies, k < D/2
 };
 
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch() { asm volatile("griddepcontrol.launch_dependents;"); }
 
 __device__ __forceinline__ bool seq_ok(int L, const DecodeArgs& a) {
   return L >= 1 && L <= a.max_seq_len;
@@ -98,13 +102,19 @@ __device__ __forceinline__ float block_max(float v, float* sm) {
   return r;
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
-__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+__device__ __forceinline__ unsigned warp_sum_u32(unsigned v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
@@ -134,7 +144,7 @@ __device__ void rope_query(const DecodeArgs& a, int b, int h, int pos, float* s_
     const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * G + g) * D;
     const float x1 = to_f32(q[k]), x2 = to_f32(q[k + D / 2]);
     float c, s;
-    rope_cos_sin(pos, k, D, a.rope_base, c, s);
+    rope_cos_sin(pos, a.inv_freq[k], c, s);
     s_q[g * D + k] = (x1 * c - x2 * s) * qscale;
     s_q[g * D + k + D / 2] = (x2 * c + x1 * s) * qscale;
   }
@@ -312,137 +322,240 @@ __device__ void write_partial(const DecodeArgs& a, WA& wa, size_t part, float* s
   }
 }
 
-// ---------------------------------------------------------------------------
-// 1. score kernel: indexer scores (+ this call's counters zeroed)
-// ---------------------------------------------------------------------------
+// Merge every partial (m, l, o) of KV head (b, h) into the output (one CTA).
+// Stage 1 combines the sink/window partials and runs before the selection has
+// finished; griddep_wait() then waits for the select kernel, and stage 2 adds
+// its n_sel partials (one per select CTA and query head).  Partials with
+// m = -inf are empty and carry weight 0.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) score_kernel(DecodeArgs a) {
-  griddep_wait();
-  griddep_launch();
-  __shared__ __align__(16) float s_q[G * kIdxDim];
-  __shared__ float s_ml[kWarps * G];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (blockIdx.x == 0) {  // zero this call's counters (read by later kernels)
-    for (int i = tid; i < a.n_ctl; i += kThreads) a.ctl[i] = 0u;
-    if (a.sel_count)
-      for (int i = tid; i < a.B * a.NR; i += kThreads) a.sel_count[i] = 0;
+__device__ void merge_partials(const DecodeArgs& a, int b, int h, int n_sel, float* s_buf) {
+  constexpr int kPer = (G * D + kThreads - 1) / kThreads;  // (head, dim) outputs per thread
+  const int tid = threadIdx.x;
+  const int n_sw = a.n_sw_tiles;
+  const size_t pbase = ((size_t)b * a.Hkv + h) * a.n_parts_max;
+  float* s_w = s_buf;                        // [n_parts_max][G] part weights
+  float* s_pl = s_buf + a.n_parts_max * G;   // [n_parts_max][G] part denominators
+  float* s_st = s_pl + a.n_parts_max * G;    // [G][3]: max, denominator, stage-1 scale
+  __syncthreads();
+  for (int i = tid; i < n_sw * G; i += kThreads) {
+    s_w[i] = __ldcg(a.pm + pbase * G + i);
+    s_pl[i] = __ldcg(a.pl + pbase * G + i);
   }
-  {
-    // ---- indexer scores ----
-    const int nch = a.n_score_ctas / (a.B * a.R);
-    const int chunk = blockIdx.x % nch;
-    const int br = blockIdx.x / nch;
-    const int b = br / a.R, r = br % a.R;
-    const int L = a.seq_len[b];
-    if (!seq_ok(L, a)) {
-      if (chunk == 0 && r == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
-      return;
+  __syncthreads();
+  if (tid < G) {
+    float mn = -CUDART_INF_F;
+    for (int t = 0; t < n_sw; ++t) mn = fmaxf(mn, s_w[t * G + tid]);
+    float den = 0.f;
+    for (int t = 0; t < n_sw; ++t) {
+      const float pmv = s_w[t * G + tid];
+      const float w = (pmv == -CUDART_INF_F) ? 0.f : exp2f(pmv - mn);
+      s_w[t * G + tid] = w;
+      den = fmaf(s_pl[t * G + tid], w, den);
     }
-    const int j0 = chunk * kScoreChunk;
-    if (j0 >= L) return;
-    const int j1 = min(L, j0 + kScoreChunk);
-    const int h = a.ret_head[r];
-    // issue this thread's indexer-key loads first (they stay in flight while q~ is formed)
-    constexpr int TPT = kScoreChunk / kThreads;
-    constexpr int NV = kIdxDim * sizeof(T) / 16;
-    const uint4* kidx = reinterpret_cast<const uint4*>(static_cast<const T*>(a.kidx) +
-                                                       ((size_t)b * a.R + r) * a.Lmax * kIdxDim);
-    uint4 kr[TPT][NV];
+    s_st[tid * 3] = mn;
+    s_st[tid * 3 + 1] = den;
+    s_st[tid * 3 + 2] = 1.f;
+  }
+  __syncthreads();
+  float acc[kPer];
 #pragma unroll
-    for (int t = 0; t < TPT; ++t) {
-      const int j = j0 + t * kThreads + tid;
-#pragma unroll
-      for (int v = 0; v < NV; ++v) kr[t][v] = (j < j1) ? __ldg(kidx + (size_t)j * NV + v) : make_uint4(0u, 0u, 0u, 0u);
-    }
-    // q~ = W_q q_pre: four threads per output, a quarter of the dims each
-    float* s_qi = s_q;  // [G][16]
-    for (int o4 = tid; o4 < G * kIdxDim * 4; o4 += kThreads) {
-      const int o = o4 >> 2, qd = o4 & 3;
-      const int g = o / kIdxDim, i = o % kIdxDim;
-      constexpr int DQ = D / 4;
-      const float4* w = reinterpret_cast<const float4*>(a.w_q + ((size_t)r * kIdxDim + i) * D + qd * DQ);
-      const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * G + g) * D + qd * DQ;
-      float wv[DQ], qv[DQ];
-#pragma unroll
-      for (int k = 0; k < DQ / 4; ++k) {
-        const float4 f = __ldg(w + k);
-        wv[4 * k] = f.x; wv[4 * k + 1] = f.y; wv[4 * k + 2] = f.z; wv[4 * k + 3] = f.w;
+  for (int u = 0; u < kPer; ++u) {
+    acc[u] = 0.f;
+    const int i = tid + u * kThreads;
+    if (i < G * D) {
+      const int g = i / D, d = i % D;
+#pragma unroll 4
+      for (int t = 0; t < n_sw; ++t) {
+        const float w = s_w[t * G + g];
+        const float pv = __ldcg(a.po + ((pbase + t) * G + g) * D + d);  // stale if w == 0
+        acc[u] = w > 0.f ? fmaf(pv, w, acc[u]) : acc[u];
       }
-      load_row<T, DQ>(q, qv);
-      float acc = 0.f;
-#pragma unroll
-      for (int k = 0; k < DQ; ++k) acc = fmaf(wv[k], qv[k], acc);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      if (qd == 0) s_qi[g * kIdxDim + i] = acc;
     }
+  }
+  griddep_wait();  // the select kernel's partials are complete
+  if (n_sel > 0) {
+    const size_t sbase = pbase + n_sw;
     __syncthreads();
-    float qr[G][kIdxDim];
-#pragma unroll
-    for (int g = 0; g < G; ++g)
-#pragma unroll
-      for (int i = 0; i < kIdxDim; ++i) qr[g][i] = s_qi[g * kIdxDim + i];
-    float* lg = a.logits + ((size_t)b * a.NR + (size_t)r * G) * a.lstride;
-    float mx[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) mx[g] = -CUDART_INF_F;
-#pragma unroll
-    for (int t = 0; t < TPT; ++t) {
-      const int j = j0 + t * kThreads + tid;
-      if (j >= j1) continue;
-      float kv[kIdxDim];
-      if constexpr (sizeof(T) == 2) {
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kr[t][v]);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 f = __bfloat1622float2(h2[q]);
-            kv[v * 8 + 2 * q] = f.x;
-            kv[v * 8 + 2 * q + 1] = f.y;
-          }
-        }
-      } else {
-#pragma unroll
-        for (int v = 0; v < NV; ++v) {
-          kv[v * 4 + 0] = __uint_as_float(kr[t][v].x); kv[v * 4 + 1] = __uint_as_float(kr[t][v].y);
-          kv[v * 4 + 2] = __uint_as_float(kr[t][v].z); kv[v * 4 + 3] = __uint_as_float(kr[t][v].w);
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float s = 0.f;
-#pragma unroll
-        for (int i = 0; i < kIdxDim; ++i) s = fmaf(qr[g][i], kv[i], s);
-        s = s * kIdxScale + 0.0f;  // exact scaling; +0 turns -0 into +0
-        lg[(size_t)g * a.lstride + j] = s;
-        mx[g] = fmaxf(mx[g], s);
-      }
-    }
-    // one block reduction for the G chunk maxima
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float v = warp_max(mx[g]);
-      if (lane == 0) s_ml[warp * G + g] = v;
+    for (int i = tid; i < n_sel * G; i += kThreads) {
+      s_w[i] = __ldcg(a.pm + sbase * G + i);
+      s_pl[i] = __ldcg(a.pl + sbase * G + i);
     }
     __syncthreads();
     if (tid < G) {
-      float v = s_ml[tid];
-#pragma unroll
-      for (int w = 1; w < kWarps; ++w) v = fmaxf(v, s_ml[w * G + tid]);
-      a.cmax[((size_t)b * a.NR + r * G + tid) * a.nch_score_max + chunk] = v;
+      const float m1 = s_st[tid * 3];
+      float mn = m1;
+      for (int t = 0; t < n_sel; ++t) mn = fmaxf(mn, s_w[t * G + tid]);
+      const float w1 = (m1 == -CUDART_INF_F) ? 0.f : exp2f(m1 - mn);
+      float den = s_st[tid * 3 + 1] * w1;
+      for (int t = 0; t < n_sel; ++t) {
+        const float pmv = s_w[t * G + tid];
+        const float w = (pmv == -CUDART_INF_F) ? 0.f : exp2f(pmv - mn);
+        s_w[t * G + tid] = w;
+        den = fmaf(s_pl[t * G + tid], w, den);
+      }
+      s_st[tid * 3 + 1] = den;
+      s_st[tid * 3 + 2] = w1;
     }
-    return;
+    __syncthreads();
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = tid + u * kThreads;
+      if (i < G * D) {
+        const int g = i / D, d = i % D;
+        float v = acc[u] * s_st[g * 3 + 2];
+#pragma unroll 4
+        for (int t = 0; t < n_sel; ++t) {
+          const float w = s_w[t * G + g];
+          const float pv = __ldcg(a.po + ((sbase + t) * G + g) * D + d);  // stale if w == 0
+          v = w > 0.f ? fmaf(pv, w, v) : v;
+        }
+        acc[u] = v;
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kPer; ++u) {
+    const int i = tid + u * kThreads;
+    if (i < G * D) {
+      const int g = i / D, d = i % D;
+      T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + h * G + g) * D + d;
+      *out = from_f32<T>(acc[u] / s_st[g * 3 + 1]);
+    }
   }
 }
 
 // ---------------------------------------------------------------------------
-// 2b. sink/window kernel: exact attention over the sinks and the window of
-// every KV head.  These rows do not depend on the selection, so this kernel is
-// launched after the select kernel without waiting for it: it runs while the
-// selection runs and waits for the select kernel only before it exits (so its
-// completion implies the selection's).  Everything it reads was finished by
-// rtp_append_kv before the select kernel could start; it reads through L2.
+// 1. score kernel: indexer scores + per-chunk maxima (+ this call's tickets zeroed)
+// ---------------------------------------------------------------------------
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads, 2) score_kernel(DecodeArgs a) {
+  // q~ is formed from the caller's inputs before waiting for rtp_append_kv;
+  // the select kernel may launch meanwhile (it waits for this grid).
+  griddep_launch();
+  constexpr int kChunk = score_chunk(sizeof(T));
+  constexpr int TPT = kChunk / kThreads;        // keys per thread
+  constexpr int NV = kIdxDim * sizeof(T) / 16;  // 16-byte vectors per key
+  __shared__ __align__(16) float s_q[G * kIdxDim];
+  __shared__ float s_ml[kWarps * G];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nch = a.n_score_ctas / (a.B * a.R);
+  const int chunk = blockIdx.x % nch;
+  const int br = blockIdx.x / nch;
+  const int b = br / a.R, r = br % a.R;
+  const int h = a.ret_head[r];
+  const int L = a.seq_len[b];
+  // q~ = W_q q_pre: four threads per output, a quarter of the dims each
+  for (int o4 = tid; o4 < G * kIdxDim * 4; o4 += kThreads) {
+    const int o = o4 >> 2, qd = o4 & 3;
+    const int g = o / kIdxDim, i = o % kIdxDim;
+    constexpr int DQ = D / 4;
+    const float4* w = reinterpret_cast<const float4*>(a.w_q + ((size_t)r * kIdxDim + i) * D + qd * DQ);
+    const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * G + g) * D + qd * DQ;
+    float wv[DQ], qv[DQ];
+#pragma unroll
+    for (int k = 0; k < DQ / 4; ++k) {
+      const float4 f = __ldg(w + k);
+      wv[4 * k] = f.x; wv[4 * k + 1] = f.y; wv[4 * k + 2] = f.z; wv[4 * k + 3] = f.w;
+    }
+    load_row<T, DQ>(q, qv);
+    float acc = 0.f;
+#pragma unroll
+    for (int k = 0; k < DQ; ++k) acc = fmaf(wv[k], qv[k], acc);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    if (qd == 0) s_q[g * kIdxDim + i] = acc;
+  }
+  griddep_wait();  // the appended token's indexer key; the previous call's tickets are done
+  if (blockIdx.x == 0)  // merge tickets of this call
+    for (int i = tid; i < a.n_ctl; i += kThreads) a.ctl[i] = 0u;
+  // The keys are requested up to the call's maximum length without waiting for
+  // seq_len (rows past seq_len are in bounds and their scores are never used).
+  const int j0 = chunk * kChunk;
+  const int jh = min(a.max_seq_len, j0 + kChunk);
+  const uint4* kidx = reinterpret_cast<const uint4*>(static_cast<const T*>(a.kidx) +
+                                                     ((size_t)b * a.R + r) * a.Lmax * kIdxDim);
+  uint4 kr[TPT][NV];
+#pragma unroll
+  for (int t = 0; t < TPT; ++t) {
+    const int j = j0 + t * kThreads + tid;
+#pragma unroll
+    for (int v = 0; v < NV; ++v) kr[t][v] = (j < jh) ? __ldcg(kidx + (size_t)j * NV + v) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  __syncthreads();  // q~ visible
+  if (!seq_ok(L, a)) {
+    if (chunk == 0 && r == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
+    return;
+  }
+  const int j1 = min(L, jh);
+  if (j0 >= j1) return;  // chunk past this sequence's length (uniform over the CTA)
+  float* lg = a.logits + ((size_t)b * a.NR + (size_t)r * G) * a.lstride;
+  float mx[G];
+#pragma unroll
+  for (int g = 0; g < G; ++g) mx[g] = -CUDART_INF_F;
+#pragma unroll
+  for (int t = 0; t < TPT; ++t) {
+    const int j = j0 + t * kThreads + tid;
+    if (j >= j1) continue;
+    float kv[kIdxDim];
+    if constexpr (sizeof(T) == 2) {
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kr[t][v]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __bfloat1622float2(h2[q]);
+          kv[v * 8 + 2 * q] = f.x;
+          kv[v * 8 + 2 * q + 1] = f.y;
+        }
+      }
+    } else {
+#pragma unroll
+      for (int v = 0; v < NV; ++v) {
+        kv[v * 4 + 0] = __uint_as_float(kr[t][v].x); kv[v * 4 + 1] = __uint_as_float(kr[t][v].y);
+        kv[v * 4 + 2] = __uint_as_float(kr[t][v].z); kv[v * 4 + 3] = __uint_as_float(kr[t][v].w);
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float4* q4 = reinterpret_cast<const float4*>(s_q + g * kIdxDim);
+      float s = 0.f;
+#pragma unroll
+      for (int i4 = 0; i4 < kIdxDim / 4; ++i4) {
+        const float4 qq = q4[i4];
+        s = fmaf(qq.x, kv[4 * i4], s);
+        s = fmaf(qq.y, kv[4 * i4 + 1], s);
+        s = fmaf(qq.z, kv[4 * i4 + 2], s);
+        s = fmaf(qq.w, kv[4 * i4 + 3], s);
+      }
+      s = s * kIdxScale + 0.0f;  // exact scaling; +0 turns -0 into +0
+      lg[(size_t)g * a.lstride + j] = s;
+      mx[g] = fmaxf(mx[g], s);
+    }
+  }
+  // one block reduction for the G chunk maxima
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float v = warp_max(mx[g]);
+    if (lane == 0) s_ml[warp * G + g] = v;
+  }
+  __syncthreads();
+  if (tid < G) {
+    float v = s_ml[tid];
+#pragma unroll
+    for (int w = 1; w < kWarps; ++w) v = fmaxf(v, s_ml[w * G + tid]);
+    a.cmax[((size_t)b * a.NR + r * G + tid) * a.nch_score_max + chunk] = v;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 3. sink/window kernel: exact attention over the sinks and the window of
+// every KV head, then the merge.  The sink/window rows do not depend on the
+// selection, so this kernel is launched after the select kernel without
+// waiting for it: it runs while the selection runs.  The last CTA of each KV
+// head merges the sink/window partials, then waits for the select kernel and
+// adds its partials (so this grid completes only after the selection has).
+// Everything it reads before that wait was finished by rtp_append_kv before
+// the select kernel triggered this launch; it reads through L2.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(kThreads, 2) sw_kernel(DecodeArgs a) {
@@ -450,10 +563,10 @@ __global__ void __launch_bounds__(kThreads, 2) sw_kernel(DecodeArgs a) {
   __shared__ __align__(16) float s_q[G * D];
   __shared__ __align__(16) float s_o[kWarps * G * D];
   __shared__ float s_ml[kWarps * G * 2];
+  __shared__ int s_flag;
   const int tid = threadIdx.x;
-  const int idx = blockIdx.x;
-  const int tile = idx % a.n_sw_tiles;
-  const int bkv = idx / a.n_sw_tiles;
+  const int tile = blockIdx.x % a.n_sw_tiles;
+  const int bkv = blockIdx.x / a.n_sw_tiles;
   const int b = bkv / a.Hkv, h = bkv % a.Hkv;
   const int L = a.seq_len[b];
   if (!seq_ok(L, a)) {
@@ -474,29 +587,24 @@ __global__ void __launch_bounds__(kThreads, 2) sw_kernel(DecodeArgs a) {
   wa.load(kb, vb, row, ok ? ((1u << G) - 1u) : 0u);  // in flight during RoPE
   rope_query<T, D, G>(a, b, h, L - 1, s_q);
   __syncthreads();
-  if (tile == 0)  // the gather kernel reuses this KV head's RoPE'd queries
-    for (int e2 = tid; e2 < G * D; e2 += kThreads) a.qrope[(size_t)bkv * G * D + e2] = s_q[e2];
   wa.compute(s_q);
   write_partial<D, G>(a, wa, (size_t)bkv * a.n_parts_max + tile, s_o, s_ml);
-  griddep_wait();  // complete only after the selection has
+  // The last sink/window CTA of this KV head merges; it alone waits for the
+  // selection (so this grid completes only after the select kernel has).
+  if (!take_ticket(&a.ctl[bkv], a.n_sw_tiles, &s_flag)) return;
+  const int r = a.ret_rank[h];
+  merge_partials<T, D, G>(a, b, h, r >= 0 ? a.sel_cs : 0, s_o);
+  if (r >= 0 && a.sel_count && tid < G) {
+    const size_t bh = (size_t)b * a.NR + r * G + tid;
+    int c = 0;
+    for (int q = 0; q < a.sel_cs; ++q) c += __ldcg(a.rank_cnt + bh * kMaxCS + q);
+    a.sel_count[bh] = c;
+  }
 }
 
 // ---------------------------------------------------------------------------
-// 2a. select kernel (cluster per head): exact top-p threshold + bitmask
+// selection helpers
 // ---------------------------------------------------------------------------
-template <int CS>
-struct SelShared {
-  unsigned long long slice[CS];   // per-rank slice totals of the approximate histogram
-  unsigned long long zpart[CS];   // [0]: mass above the boundary bucket (broadcast)
-  int bucket;                     // boundary bucket (broadcast)
-  float tau;                      // final threshold (broadcast)
-  int jcut;
-  unsigned n_cand;                // leader: candidates reserved
-  float red[kSelThreads / 32];
-  unsigned long long scan_a[kSelThreads / 32];
-  unsigned scan_c[kSelThreads / 32];
-};
-
 // Softmax mass exp(s - max) in 2^-36 fixed point.  Integer sums of these are
 // exact and order independent, so the histogram and the exact solve agree bit
 // for bit.  The selection accumulates it per bucket as two 18-bit halves with
@@ -523,20 +631,14 @@ struct DigitResult {
   unsigned cnt_digit;
 };
 
-// Items for the exact solve: a list of (order key, index), or the scores
-// [0, n) of one head themselves (every score is an item).
+// Items for the exact solve: a list of (order key, index) in shared memory,
+// or in global scratch (read through L2: other CTAs of the cluster wrote it).
 struct Items {
   const uint2* list;
-  const float* scores;
-  int bucket;  // scan mode: only scores of this bucket are items
+  bool global;
   __device__ __forceinline__ bool get(int i, uint2& e) const {
-    if (list) {
-      e = list[i];
-      return true;
-    }
-    const float s = scores[i];
-    e = make_uint2(score_key(s), (unsigned)i);
-    return score_bucket(s) == bucket;
+    e = global ? __ldcg(list + i) : list[i];
+    return true;
   }
 };
 
@@ -710,36 +812,82 @@ __device__ void solve_brute(const uint2* items, int n, float m, unsigned long lo
   jcut = *s_jmax;
 }
 
+// Rungs m - rung_delta(k) at which the selection sums mass and count in its first
+// pass: when the scores at or above one rung hold the target mass and number
+// at most kCandSmem, the leader solves over exactly those (no histogram).
+constexpr int kRungs = 6;
+__host__ __device__ constexpr float rung_delta(int k) { return k == 0 ? 0.5f : (float)(1 << (k - 1)); }  // 0.5 .. 16
+
+template <int CS>
+struct SelShared {
+  unsigned long long pre_m[CS][1 + kRungs];  // per rank: Z, then the mass at or above each rung
+  unsigned pre_c[CS][kRungs];                // per rank: count at or above each rung
+  unsigned long long wpre_m[kSelWarps][1 + kRungs];
+  unsigned wpre_c[kSelWarps][kRungs];
+  unsigned long long tot_m[1 + kRungs];      // cluster totals
+  unsigned tot_c[kRungs];
+  unsigned long long slice[CS];   // per-rank slice totals of the histogram
+  unsigned long long zpart[CS];   // [0]: mass above the boundary bucket (broadcast)
+  int bucket;                     // boundary bucket (broadcast)
+  float tau;                      // final threshold (broadcast)
+  int jcut;
+  unsigned n_cand;                // leader: candidates reserved
+  float red[kSelWarps];
+  unsigned long long scan_a[kSelWarps];
+  unsigned scan_c[kSelWarps];
+  int cnt[kSelWarps];
+};
+
 template <int CS>
 struct SelCfg {
-  static constexpr int kLgCap = 131072 / CS;  // scores cached in shared memory per CTA
   static constexpr size_t kSmem = (size_t)kLgCap * sizeof(float) +
                                   kNumBuckets * (2 * sizeof(unsigned) + sizeof(unsigned long long)) +
                                   kBruteMax * sizeof(unsigned long long) + sizeof(SelShared<CS>);
 };
+// The histogram's bytes are reused: by the leader for the candidates, then by
+// every CTA for its warps' kept-row lists (kLgCap / kSelWarps rows per warp).
 static_assert(kNumBuckets * (2 * sizeof(unsigned) + sizeof(unsigned long long)) >= kCandSmem * sizeof(uint2),
-              "the leader stages candidates in the histogram's bytes");
+              "candidates fit in the histogram's bytes");
+static_assert(kNumBuckets * (2 * sizeof(unsigned) + sizeof(unsigned long long)) >= kLgCap * sizeof(int),
+              "row lists fit in the histogram's bytes");
 
 // Every kFold scores the 18-bit halves of the histogram are folded into the
 // 64-bit bins, so no 32-bit sum can overflow.
 constexpr int kFold = 8192;
 
-template <int CS>
-__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads) select_kernel(DecodeArgs a) {
-  griddep_wait();
-  griddep_launch();
-  constexpr int kLgCap = SelCfg<CS>::kLgCap;
+// Raw vector of one lane's D/32 dims of a cache row.
+template <typename T, int D>
+struct LaneRaw {
+  static constexpr int DL = D / 32;
+  static constexpr int VB = DL * sizeof(T);
+  using type = typename std::conditional<VB == 16, uint4,
+               typename std::conditional<VB == 8, uint2,
+               typename std::conditional<VB == 4, unsigned, unsigned short>::type>::type>::type;
+};
+
+// ---------------------------------------------------------------------------
+// 2. select kernel (cluster per retrieval q head): exact top-p threshold,
+// bitmask, and this head's attention over its kept rows outside sinks/window
+// ---------------------------------------------------------------------------
+template <typename T, int D, int CS>
+__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) select_kernel(DecodeArgs a) {
+  constexpr int kChunk = score_chunk(sizeof(T));
+  constexpr int DL = D / 32;
+  using Raw = typename LaneRaw<T, D>::type;
   cg::cluster_group cl = cg::this_cluster();
   const int rank = (int)cl.block_rank();
   const int bh = blockIdx.y;
-  const int b = bh / a.NR;
+  const int b = bh / a.NR, rq = bh % a.NR;
+  const int r = rq / a.G, g = rq % a.G;
+  const int h = a.ret_head[r];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   extern __shared__ __align__(16) unsigned char dsm[];
   float* s_lg = reinterpret_cast<float*>(dsm);                                           // kLgCap
   unsigned* s_hi = reinterpret_cast<unsigned*>(s_lg + kLgCap);                           // 2048
   unsigned* s_lo = s_hi + kNumBuckets;                                                   // 2048
   unsigned long long* s_h = reinterpret_cast<unsigned long long*>(s_lo + kNumBuckets);   // 2048
-  uint2* s_cand = reinterpret_cast<uint2*>(s_hi);  // leader, after the histogram is dead
+  uint2* s_cand = reinterpret_cast<uint2*>(s_hi);  // leader, once the histogram is dead
+  int* s_rows = reinterpret_cast<int*>(s_hi);      // every CTA, once the selection is done
   unsigned long long* s_w = reinterpret_cast<unsigned long long*>(s_h + kNumBuckets);    // kBruteMax
   SelShared<CS>* sh = reinterpret_cast<SelShared<CS>*>(s_w + kBruteMax);
   __shared__ unsigned long long r_hm[256];
@@ -748,423 +896,522 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads) select
   __shared__ uint32_t s_kr[96];
   __shared__ uint32_t s_min;
   __shared__ int s_jmax;
+  __shared__ __align__(16) float s_qh[D];
+  __shared__ __align__(16) float s_wo[kSelWarps * D];
+  __shared__ float s_wml[kSelWarps * 2];
 
-  const int L = a.seq_len[b];
-  if (!seq_ok(L, a)) return;  // uniform over the cluster; the stream kernel flagged it
-  const int per = (((L + CS - 1) / CS) + 31) & ~31;
-  const int j0 = min(L, rank * per);
-  const int j1 = min(L, j0 + per);
-  uint32_t* mask = a.mask + (size_t)bh * a.words;
+  // This CTA's share of the context comes from the call's maximum length, so
+  // the score loads below do not wait for seq_len.
+  const int Lh = a.max_seq_len;
+  const int per = (((Lh + CS - 1) / CS) + 31) & ~31;
+  const int j0 = min(Lh, rank * per);
+  const int jh = min(Lh, j0 + per);
+  const bool cached = (jh - j0) <= kLgCap;  // uniform over the grid
   const float* lg_g = a.logits + (size_t)bh * a.lstride;
-
-  if (a.top_p >= 1.0f) {  // keep every token
-    for (int w = (j0 >> 5) + tid; w < ((j1 + 31) >> 5); w += kSelThreads) {
-      const int nb = min(32, L - w * 32);
-      mask[w] = nb >= 32 ? 0xffffffffu : ((1u << nb) - 1u);
-    }
-    if (rank == 0 && tid == 0 && a.sel_count) a.sel_count[bh] = L;
-    return;
-  }
-
-  // maximum score (per-chunk maxima of the stream kernel)
-  float m = -CUDART_INF_F;
-  {
-    const int nch = (L + kScoreChunk - 1) / kScoreChunk;
-    const float* cm = a.cmax + (size_t)bh * a.nch_score_max;
-    for (int c = tid; c < nch; c += kSelThreads) m = fmaxf(m, cm[c]);
-    m = block_max<kSelThreads>(m, sh->red);
-  }
   // Scores are staged in shared memory kLgCap at a time with 16-byte loads
   // issued together (rows are 16-byte aligned, j0 a multiple of 32); when the
-  // whole range fits, it is staged once and reused by every pass.
-  const bool cached = (j1 - j0) <= kLgCap;
+  // whole share fits, it is staged once and reused by every pass.
   auto stage = [&](int c0, int c1) {
     const float4* src = reinterpret_cast<const float4*>(lg_g + c0);
     float4* dst = reinterpret_cast<float4*>(s_lg);
     const int nv = (c1 - c0 + 3) >> 2;
-#pragma unroll 8
+#pragma unroll 4
     for (int i = tid; i < nv; i += kSelThreads) dst[i] = __ldcg(src + i);
   };
-  for (int i = tid; i < kNumBuckets; i += kSelThreads) { s_hi[i] = 0u; s_lo[i] = 0u; s_h[i] = 0ull; }
-  if (rank == 0 && tid == 0) sh->n_cand = 0u;
-  for (int c0 = j0; c0 < j1; c0 += kLgCap) {
-    const int c1 = min(j1, c0 + kLgCap);
-    __syncthreads();
-    stage(c0, c1);
-    __syncthreads();
-    for (int f0 = c0; f0 < c1; f0 += kFold) {
-      const int f1 = min(c1, f0 + kFold);
-      for (int j = f0 + tid; j < f1; j += 4 * kSelThreads) {  // 4 independent scores per step
-        float sv[4];
-        bool on[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int jj = j + u * kSelThreads;
-          on[u] = jj < f1;
-          sv[u] = on[u] ? s_lg[jj - c0] : -CUDART_INF_F;
-          on[u] = on[u] && sv[u] > m - 25.0f;  // e^-25 < 2^-36: adds nothing
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          if (!on[u]) continue;
-          unsigned hi, lo;
-          mass_split36(sv[u], m, hi, lo);
-          const int bk = score_bucket(sv[u]);
-          if (hi) atomicAdd(&s_hi[bk], hi);
-          if (lo) atomicAdd(&s_lo[bk], lo);
-        }
-      }
-      __syncthreads();
-      for (int i = tid; i < kNumBuckets; i += kSelThreads) {  // fold into the 64-bit bins
-        s_h[i] += ((unsigned long long)s_hi[i] << 18) + s_lo[i];
-        s_hi[i] = 0u;
-        s_lo[i] = 0u;
-      }
-      __syncthreads();
-    }
+  // Before waiting for the score kernel: seq_len and this head's RoPE'd query
+  // (scaled by log2(e)/sqrt(D)) from the caller's inputs.  The trigger comes
+  // only after the wait, so the sink/window kernel starts once the appended
+  // token is in the cache.
+  const int L = a.seq_len[b];
+  if (tid < D / 2 && seq_ok(L, a)) {
+    const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * a.G + g) * D;
+    const float qx1 = to_f32(q[tid]), qx2 = to_f32(q[tid + D / 2]);
+    const float qscale = 1.4426950408889634f * rsqrtf((float)D);
+    float c, s;
+    rope_cos_sin(L - 1, a.inv_freq[tid], c, s);
+    s_qh[tid] = (qx1 * c - qx2 * s) * qscale;
+    s_qh[tid + D / 2] = (qx2 * c + qx1 * s) * qscale;
   }
-  cl.sync();  // (1) every rank's exact histogram is complete
+  griddep_wait();
+  griddep_launch();
+  const int nch_h = (Lh + kChunk - 1) / kChunk;
+  const float* cm = a.cmax + (size_t)bh * a.nch_score_max;
+  const float cm0 = tid < nch_h ? __ldcg(cm + tid) : -CUDART_INF_F;
+  if (cached) stage(j0, jh);
+  if (!seq_ok(L, a)) return;  // uniform over the cluster; the score kernel flagged it
+  const int j1 = min(L, jh);  // j1 <= j0: nothing of this sequence in this CTA's share
+  uint32_t* mask = a.mask + (size_t)bh * a.words;
+  const bool keep_all = a.top_p >= 1.0f;
+  float tau = -CUDART_INF_F;
+  int jcut = INT_MAX;
 
-  // reduce this rank's slice of buckets over the cluster; broadcast its total
-  constexpr int NS = kNumBuckets / CS;
-  {
-    unsigned long long sm_ = 0ull;
-    if (tid < NS) {
-      const int bk = rank * NS + tid;
-#pragma unroll
-      for (int q = 0; q < CS; ++q) sm_ += *cl.map_shared_rank(s_h + bk, q);
-      r_hm[tid] = sm_;
+  if (!keep_all) {  // uniform over the grid
+    // maximum score (per-chunk maxima of the score kernel)
+    float m;
+    {
+      const int nch = (L + kChunk - 1) / kChunk;
+      float v = tid < nch ? cm0 : -CUDART_INF_F;
+      for (int c = tid + kSelThreads; c < nch; c += kSelThreads) v = fmaxf(v, __ldcg(cm + c));
+      m = block_max<kSelThreads>(v, sh->red);
     }
-    unsigned long long ex_m, tot_m;
-    unsigned ex_c, tot_c;
-    block_excl_scan2<kSelThreads>(sm_, 0u, ex_m, ex_c, tot_m, tot_c, sh->scan_a, sh->scan_c);
-    if (tid < CS) cl.map_shared_rank(sh, tid)->slice[rank] = tot_m;
-  }
-  cl.sync();  // (2) slice totals everywhere
+    if (rank == 0 && tid == 0) sh->n_cand = 0u;
+    const float m_lo = m - 26.0f;  // exp(s - m) 2^36 rounds to 0 below m - 25.65
 
-  unsigned long long target;
-  {  // exact boundary bucket: highest buckets live in the highest rank's slice
-    unsigned long long Z = 0ull;
-    for (int q = 0; q < CS; ++q) Z += sh->slice[q];
-    target = (unsigned long long)ceil((double)a.top_p * (double)Z);
-    if (target > Z) target = Z;
-    if (target < 1ull) target = 1ull;
-    int kslice = 0;
-    unsigned long long above_slice = 0ull;
-    for (int q = CS - 1; q >= 0; --q) {
-      if (above_slice + sh->slice[q] >= target) { kslice = q; break; }
-      above_slice += sh->slice[q];
-    }
-    if (rank == kslice && warp == 0) {
-      constexpr int PL = NS / 32;
-      unsigned long long w8[PL];
-      unsigned long long sw = 0ull;
+    // ---- pass 1: the exact total mass Z and, for each rung of the ladder
+    // m - rung_delta(k), the mass and the count of the scores at or above it ----
+    {
+      unsigned long long zs = 0ull, ms[kRungs];
+      unsigned cs[kRungs];
 #pragma unroll
-      for (int k = 0; k < PL; ++k) {
-        w8[k] = r_hm[NS - 1 - (lane * PL + k)];
-        sw += w8[k];
-      }
-      const unsigned long long incl = warp_incl_scan_u64(sw);
-      unsigned long long cum = above_slice + incl - sw;
-      int found = -1;
-      unsigned long long fab = 0ull;
-#pragma unroll
-      for (int k = 0; k < PL; ++k) {
-        if (found < 0 && cum < target && cum + w8[k] >= target) {
-          found = rank * NS + NS - 1 - (lane * PL + k);
-          fab = cum;
+      for (int k = 0; k < kRungs; ++k) { ms[k] = 0ull; cs[k] = 0u; }
+      const float top_lo = m - rung_delta(kRungs - 1);
+      for (int c0 = j0; c0 < j1; c0 += kLgCap) {
+        const int c1 = min(j1, c0 + kLgCap);
+        if (!cached) {
+          __syncthreads();
+          stage(c0, c1);
         }
-        cum += w8[k];
-      }
-      const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
-      const int src = who ? __ffs(who) - 1 : 0;
-      found = who ? __shfl_sync(0xffffffffu, found, src) : -1;
-      fab = __shfl_sync(0xffffffffu, fab, src);
-      if (lane < CS) {
-        SelShared<CS>* rem = cl.map_shared_rank(sh, lane);
-        rem->bucket = found;
-        rem->zpart[0] = fab;  // mass above the boundary bucket
-      }
-    }
-  }
-  cl.sync();  // (3) boundary bucket everywhere
-
-  const int bucket = sh->bucket;
-  const unsigned long long above = sh->zpart[0];
-  uint2* gcand = a.cand + (size_t)bh * a.lstride;
-  if (bucket >= 0) {  // candidates of the boundary bucket -> scratch (order does not matter)
-    SelShared<CS>* lead = cl.map_shared_rank(sh, 0);
-    for (int c0 = j0; c0 < j1; c0 += kLgCap) {
-      const int c1 = min(j1, c0 + kLgCap);
-      if (!cached) {
         __syncthreads();
-        stage(c0, c1);
-        __syncthreads();
-      }
-      for (int jb = c0; jb < c1; jb += 4 * kSelThreads) {
-        float sv[4];
-        bool in[4];
+#pragma unroll 4
+        for (int j = c0 + tid; j < c1; j += kSelThreads) {
+          const float sv = s_lg[j - c0];
+          if (sv > m_lo) {
+            const unsigned long long w = mass_fx36(sv, m);
+            zs += w;
+            if (sv >= top_lo) {
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int j = jb + u * kSelThreads + tid;
-          in[u] = false;
-          sv[u] = 0.f;
-          if (j < c1) {
-            sv[u] = s_lg[j - c0];
-            in[u] = score_bucket(sv[u]) == bucket && sv[u] > m - 25.0f && mass_fx36(sv[u], m) != 0ull;
+              for (int k = 0; k < kRungs; ++k)
+                if (sv >= m - rung_delta(k)) { ms[k] += w; ++cs[k]; }
+            }
           }
         }
+      }
+      // this rank's sums -> every rank of the cluster
+      zs = warp_sum_u64(zs);
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const unsigned bal = __ballot_sync(0xffffffffu, in[u]);
+      for (int k = 0; k < kRungs; ++k) { ms[k] = warp_sum_u64(ms[k]); cs[k] = warp_sum_u32(cs[k]); }
+      if (lane == 0) {
+        sh->wpre_m[warp][0] = zs;
+#pragma unroll
+        for (int k = 0; k < kRungs; ++k) { sh->wpre_m[warp][1 + k] = ms[k]; sh->wpre_c[warp][k] = cs[k]; }
+      }
+      __syncthreads();
+      if (tid < 1 + kRungs) {
+        unsigned long long t = 0ull;
+#pragma unroll
+        for (int w = 0; w < kSelWarps; ++w) t += sh->wpre_m[w][tid];
+#pragma unroll
+        for (int q = 0; q < CS; ++q) cl.map_shared_rank(sh, q)->pre_m[rank][tid] = t;
+      } else if (tid >= 32 && tid < 32 + kRungs) {
+        unsigned t = 0u;
+#pragma unroll
+        for (int w = 0; w < kSelWarps; ++w) t += sh->wpre_c[w][tid - 32];
+#pragma unroll
+        for (int q = 0; q < CS; ++q) cl.map_shared_rank(sh, q)->pre_c[rank][tid - 32] = t;
+      }
+    }
+    cl.sync();  // (A) every rank's sums everywhere
+
+    if (tid < 1 + kRungs) {
+      unsigned long long t = 0ull;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) t += sh->pre_m[q][tid];
+      sh->tot_m[tid] = t;
+    } else if (tid >= 32 && tid < 32 + kRungs) {
+      unsigned t = 0u;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) t += sh->pre_c[q][tid - 32];
+      sh->tot_c[tid - 32] = t;
+    }
+    __syncthreads();
+    const unsigned long long Z = sh->tot_m[0];
+    unsigned long long Mk[kRungs];
+    unsigned Ck[kRungs];
+#pragma unroll
+    for (int k = 0; k < kRungs; ++k) { Mk[k] = sh->tot_m[1 + k]; Ck[k] = sh->tot_c[k]; }
+    unsigned long long target = (unsigned long long)ceil((double)a.top_p * (double)Z);
+    if (target > Z) target = Z;
+    if (target < 1ull) target = 1ull;
+    // lowest rung whose scores already hold the target mass: the kept set lies
+    // at or above it (every other score is ordered after all of those)
+    int kf = -1;
+#pragma unroll
+    for (int k = kRungs - 1; k >= 0; --k)
+      if (Mk[k] >= target) kf = k;
+    const bool fast = kf >= 0 && Ck[kf] <= (unsigned)kCandSmem;
+    float t_lo = m_lo;
+#pragma unroll
+    for (int k = 0; k < kRungs; ++k)
+      if (k == kf) t_lo = m - rung_delta(k);
+
+    uint2* gcand = a.cand + (size_t)bh * a.lstride;
+    SelShared<CS>* lead = cl.map_shared_rank(sh, 0);
+    uint2* lead_cand = cl.map_shared_rank(s_cand, 0);
+    if (fast) {
+      // ---- every score at or above the rung -> the leader; it solves exactly ----
+      for (int c0 = j0; c0 < j1; c0 += kLgCap) {
+        const int c1 = min(j1, c0 + kLgCap);
+        if (!cached) {
+          __syncthreads();
+          stage(c0, c1);
+          __syncthreads();
+        }
+#pragma unroll 4
+        for (int jb = c0; jb < c1; jb += kSelThreads) {
+          const int j = jb + tid;
+          float sv = 0.f;
+          bool in = false;
+          if (j < c1) {
+            sv = s_lg[j - c0];
+            in = sv >= t_lo;
+          }
+          const unsigned bal = __ballot_sync(0xffffffffu, in);
           if (bal) {
             unsigned base = 0u;
             if (lane == 0) base = atomicAdd(&lead->n_cand, (unsigned)__popc(bal));
             base = __shfl_sync(0xffffffffu, base, 0);
-            const unsigned slot = base + __popc(bal & ((1u << lane) - 1u));
-            if (in[u]) gcand[slot] = make_uint2(score_key(sv[u]), (unsigned)(jb + u * kSelThreads + tid));
+            if (in) lead_cand[base + __popc(bal & ((1u << lane) - 1u))] = make_uint2(score_key(sv), (unsigned)j);
           }
         }
       }
-    }
-  }
-  __threadfence();
-  cl.sync();  // (4) candidates complete
-
-  if (rank == 0) {
-    float tau = -CUDART_INF_F;  // no boundary (unreachable): keep every token
-    int jcut = INT_MAX;
-    if (bucket >= 0) {
-      const int n = (int)sh->n_cand;
-      const unsigned long long need = target - above;
-      const uint2* items = gcand;
-      if (n <= kCandSmem) {  // stage them where the histogram was
-        for (int i = tid; i < n; i += kSelThreads) s_cand[i] = __ldcg(gcand + i);
-        __syncthreads();
-        items = s_cand;
+      cl.sync();  // (B) the leader holds every item
+      if (rank == 0) {
+        const int n = (int)sh->n_cand;  // == Ck[kf] <= kCandSmem
+        float t_tau;
+        int t_jcut;
+        if (n <= kBruteMax)
+          solve_brute(s_cand, n, m, target, s_w, &s_min, &s_jmax, t_tau, t_jcut);
+        else
+          solve_radix(Items{s_cand, false}, n, m, target, r_hm, r_hc, &s_dres, s_kr, t_tau, t_jcut);
+        if (tid < CS) {
+          SelShared<CS>* rem = cl.map_shared_rank(sh, tid);
+          rem->tau = t_tau;
+          rem->jcut = t_jcut;
+        }
       }
-      if (n <= kBruteMax)
-        solve_brute(items, n, m, need, s_w, &s_min, &s_jmax, tau, jcut);
-      else
-        solve_radix(Items{items, nullptr, bucket}, n, m, need, r_hm, r_hc, &s_dres, s_kr, tau, jcut);
-    }
-    if (tid < CS) {
-      SelShared<CS>* rem = cl.map_shared_rank(sh, tid);
-      rem->tau = tau;
-      rem->jcut = jcut;
-    }
-  }
-  cl.sync();  // (5) final threshold everywhere (no DSMEM access after this)
+      cl.sync();  // (C) final threshold everywhere (no DSMEM access after this)
+    } else {
+      // ---- 2048-bucket histogram of the scores at or above the rung ----
+      for (int i = tid; i < kNumBuckets; i += kSelThreads) { s_hi[i] = 0u; s_lo[i] = 0u; s_h[i] = 0ull; }
+      for (int c0 = j0; c0 < j1; c0 += kLgCap) {
+        const int c1 = min(j1, c0 + kLgCap);
+        if (!cached) {
+          __syncthreads();
+          stage(c0, c1);
+        }
+        __syncthreads();
+        for (int f0 = c0; f0 < c1; f0 += kFold) {
+          const int f1 = min(c1, f0 + kFold);
+          for (int j = f0 + tid; j < f1; j += 4 * kSelThreads) {  // 4 independent scores per step
+            float sv[4];
+            bool on[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int jj = j + u * kSelThreads;
+              on[u] = jj < f1;
+              sv[u] = on[u] ? s_lg[jj - c0] : -CUDART_INF_F;
+              on[u] = on[u] && sv[u] > m_lo && sv[u] >= t_lo;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if (!on[u]) continue;
+              unsigned hi, lo;
+              mass_split36(sv[u], m, hi, lo);
+              const int bk = score_bucket(sv[u]);
+              if (hi) atomicAdd(&s_hi[bk], hi);
+              if (lo) atomicAdd(&s_lo[bk], lo);
+            }
+          }
+          __syncthreads();
+          for (int i = tid; i < kNumBuckets; i += kSelThreads) {  // fold into the 64-bit bins
+            s_h[i] += ((unsigned long long)s_hi[i] << 18) + s_lo[i];
+            s_hi[i] = 0u;
+            s_lo[i] = 0u;
+          }
+          __syncthreads();
+        }
+      }
+      cl.sync();  // (1) every rank's histogram is complete
 
-  const float tau = sh->tau;
-  const int jcut = sh->jcut;
+      // reduce this rank's slice of buckets over the cluster; broadcast its total
+      constexpr int NS = kNumBuckets / CS;
+      {
+        unsigned long long sm_ = 0ull;
+        if (tid < NS) {
+          const int bk = rank * NS + tid;
+#pragma unroll
+          for (int q = 0; q < CS; ++q) sm_ += *cl.map_shared_rank(s_h + bk, q);
+          r_hm[tid] = sm_;
+        }
+        unsigned long long ex_m, tot_m;
+        unsigned ex_c, tot_c;
+        block_excl_scan2<kSelThreads>(sm_, 0u, ex_m, ex_c, tot_m, tot_c, sh->scan_a, sh->scan_c);
+        if (tid < CS) cl.map_shared_rank(sh, tid)->slice[rank] = tot_m;
+      }
+      cl.sync();  // (2) slice totals everywhere
+
+      {  // boundary bucket: the histogram holds every score at or above the
+         // rung, whose mass reaches the target; highest buckets live in the
+         // highest rank's slice
+        int kslice = 0;
+        unsigned long long above_slice = 0ull;
+        for (int q = CS - 1; q >= 0; --q) {
+          if (above_slice + sh->slice[q] >= target) { kslice = q; break; }
+          above_slice += sh->slice[q];
+        }
+        if (rank == kslice && warp == 0) {
+          constexpr int PL = NS / 32;
+          unsigned long long w8[PL];
+          unsigned long long sw = 0ull;
+#pragma unroll
+          for (int k = 0; k < PL; ++k) {
+            w8[k] = r_hm[NS - 1 - (lane * PL + k)];
+            sw += w8[k];
+          }
+          const unsigned long long incl = warp_incl_scan_u64(sw);
+          unsigned long long cum = above_slice + incl - sw;
+          int found = -1;
+          unsigned long long fab = 0ull;
+#pragma unroll
+          for (int k = 0; k < PL; ++k) {
+            if (found < 0 && cum < target && cum + w8[k] >= target) {
+              found = rank * NS + NS - 1 - (lane * PL + k);
+              fab = cum;
+            }
+            cum += w8[k];
+          }
+          const unsigned who = __ballot_sync(0xffffffffu, found >= 0);
+          const int src = who ? __ffs(who) - 1 : 0;
+          found = who ? __shfl_sync(0xffffffffu, found, src) : -1;
+          fab = __shfl_sync(0xffffffffu, fab, src);
+          if (lane < CS) {
+            SelShared<CS>* rem = cl.map_shared_rank(sh, lane);
+            rem->bucket = found;
+            rem->zpart[0] = fab;  // mass above the boundary bucket
+          }
+        }
+      }
+      cl.sync();  // (3) boundary bucket everywhere; every histogram is dead
+
+      // Candidates of the boundary bucket go straight into the leader's shared
+      // memory (order does not matter); past kCandSmem into global scratch.
+      // Scores of that bucket below the rung may join: they are ordered after
+      // the ones above it, whose mass already covers what is needed.
+      const int bucket = sh->bucket;
+      const unsigned long long above = sh->zpart[0];
+      bool wrote_global = false;
+      if (bucket >= 0) {
+        for (int c0 = j0; c0 < j1; c0 += kLgCap) {
+          const int c1 = min(j1, c0 + kLgCap);
+          if (!cached) {
+            __syncthreads();
+            stage(c0, c1);
+            __syncthreads();
+          }
+          for (int jb = c0; jb < c1; jb += 4 * kSelThreads) {
+            float sv[4];
+            bool in[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int j = jb + u * kSelThreads + tid;
+              in[u] = false;
+              sv[u] = 0.f;
+              if (j < c1) {
+                sv[u] = s_lg[j - c0];
+                in[u] = sv[u] > m_lo && score_bucket(sv[u]) == bucket && mass_fx36(sv[u], m) != 0ull;
+              }
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const unsigned bal = __ballot_sync(0xffffffffu, in[u]);
+              if (bal) {
+                unsigned base = 0u;
+                if (lane == 0) base = atomicAdd(&lead->n_cand, (unsigned)__popc(bal));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                const unsigned slot = base + __popc(bal & ((1u << lane) - 1u));
+                if (in[u]) {
+                  const uint2 item = make_uint2(score_key(sv[u]), (unsigned)(jb + u * kSelThreads + tid));
+                  if (slot < (unsigned)kCandSmem) {
+                    lead_cand[slot] = item;
+                  } else {
+                    gcand[slot] = item;
+                    wrote_global = true;
+                  }
+                }
+              }
+            }
+          }
+        }
+      }
+      if (wrote_global) __threadfence();
+      cl.sync();  // (4) candidates complete
+
+      if (rank == 0) {
+        float t_tau = -CUDART_INF_F;  // no boundary (unreachable): keep every token
+        int t_jcut = INT_MAX;
+        if (bucket >= 0) {
+          const int n = (int)sh->n_cand;
+          const unsigned long long need = target - above;
+          Items items{s_cand, false};
+          if (n > kCandSmem) {  // the list continues in global scratch: put its head there too
+            for (int i = tid; i < kCandSmem; i += kSelThreads) gcand[i] = s_cand[i];
+            __threadfence();
+            __syncthreads();
+            items = Items{gcand, true};
+          }
+          if (n <= kBruteMax)
+            solve_brute(s_cand, n, m, need, s_w, &s_min, &s_jmax, t_tau, t_jcut);
+          else
+            solve_radix(items, n, m, need, r_hm, r_hc, &s_dres, s_kr, t_tau, t_jcut);
+        }
+        if (tid < CS) {
+          SelShared<CS>* rem = cl.map_shared_rank(sh, tid);
+          rem->tau = t_tau;
+          rem->jcut = t_jcut;
+        }
+      }
+      cl.sync();  // (5) final threshold everywhere (no DSMEM access after this)
+    }
+    tau = sh->tau;
+    jcut = sh->jcut;
+  }
+
+  // ---- bitmask, then this head's attention over its kept rows outside
+  // sinks/window: each warp lists the rows of its own positions and attends
+  // them kGroup at a time (keys and values of a group in one round trip) ----
+  const int s_cnt = min(a.S, L);
+  const int sw0 = max(s_cnt, L - a.W);
+  const T* kb = static_cast<const T*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+  const T* vb = static_cast<const T*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+  int* wrows = s_rows + warp * (kLgCap / kSelWarps);
+  __syncthreads();  // s_qh visible
+  float qv[DL];
+#pragma unroll
+  for (int d = 0; d < DL; ++d) qv[d] = s_qh[lane * DL + d];
+  float am = -CUDART_INF_F, al = 0.f, ao[DL];
+#pragma unroll
+  for (int d = 0; d < DL; ++d) ao[d] = 0.f;
   int cnt = 0;
   for (int c0 = j0; c0 < j1; c0 += kLgCap) {
     const int c1 = min(j1, c0 + kLgCap);
     if (!cached) {
       __syncthreads();
       stage(c0, c1);
-      __syncthreads();
     }
-    for (int jb = c0; jb < c1; jb += 4 * kSelThreads) {
-      bool in[4];
+    __syncthreads();  // staged scores visible; the row lists' bytes are free
+    int wn = 0;
+#pragma unroll 4
+    for (int jb = c0; jb < c1; jb += kSelThreads) {
+      const int j = jb + tid;
+      bool in = false;
+      if (j < c1) {
+        const float sv = s_lg[j - c0];
+        in = keep_all || sv > tau || (sv == tau && j <= jcut);
+      }
+      const unsigned word = __ballot_sync(0xffffffffu, in);
+      const int jw = jb + warp * 32;
+      if (lane == 0 && jw < c1) mask[jw >> 5] = word;
+      cnt += in ? 1 : 0;
+      const bool o = in && j >= s_cnt && j < sw0;
+      const unsigned ob = __ballot_sync(0xffffffffu, o);
+      if (o) wrows[wn + __popc(ob & ((1u << lane) - 1u))] = j;
+      wn += __popc(ob);
+    }
+    __syncwarp();
+    for (int i0 = 0; i0 < wn; i0 += kGroup) {  // wn is warp-uniform
+      int rw[kGroup];
+      Raw kr[kGroup], vr[kGroup];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int j = jb + u * kSelThreads + tid;
-        in[u] = false;
-        if (j < c1) {
-          const float sv = s_lg[j - c0];
-          in[u] = sv > tau || (sv == tau && j <= jcut);
+      for (int k = 0; k < kGroup; ++k) {
+        kr[k] = Raw();
+        vr[k] = Raw();
+        rw[k] = (i0 + k < wn) ? wrows[i0 + k] : -1;
+        if (rw[k] >= 0) {
+          kr[k] = __ldcg(reinterpret_cast<const Raw*>(kb + (size_t)rw[k] * D + lane * DL));
+          vr[k] = __ldcg(reinterpret_cast<const Raw*>(vb + (size_t)rw[k] * D + lane * DL));
         }
       }
+      float sc[kGroup];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const unsigned word = __ballot_sync(0xffffffffu, in[u]);
-        const int jw = jb + u * kSelThreads + warp * 32;
-        if (lane == 0 && jw < c1) mask[jw >> 5] = word;
-        cnt += in[u] ? 1 : 0;
+      for (int k = 0; k < kGroup; ++k) {
+        const T* kt = reinterpret_cast<const T*>(&kr[k]);
+        float s = 0.f;
+#pragma unroll
+        for (int d = 0; d < DL; ++d) s = fmaf(qv[d], to_f32(kt[d]), s);
+        sc[k] = s;
       }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int k = 0; k < kGroup; ++k) sc[k] += __shfl_xor_sync(0xffffffffu, sc[k], o);
+      float mx = -CUDART_INF_F;
+#pragma unroll
+      for (int k = 0; k < kGroup; ++k)
+        if (rw[k] >= 0) mx = fmaxf(mx, sc[k]);
+      const float mn = fmaxf(am, mx);
+      const float alpha = exp2f(am - mn);  // 0 while nothing was attended (am = -inf)
+      al *= alpha;
+#pragma unroll
+      for (int d = 0; d < DL; ++d) ao[d] *= alpha;
+#pragma unroll
+      for (int k = 0; k < kGroup; ++k) {
+        if (rw[k] < 0) continue;
+        const float e = exp2f(sc[k] - mn);
+        const T* vt = reinterpret_cast<const T*>(&vr[k]);
+        al += e;
+#pragma unroll
+        for (int d = 0; d < DL; ++d) ao[d] = fmaf(e, to_f32(vt[d]), ao[d]);
+      }
+      am = mn;
     }
   }
-  if (a.sel_count) {
-    cnt = warp_sum_i(cnt);
-    if (lane == 0 && cnt) atomicAdd(&a.sel_count[bh], cnt);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// 3. gather kernel: kept rows outside sinks/window + log-sum-exp merge
-// ---------------------------------------------------------------------------
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads) gather_kernel(DecodeArgs a) {
-  griddep_wait();
-  griddep_launch();
-  // The row list and the warp-merge buffer are never live at the same time.
-  constexpr size_t kRowBytes = (size_t)kGatherTile * (sizeof(int) + 1);
-  constexpr size_t kMergeBytes = (size_t)kWarps * G * D * sizeof(float);
-  __shared__ __align__(16) unsigned char s_buf[kRowBytes > kMergeBytes ? kRowBytes : kMergeBytes];
-  __shared__ __align__(16) float s_q[G * D];
-  __shared__ float s_ml[kWarps * G * 2];
-  __shared__ unsigned s_wcnt[kWarps];
-  __shared__ int s_flag;
-  int* s_row = reinterpret_cast<int*>(s_buf);
-  unsigned char* s_msk = s_buf + (size_t)kGatherTile * sizeof(int);
-  float* s_o = reinterpret_cast<float*>(s_buf);
-  const int tile = blockIdx.x;
-  const int bkv = blockIdx.y;
-  const int b = bkv / a.Hkv, h = bkv % a.Hkv;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int r = a.ret_rank[h];
-  const int L = a.seq_len[b];
-  if (!seq_ok(L, a)) return;
-  const size_t pbase = (size_t)bkv * a.n_parts_max;
-  int n_parts = a.n_sw_tiles;
-  if (r >= 0) {
-    const int s_cnt = min(a.S, L);
-    const int sw0 = max(s_cnt, L - a.W);
-    const int jt0 = tile * kGatherTile;
-    int n_rows = 0;
-    if (jt0 < L) {
-      // union of the G heads' kept rows in [jt0, jt0 + kGatherTile), outside sinks/window
-      unsigned wg[G];
-      unsigned uni = 0u;
-      const int w = (jt0 >> 5) + tid;  // one 32-token word per thread
-      const int jw = w * 32;
+  // merge the warps' states into this CTA's partial for query head g
+  cnt = warp_sum_i(cnt);
 #pragma unroll
-      for (int g = 0; g < G; ++g) wg[g] = 0u;
-      if (jw < L) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          wg[g] = a.mask[((size_t)b * a.NR + r * G + g) * a.words + w];
-          uni |= wg[g];
-        }
-        // keep positions in [s_cnt, sw0): drop sinks, window and positions >= L
-        const int lo = max(0, s_cnt - jw), hi = min(32, sw0 - jw);
-        if (hi <= lo) uni = 0u;
-        else {
-          const unsigned keep_hi = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
-          const unsigned keep_lo = lo <= 0 ? 0xffffffffu : ~((1u << lo) - 1u);
-          uni &= keep_hi & keep_lo;
-        }
-      }
-      const unsigned cntw = __popc(uni);
-      unsigned incl = cntw;  // block exclusive scan of cntw, in index order
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const unsigned n2 = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n2;
-      }
-      if (lane == 31) s_wcnt[warp] = incl;
-      __syncthreads();
-      unsigned off = incl - cntw;
-      unsigned tot = 0u;
-#pragma unroll
-      for (int q = 0; q < kWarps; ++q) {
-        if (q < warp) off += s_wcnt[q];
-        tot += s_wcnt[q];
-      }
-      unsigned bits = uni;
-      while (bits) {
-        const int k = __ffs(bits) - 1;
-        bits &= bits - 1u;
-        unsigned msk = 0u;
-#pragma unroll
-        for (int g = 0; g < G; ++g) msk |= ((wg[g] >> k) & 1u) << g;
-        s_row[off] = jw + k;
-        s_msk[off] = (unsigned char)msk;
-        ++off;
-      }
-      n_rows = (int)tot;
-      __syncthreads();
-    }
-    if (n_rows > 0) {
-      WarpAttn<T, D, G> wa;
-      wa.init();
-      const T* kb = static_cast<const T*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
-      const T* vb = static_cast<const T*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
-      const int n_it = (n_rows + kThreads - 1) / kThreads;  // same trip count in every warp
-      {
-        const int e = warp * 32 + lane;
-        const bool ok = e < n_rows;
-        wa.load(kb, vb, ok ? s_row[e] : 0, ok ? (unsigned)s_msk[e] : 0u);
-      }
-      for (int e2 = tid; e2 < G * D; e2 += kThreads) s_q[e2] = __ldcg(a.qrope + (size_t)bkv * G * D + e2);
-      __syncthreads();
-      for (int it = 0; it < n_it; ++it) {
-        if (it > 0) {
-          const int e = it * kThreads + warp * 32 + lane;
-          const bool ok = e < n_rows;
-          wa.load(kb, vb, ok ? s_row[e] : 0, ok ? (unsigned)s_msk[e] : 0u);
-        }
-        wa.compute(s_q);
-      }
-      __syncthreads();  // the row list is dead; its bytes become the merge buffer
-      write_partial<D, G>(a, wa, pbase + a.n_sw_tiles + tile, s_o, s_ml);
-    } else if (tid < G) {
-      a.pm[(pbase + a.n_sw_tiles + tile) * G + tid] = -CUDART_INF_F;
-      a.pl[(pbase + a.n_sw_tiles + tile) * G + tid] = 0.f;
-    }
-    if (!take_ticket(&a.ctl[bkv], gridDim.x, &s_flag)) return;
-    n_parts = a.n_sw_tiles + gridDim.x;
-  } else if (tile != 0) {
-    return;  // local KV heads: tile 0 merges the sink/window partials
-  }
-  // ---- merge all partials of this KV head ----
-  float* s_pm = s_o;  // [n_parts][G] (reuse)
-  float* s_pl = s_o + a.n_parts_max * G;
-  __syncthreads();
-  for (int i = tid; i < n_parts * G; i += kThreads) {
-    s_pm[i] = __ldcg(a.pm + pbase * G + i);
-    s_pl[i] = __ldcg(a.pl + pbase * G + i);
+  for (int d = 0; d < DL; ++d) s_wo[warp * D + lane * DL + d] = ao[d];
+  if (lane == 0) {
+    s_wml[warp * 2] = am;
+    s_wml[warp * 2 + 1] = al;
+    sh->cnt[warp] = cnt;
   }
   __syncthreads();
-  if (tid < G) {  // per-part weights exp2(m_t - max) (0 for empty parts)
+  const size_t slot = (((size_t)b * a.Hkv + h) * a.n_parts_max + a.n_sw_tiles + rank) * a.G + g;
+  for (int d = tid; d < D; d += kSelThreads) {
     float mn = -CUDART_INF_F;
-    for (int t = 0; t < n_parts; ++t) mn = fmaxf(mn, s_pm[t * G + tid]);
-    for (int t = 0; t < n_parts; ++t) {
-      const float pmv = s_pm[t * G + tid];
-      s_pm[t * G + tid] = (pmv == -CUDART_INF_F) ? 0.f : exp2f(pmv - mn);
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) mn = fmaxf(mn, s_wml[w * 2]);
+    float acc = 0.f, den = 0.f;
+    if (mn != -CUDART_INF_F) {
+#pragma unroll
+      for (int w = 0; w < kSelWarps; ++w) {
+        const float mw = s_wml[w * 2];
+        if (mw == -CUDART_INF_F) continue;
+        const float sc = exp2f(mw - mn);
+        acc = fmaf(s_wo[w * D + d], sc, acc);
+        den = fmaf(s_wml[w * 2 + 1], sc, den);
+      }
+    }
+    a.po[slot * D + d] = acc;
+    if (d == 0) {
+      a.pm[slot] = mn;
+      a.pl[slot] = den;
     }
   }
-  __syncthreads();
-  for (int i = tid; i < G * D; i += kThreads) {
-    const int g = i / D, d = i % D;
-    float acc = 0.f, den = 0.f;
-#pragma unroll 8
-    for (int t = 0; t < n_parts; ++t) {
-      const float sc = s_pm[t * G + g];
-      const float pv = __ldcg(a.po + ((pbase + t) * G + g) * D + d);  // stale if sc == 0
-      acc = sc > 0.f ? fmaf(pv, sc, acc) : acc;
-      den = fmaf(s_pl[t * G + g], sc, den);
-    }
-    T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + h * G + g) * D + d;
-    *out = from_f32<T>(acc / den);
+  if (tid == 0) {
+    int c = 0;
+#pragma unroll
+    for (int w = 0; w < kSelWarps; ++w) c += sh->cnt[w];
+    a.rank_cnt[(size_t)bh * kMaxCS + rank] = c;
   }
 }
 
 // ---------------------------------------------------------------------------
 // launch helpers
 // ---------------------------------------------------------------------------
-cudaError_t launch_pdl(void (*k)(DecodeArgs), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
-                       const DecodeArgs& a) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k, a);
-}
-
 template <typename T, int D, int G>
 cudaError_t launch_dg(const DecodeArgs& a, int kind, dim3 grid, cudaStream_t st) {
   if (kind == 0) return launch_pdl(score_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
-  if (kind == 2) return launch_pdl(sw_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
-  return launch_pdl(gather_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
+  return launch_pdl(sw_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
 }
 
 template <typename T, int D>
@@ -1184,19 +1431,21 @@ cudaError_t launch_kind(const Shape& sh, const DecodeArgs& a, int kind, dim3 gri
   return sh.D == 128 ? launch_d<float, 128>(a, kind, grid, st) : launch_d<float, 64>(a, kind, grid, st);
 }
 
-// Cluster size of the select kernel: 16 CTAs when the device can keep all of
-// this call's clusters resident at once, else 8 (its clusters always fit in
-// fewer SMs per GPC); one wave of clusters keeps the kernel as short as one
+// Select kernel with 16-CTA clusters when the device can keep all of this
+// call's clusters resident at once, else 8-CTA clusters (which always fit in
+// fewer SMs per GPC): one wave of clusters keeps the kernel as short as one
 // cluster's work.
-int select_cluster_size(int n_clusters_needed) {
+template <typename T, int D>
+cudaError_t launch_select(DecodeArgs& a, int n_clusters, cudaStream_t st) {
   static int s_max16[64] = {};
   static bool s_done[64] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 8;
-  if (!s_done[dev]) {
-    cudaFuncSetAttribute(select_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<8>::kSmem);
-    cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<16>::kSmem);
-    cudaFuncSetAttribute(select_kernel<16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev >= 0 && dev < 64 && !s_done[dev]) {
+    cudaFuncSetAttribute(select_kernel<T, D, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<8>::kSmem);
+    cudaFuncSetAttribute(select_kernel<T, D, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<16>::kSmem);
+    cudaFuncSetAttribute(select_kernel<T, D, 16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(16, 1);
     cfg.blockDim = dim3(kSelThreads);
@@ -1209,12 +1458,23 @@ int select_cluster_size(int n_clusters_needed) {
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, select_kernel<16>, &cfg) != cudaSuccess) n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, select_kernel<T, D, 16>, &cfg) != cudaSuccess) n = 0;
     cudaGetLastError();  // clear a refused query
     s_max16[dev] = n;
     s_done[dev] = true;
   }
-  return (s_max16[dev] >= n_clusters_needed) ? 16 : 8;
+  const int cs = (dev >= 0 && dev < 64 && s_max16[dev] >= n_clusters) ? 16 : 8;
+  a.sel_cs = cs;
+  if (cs == 16)
+    return launch_pdl(select_kernel<T, D, 16>, dim3(16, n_clusters), dim3(kSelThreads), SelCfg<16>::kSmem, st, a);
+  return launch_pdl(select_kernel<T, D, 8>, dim3(8, n_clusters), dim3(kSelThreads), SelCfg<8>::kSmem, st, a);
+}
+
+cudaError_t launch_select_any(const Shape& sh, DecodeArgs& a, int n_clusters, cudaStream_t st) {
+  if (sh.dtype == RTP_BF16)
+    return sh.D == 128 ? launch_select<__nv_bfloat16, 128>(a, n_clusters, st)
+                       : launch_select<__nv_bfloat16, 64>(a, n_clusters, st);
+  return sh.D == 128 ? launch_select<float, 128>(a, n_clusters, st) : launch_select<float, 64>(a, n_clusters, st);
 }
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -1224,26 +1484,24 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 DecodeLayout decode_layout(const Shape& sh) {
   DecodeLayout l;
   const size_t NRt = (size_t)sh.B * sh.NR;
-  l.nch_score_max = (sh.Lmax + kScoreChunk - 1) / kScoreChunk;
-  l.nch_sel_max = (sh.Lmax + kGatherTile - 1) / kGatherTile;
+  const int chunk = score_chunk(sh.esize);
+  l.nch_score_max = (sh.Lmax + chunk - 1) / chunk;
   l.n_sw_tiles = (sh.S + sh.W + kSwTile - 1) / kSwTile;
-  l.n_sel_tiles_max = (sh.Lmax + kGatherTile - 1) / kGatherTile;
-  l.n_tiles_max = l.n_sw_tiles + (sh.R > 0 ? l.n_sel_tiles_max : 0);
+  l.n_tiles_max = l.n_sw_tiles + (sh.R > 0 ? kMaxCS : 0);
   l.n_ctl = (int)((size_t)sh.B * sh.Hkv);
   const size_t words = (size_t)(sh.Lmax + 31) / 32;
   const size_t lstride = ((size_t)sh.Lmax + 31) & ~size_t(31);
   size_t off = 0;
-  l.logits = off; off = align256(off + NRt * lstride * sizeof(float));
-  l.cmax = off;   off = align256(off + NRt * l.nch_score_max * sizeof(float));
-  l.hmass = off;  off = align256(off + NRt * words * sizeof(uint32_t));  // scratch bitmask
-  l.hcnt = off;
-  l.ctl = off;    off = align256(off + (size_t)l.n_ctl * sizeof(unsigned));
-  l.cand = off;   off = align256(off + NRt * lstride * sizeof(uint2));
-  l.heads = off;  off = align256(off + (size_t)sh.B * sh.Hkv * sh.G * sh.D * sizeof(float));  // RoPE'd queries
+  l.logits = off;   off = align256(off + NRt * lstride * sizeof(float));
+  l.cmax = off;     off = align256(off + NRt * l.nch_score_max * sizeof(float));
+  l.mask = off;     off = align256(off + NRt * words * sizeof(uint32_t));  // bitmask when the caller passes none
+  l.ctl = off;      off = align256(off + (size_t)l.n_ctl * sizeof(unsigned));
+  l.rank_cnt = off; off = align256(off + NRt * kMaxCS * sizeof(int));
+  l.cand = off;     off = align256(off + NRt * lstride * sizeof(uint2));
   const size_t nparts = (size_t)sh.B * sh.Hkv * l.n_tiles_max * sh.G;
-  l.pm = off;     off = align256(off + nparts * sizeof(float));
-  l.pl = off;     off = align256(off + nparts * sizeof(float));
-  l.po = off;     off = align256(off + nparts * sh.D * sizeof(float));
+  l.pm = off;       off = align256(off + nparts * sizeof(float));
+  l.pl = off;       off = align256(off + nparts * sizeof(float));
+  l.po = off;       off = align256(off + nparts * sh.D * sizeof(float));
   l.total = off;
   return l;
 }
@@ -1264,49 +1522,41 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   char* w = static_cast<char*>(ws);
   a.logits = reinterpret_cast<float*>(w + lay.logits);
   a.cmax = reinterpret_cast<float*>(w + lay.cmax);
-  a.mask = sel_bitmask ? sel_bitmask : reinterpret_cast<uint32_t*>(w + lay.hmass);
+  a.mask = sel_bitmask ? sel_bitmask : reinterpret_cast<uint32_t*>(w + lay.mask);
   a.ctl = reinterpret_cast<unsigned*>(w + lay.ctl);
+  a.rank_cnt = reinterpret_cast<int*>(w + lay.rank_cnt);
   a.cand = reinterpret_cast<uint2*>(w + lay.cand);
-  a.qrope = reinterpret_cast<float*>(w + lay.heads);
   a.pm = reinterpret_cast<float*>(w + lay.pm);
   a.pl = reinterpret_cast<float*>(w + lay.pl);
   a.po = reinterpret_cast<float*>(w + lay.po);
   a.n_ctl = lay.n_ctl; a.nch_score_max = lay.nch_score_max; a.n_sw_tiles = lay.n_sw_tiles;
   a.n_parts_max = lay.n_tiles_max;
+  a.sel_cs = 0;
   for (int i = 0; i < kMaxRetrieval; ++i) { a.ret_head[i] = sh.ret_head[i]; a.ret_rank[i] = sh.ret_rank[i]; }
+  for (int i = 0; i < 64; ++i) a.inv_freq[i] = sh.inv_freq[i];
 
   const int Lh = a.max_seq_len;
-  const int nch_score = (Lh + kScoreChunk - 1) / kScoreChunk;
-  const int n_gtiles = (Lh + kGatherTile - 1) / kGatherTile;
-  a.n_score_ctas = sh.R > 0 ? sh.B * sh.R * nch_score : 0;
+  const int chunk = score_chunk(sh.esize);
+  a.n_score_ctas = sh.R > 0 ? sh.B * sh.R * ((Lh + chunk - 1) / chunk) : 0;
   a.n_sw_ctas = sh.B * sh.Hkv * lay.n_sw_tiles;
-  const int cs = sh.R > 0 ? select_cluster_size(sh.B * sh.NR) : 8;
 
   cudaError_t e = cudaSuccess;
   if (sh.R > 0) {
-    trace_begin(RTP_STAGE_DECODE_STREAM, st);
+    trace_begin(RTP_STAGE_DECODE_SCORE, st);
     e = launch_kind(sh, a, 0, dim3(a.n_score_ctas), st);
-    trace_end(RTP_STAGE_DECODE_STREAM, st);
+    trace_end(RTP_STAGE_DECODE_SCORE, st);
     if (e == cudaSuccess) {
       trace_begin(RTP_STAGE_DECODE_SELECT, st);
-      if (cs == 16)
-        e = launch_pdl(select_kernel<16>, dim3(16, sh.B * sh.NR), dim3(kSelThreads), SelCfg<16>::kSmem, st, a);
-      else
-        e = launch_pdl(select_kernel<8>, dim3(8, sh.B * sh.NR), dim3(kSelThreads), SelCfg<8>::kSmem, st, a);
+      e = launch_select_any(sh, a, sh.B * sh.NR, st);
       trace_end(RTP_STAGE_DECODE_SELECT, st);
     }
   } else {
-    cudaMemsetAsync(a.ctl, 0, (size_t)a.n_ctl * sizeof(unsigned), st);
+    e = cudaMemsetAsync(a.ctl, 0, (size_t)a.n_ctl * sizeof(unsigned), st);
   }
   if (e == cudaSuccess) {
-    trace_begin(RTP_STAGE_DECODE_SINKWIN, st);
-    e = launch_kind(sh, a, 2, dim3(a.n_sw_ctas), st);
-    trace_end(RTP_STAGE_DECODE_SINKWIN, st);
-  }
-  if (e == cudaSuccess) {
-    trace_begin(RTP_STAGE_DECODE_GATHER, st);
-    e = launch_kind(sh, a, 1, dim3(sh.R > 0 ? n_gtiles : 1, sh.B * sh.Hkv), st);
-    trace_end(RTP_STAGE_DECODE_GATHER, st);
+    trace_begin(RTP_STAGE_DECODE_LOCAL, st);
+    e = launch_kind(sh, a, 1, dim3(a.n_sw_ctas), st);
+    trace_end(RTP_STAGE_DECODE_LOCAL, st);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {

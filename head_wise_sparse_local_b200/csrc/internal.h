@@ -25,6 +25,7 @@ struct Shape {
   int esize;  // bytes per element
   int ret_head[64];  // rank -> kv head
   int ret_rank[64];  // kv head -> rank or -1
+  double inv_freq[64];  // RoPE frequencies base^(-2k/D), k < D/2, fp64 on the host
 };
 
 // Validates cfg and fills Shape; returns RTP_OK or an error (message set).
@@ -32,8 +33,8 @@ int make_shape(const rtp_layer_cfg* cfg, Shape* sh);
 
 // Decode scratch layout (byte offsets into the workspace).
 struct DecodeLayout {
-  size_t logits, cmax, hmass, hcnt, heads, ctl, cand, pm, pl, po, total;
-  int nch_score_max, nch_sel_max, n_sw_tiles, n_sel_tiles_max, n_tiles_max;
+  size_t logits, cmax, mask, ctl, rank_cnt, cand, pm, pl, po, total;
+  int nch_score_max, n_sw_tiles, n_tiles_max;
   int n_ctl;  // u32 control words
 };
 DecodeLayout decode_layout(const Shape& sh);

@@ -47,6 +47,7 @@ struct PrefillArgs {
   uint32_t* mask;  // [B][NR][T][words] top-p bitmask per query row
   int ret_head[kMaxRetrieval];
   int ret_rank[kMaxRetrieval];
+  double inv_freq[64];  // RoPE frequencies, k < D/2
 };
 
 __device__ __forceinline__ unsigned long long mass36(float s, float m) {
@@ -514,7 +515,7 @@ __global__ void __launch_bounds__(128) attn_rows_kernel(PrefillArgs a) {
       const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q_pre) + (((size_t)b * a.T + t) * a.Hq + hq) * D;
       const float x1 = __bfloat162float(q[kk]), x2 = __bfloat162float(q[kk + D / 2]);
       float c, sn;
-      rope_cos_sin(start + t, kk, D, a.rope_base, c, sn);
+      rope_cos_sin(start + t, a.inv_freq[kk], c, sn);
       y1 = (x1 * c - x2 * sn) * qscale;
       y2 = (x2 * c + x1 * sn) * qscale;
     }
@@ -712,6 +713,7 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
   a.sel_tau = sel_tau; a.sel_jcut = sel_jcut; a.sel_count = sel_count;
   a.mask = sel_bitmask ? sel_bitmask : static_cast<uint32_t*>(ws);
   for (int i = 0; i < kMaxRetrieval; ++i) { a.ret_head[i] = sh.ret_head[i]; a.ret_rank[i] = sh.ret_rank[i]; }
+  for (int i = 0; i < 64; ++i) a.inv_freq[i] = sh.inv_freq[i];
 
   static bool s_attr[64] = {};
   int dev = 0;

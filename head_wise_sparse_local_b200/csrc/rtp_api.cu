@@ -5,6 +5,7 @@
 #include <cstring>
 #include <string>
 
+#include <cmath>
 #include "internal.h"
 
 namespace rtp {
@@ -88,6 +89,8 @@ int make_shape(const rtp_layer_cfg* cfg, Shape* sh) {
   }
   sh->R = r;
   sh->NR = r * G;
+  for (int k = 0; k < 64; ++k)
+    sh->inv_freq[k] = k < sh->D / 2 ? std::pow((double)sh->rope_base, -2.0 * k / (double)sh->D) : 0.0;
   return RTP_OK;
 }
 
