@@ -17,7 +17,7 @@ from typing import Optional, Sequence
 import torch
 
 from . import _abi
-from ._abi import (EXPORTS, RTP_BF16, RTP_DEV_POSITION, RTP_DEV_SEQ_LEN, RTP_FP32,
+from ._abi import (EXPORTS, RTP_BF16, RTP_DEV_POSITION, RTP_DEV_SEQ_LEN, RTP_DEV_TIMEOUT, RTP_FP32,
                    RTP_NOALLOC_SCRATCH_BYTES, STAGES, RtpError, rtp_cache, rtp_layer_cfg)
 
 _lib = _abi.load()
@@ -28,7 +28,7 @@ __all__ = ["Layer", "RtpError", "rtp_layer_cfg", "rtp_cache", "rtp_cache_bytes",
            "rtp_last_error", "RTP_NOALLOC_SCRATCH_BYTES",
            "rtp_version", "make_cfg", "STAGES",
            "library_path", "EXPORTS", "RTP_BF16", "RTP_FP32", "RTP_DEV_SEQ_LEN",
-           "RTP_DEV_POSITION"]
+           "RTP_DEV_POSITION", "RTP_DEV_TIMEOUT"]
 
 
 def library_path() -> str:

@@ -16,6 +16,7 @@ RTP_ERR_WORKSPACE = 4
 RTP_ERR_CUDA = 5
 RTP_DEV_SEQ_LEN = 0x1
 RTP_DEV_POSITION = 0x2
+RTP_DEV_TIMEOUT = 0x4
 RTP_BF16 = 0
 RTP_FP32 = 1
 RTP_NOALLOC_SCRATCH_BYTES = 32 << 20

@@ -104,12 +104,19 @@ __device__ __forceinline__ int score_bucket(float s) {
   return (u >> 31) ? 1023 - t : 1024 + t;
 }
 
-// Softmax mass of a score relative to the maximum, in 2^-40 fixed point.
-// exp(s - m) is in (0, 1]; integer sums are exact and order independent, so
-// every kernel that accumulates these weights agrees bit for bit.
-__device__ __forceinline__ unsigned long long mass_fx(float s, float m) {
-  const float w = expf(s - m);
-  return __float2ull_rn(w * 1099511627776.0f);
+// Softmax mass of score s relative to the row maximum m, in 2^-36 fixed point:
+// x = 2^((s - m) log2(e)) * 2^36 from the hardware base-2 exponential, rounded
+// to the nearest integer.  Decode and prefill use this one definition, so their
+// integer sums (exact and order independent), and with them their selections,
+// agree bit for bit.  x rounds to 0 below s - m = -25.65.
+__device__ __forceinline__ float mass_x36(float s, float m) {
+  const float t = (s - m) * 1.4426950408889634f;
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(t));
+  return e * 68719476736.0f;  // 2^36
+}
+__device__ __forceinline__ unsigned long long mass36(float s, float m) {
+  return __float2ull_rn(mass_x36(s, m));
 }
 
 // ---------------------------------------------------------------------------
@@ -180,8 +187,37 @@ __device__ __forceinline__ void block_excl_scan2(unsigned long long a, unsigned 
 __device__ __forceinline__ void rope_cos_sin(int pos, double inv_freq, float& c, float& s) {
   const double th = (double)pos * inv_freq;
   const double two_pi = 6.283185307179586476925286766559;
-  const double r = th - two_pi * rint(th / two_pi);
+  const double r = th - two_pi * rint(th * 0.15915494309189533577);  // any integer multiple works
   sincosf((float)r, &s, &c);
+}
+
+// Loads of data read once per call (the key and value streams): L2
+// evict-first, so they do not push code and reused data out of L2; L1 bypass.
+__device__ __forceinline__ uint64_t l2_evict_first() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+template <typename V>
+__device__ __forceinline__ V ld_stream(const V* ptr, uint64_t pol);
+template <>
+__device__ __forceinline__ uint4 ld_stream<uint4>(const uint4* ptr, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.cg.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(ptr), "l"(pol));
+  return v;
+}
+template <>
+__device__ __forceinline__ uint2 ld_stream<uint2>(const uint2* ptr, uint64_t pol) {
+  uint2 v;
+  asm volatile("ld.global.cg.L2::cache_hint.v2.u32 {%0, %1}, [%2], %3;" : "=r"(v.x), "=r"(v.y) : "l"(ptr), "l"(pol));
+  return v;
+}
+template <>
+__device__ __forceinline__ unsigned ld_stream<unsigned>(const unsigned* ptr, uint64_t pol) {
+  unsigned v;
+  asm volatile("ld.global.cg.L2::cache_hint.u32 %0, [%1], %2;" : "=r"(v) : "l"(ptr), "l"(pol));
+  return v;
 }
 
 // Programmatic dependent launch: a kernel launched with launch_pdl may start

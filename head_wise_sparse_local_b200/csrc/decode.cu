@@ -52,6 +52,8 @@ constexpr int kLgCap = 8192;        // scores a select CTA holds in shared memor
 constexpr int kCandSmem = 4096;     // candidates the leader holds in shared memory
 constexpr int kBruteMax = kSelThreads;  // exact solve by pairwise ranks up to this many candidates
 constexpr int kGroup = 4;           // kept rows a warp attends per memory round trip
+constexpr int kPos = kLgCap / kSelThreads;  // positions a select thread owns per staged chunk
+constexpr int kTopPerWarp = 16;     // top-rung items a warp hands the leader in the first pass
 
 // Tokens per score CTA: eight (bf16) or four (fp32) 16-d keys per thread.
 __host__ __device__ constexpr int score_chunk(int esize) { return kThreads * (esize == 2 ? 8 : 4); }
@@ -75,7 +77,7 @@ struct DecodeArgs {
   float* pm;        // [B][Hkv][n_parts_max][G]: sink/window tiles, then select CTAs
   float* pl;
   float* po;        // [B][Hkv][n_parts_max][G][D]
-  unsigned* ctl;    // [B*Hkv] merge tickets
+  unsigned* ctl;    // [B*Hkv] merge tickets, then [B*Hkv] select partials written
   int* rank_cnt;    // [B][NR][kMaxCS] kept tokens per select CTA
   uint2* cand;      // [B][NR][lstride] boundary-bucket candidates past kCandSmem
   int n_ctl, nch_score_max, n_sw_tiles, n_parts_max, n_score_ctas, n_sw_ctas, sel_cs;
@@ -84,6 +86,21 @@ struct DecodeArgs {
   double inv_freq[64];  // RoPE frequencies, k < D/2
 };
 
+
+// Split cluster barrier (every thread of every CTA of the cluster calls both).
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" :: "l"(p)); }
+
+__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Polls of a bounded wait (about 100 ns each) before it gives up.
+constexpr int kSpinLimit = 1 << 22;
 
 __device__ __forceinline__ bool seq_ok(int L, const DecodeArgs& a) {
   return L >= 1 && L <= a.max_seq_len;
@@ -121,10 +138,12 @@ __device__ __forceinline__ float warp_sum(float v) {
 }
 
 // "Last CTA of the group" ticket: every CTA of the group calls this once.
+// The barrier orders every thread's earlier writes before thread 0's fence,
+// whose release makes them visible before the counter moves.
 __device__ __forceinline__ bool take_ticket(unsigned* counter, unsigned n, int* s_flag) {
-  __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) {
+    __threadfence();
     const unsigned t = atomicAdd(counter, 1u);
     *s_flag = (t == n - 1);
   }
@@ -169,6 +188,7 @@ struct WarpAttn {
   float m[G], l[G], o[G][DL];
   uint4 kraw[KV];
   const T* vb;
+  uint64_t pol;
   int row;
   unsigned msk, live;
 
@@ -192,8 +212,9 @@ struct WarpAttn {
     vb = vb_;
     live = __ballot_sync(0xffffffffu, msk_ != 0u);
     const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)row * D);
+    pol = l2_evict_first();
 #pragma unroll
-    for (int i = 0; i < KV; ++i) kraw[i] = msk ? __ldcg(kr + i) : make_uint4(0u, 0u, 0u, 0u);
+    for (int i = 0; i < KV; ++i) kraw[i] = msk ? ld_stream(kr + i, pol) : make_uint4(0u, 0u, 0u, 0u);
   }
 
   __device__ __forceinline__ void compute(const float* __restrict__ s_q) {
@@ -260,7 +281,7 @@ struct WarpAttn {
       for (int r = 0; r < 16; ++r) {
         const int rr = __shfl_sync(0xffffffffu, row, half * 16 + r);
         if ((live >> (half * 16 + r)) & 1u)
-          vraw[r] = __ldcg(reinterpret_cast<const VRaw*>(vb + (size_t)rr * D + lane * DL));
+          vraw[r] = ld_stream(reinterpret_cast<const VRaw*>(vb + (size_t)rr * D + lane * DL), pol);
         else
           vraw[r] = VRaw();
       }
@@ -324,8 +345,8 @@ __device__ void write_partial(const DecodeArgs& a, WA& wa, size_t part, float* s
 
 // Merge every partial (m, l, o) of KV head (b, h) into the output (one CTA).
 // Stage 1 combines the sink/window partials and runs before the selection has
-// finished; griddep_wait() then waits for the select kernel, and stage 2 adds
-// its n_sel partials (one per select CTA and query head).  Partials with
+// finished; stage 2 waits until the select CTAs of this KV head have counted
+// their partials written and adds those n_sel per query head.  Partials with
 // m = -inf are empty and carry weight 0.
 template <typename T, int D, int G>
 __device__ void merge_partials(const DecodeArgs& a, int b, int h, int n_sel, float* s_buf) {
@@ -364,7 +385,7 @@ __device__ void merge_partials(const DecodeArgs& a, int b, int h, int n_sel, flo
     const int i = tid + u * kThreads;
     if (i < G * D) {
       const int g = i / D, d = i % D;
-#pragma unroll 4
+#pragma unroll 8
       for (int t = 0; t < n_sw; ++t) {
         const float w = s_w[t * G + g];
         const float pv = __ldcg(a.po + ((pbase + t) * G + g) * D + d);  // stale if w == 0
@@ -372,8 +393,22 @@ __device__ void merge_partials(const DecodeArgs& a, int b, int h, int n_sel, flo
       }
     }
   }
-  griddep_wait();  // the select kernel's partials are complete
   if (n_sel > 0) {
+    // Wait until every select CTA of this KV head has written its partial
+    // (they are all running: this grid launched only after each of them
+    // started, and they wait for nothing of this grid).
+    if (tid == 0) {
+      const unsigned need = (unsigned)(G * n_sel);
+      const unsigned* done = a.ctl + (size_t)a.B * a.Hkv + (size_t)b * a.Hkv + h;
+      int spins = 0;
+      while (ld_acquire(done) < need) {
+        if (++spins > kSpinLimit) {
+          atomicOr(a.status, RTP_DEV_TIMEOUT);
+          break;
+        }
+        __nanosleep(100);
+      }
+    }
     const size_t sbase = pbase + n_sw;
     __syncthreads();
     for (int i = tid; i < n_sel * G; i += kThreads) {
@@ -402,13 +437,14 @@ __device__ void merge_partials(const DecodeArgs& a, int b, int h, int n_sel, flo
       const int i = tid + u * kThreads;
       if (i < G * D) {
         const int g = i / D, d = i % D;
+        float pv[kMaxCS];  // every load in flight at once (empty partials are skipped)
+#pragma unroll
+        for (int t = 0; t < kMaxCS; ++t)
+          pv[t] = (t < n_sel && s_w[t * G + g] > 0.f) ? __ldcg(a.po + ((sbase + t) * G + g) * D + d) : 0.f;
         float v = acc[u] * s_st[g * 3 + 2];
-#pragma unroll 4
-        for (int t = 0; t < n_sel; ++t) {
-          const float w = s_w[t * G + g];
-          const float pv = __ldcg(a.po + ((sbase + t) * G + g) * D + d);  // stale if w == 0
-          v = w > 0.f ? fmaf(pv, w, v) : v;
-        }
+#pragma unroll
+        for (int t = 0; t < kMaxCS; ++t)
+          if (t < n_sel) v = fmaf(pv[t], s_w[t * G + g], v);
         acc[u] = v;
       }
     }
@@ -422,6 +458,7 @@ __device__ void merge_partials(const DecodeArgs& a, int b, int h, int n_sel, flo
       *out = from_f32<T>(acc[u] / s_st[g * 3 + 1]);
     }
   }
+  griddep_wait();  // this grid completes only after the select kernel has
 }
 
 // ---------------------------------------------------------------------------
@@ -474,12 +511,13 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(DecodeArgs a) {
   const int jh = min(a.max_seq_len, j0 + kChunk);
   const uint4* kidx = reinterpret_cast<const uint4*>(static_cast<const T*>(a.kidx) +
                                                      ((size_t)b * a.R + r) * a.Lmax * kIdxDim);
+  const uint64_t pol = l2_evict_first();
   uint4 kr[TPT][NV];
 #pragma unroll
   for (int t = 0; t < TPT; ++t) {
     const int j = j0 + t * kThreads + tid;
 #pragma unroll
-    for (int v = 0; v < NV; ++v) kr[t][v] = (j < jh) ? __ldcg(kidx + (size_t)j * NV + v) : make_uint4(0u, 0u, 0u, 0u);
+    for (int v = 0; v < NV; ++v) kr[t][v] = (j < jh) ? ld_stream(kidx + (size_t)j * NV + v, pol) : make_uint4(0u, 0u, 0u, 0u);
   }
   __syncthreads();  // q~ visible
   if (!seq_ok(L, a)) {
@@ -605,20 +643,15 @@ __global__ void __launch_bounds__(kThreads, 2) sw_kernel(DecodeArgs a) {
 // ---------------------------------------------------------------------------
 // selection helpers
 // ---------------------------------------------------------------------------
-// Softmax mass exp(s - max) in 2^-36 fixed point.  Integer sums of these are
-// exact and order independent, so the histogram and the exact solve agree bit
-// for bit.  The selection accumulates it per bucket as two 18-bit halves with
-// 32-bit shared atomics (native and robust to contention); a score whose mass
-// rounds to zero adds nothing and is skipped.
-__device__ __forceinline__ unsigned long long mass_fx36(float s, float m) {
-  return __float2ull_rn(expf(s - m) * 68719476736.0f);  // 2^36
-}
-// The same integer as two 32-bit halves, hi * 2^18 + lo, computed in fp32
-// without a 64-bit conversion: x = e^(s-m) 2^36 is exact (power-of-two
-// scale); hi = floor(x / 2^18) and x - hi 2^18 are exact; rounding the
-// remainder gives rint(x) - hi 2^18 because hi 2^18 is an even integer.
+// Softmax mass exp(s - max) in 2^-36 fixed point (mass36): integer sums are
+// exact and order independent, so the first pass, the histogram and the exact
+// solve agree bit for bit.  The histogram accumulates it per bucket as two
+// 18-bit halves with 32-bit shared atomics (native and robust to contention):
+// with x = mass_x36(s, m), hi = floor(x / 2^18) and x - hi 2^18 are exact in
+// fp32, and rounding the remainder gives rint(x) - hi 2^18 because hi 2^18 is
+// an even integer.
 __device__ __forceinline__ void mass_split36(float s, float m, unsigned& hi, unsigned& lo) {
-  const float x = expf(s - m) * 68719476736.0f;
+  const float x = mass_x36(s, m);
   const float hf = floorf(x * 3.814697265625e-06f);  // 2^-18
   hi = (unsigned)hf;
   lo = __float2uint_rn(fmaf(hf, -262144.0f, x));
@@ -660,7 +693,7 @@ __device__ DigitResult radix_step(const Items& it, int n, uint32_t prefix, uint3
     if constexpr (kMass) {
       if ((e.x & mask) == prefix) {
         const int dg = (e.x >> shift) & 255;
-        atomicAdd(&h_m[dg], mass_fx36(key_score(e.x), m));
+        atomicAdd(&h_m[dg], mass36(key_score(e.x), m));
         atomicAdd(&h_c[dg], 1u);
       }
     } else {
@@ -761,7 +794,7 @@ __device__ void solve_radix(const Items& it, int n, float m, unsigned long long 
     cnt_eq = n_items;  // every item has the same key
   }
   const uint32_t tau_key = prefix;
-  const unsigned long long w_tau = mass_fx36(key_score(tau_key), m);
+  const unsigned long long w_tau = mass36(key_score(tau_key), m);
   unsigned long long kk = (w_tau > 0ull) ? (need + w_tau - 1ull) / w_tau : (unsigned long long)cnt_eq;
   if (kk < 1ull) kk = 1ull;
   if (kk > cnt_eq) kk = cnt_eq;
@@ -790,16 +823,18 @@ __device__ void solve_brute(const uint2* items, int n, float m, unsigned long lo
   uint2 me = make_uint2(0u, 0u);
   if (tid < n) {
     me = items[tid];
-    s_w[tid] = mass_fx36(key_score(me.x), m);
+    s_w[tid] = mass36(key_score(me.x), m);
   }
   if (tid == 0) { *s_min = 0xffffffffu; *s_jmax = -1; }
   __syncthreads();
   bool kept = false;
   if (tid < n) {
     unsigned long long before = 0ull;
+#pragma unroll 4
     for (int j = 0; j < n; ++j) {
       const uint2 o = items[j];
-      if (o.x > me.x || (o.x == me.x && o.y < me.y)) before += s_w[j];
+      const unsigned long long ow = s_w[j];
+      if (o.x > me.x || (o.x == me.x && o.y < me.y)) before += ow;
     }
     kept = before < need;
     if (kept) atomicMin(s_min, me.x);
@@ -815,28 +850,55 @@ __device__ void solve_brute(const uint2* items, int n, float m, unsigned long lo
 // Rungs m - rung_delta(k) at which the selection sums mass and count in its first
 // pass: when the scores at or above one rung hold the target mass and number
 // at most kCandSmem, the leader solves over exactly those (no histogram).
-constexpr int kRungs = 6;
-__host__ __device__ constexpr float rung_delta(int k) { return k == 0 ? 0.5f : (float)(1 << (k - 1)); }  // 0.5 .. 16
+constexpr int kRungs = 4;
+__host__ __device__ constexpr float rung_delta(int k) { return (float)(1 << k); }  // 1, 2, 4, 8
 
 template <int CS>
 struct SelShared {
   unsigned long long pre_m[CS][1 + kRungs];  // per rank: Z, then the mass at or above each rung
-  unsigned pre_c[CS][kRungs];                // per rank: count at or above each rung
+  unsigned pre_c[CS][kRungs + 1];            // per rank: count at or above each rung, overflowed warps
+  unsigned wcnt[CS * kSelWarps];             // leader: top-rung items per (rank, warp) region
   unsigned long long wpre_m[kSelWarps][1 + kRungs];
-  unsigned wpre_c[kSelWarps][kRungs];
+  unsigned wpre_c[kSelWarps][kRungs + 1];
   unsigned long long tot_m[1 + kRungs];      // cluster totals
-  unsigned tot_c[kRungs];
+  unsigned tot_c[kRungs + 1];
   unsigned long long slice[CS];   // per-rank slice totals of the histogram
   unsigned long long zpart[CS];   // [0]: mass above the boundary bucket (broadcast)
   int bucket;                     // boundary bucket (broadcast)
   float tau;                      // final threshold (broadcast)
   int jcut;
-  unsigned n_cand;                // leader: candidates reserved
+  unsigned n_cand2;               // leader: items / candidates reserved after the first pass
   float red[kSelWarps];
   unsigned long long scan_a[kSelWarps];
   unsigned scan_c[kSelWarps];
   int cnt[kSelWarps];
 };
+
+// Exact tau / j_cut for n <= 32 items by one warp (lane i owns item i): an item
+// is kept iff the mass of the items ordered before it is below `need`.
+__device__ void solve_warp(const uint2* items, int n, float m, unsigned long long need, float& tau,
+                           int& jcut) {
+  const int lane = threadIdx.x & 31;
+  const uint2 me = lane < n ? items[lane] : make_uint2(0u, 0u);
+  const unsigned long long w = lane < n ? mass36(key_score(me.x), m) : 0ull;
+  unsigned long long before = 0ull;
+#pragma unroll 1
+  for (int j = 0; j < n; ++j) {
+    const unsigned ox = __shfl_sync(0xffffffffu, me.x, j);
+    const unsigned oy = __shfl_sync(0xffffffffu, me.y, j);
+    const unsigned long long ow = __shfl_sync(0xffffffffu, w, j);
+    if (ox > me.x || (ox == me.x && oy < me.y)) before += ow;
+  }
+  const bool kept = lane < n && before < need;
+  unsigned tk = kept ? me.x : 0xffffffffu;  // the smallest kept key ...
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tk = min(tk, __shfl_xor_sync(0xffffffffu, tk, o));
+  int jm = (kept && me.x == tk) ? (int)me.y : -1;  // ... and its largest kept index
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) jm = max(jm, __shfl_xor_sync(0xffffffffu, jm, o));
+  tau = key_score(tk);
+  jcut = jm;
+}
 
 template <int CS>
 struct SelCfg {
@@ -896,9 +958,12 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   __shared__ uint32_t s_kr[96];
   __shared__ uint32_t s_min;
   __shared__ int s_jmax;
+  __shared__ uint2 s_small[32];
   __shared__ __align__(16) float s_qh[D];
   __shared__ __align__(16) float s_wo[kSelWarps * D];
   __shared__ float s_wml[kSelWarps * 2];
+  const T* kb = static_cast<const T*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+  const T* vb = static_cast<const T*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
 
   // This CTA's share of the context comes from the call's maximum length, so
   // the score loads below do not wait for seq_len.
@@ -932,12 +997,15 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
     s_qh[tid] = (qx1 * c - qx2 * s) * qscale;
     s_qh[tid + D / 2] = (qx2 * c + qx1 * s) * qscale;
   }
+  if (rank == 0 && tid == 0) sh->n_cand2 = 0u;
+  cluster_arrive();  // counter zeroed; every CTA of the cluster running
   griddep_wait();
   griddep_launch();
   const int nch_h = (Lh + kChunk - 1) / kChunk;
   const float* cm = a.cmax + (size_t)bh * a.nch_score_max;
   const float cm0 = tid < nch_h ? __ldcg(cm + tid) : -CUDART_INF_F;
   if (cached) stage(j0, jh);
+  cluster_wait();
   if (!seq_ok(L, a)) return;  // uniform over the cluster; the score kernel flagged it
   const int j1 = min(L, jh);  // j1 <= j0: nothing of this sequence in this CTA's share
   uint32_t* mask = a.mask + (size_t)bh * a.words;
@@ -954,17 +1022,22 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
       for (int c = tid + kSelThreads; c < nch; c += kSelThreads) v = fmaxf(v, __ldcg(cm + c));
       m = block_max<kSelThreads>(v, sh->red);
     }
-    if (rank == 0 && tid == 0) sh->n_cand = 0u;
     const float m_lo = m - 26.0f;  // exp(s - m) 2^36 rounds to 0 below m - 25.65
+    SelShared<CS>* lead = cl.map_shared_rank(sh, 0);
+    uint2* lead_cand = cl.map_shared_rank(s_cand, 0);
 
     // ---- pass 1: the exact total mass Z and, for each rung of the ladder
     // m - rung_delta(k), the mass and the count of the scores at or above it ----
     {
+      // Z: masses of scores below the lowest rung m - 8 (below 2^25; nearly
+      // every score) are summed in 32 bits (at most kLgCap / kSelThreads = 16
+      // per thread per chunk, so below 2^29), the rest in 64 bits.
       unsigned long long zs = 0ull, ms[kRungs];
-      unsigned cs[kRungs];
+      unsigned zs32 = 0u, cs[kRungs];
 #pragma unroll
       for (int k = 0; k < kRungs; ++k) { ms[k] = 0ull; cs[k] = 0u; }
       const float top_lo = m - rung_delta(kRungs - 1);
+      unsigned wtop = 0u;  // warp-uniform: this warp's top-rung items so far
       for (int c0 = j0; c0 < j1; c0 += kLgCap) {
         const int c1 = min(j1, c0 + kLgCap);
         if (!cached) {
@@ -972,28 +1045,67 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
           stage(c0, c1);
         }
         __syncthreads();
+        // this thread's positions c0 + u * kSelThreads + tid, u < kPos: sums,
+        // and a bit per position at or above the top rung
+        unsigned topbits = 0u;
 #pragma unroll 4
-        for (int j = c0 + tid; j < c1; j += kSelThreads) {
-          const float sv = s_lg[j - c0];
+        for (int u = 0; u < kPos; ++u) {
+          const int j = c0 + u * kSelThreads + tid;
+          const float sv = j < c1 ? s_lg[j - c0] : -CUDART_INF_F;
           if (sv > m_lo) {
-            const unsigned long long w = mass_fx36(sv, m);
-            zs += w;
-            if (sv >= top_lo) {
+            const float x = mass_x36(sv, m);
+            if (sv < top_lo) {  // x < 2^36 e^-8 < 2^25
+              zs32 += __float2uint_rn(x);
+            } else {
+              const unsigned long long w = __float2ull_rn(x);
+              zs += w;
 #pragma unroll
               for (int k = 0; k < kRungs; ++k)
                 if (sv >= m - rung_delta(k)) { ms[k] += w; ++cs[k]; }
+              topbits |= 1u << u;
             }
           }
         }
-      }
-      // this rank's sums -> every rank of the cluster
-      zs = warp_sum_u64(zs);
+        zs += zs32;
+        zs32 = 0u;
+        // Scores at or above the top rung go to this warp's region of the
+        // leader's item space (kTopPerWarp slots, no atomics); their key and
+        // value rows are pulled into L2 meanwhile (the kept rows are among them
+        // whenever the leader solves over these items).
+        if (__any_sync(0xffffffffu, topbits != 0u)) {
+          uint2* region = lead_cand + (rank * kSelWarps + warp) * kTopPerWarp;
+          for (int u = 0; u < kPos; ++u) {
+            const bool top = (topbits >> u) & 1u;
+            const unsigned bal = __ballot_sync(0xffffffffu, top);
+            if (!bal) continue;
+            const unsigned slot = wtop + __popc(bal & ((1u << lane) - 1u));
+            if (top) {
+              const int j = c0 + u * kSelThreads + tid;
+              if (slot < (unsigned)kTopPerWarp) region[slot] = make_uint2(score_key(s_lg[j - c0]), (unsigned)j);
 #pragma unroll
-      for (int k = 0; k < kRungs; ++k) { ms[k] = warp_sum_u64(ms[k]); cs[k] = warp_sum_u32(cs[k]); }
+              for (int o = 0; o < D * (int)sizeof(T); o += 128) {
+                prefetch_l2(reinterpret_cast<const char*>(kb + (size_t)j * D) + o);
+                prefetch_l2(reinterpret_cast<const char*>(vb + (size_t)j * D) + o);
+              }
+            }
+            wtop += __popc(bal);
+          }
+        }
+      }
+      // this rank's sums -> every rank of the cluster (the rung sums are zero
+      // in most warps: reduce them only where some lane has one)
+      zs = warp_sum_u64(zs);
+      const bool any_top = __any_sync(0xffffffffu, cs[kRungs - 1] != 0u);
+      if (any_top) {
+#pragma unroll
+        for (int k = 0; k < kRungs; ++k) { ms[k] = warp_sum_u64(ms[k]); cs[k] = warp_sum_u32(cs[k]); }
+      }
       if (lane == 0) {
         sh->wpre_m[warp][0] = zs;
 #pragma unroll
         for (int k = 0; k < kRungs; ++k) { sh->wpre_m[warp][1 + k] = ms[k]; sh->wpre_c[warp][k] = cs[k]; }
+        sh->wpre_c[warp][kRungs] = wtop > (unsigned)kTopPerWarp ? 1u : 0u;
+        lead->wcnt[rank * kSelWarps + warp] = wtop;
       }
       __syncthreads();
       if (tid < 1 + kRungs) {
@@ -1002,7 +1114,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         for (int w = 0; w < kSelWarps; ++w) t += sh->wpre_m[w][tid];
 #pragma unroll
         for (int q = 0; q < CS; ++q) cl.map_shared_rank(sh, q)->pre_m[rank][tid] = t;
-      } else if (tid >= 32 && tid < 32 + kRungs) {
+      } else if (tid >= 32 && tid < 32 + kRungs + 1) {
         unsigned t = 0u;
 #pragma unroll
         for (int w = 0; w < kSelWarps; ++w) t += sh->wpre_c[w][tid - 32];
@@ -1017,7 +1129,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
 #pragma unroll
       for (int q = 0; q < CS; ++q) t += sh->pre_m[q][tid];
       sh->tot_m[tid] = t;
-    } else if (tid >= 32 && tid < 32 + kRungs) {
+    } else if (tid >= 32 && tid < 32 + kRungs + 1) {
       unsigned t = 0u;
 #pragma unroll
       for (int q = 0; q < CS; ++q) t += sh->pre_c[q][tid - 32];
@@ -1038,53 +1150,117 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
 #pragma unroll
     for (int k = kRungs - 1; k >= 0; --k)
       if (Mk[k] >= target) kf = k;
-    const bool fast = kf >= 0 && Ck[kf] <= (unsigned)kCandSmem;
+    // tier 1: the first pass already put every score at or above the top rung
+    // with the leader, and they hold the target; tier 2: a lower rung's
+    // scores hold it and fit (one more pass collects them); else the histogram
+    const bool tier1 = Mk[kRungs - 1] >= target && sh->tot_c[kRungs] == 0u;  // no region overflowed
+    const bool tier2 = !tier1 && kf >= 0 && Ck[kf] <= (unsigned)kCandSmem;
     float t_lo = m_lo;
 #pragma unroll
     for (int k = 0; k < kRungs; ++k)
       if (k == kf) t_lo = m - rung_delta(k);
 
     uint2* gcand = a.cand + (size_t)bh * a.lstride;
-    SelShared<CS>* lead = cl.map_shared_rank(sh, 0);
-    uint2* lead_cand = cl.map_shared_rank(s_cand, 0);
-    if (fast) {
-      // ---- every score at or above the rung -> the leader; it solves exactly ----
-      for (int c0 = j0; c0 < j1; c0 += kLgCap) {
-        const int c1 = min(j1, c0 + kLgCap);
-        if (!cached) {
-          __syncthreads();
-          stage(c0, c1);
-          __syncthreads();
-        }
-#pragma unroll 4
-        for (int jb = c0; jb < c1; jb += kSelThreads) {
-          const int j = jb + tid;
-          float sv = 0.f;
-          bool in = false;
-          if (j < c1) {
-            sv = s_lg[j - c0];
-            in = sv >= t_lo;
+    if (tier1 || tier2) {
+      if (tier2) {  // every score at or above rung kf -> the leader
+        for (int c0 = j0; c0 < j1; c0 += kLgCap) {
+          const int c1 = min(j1, c0 + kLgCap);
+          if (!cached) {
+            __syncthreads();
+            stage(c0, c1);
+            __syncthreads();
           }
-          const unsigned bal = __ballot_sync(0xffffffffu, in);
-          if (bal) {
-            unsigned base = 0u;
-            if (lane == 0) base = atomicAdd(&lead->n_cand, (unsigned)__popc(bal));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (in) lead_cand[base + __popc(bal & ((1u << lane) - 1u))] = make_uint2(score_key(sv), (unsigned)j);
+          unsigned inbits = 0u;
+#pragma unroll
+          for (int u = 0; u < kPos; ++u) {
+            const int j = c0 + u * kSelThreads + tid;
+            if (j < c1 && s_lg[j - c0] >= t_lo) inbits |= 1u << u;
+          }
+          if (__any_sync(0xffffffffu, inbits != 0u)) {
+            for (int u = 0; u < kPos; ++u) {
+              const bool in = (inbits >> u) & 1u;
+              const unsigned bal = __ballot_sync(0xffffffffu, in);
+              if (!bal) continue;
+              unsigned base = 0u;
+              if (lane == 0) base = atomicAdd(&lead->n_cand2, (unsigned)__popc(bal));
+              base = __shfl_sync(0xffffffffu, base, 0);
+              if (in) {
+                const int j = c0 + u * kSelThreads + tid;
+                lead_cand[base + __popc(bal & ((1u << lane) - 1u))] = make_uint2(score_key(s_lg[j - c0]), (unsigned)j);
+              }
+            }
           }
         }
+        cl.sync();  // (B) the leader holds every item
       }
-      cl.sync();  // (B) the leader holds every item
       if (rank == 0) {
-        const int n = (int)sh->n_cand;  // == Ck[kf] <= kCandSmem
-        float t_tau;
-        int t_jcut;
-        if (n <= kBruteMax)
+        int n = (int)Ck[kf];
+        bool done = false;
+        float t_tau = 0.f;
+        int t_jcut = 0;
+        if (tier1 && Ck[kRungs - 1] <= 32u) {
+          // few items: warp 0 gathers the regions' items at or above rung kf and solves
+          if (warp == 0) {
+            const uint32_t klo = score_key(t_lo);
+            if (lane == 0) s_min = 0u;
+            __syncwarp();
+#pragma unroll 1
+            for (int rg = lane; rg < CS * kSelWarps; rg += 32) {
+              const int cnt_r = (int)sh->wcnt[rg];
+#pragma unroll 1
+              for (int i = 0; i < cnt_r; ++i) {
+                const uint2 e = s_cand[rg * kTopPerWarp + i];
+                if (e.x >= klo) s_small[atomicAdd(&s_min, 1u)] = e;
+              }
+            }
+            __syncwarp();
+            n = (int)s_min;
+            solve_warp(s_small, n, m, target, t_tau, t_jcut);
+          }
+          done = true;
+        } else if (tier1) {
+          // gather the regions' items (only those at or above rung kf can be
+          // kept) into one list; read everything before writing
+          constexpr int kRegions = kMaxCS * kSelWarps;
+          constexpr int kRPT = (kRegions + kSelThreads - 1) / kSelThreads;
+          static_assert(kRegions * kTopPerWarp <= kCandSmem, "regions fit in the item space");
+          const uint32_t klo = score_key(t_lo);
+          uint2 it[kRPT][kTopPerWarp];
+          unsigned c = 0u;
+#pragma unroll
+          for (int rr = 0; rr < kRPT; ++rr) {
+            const int rg = tid + rr * kSelThreads;
+            const int cnt_r = rg < CS * kSelWarps ? (int)sh->wcnt[rg] : 0;
+#pragma unroll
+            for (int i = 0; i < kTopPerWarp; ++i) {
+              it[rr][i] = make_uint2(0u, 0u);
+              if (i < cnt_r) {
+                it[rr][i] = s_cand[rg * kTopPerWarp + i];
+                if (it[rr][i].x >= klo) ++c;
+              }
+            }
+          }
+          unsigned long long ex_m, tot_m;
+          unsigned off, tot;
+          block_excl_scan2<kSelThreads>(0ull, c, ex_m, off, tot_m, tot, sh->scan_a, sh->scan_c);
+#pragma unroll
+          for (int rr = 0; rr < kRPT; ++rr)
+#pragma unroll
+            for (int i = 0; i < kTopPerWarp; ++i)
+              if (it[rr][i].x >= klo && it[rr][i].x != 0u) s_cand[off++] = it[rr][i];
+          __syncthreads();
+          n = (int)tot;
+        }
+        if (done) {
+        } else if (n <= 32) {
+          if (warp == 0) solve_warp(s_cand, n, m, target, t_tau, t_jcut);
+        } else if (n <= kBruteMax) {
           solve_brute(s_cand, n, m, target, s_w, &s_min, &s_jmax, t_tau, t_jcut);
-        else
+        } else {
           solve_radix(Items{s_cand, false}, n, m, target, r_hm, r_hc, &s_dres, s_kr, t_tau, t_jcut);
-        if (tid < CS) {
-          SelShared<CS>* rem = cl.map_shared_rank(sh, tid);
+        }
+        if (warp == 0 && lane < CS) {
+          SelShared<CS>* rem = cl.map_shared_rank(sh, lane);
           rem->tau = t_tau;
           rem->jcut = t_jcut;
         }
@@ -1218,7 +1394,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
               sv[u] = 0.f;
               if (j < c1) {
                 sv[u] = s_lg[j - c0];
-                in[u] = sv[u] > m_lo && score_bucket(sv[u]) == bucket && mass_fx36(sv[u], m) != 0ull;
+                in[u] = sv[u] > m_lo && score_bucket(sv[u]) == bucket && mass36(sv[u], m) != 0ull;
               }
             }
 #pragma unroll
@@ -1226,7 +1402,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
               const unsigned bal = __ballot_sync(0xffffffffu, in[u]);
               if (bal) {
                 unsigned base = 0u;
-                if (lane == 0) base = atomicAdd(&lead->n_cand, (unsigned)__popc(bal));
+                if (lane == 0) base = atomicAdd(&lead->n_cand2, (unsigned)__popc(bal));
                 base = __shfl_sync(0xffffffffu, base, 0);
                 const unsigned slot = base + __popc(bal & ((1u << lane) - 1u));
                 if (in[u]) {
@@ -1250,7 +1426,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         float t_tau = -CUDART_INF_F;  // no boundary (unreachable): keep every token
         int t_jcut = INT_MAX;
         if (bucket >= 0) {
-          const int n = (int)sh->n_cand;
+          const int n = (int)sh->n_cand2;
           const unsigned long long need = target - above;
           Items items{s_cand, false};
           if (n > kCandSmem) {  // the list continues in global scratch: put its head there too
@@ -1281,9 +1457,8 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   // them kGroup at a time (keys and values of a group in one round trip) ----
   const int s_cnt = min(a.S, L);
   const int sw0 = max(s_cnt, L - a.W);
-  const T* kb = static_cast<const T*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
-  const T* vb = static_cast<const T*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
   int* wrows = s_rows + warp * (kLgCap / kSelWarps);
+  const uint64_t pol = l2_evict_first();
   __syncthreads();  // s_qh visible
   float qv[DL];
 #pragma unroll
@@ -1299,22 +1474,27 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
       stage(c0, c1);
     }
     __syncthreads();  // staged scores visible; the row lists' bytes are free
-    int wn = 0;
+    unsigned inbits = 0u, outbits = 0u;
 #pragma unroll 4
-    for (int jb = c0; jb < c1; jb += kSelThreads) {
-      const int j = jb + tid;
-      bool in = false;
+    for (int u = 0; u < kPos; ++u) {
+      const int j = c0 + u * kSelThreads + tid;
       if (j < c1) {
         const float sv = s_lg[j - c0];
-        in = keep_all || sv > tau || (sv == tau && j <= jcut);
+        if (keep_all || sv > tau || (sv == tau && j <= jcut)) {
+          inbits |= 1u << u;
+          if (j >= s_cnt && j < sw0) outbits |= 1u << u;
+        }
       }
-      const unsigned word = __ballot_sync(0xffffffffu, in);
-      const int jw = jb + warp * 32;
+    }
+    cnt += __popc(inbits);
+    int wn = 0;
+#pragma unroll 2
+    for (int u = 0; u < kPos; ++u) {
+      const unsigned word = __ballot_sync(0xffffffffu, (inbits >> u) & 1u);
+      const int jw = c0 + u * kSelThreads + warp * 32;
       if (lane == 0 && jw < c1) mask[jw >> 5] = word;
-      cnt += in ? 1 : 0;
-      const bool o = in && j >= s_cnt && j < sw0;
-      const unsigned ob = __ballot_sync(0xffffffffu, o);
-      if (o) wrows[wn + __popc(ob & ((1u << lane) - 1u))] = j;
+      const unsigned ob = __ballot_sync(0xffffffffu, (outbits >> u) & 1u);
+      if ((outbits >> u) & 1u) wrows[wn + __popc(ob & ((1u << lane) - 1u))] = jw + lane;
       wn += __popc(ob);
     }
     __syncwarp();
@@ -1327,8 +1507,8 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         vr[k] = Raw();
         rw[k] = (i0 + k < wn) ? wrows[i0 + k] : -1;
         if (rw[k] >= 0) {
-          kr[k] = __ldcg(reinterpret_cast<const Raw*>(kb + (size_t)rw[k] * D + lane * DL));
-          vr[k] = __ldcg(reinterpret_cast<const Raw*>(vb + (size_t)rw[k] * D + lane * DL));
+          kr[k] = ld_stream(reinterpret_cast<const Raw*>(kb + (size_t)rw[k] * D + lane * DL), pol);
+          vr[k] = ld_stream(reinterpret_cast<const Raw*>(vb + (size_t)rw[k] * D + lane * DL), pol);
         }
       }
       float sc[kGroup];
@@ -1402,6 +1582,12 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
 #pragma unroll
     for (int w = 0; w < kSelWarps; ++w) c += sh->cnt[w];
     a.rank_cnt[(size_t)bh * kMaxCS + rank] = c;
+  }
+  // this CTA's partial and count are written: count them for the merge
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(a.ctl + (size_t)a.B * a.Hkv + (size_t)b * a.Hkv + h, 1u);
   }
 }
 
@@ -1488,7 +1674,7 @@ DecodeLayout decode_layout(const Shape& sh) {
   l.nch_score_max = (sh.Lmax + chunk - 1) / chunk;
   l.n_sw_tiles = (sh.S + sh.W + kSwTile - 1) / kSwTile;
   l.n_tiles_max = l.n_sw_tiles + (sh.R > 0 ? kMaxCS : 0);
-  l.n_ctl = (int)((size_t)sh.B * sh.Hkv);
+  l.n_ctl = (int)(2 * (size_t)sh.B * sh.Hkv);  // merge tickets, select-partial counters
   const size_t words = (size_t)(sh.Lmax + 31) / 32;
   const size_t lstride = ((size_t)sh.Lmax + 31) & ~size_t(31);
   size_t off = 0;

@@ -8,7 +8,8 @@
 //       so a row's selection equals the decode selection at that position.
 //       The exact top-p threshold is found by splitting the score interval
 //       that contains the boundary 8 ways per pass, with the softmax mass
-//       exp(s - max) of every score in 2^-36 fixed point (exact integer sums
+//       exp(s - max) of every score in 2^-36 fixed point (mass36, shared with
+//       the decode path; exact integer sums
 //       in registers), until at most kCand tokens remain; a warp-level exact
 //       solve finishes (ties to the lower index).  The row's top-p set is
 //       written as a bitmask.
@@ -50,9 +51,6 @@ struct PrefillArgs {
   double inv_freq[64];  // RoPE frequencies, k < D/2
 };
 
-__device__ __forceinline__ unsigned long long mass36(float s, float m) {
-  return __float2ull_rn(expf(s - m) * 68719476736.0f);  // 2^36
-}
 __device__ __forceinline__ unsigned long long wsum64(unsigned long long v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
