@@ -44,6 +44,9 @@ import torch  # noqa: E402
 
 METRIC = "sparse-attn layer decode µs/token & HBM GB/s at 128K–1M; prefill ms @32K"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_MD = os.path.join(ROOT, "profiles", "decode_128k_bf16_dram_bytes.md")
+STAGE_KERNEL = {"append": "append_kernel", "decode_score": "score_kernel", "decode_select": "select_kernel",
+                "decode_local": "sw_kernel"}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -184,6 +187,28 @@ def kept_rows_outside_sw(shape, seq_len, bitmask: torch.Tensor) -> int:
             bits = np.unpackbits(words.view(np.uint8), bitorder="little")[:L]
             tot += int(bits[s_cnt:sw0].sum())
     return tot
+
+
+def measured_traffic(stage: str, workload: str):
+    """DRAM bytes (read + write) per launch of `stage`'s kernel from the committed
+    ncu summary, or None when there is none for this workload or the kernel
+    sources changed since it was captured."""
+    import hashlib
+    import re
+    if workload != "decode_128k_bf16" or not os.path.exists(TRAFFIC_MD):
+        return None
+    text = open(TRAFFIC_MD).read()
+    m = re.search(r"source-sha256-16: (.*)", text)
+    if not m:
+        return None
+    csrc = os.path.join(ROOT, "head_wise_sparse_local_b200", "csrc")
+    for item in m.group(1).split():
+        fname, digest = item.split("=")
+        path = os.path.join(csrc, fname)
+        if not os.path.exists(path) or hashlib.sha256(open(path, "rb").read()).hexdigest()[:16] != digest:
+            return None
+    row = re.search(r"^\| %s \| (\d+) \| (\d+) \|" % STAGE_KERNEL[stage], text, re.M)
+    return int(row.group(1)) + int(row.group(2)) if row else None
 
 
 def l2_bytes() -> int:
@@ -388,12 +413,178 @@ def run_ours(args, dist: Dist) -> dict:
         kept_out=kept_out, counts=cnt.cpu().numpy(), kern_us=kern_us, dominant=dominant,
         roofline={"bound": "hbm", "kernel": dominant, "achieved": round(ach, 1), "peak": peak,
                   "peak_source": peak_src, "unit": "GB/s", "frac": round(ach / peak, 4),
-                  "bytes_per_launch": kbytes[dominant], "traffic": None},
+                  "bytes_per_launch": kbytes[dominant],
+                  "traffic": measured_traffic(dominant, args.workload)},
         e2e={"value": e2e_s * 1e6 / (n_e * B * dist.world), "unit": "µs/token",
              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e},
         clocks=(clocks.summary(t_wall0, t_wall1) if clocks else None),
         gpu_launches=K * (4 if R else 2), l2=l2, inp=inp, Lh=Lh,
     )
+
+
+# ---------------------------------------------------------------------------
+# extra lines of the metric: 1M-token decode and the 32K prefill chunk
+# ---------------------------------------------------------------------------
+def decode_extra(name: str, dev, steps: int) -> dict:
+    """µs/token of (append + decode) on workload `name`: CUDA-graph replays over
+    replica caches whose bytes per step sum to more than twice the L2."""
+    import head_wise_sparse_local_b200 as rtp
+    from synth import make_decode_inputs, workload
+    inp = make_decode_inputs(workload(name))
+    sh = inp["shape"]
+    B, Hq, D = sh.batch, sh.n_q_heads, sh.head_dim
+    Lmax, seq_len = inp["max_ctx"], inp["seq_len"]
+    Lh = int(seq_len.max())
+    dt = sh.torch_dtype
+    w_q, w_k = inp["w_q"].to(dev), inp["w_k"].to(dev)
+    seq = torch.from_numpy(seq_len).to(dev)
+    last = (seq - 1).to(torch.int32)
+    bidx, lastc = torch.arange(B), torch.from_numpy(seq_len.astype(np.int64) - 1)
+    k_new = inp["k_pre"][bidx, lastc][:, None].contiguous().to(dev)
+    v_new = inp["v"][bidx, lastc][:, None].contiguous().to(dev)
+    q = inp["q_pre"].to(dev)
+    lay0 = rtp.Layer(sh, Lmax, device=dev)
+    lay0.append(inp["k_pre"].to(dev), inp["v"].to(dev), torch.zeros(B, dtype=torch.int32, device=dev), w_k)
+    NR = max(sh.n_retrieval * sh.group, 1)
+    bm = torch.zeros((B, NR, (Lmax + 31) // 32), dtype=torch.int32, device=dev)
+    cnt = torch.zeros((B, NR), dtype=torch.int32, device=dev)
+    out = torch.empty((B, Hq, D), dtype=dt, device=dev)
+    lay0.append(k_new, v_new, last, w_k)
+    lay0.decode(q, seq, w_q, out, max_seq_len=Lh, sel_bitmask=bm, sel_count=cnt)
+    torch.cuda.synchronize()
+    nbytes = algorithmic_bytes(sh, seq_len, kept_rows_outside_sw(sh, seq_len, bm) if sh.n_retrieval else 0)
+    n_rep = max(3, math.ceil(2.0 * l2_bytes() / nbytes["total"]) + 1)
+    per_rep = lay0.k.numel() * lay0.k.element_size() * 2 + lay0.kidx.numel() * lay0.kidx.element_size()
+    n_rep = int(max(1, min(n_rep, (torch.cuda.mem_get_info(dev)[0] * 0.7) // per_rep + 1)))
+    reps = []
+    for i in range(n_rep):
+        k, v, ki = (lay0.k, lay0.v, lay0.kidx) if i == 0 else (lay0.k.clone(), lay0.v.clone(), lay0.kidx.clone())
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        reps.append(dict(k=k, v=v, kidx=ki, status=st, out=torch.empty_like(out),
+                         cache=rtp.rtp_cache(k.data_ptr(), v.data_ptr(), ki.data_ptr(), st.data_ptr())))
+    cap = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(cap):
+        for r in reps:  # eager warm-up
+            rtp.rtp_append_kv(lay0.cfg, r["cache"], k_new, v_new, last, 1, w_k)
+            rtp.rtp_decode_attn(lay0.cfg, r["cache"], q, seq, Lh, w_q, r["out"], None, None,
+                                lay0.ws_decode, lay0.ws_decode_bytes)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for r in reps:
+            rtp.rtp_append_kv(lay0.cfg, r["cache"], k_new, v_new, last, 1, w_k)
+            rtp.rtp_decode_attn(lay0.cfg, r["cache"], q, seq, Lh, w_q, r["out"], None, None,
+                                lay0.ws_decode, lay0.ws_decode_bytes)
+    n_graph = max(1, steps // n_rep)
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(int(2e7))
+    e0.record()
+    for _ in range(n_graph):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if sum(int(r["status"].item()) for r in reps):
+        raise RuntimeError(f"device status set during the {name} steps")
+    us = e0.elapsed_time(e1) * 1e3 / (n_graph * n_rep * B)
+    return {"us_per_token": round(us, 3), "hbm_gbs": round(nbytes["total"] / (us * B * 1e-6) / 1e9, 1),
+            "bytes_per_step": nbytes["total"], "steps": n_graph * n_rep, "replicas": n_rep,
+            "kept_per_head": cnt.cpu().numpy().tolist()}
+
+
+def _popcount_words(w: torch.Tensor, lut: torch.Tensor) -> torch.Tensor:
+    """Set bits of each int32 word (same shape, int64)."""
+    by = lut[w.contiguous().view(torch.uint8).long()]
+    return by.view(*w.shape, 4).sum(-1)
+
+
+def prefill_pairs(sh, bm: torch.Tensor, start: int, T: int) -> int:
+    """(query row, key) pairs the prefill chunk attends: every row keeps its
+    sinks and window; retrieval rows add their top-p tokens outside those,
+    counted exactly from the bitmask (prefix popcounts per row)."""
+    dev = bm.device
+    lut = torch.tensor([bin(i).count("1") for i in range(256)], dtype=torch.int64, device=dev)
+    pos = start + torch.arange(T, device=dev, dtype=torch.int64)
+    s_cnt = torch.clamp(pos + 1, max=sh.n_sink)
+    sw0 = torch.maximum(s_cnt, pos + 1 - sh.window)
+    sw_rows = int((s_cnt + (pos + 1 - sw0)).sum().item())
+    B, NR, _, words = bm.shape
+    extra = 0
+    for b in range(B):
+        for hh in range(NR):
+            wd = bm[b, hh]  # [T, words]
+            cum = torch.cumsum(_popcount_words(wd, lut), dim=1)
+
+            def below(x):  # kept bits at positions < x, per row
+                wi, bi = x >> 5, x & 31
+                full = torch.where(wi > 0, cum.gather(1, (wi - 1).clamp(min=0)[:, None]).squeeze(1),
+                                   torch.zeros_like(wi))
+                word = wd.gather(1, wi.clamp(max=words - 1)[:, None]).squeeze(1).to(torch.int64) & 0xFFFFFFFF
+                part = _popcount_words((word & ((1 << bi) - 1)).to(torch.int32), lut)
+                return full + part
+            extra += int((below(sw0) - below(s_cnt)).sum().item())
+    return B * sh.n_q_heads * sw_rows + extra
+
+
+def prefill_extra(dev, reps: int) -> dict:
+    """ms per 32K causal prefill chunk (rtp_prefill_attn) and the attention
+    kernel's tensor-pipe roofline."""
+    import head_wise_sparse_local_b200 as rtp
+    from synth import make_prefill_inputs, workload
+    w = workload("prefill_32k_bf16")
+    inp = make_prefill_inputs(w)
+    sh = inp["shape"]
+    B, T, Hq, D = sh.batch, int(w["ctx"]), sh.n_q_heads, sh.head_dim
+    lay = rtp.Layer(sh, inp["max_ctx"], device=dev, prefill_T=T)
+    w_q, w_k = inp["w_q"].to(dev), inp["w_k"].to(dev)
+    start = torch.zeros(B, dtype=torch.int32, device=dev)
+    lay.append(inp["k_pre"][:, :T].contiguous().to(dev), inp["v"][:, :T].contiguous().to(dev), start, w_k)
+    q = inp["q_pre"].to(dev)
+    out = torch.empty((B, T, Hq, D), dtype=sh.torch_dtype, device=dev)
+    NR = sh.n_retrieval * sh.group
+    words = (inp["max_ctx"] + 31) // 32
+    bm = torch.zeros((B, NR, T, words), dtype=torch.int32, device=dev)
+    lay.prefill(q, start, w_q, out, sel_bitmask=bm)
+    torch.cuda.synchronize()
+    pairs = prefill_pairs(sh, bm, 0, T)
+    del bm
+    flops = 4.0 * D * pairs
+    for _ in range(2):
+        lay.prefill(q, start, w_q, out)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lay.prefill(q, start, w_q, out)
+        e1.record()
+        torch.cuda.synchronize()
+        ts.append(e0.elapsed_time(e1))
+    # per-kernel times (CUDA events around each launch on the launching stream)
+    kern = {}
+    for stage in ("prefill_index", "prefill_attn"):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        v = []
+        for _ in range(reps):
+            rtp.rtp_trace_stage(stage, e0, e1)
+            lay.prefill(q, start, w_q, out)
+            torch.cuda.synchronize()
+            v.append(e0.elapsed_time(e1))
+        kern[stage] = float(np.median(v))
+    if lay.device_status():
+        raise RuntimeError("device status set during the prefill runs")
+    peaks = json.load(open(PEAKS_PATH)) if os.path.exists(PEAKS_PATH) else {}
+    peak = float(peaks.get("bf16_tflops", 1590.0))
+    att_tf = flops / (kern["prefill_attn"] * 1e-3) / 1e12
+    return {"ms": round(float(np.median(ts)), 4), "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
+            "attended_pairs": pairs, "attn_flop": flops,
+            "roofline": {"bound": "tensor", "kernel": "prefill_attn", "achieved": round(att_tf, 1),
+                         "peak": peak, "peak_source": "measured" if "bf16_tflops" in peaks else "fallback",
+                         "unit": "TFLOP/s", "frac": round(att_tf / peak, 4),
+                         "note": "mma.sync m16n8k16 bf16 path (legacy tensor-core instructions)"},
+            "data": "inputs larger than L2 (q 268 MB)"}
 
 
 # ---------------------------------------------------------------------------
@@ -448,6 +639,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=300)
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle timing")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true", help="skip the 1M decode and 32K prefill lines")
+    ap.add_argument("--extra-steps", type=int, default=1000)
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -486,6 +679,17 @@ def main():
                "kind": "oracle",
                "sample": f"{n} full oracle steps (append the decode token + decode) of {args.workload}; "
                          f"context built untimed"}
+    extras = None
+    if dist.rank == 0 and dist.world == 1 and not args.no_extras:
+        dev = torch.device("cuda", dist.local_rank)
+        extras = {}
+        for name, fn in (("decode_1m_bf16", lambda: decode_extra("decode_1m_bf16", dev, args.extra_steps)),
+                         ("prefill_32k_bf16", lambda: prefill_extra(dev, 5))):
+            try:
+                extras[name] = fn()
+            except torch.cuda.OutOfMemoryError as e:  # pragma: no cover - depends on the device
+                extras[name] = {"skipped": f"out of device memory: {e}"}
+            torch.cuda.empty_cache()
     if dist.rank == 0:
         tot_bytes = r["nbytes"]["total"]
         gbs = tot_bytes * args.steps * dist.world / (r["ms_per_step"] * args.steps * 1e-3) / 1e9
@@ -509,6 +713,7 @@ def main():
             "e2e": {k: (round(v, 3) if isinstance(v, float) else v) for k, v in r["e2e"].items()},
             "gpu_launches": r["gpu_launches"],
             "clocks": r["clocks"],
+            "extras": extras,
         }
         print(json.dumps(line), flush=True)
     dist.close()
