@@ -4,8 +4,10 @@
 //
 //   select_rows_kernel  retrieval query heads only.  One warp per query row,
 //       8 rows per CTA sharing the 16-d indexer-key tiles staged in shared
-//       memory.  Scores use the same fp32 FMA sequence as the decode path,
-//       so a row's selection equals the decode selection at that position.
+//       memory.  Each pass computes a tile's scores for all 8 rows on tensor
+//       cores (q~ as bf16 hi + lo parts: the fp32 score to about 2^-17), so a
+//       row's selection equals the decode step's at that position except for
+//       tokens within that rounding of the threshold.
 //       The exact top-p threshold is found by splitting the score interval
 //       that contains the boundary 8 ways per pass, with the softmax mass
 //       exp(s - max) of every score in 2^-36 fixed point (mass36, shared with
@@ -27,7 +29,7 @@ namespace {
 
 constexpr int kSelRows = 8;       // query rows (warps) per selection CTA
 constexpr int kKeyTile = 256;     // indexer keys staged per step
-constexpr int kCand = 256;        // tokens the exact solve takes per row
+constexpr int kCand = 160;        // tokens the exact solve takes per row
 constexpr int kBQ = 64;           // attention: query rows per CTA (16 per warp)
 constexpr int kBK = 64;           // attention: keys per tile
 
@@ -77,6 +79,35 @@ __device__ __forceinline__ unsigned wmaxu(unsigned v) {
   return v;
 }
 
+// ---------------------------------------------------------------------------
+// tensor-core helpers (mma.sync m16n8k16 bf16, fp32 accumulate; ldmatrix)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(unsigned& r0, unsigned& r1, unsigned& r2, unsigned& r3, const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x2(unsigned& r0, unsigned& r1, const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(a));
+}
+__device__ __forceinline__ void ldsm_x2_t(unsigned& r0, unsigned& r1, const void* p) {
+  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(a));
+}
+__device__ __forceinline__ void mma_bf16(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
+                                         unsigned b0, unsigned b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ unsigned pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const unsigned*>(&v);
+}
+
 // What a row's warp does with each of its scores in one pass over its keys.
 enum : int {
   kOpMax = 0,    // row maximum
@@ -111,8 +142,10 @@ struct RowSel {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kSelRows * 32) select_rows_kernel(PrefillArgs a) {
-  __shared__ __align__(16) __nv_bfloat16 s_k[kKeyTile * kIdxDim];
+__global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillArgs a) {
+  __shared__ __align__(16) __nv_bfloat16 s_k[2][kKeyTile * kIdxDim];  // double-buffered key tiles
+  __shared__ float s_sc[kSelRows][kKeyTile + 4];  // this tile's scores of the CTA's rows
+  __shared__ float s_qi[kSelRows][kIdxDim];
   __shared__ uint2 s_cand[kSelRows][kCand];
   __shared__ unsigned long long s_cw[kSelRows][kCand];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -162,6 +195,27 @@ __global__ void __launch_bounds__(kSelRows * 32) select_rows_kernel(PrefillArgs 
 #pragma unroll
     for (int o = 0; o < kIdxDim; ++o) qi[o] = __shfl_sync(0xffffffffu, part[o >> 3], (o & 7) * 4);
   }
+  if (lane < kIdxDim) s_qi[warp][lane] = qi[lane];
+  __syncthreads();
+  // Scores on tensor cores: S = K~ Q~^T with K = 16, q~ split into bf16 hi and
+  // lo parts (the products are exact; fp32 accumulation), so the score is the
+  // fp32 q~ . k~ to about 2^-17 relative.  B fragments (16 dims x 8 rows): lane
+  // holds row lane/4, dims 2t, 2t+1 (b0) and 2t+8, 2t+9 (b1), t = lane % 4.
+  unsigned bh0, bh1, bl0, bl1;
+  {
+    const int n = lane >> 2, k0 = (lane & 3) * 2;
+    float v[4] = {s_qi[n][k0], s_qi[n][k0 + 1], s_qi[n][k0 + 8], s_qi[n][k0 + 9]};
+    float hi[4], lo[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      hi[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+      lo[e] = v[e] - hi[e];
+    }
+    bh0 = pack_bf16(hi[0], hi[1]);
+    bh1 = pack_bf16(hi[2], hi[3]);
+    bl0 = pack_bf16(lo[0], lo[1]);
+    bl1 = pack_bf16(lo[2], lo[3]);
+  }
 
   RowSel rs;
   rs.op = row_ok ? kOpMax : kOpDone;
@@ -189,13 +243,37 @@ __global__ void __launch_bounds__(kSelRows * 32) select_rows_kernel(PrefillArgs 
     tie_cnt = 0u;
     zsum = 0ull;
     const bool first_split = (op == kOpSplit) && rs.first;
-    for (int kt = 0; kt <= i_last; kt += kKeyTile) {
-      __syncthreads();
-      {  // stage keys [kt, kt + kKeyTile) (only up to i_last)
-        const int n = min(kKeyTile, i_last + 1 - kt);
-        const uint4* src = reinterpret_cast<const uint4*>(kidx + (size_t)kt * kIdxDim);
-        uint4* dst = reinterpret_cast<uint4*>(s_k);
-        for (int v = threadIdx.x; v < n * 2; v += kSelRows * 32) dst[v] = __ldg(src + v);
+    // key tiles [kt, kt + kKeyTile) up to i_last, copied asynchronously one
+    // tile ahead of their use
+    auto stage_async = [&](int kt_, int buf) {
+      const int n = min(kKeyTile, i_last + 1 - kt_);
+      const char* src = reinterpret_cast<const char*>(kidx + (size_t)kt_ * kIdxDim);
+      const unsigned dst = (unsigned)__cvta_generic_to_shared(s_k[buf]);
+      for (int v = threadIdx.x; v < n * 2; v += kSelRows * 32)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst + 16u * v), "l"(src + 16 * (size_t)v));
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    __syncthreads();  // the previous pass is done with both buffers
+    stage_async(0, 0);
+    int buf = 0;
+    for (int kt = 0; kt <= i_last; kt += kKeyTile, buf ^= 1) {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      __syncthreads();  // tile kt landed for every thread; the other buffer is free
+      if (kt + kKeyTile <= i_last) stage_async(kt + kKeyTile, buf ^ 1);
+      // warp w: the scores of keys [32 w, 32 w + 32) of this tile for all rows
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int kb = warp * 32 + half * 16;  // first key (M row) of this 16 x 8 tile
+        unsigned a0, a1, a2, a3;
+        ldsm_x4(a0, a1, a2, a3, s_k[buf] + (size_t)(kb + (lane & 7) + ((lane >> 3) & 1) * 8) * kIdxDim + (lane >> 4) * 8);
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+        mma_bf16(c, a0, a1, a2, a3, bh0, bh1);
+        mma_bf16(c, a0, a1, a2, a3, bl0, bl1);
+        const int key0 = kb + (lane >> 2), row0 = (lane & 3) * 2;
+        s_sc[row0][key0] = c[0] * kIdxScale + 0.0f;  // +0 turns -0 into +0
+        s_sc[row0 + 1][key0] = c[1] * kIdxScale + 0.0f;
+        s_sc[row0][key0 + 8] = c[2] * kIdxScale + 0.0f;
+        s_sc[row0 + 1][key0 + 8] = c[3] * kIdxScale + 0.0f;
       }
       __syncthreads();
       if (op == kOpDone || kt > i) continue;  // uniform per warp
@@ -203,27 +281,7 @@ __global__ void __launch_bounds__(kSelRows * 32) select_rows_kernel(PrefillArgs 
       for (int u = 0; u < kKeyTile / 32; ++u) {
         const int j = kt + u * 32 + lane;
         const bool on = j <= i;
-        float s = 0.f;
-        if (on) {
-          float kv[kIdxDim];
-          {  // shared-memory row (plain loads: this is not global memory)
-            const uint4* kp = reinterpret_cast<const uint4*>(s_k + (size_t)(u * 32 + lane) * kIdxDim);
-#pragma unroll
-            for (int v = 0; v < 2; ++v) {
-              const uint4 raw = kp[v];
-              const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const float2 f = __bfloat1622float2(h2[q]);
-                kv[v * 8 + 2 * q] = f.x;
-                kv[v * 8 + 2 * q + 1] = f.y;
-              }
-            }
-          }
-#pragma unroll
-          for (int q = 0; q < kIdxDim; ++q) s = fmaf(qi[q], kv[q], s);
-          s = s * kIdxScale + 0.0f;
-        }
+        const float s = on ? s_sc[warp][u * 32 + lane] : 0.f;
         const unsigned key = score_key(s);
         if (op == kOpMax) {
           if (on) fmx = fmaxf(fmx, s);
@@ -233,9 +291,10 @@ __global__ void __launch_bounds__(kSelRows * 32) select_rows_kernel(PrefillArgs 
           if (lane == 0 && kt + u * 32 <= i) mrow[(kt >> 5) + u] = wd;
         } else if (on) {
           const float d = rs.m - s;
-          const unsigned long long w = mass36(s, rs.m);
-          if (first_split) zsum += w;
           const bool inside = d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi;
+          unsigned long long w = 0ull;
+          if (first_split || (op == kOpSplit && inside)) w = mass36(s, rs.m);
+          if (first_split) zsum += w;
           if (inside) {
             if (op == kOpSplit) {
               int q = 0;
@@ -451,32 +510,6 @@ __global__ void __launch_bounds__(kSelRows * 32) select_rows_kernel(PrefillArgs 
 // ---------------------------------------------------------------------------
 // masked causal attention on tensor cores
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void ldsm_x4(unsigned& r0, unsigned& r1, unsigned& r2, unsigned& r3, const void* p) {
-  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(a));
-}
-__device__ __forceinline__ void ldsm_x2(unsigned& r0, unsigned& r1, const void* p) {
-  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(a));
-}
-__device__ __forceinline__ void ldsm_x2_t(unsigned& r0, unsigned& r1, const void* p) {
-  const unsigned a = (unsigned)__cvta_generic_to_shared(p);
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(a));
-}
-__device__ __forceinline__ void mma_bf16(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
-                                         unsigned b0, unsigned b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ unsigned pack_bf16(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const unsigned*>(&v);
-}
-
 template <int D>
 struct AttnSmem {
   static constexpr int kStride = D + 8;  // bf16 elements per shared row (pad: no ldmatrix conflicts)
