@@ -360,37 +360,51 @@ def run_ours(args, dist: Dist) -> dict:
         per_stage[stages[i % len(stages)]].append(evs[i][0].elapsed_time(evs[i][1]) * 1e3)
     kern_us = {s: float(np.mean(v)) for s, v in per_stage.items()}
 
-    # end to end: pinned host inputs -> device -> layer -> pinned host output, per step
-    h_q = torch.empty(q.shape, dtype=dt, pin_memory=True).copy_(q.cpu())
-    h_k = torch.empty(k_new.shape, dtype=dt, pin_memory=True).copy_(k_new.cpu())
-    h_v = torch.empty(v_new.shape, dtype=dt, pin_memory=True).copy_(v_new.cpu())
-    h_seq = torch.empty(seq.shape, dtype=torch.int32, pin_memory=True).copy_(seq.cpu())
-    h_pos = torch.empty(seq.shape, dtype=torch.int32, pin_memory=True).copy_(last.cpu())
-    h_out = torch.empty((B, Hq, D), dtype=dt, pin_memory=True)
-    d_q, d_k, d_v = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
-    d_seq, d_pos = torch.empty_like(seq), torch.empty_like(last)
-    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_seq, h_pos))
-    d2h = h_out.numel() * h_out.element_size()
+    # end to end: pinned host inputs -> device -> layer -> pinned host output, per step.
+    # The step's inputs travel packed in one pinned buffer (one copy each way);
+    # the copies and the two public-API calls are captured once per replica in a
+    # CUDA graph, replayed and synchronised every step.
+    segs = [("q", q), ("k", k_new), ("v", v_new), ("seq", seq), ("pos", last)]
+    offs, total = {}, 0
+    for name, t in segs:
+        offs[name] = total
+        total += -(-t.numel() * t.element_size() // 256) * 256
+    h_in = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    d_in = torch.empty(total, dtype=torch.uint8, device=dev)
 
-    def e2e_step(rep):
-        d_q.copy_(h_q, non_blocking=True)
-        d_k.copy_(h_k, non_blocking=True)
-        d_v.copy_(h_v, non_blocking=True)
-        d_seq.copy_(h_seq, non_blocking=True)
-        d_pos.copy_(h_pos, non_blocking=True)
-        rtp.rtp_append_kv(cfg, rep["cache"], d_k, d_v, d_pos, 1, w_k)
-        rtp.rtp_decode_attn(cfg, rep["cache"], d_q, d_seq, Lh, w_q, rep["out"], None, None, ws, ws_bytes)
-        h_out.copy_(rep["out"], non_blocking=True)
-        torch.cuda.current_stream().synchronize()
+    def view(buf, name, like):
+        n = like.numel() * like.element_size()
+        return buf[offs[name]:offs[name] + n].view(like.dtype).view(like.shape)
+
+    for name, t in segs:
+        view(h_in, name, t).copy_(t.cpu())
+    dq, dk, dv, dseq, dpos = (view(d_in, name, t) for name, t in segs)
+    h_out = torch.empty((B, Hq, D), dtype=dt, pin_memory=True)
+    h2d = total
+    d2h = h_out.numel() * h_out.element_size()
+    e2e_graphs = []
+    for rep in reps:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap):
+            d_in.copy_(h_in, non_blocking=True)
+            rtp.rtp_append_kv(cfg, rep["cache"], dk, dv, dpos, 1, w_k)
+            rtp.rtp_decode_attn(cfg, rep["cache"], dq, dseq, Lh, w_q, rep["out"], None, None, ws, ws_bytes)
+            h_out.copy_(rep["out"], non_blocking=True)
+        e2e_graphs.append(g)
+    stream = torch.cuda.current_stream()
+
+    def e2e_step(i):
+        e2e_graphs[i % n_rep].replay()
+        stream.synchronize()
 
     for i in range(5):
-        e2e_step(reps[i % n_rep])
+        e2e_step(i)
     n_e = args.e2e_steps
     dist.barrier()
     torch.cuda.synchronize()
     te0 = time.perf_counter()
     for i in range(n_e):
-        e2e_step(reps[i % n_rep])
+        e2e_step(i)
     te1 = time.perf_counter()
     e2e_s = dist.max(te1 - te0)
     if not torch.equal(h_out, out0.cpu()):
