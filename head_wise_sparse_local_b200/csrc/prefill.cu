@@ -297,17 +297,18 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
           if (first_split) zsum += w;
           if (inside) {
             if (op == kOpSplit) {
-              int q = 0;
+              // cumulative sums: pm[e] / pc[e] (e < 7) gather what lies past
+              // threshold e, pm[7] / pc[7] everything inside
+              pm[7] += w;
+              pc[7] += 1u;
               if (!rs.by_key) {
 #pragma unroll
-                for (int e = 0; e < 7; ++e) q += (d >= rs.th[e]) ? 1 : 0;
+                for (int e = 0; e < 7; ++e)
+                  if (d >= rs.th[e]) { pm[e] += w; pc[e] += 1u; }
               } else {
 #pragma unroll
-                for (int e = 0; e < 7; ++e) q += (key < rs.kth[e]) ? 1 : 0;
-              }
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                if (q == e) { pm[e] += w; pc[e] += 1u; }
+                for (int e = 0; e < 7; ++e)
+                  if (key < rs.kth[e]) { pm[e] += w; pc[e] += 1u; }
               }
             } else if (op == kOpRange) {
               kmn = min(kmn, key);
@@ -360,6 +361,16 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
     } else if (op == kOpSplit) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) { pm[e] = wsum64(pm[e]); pc[e] = wsum32(pc[e]); }
+      {  // cumulative -> per sub-interval (e = 0 holds the highest scores)
+        const unsigned long long tm = pm[7];
+        const unsigned tc = pc[7];
+        pm[7] = pm[6];
+        pc[7] = pc[6];
+#pragma unroll
+        for (int e = 6; e >= 1; --e) { pm[e] = pm[e - 1] - pm[e]; pc[e] = pc[e - 1] - pc[e]; }
+        pm[0] = tm - pm[0];
+        pc[0] = tc - pc[0];
+      }
       if (first_split) {
         const unsigned long long Z = wsum64(zsum);
         unsigned long long target = (unsigned long long)ceil((double)a.top_p * (double)Z);
