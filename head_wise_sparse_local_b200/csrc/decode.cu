@@ -54,6 +54,7 @@ constexpr int kBruteMax = kSelThreads;  // exact solve by pairwise ranks up to t
 constexpr int kGroup = 4;           // kept rows a warp attends per memory round trip
 constexpr int kPos = kLgCap / kSelThreads;  // positions a select thread owns per staged chunk
 constexpr int kTopPerWarp = 16;     // top-rung items a warp hands the leader in the first pass
+constexpr int kSpec = 2;            // of those, rows whose keys and values a warp stages early
 
 // Tokens per score CTA: eight (bf16) or four (fp32) 16-d keys per thread.
 __host__ __device__ constexpr int score_chunk(int esize) { return kThreads * (esize == 2 ? 8 : 4); }
@@ -679,8 +680,11 @@ struct Items {
 // their softmax mass, digits ranked high to low.  !kMass: items with key ==
 // key_eq counted, index digits ranked low to high.  Finds the first digit at
 // which the running total reaches `need`.
+// The general solvers below are rarely reached by a decode step; kept out of
+// line so that the common path's code stays compact (each code block a
+// launch reaches for the first time costs an instruction fetch from L2).
 template <bool kMass>
-__device__ DigitResult radix_step(const Items& it, int n, uint32_t prefix, uint32_t mask,
+__device__ __noinline__ DigitResult radix_step(const Items& it, int n, uint32_t prefix, uint32_t mask,
                                   uint32_t key_eq, int shift, float m, unsigned long long need,
                                   unsigned long long* h_m, unsigned* h_c, DigitResult* s_res) {
   const int tid = threadIdx.x;
@@ -744,7 +748,7 @@ __device__ DigitResult radix_step(const Items& it, int n, uint32_t prefix, uint3
 // Exact tau / j_cut among n items whose mass must supply `need` (one CTA).
 // Order: key descending, index ascending.  The kept set is the shortest prefix
 // whose mass reaches `need`.
-__device__ void solve_radix(const Items& it, int n, float m, unsigned long long need,
+__device__ __noinline__ void solve_radix(const Items& it, int n, float m, unsigned long long need,
                             unsigned long long* h_m, unsigned* h_c, DigitResult* s_res,
                             uint32_t* s_kr, float& tau, int& jcut) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -816,7 +820,7 @@ __device__ void solve_radix(const Items& it, int n, float m, unsigned long long 
 
 // Exact tau / j_cut for n <= blockDim.x list items: item i is kept iff the
 // mass of the items ordered before it is below `need`.
-__device__ void solve_brute(const uint2* items, int n, float m, unsigned long long need,
+__device__ __noinline__ void solve_brute(const uint2* items, int n, float m, unsigned long long need,
                             unsigned long long* s_w, uint32_t* s_min, int* s_jmax, float& tau,
                             int& jcut) {
   const int tid = threadIdx.x;
@@ -882,7 +886,7 @@ __device__ void solve_warp(const uint2* items, int n, float m, unsigned long lon
   const uint2 me = lane < n ? items[lane] : make_uint2(0u, 0u);
   const unsigned long long w = lane < n ? mass36(key_score(me.x), m) : 0ull;
   unsigned long long before = 0ull;
-#pragma unroll 1
+#pragma unroll 4
   for (int j = 0; j < n; ++j) {
     const unsigned ox = __shfl_sync(0xffffffffu, me.x, j);
     const unsigned oy = __shfl_sync(0xffffffffu, me.y, j);
@@ -959,6 +963,8 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   __shared__ uint32_t s_min;
   __shared__ int s_jmax;
   __shared__ uint2 s_small[32];
+  __shared__ __align__(16) T s_spec[kSelWarps][kSpec][2][D];  // early-staged K, V rows per warp
+  __shared__ int s_spec_j[kSelWarps][kSpec];
   __shared__ __align__(16) float s_qh[D];
   __shared__ __align__(16) float s_wo[kSelWarps * D];
   __shared__ float s_wml[kSelWarps * 2];
@@ -998,6 +1004,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
     s_qh[tid + D / 2] = (qx2 * c + qx1 * s) * qscale;
   }
   if (rank == 0 && tid == 0) sh->n_cand2 = 0u;
+  if (lane < kSpec) s_spec_j[warp][lane] = -1;
   cluster_arrive();  // counter zeroed; every CTA of the cluster running
   griddep_wait();
   griddep_launch();
@@ -1013,7 +1020,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   float tau = -CUDART_INF_F;
   int jcut = INT_MAX;
 
-  if (!keep_all) {  // uniform over the grid
+  if (__builtin_expect(!keep_all, 1)) {  // uniform over the grid
     // maximum score (per-chunk maxima of the score kernel)
     float m;
     {
@@ -1075,20 +1082,35 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         if (__any_sync(0xffffffffu, topbits != 0u)) {
           uint2* region = lead_cand + (rank * kSelWarps + warp) * kTopPerWarp;
           for (int u = 0; u < kPos; ++u) {
-            const bool top = (topbits >> u) & 1u;
-            const unsigned bal = __ballot_sync(0xffffffffu, top);
-            if (!bal) continue;
-            const unsigned slot = wtop + __popc(bal & ((1u << lane) - 1u));
-            if (top) {
-              const int j = c0 + u * kSelThreads + tid;
-              if (slot < (unsigned)kTopPerWarp) region[slot] = make_uint2(score_key(s_lg[j - c0]), (unsigned)j);
+            unsigned bal = __ballot_sync(0xffffffffu, (topbits >> u) & 1u);
+            while (bal) {  // warp-uniform, one item at a time
+              const int src = __ffs(bal) - 1;
+              bal &= bal - 1u;
+              const int j = c0 + u * kSelThreads + warp * 32 + src;
+              if (lane == src && wtop < (unsigned)kTopPerWarp)
+                region[wtop] = make_uint2(score_key(s_lg[j - c0]), (unsigned)j);
+              if (wtop < (unsigned)kSpec && cached) {
+                // the warp's first rows: keys and values into shared memory
+                constexpr int NC = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
+                const unsigned dk = (unsigned)__cvta_generic_to_shared(s_spec[warp][wtop][0]);
+                const unsigned dv = (unsigned)__cvta_generic_to_shared(s_spec[warp][wtop][1]);
+                for (int c = lane; c < 2 * NC; c += 32) {
+                  const bool isv = c >= NC;
+                  const int cc = isv ? c - NC : c;
+                  const char* src_p = reinterpret_cast<const char*>((isv ? vb : kb) + (size_t)j * D) + 16 * cc;
+                  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"((isv ? dv : dk) + 16u * cc), "l"(src_p));
+                }
+                asm volatile("cp.async.commit_group;" ::: "memory");
+                if (lane == 0) s_spec_j[warp][wtop] = j;
+              } else if (lane == src) {
 #pragma unroll
-              for (int o = 0; o < D * (int)sizeof(T); o += 128) {
-                prefetch_l2(reinterpret_cast<const char*>(kb + (size_t)j * D) + o);
-                prefetch_l2(reinterpret_cast<const char*>(vb + (size_t)j * D) + o);
+                for (int o = 0; o < D * (int)sizeof(T); o += 128) {
+                  prefetch_l2(reinterpret_cast<const char*>(kb + (size_t)j * D) + o);
+                  prefetch_l2(reinterpret_cast<const char*>(vb + (size_t)j * D) + o);
+                }
               }
+              ++wtop;
             }
-            wtop += __popc(bal);
           }
         }
       }
@@ -1161,8 +1183,8 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
       if (k == kf) t_lo = m - rung_delta(k);
 
     uint2* gcand = a.cand + (size_t)bh * a.lstride;
-    if (tier1 || tier2) {
-      if (tier2) {  // every score at or above rung kf -> the leader
+    if (__builtin_expect(tier1 || tier2, 1)) {
+      if (__builtin_expect(tier2, 0)) {  // every score at or above rung kf -> the leader
         for (int c0 = j0; c0 < j1; c0 += kLgCap) {
           const int c1 = min(j1, c0 + kLgCap);
           if (!cached) {
@@ -1198,23 +1220,32 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         bool done = false;
         float t_tau = 0.f;
         int t_jcut = 0;
-        if (tier1 && Ck[kRungs - 1] <= 32u) {
+        if (__builtin_expect(tier1 && Ck[kRungs - 1] <= 32u, 1)) {
           // few items: warp 0 gathers the regions' items at or above rung kf and solves
+          // (items below rung kf cannot be kept: the mass before them already
+          // reaches the target, so the solve needs no filtering)
           if (warp == 0) {
-            const uint32_t klo = score_key(t_lo);
-            if (lane == 0) s_min = 0u;
-            __syncwarp();
-#pragma unroll 1
-            for (int rg = lane; rg < CS * kSelWarps; rg += 32) {
-              const int cnt_r = (int)sh->wcnt[rg];
-#pragma unroll 1
-              for (int i = 0; i < cnt_r; ++i) {
-                const uint2 e = s_cand[rg * kTopPerWarp + i];
-                if (e.x >= klo) s_small[atomicAdd(&s_min, 1u)] = e;
-              }
+            constexpr int RPL = kMaxCS * kSelWarps / 32;  // regions per lane
+            const int nreg = CS * kSelWarps;
+            unsigned cr[RPL], c = 0u;
+#pragma unroll
+            for (int k = 0; k < RPL; ++k) {
+              const int rg = lane * RPL + k;
+              cr[k] = rg < nreg ? sh->wcnt[rg] : 0u;
+              c += cr[k];
             }
+            unsigned off = c;  // exclusive warp prefix of the lanes' counts
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const unsigned v = __shfl_up_sync(0xffffffffu, off, o);
+              if (lane >= o) off += v;
+            }
+            off -= c;
+            n = (int)__shfl_sync(0xffffffffu, off + c, 31);
+#pragma unroll
+            for (int k = 0; k < RPL; ++k)
+              for (unsigned i = 0; i < cr[k]; ++i) s_small[off++] = s_cand[(lane * RPL + k) * kTopPerWarp + i];
             __syncwarp();
-            n = (int)s_min;
             solve_warp(s_small, n, m, target, t_tau, t_jcut);
           }
           done = true;
@@ -1497,7 +1528,9 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
       if ((outbits >> u) & 1u) wrows[wn + __popc(ob & ((1u << lane) - 1u))] = jw + lane;
       wn += __popc(ob);
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's early copies
     __syncwarp();
+    const int sj0 = s_spec_j[warp][0], sj1 = s_spec_j[warp][1];
     for (int i0 = 0; i0 < wn; i0 += kGroup) {  // wn is warp-uniform
       int rw[kGroup];
       Raw kr[kGroup], vr[kGroup];
@@ -1507,8 +1540,14 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         vr[k] = Raw();
         rw[k] = (i0 + k < wn) ? wrows[i0 + k] : -1;
         if (rw[k] >= 0) {
-          kr[k] = ld_stream(reinterpret_cast<const Raw*>(kb + (size_t)rw[k] * D + lane * DL), pol);
-          vr[k] = ld_stream(reinterpret_cast<const Raw*>(vb + (size_t)rw[k] * D + lane * DL), pol);
+          const int sp = rw[k] == sj0 ? 0 : (rw[k] == sj1 ? 1 : -1);
+          if (sp >= 0) {
+            kr[k] = *reinterpret_cast<const Raw*>(&s_spec[warp][sp][0][lane * DL]);
+            vr[k] = *reinterpret_cast<const Raw*>(&s_spec[warp][sp][1][lane * DL]);
+          } else {
+            kr[k] = ld_stream(reinterpret_cast<const Raw*>(kb + (size_t)rw[k] * D + lane * DL), pol);
+            vr[k] = ld_stream(reinterpret_cast<const Raw*>(vb + (size_t)rw[k] * D + lane * DL), pol);
+          }
         }
       }
       float sc[kGroup];

@@ -181,3 +181,19 @@ def test_decode_all_scores_equal(p):
     for s in sets:
         assert np.array_equal(s, np.arange(want)), (len(s), want)
     check_decode_parity(inp, top_p=p)
+
+
+def test_decode_tiny_p_keeps_the_top_token():
+    # p far below any single token's probability: the set is the top token
+    inp = _small(ctx=3000, needles=8)
+    st = check_decode_parity(inp, top_p=1e-6)
+    assert np.all(st["counts"] == 1), st["counts"]
+
+
+def test_decode_many_needles_second_tier():
+    # every other token a needle: more than 4096 scores lie within 8 of the
+    # maximum, so the selection collects a lower rung's scores in a second pass
+    # (or falls back to the histogram); both must stay exact
+    inp = _small(ctx=20000, needles=10000)
+    st = check_decode_parity(inp, top_p=0.9)
+    assert st["exact"] >= st["heads"] - 1

@@ -86,3 +86,12 @@ def test_prefill_32k_sampled_rows():
     rows = [0, 1, 64, 2047, 2048, 5000, 16383, 16384, 30000, 32767]
     st = check_prefill_parity(inp, rows=rows)
     assert st["exact"] >= st["heads"] - 2
+
+
+def test_prefill_single_row_and_tiny_p():
+    inp = _inp(T=1, start=0, n_sink=4, window=16, top_p=0.9)
+    st = check_prefill_parity(inp)
+    assert st["exact"] == st["heads"]
+    inp = _inp(T=300, start=100, n_sink=4, window=16, top_p=1e-6)
+    st = check_prefill_parity(inp)
+    assert np.all(st["g"]["count"] == 1)
