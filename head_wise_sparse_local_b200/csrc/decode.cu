@@ -821,23 +821,25 @@ __device__ __noinline__ void solve_radix(const Items& it, int n, float m, unsign
 // Exact tau / j_cut for n <= blockDim.x list items: item i is kept iff the
 // mass of the items ordered before it is below `need`.
 __device__ __noinline__ void solve_brute(const uint2* items, int n, float m, unsigned long long need,
-                            unsigned long long* s_w, uint32_t* s_min, int* s_jmax, float& tau,
-                            int& jcut) {
+                                         uint4* pack, uint32_t* s_min, int* s_jmax, float& tau, int& jcut) {
+  // pack[i] = (key, index, mass lo, mass hi): one 16-byte broadcast load per
+  // item in the pairwise loop (pack must not overlap items)
   const int tid = threadIdx.x;
   uint2 me = make_uint2(0u, 0u);
   if (tid < n) {
     me = items[tid];
-    s_w[tid] = mass36(key_score(me.x), m);
+    const unsigned long long w = mass36(key_score(me.x), m);
+    pack[tid] = make_uint4(me.x, me.y, (unsigned)w, (unsigned)(w >> 32));
   }
   if (tid == 0) { *s_min = 0xffffffffu; *s_jmax = -1; }
   __syncthreads();
   bool kept = false;
   if (tid < n) {
     unsigned long long before = 0ull;
-#pragma unroll 4
+#pragma unroll 8
     for (int j = 0; j < n; ++j) {
-      const uint2 o = items[j];
-      const unsigned long long ow = s_w[j];
+      const uint4 o = pack[j];
+      const unsigned long long ow = ((unsigned long long)o.w << 32) | o.z;
       if (o.x > me.x || (o.x == me.x && o.y < me.y)) before += ow;
     }
     kept = before < need;
@@ -1286,7 +1288,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         } else if (n <= 32) {
           if (warp == 0) solve_warp(s_cand, n, m, target, t_tau, t_jcut);
         } else if (n <= kBruteMax) {
-          solve_brute(s_cand, n, m, target, s_w, &s_min, &s_jmax, t_tau, t_jcut);
+          solve_brute(s_cand, n, m, target, reinterpret_cast<uint4*>(s_cand + kCandSmem / 2), &s_min, &s_jmax, t_tau, t_jcut);
         } else {
           solve_radix(Items{s_cand, false}, n, m, target, r_hm, r_hc, &s_dres, s_kr, t_tau, t_jcut);
         }
@@ -1467,7 +1469,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
             items = Items{gcand, true};
           }
           if (n <= kBruteMax)
-            solve_brute(s_cand, n, m, need, s_w, &s_min, &s_jmax, t_tau, t_jcut);
+            solve_brute(s_cand, n, m, need, reinterpret_cast<uint4*>(s_cand + kCandSmem / 2), &s_min, &s_jmax, t_tau, t_jcut);
           else
             solve_radix(items, n, m, need, r_hm, r_hc, &s_dres, s_kr, t_tau, t_jcut);
         }
