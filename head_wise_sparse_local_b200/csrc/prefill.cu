@@ -277,28 +277,59 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
       }
       __syncthreads();
       if (op == kOpDone || kt > i) continue;  // uniform per warp
-#pragma unroll 2
-      for (int u = 0; u < kKeyTile / 32; ++u) {
-        const int j = kt + u * 32 + lane;
-        const bool on = j <= i;
-        const float s = on ? s_sc[warp][u * 32 + lane] : 0.f;
-        const unsigned key = score_key(s);
-        if (op == kOpMax) {
-          if (on) fmx = fmaxf(fmx, s);
-        } else if (op == kOpEmit) {
-          const bool in = on && (s > rs.tau || (s == rs.tau && j <= rs.jcut));
-          const unsigned wd = __ballot_sync(0xffffffffu, in);
-          if (lane == 0 && kt + u * 32 <= i) mrow[(kt >> 5) + u] = wd;
-        } else if (on) {
-          const float d = rs.m - s;
-          const bool inside = d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi;
-          unsigned long long w = 0ull;
-          if (first_split || (op == kOpSplit && inside)) w = mass36(s, rs.m);
-          if (first_split) zsum += w;
-          if (inside) {
-            if (op == kOpSplit) {
-              // cumulative sums: pm[e] / pc[e] (e < 7) gather what lies past
-              // threshold e, pm[7] / pc[7] everything inside
+      // One tight loop per kind of pass over this tile's 8 groups of 32 keys
+      // (the row's op is warp-uniform).  Keys past the row (j > i) are off.
+      const float* srow = s_sc[warp];
+      const int ulim = min(kKeyTile / 32, (i - kt) / 32 + 1);  // groups holding keys <= i
+      switch (op) {
+        case kOpMax: {
+#pragma unroll 8
+          for (int u = 0; u < kKeyTile / 32; ++u) {
+            const int j = kt + u * 32 + lane;
+            if (u < ulim && j <= i) fmx = fmaxf(fmx, srow[u * 32 + lane]);
+          }
+          break;
+        }
+        case kOpEmit: {
+#pragma unroll 8
+          for (int u = 0; u < kKeyTile / 32; ++u) {
+            if (u >= ulim) break;
+            const int j = kt + u * 32 + lane;
+            const float sv = srow[u * 32 + lane];
+            const bool in = j <= i && (sv > rs.tau || (sv == rs.tau && j <= rs.jcut));
+            const unsigned wd = __ballot_sync(0xffffffffu, in);
+            if (lane == 0) mrow[(kt >> 5) + u] = wd;
+          }
+          break;
+        }
+        case kOpSplit: {
+          if (first_split) {  // every key is inside: total mass and d-thresholds
+#pragma unroll 4
+            for (int u = 0; u < kKeyTile / 32; ++u) {
+              const int j = kt + u * 32 + lane;
+              if (u >= ulim || j > i) continue;
+              const float sv = srow[u * 32 + lane];
+              const float d = rs.m - sv;
+              const unsigned long long w = mass36(sv, rs.m);
+              zsum += w;
+              pm[7] += w;
+              pc[7] += 1u;
+#pragma unroll
+              for (int e = 0; e < 7; ++e)
+                if (d >= rs.th[e]) { pm[e] += w; pc[e] += 1u; }
+            }
+          } else {
+            // cumulative sums: pm[e] / pc[e] (e < 7) gather what lies past
+            // threshold e, pm[7] / pc[7] everything inside
+#pragma unroll 4
+            for (int u = 0; u < kKeyTile / 32; ++u) {
+              const int j = kt + u * 32 + lane;
+              if (u >= ulim || j > i) continue;
+              const float sv = srow[u * 32 + lane];
+              const float d = rs.m - sv;
+              const unsigned key = score_key(sv);
+              if (!(d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi)) continue;
+              const unsigned long long w = mass36(sv, rs.m);
               pm[7] += w;
               pc[7] += 1u;
               if (!rs.by_key) {
@@ -310,28 +341,56 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
                 for (int e = 0; e < 7; ++e)
                   if (key < rs.kth[e]) { pm[e] += w; pc[e] += 1u; }
               }
-            } else if (op == kOpRange) {
-              kmn = min(kmn, key);
-              kmx = max(kmx, key);
-            } else if (op == kOpTies) {
-              if (key == rs.tie_key && (unsigned)j <= rs.tie_hi) tie_cnt += 1u;
             }
           }
+          break;
         }
-        if (op == kOpCand) {
-          bool inside = false;
-          if (on) {
-            const float d = rs.m - s;
-            inside = d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi;
+        case kOpRange: {
+#pragma unroll 4
+          for (int u = 0; u < kKeyTile / 32; ++u) {
+            const int j = kt + u * 32 + lane;
+            if (u >= ulim || j > i) continue;
+            const float sv = srow[u * 32 + lane];
+            const float d = rs.m - sv;
+            const unsigned key = score_key(sv);
+            if (d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi) {
+              kmn = min(kmn, key);
+              kmx = max(kmx, key);
+            }
           }
-          const unsigned bal = __ballot_sync(0xffffffffu, inside);
-          const unsigned slot = n_cand + __popc(bal & ((1u << lane) - 1u));
-          if (inside && slot < (unsigned)kCand) {
-            s_cand[warp][slot] = make_uint2(key, (unsigned)j);
-            s_cw[warp][slot] = mass36(s, rs.m);
-          }
-          n_cand += __popc(bal);
+          break;
         }
+        case kOpTies: {
+#pragma unroll 4
+          for (int u = 0; u < kKeyTile / 32; ++u) {
+            const int j = kt + u * 32 + lane;
+            if (u >= ulim || j > i) continue;
+            const unsigned key = score_key(srow[u * 32 + lane]);
+            if (key == rs.tie_key && (unsigned)j <= rs.tie_hi) tie_cnt += 1u;
+          }
+          break;
+        }
+        case kOpCand: {
+#pragma unroll 2
+          for (int u = 0; u < kKeyTile / 32; ++u) {
+            if (u >= ulim) break;
+            const int j = kt + u * 32 + lane;
+            const float sv = srow[u * 32 + lane];
+            const float d = rs.m - sv;
+            const unsigned key = score_key(sv);
+            const bool inside = j <= i && d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi;
+            const unsigned bal = __ballot_sync(0xffffffffu, inside);
+            const unsigned slot = n_cand + __popc(bal & ((1u << lane) - 1u));
+            if (inside && slot < (unsigned)kCand) {
+              s_cand[warp][slot] = make_uint2(key, (unsigned)j);
+              s_cw[warp][slot] = mass36(sv, rs.m);
+            }
+            n_cand += __popc(bal);
+          }
+          break;
+        }
+        default:
+          break;
       }
     }
     // ---- reduce this pass and choose the next step (warp-uniform) ----
