@@ -28,7 +28,8 @@ namespace rtp {
 namespace {
 
 constexpr int kSelRows = 8;       // query rows (warps) per selection CTA
-constexpr int kKeyTile = 256;     // indexer keys staged per step
+constexpr int kKeyTile = 512;     // indexer keys staged per step
+constexpr size_t kSelDynSmem = 2 * kKeyTile * kIdxDim * sizeof(__nv_bfloat16) + kSelRows * (kKeyTile + 4) * sizeof(float);
 constexpr int kCand = 160;        // tokens the exact solve takes per row
 constexpr int kBQ = 64;           // attention: query rows per CTA (16 per warp)
 constexpr int kBK = 64;           // attention: keys per tile
@@ -143,8 +144,11 @@ struct RowSel {
 
 template <int D>
 __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillArgs a) {
-  __shared__ __align__(16) __nv_bfloat16 s_k[2][kKeyTile * kIdxDim];  // double-buffered key tiles
-  __shared__ float s_sc[kSelRows][kKeyTile + 4];  // this tile's scores of the CTA's rows
+  // dynamic shared memory: double-buffered key tiles, then this tile's scores
+  // of the CTA's rows
+  extern __shared__ __align__(16) unsigned char sel_dsm[];
+  auto s_k = reinterpret_cast<__nv_bfloat16 (*)[kKeyTile * kIdxDim]>(sel_dsm);
+  auto s_sc = reinterpret_cast<float (*)[kKeyTile + 4]>(sel_dsm + 2 * kKeyTile * kIdxDim * sizeof(__nv_bfloat16));
   __shared__ float s_qi[kSelRows][kIdxDim];
   __shared__ uint2 s_cand[kSelRows][kCand];
   __shared__ unsigned long long s_cw[kSelRows][kCand];
@@ -260,10 +264,10 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
       asm volatile("cp.async.wait_group 0;" ::: "memory");
       __syncthreads();  // tile kt landed for every thread; the other buffer is free
       if (kt + kKeyTile <= i_last) stage_async(kt + kKeyTile, buf ^ 1);
-      // warp w: the scores of keys [32 w, 32 w + 32) of this tile for all rows
+      // warp w: the scores of keys [64 w, 64 w + 64) of this tile for all rows
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int kb = warp * 32 + half * 16;  // first key (M row) of this 16 x 8 tile
+      for (int half = 0; half < kKeyTile / kSelRows / 16; ++half) {
+        const int kb = warp * (kKeyTile / kSelRows) + half * 16;  // first key (M row) of this 16 x 8 tile
         unsigned a0, a1, a2, a3;
         ldsm_x4(a0, a1, a2, a3, s_k[buf] + (size_t)(kb + (lane & 7) + ((lane >> 3) & 1) * 8) * kIdxDim + (lane >> 4) * 8);
         float c[4] = {0.f, 0.f, 0.f, 0.f};
@@ -277,7 +281,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
       }
       __syncthreads();
       if (op == kOpDone || kt > i) continue;  // uniform per warp
-      // One tight loop per kind of pass over this tile's 8 groups of 32 keys
+      // One tight loop per kind of pass over this tile's 16 groups of 32 keys
       // (the row's op is warp-uniform).  Keys past the row (j > i) are off.
       const float* srow = s_sc[warp];
       const int ulim = min(kKeyTile / 32, (i - kt) / 32 + 1);  // groups holding keys <= i
@@ -660,6 +664,13 @@ __global__ void __launch_bounds__(128) attn_rows_kernel(PrefillArgs a) {
   const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
 
   for (int kt = 0; kt <= i_max; kt += kBK) {
+    if (r < 0 && kt >= a.S) {  // local head: jump from the sinks to the first window tile
+      const int kw = (max(0, i_min - a.W + 1) / kBK) * kBK;
+      if (kt < kw) {
+        kt = kw - kBK;
+        continue;
+      }
+    }
     // does any row of the tile keep a key of this tile?
     const bool sink_tile = kt < a.S;
     const bool win_tile = kt + kBK - 1 >= i_min - a.W + 1;
@@ -824,13 +835,15 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
                          (int)AttnSmem<128>::kBytes);
     cudaFuncSetAttribute(attn_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)AttnSmem<64>::kBytes);
+    cudaFuncSetAttribute(select_rows_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDynSmem);
+    cudaFuncSetAttribute(select_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDynSmem);
     s_attr[dev] = true;
   }
   if (sh.R > 0) {
     const dim3 gs((T + kSelRows - 1) / kSelRows, sh.B * sh.NR);
     trace_begin(RTP_STAGE_PREFILL_INDEX, st);
-    if (sh.D == 128) select_rows_kernel<128><<<gs, kSelRows * 32, 0, st>>>(a);
-    else select_rows_kernel<64><<<gs, kSelRows * 32, 0, st>>>(a);
+    if (sh.D == 128) select_rows_kernel<128><<<gs, kSelRows * 32, kSelDynSmem, st>>>(a);
+    else select_rows_kernel<64><<<gs, kSelRows * 32, kSelDynSmem, st>>>(a);
     trace_end(RTP_STAGE_PREFILL_INDEX, st);
   }
   const dim3 ga((T + kBQ - 1) / kBQ, sh.B * sh.Hq);
