@@ -587,7 +587,8 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
 template <int D>
 struct AttnSmem {
   static constexpr int kStride = D + 8;  // bf16 elements per shared row (pad: no ldmatrix conflicts)
-  static constexpr size_t kBytes = (size_t)(kBQ + 2 * kBK) * kStride * sizeof(__nv_bfloat16);
+  // Q tile, then two buffers of (K tile, V tile)
+  static constexpr size_t kBytes = (size_t)(kBQ + 4 * kBK) * kStride * sizeof(__nv_bfloat16);
 };
 
 template <int D>
@@ -597,8 +598,7 @@ __global__ void __launch_bounds__(128) attn_rows_kernel(PrefillArgs a) {
   constexpr int NO = D / 8;   // n8 tiles of the output
   extern __shared__ __align__(16) unsigned char smem[];
   __nv_bfloat16* s_q = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* s_k = s_q + kBQ * ST;
-  __nv_bfloat16* s_v = s_k + kBK * ST;
+  __nv_bfloat16* s_kv = s_q + kBQ * ST;  // buffer u: K at s_kv + 2u kBK ST, V right after
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
   const int bq = blockIdx.y;
@@ -663,45 +663,71 @@ __global__ void __launch_bounds__(128) attn_rows_kernel(PrefillArgs a) {
   const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
   const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
 
-  for (int kt = 0; kt <= i_max; kt += kBK) {
-    if (r < 0 && kt >= a.S) {  // local head: jump from the sinks to the first window tile
-      const int kw = (max(0, i_min - a.W + 1) / kBK) * kBK;
-      if (kt < kw) {
-        kt = kw - kBK;
-        continue;
-      }
+  // Key tiles in order, local heads jumping from the sinks to the first window
+  // tile; each tile's K, V (cp.async, rows past the chunk zero-filled) and
+  // mask words are requested one tile ahead.
+  auto next_tile = [&](int kt_) {
+    int n = kt_ + kBK;
+    if (r < 0 && n >= a.S) n = max(n, (max(0, i_min - a.W + 1) / kBK) * kBK);
+    return n;
+  };
+  auto issue_kv = [&](int kt_, int u) {
+    const unsigned dk = (unsigned)__cvta_generic_to_shared(s_kv + (size_t)(2 * u) * kBK * ST);
+    const unsigned dv = (unsigned)__cvta_generic_to_shared(s_kv + (size_t)(2 * u + 1) * kBK * ST);
+    for (int e = threadIdx.x; e < kBK * (D / 8); e += blockDim.x) {
+      const int kr = e / (D / 8), c8 = e % (D / 8);
+      const int j = kt_ + kr;
+      const unsigned sz = j <= i_max ? 16u : 0u;  // 0: zero fill
+      const int jj = j <= i_max ? j : 0;
+      const unsigned off = (unsigned)((kr * ST + c8 * 8) * sizeof(__nv_bfloat16));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dk + off),
+                   "l"(kg + (size_t)jj * D + c8 * 8), "r"(sz));
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dv + off),
+                   "l"(vg + (size_t)jj * D + c8 * 8), "r"(sz));
     }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  };
+  auto load_mw = [&](int kt_, unsigned (&m_)[2][2]) {
+#pragma unroll
+    for (int x = 0; x < 2; ++x)
+#pragma unroll
+      for (int y = 0; y < 2; ++y) {
+        const int wd = (kt_ >> 5) + y;
+        m_[x][y] = (r >= 0 && rv[x] && wd * 32 <= pi[x]) ? __ldg(mrow[x] + wd) : 0u;
+      }
+  };
+  unsigned mw[2][2];
+  load_mw(0, mw);
+  issue_kv(0, 0);
+  int ub = 0;
+  for (int kt = 0; kt <= i_max; ub ^= 1) {
+    const int kn = next_tile(kt);
+    unsigned mwn[2][2];
+    if (kn <= i_max) {
+      issue_kv(kn, ub ^ 1);
+      load_mw(kn, mwn);
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+    } else {
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+    }
+    const __nv_bfloat16* s_k = s_kv + (size_t)(2 * ub) * kBK * ST;
+    const __nv_bfloat16* s_v = s_k + kBK * ST;
     // does any row of the tile keep a key of this tile?
     const bool sink_tile = kt < a.S;
     const bool win_tile = kt + kBK - 1 >= i_min - a.W + 1;
-    unsigned mw[2][2] = {{0u, 0u}, {0u, 0u}};
     bool any = false;
-    if (r >= 0) {
 #pragma unroll
-      for (int x = 0; x < 2; ++x) {
-        if (!rv[x]) continue;
+    for (int x = 0; x < 2; ++x)
 #pragma unroll
-        for (int y = 0; y < 2; ++y) {
-          const int wd = (kt >> 5) + y;
-          if (wd * 32 <= pi[x]) mw[x][y] = __ldg(mrow[x] + wd);
-          any |= mw[x][y] != 0u;
-        }
-      }
+      for (int y = 0; y < 2; ++y) any |= mw[x][y] != 0u;
+    if (!__syncthreads_or(any || sink_tile || win_tile)) {  // also: tile kt's K, V visible
+      kt = kn;
+#pragma unroll
+      for (int x = 0; x < 2; ++x)
+#pragma unroll
+        for (int y = 0; y < 2; ++y) mw[x][y] = mwn[x][y];
+      continue;
     }
-    if (!__syncthreads_or(any || sink_tile || win_tile)) continue;
-    // stage K and V tiles
-    for (int e = threadIdx.x; e < kBK * (D / 8); e += blockDim.x) {
-      const int kr = e / (D / 8), c8 = e % (D / 8);
-      const int j = kt + kr;
-      uint4 kv = make_uint4(0u, 0u, 0u, 0u), vv = make_uint4(0u, 0u, 0u, 0u);
-      if (j <= i_max) {
-        kv = __ldg(reinterpret_cast<const uint4*>(kg + (size_t)j * D) + c8);
-        vv = __ldg(reinterpret_cast<const uint4*>(vg + (size_t)j * D) + c8);
-      }
-      *reinterpret_cast<uint4*>(s_k + kr * ST + c8 * 8) = kv;
-      *reinterpret_cast<uint4*>(s_v + kr * ST + c8 * 8) = vv;
-    }
-    __syncthreads();
     // S = Q K^T for this warp's 16 rows x 64 keys
     float sc[kBK / 8][4];
 #pragma unroll
@@ -775,7 +801,12 @@ __global__ void __launch_bounds__(128) attn_rows_kernel(PrefillArgs a) {
         mma_bf16(o[n], pa0, pa1, pa2, pa3, b0, b1);
       }
     }
-    __syncthreads();
+    __syncthreads();  // this buffer is free for the tile after next
+    kt = kn;
+#pragma unroll
+    for (int x = 0; x < 2; ++x)
+#pragma unroll
+      for (int y = 0; y < 2; ++y) mw[x][y] = mwn[x][y];
   }
   // ---- epilogue ----
 #pragma unroll
