@@ -542,15 +542,17 @@ def prefill_pairs(sh, bm: torch.Tensor, start: int, T: int) -> int:
     return B * sh.n_q_heads * sw_rows + extra
 
 
-def prefill_extra(dev, reps: int) -> dict:
-    """ms per 32K causal prefill chunk (rtp_prefill_attn) and the attention
-    kernel's tensor-pipe roofline."""
+def prefill_extra(dev, reps: int, T: int = 0) -> dict:
+    """ms per causal prefill chunk of the 32K prefill workload (T tokens,
+    default the workload's 32768; rtp_prefill_attn) and the attention kernel's
+    tensor-pipe roofline."""
     import head_wise_sparse_local_b200 as rtp
     from synth import make_prefill_inputs, workload
     w = workload("prefill_32k_bf16")
-    inp = make_prefill_inputs(w)
+    T = int(T or w["ctx"])
+    inp = make_prefill_inputs(w, T=T)
     sh = inp["shape"]
-    B, T, Hq, D = sh.batch, int(w["ctx"]), sh.n_q_heads, sh.head_dim
+    B, Hq, D = sh.batch, sh.n_q_heads, sh.head_dim
     lay = rtp.Layer(sh, inp["max_ctx"], device=dev, prefill_T=T)
     w_q, w_k = inp["w_q"].to(dev), inp["w_k"].to(dev)
     start = torch.zeros(B, dtype=torch.int32, device=dev)
@@ -598,7 +600,7 @@ def prefill_extra(dev, reps: int) -> dict:
                          "peak": peak, "peak_source": "measured" if "bf16_tflops" in peaks else "fallback",
                          "unit": "TFLOP/s", "frac": round(att_tf / peak, 4),
                          "note": "mma.sync m16n8k16 bf16 path (legacy tensor-core instructions)"},
-            "data": "inputs larger than L2 (q 268 MB)"}
+            "data": f"T = {T}; q alone {B * T * Hq * D * 2 / 1e6:.0f} MB" + (" (larger than L2)" if B * T * Hq * D * 2 > l2_bytes() else "")}
 
 
 # ---------------------------------------------------------------------------
@@ -655,6 +657,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true", help="skip the 1M decode and 32K prefill lines")
     ap.add_argument("--extra-steps", type=int, default=1000)
+    ap.add_argument("--prefill-only", action="store_true",
+                    help="time only the prefill chunk (profiling); prints its JSON object")
+    ap.add_argument("--prefill-T", type=int, default=0, help="prefill chunk length (default 32768)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -681,6 +686,12 @@ def main():
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         dist.close()
+        return
+
+    if args.prefill_only:
+        torch.cuda.set_device(0)
+        res = prefill_extra(torch.device("cuda", 0), 3, args.prefill_T)
+        print(json.dumps({"prefill": res, "T": args.prefill_T or 32768}), flush=True)
         return
 
     dist = Dist("nccl")
