@@ -54,6 +54,7 @@ constexpr int kBruteMax = kSelThreads;  // exact solve by pairwise ranks up to t
 constexpr int kGroup = 4;           // kept rows a warp attends per memory round trip
 constexpr int kPos = kLgCap / kSelThreads;  // positions a select thread owns per staged chunk
 constexpr int kTopPerWarp = 16;     // top-rung items a warp hands the leader in the first pass
+static_assert(kTopPerWarp <= 32, "the tail gives each top-rung item of a warp its own lane");
 constexpr int kSpec = 2;            // of those, rows whose keys and values a warp stages early
 
 // Tokens per score CTA: eight (bf16) or four (fp32) 16-d keys per thread.
@@ -82,6 +83,7 @@ struct DecodeArgs {
   int* rank_cnt;    // [B][NR][kMaxCS] kept tokens per select CTA
   uint2* cand;      // [B][NR][lstride] boundary-bucket candidates past kCandSmem
   int n_ctl, nch_score_max, n_sw_tiles, n_parts_max, n_score_ctas, n_sw_ctas, sel_cs;
+  int want_mask;    // 1: the caller asked for the top-p bitmask
   int ret_head[kMaxRetrieval];
   int ret_rank[kMaxRetrieval];
   double inv_freq[64];  // RoPE frequencies, k < D/2
@@ -967,6 +969,8 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   __shared__ uint2 s_small[32];
   __shared__ __align__(16) T s_spec[kSelWarps][kSpec][2][D];  // early-staged K, V rows per warp
   __shared__ int s_spec_j[kSelWarps][kSpec];
+  __shared__ uint2 s_top[kSelWarps][kTopPerWarp];  // this CTA's top-rung items per warp (key, index)
+  __shared__ int s_wtop[kSelWarps];
   __shared__ __align__(16) float s_qh[D];
   __shared__ __align__(16) float s_wo[kSelWarps * D];
   __shared__ float s_wml[kSelWarps * 2];
@@ -1021,6 +1025,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   const bool keep_all = a.top_p >= 1.0f;
   float tau = -CUDART_INF_F;
   int jcut = INT_MAX;
+  bool via_top = false;  // the tail reads only the top-rung items (tier 1, no bitmask)
 
   if (__builtin_expect(!keep_all, 1)) {  // uniform over the grid
     // maximum score (per-chunk maxima of the score kernel)
@@ -1089,8 +1094,11 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
               const int src = __ffs(bal) - 1;
               bal &= bal - 1u;
               const int j = c0 + u * kSelThreads + warp * 32 + src;
-              if (lane == src && wtop < (unsigned)kTopPerWarp)
-                region[wtop] = make_uint2(score_key(s_lg[j - c0]), (unsigned)j);
+              if (lane == src && wtop < (unsigned)kTopPerWarp) {
+                const uint2 item = make_uint2(score_key(s_lg[j - c0]), (unsigned)j);
+                region[wtop] = item;
+                s_top[warp][wtop] = item;
+              }
               if (wtop < (unsigned)kSpec && cached) {
                 // the warp's first rows: keys and values into shared memory
                 constexpr int NC = D * (int)sizeof(T) / 16;  // 16-byte chunks per row
@@ -1129,6 +1137,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
 #pragma unroll
         for (int k = 0; k < kRungs; ++k) { sh->wpre_m[warp][1 + k] = ms[k]; sh->wpre_c[warp][k] = cs[k]; }
         sh->wpre_c[warp][kRungs] = wtop > (unsigned)kTopPerWarp ? 1u : 0u;
+        s_wtop[warp] = (int)min(wtop, (unsigned)kTopPerWarp);
         lead->wcnt[rank * kSelWarps + warp] = wtop;
       }
       __syncthreads();
@@ -1179,6 +1188,9 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
     // scores hold it and fit (one more pass collects them); else the histogram
     const bool tier1 = Mk[kRungs - 1] >= target && sh->tot_c[kRungs] == 0u;  // no region overflowed
     const bool tier2 = !tier1 && kf >= 0 && Ck[kf] <= (unsigned)kCandSmem;
+    // tau is one of the top-rung scores under tier 1, so every kept token is a
+    // top-rung item: without a bitmask to write, the tail tests only those
+    via_top = tier1 && !a.want_mask;
     float t_lo = m_lo;
 #pragma unroll
     for (int k = 0; k < kRungs; ++k)
@@ -1499,37 +1511,8 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   float am = -CUDART_INF_F, al = 0.f, ao[DL];
 #pragma unroll
   for (int d = 0; d < DL; ++d) ao[d] = 0.f;
-  int cnt = 0;
-  for (int c0 = j0; c0 < j1; c0 += kLgCap) {
-    const int c1 = min(j1, c0 + kLgCap);
-    if (!cached) {
-      __syncthreads();
-      stage(c0, c1);
-    }
-    __syncthreads();  // staged scores visible; the row lists' bytes are free
-    unsigned inbits = 0u, outbits = 0u;
-#pragma unroll 4
-    for (int u = 0; u < kPos; ++u) {
-      const int j = c0 + u * kSelThreads + tid;
-      if (j < c1) {
-        const float sv = s_lg[j - c0];
-        if (keep_all || sv > tau || (sv == tau && j <= jcut)) {
-          inbits |= 1u << u;
-          if (j >= s_cnt && j < sw0) outbits |= 1u << u;
-        }
-      }
-    }
-    cnt += __popc(inbits);
-    int wn = 0;
-#pragma unroll 2
-    for (int u = 0; u < kPos; ++u) {
-      const unsigned word = __ballot_sync(0xffffffffu, (inbits >> u) & 1u);
-      const int jw = c0 + u * kSelThreads + warp * 32;
-      if (lane == 0 && jw < c1) mask[jw >> 5] = word;
-      const unsigned ob = __ballot_sync(0xffffffffu, (outbits >> u) & 1u);
-      if ((outbits >> u) & 1u) wrows[wn + __popc(ob & ((1u << lane) - 1u))] = jw + lane;
-      wn += __popc(ob);
-    }
+  // this warp attends its rows wrows[0, wn) (wn warp-uniform) for query head g
+  auto attend_rows = [&](int wn) {
     asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's early copies
     __syncwarp();
     const int sj0 = s_spec_j[warp][0], sj1 = s_spec_j[warp][1];
@@ -1584,6 +1567,58 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         for (int d = 0; d < DL; ++d) ao[d] = fmaf(e, to_f32(vt[d]), ao[d]);
       }
       am = mn;
+    }
+  };
+  int cnt = 0;
+  if (via_top) {
+    // this warp's top-rung items (one per lane at most) are its only candidates
+    const int nt = s_wtop[warp];
+    bool in = false, o = false;
+    int jj = 0;
+    if (lane < nt) {
+      const uint2 e = s_top[warp][lane];
+      const float sv = key_score(e.x);
+      jj = (int)e.y;
+      in = sv > tau || (sv == tau && jj <= jcut);
+      o = in && jj >= s_cnt && jj < sw0;
+    }
+    cnt = in ? 1 : 0;
+    const unsigned ob = __ballot_sync(0xffffffffu, o);
+    if (o) wrows[__popc(ob & ((1u << lane) - 1u))] = jj;
+    __syncwarp();
+    attend_rows(__popc(ob));
+  } else {
+    for (int c0 = j0; c0 < j1; c0 += kLgCap) {
+      const int c1 = min(j1, c0 + kLgCap);
+      if (!cached) {
+        __syncthreads();
+        stage(c0, c1);
+      }
+      __syncthreads();  // staged scores visible; the row lists' bytes are free
+      unsigned inbits = 0u, outbits = 0u;
+#pragma unroll 4
+      for (int u = 0; u < kPos; ++u) {
+        const int j = c0 + u * kSelThreads + tid;
+        if (j < c1) {
+          const float sv = s_lg[j - c0];
+          if (keep_all || sv > tau || (sv == tau && j <= jcut)) {
+            inbits |= 1u << u;
+            if (j >= s_cnt && j < sw0) outbits |= 1u << u;
+          }
+        }
+      }
+      cnt += __popc(inbits);
+      int wn = 0;
+#pragma unroll 2
+      for (int u = 0; u < kPos; ++u) {
+        const unsigned word = __ballot_sync(0xffffffffu, (inbits >> u) & 1u);
+        const int jw = c0 + u * kSelThreads + warp * 32;
+        if (lane == 0 && jw < c1) mask[jw >> 5] = word;
+        const unsigned ob = __ballot_sync(0xffffffffu, (outbits >> u) & 1u);
+        if ((outbits >> u) & 1u) wrows[wn + __popc(ob & ((1u << lane) - 1u))] = jw + lane;
+        wn += __popc(ob);
+      }
+      attend_rows(wn);
     }
   }
   // merge the warps' states into this CTA's partial for query head g
@@ -1750,6 +1785,7 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   a.logits = reinterpret_cast<float*>(w + lay.logits);
   a.cmax = reinterpret_cast<float*>(w + lay.cmax);
   a.mask = sel_bitmask ? sel_bitmask : reinterpret_cast<uint32_t*>(w + lay.mask);
+  a.want_mask = sel_bitmask != nullptr;
   a.ctl = reinterpret_cast<unsigned*>(w + lay.ctl);
   a.rank_cnt = reinterpret_cast<int*>(w + lay.rank_cnt);
   a.cand = reinterpret_cast<uint2*>(w + lay.cand);

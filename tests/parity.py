@@ -63,10 +63,11 @@ def oracle_cache_from_inputs(inp) -> OracleCache:
     return c
 
 
-def run_gpu_decode(inp, top_p=None, append_last_separately=True):
+def run_gpu_decode(inp, top_p=None, append_last_separately=True, with_bitmask=True):
     """Fill a device cache with the context, append the decode token, decode.
 
-    Returns dict(out [B,Hq,D] float64 numpy, bitmask, count, status, layer)."""
+    Returns dict(out [B,Hq,D] float64 numpy, bitmask, count, status, layer);
+    with_bitmask=False passes no bitmask (bitmask None in the result)."""
     from head_wise_sparse_local_b200 import Layer
     sh = inp["shape"]
     if top_p is not None:
@@ -95,6 +96,8 @@ def run_gpu_decode(inp, top_p=None, append_last_separately=True):
     NR = sh.n_retrieval * sh.group
     bm = torch.zeros((sh.batch, max(NR, 1), words), dtype=torch.int32, device=dev)
     cnt = torch.full((sh.batch, max(NR, 1)), -1, dtype=torch.int32, device=dev)
+    if not with_bitmask:
+        bm = None
     lay.decode(q, seq, w_q, out, max_seq_len=int(inp["seq_len"].max()), sel_bitmask=bm, sel_count=cnt)
     torch.cuda.synchronize()
     return dict(out=out.double().cpu().numpy(), bitmask=bm, count=cnt.cpu().numpy(),

@@ -197,3 +197,38 @@ def test_decode_many_needles_second_tier():
     inp = _small(ctx=20000, needles=10000)
     st = check_decode_parity(inp, top_p=0.9)
     assert st["exact"] >= st["heads"] - 1
+
+
+@pytest.mark.parametrize("case", ["needles_p03", "needles_p09", "needles_p0999", "flat", "ragged",
+                                  "many_needles", "full_128k", "full_1m"])
+def test_decode_without_bitmask_matches(case):
+    """Without a bitmask to write, a selection settled over the top-rung items
+    reads only those items in its tail. The kept counts must equal those of the
+    call that writes the bitmask; so must the output, bitwise where each CTA's
+    scores fit in shared memory (the kept rows are then attended in the same
+    groups), within the bf16 tolerance at 1M (grouped per staged chunk there)."""
+    p = None
+    if case.startswith("needles"):
+        inp = _small(ctx=5000, needles=16)
+        p = {"needles_p03": 0.3, "needles_p09": 0.9, "needles_p0999": 0.999}[case]
+    elif case == "flat":
+        inp, p = _small(ctx=20000, needles=0), 0.8
+    elif case == "ragged":
+        w = workload("ragged_decode_b8_8k_32k_bf16", shape_batch=5, ctx=(1, 9000), needles=4)
+        inp = make_decode_inputs(w, max_ctx=9100)
+        inp["seq_len"] = np.array([1, 37, 2100, 2113, 9000], dtype=np.int32)
+    elif case == "many_needles":
+        inp, p = _small(ctx=20000, needles=10000), 0.9
+    elif case == "full_128k":
+        inp = make_decode_inputs(workload("decode_128k_bf16"))
+    else:
+        inp = make_decode_inputs(workload("decode_1m_bf16"))
+    a = run_gpu_decode(inp, top_p=p)
+    b = run_gpu_decode(inp, top_p=p, with_bitmask=False)
+    assert a["status"] == 0 and b["status"] == 0
+    assert np.array_equal(a["count"], b["count"])
+    if case != "full_1m":
+        assert np.array_equal(a["out"], b["out"])
+    else:
+        atol, rtol = TOL["bf16"]
+        assert np.all(np.abs(a["out"] - b["out"]) <= atol + rtol * np.abs(a["out"]))
