@@ -143,7 +143,7 @@ struct RowSel {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __grid_constant__ PrefillArgs a) {
   // dynamic shared memory: double-buffered key tiles, then this tile's scores
   // of the CTA's rows
   extern __shared__ __align__(16) unsigned char sel_dsm[];
@@ -152,6 +152,10 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
   __shared__ float s_qi[kSelRows][kIdxDim];
   __shared__ uint2 s_cand[kSelRows][kCand];
   __shared__ unsigned long long s_cw[kSelRows][kCand];
+  // Each row's selection state lives in shared memory: a pass loads only the
+  // few fields its op tests into registers, and the step between passes works
+  // on a copy, which keeps the per-key loops' registers free of it.
+  __shared__ RowSel s_rs[kSelRows];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int b = bh / a.NR, hh = bh % a.NR;
@@ -199,7 +203,14 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
 #pragma unroll
     for (int o = 0; o < kIdxDim; ++o) qi[o] = __shfl_sync(0xffffffffu, part[o >> 3], (o & 7) * 4);
   }
-  if (lane < kIdxDim) s_qi[warp][lane] = qi[lane];
+  {
+    // lane l < 16 stores q~[l] (constant register indices only)
+    float mine = 0.f;
+#pragma unroll
+    for (int o = 0; o < kIdxDim; ++o)
+      if (lane == o) mine = qi[o];
+    if (lane < kIdxDim) s_qi[warp][lane] = mine;
+  }
   __syncthreads();
   // Scores on tensor cores: S = K~ Q~^T with K = 16, q~ split into bf16 hi and
   // lo parts (the products are exact; fp32 accumulation), so the score is the
@@ -221,10 +232,13 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
     bl1 = pack_bf16(lo[2], lo[3]);
   }
 
-  RowSel rs;
-  rs.op = row_ok ? kOpMax : kOpDone;
-  rs.m = -CUDART_INF_F;
-  rs.first = false;
+  if (lane == 0) {
+    s_rs[warp].op = row_ok ? kOpMax : kOpDone;
+    s_rs[warp].m = -CUDART_INF_F;
+    s_rs[warp].first = false;
+  }
+  __syncwarp();
+  const RowSel& R = s_rs[warp];
   const __nv_bfloat16* kidx = static_cast<const __nv_bfloat16*>(a.kidx) + ((size_t)b * a.R + r) * a.Lmax * kIdxDim;
   uint32_t* mrow = a.mask + (((size_t)b * a.NR + hh) * a.T + (row_ok ? t : 0)) * a.words;
 
@@ -236,7 +250,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
   unsigned long long zsum;
 
   for (int pass = 0; pass < 200; ++pass) {
-    const int op = rs.op;
+    const int op = R.op;
     // reset accumulators
 #pragma unroll
     for (int q = 0; q < 8; ++q) { pm[q] = 0ull; pc[q] = 0u; }
@@ -246,7 +260,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
     n_cand = 0u;
     tie_cnt = 0u;
     zsum = 0ull;
-    const bool first_split = (op == kOpSplit) && rs.first;
+    const bool first_split = (op == kOpSplit) && R.first;
     // key tiles [kt, kt + kKeyTile) up to i_last, copied asynchronously one
     // tile ahead of their use
     auto stage_async = [&](int kt_, int buf) {
@@ -295,69 +309,97 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
           break;
         }
         case kOpEmit: {
+          const float tau = R.tau;
+          const int jcut = R.jcut;
 #pragma unroll 8
           for (int u = 0; u < kKeyTile / 32; ++u) {
             if (u >= ulim) break;
             const int j = kt + u * 32 + lane;
             const float sv = srow[u * 32 + lane];
-            const bool in = j <= i && (sv > rs.tau || (sv == rs.tau && j <= rs.jcut));
+            const bool in = j <= i && (sv > tau || (sv == tau && j <= jcut));
             const unsigned wd = __ballot_sync(0xffffffffu, in);
             if (lane == 0) mrow[(kt >> 5) + u] = wd;
           }
           break;
         }
         case kOpSplit: {
+          const float m = R.m;
           if (first_split) {  // every key is inside: total mass and d-thresholds
+            float th[7];
+#pragma unroll
+            for (int e = 0; e < 7; ++e) th[e] = R.th[e];
 #pragma unroll 4
             for (int u = 0; u < kKeyTile / 32; ++u) {
               const int j = kt + u * 32 + lane;
               if (u >= ulim || j > i) continue;
               const float sv = srow[u * 32 + lane];
-              const float d = rs.m - sv;
-              const unsigned long long w = mass36(sv, rs.m);
+              const float d = m - sv;
+              const unsigned long long w = mass36(sv, m);
               zsum += w;
               pm[7] += w;
               pc[7] += 1u;
 #pragma unroll
               for (int e = 0; e < 7; ++e)
-                if (d >= rs.th[e]) { pm[e] += w; pc[e] += 1u; }
+                if (d >= th[e]) { pm[e] += w; pc[e] += 1u; }
             }
           } else {
             // cumulative sums: pm[e] / pc[e] (e < 7) gather what lies past
             // threshold e, pm[7] / pc[7] everything inside
+            const float dlo = R.dlo, dhi = R.dhi;
+            const unsigned klo = R.klo, khi = R.khi;
+            if (!R.by_key) {
+              float th[7];
+#pragma unroll
+              for (int e = 0; e < 7; ++e) th[e] = R.th[e];
 #pragma unroll 4
-            for (int u = 0; u < kKeyTile / 32; ++u) {
-              const int j = kt + u * 32 + lane;
-              if (u >= ulim || j > i) continue;
-              const float sv = srow[u * 32 + lane];
-              const float d = rs.m - sv;
-              const unsigned key = score_key(sv);
-              if (!(d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi)) continue;
-              const unsigned long long w = mass36(sv, rs.m);
-              pm[7] += w;
-              pc[7] += 1u;
-              if (!rs.by_key) {
+              for (int u = 0; u < kKeyTile / 32; ++u) {
+                const int j = kt + u * 32 + lane;
+                if (u >= ulim || j > i) continue;
+                const float sv = srow[u * 32 + lane];
+                const float d = m - sv;
+                const unsigned key = score_key(sv);
+                if (!(d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi)) continue;
+                const unsigned long long w = mass36(sv, m);
+                pm[7] += w;
+                pc[7] += 1u;
 #pragma unroll
                 for (int e = 0; e < 7; ++e)
-                  if (d >= rs.th[e]) { pm[e] += w; pc[e] += 1u; }
-              } else {
+                  if (d >= th[e]) { pm[e] += w; pc[e] += 1u; }
+              }
+            } else {
+              unsigned kth[7];
+#pragma unroll
+              for (int e = 0; e < 7; ++e) kth[e] = R.kth[e];
+#pragma unroll 4
+              for (int u = 0; u < kKeyTile / 32; ++u) {
+                const int j = kt + u * 32 + lane;
+                if (u >= ulim || j > i) continue;
+                const float sv = srow[u * 32 + lane];
+                const float d = m - sv;
+                const unsigned key = score_key(sv);
+                if (!(d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi)) continue;
+                const unsigned long long w = mass36(sv, m);
+                pm[7] += w;
+                pc[7] += 1u;
 #pragma unroll
                 for (int e = 0; e < 7; ++e)
-                  if (key < rs.kth[e]) { pm[e] += w; pc[e] += 1u; }
+                  if (key < kth[e]) { pm[e] += w; pc[e] += 1u; }
               }
             }
           }
           break;
         }
         case kOpRange: {
+          const float m = R.m, dlo = R.dlo, dhi = R.dhi;
+          const unsigned klo = R.klo, khi = R.khi;
 #pragma unroll 4
           for (int u = 0; u < kKeyTile / 32; ++u) {
             const int j = kt + u * 32 + lane;
             if (u >= ulim || j > i) continue;
             const float sv = srow[u * 32 + lane];
-            const float d = rs.m - sv;
+            const float d = m - sv;
             const unsigned key = score_key(sv);
-            if (d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi) {
+            if (d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi) {
               kmn = min(kmn, key);
               kmx = max(kmx, key);
             }
@@ -365,29 +407,32 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
           break;
         }
         case kOpTies: {
+          const unsigned tie_key = R.tie_key, tie_hi = R.tie_hi;
 #pragma unroll 4
           for (int u = 0; u < kKeyTile / 32; ++u) {
             const int j = kt + u * 32 + lane;
             if (u >= ulim || j > i) continue;
             const unsigned key = score_key(srow[u * 32 + lane]);
-            if (key == rs.tie_key && (unsigned)j <= rs.tie_hi) tie_cnt += 1u;
+            if (key == tie_key && (unsigned)j <= tie_hi) tie_cnt += 1u;
           }
           break;
         }
         case kOpCand: {
+          const float m = R.m, dlo = R.dlo, dhi = R.dhi;
+          const unsigned klo = R.klo, khi = R.khi;
 #pragma unroll 2
           for (int u = 0; u < kKeyTile / 32; ++u) {
             if (u >= ulim) break;
             const int j = kt + u * 32 + lane;
             const float sv = srow[u * 32 + lane];
-            const float d = rs.m - sv;
+            const float d = m - sv;
             const unsigned key = score_key(sv);
-            const bool inside = j <= i && d >= rs.dlo && (rs.dhi < 0.f || d < rs.dhi) && key >= rs.klo && key <= rs.khi;
+            const bool inside = j <= i && d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi;
             const unsigned bal = __ballot_sync(0xffffffffu, inside);
             const unsigned slot = n_cand + __popc(bal & ((1u << lane) - 1u));
             if (inside && slot < (unsigned)kCand) {
               s_cand[warp][slot] = make_uint2(key, (unsigned)j);
-              s_cw[warp][slot] = mass36(sv, rs.m);
+              s_cw[warp][slot] = mass36(sv, m);
             }
             n_cand += __popc(bal);
           }
@@ -398,6 +443,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
       }
     }
     // ---- reduce this pass and choose the next step (warp-uniform) ----
+    RowSel rs = R;
     if (op == kOpDone) {
       // nothing
     } else if (op == kOpMax) {
@@ -443,28 +489,39 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
         rs.cnt_in = (unsigned)(i + 1);
         rs.first = false;
       }
-      // sub-intervals are ordered from the highest scores (e = 0) down
+      // sub-intervals are ordered from the highest scores (e = 0) down; the
+      // first one that reaches the mass still needed holds the boundary.
+      // (Constant indices only, so that these arrays stay in registers.)
       unsigned long long cum = 0ull;
-      unsigned cc = 0u;
+      unsigned cc = 0u, pc_sel = pc[7];
       int sel = 7;
+      bool found = false;
+#pragma unroll
       for (int e = 0; e < 8; ++e) {
-        if (cum + pm[e] >= rs.need) { sel = e; break; }
-        cum += pm[e];
-        cc += pc[e];
+        if (!found && cum + pm[e] >= rs.need) { sel = e; found = true; pc_sel = pc[e]; }
+        if (!found) { cum += pm[e]; cc += pc[e]; }
       }
       rs.need -= cum;
       rs.cnt_above += cc;
       const unsigned before = rs.cnt_in;
-      rs.cnt_in = pc[sel];
+      rs.cnt_in = pc_sel;
       if (!rs.by_key) {
-        const float lo = sel == 0 ? rs.dlo : rs.th[sel - 1];
-        const float hi = sel == 7 ? rs.dhi : rs.th[sel];
+        float lo = rs.dlo, hi = rs.dhi;
+#pragma unroll
+        for (int e = 0; e < 7; ++e) {
+          if (e == sel - 1) lo = rs.th[e];
+          if (e == sel) hi = rs.th[e];
+        }
         rs.dlo = lo;
         rs.dhi = hi;
       } else {
         // key sub-intervals: e = 0 holds the highest keys
-        const unsigned hi = sel == 0 ? rs.khi : rs.kth[sel - 1] - 1u;
-        const unsigned lo = sel == 7 ? rs.klo : rs.kth[sel];
+        unsigned hi = rs.khi, lo = rs.klo;
+#pragma unroll
+        for (int e = 0; e < 7; ++e) {
+          if (e == sel - 1) hi = rs.kth[e] - 1u;
+          if (e == sel) lo = rs.kth[e];
+        }
         rs.klo = lo;
         rs.khi = hi;
       }
@@ -577,6 +634,9 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(PrefillAr
       }
       rs.op = kOpDone;
     }
+    __syncwarp();
+    if (lane == 0) s_rs[warp] = rs;
+    __syncwarp();
     if (!__syncthreads_or(rs.op != kOpDone)) break;
   }
 }
