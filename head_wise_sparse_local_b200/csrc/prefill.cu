@@ -29,7 +29,8 @@ namespace {
 
 constexpr int kSelRows = 8;       // query rows (warps) per selection CTA
 constexpr int kKeyTile = 512;     // indexer keys staged per step
-constexpr size_t kSelDynSmem = 2 * kKeyTile * kIdxDim * sizeof(__nv_bfloat16) + kSelRows * (kKeyTile + 4) * sizeof(float);
+constexpr int kKeyStages = 4;     // key tiles in flight: the one in use and three ahead
+constexpr size_t kSelDynSmem = kKeyStages * kKeyTile * kIdxDim * sizeof(__nv_bfloat16) + kSelRows * (kKeyTile + 4) * sizeof(float);
 constexpr int kCand = 160;        // tokens the exact solve takes per row
 constexpr int kBQ = 64;           // attention: query rows per CTA (16 per warp)
 constexpr int kBK = 64;           // attention: keys per tile
@@ -60,6 +61,11 @@ __device__ __forceinline__ unsigned long long wsum64(unsigned long long v) {
   return v;
 }
 __device__ __forceinline__ unsigned wsum32(unsigned v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+__device__ __forceinline__ float wsumf(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
@@ -114,9 +120,10 @@ enum : int {
   kOpMax = 0,    // row maximum
   kOpSplit = 1,  // mass/count of the 8 sub-intervals of the current interval
   kOpRange = 2,  // min/max order key inside the current interval
-  kOpCand = 3,   // collect the current interval's tokens for the exact solve
+  kOpCand = 3,   // collect the current interval's tokens for the exact solve; write the bitmask
   kOpTies = 4,   // count tied tokens with index <= probe (index bisection)
-  kOpEmit = 5,   // write the top-p bitmask
+  kOpEmit = 5,   // write the top-p bitmask (after exact ties or p >= 1; the
+                 // candidate pass writes it itself)
   kOpDone = 6
 };
 
@@ -144,11 +151,11 @@ struct RowSel {
 
 template <int D>
 __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __grid_constant__ PrefillArgs a) {
-  // dynamic shared memory: double-buffered key tiles, then this tile's scores
-  // of the CTA's rows
+  // dynamic shared memory: a ring of key tiles, then this tile's scores of
+  // the CTA's rows
   extern __shared__ __align__(16) unsigned char sel_dsm[];
   auto s_k = reinterpret_cast<__nv_bfloat16 (*)[kKeyTile * kIdxDim]>(sel_dsm);
-  auto s_sc = reinterpret_cast<float (*)[kKeyTile + 4]>(sel_dsm + 2 * kKeyTile * kIdxDim * sizeof(__nv_bfloat16));
+  auto s_sc = reinterpret_cast<float (*)[kKeyTile + 4]>(sel_dsm + kKeyStages * kKeyTile * kIdxDim * sizeof(__nv_bfloat16));
   __shared__ float s_qi[kSelRows][kIdxDim];
   __shared__ uint2 s_cand[kSelRows][kCand];
   __shared__ unsigned long long s_cw[kSelRows][kCand];
@@ -156,6 +163,8 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
   // few fields its op tests into registers, and the step between passes works
   // on a copy, which keeps the per-key loops' registers free of it.
   __shared__ RowSel s_rs[kSelRows];
+  // later splits: the scores inside the interval, gathered 32 at a time
+  __shared__ float s_ring[kSelRows][64];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bh = blockIdx.y;
   const int b = bh / a.NR, hh = bh % a.NR;
@@ -233,6 +242,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
   }
 
   if (lane == 0) {
+    s_rs[warp] = RowSel{};
     s_rs[warp].op = row_ok ? kOpMax : kOpDone;
     s_rs[warp].m = -CUDART_INF_F;
     s_rs[warp].first = false;
@@ -245,7 +255,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
   // pass accumulators
   unsigned long long pm[8];
   unsigned pc[8];
-  float fmx;
+  float fmx, fs, fs2;
   unsigned kmn, kmx, n_cand, tie_cnt;
   unsigned long long zsum;
 
@@ -255,29 +265,60 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
 #pragma unroll
     for (int q = 0; q < 8; ++q) { pm[q] = 0ull; pc[q] = 0u; }
     fmx = -CUDART_INF_F;
+    fs = 0.f;
+    fs2 = 0.f;
     kmn = 0xffffffffu;
     kmx = 0u;
     n_cand = 0u;
     tie_cnt = 0u;
     zsum = 0ull;
     const bool first_split = (op == kOpSplit) && R.first;
-    // key tiles [kt, kt + kKeyTile) up to i_last, copied asynchronously one
-    // tile ahead of their use
+    // the interval and the split edges, for the ops that test them
+    const float m = R.m, dlo = R.dlo, dhi = R.dhi;
+    const unsigned klo = R.klo, khi = R.khi;
+    const bool by_key = R.by_key;
+    float thr[7];  // split edges: d thresholds, or order keys (as bits) when by_key
+#pragma unroll
+    for (int e = 0; e < 7; ++e) thr[e] = by_key ? __uint_as_float(R.kth[e]) : R.th[e];
+    // one score inside the interval of a later split: its mass into the
+    // cumulative sums (pm[e] / pc[e], e < 7: past edge e; [7]: everything)
+    auto split_item = [&](float sv) {
+      const float d = m - sv;
+      const unsigned key = score_key(sv);
+      const unsigned long long w = mass36(sv, m);
+      pm[7] += w;
+      pc[7] += 1u;
+      if (!by_key) {
+#pragma unroll
+        for (int e = 0; e < 7; ++e)
+          if (d >= thr[e]) { pm[e] += w; pc[e] += 1u; }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 7; ++e)
+          if (key < __float_as_uint(thr[e])) { pm[e] += w; pc[e] += 1u; }
+      }
+    };
+    unsigned q_head = 0u, q_tail = 0u;  // s_ring[warp] positions (warp-uniform)
+    // key tiles [kt, kt + kKeyTile) up to i_last, copied asynchronously
+    // kKeyStages - 1 tiles ahead of their use (an empty group past the end)
     auto stage_async = [&](int kt_, int buf) {
-      const int n = min(kKeyTile, i_last + 1 - kt_);
-      const char* src = reinterpret_cast<const char*>(kidx + (size_t)kt_ * kIdxDim);
-      const unsigned dst = (unsigned)__cvta_generic_to_shared(s_k[buf]);
-      for (int v = threadIdx.x; v < n * 2; v += kSelRows * 32)
-        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst + 16u * v), "l"(src + 16 * (size_t)v));
+      if (kt_ <= i_last) {
+        const int n = min(kKeyTile, i_last + 1 - kt_);
+        const char* src = reinterpret_cast<const char*>(kidx + (size_t)kt_ * kIdxDim);
+        const unsigned dst = (unsigned)__cvta_generic_to_shared(s_k[buf]);
+        for (int v = threadIdx.x; v < n * 2; v += kSelRows * 32)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst + 16u * v), "l"(src + 16 * (size_t)v));
+      }
       asm volatile("cp.async.commit_group;" ::: "memory");
     };
-    __syncthreads();  // the previous pass is done with both buffers
-    stage_async(0, 0);
+    __syncthreads();  // the previous pass is done with every buffer
+#pragma unroll
+    for (int s0 = 0; s0 < kKeyStages - 1; ++s0) stage_async(s0 * kKeyTile, s0);
     int buf = 0;
-    for (int kt = 0; kt <= i_last; kt += kKeyTile, buf ^= 1) {
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      __syncthreads();  // tile kt landed for every thread; the other buffer is free
-      if (kt + kKeyTile <= i_last) stage_async(kt + kKeyTile, buf ^ 1);
+    for (int kt = 0; kt <= i_last; kt += kKeyTile) {
+      asm volatile("cp.async.wait_group %0;" :: "n"(kKeyStages - 2) : "memory");
+      __syncthreads();  // tile kt landed for every thread; the previous tile's buffer is free
+      stage_async(kt + (kKeyStages - 1) * kKeyTile, buf == 0 ? kKeyStages - 1 : buf - 1);
       // warp w: the scores of keys [64 w, 64 w + 64) of this tile for all rows
 #pragma unroll
       for (int half = 0; half < kKeyTile / kSelRows / 16; ++half) {
@@ -294,6 +335,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
         s_sc[row0 + 1][key0 + 8] = c[3] * kIdxScale + 0.0f;
       }
       __syncthreads();
+      buf = buf + 1 == kKeyStages ? 0 : buf + 1;  // the next tile's buffer
       if (op == kOpDone || kt > i) continue;  // uniform per warp
       // One tight loop per kind of pass over this tile's 16 groups of 32 keys
       // (the row's op is warp-uniform).  Keys past the row (j > i) are off.
@@ -304,7 +346,12 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
 #pragma unroll 8
           for (int u = 0; u < kKeyTile / 32; ++u) {
             const int j = kt + u * 32 + lane;
-            if (u < ulim && j <= i) fmx = fmaxf(fmx, srow[u * 32 + lane]);
+            if (u < ulim && j <= i) {
+              const float sv = srow[u * 32 + lane];
+              fmx = fmaxf(fmx, sv);
+              fs += sv;
+              fs2 = fmaf(sv, sv, fs2);
+            }
           }
           break;
         }
@@ -323,11 +370,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
           break;
         }
         case kOpSplit: {
-          const float m = R.m;
           if (first_split) {  // every key is inside: total mass and d-thresholds
-            float th[7];
-#pragma unroll
-            for (int e = 0; e < 7; ++e) th[e] = R.th[e];
 #pragma unroll 4
             for (int u = 0; u < kKeyTile / 32; ++u) {
               const int j = kt + u * 32 + lane;
@@ -340,58 +383,36 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
               pc[7] += 1u;
 #pragma unroll
               for (int e = 0; e < 7; ++e)
-                if (d >= th[e]) { pm[e] += w; pc[e] += 1u; }
+                if (d >= thr[e]) { pm[e] += w; pc[e] += 1u; }
             }
           } else {
-            // cumulative sums: pm[e] / pc[e] (e < 7) gather what lies past
-            // threshold e, pm[7] / pc[7] everything inside
-            const float dlo = R.dlo, dhi = R.dhi;
-            const unsigned klo = R.klo, khi = R.khi;
-            if (!R.by_key) {
-              float th[7];
-#pragma unroll
-              for (int e = 0; e < 7; ++e) th[e] = R.th[e];
+            // a small share of the keys lies inside: gather those scores in
+            // the warp's ring and add them 32 at a time (no divergent lanes)
+            float* ring = s_ring[warp];
 #pragma unroll 4
-              for (int u = 0; u < kKeyTile / 32; ++u) {
-                const int j = kt + u * 32 + lane;
-                if (u >= ulim || j > i) continue;
-                const float sv = srow[u * 32 + lane];
-                const float d = m - sv;
-                const unsigned key = score_key(sv);
-                if (!(d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi)) continue;
-                const unsigned long long w = mass36(sv, m);
-                pm[7] += w;
-                pc[7] += 1u;
-#pragma unroll
-                for (int e = 0; e < 7; ++e)
-                  if (d >= th[e]) { pm[e] += w; pc[e] += 1u; }
-              }
-            } else {
-              unsigned kth[7];
-#pragma unroll
-              for (int e = 0; e < 7; ++e) kth[e] = R.kth[e];
-#pragma unroll 4
-              for (int u = 0; u < kKeyTile / 32; ++u) {
-                const int j = kt + u * 32 + lane;
-                if (u >= ulim || j > i) continue;
-                const float sv = srow[u * 32 + lane];
-                const float d = m - sv;
-                const unsigned key = score_key(sv);
-                if (!(d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi)) continue;
-                const unsigned long long w = mass36(sv, m);
-                pm[7] += w;
-                pc[7] += 1u;
-#pragma unroll
-                for (int e = 0; e < 7; ++e)
-                  if (key < kth[e]) { pm[e] += w; pc[e] += 1u; }
+            for (int u = 0; u < kKeyTile / 32; ++u) {
+              if (u >= ulim) break;
+              const int j = kt + u * 32 + lane;
+              const float sv = srow[u * 32 + lane];
+              const float d = m - sv;
+              const unsigned key = score_key(sv);
+              const bool inside = j <= i && d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi;
+              const unsigned bal = __ballot_sync(0xffffffffu, inside);
+              if (bal == 0u) continue;
+              if (inside) ring[(q_tail + __popc(bal & ((1u << lane) - 1u))) & 63u] = sv;
+              q_tail += (unsigned)__popc(bal);
+              if (q_tail - q_head >= 32u) {
+                __syncwarp();
+                const float sq = ring[(q_head + lane) & 63u];
+                __syncwarp();
+                q_head += 32u;
+                split_item(sq);
               }
             }
           }
           break;
         }
         case kOpRange: {
-          const float m = R.m, dlo = R.dlo, dhi = R.dhi;
-          const unsigned klo = R.klo, khi = R.khi;
 #pragma unroll 4
           for (int u = 0; u < kKeyTile / 32; ++u) {
             const int j = kt + u * 32 + lane;
@@ -418,8 +439,6 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
           break;
         }
         case kOpCand: {
-          const float m = R.m, dlo = R.dlo, dhi = R.dhi;
-          const unsigned klo = R.klo, khi = R.khi;
 #pragma unroll 2
           for (int u = 0; u < kKeyTile / 32; ++u) {
             if (u >= ulim) break;
@@ -427,7 +446,12 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
             const float sv = srow[u * 32 + lane];
             const float d = m - sv;
             const unsigned key = score_key(sv);
-            const bool inside = j <= i && d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi;
+            const bool below_hi = dhi < 0.f || d < dhi;
+            const bool inside = j <= i && d >= dlo && below_hi && key >= klo && key <= khi;
+            // ordered before every candidate: kept whatever the solve finds
+            const bool above = j <= i && (d < dlo || (below_hi && key > khi));
+            const unsigned wd = __ballot_sync(0xffffffffu, above);
+            if (lane == 0) mrow[(kt >> 5) + u] = wd;
             const unsigned bal = __ballot_sync(0xffffffffu, inside);
             const unsigned slot = n_cand + __popc(bal & ((1u << lane) - 1u));
             if (inside && slot < (unsigned)kCand) {
@@ -441,6 +465,10 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
         default:
           break;
       }
+    }
+    if (op == kOpSplit && !first_split && q_tail != q_head) {  // the ring's last (< 32) scores
+      __syncwarp();
+      if (lane < q_tail - q_head) split_item(s_ring[warp][(q_head + lane) & 63u]);
     }
     // ---- reduce this pass and choose the next step (warp-uniform) ----
     RowSel rs = R;
@@ -457,10 +485,24 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
       rs.first = true;
       rs.cnt_above = 0u;
       rs.need = 0ull;
-      // first split: fixed d edges (scores within 0.5, 1, 2, 3, 4.5, 7, 12 of the max)
-      const float edges[7] = {0.5f, 1.f, 2.f, 3.f, 4.5f, 7.f, 12.f};
+      // First split: edges around a guess of the boundary's distance below the
+      // max. For scores ~ N(mu, sd^2) the softmax-weighted scores are
+      // ~ N(mu + sd^2, sd^2), whose upper p-quantile lies z_p sd below
+      // mu + sd^2. Large scores beyond the bulk move the boundary towards the
+      // max, hence the wider bins on that side. The guess only places the
+      // edges: the split stays exact wherever the boundary falls.
+      {
+        const float n = (float)(i + 1);
+        const float mu = __shfl_sync(0xffffffffu, wsumf(fs), 0) / n;
+        const float var = fmaxf(__shfl_sync(0xffffffffu, wsumf(fs2), 0) / n - mu * mu, 0.f);
+        const float sd = sqrtf(var);
+        const float c = rs.m - (mu + var - normcdfinvf(a.top_p) * sd);
+        const float off[7] = {-0.8f, -0.4f, -0.2f, -0.08f, 0.f, 0.08f, 0.25f};
+        const float fixed[7] = {0.5f, 1.f, 2.f, 3.f, 4.5f, 7.f, 12.f};
+        const bool ok = isfinite(c) && isfinite(sd);
 #pragma unroll
-      for (int e = 0; e < 7; ++e) rs.th[e] = edges[e];
+        for (int e = 0; e < 7; ++e) rs.th[e] = ok ? c + off[e] * sd : fixed[e];
+      }
       if (a.top_p >= 1.0f) {  // keep everything
         rs.tau = -CUDART_INF_F;
         rs.jcut = INT_MAX;
@@ -620,11 +662,22 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) jc = max(jc, __shfl_xor_sync(0xffffffffu, jc, o));
+      // the pass wrote the bitmask words with the tokens above the interval;
+      // add the kept candidates
+      for (int c = lane; c < n; c += 32) {
+        const uint2 me = s_cand[warp][c];
+        if (me.x > tkey || (me.x == tkey && (int)me.y <= jc)) atomicOr(&mrow[me.y >> 5], 1u << (me.y & 31u));
+      }
       __syncwarp();
       rs.tau = key_score(tkey);
       rs.jcut = jc;
       rs.count = rs.cnt_above + kept_n;
-      rs.op = kOpEmit;
+      if (lane == 0) {
+        if (a.sel_tau) a.sel_tau[((size_t)b * a.NR + hh) * a.T + t] = rs.tau;
+        if (a.sel_jcut) a.sel_jcut[((size_t)b * a.NR + hh) * a.T + t] = rs.jcut;
+        if (a.sel_count) a.sel_count[((size_t)b * a.NR + hh) * a.T + t] = (int)rs.count;
+      }
+      rs.op = kOpDone;
     } else if (op == kOpEmit) {
       // last word(s) past i inside the row stay as written (bits > i are zero)
       if (lane == 0) {

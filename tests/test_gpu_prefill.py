@@ -31,6 +31,13 @@ def test_prefill_chunk_after_context():
     check_prefill_parity(inp)
 
 
+def test_prefill_rows_longer_than_the_key_ring():
+    # rows of 3000-3200 keys: 6-7 key tiles of 512, more than the tiles in flight
+    inp = _inp(T=200, start=3000, n_sink=8, window=100, top_p=0.9, needles=12)
+    st = check_prefill_parity(inp)
+    assert st["exact"] >= st["heads"] - 2
+
+
 def test_prefill_p1_is_dense_causal():
     inp = _inp(T=300, n_sink=4, window=50, top_p=1.0)
     st = check_prefill_parity(inp)
@@ -95,3 +102,48 @@ def test_prefill_single_row_and_tiny_p():
     inp = _inp(T=300, start=100, n_sink=4, window=16, top_p=1e-6)
     st = check_prefill_parity(inp)
     assert np.all(st["g"]["count"] == 1)
+
+
+@pytest.mark.parametrize("p", [0.5, 0.77])
+def test_prefill_all_scores_equal(p):
+    """Every indexer key of the retrieval heads identical: each row's scores
+    are all tied, so the selection resolves the cut by index alone (the tie
+    passes); row t keeps its first ceil(p (t + 1)) tokens."""
+    inp = _inp(T=300, n_sink=4, window=16, top_p=p, needles=0)
+    sh = inp["shape"]
+    for h in sh.retrieval:
+        inp["k_pre"][0, :, h] = inp["k_pre"][0, 0, h]
+    g = run_gpu_prefill(inp)
+    assert g["status"] == 0
+    bm = g["bitmask"].cpu().numpy().view(np.uint32)
+    pf = float(np.float32(p))
+    for t in [0, 1, 2, 31, 32, 100, 299]:
+        want = int(np.ceil(pf * (t + 1)))
+        for rg in range(sh.n_retrieval * sh.group):
+            bits = np.unpackbits(bm[0, rg, t].view(np.uint8), bitorder="little")[: t + 1]
+            assert np.array_equal(np.nonzero(bits)[0], np.arange(want)), (t, rg, int(bits.sum()), want)
+            assert g["count"][0, rg, t] == want
+    check_prefill_parity(inp, rows=[0, 5, 77, 299], g=g)
+
+
+def test_prefill_tied_block_keeps_lowest_indices():
+    """A block of identical indexer keys at a needle's key: for rows where the
+    block holds the cut, the kept part of the block is its lowest indices."""
+    inp = _inp(T=900, n_sink=4, window=32, top_p=0.6, needles=8)
+    sh = inp["shape"]
+    h = sh.retrieval[0]
+    src = int(inp["needles"][0][0][0])
+    inp["k_pre"][0, 300:600, h] = inp["k_pre"][0, src, h]
+    g = run_gpu_prefill(inp)
+    assert g["status"] == 0
+    bm = g["bitmask"].cpu().numpy().view(np.uint32)
+    n_cut = 0
+    for t in range(600, 900, 7):
+        for gg in range(sh.group):
+            bits = np.unpackbits(bm[0, gg, t].view(np.uint8), bitorder="little")[: t + 1]
+            kept = np.nonzero(bits[300:600])[0]
+            if 0 < len(kept) < 300:
+                n_cut += 1
+                assert np.array_equal(kept, np.arange(len(kept))), (t, gg, kept[:8])
+    check_prefill_parity(inp, rows=list(range(600, 900, 37)), g=g)
+    assert n_cut > 0
