@@ -29,7 +29,7 @@ namespace {
 
 constexpr int kSelRows = 8;       // query rows (warps) per selection CTA
 constexpr int kKeyTile = 512;     // indexer keys staged per step
-constexpr int kKeyStages = 4;     // key tiles in flight: the one in use and three ahead
+constexpr int kKeyStages = 2;     // key tiles in flight: the one in use and one ahead
 constexpr size_t kSelDynSmem = kKeyStages * kKeyTile * kIdxDim * sizeof(__nv_bfloat16) + kSelRows * (kKeyTile + 4) * sizeof(float);
 constexpr int kCand = 160;        // tokens the exact solve takes per row
 constexpr int kBQ = 64;           // attention: query rows per CTA (16 per warp)
@@ -150,7 +150,7 @@ struct RowSel {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __grid_constant__ PrefillArgs a) {
+__global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __grid_constant__ PrefillArgs a) {
   // dynamic shared memory: a ring of key tiles, then this tile's scores of
   // the CTA's rows
   extern __shared__ __align__(16) unsigned char sel_dsm[];
@@ -700,18 +700,20 @@ __global__ void __launch_bounds__(kSelRows * 32, 2) select_rows_kernel(const __g
 template <int D>
 struct AttnSmem {
   static constexpr int kStride = D + 8;  // bf16 elements per shared row (pad: no ldmatrix conflicts)
-  // Q tile, then two buffers of (K tile, V tile)
-  static constexpr size_t kBytes = (size_t)(kBQ + 4 * kBK) * kStride * sizeof(__nv_bfloat16);
+  // two buffers of (K tile, V tile); the Q tile borrows the first K tile
+  // until its fragments are in registers
+  static_assert(kBQ <= kBK, "the Q tile fits in one K tile");
+  static constexpr size_t kBytes = (size_t)(4 * kBK) * kStride * sizeof(__nv_bfloat16);
 };
 
 template <int D>
-__global__ void __launch_bounds__(128) attn_rows_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(128, 3) attn_rows_kernel(PrefillArgs a) {
   constexpr int ST = AttnSmem<D>::kStride;
   constexpr int KS = D / 16;  // k-steps of Q K^T
   constexpr int NO = D / 8;   // n8 tiles of the output
   extern __shared__ __align__(16) unsigned char smem[];
   __nv_bfloat16* s_q = reinterpret_cast<__nv_bfloat16*>(smem);
-  __nv_bfloat16* s_kv = s_q + kBQ * ST;  // buffer u: K at s_kv + 2u kBK ST, V right after
+  __nv_bfloat16* s_kv = s_q;  // buffer u: K at s_kv + 2u kBK ST, V right after
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
   const int bq = blockIdx.y;
@@ -811,6 +813,7 @@ __global__ void __launch_bounds__(128) attn_rows_kernel(PrefillArgs a) {
   };
   unsigned mw[2][2];
   load_mw(0, mw);
+  __syncthreads();  // every warp holds its Q fragments: the first K tile may overwrite them
   issue_kv(0, 0);
   int ub = 0;
   for (int kt = 0; kt <= i_max; ub ^= 1) {
