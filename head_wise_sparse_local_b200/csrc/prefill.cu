@@ -149,6 +149,45 @@ struct RowSel {
   int op;
 };
 
+// The edges and interval a split pass tests, loaded from the row's state.
+struct SplitView {
+  float m, dlo, dhi;
+  unsigned klo, khi;
+  bool by_key;
+  float thr[7];  // d thresholds, or order keys (as bits) when by_key
+};
+__device__ __forceinline__ SplitView load_split(const RowSel& R) {
+  SplitView v;
+  v.m = R.m;
+  v.dlo = R.dlo;
+  v.dhi = R.dhi;
+  v.klo = R.klo;
+  v.khi = R.khi;
+  v.by_key = R.by_key;
+#pragma unroll
+  for (int e = 0; e < 7; ++e) v.thr[e] = v.by_key ? __uint_as_float(R.kth[e]) : R.th[e];
+  return v;
+}
+// One score inside the interval of a later split: its mass into the cumulative
+// sums (pm[e] / pc[e], e < 7: past edge e; [7]: everything inside).
+__device__ __forceinline__ void split_item(const SplitView& v, float sv, unsigned long long (&pm)[8],
+                                           unsigned (&pc)[8]) {
+  const float d = v.m - sv;
+  const unsigned key = score_key(sv);
+  const unsigned long long w = mass36(sv, v.m);
+  pm[7] += w;
+  pc[7] += 1u;
+  if (!v.by_key) {
+#pragma unroll
+    for (int e = 0; e < 7; ++e)
+      if (d >= v.thr[e]) { pm[e] += w; pc[e] += 1u; }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 7; ++e)
+      if (key < __float_as_uint(v.thr[e])) { pm[e] += w; pc[e] += 1u; }
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __grid_constant__ PrefillArgs a) {
   // dynamic shared memory: a ring of key tiles, then this tile's scores of
@@ -255,49 +294,20 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
   // pass accumulators
   unsigned long long pm[8];
   unsigned pc[8];
-  float fmx, fs, fs2;
-  unsigned kmn, kmx, n_cand, tie_cnt;
-  unsigned long long zsum;
+  // the small accumulators of the other ops share three registers:
+  //   max: x0 = max score, x1 = sum of s, x2 = sum of s^2 (float bits)
+  //   range: x0 = min key, x1 = max key; candidates: x0 = count; ties: x0 = count
+  unsigned x0, x1, x2;
 
   for (int pass = 0; pass < 200; ++pass) {
     const int op = R.op;
     // reset accumulators
 #pragma unroll
     for (int q = 0; q < 8; ++q) { pm[q] = 0ull; pc[q] = 0u; }
-    fmx = -CUDART_INF_F;
-    fs = 0.f;
-    fs2 = 0.f;
-    kmn = 0xffffffffu;
-    kmx = 0u;
-    n_cand = 0u;
-    tie_cnt = 0u;
-    zsum = 0ull;
+    x0 = op == kOpMax ? __float_as_uint(-CUDART_INF_F) : (op == kOpRange ? 0xffffffffu : 0u);
+    x1 = 0u;  // also 0.f
+    x2 = 0u;
     const bool first_split = (op == kOpSplit) && R.first;
-    // the interval and the split edges, for the ops that test them
-    const float m = R.m, dlo = R.dlo, dhi = R.dhi;
-    const unsigned klo = R.klo, khi = R.khi;
-    const bool by_key = R.by_key;
-    float thr[7];  // split edges: d thresholds, or order keys (as bits) when by_key
-#pragma unroll
-    for (int e = 0; e < 7; ++e) thr[e] = by_key ? __uint_as_float(R.kth[e]) : R.th[e];
-    // one score inside the interval of a later split: its mass into the
-    // cumulative sums (pm[e] / pc[e], e < 7: past edge e; [7]: everything)
-    auto split_item = [&](float sv) {
-      const float d = m - sv;
-      const unsigned key = score_key(sv);
-      const unsigned long long w = mass36(sv, m);
-      pm[7] += w;
-      pc[7] += 1u;
-      if (!by_key) {
-#pragma unroll
-        for (int e = 0; e < 7; ++e)
-          if (d >= thr[e]) { pm[e] += w; pc[e] += 1u; }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 7; ++e)
-          if (key < __float_as_uint(thr[e])) { pm[e] += w; pc[e] += 1u; }
-      }
-    };
     unsigned q_head = 0u, q_tail = 0u;  // s_ring[warp] positions (warp-uniform)
     // key tiles [kt, kt + kKeyTile) up to i_last, copied asynchronously
     // kKeyStages - 1 tiles ahead of their use (an empty group past the end)
@@ -343,6 +353,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
       const int ulim = min(kKeyTile / 32, (i - kt) / 32 + 1);  // groups holding keys <= i
       switch (op) {
         case kOpMax: {
+          float fmx = __uint_as_float(x0), fs = __uint_as_float(x1), fs2 = __uint_as_float(x2);
 #pragma unroll 8
           for (int u = 0; u < kKeyTile / 32; ++u) {
             const int j = kt + u * 32 + lane;
@@ -353,6 +364,9 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
               fs2 = fmaf(sv, sv, fs2);
             }
           }
+          x0 = __float_as_uint(fmx);
+          x1 = __float_as_uint(fs);
+          x2 = __float_as_uint(fs2);
           break;
         }
         case kOpEmit: {
@@ -370,6 +384,8 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
           break;
         }
         case kOpSplit: {
+          const SplitView v = load_split(R);
+          const float m = v.m;
           if (first_split) {  // every key is inside: total mass and d-thresholds
 #pragma unroll 4
             for (int u = 0; u < kKeyTile / 32; ++u) {
@@ -378,12 +394,11 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
               const float sv = srow[u * 32 + lane];
               const float d = m - sv;
               const unsigned long long w = mass36(sv, m);
-              zsum += w;
-              pm[7] += w;
+              pm[7] += w;  // every key: the total mass
               pc[7] += 1u;
 #pragma unroll
               for (int e = 0; e < 7; ++e)
-                if (d >= thr[e]) { pm[e] += w; pc[e] += 1u; }
+                if (d >= v.thr[e]) { pm[e] += w; pc[e] += 1u; }
             }
           } else {
             // a small share of the keys lies inside: gather those scores in
@@ -396,7 +411,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
               const float sv = srow[u * 32 + lane];
               const float d = m - sv;
               const unsigned key = score_key(sv);
-              const bool inside = j <= i && d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi;
+              const bool inside = j <= i && d >= v.dlo && (v.dhi < 0.f || d < v.dhi) && key >= v.klo && key <= v.khi;
               const unsigned bal = __ballot_sync(0xffffffffu, inside);
               if (bal == 0u) continue;
               if (inside) ring[(q_tail + __popc(bal & ((1u << lane) - 1u))) & 63u] = sv;
@@ -406,13 +421,15 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
                 const float sq = ring[(q_head + lane) & 63u];
                 __syncwarp();
                 q_head += 32u;
-                split_item(sq);
+                split_item(v, sq, pm, pc);
               }
             }
           }
           break;
         }
         case kOpRange: {
+          const float m = R.m, dlo = R.dlo, dhi = R.dhi;
+          const unsigned klo = R.klo, khi = R.khi;
 #pragma unroll 4
           for (int u = 0; u < kKeyTile / 32; ++u) {
             const int j = kt + u * 32 + lane;
@@ -421,8 +438,8 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
             const float d = m - sv;
             const unsigned key = score_key(sv);
             if (d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi) {
-              kmn = min(kmn, key);
-              kmx = max(kmx, key);
+              x0 = min(x0, key);
+              x1 = max(x1, key);
             }
           }
           break;
@@ -434,11 +451,13 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
             const int j = kt + u * 32 + lane;
             if (u >= ulim || j > i) continue;
             const unsigned key = score_key(srow[u * 32 + lane]);
-            if (key == tie_key && (unsigned)j <= tie_hi) tie_cnt += 1u;
+            if (key == tie_key && (unsigned)j <= tie_hi) x0 += 1u;
           }
           break;
         }
         case kOpCand: {
+          const float m = R.m, dlo = R.dlo, dhi = R.dhi;
+          const unsigned klo = R.klo, khi = R.khi;
 #pragma unroll 2
           for (int u = 0; u < kKeyTile / 32; ++u) {
             if (u >= ulim) break;
@@ -453,12 +472,12 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
             const unsigned wd = __ballot_sync(0xffffffffu, above);
             if (lane == 0) mrow[(kt >> 5) + u] = wd;
             const unsigned bal = __ballot_sync(0xffffffffu, inside);
-            const unsigned slot = n_cand + __popc(bal & ((1u << lane) - 1u));
+            const unsigned slot = x0 + __popc(bal & ((1u << lane) - 1u));
             if (inside && slot < (unsigned)kCand) {
               s_cand[warp][slot] = make_uint2(key, (unsigned)j);
               s_cw[warp][slot] = mass36(sv, m);
             }
-            n_cand += __popc(bal);
+            x0 += __popc(bal);
           }
           break;
         }
@@ -468,14 +487,14 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
     }
     if (op == kOpSplit && !first_split && q_tail != q_head) {  // the ring's last (< 32) scores
       __syncwarp();
-      if (lane < q_tail - q_head) split_item(s_ring[warp][(q_head + lane) & 63u]);
+      if (lane < q_tail - q_head) split_item(load_split(R), s_ring[warp][(q_head + lane) & 63u], pm, pc);
     }
     // ---- reduce this pass and choose the next step (warp-uniform) ----
     RowSel rs = R;
     if (op == kOpDone) {
       // nothing
     } else if (op == kOpMax) {
-      rs.m = wmaxf(fmx);
+      rs.m = wmaxf(__uint_as_float(x0));
       rs.op = kOpSplit;
       rs.dlo = 0.f;
       rs.dhi = -1.f;
@@ -493,8 +512,8 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
       // edges: the split stays exact wherever the boundary falls.
       {
         const float n = (float)(i + 1);
-        const float mu = __shfl_sync(0xffffffffu, wsumf(fs), 0) / n;
-        const float var = fmaxf(__shfl_sync(0xffffffffu, wsumf(fs2), 0) / n - mu * mu, 0.f);
+        const float mu = __shfl_sync(0xffffffffu, wsumf(__uint_as_float(x1)), 0) / n;
+        const float var = fmaxf(__shfl_sync(0xffffffffu, wsumf(__uint_as_float(x2)), 0) / n - mu * mu, 0.f);
         const float sd = sqrtf(var);
         const float c = rs.m - (mu + var - normcdfinvf(a.top_p) * sd);
         const float off[7] = {-0.8f, -0.4f, -0.2f, -0.08f, 0.f, 0.08f, 0.25f};
@@ -512,6 +531,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
     } else if (op == kOpSplit) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) { pm[e] = wsum64(pm[e]); pc[e] = wsum32(pc[e]); }
+      const unsigned long long inside_mass = pm[7];  // first split: every key, Z
       {  // cumulative -> per sub-interval (e = 0 holds the highest scores)
         const unsigned long long tm = pm[7];
         const unsigned tc = pc[7];
@@ -523,7 +543,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
         pc[0] = tc - pc[0];
       }
       if (first_split) {
-        const unsigned long long Z = wsum64(zsum);
+        const unsigned long long Z = inside_mass;
         unsigned long long target = (unsigned long long)ceil((double)a.top_p * (double)Z);
         if (target > Z) target = Z;
         if (target < 1ull) target = 1ull;
@@ -584,10 +604,8 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
         }
       }
     } else if (op == kOpRange) {
-      kmn = wminu(kmn);
-      kmx = wmaxu(kmx);
-      rs.klo = max(rs.klo, kmn);
-      rs.khi = min(rs.khi, kmx);
+      rs.klo = max(rs.klo, wminu(x0));
+      rs.khi = min(rs.khi, wmaxu(x1));
       rs.by_key = true;
       if (rs.klo == rs.khi) {  // exact ties: keep the first ceil(need / w) by index
         const unsigned long long w = mass36(key_score(rs.klo), rs.m);
@@ -618,7 +636,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
       }
     } else if (op == kOpTies) {
       // bisection on the index: smallest probe with count(ties <= probe) >= need_ties
-      tie_cnt = wsum32(tie_cnt);
+      const unsigned tie_cnt = wsum32(x0);
       unsigned lo = rs.tie_lo, hi = rs.kth[0];
       if (tie_cnt >= rs.need_ties) hi = rs.tie_hi;
       else lo = rs.tie_hi + 1u;
@@ -632,7 +650,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
       }
     } else if (op == kOpCand) {
       // exact solve: candidate c is kept iff the mass ordered before it is < need
-      const int n = (int)min(n_cand, (unsigned)kCand);
+      const int n = (int)min(x0, (unsigned)kCand);
       unsigned kept_n = 0u, tkey = 0xffffffffu;
       __syncwarp();
       for (int c = lane; c < n; c += 32) {
