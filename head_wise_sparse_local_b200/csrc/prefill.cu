@@ -11,10 +11,12 @@
 //       The exact top-p threshold is found by splitting the score interval
 //       that contains the boundary 8 ways per pass, with the softmax mass
 //       exp(s - max) of every score in 2^-36 fixed point (mass36, shared with
-//       the decode path; exact integer sums
-//       in registers), until at most kCand tokens remain; a warp-level exact
-//       solve finishes (ties to the lower index).  The row's top-p set is
-//       written as a bitmask.
+//       the decode path; exact integer sums in registers), until at most
+//       kCand tokens remain; a warp-level exact solve finishes (ties to the
+//       lower index).  The first pass also takes the scores' mean and spread,
+//       and the first split's edges go around the boundary a Gaussian score
+//       model predicts (a guess that only places them).  The pass that
+//       collects the last candidates also writes the row's top-p bitmask.
 //   attn_rows_kernel  tensor-core (mma.sync m16n8k16 bf16, fp32 accumulate)
 //       flash attention over 64-row query tiles and 64-key tiles, masked by
 //       causality, sinks, the window and (retrieval heads) the bitmask; key
