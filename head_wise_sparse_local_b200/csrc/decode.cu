@@ -8,17 +8,23 @@
 //                  s_j = q~ . k~_j / 4 of the G query heads of a retrieval KV
 //                  head plus a per-chunk maximum.
 //   select_kernel  one thread-block cluster per (sequence, retrieval q head).
-//                  The softmax mass exp(s - max) of every score, in 2^-36
-//                  fixed point (integer sums: exact and order independent),
-//                  goes into a 2048-bucket histogram ordered by score; the
-//                  cluster merges it through distributed shared memory, finds
-//                  the bucket where the mass of the highest scores reaches
-//                  ceil(p * Z), gathers that bucket's scores in the leader CTA,
-//                  and the leader resolves the exact threshold score tau and,
-//                  for ties at tau, the last kept index j_cut.  Every CTA then
-//                  writes its share of the top-p bitmask and attends, for its
-//                  query head, the kept rows of its share that lie outside
-//                  the sinks and the window (one partial per CTA).
+//                  The softmax mass exp(s - max) of every score is taken in
+//                  2^-36 fixed point (integer sums: exact and order
+//                  independent).  One pass sums the total mass and the mass
+//                  and count at or above rungs 1, 2, 4 and 8 below the
+//                  maximum, and hands every score at or above the top rung to
+//                  the leader CTA through distributed shared memory.  When
+//                  those scores hold ceil(p * Z), the leader solves the exact
+//                  threshold score tau (and, for ties at tau, the last kept
+//                  index j_cut) over them.  Otherwise a lower rung's scores
+//                  are collected in one more pass, or a 2048-bucket mass
+//                  histogram finds the boundary bucket whose scores are
+//                  solved.  Every CTA then writes its share of the top-p
+//                  bitmask and attends, for its query head, the kept rows of
+//                  its share that lie outside the sinks and the window (one
+//                  partial per CTA).  With no bitmask asked for and the solve
+//                  over the top-rung scores, each warp tests only its own
+//                  top-rung items instead of its whole share.
 //   sw_kernel      exact attention over the sinks and the window of every KV
 //                  head.  It is launched after the select kernel and does not
 //                  wait for it until its own partial is written, so this HBM
