@@ -25,6 +25,7 @@ _lib = _abi.load()
 __all__ = ["Layer", "RtpError", "rtp_layer_cfg", "rtp_cache", "rtp_cache_bytes",
            "rtp_decode_workspace_bytes", "rtp_prefill_workspace_bytes", "rtp_append_kv",
            "rtp_decode_attn", "rtp_decode_attn_noalloc", "rtp_prefill_attn", "rtp_trace_stage",
+           "rtp_debug_wait_expiry",
            "rtp_last_error", "RTP_NOALLOC_SCRATCH_BYTES",
            "rtp_version", "make_cfg", "STAGES",
            "library_path", "EXPORTS", "RTP_BF16", "RTP_FP32", "RTP_DEV_SEQ_LEN",
@@ -59,12 +60,14 @@ def _stream(stream) -> Optional[int]:
 
 def make_cfg(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int, max_ctx: int,
              n_sink: int, window: int, top_p: float, retrieval: Sequence[int],
-             dtype: str = "bf16", rope_base: float = 10000.0, idx_dim: int = 16) -> rtp_layer_cfg:
+             dtype: str = "bf16", rope_base: float = 10000.0, idx_dim: int = 16,
+             local_cap: int = 0) -> rtp_layer_cfg:
     mask = 0
     for h in retrieval:
         mask |= 1 << int(h)
     return rtp_layer_cfg(batch, n_q_heads, n_kv_heads, head_dim, idx_dim, max_ctx, n_sink, window,
-                         top_p, rope_base, mask, RTP_BF16 if dtype == "bf16" else RTP_FP32)
+                         top_p, rope_base, mask, RTP_BF16 if dtype == "bf16" else RTP_FP32,
+                         int(local_cap))
 
 
 def rtp_version() -> str:
@@ -87,6 +90,11 @@ def rtp_trace_stage(stage, start_event=None, stop_event=None) -> None:
             ev.record()
         handles.append(ev.cuda_event)
     _abi.check(_lib.rtp_trace_stage(sid, handles[0], handles[1]))
+
+
+def rtp_debug_wait_expiry(polls: int) -> None:
+    """Arm the next rtp_decode_attn call on this thread to let its bounded waits expire."""
+    _abi.check(_lib.rtp_debug_wait_expiry(int(polls)))
 
 
 def rtp_cache_bytes(cfg: rtp_layer_cfg):
@@ -139,17 +147,28 @@ def rtp_prefill_attn(cfg, cache, q_pre, start_pos, T, w_q, out, sel_bitmask=None
 
 
 class Layer:
-    """One layer's configuration plus its device cache and scratch (torch-allocated)."""
+    """One layer's configuration plus its device cache and scratch (torch-allocated).
 
-    def __init__(self, shape, max_ctx: int, device="cuda", prefill_T: int = 0):
+    local_cap > 0 selects ring mode: local heads keep only their sinks and a
+    ring of local_cap window rows.  k and v are then flat [B, rows, D] buffers
+    (head_rows() gives each head's slice); otherwise [B, Hkv, max_ctx, D]."""
+
+    def __init__(self, shape, max_ctx: int, device="cuda", prefill_T: int = 0, local_cap: int = 0):
         self.shape = shape
         self.cfg = make_cfg(shape.batch, shape.n_q_heads, shape.n_kv_heads, shape.head_dim, max_ctx,
                             shape.n_sink, shape.window, shape.top_p, shape.retrieval, shape.dtype,
-                            shape.rope_base, shape.idx_dim)
+                            shape.rope_base, shape.idx_dim, local_cap)
         self.max_ctx = max_ctx
         dt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
         B, Hkv, D, R = shape.batch, shape.n_kv_heads, shape.head_dim, shape.n_retrieval
-        self.k = torch.empty((B, Hkv, max_ctx, D), dtype=dt, device=device)
+        es = 2 if shape.dtype == "bf16" else 4
+        k_bytes, _, _ = rtp_cache_bytes(self.cfg)
+        rows = k_bytes // (B * D * es)
+        self.ring = rows != Hkv * max_ctx
+        if self.ring:
+            self.k = torch.empty((B, rows, D), dtype=dt, device=device)
+        else:
+            self.k = torch.empty((B, Hkv, max_ctx, D), dtype=dt, device=device)
         self.v = torch.empty_like(self.k)
         self.kidx = torch.empty((B, max(R, 1), max_ctx, 16), dtype=dt, device=device)
         self.status = torch.zeros(1, dtype=torch.int32, device=device)

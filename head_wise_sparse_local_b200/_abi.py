@@ -27,11 +27,10 @@ STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_INVALID", 2: "RTP_ERR_SHAPE", 3: "RTP_E
 # Every entry point declared in include/rtp.h.
 EXPORTS = ("rtp_cache_bytes", "rtp_decode_workspace_bytes", "rtp_prefill_workspace_bytes",
            "rtp_append_kv", "rtp_decode_attn", "rtp_decode_attn_noalloc", "rtp_prefill_attn",
-           "rtp_trace_stage",
+           "rtp_trace_stage", "rtp_debug_wait_expiry",
            "rtp_last_error", "rtp_version")
 
-STAGES = {"append": 0, "decode_score": 1, "decode_select": 2, "decode_local": 3,
-          "prefill_index": 4, "prefill_attn": 5}
+STAGES = {"append": 0, "decode_stream": 1, "decode_select": 2, "prefill_index": 3, "prefill_attn": 4}
 
 
 class rtp_layer_cfg(ctypes.Structure):
@@ -39,7 +38,7 @@ class rtp_layer_cfg(ctypes.Structure):
                 ("head_dim", ctypes.c_int), ("idx_dim", ctypes.c_int), ("max_ctx", ctypes.c_int),
                 ("n_sink", ctypes.c_int), ("window", ctypes.c_int), ("top_p", ctypes.c_float),
                 ("rope_base", ctypes.c_float), ("retrieval_mask", ctypes.c_uint64),
-                ("dtype", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("local_cap", ctypes.c_int)]
 
 
 class rtp_cache(ctypes.Structure):
@@ -74,6 +73,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rtp_decode_attn.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp, sz, vp]
     lib.rtp_prefill_attn.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.rtp_trace_stage.argtypes = [i32, vp, vp]
+    lib.rtp_debug_wait_expiry.argtypes = [i32]
     lib.rtp_decode_attn_noalloc.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp]
     for name in EXPORTS:
         getattr(lib, name).restype = ctypes.c_char_p if name in ("rtp_last_error", "rtp_version") \

@@ -23,12 +23,13 @@ struct AppendArgs {
   void* v;
   void* kidx;
   int* status;
+  KvMap kv;
   int ret_rank[kMaxRetrieval];
   double inv_freq[64];
 };
 
 template <typename T, int D>
-__global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
+__global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendArgs a) {
   // The inputs (k_pre, v, start_pos, W_k) are read and the rotated key and the
   // indexer key formed before waiting for the previous kernel on the stream;
   // only the cache stores wait (a decode step still running may read the cache).
@@ -42,11 +43,17 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
   const int h = int(row % a.Hkv);
   const int t = int((row / a.Hkv) % a.T);
   const int b = int(row / ((long long)a.Hkv * a.T));
-  const int pos = a.start_pos[b] + t;
+  const int s0 = a.start_pos[b];
+  const int pos = s0 + t;
   if (pos < 0 || pos >= a.Lmax) {
     if (lane == 0) atomicOr(a.status, RTP_DEV_POSITION);
     return;
   }
+  // A local head in ring mode keeps the sinks and the last `ring` positions:
+  // an earlier position of this call whose slot a later one takes is skipped
+  // (two writes to one slot in one launch would race).
+  const bool ringed = (a.kv.ring_mask >> h) & 1ull;
+  if (ringed && pos >= a.kv.S && pos < s0 + a.T - a.kv.ring) return;
   const T* kp = static_cast<const T*>(a.k_pre) + row * D;
   const T* vp = static_cast<const T*>(a.v_in) + row * D;
   float x1[PP], x2[PP];
@@ -90,7 +97,7 @@ __global__ void __launch_bounds__(256) append_kernel(AppendArgs a) {
     }
   }
   griddep_wait();
-  const size_t dst = (((size_t)b * a.Hkv + h) * a.Lmax + pos) * D;
+  const size_t dst = a.kv.row(b, h, pos) * D;
   T* ko = static_cast<T*>(a.k) + dst;
   T* vo = static_cast<T*>(a.v) + dst;
 #pragma unroll
@@ -118,6 +125,7 @@ int launch_append(const Shape& sh, const rtp_cache* cache, const void* k_pre, co
   a.rope_base = sh.rope_base;
   a.k_pre = k_pre; a.v_in = v_in; a.start_pos = start_pos; a.w_k = w_k;
   a.k = cache->k; a.v = cache->v; a.kidx = cache->kidx; a.status = cache->status;
+  a.kv = sh.kv;
   for (int i = 0; i < kMaxRetrieval; ++i) a.ret_rank[i] = sh.ret_rank[i];
   for (int i = 0; i < 64; ++i) a.inv_freq[i] = sh.inv_freq[i];
   const long long rows = (long long)sh.B * T * sh.Hkv;

@@ -1,41 +1,50 @@
 // rtp_decode_attn: one decode step of the head-wise sparse attention layer.
 //
-// Three kernels on the caller's stream, chained with programmatic dependent
+// Two kernels on the caller's stream, chained with programmatic dependent
 // launch, scratch in the caller's workspace:
 //
-//   score_kernel   reads the 16-d indexer-key cache once (two 16-byte loads
-//                  per token for bf16) and writes the fp32 scores
-//                  s_j = q~ . k~_j / 4 of the G query heads of a retrieval KV
-//                  head plus a per-chunk maximum.
+//   stream_kernel  the two HBM streams of the step, side by side in one grid
+//                  that covers every SM, each CTA pulling its whole share into
+//                  shared memory with bulk asynchronous copies (TMA) that
+//                  complete on an mbarrier:
+//                  * score CTAs take a chunk of the 16-d indexer-key cache
+//                    (contiguous rows) and write the fp32 scores
+//                    s_j = q~ . k~_j / 4 of the G query heads of a retrieval
+//                    KV head plus a per-chunk maximum;
+//                  * sink/window clusters (one per sequence and KV head)
+//                    attend the sinks and the window of every KV head: a
+//                    half-warp per row, all G query heads per row, log-sum-exp
+//                    merged across the cluster through distributed shared
+//                    memory.  Local heads write their output here; retrieval
+//                    heads leave one partial per query head.
 //   select_kernel  one thread-block cluster per (sequence, retrieval q head).
-//                  The softmax mass exp(s - max) of every score is taken in
-//                  2^-36 fixed point (integer sums: exact and order
-//                  independent).  One pass sums the total mass and the mass
-//                  and count at or above rungs 1, 2, 4 and 8 below the
-//                  maximum, and hands every score at or above the top rung to
-//                  the leader CTA through distributed shared memory.  When
-//                  those scores hold ceil(p * Z), the leader solves the exact
-//                  threshold score tau (and, for ties at tau, the last kept
-//                  index j_cut) over them.  Otherwise a lower rung's scores
-//                  are collected in one more pass, or a 2048-bucket mass
-//                  histogram finds the boundary bucket whose scores are
-//                  solved.  Every CTA then writes its share of the top-p
-//                  bitmask and attends, for its query head, the kept rows of
-//                  its share that lie outside the sinks and the window (one
-//                  partial per CTA).  With no bitmask asked for and the solve
-//                  over the top-rung scores, each warp tests only its own
-//                  top-rung items instead of its whole share.
-//   sw_kernel      exact attention over the sinks and the window of every KV
-//                  head.  It is launched after the select kernel and does not
-//                  wait for it until its own partial is written, so this HBM
-//                  stream overlaps the selection; then the last CTA of each KV
-//                  head merges every partial of that head (log-sum-exp) into
-//                  the output.
+//                  It launches at once and prepares its query, then waits for
+//                  the stream kernel to complete.  The softmax mass
+//                  exp(s - max) of every score is taken in 2^-36 fixed point
+//                  (integer sums: exact and order independent).  One pass sums
+//                  the total mass and the mass and count at or above rungs 1,
+//                  2, 4 and 8 below the maximum, and hands every score at or
+//                  above the top rung to the leader CTA through distributed
+//                  shared memory.  When those scores hold ceil(p * Z), the
+//                  leader solves the exact threshold score tau (and, for ties
+//                  at tau, the last kept index j_cut) over them.  Otherwise a
+//                  lower rung's scores are collected in one more pass, or a
+//                  2048-bucket mass histogram finds the boundary bucket whose
+//                  scores are solved.  Every CTA then writes its share of the
+//                  top-p bitmask and attends, for its query head, the kept
+//                  rows of its share that lie outside the sinks and the
+//                  window.  The cluster merges its partials with the head's
+//                  sink/window partial and writes the output.
+//
+// Every in-kernel wait is either a hardware barrier reached uniformly or a
+// bounded wait on a copy barrier (RTP_DEV_TIMEOUT when it gives up).
 //
 // Top-p follows the abstract's observation (3) and the atlas.scime.ai summary
 // ("query-adaptive top-p threshold"); sinks + window follow that summary's
 // "Approach"; the 16-d pre-RoPE indexer follows observation (2).
+#include <atomic>
 #include <climits>
+#include <mutex>
 #include <type_traits>
 
 #include <cooperative_groups.h>
@@ -50,7 +59,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSwTile = 256;        // sink/window rows per attention CTA (32 per warp)
+constexpr int kSwCluster = 16;      // CTAs per sink/window cluster (one cluster per sequence and KV head)
+constexpr int kStreamSmem = 80 * 1024;  // stream kernel: bytes of staged keys (score) or K/V rows (two stages)
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
 constexpr int kMaxCS = 16;          // largest select cluster
@@ -82,14 +92,13 @@ struct DecodeArgs {
   int* sel_count;   // optional [B][NR]
   float* logits;    // [B][NR][lstride]
   float* cmax;      // [B][NR][nch_score_max]
-  float* pm;        // [B][Hkv][n_parts_max][G]: sink/window tiles, then select CTAs
-  float* pl;
-  float* po;        // [B][Hkv][n_parts_max][G][D]
-  unsigned* ctl;    // [B*Hkv] merge tickets, then [B*Hkv] select partials written
-  int* rank_cnt;    // [B][NR][kMaxCS] kept tokens per select CTA
+  float* sw_part;   // [B][Hkv][G][D + 2]: sink/window partial per query head (o[D], m, l)
   uint2* cand;      // [B][NR][lstride] boundary-bucket candidates past kCandSmem
-  int n_ctl, nch_score_max, n_sw_tiles, n_parts_max, n_score_ctas, n_sw_ctas, sel_cs;
+  int nch_score_max, n_score_ctas, n_score_pad, sel_cs;
   int want_mask;    // 1: the caller asked for the top-p bitmask
+  unsigned tx_extra;   // bytes a copy barrier expects beyond its copies (0; 16 when a test arms expiry)
+  unsigned long long wait_ns;  // time a bounded wait allows before it gives up
+  KvMap kv;
   int ret_head[kMaxRetrieval];
   int ret_rank[kMaxRetrieval];
   double inv_freq[64];  // RoPE frequencies, k < D/2
@@ -101,15 +110,6 @@ __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void prefetch_l2(const void* p) { asm volatile("prefetch.global.L2 [%0];" :: "l"(p)); }
-
-__device__ __forceinline__ unsigned ld_acquire(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Polls of a bounded wait (about 100 ns each) before it gives up.
-constexpr int kSpinLimit = 1 << 22;
 
 __device__ __forceinline__ bool seq_ok(int L, const DecodeArgs& a) {
   return L >= 1 && L <= a.max_seq_len;
@@ -140,28 +140,6 @@ __device__ __forceinline__ unsigned warp_sum_u32(unsigned v) {
   return v;
 }
 
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-
-// "Last CTA of the group" ticket: every CTA of the group calls this once.
-// The barrier orders every thread's earlier writes before thread 0's fence,
-// whose release makes them visible before the counter moves.
-__device__ __forceinline__ bool take_ticket(unsigned* counter, unsigned n, int* s_flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const unsigned t = atomicAdd(counter, 1u);
-    *s_flag = (t == n - 1);
-  }
-  __syncthreads();
-  const bool last = *s_flag;
-  if (last) __threadfence();
-  return last;
-}
-
 // RoPE'd query of the G heads of KV head h at position pos, scaled by
 // log2(e)/sqrt(D), into shared memory [G][D].
 template <typename T, int D, int G>
@@ -179,318 +157,29 @@ __device__ void rope_query(const DecodeArgs& a, int b, int h, int pos, float* s_
 }
 
 // ---------------------------------------------------------------------------
-// warp-level attention over tiles of 32 rows
+// 1a. score CTA: indexer scores + per-chunk maxima of one retrieval KV head
 // ---------------------------------------------------------------------------
-// load(): lane i requests row i's whole key and, for every live row of the
-// tile, its own D/32 value dims, so a tile costs one memory round trip.
-// compute(): lane-per-row dot products against the G queries (broadcast from
-// shared memory), the tile's softmax per head with one exp2 per (row, head),
-// and P V with the row weights broadcast by shuffle.
+// The chunk's indexer keys (contiguous rows of the key cache) arrive in shared
+// memory with one bulk asynchronous copy; the scores are then formed there.
 template <typename T, int D, int G>
-struct WarpAttn {
-  static constexpr int DL = D / 32;             // output dims per lane
-  static constexpr int KV = D * sizeof(T) / 16; // 16-byte vectors per key row
-  static constexpr int VB = DL * sizeof(T);     // value bytes per lane per row
-  using VRaw = typename std::conditional<VB == 16, uint4,
-               typename std::conditional<VB == 8, uint2,
-               typename std::conditional<VB == 4, unsigned, unsigned short>::type>::type>::type;
-  float m[G], l[G], o[G][DL];
-  uint4 kraw[KV];
-  const T* vb;
-  uint64_t pol;
-  int row;
-  unsigned msk, live;
-
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      m[g] = -CUDART_INF_F;
-      l[g] = 0.f;
-#pragma unroll
-      for (int d = 0; d < DL; ++d) o[g][d] = 0.f;
-    }
-  }
-
-  // row_: this lane's row (ignored when msk_ == 0); msk_: head bits.  Issues
-  // the key loads; the value loads are issued inside compute(), after the
-  // scores, so keys and values are never live in registers together.
-  __device__ __forceinline__ void load(const T* __restrict__ kb, const T* __restrict__ vb_, int row_,
-                                       unsigned msk_) {
-    row = msk_ ? row_ : 0;
-    msk = msk_;
-    vb = vb_;
-    live = __ballot_sync(0xffffffffu, msk_ != 0u);
-    const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)row * D);
-    pol = l2_evict_first();
-#pragma unroll
-    for (int i = 0; i < KV; ++i) kraw[i] = msk ? ld_stream(kr + i, pol) : make_uint4(0u, 0u, 0u, 0u);
-  }
-
-  __device__ __forceinline__ void compute(const float* __restrict__ s_q) {
-    float s4[G][4];  // four independent partial sums per head
-#pragma unroll
-    for (int g = 0; g < G; ++g) s4[g][0] = s4[g][1] = s4[g][2] = s4[g][3] = 0.f;
-    constexpr int E = 16 / sizeof(T);
-#pragma unroll
-    for (int i = 0; i < KV; ++i) {
-      float kf[E];
-      if constexpr (sizeof(T) == 2) {
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kraw[i]);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(h2[q]);
-          kf[2 * q] = f.x;
-          kf[2 * q + 1] = f.y;
-        }
-      } else {
-        kf[0] = __uint_as_float(kraw[i].x); kf[1] = __uint_as_float(kraw[i].y);
-        kf[2] = __uint_as_float(kraw[i].z); kf[3] = __uint_as_float(kraw[i].w);
-      }
-#pragma unroll
-      for (int e = 0; e < E; e += 4) {
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float4 qv = *reinterpret_cast<const float4*>(s_q + g * D + i * E + e);
-          float* acc = s4[g];
-          acc[0] = fmaf(qv.x, kf[e], acc[0]);
-          acc[1] = fmaf(qv.y, kf[e + 1], acc[1]);
-          acc[2] = fmaf(qv.z, kf[e + 2], acc[2]);
-          acc[3] = fmaf(qv.w, kf[e + 3], acc[3]);
-        }
-      }
-    }
-    float s[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) s[g] = (s4[g][0] + s4[g][1]) + (s4[g][2] + s4[g][3]);
-    float p[G];
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const bool on = (msk >> g) & 1u;
-      const float sv = on ? s[g] : -CUDART_INF_F;
-      const float tm = warp_max(sv);
-      const float mn = fmaxf(m[g], tm);
-      if (mn == -CUDART_INF_F) {  // nothing kept for this head yet (warp-uniform)
-        p[g] = 0.f;
-        continue;
-      }
-      const float al = exp2f(m[g] - mn);
-      p[g] = on ? exp2f(sv - mn) : 0.f;
-      l[g] = l[g] * al + p[g];
-#pragma unroll
-      for (int d = 0; d < DL; ++d) o[g][d] *= al;
-      m[g] = mn;
-    }
-    // value slices of the tile's live rows (lane owns dims [lane*DL, lane*DL + DL)),
-    // 16 rows at a time
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      VRaw vraw[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        const int rr = __shfl_sync(0xffffffffu, row, half * 16 + r);
-        if ((live >> (half * 16 + r)) & 1u)
-          vraw[r] = ld_stream(reinterpret_cast<const VRaw*>(vb + (size_t)rr * D + lane * DL), pol);
-        else
-          vraw[r] = VRaw();
-      }
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        if (!((live >> (half * 16 + r)) & 1u)) continue;  // warp-uniform
-        float vv[DL];
-        const T* vt = reinterpret_cast<const T*>(&vraw[r]);
-#pragma unroll
-        for (int d = 0; d < DL; ++d) vv[d] = to_f32(vt[d]);
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float pr = __shfl_sync(0xffffffffu, p[g], half * 16 + r);
-#pragma unroll
-          for (int d = 0; d < DL; ++d) o[g][d] = fmaf(pr, vv[d], o[g][d]);
-        }
-      }
-    }
-  }
-};
-
-// Merge the warps' WarpAttn states of a CTA and write one partial (m, l, o)
-// per query head at slot `part`.
-template <int D, int G, typename WA>
-__device__ void write_partial(const DecodeArgs& a, WA& wa, size_t part, float* s_o, float* s_ml) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float lw = warp_sum(wa.l[g]);
-#pragma unroll
-    for (int d = 0; d < WA::DL; ++d) s_o[(warp * G + g) * D + lane * WA::DL + d] = wa.o[g][d];
-    if (lane == 0) {
-      s_ml[(warp * G + g) * 2] = wa.m[g];
-      s_ml[(warp * G + g) * 2 + 1] = lw;
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < G * D; i += blockDim.x) {
-    const int g = i / D, d = i % D;
-    float mn = -CUDART_INF_F;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) mn = fmaxf(mn, s_ml[(w * G + g) * 2]);
-    float acc = 0.f, den = 0.f;
-    if (mn != -CUDART_INF_F) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        const float mw = s_ml[(w * G + g) * 2];
-        if (mw == -CUDART_INF_F) continue;
-        const float sc = exp2f(mw - mn);
-        acc = fmaf(s_o[(w * G + g) * D + d], sc, acc);
-        den = fmaf(s_ml[(w * G + g) * 2 + 1], sc, den);
-      }
-    }
-    a.po[(part * G + g) * D + d] = acc;
-    if (d == 0) {
-      a.pm[part * G + g] = mn;
-      a.pl[part * G + g] = den;
-    }
-  }
-}
-
-// Merge every partial (m, l, o) of KV head (b, h) into the output (one CTA).
-// Stage 1 combines the sink/window partials and runs before the selection has
-// finished; stage 2 waits until the select CTAs of this KV head have counted
-// their partials written and adds those n_sel per query head.  Partials with
-// m = -inf are empty and carry weight 0.
-template <typename T, int D, int G>
-__device__ void merge_partials(const DecodeArgs& a, int b, int h, int n_sel, float* s_buf) {
-  constexpr int kPer = (G * D + kThreads - 1) / kThreads;  // (head, dim) outputs per thread
-  const int tid = threadIdx.x;
-  const int n_sw = a.n_sw_tiles;
-  const size_t pbase = ((size_t)b * a.Hkv + h) * a.n_parts_max;
-  float* s_w = s_buf;                        // [n_parts_max][G] part weights
-  float* s_pl = s_buf + a.n_parts_max * G;   // [n_parts_max][G] part denominators
-  float* s_st = s_pl + a.n_parts_max * G;    // [G][3]: max, denominator, stage-1 scale
-  __syncthreads();
-  for (int i = tid; i < n_sw * G; i += kThreads) {
-    s_w[i] = __ldcg(a.pm + pbase * G + i);
-    s_pl[i] = __ldcg(a.pl + pbase * G + i);
-  }
-  __syncthreads();
-  if (tid < G) {
-    float mn = -CUDART_INF_F;
-    for (int t = 0; t < n_sw; ++t) mn = fmaxf(mn, s_w[t * G + tid]);
-    float den = 0.f;
-    for (int t = 0; t < n_sw; ++t) {
-      const float pmv = s_w[t * G + tid];
-      const float w = (pmv == -CUDART_INF_F) ? 0.f : exp2f(pmv - mn);
-      s_w[t * G + tid] = w;
-      den = fmaf(s_pl[t * G + tid], w, den);
-    }
-    s_st[tid * 3] = mn;
-    s_st[tid * 3 + 1] = den;
-    s_st[tid * 3 + 2] = 1.f;
-  }
-  __syncthreads();
-  float acc[kPer];
-#pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    acc[u] = 0.f;
-    const int i = tid + u * kThreads;
-    if (i < G * D) {
-      const int g = i / D, d = i % D;
-#pragma unroll 8
-      for (int t = 0; t < n_sw; ++t) {
-        const float w = s_w[t * G + g];
-        const float pv = __ldcg(a.po + ((pbase + t) * G + g) * D + d);  // stale if w == 0
-        acc[u] = w > 0.f ? fmaf(pv, w, acc[u]) : acc[u];
-      }
-    }
-  }
-  if (n_sel > 0) {
-    // Wait until every select CTA of this KV head has written its partial
-    // (they are all running: this grid launched only after each of them
-    // started, and they wait for nothing of this grid).
-    if (tid == 0) {
-      const unsigned need = (unsigned)(G * n_sel);
-      const unsigned* done = a.ctl + (size_t)a.B * a.Hkv + (size_t)b * a.Hkv + h;
-      int spins = 0;
-      while (ld_acquire(done) < need) {
-        if (++spins > kSpinLimit) {
-          atomicOr(a.status, RTP_DEV_TIMEOUT);
-          break;
-        }
-        __nanosleep(100);
-      }
-    }
-    const size_t sbase = pbase + n_sw;
-    __syncthreads();
-    for (int i = tid; i < n_sel * G; i += kThreads) {
-      s_w[i] = __ldcg(a.pm + sbase * G + i);
-      s_pl[i] = __ldcg(a.pl + sbase * G + i);
-    }
-    __syncthreads();
-    if (tid < G) {
-      const float m1 = s_st[tid * 3];
-      float mn = m1;
-      for (int t = 0; t < n_sel; ++t) mn = fmaxf(mn, s_w[t * G + tid]);
-      const float w1 = (m1 == -CUDART_INF_F) ? 0.f : exp2f(m1 - mn);
-      float den = s_st[tid * 3 + 1] * w1;
-      for (int t = 0; t < n_sel; ++t) {
-        const float pmv = s_w[t * G + tid];
-        const float w = (pmv == -CUDART_INF_F) ? 0.f : exp2f(pmv - mn);
-        s_w[t * G + tid] = w;
-        den = fmaf(s_pl[t * G + tid], w, den);
-      }
-      s_st[tid * 3 + 1] = den;
-      s_st[tid * 3 + 2] = w1;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int u = 0; u < kPer; ++u) {
-      const int i = tid + u * kThreads;
-      if (i < G * D) {
-        const int g = i / D, d = i % D;
-        float pv[kMaxCS];  // every load in flight at once (empty partials are skipped)
-#pragma unroll
-        for (int t = 0; t < kMaxCS; ++t)
-          pv[t] = (t < n_sel && s_w[t * G + g] > 0.f) ? __ldcg(a.po + ((sbase + t) * G + g) * D + d) : 0.f;
-        float v = acc[u] * s_st[g * 3 + 2];
-#pragma unroll
-        for (int t = 0; t < kMaxCS; ++t)
-          if (t < n_sel) v = fmaf(pv[t], s_w[t * G + g], v);
-        acc[u] = v;
-      }
-    }
-  }
-#pragma unroll
-  for (int u = 0; u < kPer; ++u) {
-    const int i = tid + u * kThreads;
-    if (i < G * D) {
-      const int g = i / D, d = i % D;
-      T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + h * G + g) * D + d;
-      *out = from_f32<T>(acc[u] / s_st[g * 3 + 1]);
-    }
-  }
-  griddep_wait();  // this grid completes only after the select kernel has
-}
-
-// ---------------------------------------------------------------------------
-// 1. score kernel: indexer scores + per-chunk maxima (+ this call's tickets zeroed)
-// ---------------------------------------------------------------------------
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads, 2) score_kernel(DecodeArgs a) {
-  // q~ is formed from the caller's inputs before waiting for rtp_append_kv;
-  // the select kernel may launch meanwhile (it waits for this grid).
-  griddep_launch();
+__device__ __forceinline__ void score_cta(const DecodeArgs& a, int sc, unsigned char* dsm, uint64_t* bar) {
   constexpr int kChunk = score_chunk(sizeof(T));
   constexpr int TPT = kChunk / kThreads;        // keys per thread
   constexpr int NV = kIdxDim * sizeof(T) / 16;  // 16-byte vectors per key
+  constexpr int KB = kIdxDim * sizeof(T);       // bytes per key
+  static_assert(kChunk * KB <= kStreamSmem, "a score chunk fits in the stream kernel's shared memory");
   __shared__ __align__(16) float s_q[G * kIdxDim];
   __shared__ float s_ml[kWarps * G];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = a.n_score_ctas / (a.B * a.R);
-  const int chunk = blockIdx.x % nch;
-  const int br = blockIdx.x / nch;
+  const int chunk = sc % nch;
+  const int br = sc / nch;
   const int b = br / a.R, r = br % a.R;
   const int h = a.ret_head[r];
   const int L = a.seq_len[b];
-  // q~ = W_q q_pre: four threads per output, a quarter of the dims each
+  if (tid == 0) mbar_init(bar, 1);
+  // q~ = W_q q_pre from the caller's inputs, before waiting for rtp_append_kv:
+  // four threads per output, a quarter of the dims each
   for (int o4 = tid; o4 < G * kIdxDim * 4; o4 += kThreads) {
     const int o = o4 >> 2, qd = o4 & 3;
     const int g = o / kIdxDim, i = o % kIdxDim;
@@ -511,43 +200,45 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(DecodeArgs a) {
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
     if (qd == 0) s_q[g * kIdxDim + i] = acc;
   }
-  griddep_wait();  // the appended token's indexer key; the previous call's tickets are done
-  if (blockIdx.x == 0)  // merge tickets of this call
-    for (int i = tid; i < a.n_ctl; i += kThreads) a.ctl[i] = 0u;
-  // The keys are requested up to the call's maximum length without waiting for
-  // seq_len (rows past seq_len are in bounds and their scores are never used).
-  const int j0 = chunk * kChunk;
-  const int jh = min(a.max_seq_len, j0 + kChunk);
-  const uint4* kidx = reinterpret_cast<const uint4*>(static_cast<const T*>(a.kidx) +
-                                                     ((size_t)b * a.R + r) * a.Lmax * kIdxDim);
-  const uint64_t pol = l2_evict_first();
-  uint4 kr[TPT][NV];
-#pragma unroll
-  for (int t = 0; t < TPT; ++t) {
-    const int j = j0 + t * kThreads + tid;
-#pragma unroll
-    for (int v = 0; v < NV; ++v) kr[t][v] = (j < jh) ? ld_stream(kidx + (size_t)j * NV + v, pol) : make_uint4(0u, 0u, 0u, 0u);
-  }
-  __syncthreads();  // q~ visible
-  if (!seq_ok(L, a)) {
+  __syncthreads();  // barrier initialised, q~ visible
+  griddep_wait();   // rtp_append_kv (and with it the previous decode step) has completed
+  if (!seq_ok(L, a)) {  // uniform over the CTA
     if (chunk == 0 && r == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
     return;
   }
+  // The keys are fetched up to the call's maximum length without looking at
+  // seq_len (rows past seq_len are in bounds and their scores are never used).
+  const int j0 = chunk * kChunk;
+  const int jh = min(a.max_seq_len, j0 + kChunk);
+  const unsigned char* src = static_cast<const unsigned char*>(a.kidx) +
+                             (((size_t)b * a.R + r) * a.Lmax + j0) * KB;
+  if (tid == 0) {
+    const uint32_t bytes = (uint32_t)(jh - j0) * KB;
+    mbar_expect_tx(bar, bytes + a.tx_extra);
+    bulk_g2s(dsm, src, bytes, bar, l2_evict_first());
+  }
+  if (!mbar_wait_bounded(bar, 0, a.wait_ns, a.status)) {
+    mbar_wait_bounded(bar, 0, a.wait_ns, a.status);  // the copy, before leaving (output invalid)
+    return;
+  }
   const int j1 = min(L, jh);
-  if (j0 >= j1) return;  // chunk past this sequence's length (uniform over the CTA)
   float* lg = a.logits + ((size_t)b * a.NR + (size_t)r * G) * a.lstride;
   float mx[G];
 #pragma unroll
   for (int g = 0; g < G; ++g) mx[g] = -CUDART_INF_F;
 #pragma unroll
   for (int t = 0; t < TPT; ++t) {
-    const int j = j0 + t * kThreads + tid;
+    const int jl = t * kThreads + tid;
+    const int j = j0 + jl;
     if (j >= j1) continue;
+    uint4 kr[NV];
+#pragma unroll
+    for (int v = 0; v < NV; ++v) kr[v] = reinterpret_cast<const uint4*>(dsm + (size_t)jl * KB)[v];
     float kv[kIdxDim];
     if constexpr (sizeof(T) == 2) {
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kr[t][v]);
+        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kr[v]);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float2 f = __bfloat1622float2(h2[q]);
@@ -558,8 +249,8 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(DecodeArgs a) {
     } else {
 #pragma unroll
       for (int v = 0; v < NV; ++v) {
-        kv[v * 4 + 0] = __uint_as_float(kr[t][v].x); kv[v * 4 + 1] = __uint_as_float(kr[t][v].y);
-        kv[v * 4 + 2] = __uint_as_float(kr[t][v].z); kv[v * 4 + 3] = __uint_as_float(kr[t][v].w);
+        kv[v * 4 + 0] = __uint_as_float(kr[v].x); kv[v * 4 + 1] = __uint_as_float(kr[v].y);
+        kv[v * 4 + 2] = __uint_as_float(kr[v].z); kv[v * 4 + 3] = __uint_as_float(kr[v].w);
       }
     }
 #pragma unroll
@@ -579,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(DecodeArgs a) {
       mx[g] = fmaxf(mx[g], s);
     }
   }
-  // one block reduction for the G chunk maxima
+  // one block reduction for the G chunk maxima (-inf for a chunk past seq_len)
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     const float v = warp_max(mx[g]);
@@ -595,58 +286,291 @@ __global__ void __launch_bounds__(kThreads, 2) score_kernel(DecodeArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// 3. sink/window kernel: exact attention over the sinks and the window of
-// every KV head, then the merge.  The sink/window rows do not depend on the
-// selection, so this kernel is launched after the select kernel without
-// waiting for it: it runs while the selection runs.  The last CTA of each KV
-// head merges the sink/window partials, then waits for the select kernel and
-// adds its partials (so this grid completes only after the selection has).
-// Everything it reads before that wait was finished by rtp_append_kv before
-// the select kernel triggered this launch; it reads through L2.
+// 1b. sink/window CTA: rank `crank` of the cluster of (sequence b, KV head h)
 // ---------------------------------------------------------------------------
+// The CTA's rows arrive in shared memory by bulk asynchronous copies, one per
+// contiguous run of cache rows (the sinks, the window, and a second window run
+// where a ring wraps), in stages of kStreamSmem / 2 bytes (K and V), two stages
+// in flight.  A half-warp then owns a row: lane (half, c) reads dims
+// [c*EPL, c*EPL + EPL) of the row's key and value, so a warp covers two rows.
+// Scores of the G query heads are reduced over the half-warp by shuffles;
+// every lane keeps the running (max, sum) of its half and the weighted value
+// sum of its own dims.
+template <typename T, int D>
+struct SwLane {
+  static constexpr int EPL = D / 16;                 // elements per lane per row
+  static constexpr int VB = EPL * (int)sizeof(T);    // bytes per lane per row
+  static constexpr int NV = VB >= 16 ? VB / 16 : 1;
+  using Vec = typename std::conditional<VB >= 16, uint4, uint2>::type;
+  Vec v[NV];
+  __device__ __forceinline__ void load(const unsigned char* p) {
+    const Vec* q = reinterpret_cast<const Vec*>(p);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) v[i] = q[i];
+  }
+  __device__ __forceinline__ void to_f32(float (&f)[EPL]) const {
+    if constexpr (sizeof(T) == 2) {
+      const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(v);
+#pragma unroll
+      for (int i = 0; i < EPL / 2; ++i) {
+        const float2 x = __bfloat1622float2(h2[i]);
+        f[2 * i] = x.x;
+        f[2 * i + 1] = x.y;
+      }
+    } else {
+      const float* x = reinterpret_cast<const float*>(v);
+#pragma unroll
+      for (int i = 0; i < EPL; ++i) f[i] = x[i];
+    }
+  }
+};
+
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads, 2) sw_kernel(DecodeArgs a) {
-  griddep_launch();
+__device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, int csw, unsigned char* dsm,
+                                       uint64_t* bar) {
+  using Lane = SwLane<T, D>;
+  constexpr int EPL = Lane::EPL;
+  constexpr int RB = D * (int)sizeof(T);             // bytes per cache row
+  constexpr int SR = kStreamSmem / 4 / RB;           // rows per stage (K and V of a stage: half the buffer)
+  static_assert(SR >= 2 && SR % 2 == 0, "a stage holds whole row pairs");
   __shared__ __align__(16) float s_q[G * D];
-  __shared__ __align__(16) float s_o[kWarps * G * D];
-  __shared__ float s_ml[kWarps * G * 2];
-  __shared__ int s_flag;
-  const int tid = threadIdx.x;
-  const int tile = blockIdx.x % a.n_sw_tiles;
-  const int bkv = blockIdx.x / a.n_sw_tiles;
+  __shared__ __align__(16) float s_wo[kWarps][G][D];
+  __shared__ float s_wml[kWarps][G][2];
+  __shared__ __align__(16) float s_part[G][D + 2];  // this CTA's (o[D], m, l) per query head
+  cg::cluster_group cl = cg::this_cluster();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int half = lane >> 4, c = lane & 15;
   const int b = bkv / a.Hkv, h = bkv % a.Hkv;
+  const int r = a.ret_rank[h];
   const int L = a.seq_len[b];
-  if (!seq_ok(L, a)) {
-    if (tile == 0 && h == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
-    griddep_wait();
+  if (!seq_ok(L, a)) {  // uniform over the cluster
+    if (crank == 0 && h == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
     return;
   }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+  }
+  rope_query<T, D, G>(a, b, h, L - 1, s_q);  // caller's inputs: before the wait
+  __syncthreads();  // barriers initialised, s_q visible
+  griddep_wait();
+
   const int s_cnt = min(a.S, L);
   const int sw0 = max(s_cnt, L - a.W);
-  const int n_sw = s_cnt + (L - sw0);
-  const int e = tile * kSwTile + threadIdx.x;  // one row per thread, 32 per warp
-  const bool ok = e < n_sw;
-  const int row = ok ? (e < s_cnt ? e : sw0 + (e - s_cnt)) : 0;
-  WarpAttn<T, D, G> wa;
-  wa.init();
-  const T* kb = static_cast<const T*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
-  const T* vb = static_cast<const T*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
-  wa.load(kb, vb, row, ok ? ((1u << G) - 1u) : 0u);  // in flight during RoPE
-  rope_query<T, D, G>(a, b, h, L - 1, s_q);
-  __syncthreads();
-  wa.compute(s_q);
-  write_partial<D, G>(a, wa, (size_t)bkv * a.n_parts_max + tile, s_o, s_ml);
-  // The last sink/window CTA of this KV head merges; it alone waits for the
-  // selection (so this grid completes only after the select kernel has).
-  if (!take_ticket(&a.ctl[bkv], a.n_sw_tiles, &s_flag)) return;
-  const int r = a.ret_rank[h];
-  merge_partials<T, D, G>(a, b, h, r >= 0 ? a.sel_cs : 0, s_o);
-  if (r >= 0 && a.sel_count && tid < G) {
-    const size_t bh = (size_t)b * a.NR + r * G + tid;
-    int c = 0;
-    for (int q = 0; q < a.sel_cs; ++q) c += __ldcg(a.rank_cnt + bh * kMaxCS + q);
-    a.sel_count[bh] = c;
+  const int n_sw = s_cnt + (L - sw0);      // rows e: sinks e < s_cnt, then window positions
+  const int npair_all = (n_sw + 1) / 2;
+  const int per = (npair_all + csw - 1) / csw;
+  const int e_lo = min(n_sw, 2 * crank * per), e_hi = min(n_sw, 2 * (crank + 1) * per);
+  const int n_st = (e_hi - e_lo + SR - 1) / SR;
+  const unsigned char* kbase = static_cast<const unsigned char*>(a.k);
+  const unsigned char* vbase = static_cast<const unsigned char*>(a.v);
+  const bool ringed = (a.kv.ring_mask >> h) & 1ull;
+
+  // stage st: rows [e_lo + st*SR, ...) into buffer st & 1 (K, then V)
+  auto issue = [&](int st) {
+    const int e0 = e_lo + st * SR, e1 = min(e_hi, e0 + SR);
+    uint64_t* bb = bar + (st & 1);
+    unsigned char* dk = dsm + (size_t)(st & 1) * (kStreamSmem / 2);
+    unsigned char* dv = dk + (size_t)SR * RB;
+    mbar_expect_tx(bb, (uint32_t)(e1 - e0) * 2u * RB + a.tx_extra);
+    const uint64_t pol = l2_evict_first();
+    for (int e = e0; e < e1;) {
+      const int pos = e < s_cnt ? e : sw0 + (e - s_cnt);
+      int n = (e < s_cnt ? s_cnt : e1) - e;
+      if (e < s_cnt && n > e1 - e) n = e1 - e;
+      if (ringed && pos >= a.kv.S) n = min(n, a.kv.S + a.kv.ring - (a.kv.S + (pos - a.kv.S) % a.kv.ring));
+      const size_t row = a.kv.row(b, h, pos);
+      bulk_g2s(dk + (size_t)(e - e0) * RB, kbase + row * RB, (uint32_t)n * RB, bb, pol);
+      bulk_g2s(dv + (size_t)(e - e0) * RB, vbase + row * RB, (uint32_t)n * RB, bb, pol);
+      e += n;
+    }
+  };
+  if (tid == 0) {
+    if (n_st > 0) issue(0);
+    if (n_st > 1) issue(1);
   }
+
+  float m[G], l[G], o[G][EPL];
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    m[g] = -CUDART_INF_F;
+    l[g] = 0.f;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
+  }
+  int failed = -1;
+  for (int st = 0; st < n_st; ++st) {
+    if (!mbar_wait_bounded(bar + (st & 1), (uint32_t)(st >> 1) & 1u, a.wait_ns, a.status)) {
+      failed = st;
+      break;
+    }
+    const int n = min(e_hi, e_lo + (st + 1) * SR) - (e_lo + st * SR);
+    const unsigned char* sk = dsm + (size_t)(st & 1) * (kStreamSmem / 2);
+    const unsigned char* sv = sk + (size_t)SR * RB;
+    for (int p = warp; 2 * p < n; p += kWarps) {
+      const int i = 2 * p + half;
+      const bool ok = i < n;  // uniform over the half-warp
+      Lane kr, vr;
+      kr.load(sk + (size_t)(ok ? i : 0) * RB + c * Lane::VB);
+      vr.load(sv + (size_t)(ok ? i : 0) * RB + c * Lane::VB);
+      float kf[EPL];
+      kr.to_f32(kf);
+      float s[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float* qg = s_q + g * D + c * EPL;
+        float acc = 0.f;
+#pragma unroll
+        for (int e4 = 0; e4 < EPL; e4 += 4) {
+          const float4 qq = *reinterpret_cast<const float4*>(qg + e4);
+          acc = fmaf(qq.x, kf[e4], acc);
+          acc = fmaf(qq.y, kf[e4 + 1], acc);
+          acc = fmaf(qq.z, kf[e4 + 2], acc);
+          acc = fmaf(qq.w, kf[e4 + 3], acc);
+        }
+        s[g] = acc;
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        s[g] += __shfl_xor_sync(0xffffffffu, s[g], 8);
+        s[g] += __shfl_xor_sync(0xffffffffu, s[g], 4);
+        s[g] += __shfl_xor_sync(0xffffffffu, s[g], 2);
+        s[g] += __shfl_xor_sync(0xffffffffu, s[g], 1);
+      }
+      if (ok) {
+        float vf[EPL];
+        vr.to_f32(vf);
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float mn = fmaxf(m[g], s[g]);
+          const float al = exp2f(m[g] - mn);  // 0 while nothing was attended (m = -inf)
+          const float pv = exp2f(s[g] - mn);
+          l[g] = fmaf(l[g], al, pv);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) o[g][e] = fmaf(o[g][e], al, pv * vf[e]);
+          m[g] = mn;
+        }
+      }
+    }
+    __syncthreads();  // buffer st & 1 is free
+    if (tid == 0 && st + 2 < n_st) issue(st + 2);
+  }
+  if (failed >= 0) {
+    // a copy did not complete in time (RTP_DEV_TIMEOUT is set): wait, again
+    // with a limit, for the stages still in flight before leaving; the
+    // output is invalid
+    for (int st = failed; st < min(n_st, failed + 2); ++st)
+      mbar_wait_bounded(bar + (st & 1), (uint32_t)(st >> 1) & 1u, a.wait_ns, a.status);
+  }
+  // the two halves of the warp, then the warps of the CTA
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m[g], 16);
+    const float l2 = __shfl_xor_sync(0xffffffffu, l[g], 16);
+    const float mn = fmaxf(m[g], m2);
+    const float a1 = (m[g] == -CUDART_INF_F) ? 0.f : exp2f(m[g] - mn);
+    const float a2 = (m2 == -CUDART_INF_F) ? 0.f : exp2f(m2 - mn);
+    l[g] = l[g] * a1 + l2 * a2;
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) {
+      const float o2 = __shfl_xor_sync(0xffffffffu, o[g][e], 16);
+      o[g][e] = o[g][e] * a1 + o2 * a2;
+    }
+    m[g] = mn;
+    if (half == 0) {
+#pragma unroll
+      for (int e = 0; e < EPL; ++e) s_wo[warp][g][c * EPL + e] = o[g][e];
+    }
+    if (lane == 0) {
+      s_wml[warp][g][0] = m[g];
+      s_wml[warp][g][1] = l[g];
+    }
+  }
+  __syncthreads();
+  for (int i = tid; i < G * D; i += kThreads) {
+    const int g = i / D, d = i % D;
+    float mn = -CUDART_INF_F;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mn = fmaxf(mn, s_wml[w][g][0]);
+    float acc = 0.f, den = 0.f;
+    if (mn != -CUDART_INF_F) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        const float mw = s_wml[w][g][0];
+        if (mw == -CUDART_INF_F) continue;
+        const float sc = exp2f(mw - mn);
+        acc = fmaf(s_wo[w][g][d], sc, acc);
+        den = fmaf(s_wml[w][g][1], sc, den);
+      }
+    }
+    s_part[g][d] = acc;
+    if (d == 0) {
+      s_part[g][D] = mn;
+      s_part[g][D + 1] = den;
+    }
+  }
+  cl.sync();  // every rank's partial in its shared memory
+  // The cluster's merge is spread over its ranks: element i of the G x D
+  // outputs goes to rank i mod csw.  Each thread issues its loads of every
+  // rank's partial at once (distributed shared memory, one round trip).
+  for (int i = crank + csw * tid; i < G * D; i += csw * kThreads) {
+    const int g = i / D, d = i % D;
+    float mq[kSwCluster], lq[kSwCluster], oq[kSwCluster];
+#pragma unroll
+    for (int q = 0; q < kSwCluster; ++q) {
+      mq[q] = -CUDART_INF_F;
+      lq[q] = 0.f;
+      oq[q] = 0.f;
+      if (q < csw) {
+        const float* pq = cl.map_shared_rank(&s_part[g][0], q);
+        mq[q] = pq[D];
+        lq[q] = pq[D + 1];
+        oq[q] = pq[d];
+      }
+    }
+    float mn = -CUDART_INF_F;
+#pragma unroll
+    for (int q = 0; q < kSwCluster; ++q) mn = fmaxf(mn, mq[q]);
+    float acc = 0.f, den = 0.f;
+#pragma unroll
+    for (int q = 0; q < kSwCluster; ++q) {
+      const float sc = mq[q] == -CUDART_INF_F ? 0.f : exp2f(mq[q] - mn);
+      acc = fmaf(oq[q], sc, acc);
+      den = fmaf(lq[q], sc, den);
+    }
+    if (r < 0) {  // local head: this is the whole attention
+      T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + h * G + g) * D + d;
+      *out = from_f32<T>(acc / den);
+    } else {      // retrieval head: the select kernel adds its kept rows
+      float* sp = a.sw_part + ((size_t)bkv * G + g) * (D + 2);
+      sp[d] = acc;
+      if (d == 0) {
+        sp[D] = mn;
+        sp[D + 1] = den;
+      }
+    }
+  }
+  cl.sync();  // no rank reads another's shared memory after this
+}
+
+// ---------------------------------------------------------------------------
+// 1. stream kernel: [score CTAs, padded to whole clusters][sink/window clusters]
+// ---------------------------------------------------------------------------
+// It lets the select kernel launch at once (its CTAs start with the work that
+// needs no scores); the select kernel waits for this whole grid to complete.
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_constant__ DecodeArgs a) {
+  extern __shared__ __align__(128) unsigned char dsm[];
+  __shared__ __align__(8) uint64_t s_bar[2];
+  griddep_launch();
+  const int blk = blockIdx.x;
+  if (blk < a.n_score_pad) {
+    if (blk < a.n_score_ctas) score_cta<T, D, G>(a, blk, dsm, s_bar);
+    return;
+  }
+  const int csw = (int)cg::this_cluster().num_blocks();
+  const int sw = blk - a.n_score_pad;
+  sw_cta<T, D, G>(a, sw / csw, (int)cg::this_cluster().block_rank(), csw, dsm, s_bar);
 }
 
 // ---------------------------------------------------------------------------
@@ -946,7 +870,7 @@ struct LaneRaw {
 // bitmask, and this head's attention over its kept rows outside sinks/window
 // ---------------------------------------------------------------------------
 template <typename T, int D, int CS>
-__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) select_kernel(DecodeArgs a) {
+__global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) select_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr int kChunk = score_chunk(sizeof(T));
   constexpr int DL = D / 32;
   using Raw = typename LaneRaw<T, D>::type;
@@ -980,8 +904,12 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   __shared__ __align__(16) float s_qh[D];
   __shared__ __align__(16) float s_wo[kSelWarps * D];
   __shared__ float s_wml[kSelWarps * 2];
-  const T* kb = static_cast<const T*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
-  const T* vb = static_cast<const T*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+  __shared__ __align__(16) float s_cp[D + 2];  // this CTA's partial for query head g: (o[D], m, l)
+  __shared__ int s_ccnt;                       // and its kept-token count
+  // retrieval heads keep the whole context: row pos of head h sits at row0 + pos
+  const size_t row0 = a.kv.row(b, h, 0);
+  const T* kb = static_cast<const T*>(a.k) + row0 * D;
+  const T* vb = static_cast<const T*>(a.v) + row0 * D;
 
   // This CTA's share of the context comes from the call's maximum length, so
   // the score loads below do not wait for seq_len.
@@ -1001,10 +929,10 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
 #pragma unroll 4
     for (int i = tid; i < nv; i += kSelThreads) dst[i] = __ldcg(src + i);
   };
-  // Before waiting for the score kernel: seq_len and this head's RoPE'd query
-  // (scaled by log2(e)/sqrt(D)) from the caller's inputs.  The trigger comes
-  // only after the wait, so the sink/window kernel starts once the appended
-  // token is in the cache.
+  // Before waiting for the scores: seq_len and this head's RoPE'd query
+  // (scaled by log2(e)/sqrt(D)) from the caller's inputs.  This kernel starts
+  // only once every stream CTA has passed its wait for rtp_append_kv, so the
+  // cache rows it reads are complete.
   const int L = a.seq_len[b];
   if (tid < D / 2 && seq_ok(L, a)) {
     const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * a.G + g) * D;
@@ -1017,15 +945,18 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   }
   if (rank == 0 && tid == 0) sh->n_cand2 = 0u;
   if (lane < kSpec) s_spec_j[warp][lane] = -1;
-  cluster_arrive();  // counter zeroed; every CTA of the cluster running
-  griddep_wait();
   griddep_launch();
+  cluster_arrive();  // counter zeroed; every CTA of the cluster running
+  griddep_wait();    // the stream kernel (scores, chunk maxima, sink/window partials) has completed
+  if (!seq_ok(L, a)) {  // uniform over the cluster; the stream kernel flagged it
+    cluster_wait();
+    return;
+  }
   const int nch_h = (Lh + kChunk - 1) / kChunk;
   const float* cm = a.cmax + (size_t)bh * a.nch_score_max;
   const float cm0 = tid < nch_h ? __ldcg(cm + tid) : -CUDART_INF_F;
   if (cached) stage(j0, jh);
   cluster_wait();
-  if (!seq_ok(L, a)) return;  // uniform over the cluster; the score kernel flagged it
   const int j1 = min(L, jh);  // j1 <= j0: nothing of this sequence in this CTA's share
   uint32_t* mask = a.mask + (size_t)bh * a.words;
   const bool keep_all = a.top_p >= 1.0f;
@@ -1637,7 +1568,6 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
     sh->cnt[warp] = cnt;
   }
   __syncthreads();
-  const size_t slot = (((size_t)b * a.Hkv + h) * a.n_parts_max + a.n_sw_tiles + rank) * a.G + g;
   for (int d = tid; d < D; d += kSelThreads) {
     float mn = -CUDART_INF_F;
 #pragma unroll
@@ -1653,85 +1583,194 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         den = fmaf(s_wml[w * 2 + 1], sc, den);
       }
     }
-    a.po[slot * D + d] = acc;
+    s_cp[d] = acc;
     if (d == 0) {
-      a.pm[slot] = mn;
-      a.pl[slot] = den;
+      s_cp[D] = mn;
+      s_cp[D + 1] = den;
     }
   }
   if (tid == 0) {
     int c = 0;
 #pragma unroll
     for (int w = 0; w < kSelWarps; ++w) c += sh->cnt[w];
-    a.rank_cnt[(size_t)bh * kMaxCS + rank] = c;
+    s_ccnt = c;
   }
-  // this CTA's partial and count are written: count them for the merge
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    atomicAdd(a.ctl + (size_t)a.B * a.Hkv + (size_t)b * a.Hkv + h, 1u);
+  cl.sync();  // every rank's partial and count in its shared memory
+  {
+    // The head's sink/window partial plus every rank's kept-row partial, the
+    // D output elements spread over the ranks (element d on rank d mod CS),
+    // each thread loading every rank's partial at once.
+    const int bkv = b * a.Hkv + h;
+    const float* sp = a.sw_part + ((size_t)bkv * a.G + g) * (D + 2);
+    for (int d = rank + CS * tid; d < D; d += CS * kSelThreads) {
+      float mq[CS], lq[CS], oq[CS];
+#pragma unroll
+      for (int q = 0; q < CS; ++q) {
+        const float* pq = cl.map_shared_rank(s_cp, q);
+        mq[q] = pq[D];
+        lq[q] = pq[D + 1];
+        oq[q] = pq[d];
+      }
+      const float m_sw = __ldcg(sp + D);
+      const float l_sw = __ldcg(sp + D + 1);
+      const float o_sw = __ldcg(sp + d);
+      float mn = m_sw;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) mn = fmaxf(mn, mq[q]);
+      float acc = 0.f, den = 0.f;
+      if (m_sw != -CUDART_INF_F) {
+        const float sc = exp2f(m_sw - mn);
+        acc = o_sw * sc;
+        den = l_sw * sc;
+      }
+#pragma unroll
+      for (int q = 0; q < CS; ++q) {
+        const float sc = mq[q] == -CUDART_INF_F ? 0.f : exp2f(mq[q] - mn);
+        acc = fmaf(oq[q], sc, acc);
+        den = fmaf(lq[q], sc, den);
+      }
+      T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + h * a.G + g) * D + d;
+      *out = from_f32<T>(acc / den);
+    }
+    if (rank == 0 && tid == 0 && a.sel_count) {
+      int c = 0;
+#pragma unroll
+      for (int q = 0; q < CS; ++q) c += *cl.map_shared_rank(&s_ccnt, q);
+      a.sel_count[bh] = c;
+    }
   }
+  cl.sync();  // no rank reads another's shared memory after this
 }
 
 // ---------------------------------------------------------------------------
 // launch helpers
 // ---------------------------------------------------------------------------
+// Time a bounded wait allows before it gives up (ns).
+constexpr unsigned long long kWaitNs = 400ull * 1000 * 1000;
+
+// Test hook (rtp_debug_wait_expiry): per host thread, armed for the next call.
+thread_local int t_expiry_polls = 0;
+
+cudaError_t launch_cluster_pdl(void (*k)(DecodeArgs), dim3 grid, dim3 block, size_t smem, int cluster,
+                               cudaStream_t st, const DecodeArgs& a) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, k, a);
+}
+
+// Stream kernel with 16-CTA sink/window clusters when the device can place
+// one (non-portable size), else 8.  Set up once per device under a mutex.
 template <typename T, int D, int G>
-cudaError_t launch_dg(const DecodeArgs& a, int kind, dim3 grid, cudaStream_t st) {
-  if (kind == 0) return launch_pdl(score_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
-  return launch_pdl(sw_kernel<T, D, G>, grid, dim3(kThreads), 0, st, a);
+cudaError_t launch_stream(DecodeArgs& a, int n_bkv, cudaStream_t st) {
+  static std::mutex s_mu;
+  static std::atomic<int> s_cs[64];  // chosen cluster size; 0 = not set up yet
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) dev = 63;
+  int cs = s_cs[dev].load(std::memory_order_acquire);
+  if (cs == 0) {
+    std::lock_guard<std::mutex> lock(s_mu);
+    cs = s_cs[dev].load(std::memory_order_relaxed);
+    if (cs == 0) {
+      cudaFuncSetAttribute(stream_kernel<T, D, G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      cudaFuncSetAttribute(stream_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(kSwCluster);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = kStreamSmem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = kSwCluster;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, stream_kernel<T, D, G>, &cfg) != cudaSuccess) n = 0;
+      cudaGetLastError();  // clear a refused query
+      cs = n > 0 ? kSwCluster : 8;
+      s_cs[dev].store(cs, std::memory_order_release);
+    }
+  }
+  a.n_score_pad = (a.n_score_ctas + cs - 1) / cs * cs;
+  const dim3 grid(a.n_score_pad + n_bkv * cs);
+  return launch_cluster_pdl(stream_kernel<T, D, G>, grid, dim3(kThreads), kStreamSmem, cs, st, a);
 }
 
 template <typename T, int D>
-cudaError_t launch_d(const DecodeArgs& a, int kind, dim3 grid, cudaStream_t st) {
+cudaError_t launch_stream_d(DecodeArgs& a, int n_bkv, cudaStream_t st) {
   switch (a.G) {
-    case 1: return launch_dg<T, D, 1>(a, kind, grid, st);
-    case 2: return launch_dg<T, D, 2>(a, kind, grid, st);
-    case 4: return launch_dg<T, D, 4>(a, kind, grid, st);
-    default: return launch_dg<T, D, 8>(a, kind, grid, st);
+    case 1: return launch_stream<T, D, 1>(a, n_bkv, st);
+    case 2: return launch_stream<T, D, 2>(a, n_bkv, st);
+    case 4: return launch_stream<T, D, 4>(a, n_bkv, st);
+    default: return launch_stream<T, D, 8>(a, n_bkv, st);
   }
 }
 
-cudaError_t launch_kind(const Shape& sh, const DecodeArgs& a, int kind, dim3 grid, cudaStream_t st) {
+cudaError_t launch_stream_any(const Shape& sh, DecodeArgs& a, cudaStream_t st) {
+  const int n_bkv = sh.B * sh.Hkv;
   if (sh.dtype == RTP_BF16)
-    return sh.D == 128 ? launch_d<__nv_bfloat16, 128>(a, kind, grid, st)
-                       : launch_d<__nv_bfloat16, 64>(a, kind, grid, st);
-  return sh.D == 128 ? launch_d<float, 128>(a, kind, grid, st) : launch_d<float, 64>(a, kind, grid, st);
+    return sh.D == 128 ? launch_stream_d<__nv_bfloat16, 128>(a, n_bkv, st)
+                       : launch_stream_d<__nv_bfloat16, 64>(a, n_bkv, st);
+  return sh.D == 128 ? launch_stream_d<float, 128>(a, n_bkv, st) : launch_stream_d<float, 64>(a, n_bkv, st);
 }
 
 // Select kernel with 16-CTA clusters when the device can keep all of this
 // call's clusters resident at once, else 8-CTA clusters (which always fit in
 // fewer SMs per GPC): one wave of clusters keeps the kernel as short as one
 // cluster's work.
+// The per-device attribute set-up and occupancy query run once per device
+// under a mutex (calls may come from several host threads); the result is
+// published through an atomic, so later calls read it without the lock.
 template <typename T, int D>
 cudaError_t launch_select(DecodeArgs& a, int n_clusters, cudaStream_t st) {
-  static int s_max16[64] = {};
-  static bool s_done[64] = {};
+  static std::mutex s_mu;
+  static std::atomic<int> s_max16[64];  // -1 - (clusters resident): 0 = not queried yet
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (dev >= 0 && dev < 64 && !s_done[dev]) {
-    cudaFuncSetAttribute(select_kernel<T, D, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<8>::kSmem);
-    cudaFuncSetAttribute(select_kernel<T, D, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<16>::kSmem);
-    cudaFuncSetAttribute(select_kernel<T, D, 16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(16, 1);
-    cfg.blockDim = dim3(kSelThreads);
-    cfg.dynamicSmemBytes = SelCfg<16>::kSmem;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 16;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, select_kernel<T, D, 16>, &cfg) != cudaSuccess) n = 0;
-    cudaGetLastError();  // clear a refused query
-    s_max16[dev] = n;
-    s_done[dev] = true;
+  if (dev < 0 || dev >= 64) dev = 63;  // out-of-range ordinals share the last slot
+  int cached = s_max16[dev].load(std::memory_order_acquire);
+  if (cached == 0) {
+    std::lock_guard<std::mutex> lock(s_mu);
+    cached = s_max16[dev].load(std::memory_order_relaxed);
+    if (cached == 0) {
+      cudaFuncSetAttribute(select_kernel<T, D, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<8>::kSmem);
+      cudaFuncSetAttribute(select_kernel<T, D, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<16>::kSmem);
+      cudaFuncSetAttribute(select_kernel<T, D, 16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(16, 1);
+      cfg.blockDim = dim3(kSelThreads);
+      cfg.dynamicSmemBytes = SelCfg<16>::kSmem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = 16;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, select_kernel<T, D, 16>, &cfg) != cudaSuccess) n = 0;
+      cudaGetLastError();  // clear a refused query
+      cached = -1 - n;
+      s_max16[dev].store(cached, std::memory_order_release);
+    }
   }
-  const int cs = (dev >= 0 && dev < 64 && s_max16[dev] >= n_clusters) ? 16 : 8;
+  const int max16 = cached < 0 ? -1 - cached : 0;
+  const int cs = (max16 >= n_clusters) ? 16 : 8;
   a.sel_cs = cs;
   if (cs == 16)
     return launch_pdl(select_kernel<T, D, 16>, dim3(16, n_clusters), dim3(kSelThreads), SelCfg<16>::kSmem, st, a);
@@ -1749,27 +1788,21 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+void arm_wait_expiry(int polls) { t_expiry_polls = polls; }
+
 DecodeLayout decode_layout(const Shape& sh) {
   DecodeLayout l;
   const size_t NRt = (size_t)sh.B * sh.NR;
   const int chunk = score_chunk(sh.esize);
   l.nch_score_max = (sh.Lmax + chunk - 1) / chunk;
-  l.n_sw_tiles = (sh.S + sh.W + kSwTile - 1) / kSwTile;
-  l.n_tiles_max = l.n_sw_tiles + (sh.R > 0 ? kMaxCS : 0);
-  l.n_ctl = (int)(2 * (size_t)sh.B * sh.Hkv);  // merge tickets, select-partial counters
   const size_t words = (size_t)(sh.Lmax + 31) / 32;
   const size_t lstride = ((size_t)sh.Lmax + 31) & ~size_t(31);
   size_t off = 0;
-  l.logits = off;   off = align256(off + NRt * lstride * sizeof(float));
-  l.cmax = off;     off = align256(off + NRt * l.nch_score_max * sizeof(float));
-  l.mask = off;     off = align256(off + NRt * words * sizeof(uint32_t));  // bitmask when the caller passes none
-  l.ctl = off;      off = align256(off + (size_t)l.n_ctl * sizeof(unsigned));
-  l.rank_cnt = off; off = align256(off + NRt * kMaxCS * sizeof(int));
-  l.cand = off;     off = align256(off + NRt * lstride * sizeof(uint2));
-  const size_t nparts = (size_t)sh.B * sh.Hkv * l.n_tiles_max * sh.G;
-  l.pm = off;       off = align256(off + nparts * sizeof(float));
-  l.pl = off;       off = align256(off + nparts * sizeof(float));
-  l.po = off;       off = align256(off + nparts * sh.D * sizeof(float));
+  l.logits = off;     off = align256(off + NRt * lstride * sizeof(float));
+  l.cmax = off;       off = align256(off + NRt * l.nch_score_max * sizeof(float));
+  l.mask = off;       off = align256(off + NRt * words * sizeof(uint32_t));  // bitmask when the caller passes none
+  l.cand = off;       off = align256(off + NRt * lstride * sizeof(uint2));
+  l.sw_part = off;    off = align256(off + (size_t)sh.B * sh.Hkv * sh.G * (sh.D + 2) * sizeof(float));
   l.total = off;
   return l;
 }
@@ -1792,40 +1825,32 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   a.cmax = reinterpret_cast<float*>(w + lay.cmax);
   a.mask = sel_bitmask ? sel_bitmask : reinterpret_cast<uint32_t*>(w + lay.mask);
   a.want_mask = sel_bitmask != nullptr;
-  a.ctl = reinterpret_cast<unsigned*>(w + lay.ctl);
-  a.rank_cnt = reinterpret_cast<int*>(w + lay.rank_cnt);
   a.cand = reinterpret_cast<uint2*>(w + lay.cand);
-  a.pm = reinterpret_cast<float*>(w + lay.pm);
-  a.pl = reinterpret_cast<float*>(w + lay.pl);
-  a.po = reinterpret_cast<float*>(w + lay.po);
-  a.n_ctl = lay.n_ctl; a.nch_score_max = lay.nch_score_max; a.n_sw_tiles = lay.n_sw_tiles;
-  a.n_parts_max = lay.n_tiles_max;
+  a.sw_part = reinterpret_cast<float*>(w + lay.sw_part);
+  a.nch_score_max = lay.nch_score_max;
   a.sel_cs = 0;
+  a.tx_extra = 0u;
+  a.wait_ns = kWaitNs;
+  if (t_expiry_polls > 0) {  // test hook: copy barriers that expect bytes that never come
+    a.tx_extra = 16u;
+    a.wait_ns = 100ull * (unsigned long long)t_expiry_polls;
+    t_expiry_polls = 0;
+  }
+  a.kv = sh.kv;
   for (int i = 0; i < kMaxRetrieval; ++i) { a.ret_head[i] = sh.ret_head[i]; a.ret_rank[i] = sh.ret_rank[i]; }
   for (int i = 0; i < 64; ++i) a.inv_freq[i] = sh.inv_freq[i];
 
   const int Lh = a.max_seq_len;
   const int chunk = score_chunk(sh.esize);
   a.n_score_ctas = sh.R > 0 ? sh.B * sh.R * ((Lh + chunk - 1) / chunk) : 0;
-  a.n_sw_ctas = sh.B * sh.Hkv * lay.n_sw_tiles;
 
-  cudaError_t e = cudaSuccess;
-  if (sh.R > 0) {
-    trace_begin(RTP_STAGE_DECODE_SCORE, st);
-    e = launch_kind(sh, a, 0, dim3(a.n_score_ctas), st);
-    trace_end(RTP_STAGE_DECODE_SCORE, st);
-    if (e == cudaSuccess) {
-      trace_begin(RTP_STAGE_DECODE_SELECT, st);
-      e = launch_select_any(sh, a, sh.B * sh.NR, st);
-      trace_end(RTP_STAGE_DECODE_SELECT, st);
-    }
-  } else {
-    e = cudaMemsetAsync(a.ctl, 0, (size_t)a.n_ctl * sizeof(unsigned), st);
-  }
-  if (e == cudaSuccess) {
-    trace_begin(RTP_STAGE_DECODE_LOCAL, st);
-    e = launch_kind(sh, a, 1, dim3(a.n_sw_ctas), st);
-    trace_end(RTP_STAGE_DECODE_LOCAL, st);
+  trace_begin(RTP_STAGE_DECODE_STREAM, st);
+  cudaError_t e = launch_stream_any(sh, a, st);
+  trace_end(RTP_STAGE_DECODE_STREAM, st);
+  if (e == cudaSuccess && sh.R > 0) {
+    trace_begin(RTP_STAGE_DECODE_SELECT, st);
+    e = launch_select_any(sh, a, sh.B * sh.NR, st);
+    trace_end(RTP_STAGE_DECODE_SELECT, st);
   }
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {

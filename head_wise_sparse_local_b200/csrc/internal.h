@@ -18,8 +18,30 @@ void set_error(const std::string& msg);
 void trace_begin(int stage, cudaStream_t st);
 void trace_end(int stage, cudaStream_t st);
 
+// Where row `pos` of KV head h of sequence b sits in the K and V buffers.
+// Per sequence the heads are stored one after another, head h taking
+// cap(h) rows starting at row0[h]: the whole context (Lmax rows) for
+// retrieval heads, and for local heads either the whole context as well or,
+// in ring mode, the S sinks followed by a ring of `ring` window rows (position
+// pos >= S in slot S + (pos - S) mod ring).  Plain data, passed to kernels.
+struct KvMap {
+  long long rows_per_seq;
+  int row0[64];
+  uint64_t ring_mask;  // bit h: head h keeps sinks + a window ring
+  int ring, S;
+#ifdef __CUDACC__
+  __host__ __device__ __forceinline__ size_t row(int b, int h, int pos) const {
+    int slot = pos;
+    if ((ring_mask >> h) & 1ull) slot = pos < S ? pos : S + (pos - S) % ring;
+    return (size_t)b * (size_t)rows_per_seq + (size_t)row0[h] + (size_t)slot;
+  }
+#endif
+};
+
 struct Shape {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W;
+  int ring;          // window rows a local head keeps in ring mode (0: whole context)
+  KvMap kv;
   float top_p, rope_base;
   int dtype;  // rtp_dtype
   int esize;  // bytes per element
@@ -33,11 +55,15 @@ int make_shape(const rtp_layer_cfg* cfg, Shape* sh);
 
 // Decode scratch layout (byte offsets into the workspace).
 struct DecodeLayout {
-  size_t logits, cmax, mask, ctl, rank_cnt, cand, pm, pl, po, total;
-  int nch_score_max, n_sw_tiles, n_tiles_max;
-  int n_ctl;  // u32 control words
+  size_t logits, cmax, mask, cand, sw_part, total;
+  int nch_score_max;
 };
 DecodeLayout decode_layout(const Shape& sh);
+
+// Test hook behind rtp_debug_wait_expiry: the next decode call on this host
+// thread waits on copy barriers that expect bytes that never come, giving up
+// after `polls` x 100 ns.
+void arm_wait_expiry(int polls);
 
 int launch_append(const Shape& sh, const rtp_cache* cache, const void* k_pre, const void* v_in,
                   const int* start_pos, int T, const float* w_k, cudaStream_t st);
@@ -48,6 +74,7 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
 
 struct PrefillLayout {
   size_t total;
+  int block_rows;  // query rows per selection + attention pass
 };
 PrefillLayout prefill_layout(const Shape& sh, int T);
 int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* start_pos,

@@ -51,7 +51,10 @@ struct PrefillArgs {
   float* sel_tau;
   int* sel_jcut;
   int* sel_count;
-  uint32_t* mask;  // [B][NR][T][words] top-p bitmask per query row
+  uint32_t* mask;  // [B][NR][mask_rows][words] top-p bitmask of rows [mask_t0, mask_t0 + mask_rows)
+  int t_base, t_end;         // this launch's query rows [t_base, t_end) of the chunk
+  int mask_t0, mask_rows;
+  KvMap kv;
   int ret_head[kMaxRetrieval];
   int ret_rank[kMaxRetrieval];
   double inv_freq[64];  // RoPE frequencies, k < D/2
@@ -211,15 +214,15 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
   const int b = bh / a.NR, hh = bh % a.NR;
   const int r = hh / a.G, g = hh % a.G;
   const int h = a.ret_head[r];
-  const int t = blockIdx.x * kSelRows + warp;
+  const int t = a.t_base + blockIdx.x * kSelRows + warp;
   const int start = a.start_pos[b];
   if (start < 0 || start + a.T > a.Lmax) {
     if (threadIdx.x == 0 && blockIdx.x == 0 && hh == 0) atomicOr(a.status, RTP_DEV_POSITION);
     return;  // uniform over the CTA
   }
-  const bool row_ok = t < a.T;
+  const bool row_ok = t < a.t_end;
   const int i = start + t;  // query position; keys [0, i]
-  const int i_last = start + min(a.T, (int)(blockIdx.x + 1) * kSelRows) - 1;
+  const int i_last = start + min(a.t_end, a.t_base + (int)(blockIdx.x + 1) * kSelRows) - 1;
 
   // q~ = W_q q_pre with the decode path's association: four quarter sums of
   // D/4 dims each, then butterfly adds.
@@ -291,7 +294,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
   __syncwarp();
   const RowSel& R = s_rs[warp];
   const __nv_bfloat16* kidx = static_cast<const __nv_bfloat16*>(a.kidx) + ((size_t)b * a.R + r) * a.Lmax * kIdxDim;
-  uint32_t* mrow = a.mask + (((size_t)b * a.NR + hh) * a.T + (row_ok ? t : 0)) * a.words;
+  uint32_t* mrow = a.mask + (((size_t)b * a.NR + hh) * a.mask_rows + (row_ok ? t - a.mask_t0 : 0)) * a.words;
 
   // pass accumulators
   unsigned long long pm[8];
@@ -727,7 +730,7 @@ struct AttnSmem {
 };
 
 template <int D>
-__global__ void __launch_bounds__(128, 3) attn_rows_kernel(PrefillArgs a) {
+__global__ void __launch_bounds__(128, 3) attn_rows_kernel(const __grid_constant__ PrefillArgs a) {
   constexpr int ST = AttnSmem<D>::kStride;
   constexpr int KS = D / 16;  // k-steps of Q K^T
   constexpr int NO = D / 8;   // n8 tiles of the output
@@ -742,7 +745,7 @@ __global__ void __launch_bounds__(128, 3) attn_rows_kernel(PrefillArgs a) {
   const int r = a.ret_rank[h];
   const int start = a.start_pos[b];
   if (start < 0 || start + a.T > a.Lmax) return;  // flagged by the selection kernel / host
-  const int t0 = blockIdx.x * kBQ;
+  const int t0 = a.t_base + blockIdx.x * kBQ;
   const int hh = r >= 0 ? r * a.G + g : 0;
 
   // ---- Q tile: RoPE at each row's position, scaled by log2(e)/sqrt(D), bf16 ----
@@ -751,7 +754,7 @@ __global__ void __launch_bounds__(128, 3) attn_rows_kernel(PrefillArgs a) {
     const int rr = e / (D / 2), kk = e % (D / 2);
     const int t = t0 + rr;
     float y1 = 0.f, y2 = 0.f;
-    if (t < a.T) {
+    if (t < a.t_end) {
       const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q_pre) + (((size_t)b * a.T + t) * a.Hq + hq) * D;
       const float x1 = __bfloat162float(q[kk]), x2 = __bfloat162float(q[kk + D / 2]);
       float c, sn;
@@ -778,25 +781,25 @@ __global__ void __launch_bounds__(128, 3) attn_rows_kernel(PrefillArgs a) {
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
     ti[x] = t0 + warp * 16 + gq + 8 * x;
-    rv[x] = ti[x] < a.T;
+    rv[x] = ti[x] < a.t_end;
     pi[x] = start + ti[x];
     wlo[x] = pi[x] - a.W + 1;  // window: keys >= wlo
   }
-  const int t_last = min(a.T, t0 + kBQ) - 1;
+  const int t_last = min(a.t_end, t0 + kBQ) - 1;
   const int i_max = start + t_last;
   const int i_min = start + t0;
   const uint32_t* mrow[2];
 #pragma unroll
   for (int x = 0; x < 2; ++x)
-    mrow[x] = a.mask + (((size_t)b * a.NR + hh) * a.T + (rv[x] ? ti[x] : 0)) * a.words;
+    mrow[x] = a.mask + (((size_t)b * a.NR + hh) * a.mask_rows + (rv[x] ? ti[x] - a.mask_t0 : 0)) * a.words;
 
   float o[NO][4];
 #pragma unroll
   for (int n = 0; n < NO; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
   float mrun[2] = {-CUDART_INF_F, -CUDART_INF_F}, lrun[2] = {0.f, 0.f};
 
-  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
-  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v) + ((size_t)b * a.Hkv + h) * a.Lmax * D;
+  const __nv_bfloat16* kg = static_cast<const __nv_bfloat16*>(a.k);
+  const __nv_bfloat16* vg = static_cast<const __nv_bfloat16*>(a.v);
 
   // Key tiles in order, local heads jumping from the sinks to the first window
   // tile; each tile's K, V (cp.async, rows past the chunk zero-filled) and
@@ -813,12 +816,12 @@ __global__ void __launch_bounds__(128, 3) attn_rows_kernel(PrefillArgs a) {
       const int kr = e / (D / 8), c8 = e % (D / 8);
       const int j = kt_ + kr;
       const unsigned sz = j <= i_max ? 16u : 0u;  // 0: zero fill
-      const int jj = j <= i_max ? j : 0;
+      const size_t row = a.kv.row(b, h, j <= i_max ? j : 0);
       const unsigned off = (unsigned)((kr * ST + c8 * 8) * sizeof(__nv_bfloat16));
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dk + off),
-                   "l"(kg + (size_t)jj * D + c8 * 8), "r"(sz));
+                   "l"(kg + row * D + c8 * 8), "r"(sz));
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dv + off),
-                   "l"(vg + (size_t)jj * D + c8 * 8), "r"(sz));
+                   "l"(vg + row * D + c8 * 8), "r"(sz));
     }
     asm volatile("cp.async.commit_group;" ::: "memory");
   };
@@ -967,17 +970,32 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
 
+// Rows whose top-p bitmask the workspace holds at once: the whole chunk when
+// that stays under kMaskBudget, else blocks of a multiple of the attention
+// tile (the chunk then runs block by block: selection, attention, next block).
+constexpr size_t kMaskBudget = size_t(1) << 30;
+
+int prefill_block_rows(const Shape& sh, int T) {
+  const size_t words = (size_t)(sh.Lmax + 31) / 32;
+  const size_t per_row = (size_t)sh.B * (size_t)(sh.NR > 0 ? sh.NR : 1) * words * sizeof(uint32_t);
+  size_t rows = kMaskBudget / per_row;
+  if (rows >= (size_t)T) return T;
+  rows = rows / kBQ * kBQ;
+  return rows < (size_t)kBQ ? kBQ : (int)rows;
+}
+
 PrefillLayout prefill_layout(const Shape& sh, int T) {
   PrefillLayout l;
   const size_t words = (size_t)(sh.Lmax + 31) / 32;
-  l.total = align256((size_t)sh.B * sh.NR * T * words * sizeof(uint32_t)) + 256;
+  const int rows = prefill_block_rows(sh, T);
+  l.block_rows = rows;
+  l.total = align256((size_t)sh.B * sh.NR * rows * words * sizeof(uint32_t)) + 256;
   return l;
 }
 
 int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* start_pos,
                    int T, const float* w_q, void* out, uint32_t* sel_bitmask, float* sel_tau,
                    int* sel_jcut, int* sel_count, void* ws, const PrefillLayout& lay, cudaStream_t st) {
-  (void)lay;
   if (sh.dtype != RTP_BF16) {
     set_error("rtp_prefill_attn: the prefill path computes in bf16 (dtype must be RTP_BF16)");
     return RTP_ERR_DTYPE;
@@ -991,6 +1009,7 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
   a.start_pos = start_pos;
   a.sel_tau = sel_tau; a.sel_jcut = sel_jcut; a.sel_count = sel_count;
   a.mask = sel_bitmask ? sel_bitmask : static_cast<uint32_t*>(ws);
+  a.kv = sh.kv;
   for (int i = 0; i < kMaxRetrieval; ++i) { a.ret_head[i] = sh.ret_head[i]; a.ret_rank[i] = sh.ret_rank[i]; }
   for (int i = 0; i < 64; ++i) a.inv_freq[i] = sh.inv_freq[i];
 
@@ -1006,18 +1025,27 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
     cudaFuncSetAttribute(select_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDynSmem);
     s_attr[dev] = true;
   }
-  if (sh.R > 0) {
-    const dim3 gs((T + kSelRows - 1) / kSelRows, sh.B * sh.NR);
-    trace_begin(RTP_STAGE_PREFILL_INDEX, st);
-    if (sh.D == 128) select_rows_kernel<128><<<gs, kSelRows * 32, kSelDynSmem, st>>>(a);
-    else select_rows_kernel<64><<<gs, kSelRows * 32, kSelDynSmem, st>>>(a);
-    trace_end(RTP_STAGE_PREFILL_INDEX, st);
+  // The caller's bitmask holds every row; the workspace one block of rows.
+  const int blk = sel_bitmask ? T : lay.block_rows;
+  for (int t_base = 0; t_base < T; t_base += blk) {
+    a.t_base = t_base;
+    a.t_end = min(T, t_base + blk);
+    a.mask_t0 = sel_bitmask ? 0 : t_base;
+    a.mask_rows = sel_bitmask ? T : blk;
+    const int n = a.t_end - t_base;
+    if (sh.R > 0) {
+      const dim3 gs((n + kSelRows - 1) / kSelRows, sh.B * sh.NR);
+      trace_begin(RTP_STAGE_PREFILL_INDEX, st);
+      if (sh.D == 128) select_rows_kernel<128><<<gs, kSelRows * 32, kSelDynSmem, st>>>(a);
+      else select_rows_kernel<64><<<gs, kSelRows * 32, kSelDynSmem, st>>>(a);
+      trace_end(RTP_STAGE_PREFILL_INDEX, st);
+    }
+    const dim3 ga((n + kBQ - 1) / kBQ, sh.B * sh.Hq);
+    trace_begin(RTP_STAGE_PREFILL_ATTN, st);
+    if (sh.D == 128) attn_rows_kernel<128><<<ga, 128, AttnSmem<128>::kBytes, st>>>(a);
+    else attn_rows_kernel<64><<<ga, 128, AttnSmem<64>::kBytes, st>>>(a);
+    trace_end(RTP_STAGE_PREFILL_ATTN, st);
   }
-  const dim3 ga((T + kBQ - 1) / kBQ, sh.B * sh.Hq);
-  trace_begin(RTP_STAGE_PREFILL_ATTN, st);
-  if (sh.D == 128) attn_rows_kernel<128><<<ga, 128, AttnSmem<128>::kBytes, st>>>(a);
-  else attn_rows_kernel<64><<<ga, 128, AttnSmem<64>::kBytes, st>>>(a);
-  trace_end(RTP_STAGE_PREFILL_ATTN, st);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("prefill launch: ") + cudaGetErrorString(e));

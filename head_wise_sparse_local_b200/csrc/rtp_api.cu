@@ -89,6 +89,24 @@ int make_shape(const rtp_layer_cfg* cfg, Shape* sh) {
   }
   sh->R = r;
   sh->NR = r * G;
+  if (cfg->local_cap < 0) return fail(RTP_ERR_INVALID, "local_cap must be >= 0");
+  if (cfg->local_cap > 0 && cfg->local_cap < cfg->window)
+    return fail(RTP_ERR_SHAPE, "local_cap must be 0 or at least the window");
+  // ring mode only when it actually saves rows
+  sh->ring = (cfg->local_cap > 0 && (long long)sh->S + cfg->local_cap < (long long)sh->Lmax) ? cfg->local_cap : 0;
+  sh->kv.ring = sh->ring > 0 ? sh->ring : 1;
+  sh->kv.S = sh->S;
+  sh->kv.ring_mask = 0ull;
+  long long rows = 0;
+  for (int h = 0; h < 64; ++h) sh->kv.row0[h] = 0;
+  for (int h = 0; h < sh->Hkv; ++h) {
+    sh->kv.row0[h] = (int)rows;
+    const bool ring = sh->ring > 0 && sh->ret_rank[h] < 0;
+    if (ring) sh->kv.ring_mask |= 1ull << h;
+    rows += ring ? (long long)sh->S + sh->ring : sh->Lmax;
+  }
+  if (rows > INT32_MAX) return fail(RTP_ERR_SHAPE, "cache rows per sequence exceed 2^31");
+  sh->kv.rows_per_seq = rows;
   for (int k = 0; k < 64; ++k)
     sh->inv_freq[k] = k < sh->D / 2 ? std::pow((double)sh->rope_base, -2.0 * k / (double)sh->D) : 0.0;
   return RTP_OK;
@@ -126,12 +144,17 @@ int rtp_trace_stage(int stage, void* start_event, void* stop_event) {
   return RTP_OK;
 }
 
+int rtp_debug_wait_expiry(int polls) {
+  arm_wait_expiry(polls > 0 ? polls : 0);
+  return RTP_OK;
+}
+
 int rtp_cache_bytes(const rtp_layer_cfg* cfg, size_t* k_bytes, size_t* v_bytes,
                     size_t* kidx_bytes) {
   Shape sh;
   int rc = make_shape(cfg, &sh);
   if (rc != RTP_OK) return rc;
-  const size_t kv = (size_t)sh.B * sh.Hkv * sh.Lmax * sh.D * sh.esize;
+  const size_t kv = (size_t)sh.B * (size_t)sh.kv.rows_per_seq * sh.D * sh.esize;
   if (k_bytes) *k_bytes = kv;
   if (v_bytes) *v_bytes = kv;
   if (kidx_bytes) *kidx_bytes = (size_t)sh.B * sh.R * sh.Lmax * 16 * sh.esize;
@@ -204,6 +227,8 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
   if (rc != RTP_OK) return rc;
   if ((rc = check_cache(sh, cache)) != RTP_OK) return rc;
   if (T < 1 || T > sh.Lmax) return fail(RTP_ERR_SHAPE, "T must be in [1, max_ctx]");
+  if (sh.ring > 0 && (long long)T + sh.W - 1 > sh.ring)
+    return fail(RTP_ERR_SHAPE, "ring mode: a prefill chunk needs local_cap >= T + window - 1");
   if (!q_pre || !start_pos || !out) return fail(RTP_ERR_INVALID, "q_pre/start_pos/out is NULL");
   if (sh.R > 0 && !w_q) return fail(RTP_ERR_INVALID, "w_q is NULL with retrieval heads");
   if (!aligned16(q_pre) || (w_q && !aligned16(w_q)))

@@ -76,6 +76,13 @@ typedef enum rtp_dtype { RTP_BF16 = 0, RTP_FP32 = 1 } rtp_dtype;
  *   retrieval_mask bit h set => KV head h is a retrieval head.  Retrieval
  *                 heads are ranked r = 0..R-1 in increasing h; R <= 64
  *   dtype         rtp_dtype of q, k, v, out and the caches
+ *   local_cap     0: every KV head keeps the whole context in the cache.
+ *                 > 0 (ring mode, at least `window`): local heads keep only
+ *                 the S sinks and a ring of local_cap window rows, so the cache
+ *                 holds the full context only for retrieval heads (abstract:
+ *                 the full KV cache is kept for retrieval heads only).  A
+ *                 prefill chunk of T tokens then needs local_cap >= T + W - 1.
+ *                 Ignored (whole context kept) when S + local_cap >= max_ctx.
  */
 typedef struct rtp_layer_cfg {
   int batch;
@@ -90,12 +97,18 @@ typedef struct rtp_layer_cfg {
   float rope_base;
   uint64_t retrieval_mask;
   int dtype;
+  int local_cap;
 } rtp_layer_cfg;
 
 /* The layer's cache (device memory owned by the caller; sizes from
  * rtp_cache_bytes):
  *   k       [B][Hkv][Lmax][D]  keys after RoPE at their own position
  *   v       [B][Hkv][Lmax][D]  values
+ *           In ring mode (cfg->local_cap > 0) k and v are [B][rows][D]: per
+ *           sequence the KV heads follow one another in order h = 0..Hkv-1,
+ *           a retrieval head taking Lmax rows (position j in row j) and a local
+ *           head S + local_cap rows (position j < S in row j, position j >= S
+ *           in row S + (j - S) mod local_cap).
  *   kidx    [B][R][Lmax][16]   16-d indexer keys k~ = W_k k_pre, one row per
  *                              token for each retrieval KV head (pre-RoPE)
  *   status  one int of device-side error bits (see RTP_DEV_*), zeroed by the
@@ -164,6 +177,13 @@ int rtp_append_kv(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* 
  *                contents need no initialisation and are clobbered
  * A sequence with an invalid seq_len is skipped (its out rows untouched) and
  * sets RTP_DEV_SEQ_LEN.
+ * q_pre, w_q and seq_len are read before the kernels wait for the work already
+ * on the stream (only the cache reads wait): they must not be written by a
+ * kernel that may still be running when this call's kernels start, such as an
+ * earlier kernel launched with programmatic dependent launch.
+ * Two bounded waits inside the call (for the step's indexer scores and for
+ * each head's sink/window partial) give up after about 0.4 s; the call's output
+ * is then invalid and RTP_DEV_TIMEOUT is set.
  */
 int rtp_decode_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
                     const int* seq_len, int max_seq_len, const float* w_q, void* out,
@@ -192,7 +212,8 @@ int rtp_decode_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void
  *     overlaps (several streams or threads) race on it: serialise them.
  *   - The first call on each device looks up the array's device address with
  *     that device current and caches it; make that first call before any
- *     stream capture.
+ *     stream capture.  The cached address is not looked up again: do not use
+ *     this entry point after a cudaDeviceReset in the same process.
  */
 int rtp_decode_attn_noalloc(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
                             const int* seq_len, int max_seq_len, const float* w_q, void* out,
@@ -203,11 +224,15 @@ int rtp_decode_attn_noalloc(const rtp_layer_cfg* cfg, const rtp_cache* cache, co
  * must already be in the cache (rtp_append_kv with the same start_pos and T).
  * Per row the layer computes exactly what rtp_decode_attn computes for a
  * query at position i (top-p over the indexer scores of [0, i] for retrieval
- * query heads; sinks and window [i-W+1, i] for every head); the indexer
- * scores use the same fp32 arithmetic as rtp_decode_attn, so a row's top-p
- * set equals the decode step's at that position.  The attention itself runs
- * on tensor cores in bf16 with fp32 accumulation (atlas.scime.ai summary,
- * "Approach"; abstract, observations (2)-(3)).  cfg->dtype must be RTP_BF16.
+ * query heads; sinks and window [i-W+1, i] for every head).  The indexer
+ * scores are computed on tensor cores from q~ split into a bf16 high part and
+ * a bf16 low part, with fp32 accumulation: they equal the fp32 score of
+ * rtp_decode_attn to about 2^-17 of the score, not bit for bit.  A row's
+ * top-p set can therefore differ from the decode step's at that position, but
+ * only in tokens at the cut (within the 1e-6 probability tolerance of the
+ * parity tests).  The attention itself runs on tensor cores in bf16 with fp32
+ * accumulation (atlas.scime.ai summary, "Approach"; abstract, observations
+ * (2)-(3)).  cfg->dtype must be RTP_BF16.
  *
  *   q_pre        [B][T][Hq][D] bf16, device
  *   start_pos    [B] int32, device; 0 <= start_pos[b] and start_pos[b] + T <= max_ctx
@@ -223,7 +248,12 @@ int rtp_decode_attn_noalloc(const rtp_layer_cfg* cfg, const rtp_cache* cache, co
  *                iff their index <= sel_jcut (so membership is
  *                s_j > tau || (s_j == tau && j <= jcut))
  *   sel_count    optional [B][R*G][T] int32: size of the row's top-p set
- *   workspace    >= rtp_prefill_workspace_bytes(cfg, T), 256-byte aligned
+ *   workspace    >= rtp_prefill_workspace_bytes(cfg, T), 256-byte aligned.  It
+ *                holds a per-row top-p bitmask for a block of rows at a time;
+ *                the block is sized so the workspace stays under 1 GiB, and
+ *                longer chunks run block by block.
+ * Ring mode (cfg->local_cap > 0) needs local_cap >= T + W - 1, else
+ * RTP_ERR_SHAPE.
  */
 int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
                      const int* start_pos, int T, const float* w_q, void* out,
@@ -233,12 +263,11 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
 /* Kernel stages, for rtp_trace_stage. */
 typedef enum rtp_stage {
   RTP_STAGE_APPEND = 0,         /* rtp_append_kv: RoPE + cache + indexer-key store */
-  RTP_STAGE_DECODE_SCORE = 1,   /* decode: indexer scores over the 16-d key cache */
-  RTP_STAGE_DECODE_SELECT = 2,  /* decode: exact top-p selection, bitmask, kept-row attention */
-  RTP_STAGE_DECODE_LOCAL = 3,   /* decode: sink/window attention (overlaps the selection) + merge */
-  RTP_STAGE_PREFILL_INDEX = 4,  /* prefill: per-row exact top-p selection */
-  RTP_STAGE_PREFILL_ATTN = 5,   /* prefill: masked causal attention */
-  RTP_STAGE_COUNT = 6
+  RTP_STAGE_DECODE_STREAM = 1,  /* decode: indexer scores + sink/window attention (one grid) */
+  RTP_STAGE_DECODE_SELECT = 2,  /* decode: exact top-p selection, bitmask, kept-row attention, merge */
+  RTP_STAGE_PREFILL_INDEX = 3,  /* prefill: per-row exact top-p selection */
+  RTP_STAGE_PREFILL_ATTN = 4,   /* prefill: masked causal attention */
+  RTP_STAGE_COUNT = 5
 } rtp_stage;
 
 /* Host.  Optional instrumentation (no work is skipped or added).  Arms a
@@ -247,9 +276,17 @@ typedef enum rtp_stage {
  * cudaEventRecord(stop_event) on its launch stream.  Events are cudaEvent_t
  * passed as void*, created and owned by the caller (with timing enabled to
  * read cudaEventElapsedTime).  A stage launched several times by one call
- * (none today) records around its first launch.  NULL events disarm the stage.
- * Returns RTP_ERR_INVALID for an unknown stage. */
+ * (prefill chunks longer than one row block) records around its first launch.
+ * NULL events disarm the stage.  Returns RTP_ERR_INVALID for an unknown stage. */
 int rtp_trace_stage(int stage, void* start_event, void* stop_event);
+
+/* Host.  Test hook for the bounded waits of rtp_decode_attn (no counterpart
+ * in the paper).  Arms the next rtp_decode_attn call on this host thread to
+ * wait for completion flags that never reach the awaited value, giving up
+ * after `polls` polls (about 100 ns each): the call then sets RTP_DEV_TIMEOUT,
+ * its output is invalid, and the GPU stays usable.  polls <= 0 disarms.
+ * Returns RTP_OK. */
+int rtp_debug_wait_expiry(int polls);
 
 /* Host.  Message for the last non-OK return on this thread ("" if none). */
 const char* rtp_last_error(void);

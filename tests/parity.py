@@ -9,6 +9,10 @@ within 1e-6 of p, the two cuts may differ by one token.
 Outputs: |gpu - oracle| <= atol + rtol * |oracle| with (2e-2, 1e-2) for bf16
 and (1e-5, 1e-5) for fp32, against the oracle evaluated on the GPU's own kept
 set (identical to the oracle's own set whenever the selections agree).
+
+Every decode parity check also repeats the call without a bitmask (the call
+the benchmark times, whose tail reads only the top-rung items when it can) and
+holds its kept counts and its output to the same oracle reference.
 """
 
 from __future__ import annotations
@@ -63,25 +67,61 @@ def oracle_cache_from_inputs(inp) -> OracleCache:
     return c
 
 
-def run_gpu_decode(inp, top_p=None, append_last_separately=True, with_bitmask=True):
+def append_context(lay, inp, w_k, n_rows=None, dev="cuda"):
+    """Append each sequence's context rows [0, n_rows[b]) (default seq_len[b])
+    to the layer's cache.  In ring mode every sequence is appended on its own
+    (a batch-1 view of its cache slice), so rows past its own length never
+    take ring slots of its window."""
+    import head_wise_sparse_local_b200 as rtp
+    sh = inp["shape"]
+    n_rows = inp["seq_len"] if n_rows is None else n_rows
+    if not lay.ring:
+        T = int(max(n_rows))
+        lay.append(inp["k_pre"][:, :T].contiguous().to(dev), inp["v"][:, :T].contiguous().to(dev),
+                   torch.zeros(sh.batch, dtype=torch.int32, device=dev), w_k)
+        return
+    c = lay.cfg
+    cfg1 = rtp.rtp_layer_cfg(1, c.n_q_heads, c.n_kv_heads, c.head_dim, c.idx_dim, c.max_ctx, c.n_sink,
+                             c.window, c.top_p, c.rope_base, c.retrieval_mask, c.dtype, c.local_cap)
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    for b in range(sh.batch):
+        L = int(n_rows[b])
+        cache1 = rtp.rtp_cache(lay.k[b].data_ptr(), lay.v[b].data_ptr(), lay.kidx[b].data_ptr(),
+                               lay.status.data_ptr())
+        kp = inp["k_pre"][b:b + 1, :L].contiguous().to(dev)
+        vv = inp["v"][b:b + 1, :L].contiguous().to(dev)
+        rtp.rtp_append_kv(cfg1, cache1, kp, vv, zero, L, w_k)
+        torch.cuda.synchronize()
+
+
+def run_gpu_decode(inp, top_p=None, append_last_separately=True, with_bitmask=True,
+                   also_timed_path=False, local_cap=0, ws_fill=None):
     """Fill a device cache with the context, append the decode token, decode.
 
     Returns dict(out [B,Hq,D] float64 numpy, bitmask, count, status, layer);
-    with_bitmask=False passes no bitmask (bitmask None in the result)."""
+    with_bitmask=False passes no bitmask (bitmask None in the result).
+    also_timed_path=True repeats the call without a bitmask on the same cache
+    (the call the benchmark times) and adds out_timed / count_timed.
+    local_cap > 0 runs the cache in ring mode; ws_fill fills the decode
+    workspace with that byte first (it needs no initialisation)."""
     from head_wise_sparse_local_b200 import Layer
     sh = inp["shape"]
     if top_p is not None:
         sh = sh.replace(top_p=top_p)
     dev = torch.device("cuda")
     Lmax = inp["max_ctx"]
-    lay = Layer(sh, Lmax, device=dev)
+    lay = Layer(sh, Lmax, device=dev, local_cap=local_cap)
+    if ws_fill is not None:
+        lay.ws_decode.fill_(ws_fill)
     k_pre = inp["k_pre"].to(dev)
     v = inp["v"].to(dev)
     w_q = inp["w_q"].to(dev)
     w_k = inp["w_k"].to(dev)
     seq = torch.from_numpy(inp["seq_len"]).to(dev)
-    start0 = torch.zeros(sh.batch, dtype=torch.int32, device=dev)
-    lay.append(k_pre, v, start0, w_k)
+    if lay.ring:
+        append_context(lay, inp, w_k, dev=dev)
+    else:
+        lay.append(k_pre, v, torch.zeros(sh.batch, dtype=torch.int32, device=dev), w_k)
     if append_last_separately:
         # re-append each sequence's last token as a decode step would (T = 1)
         last = (seq - 1).to(torch.int32)
@@ -98,16 +138,25 @@ def run_gpu_decode(inp, top_p=None, append_last_separately=True, with_bitmask=Tr
     cnt = torch.full((sh.batch, max(NR, 1)), -1, dtype=torch.int32, device=dev)
     if not with_bitmask:
         bm = None
-    lay.decode(q, seq, w_q, out, max_seq_len=int(inp["seq_len"].max()), sel_bitmask=bm, sel_count=cnt)
+    Lh = int(inp["seq_len"].max())
+    lay.decode(q, seq, w_q, out, max_seq_len=Lh, sel_bitmask=bm, sel_count=cnt)
+    res = dict(out=out.double().cpu().numpy(), bitmask=bm, count=cnt.cpu().numpy(), layer=lay, shape=sh)
+    if with_bitmask and also_timed_path:
+        # the call the benchmark times: no bitmask, kept counts only
+        out2 = torch.empty_like(out)
+        cnt2 = torch.full_like(cnt, -1)
+        lay.decode(q, seq, w_q, out2, max_seq_len=Lh, sel_bitmask=None, sel_count=cnt2)
+        res["out_timed"] = out2.double().cpu().numpy()
+        res["count_timed"] = cnt2.cpu().numpy()
     torch.cuda.synchronize()
-    return dict(out=out.double().cpu().numpy(), bitmask=bm, count=cnt.cpu().numpy(),
-                status=lay.device_status(), layer=lay, shape=sh)
+    res["status"] = lay.device_status()
+    return res
 
 
-def check_decode_parity(inp, top_p=None, oc=None):
+def check_decode_parity(inp, top_p=None, oc=None, local_cap=0):
     """Full parity check of one decode step; returns stats."""
     sh = inp["shape"] if top_p is None else inp["shape"].replace(top_p=top_p)
-    g = run_gpu_decode(inp, top_p)
+    g = run_gpu_decode(inp, top_p, also_timed_path=True, local_cap=local_cap)
     assert g["status"] == 0, f"device status {g['status']}"
     oc = oc or oracle_cache_from_inputs(inp)
     oc.shape = sh
@@ -143,14 +192,23 @@ def check_decode_parity(inp, top_p=None, oc=None):
     lim = atol + rtol * np.abs(ref)
     worst = float((err / lim).max())
     assert np.all(err <= lim), f"output mismatch: max err {err.max():.3e}, worst ratio {worst:.3f}"
-    return dict(heads=n_heads, exact=n_exact, diff_tokens=n_diff_tok, worst_ratio=worst,
-                max_abs_err=float(err.max()), counts=g["count"])
+    # The timed call (no bitmask) runs the same selection: its kept counts must
+    # equal the bitmask call's set sizes, and its output must match the oracle
+    # on that set directly (not only through the bitmask call).
+    assert np.array_equal(g["count_timed"], g["count"]), (g["count_timed"], g["count"])
+    err_t = np.abs(g["out_timed"] - ref)
+    worst_t = float((err_t / lim).max())
+    assert np.all(err_t <= lim), f"timed-path output mismatch: max err {err_t.max():.3e}, worst {worst_t:.3f}"
+    return dict(heads=n_heads, exact=n_exact, diff_tokens=n_diff_tok, worst_ratio=max(worst, worst_t),
+                max_abs_err=float(max(err.max(), err_t.max())), counts=g["count"])
 
 
-def run_gpu_prefill(inp, top_p=None):
+def run_gpu_prefill(inp, top_p=None, local_cap=0, with_bitmask=True):
     """Append the context and the chunk, then run one prefill over the chunk.
 
-    Returns out [B, T, Hq, D] float64, bitmask [B, NR, T, words], count [B, NR, T]."""
+    Returns out [B, T, Hq, D] float64, bitmask [B, NR, T, words], count [B, NR, T].
+    local_cap > 0 runs the cache in ring mode (the context before the chunk
+    and the chunk are appended separately, as a serving loop would)."""
     from head_wise_sparse_local_b200 import Layer
     sh = inp["shape"]
     if top_p is not None:
@@ -158,16 +216,25 @@ def run_gpu_prefill(inp, top_p=None):
     dev = torch.device("cuda")
     Lmax = inp["max_ctx"]
     T = inp["T"]
-    lay = Layer(sh, Lmax, device=dev, prefill_T=T)
+    lay = Layer(sh, Lmax, device=dev, prefill_T=T, local_cap=local_cap)
     start = torch.from_numpy(inp["start_pos"]).to(dev)
     n_ctx = int(inp["start_pos"].max()) + T
-    lay.append(inp["k_pre"][:, :n_ctx].contiguous().to(dev), inp["v"][:, :n_ctx].contiguous().to(dev),
-               torch.zeros(sh.batch, dtype=torch.int32, device=dev), inp["w_k"].to(dev))
+    w_k = inp["w_k"].to(dev)
+    if lay.ring:
+        s0 = int(inp["start_pos"][0])
+        assert np.all(inp["start_pos"] == s0)
+        if s0 > 0:
+            append_context(lay, inp, w_k, n_rows=np.full(sh.batch, s0), dev=dev)
+        lay.append(inp["k_pre"][:, s0:n_ctx].contiguous().to(dev), inp["v"][:, s0:n_ctx].contiguous().to(dev),
+                   start, w_k)
+    else:
+        lay.append(inp["k_pre"][:, :n_ctx].contiguous().to(dev), inp["v"][:, :n_ctx].contiguous().to(dev),
+                   torch.zeros(sh.batch, dtype=torch.int32, device=dev), w_k)
     q = inp["q_pre"].to(dev)
     out = torch.empty((sh.batch, T, sh.n_q_heads, sh.head_dim), dtype=sh.torch_dtype, device=dev)
     NR = max(sh.n_retrieval * sh.group, 1)
     words = (Lmax + 31) // 32
-    bm = torch.zeros((sh.batch, NR, T, words), dtype=torch.int32, device=dev)
+    bm = torch.zeros((sh.batch, NR, T, words), dtype=torch.int32, device=dev) if with_bitmask else None
     cnt = torch.full((sh.batch, NR, T), -1, dtype=torch.int32, device=dev)
     tau = torch.zeros((sh.batch, NR, T), dtype=torch.float32, device=dev)
     jcut = torch.zeros((sh.batch, NR, T), dtype=torch.int32, device=dev)
@@ -179,11 +246,11 @@ def run_gpu_prefill(inp, top_p=None):
                 layer=lay, shape=sh)
 
 
-def check_prefill_parity(inp, rows=None, top_p=None, g=None):
+def check_prefill_parity(inp, rows=None, top_p=None, g=None, local_cap=0):
     """Selection sets (per row, per retrieval q head) and outputs of the GPU
     prefill against the oracle, over `rows` (default: every row)."""
     sh = inp["shape"] if top_p is None else inp["shape"].replace(top_p=top_p)
-    g = g or run_gpu_prefill(inp, top_p)
+    g = g or run_gpu_prefill(inp, top_p, local_cap=local_cap)
     assert g["status"] == 0, f"device status {g['status']}"
     T = inp["T"]
     rows = list(range(T)) if rows is None else list(rows)

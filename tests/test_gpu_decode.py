@@ -232,3 +232,53 @@ def test_decode_without_bitmask_matches(case):
     else:
         atol, rtol = TOL["bf16"]
         assert np.all(np.abs(a["out"] - b["out"]) <= atol + rtol * np.abs(a["out"]))
+
+
+def test_decode_workspace_needs_no_initialisation():
+    """Completion flags are cleared by their owners inside every call, so a
+    workspace full of leftovers gives the same result as a zeroed one: every
+    byte 0xFF, and the raised flags (value 1) a previous call leaves behind."""
+    inp = _small(ctx=6000, needles=8)
+    ref = run_gpu_decode(inp, top_p=0.9, ws_fill=0)
+    got = run_gpu_decode(inp, top_p=0.9, ws_fill=0xFF)
+    assert got["status"] == 0
+    assert np.array_equal(got["out"], ref["out"])
+    assert torch.equal(got["bitmask"], ref["bitmask"])
+    # a second call on the same workspace, after a call with another query
+    lay, sh = got["layer"], got["shape"]
+    dev = torch.device("cuda")
+    seq = torch.from_numpy(inp["seq_len"]).to(dev)
+    w_q = inp["w_q"].to(dev)
+    out = torch.empty((1, sh.n_q_heads, sh.head_dim), dtype=torch.bfloat16, device=dev)
+    q_other = torch.randn(inp["q_pre"].shape, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    lay.decode(q_other.to(dev), seq, w_q, out, max_seq_len=6000)
+    lay.decode(inp["q_pre"].to(dev), seq, w_q, out, max_seq_len=6000)
+    torch.cuda.synchronize()
+    assert lay.device_status() == 0
+    assert np.array_equal(out.double().cpu().numpy(), ref["out"])
+
+
+def test_bounded_wait_expiry_sets_timeout_and_returns():
+    """The decode step's in-kernel waits are bounded: armed through the test
+    hook, a call waits for flags that never reach the awaited value, gives up
+    after a few thousand polls, sets RTP_DEV_TIMEOUT and returns; the GPU
+    stays usable and the next call is correct again."""
+    import head_wise_sparse_local_b200 as rtp
+    inp = _small(ctx=3000, needles=4)
+    g = run_gpu_decode(inp, top_p=0.9)
+    lay = g["layer"]
+    sh = g["shape"]
+    dev = torch.device("cuda")
+    q = inp["q_pre"].to(dev)
+    seq = torch.from_numpy(inp["seq_len"]).to(dev)
+    w_q = inp["w_q"].to(dev)
+    out = torch.empty((1, sh.n_q_heads, sh.head_dim), dtype=torch.bfloat16, device=dev)
+    rtp.rtp_debug_wait_expiry(2000)
+    lay.decode(q, seq, w_q, out, max_seq_len=3000)
+    torch.cuda.synchronize()
+    assert lay.device_status() & rtp.RTP_DEV_TIMEOUT
+    lay.status.zero_()
+    lay.decode(q, seq, w_q, out, max_seq_len=3000)  # not armed any more
+    torch.cuda.synchronize()
+    assert lay.device_status() == 0
+    assert np.array_equal(out.double().cpu().numpy(), g["out"])

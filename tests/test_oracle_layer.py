@@ -131,6 +131,44 @@ def test_indexer_scale_two_token_golden():
         assert list(topp[(0, 0)]) == case["kept"], case
 
 
+@pytest.mark.parametrize("path", ["append", "append_in_place", "prefill"])
+def test_indexer_key_storage_rounding_golden(path):
+    """The stored indexer key is rounded to the cache's storage type before it
+    is scored: a bf16 layer ties two tokens that an fp32 layer separates by
+    2^-11, which flips the kept set (hand-derived, tests/golden)."""
+    d = json.load(open(os.path.join(GOLD, "indexer_bf16_rounding.json")))
+    D = d["head_dim"]
+    for case in d["cases"]:
+        L = case["L"]
+        sh = LayerShape(batch=1, n_q_heads=1, n_kv_heads=1, head_dim=D, n_sink=0, window=1,
+                        top_p=case["p"], retrieval=(0,), dtype=case["dtype"])
+        wq = torch.zeros((1, 16, D))
+        wq[0, 0, 0] = 1.0
+        wk = torch.zeros((1, 16, D))
+        wk[0, 0] = torch.tensor(d["w_k_row0"], dtype=torch.float32)
+        k = torch.zeros((1, L, 1, D), dtype=sh.torch_dtype)
+        for j in range(L):
+            k[0, j, 0, j] = 1.0
+        v = torch.randn((1, L, 1, D)).to(sh.torch_dtype)
+        q = torch.zeros((1, 1, D), dtype=sh.torch_dtype)
+        q[0, 0, 0] = 1.0
+        c = OracleCache(sh, L)
+        if path == "append_in_place":
+            c.append_in_place(k, v, [L], wk)
+        else:
+            c.append(k, v, [0], L, wk)
+        stored = c.indexer_keys(0, 0, L)[:, 0]
+        assert list(stored) == d["stored_" + case["dtype"]][:L], (case, stored)
+        assert np.all(c.indexer_keys(0, 0, L)[:, 1:] == 0.0)
+        if path == "prefill":
+            _, topp = oracle.prefill(c, q[:, None].expand(1, L, 1, D).contiguous(), [0], wq, rows=[L - 1])
+            kept = topp[(0, L - 1, 0)]
+        else:
+            _, topp, _ = oracle.decode(c, q, [L], wq)
+            kept = topp[(0, 0)]
+        assert list(kept) == case["kept"], (path, case)
+
+
 def test_sink_window_golden():
     d = json.load(open(os.path.join(GOLD, "sink_window.json")))
     for c in d["cases"]:
