@@ -45,7 +45,8 @@ import torch  # noqa: E402
 METRIC = "sparse-attn layer decode µs/token & HBM GB/s at 128K–1M; prefill ms @32K"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
 TRAFFIC_MD = os.path.join(ROOT, "profiles", "decode_128k_bf16_dram_bytes.md")
-STAGE_KERNEL = {"append": "append_kernel", "decode_stream": "stream_kernel", "decode_select": "select_kernel"}
+STAGE_KERNEL = {"append": "append_kernel", "decode_score": "score_kernel", "decode_select": "select_kernel",
+                "decode_local": "sw_kernel"}
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -345,7 +346,7 @@ def run_ours(args, dist: Dist) -> dict:
         raise RuntimeError(f"device status {status} during the timed steps")
 
     # per-kernel CUDA-event timing (same steps, eager launches behind a pre-roll)
-    stages = ["append", "decode_stream", "decode_select"] if R else ["append", "decode_stream"]
+    stages = ["append", "decode_score", "decode_select", "decode_local"] if R else ["append", "decode_local"]
     n_k = args.kernel_steps
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_k)]
     torch.cuda.synchronize()
@@ -411,8 +412,8 @@ def run_ours(args, dist: Dist) -> dict:
 
     # roofline of the dominant kernel
     dominant = max(kern_us, key=lambda s: kern_us[s])
-    kbytes = {"append": nbytes["append"], "decode_stream": nbytes["score"] + nbytes["sw"] + nbytes["qo"],
-              "decode_select": nbytes["kept"]}
+    kbytes = {"append": nbytes["append"], "decode_score": nbytes["score"], "decode_select": nbytes["kept"],
+              "decode_local": nbytes["sw"] + nbytes["qo"]}
     peaks = {}
     if os.path.exists(PEAKS_PATH):
         peaks = json.load(open(PEAKS_PATH))
@@ -431,7 +432,7 @@ def run_ours(args, dist: Dist) -> dict:
         e2e={"value": e2e_s * 1e6 / (n_e * B * dist.world), "unit": "µs/token",
              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e},
         clocks=(clocks.summary(t_wall0, t_wall1) if clocks else None),
-        gpu_launches=K * (3 if R else 2), l2=l2, inp=inp, Lh=Lh,
+        gpu_launches=K * (4 if R else 2), l2=l2, inp=inp, Lh=Lh,
     )
 
 

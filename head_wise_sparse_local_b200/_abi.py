@@ -30,7 +30,8 @@ EXPORTS = ("rtp_cache_bytes", "rtp_decode_workspace_bytes", "rtp_prefill_workspa
            "rtp_trace_stage", "rtp_debug_wait_expiry",
            "rtp_last_error", "rtp_version")
 
-STAGES = {"append": 0, "decode_stream": 1, "decode_select": 2, "prefill_index": 3, "prefill_attn": 4}
+STAGES = {"append": 0, "decode_score": 1, "decode_select": 2, "decode_local": 3,
+          "prefill_index": 4, "prefill_attn": 5}
 
 
 class rtp_layer_cfg(ctypes.Structure):

@@ -1,22 +1,21 @@
 // rtp_decode_attn: one decode step of the head-wise sparse attention layer.
 //
-// Two kernels on the caller's stream, chained with programmatic dependent
-// launch, scratch in the caller's workspace:
+// Three kernels on the caller's stream, chained with programmatic dependent
+// launch, scratch in the caller's workspace.  The first two are the step's
+// HBM streams and run side by side; each of their CTAs pulls its whole share
+// into shared memory with bulk asynchronous copies (TMA) that complete on an
+// mbarrier:
 //
-//   stream_kernel  the two HBM streams of the step, side by side in one grid
-//                  that covers every SM, each CTA pulling its whole share into
-//                  shared memory with bulk asynchronous copies (TMA) that
-//                  complete on an mbarrier:
-//                  * score CTAs take a chunk of the 16-d indexer-key cache
-//                    (contiguous rows) and write the fp32 scores
-//                    s_j = q~ . k~_j / 4 of the G query heads of a retrieval
-//                    KV head plus a per-chunk maximum;
-//                  * sink/window clusters (one per sequence and KV head)
-//                    attend the sinks and the window of every KV head: a
-//                    half-warp per row, all G query heads per row, log-sum-exp
-//                    merged across the cluster through distributed shared
-//                    memory.  Local heads write their output here; retrieval
-//                    heads leave one partial per query head.
+//   score_kernel   a chunk of the 16-d indexer-key cache (contiguous rows) per
+//                  CTA; the fp32 scores s_j = q~ . k~_j / 4 of the G query
+//                  heads of a retrieval KV head are formed on tensor cores
+//                  (q~ as bf16 high and low parts, as in the prefill) and
+//                  written with a per-chunk maximum.
+//   sw_kernel      one cluster per (sequence, KV head) attends the sinks and
+//                  the window: S = K Q^T and O^T = V^T P on tensor cores per
+//                  16-row tile (bf16; fp32 layers on CUDA cores), log-sum-exp
+//                  merged across the cluster.  Local heads write their output
+//                  here; retrieval heads leave one partial per query head.
 //   select_kernel  one thread-block cluster per (sequence, retrieval q head).
 //                  It launches at once and prepares its query, then waits for
 //                  the stream kernel to complete.  The softmax mass
@@ -42,6 +41,7 @@
 // Top-p follows the abstract's observation (3) and the atlas.scime.ai summary
 // ("query-adaptive top-p threshold"); sinks + window follow that summary's
 // "Approach"; the 16-d pre-RoPE indexer follows observation (2).
+#include <algorithm>
 #include <atomic>
 #include <climits>
 #include <mutex>
@@ -73,8 +73,11 @@ constexpr int kTopPerWarp = 16;     // top-rung items a warp hands the leader in
 static_assert(kTopPerWarp <= 32, "the tail gives each top-rung item of a warp its own lane");
 constexpr int kSpec = 2;            // of those, rows whose keys and values a warp stages early
 
-// Tokens per score CTA: eight (bf16) or four (fp32) 16-d keys per thread.
-__host__ __device__ constexpr int score_chunk(int esize) { return kThreads * (esize == 2 ? 8 : 4); }
+// Tokens per score chunk (32 KB of indexer keys): four (bf16) or two (fp32)
+// 16-d keys per thread.
+__host__ __device__ constexpr int score_chunk(int esize) { return kThreads * (esize == 2 ? 4 : 2); }
+constexpr int kScoreSmem = 2 * 32 * 1024;  // two chunk buffers
+constexpr int kScoreCtasPerSm = 3;
 
 struct DecodeArgs {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W, max_seq_len, words;
@@ -93,8 +96,10 @@ struct DecodeArgs {
   float* logits;    // [B][NR][lstride]
   float* cmax;      // [B][NR][nch_score_max]
   float* sw_part;   // [B][Hkv][G][D + 2]: sink/window partial per query head (o[D], m, l)
+  float* sw_scratch;  // [B][Hkv][kSwCluster][G][D + 2]: partial of each CTA of a sink/window cluster
+  float* sel_scratch; // [B][NR][kMaxCS][D + 3]: partial (o[D], m, l) and kept count of each select CTA
   uint2* cand;      // [B][NR][lstride] boundary-bucket candidates past kCandSmem
-  int nch_score_max, n_score_ctas, n_score_pad, sel_cs;
+  int nch_score_max, n_score_ctas, sel_cs;
   int want_mask;    // 1: the caller asked for the top-p bitmask
   unsigned tx_extra;   // bytes a copy barrier expects beyond its copies (0; 16 when a test arms expiry)
   unsigned long long wait_ns;  // time a bounded wait allows before it gives up
@@ -157,29 +162,18 @@ __device__ void rope_query(const DecodeArgs& a, int b, int h, int pos, float* s_
 }
 
 // ---------------------------------------------------------------------------
-// 1a. score CTA: indexer scores + per-chunk maxima of one retrieval KV head
+// 1a. score CTAs: indexer scores + per-chunk maxima of the retrieval KV heads
 // ---------------------------------------------------------------------------
-// The chunk's indexer keys (contiguous rows of the key cache) arrive in shared
-// memory with one bulk asynchronous copy; the scores are then formed there.
+// A persistent grid (at most kScoreCtasPerSm per SM) walks the chunks
+// (sequence, retrieval KV head, chunk of kChunk tokens) in order, a CTA taking
+// every gridDim.x-th.  A chunk's indexer keys (contiguous rows of the key
+// cache) arrive in shared memory with one bulk asynchronous copy, two chunks in
+// flight per CTA; the scores are formed there.
 template <typename T, int D, int G>
-__device__ __forceinline__ void score_cta(const DecodeArgs& a, int sc, unsigned char* dsm, uint64_t* bar) {
-  constexpr int kChunk = score_chunk(sizeof(T));
-  constexpr int TPT = kChunk / kThreads;        // keys per thread
-  constexpr int NV = kIdxDim * sizeof(T) / 16;  // 16-byte vectors per key
-  constexpr int KB = kIdxDim * sizeof(T);       // bytes per key
-  static_assert(kChunk * KB <= kStreamSmem, "a score chunk fits in the stream kernel's shared memory");
-  __shared__ __align__(16) float s_q[G * kIdxDim];
-  __shared__ float s_ml[kWarps * G];
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int nch = a.n_score_ctas / (a.B * a.R);
-  const int chunk = sc % nch;
-  const int br = sc / nch;
-  const int b = br / a.R, r = br % a.R;
+__device__ __forceinline__ void score_q(const DecodeArgs& a, int b, int r, float* s_q) {
+  // q~ = W_q q_pre: four threads per output, a quarter of the dims each
+  const int tid = threadIdx.x;
   const int h = a.ret_head[r];
-  const int L = a.seq_len[b];
-  if (tid == 0) mbar_init(bar, 1);
-  // q~ = W_q q_pre from the caller's inputs, before waiting for rtp_append_kv:
-  // four threads per output, a quarter of the dims each
   for (int o4 = tid; o4 < G * kIdxDim * 4; o4 += kThreads) {
     const int o = o4 >> 2, qd = o4 & 3;
     const int g = o / kIdxDim, i = o % kIdxDim;
@@ -200,88 +194,189 @@ __device__ __forceinline__ void score_cta(const DecodeArgs& a, int sc, unsigned 
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
     if (qd == 0) s_q[g * kIdxDim + i] = acc;
   }
-  __syncthreads();  // barrier initialised, q~ visible
-  griddep_wait();   // rtp_append_kv (and with it the previous decode step) has completed
-  if (!seq_ok(L, a)) {  // uniform over the CTA
-    if (chunk == 0 && r == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
+}
+
+template <typename T, int D, int G>
+__device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* dsm, uint64_t* bar) {
+  constexpr int kChunk = score_chunk(sizeof(T));
+  constexpr int TPT = kChunk / kThreads;        // keys per thread
+  constexpr int NV = kIdxDim * sizeof(T) / 16;  // 16-byte vectors per key
+  constexpr int KB = kIdxDim * sizeof(T);       // bytes per key
+  constexpr int kBuf = kChunk * KB;             // bytes of one chunk buffer
+  __shared__ __align__(16) float s_q[G * kIdxDim];
+  __shared__ float s_ml[kWarps * G];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nch = a.n_score_ctas / (a.B * a.R);  // chunks per (sequence, retrieval head)
+  const int n_all = a.n_score_ctas;
+  const uint64_t pol = l2_evict_first();
+  if (blockIdx.x >= n_all) {  // no chunk for this CTA
+    griddep_wait();
+    griddep_launch();
     return;
   }
-  // The keys are fetched up to the call's maximum length without looking at
-  // seq_len (rows past seq_len are in bounds and their scores are never used).
-  const int j0 = chunk * kChunk;
-  const int jh = min(a.max_seq_len, j0 + kChunk);
-  const unsigned char* src = static_cast<const unsigned char*>(a.kidx) +
-                             (((size_t)b * a.R + r) * a.Lmax + j0) * KB;
   if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+  }
+  int cur_br = blockIdx.x / nch;
+  score_q<T, D, G>(a, cur_br / a.R, cur_br % a.R, s_q);  // the caller's inputs: before the wait
+  __syncthreads();  // barriers initialised, q~ visible
+  griddep_wait();   // rtp_append_kv (and with it the previous decode step) has completed
+  griddep_launch();
+  // chunk c: keys [j0, jh) of (sequence b, retrieval head r); rows fetched up to
+  // the call's maximum length without looking at seq_len (rows past seq_len are
+  // in bounds and their scores are never used)
+  auto issue = [&](int c, int k) {  // k-th chunk of this CTA -> buffer k & 1
+    const int br = c / nch, chunk = c % nch;
+    const int j0 = chunk * kChunk, jh = min(a.max_seq_len, j0 + kChunk);
+    const unsigned char* src = static_cast<const unsigned char*>(a.kidx) +
+                               ((size_t)br * a.Lmax + j0) * KB;
     const uint32_t bytes = (uint32_t)(jh - j0) * KB;
-    mbar_expect_tx(bar, bytes + a.tx_extra);
-    bulk_g2s(dsm, src, bytes, bar, l2_evict_first());
+    mbar_expect_tx(bar + (k & 1), bytes + a.tx_extra);
+    bulk_g2s(dsm + (size_t)(k & 1) * kBuf, src, bytes, bar + (k & 1), pol);
+  };
+  if (tid == 0) {
+    issue(blockIdx.x, 0);
+    if (blockIdx.x + gridDim.x < n_all) issue(blockIdx.x + gridDim.x, 1);
   }
-  if (!mbar_wait_bounded(bar, 0, a.wait_ns, a.status)) {
-    mbar_wait_bounded(bar, 0, a.wait_ns, a.status);  // the copy, before leaving (output invalid)
-    return;
-  }
-  const int j1 = min(L, jh);
-  float* lg = a.logits + ((size_t)b * a.NR + (size_t)r * G) * a.lstride;
-  float mx[G];
+  int k = 0;
+  for (int c = blockIdx.x; c < n_all; c += gridDim.x, ++k) {
+    const int br = c / nch, chunk = c % nch;
+    const int b = br / a.R, r = br % a.R;
+    const int L = a.seq_len[b];
+    if (br != cur_br) {  // another (sequence, retrieval head): its q~ (uniform over the CTA)
+      __syncthreads();
+      score_q<T, D, G>(a, b, r, s_q);
+      cur_br = br;
+    }
+    const bool arrived = mbar_wait_bounded(bar + (k & 1), (uint32_t)(k >> 1) & 1u, a.wait_ns, a.status);
+    if (__syncthreads_or(!arrived)) {  // every thread takes the same branch
+      // a copy did not complete in time (RTP_DEV_TIMEOUT is set): wait, again
+      // with a limit, for the copies in flight before leaving; output invalid
+      mbar_wait_bounded(bar + (k & 1), (uint32_t)(k >> 1) & 1u, a.wait_ns, a.status);
+      if (c + gridDim.x < n_all)
+        mbar_wait_bounded(bar + ((k + 1) & 1), (uint32_t)((k + 1) >> 1) & 1u, a.wait_ns, a.status);
+      return;
+    }
+    const unsigned char* kbuf = dsm + (size_t)(k & 1) * kBuf;
+    if (!seq_ok(L, a)) {  // uniform over the CTA
+      if (chunk == 0 && r == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
+    } else {
+      const int j0 = chunk * kChunk;
+      const int j1 = min(L, min(a.max_seq_len, j0 + kChunk));
+      float* lg = a.logits + ((size_t)b * a.NR + (size_t)r * G) * a.lstride;
+      if constexpr (sizeof(T) == 2) {
+        // Tensor cores, with exactly the prefill selection's arithmetic: S = K~ Q~^T
+        // (16 keys x 8 columns per mma, column n = query head n < G), q~ split
+        // into bf16 hi and lo parts accumulated in that order into one fp32
+        // accumulator.  A prefill row and the decode step at its position then
+        // see bit-identical scores.
+        const int t4 = lane & 3, gq = lane >> 2;
+        unsigned bh0 = 0u, bh1 = 0u, bl0 = 0u, bl1 = 0u;
+        if (gq < G) {
+          const int k0 = t4 * 2;
+          const float v[4] = {s_q[gq * kIdxDim + k0], s_q[gq * kIdxDim + k0 + 1], s_q[gq * kIdxDim + k0 + 8],
+                              s_q[gq * kIdxDim + k0 + 9]};
+          float hi[4], lo[4];
 #pragma unroll
-  for (int g = 0; g < G; ++g) mx[g] = -CUDART_INF_F;
+          for (int e = 0; e < 4; ++e) {
+            hi[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+            lo[e] = v[e] - hi[e];
+          }
+          bh0 = pack_bf16(hi[0], hi[1]);
+          bh1 = pack_bf16(hi[2], hi[3]);
+          bl0 = pack_bf16(lo[0], lo[1]);
+          bl1 = pack_bf16(lo[2], lo[3]);
+        }
+        // this lane's columns 2 t4, 2 t4 + 1 (query heads when < G)
+        float mxa = -CUDART_INF_F, mxb = -CUDART_INF_F;
+        const bool ca = 2 * t4 < G, cb = 2 * t4 + 1 < G;
+        constexpr int kTiles = kChunk / 16;
+        for (int tt = warp; tt < kTiles; tt += kWarps) {
+          const int kb = tt * 16;  // first key of the tile (chunk-local)
+          if (j0 + kb >= j1) break;  // warp-uniform
+          unsigned a0, a1, a2, a3;
+          ldsm_x4(a0, a1, a2, a3, kbuf + (size_t)(kb + (lane & 7) + ((lane >> 3) & 1) * 8) * KB + (lane >> 4) * 16);
+          float cc[4] = {0.f, 0.f, 0.f, 0.f};
+          mma_bf16(cc, a0, a1, a2, a3, bh0, bh1);
+          mma_bf16(cc, a0, a1, a2, a3, bl0, bl1);
 #pragma unroll
-  for (int t = 0; t < TPT; ++t) {
-    const int jl = t * kThreads + tid;
-    const int j = j0 + jl;
-    if (j >= j1) continue;
-    uint4 kr[NV];
+          for (int x = 0; x < 2; ++x) {
+            const int j = j0 + kb + gq + 8 * x;
+            if (j >= j1) continue;
+            const float sa = cc[2 * x] * kIdxScale + 0.0f;  // +0 turns -0 into +0
+            const float sb = cc[2 * x + 1] * kIdxScale + 0.0f;
+            if (ca) {
+              lg[(size_t)(2 * t4) * a.lstride + j] = sa;
+              mxa = fmaxf(mxa, sa);
+            }
+            if (cb) {
+              lg[(size_t)(2 * t4 + 1) * a.lstride + j] = sb;
+              mxb = fmaxf(mxb, sb);
+            }
+          }
+        }
 #pragma unroll
-    for (int v = 0; v < NV; ++v) kr[v] = reinterpret_cast<const uint4*>(dsm + (size_t)jl * KB)[v];
-    float kv[kIdxDim];
-    if constexpr (sizeof(T) == 2) {
+        for (int o = 4; o < 32; o <<= 1) {
+          mxa = fmaxf(mxa, __shfl_xor_sync(0xffffffffu, mxa, o));
+          mxb = fmaxf(mxb, __shfl_xor_sync(0xffffffffu, mxb, o));
+        }
+        if (gq == 0) {
+          if (ca) s_ml[warp * G + 2 * t4] = mxa;
+          if (cb) s_ml[warp * G + 2 * t4 + 1] = mxb;
+        }
+      } else {
+        float mx[G];
 #pragma unroll
-      for (int v = 0; v < NV; ++v) {
-        const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&kr[v]);
+        for (int g = 0; g < G; ++g) mx[g] = -CUDART_INF_F;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float2 f = __bfloat1622float2(h2[q]);
-          kv[v * 8 + 2 * q] = f.x;
-          kv[v * 8 + 2 * q + 1] = f.y;
+        for (int t = 0; t < TPT; ++t) {
+          const int jl = t * kThreads + tid;
+          const int j = j0 + jl;
+          if (j >= j1) continue;
+          uint4 kr[NV];
+#pragma unroll
+          for (int v = 0; v < NV; ++v) kr[v] = reinterpret_cast<const uint4*>(kbuf + (size_t)jl * KB)[v];
+          float kv[kIdxDim];
+#pragma unroll
+          for (int v = 0; v < NV; ++v) {
+            kv[v * 4 + 0] = __uint_as_float(kr[v].x); kv[v * 4 + 1] = __uint_as_float(kr[v].y);
+            kv[v * 4 + 2] = __uint_as_float(kr[v].z); kv[v * 4 + 3] = __uint_as_float(kr[v].w);
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float4* q4 = reinterpret_cast<const float4*>(s_q + g * kIdxDim);
+            float sco = 0.f;
+#pragma unroll
+            for (int i4 = 0; i4 < kIdxDim / 4; ++i4) {
+              const float4 qq = q4[i4];
+              sco = fmaf(qq.x, kv[4 * i4], sco);
+              sco = fmaf(qq.y, kv[4 * i4 + 1], sco);
+              sco = fmaf(qq.z, kv[4 * i4 + 2], sco);
+              sco = fmaf(qq.w, kv[4 * i4 + 3], sco);
+            }
+            sco = sco * kIdxScale + 0.0f;  // exact scaling; +0 turns -0 into +0
+            lg[(size_t)g * a.lstride + j] = sco;
+            mx[g] = fmaxf(mx[g], sco);
+          }
+        }
+        // one block reduction for the G chunk maxima (-inf for a chunk past seq_len)
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float v = warp_max(mx[g]);
+          if (lane == 0) s_ml[warp * G + g] = v;
         }
       }
-    } else {
+      __syncthreads();
+      if (tid < G) {
+        float v = s_ml[tid];
 #pragma unroll
-      for (int v = 0; v < NV; ++v) {
-        kv[v * 4 + 0] = __uint_as_float(kr[v].x); kv[v * 4 + 1] = __uint_as_float(kr[v].y);
-        kv[v * 4 + 2] = __uint_as_float(kr[v].z); kv[v * 4 + 3] = __uint_as_float(kr[v].w);
+        for (int w = 1; w < kWarps; ++w) v = fmaxf(v, s_ml[w * G + tid]);
+        a.cmax[((size_t)b * a.NR + r * G + tid) * a.nch_score_max + chunk] = v;
       }
     }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      const float4* q4 = reinterpret_cast<const float4*>(s_q + g * kIdxDim);
-      float s = 0.f;
-#pragma unroll
-      for (int i4 = 0; i4 < kIdxDim / 4; ++i4) {
-        const float4 qq = q4[i4];
-        s = fmaf(qq.x, kv[4 * i4], s);
-        s = fmaf(qq.y, kv[4 * i4 + 1], s);
-        s = fmaf(qq.z, kv[4 * i4 + 2], s);
-        s = fmaf(qq.w, kv[4 * i4 + 3], s);
-      }
-      s = s * kIdxScale + 0.0f;  // exact scaling; +0 turns -0 into +0
-      lg[(size_t)g * a.lstride + j] = s;
-      mx[g] = fmaxf(mx[g], s);
-    }
-  }
-  // one block reduction for the G chunk maxima (-inf for a chunk past seq_len)
-#pragma unroll
-  for (int g = 0; g < G; ++g) {
-    const float v = warp_max(mx[g]);
-    if (lane == 0) s_ml[warp * G + g] = v;
-  }
-  __syncthreads();
-  if (tid < G) {
-    float v = s_ml[tid];
-#pragma unroll
-    for (int w = 1; w < kWarps; ++w) v = fmaxf(v, s_ml[w * G + tid]);
-    a.cmax[((size_t)b * a.NR + r * G + tid) * a.nch_score_max + chunk] = v;
+    __syncthreads();  // buffer k & 1 is free
+    if (tid == 0 && c + 2 * gridDim.x < n_all) issue(c + 2 * gridDim.x, k + 2);
   }
 }
 
@@ -331,12 +426,14 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
   using Lane = SwLane<T, D>;
   constexpr int EPL = Lane::EPL;
   constexpr int RB = D * (int)sizeof(T);             // bytes per cache row
-  constexpr int SR = kStreamSmem / 4 / RB;           // rows per stage (K and V of a stage: half the buffer)
+  // rows per stage (K and V of a stage take at most half the buffer; at most
+  // 80 rows, 32 for G = 8, which keeps a warp's scores of a stage in registers)
+  constexpr int kCapRows = G >= 8 ? 32 : 80;
+  constexpr int SR = (kStreamSmem / 4 / RB) < kCapRows ? (kStreamSmem / 4 / RB) : kCapRows;
   static_assert(SR >= 2 && SR % 2 == 0, "a stage holds whole row pairs");
   __shared__ __align__(16) float s_q[G * D];
   __shared__ __align__(16) float s_wo[kWarps][G][D];
   __shared__ float s_wml[kWarps][G][2];
-  __shared__ __align__(16) float s_part[G][D + 2];  // this CTA's (o[D], m, l) per query head
   cg::cluster_group cl = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int half = lane >> 4, c = lane & 15;
@@ -351,9 +448,9 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
     mbar_init(bar, 1);
     mbar_init(bar + 1, 1);
   }
-  rope_query<T, D, G>(a, b, h, L - 1, s_q);  // caller's inputs: before the wait
+  rope_query<T, D, G>(a, b, h, L - 1, s_q);
   __syncthreads();  // barriers initialised, s_q visible
-  griddep_wait();
+  if (a.n_score_ctas == 0) griddep_wait();  // no score kernel ahead: wait for rtp_append_kv here
 
   const int s_cnt = min(a.S, L);
   const int sw0 = max(s_cnt, L - a.W);
@@ -390,6 +487,160 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
     if (n_st > 1) issue(1);
   }
 
+  int failed = -1;
+  if constexpr (sizeof(T) == 2) {
+    // Tensor cores.  Per 16-row tile of a stage: S = K Q^T (16 rows x 8
+    // columns: query head c < G from q's bf16 high part, column G + c from its
+    // low part, so a score is the fp32-query score to about 2^-17), then
+    // O^T += V^T P (D x 8: the G heads' weighted values; P in bf16, as the
+    // prefill attention rounds it).  A lane owns query heads 2 t4 and
+    // 2 t4 + 1 (t4 = lane mod 4) for the tile rows g and g + 8 (g = lane / 4).
+    constexpr int KS = D / 16;
+    constexpr int NT = (2 * G + 7) / 8;  // n-tiles of S: 1, or 2 for G = 8
+    const int t4 = lane & 3, gq = lane >> 2;
+    unsigned qb[NT][KS][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int cix = nt * 8 + gq;
+      const int hd = cix < G ? cix : cix - G;
+      const int part = cix < G ? 0 : (cix < 2 * G ? 1 : 2);
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (part < 2) {
+          const float* qg = s_q + hd * D + ks * 16 + 2 * t4;
+          const float v[4] = {qg[0], qg[1], qg[8], qg[9]};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float hi = __bfloat162float(__float2bfloat16_rn(v[e]));
+            x[e] = part == 0 ? hi : v[e] - hi;
+          }
+        }
+        qb[nt][ks][0] = pack_bf16(x[0], x[1]);
+        qb[nt][ks][1] = pack_bf16(x[2], x[3]);
+      }
+    }
+    float mh[2] = {-CUDART_INF_F, -CUDART_INF_F}, lh[2] = {0.f, 0.f};
+    float oacc[KS][4];
+#pragma unroll
+    for (int mt = 0; mt < KS; ++mt) oacc[mt][0] = oacc[mt][1] = oacc[mt][2] = oacc[mt][3] = 0.f;
+    const bool own[2] = {2 * t4 < G, 2 * t4 + 1 < G};
+    for (int st = 0; st < n_st; ++st) {
+      const bool arrived = mbar_wait_bounded(bar + (st & 1), (uint32_t)(st >> 1) & 1u, a.wait_ns, a.status);
+      if (__syncthreads_or(!arrived)) {  // every thread takes the same branch
+        failed = st;
+        break;
+      }
+      const int n = min(e_hi, e_lo + (st + 1) * SR) - (e_lo + st * SR);
+      const unsigned char* sk = dsm + (size_t)(st & 1) * (kStreamSmem / 2);
+      const unsigned char* sv = sk + (size_t)SR * RB;
+      for (int tt = warp; 16 * tt < n; tt += kWarps) {  // warp-uniform
+        const int r0 = 16 * tt;
+        // S = K Q^T; rows past n read row 0 (their weights are zeroed)
+        float sacc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
+        {
+          const int rr = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const unsigned char* krow = sk + (size_t)(rr < n ? rr : 0) * RB + (lane >> 4) * 16;
+#pragma unroll
+          for (int ks = 0; ks < KS; ++ks) {
+            unsigned a0, a1, a2, a3;
+            ldsm_x4(a0, a1, a2, a3, krow + ks * 32);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) mma_bf16(sacc[nt], a0, a1, a2, a3, qb[nt][ks][0], qb[nt][ks][1]);
+          }
+        }
+        // scores of the lane's heads: high part + low part
+        float sc[2][2];  // [row g / g + 8][head 2 t4 + e]
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float lo_part;
+          if constexpr (G == 8) lo_part = sacc[NT - 1][i];
+          else if constexpr (G == 4) lo_part = __shfl_xor_sync(0xffffffffu, sacc[0][i], 2);
+          else if constexpr (G == 2) lo_part = __shfl_xor_sync(0xffffffffu, sacc[0][i], 1);
+          else lo_part = sacc[0][i ^ 1];
+          sc[i >> 1][i & 1] = (G == 8 ? sacc[0][i] : sacc[0][i]) + lo_part;
+        }
+        float tmx[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+#pragma unroll
+          for (int x = 0; x < 2; ++x) {
+            const bool okr = r0 + gq + 8 * x < n;
+            sc[x][e] = (own[e] && okr) ? sc[x][e] : -CUDART_INF_F;
+          }
+          tmx[e] = fmaxf(sc[0][e], sc[1][e]);
+#pragma unroll
+          for (int o = 4; o < 32; o <<= 1) tmx[e] = fmaxf(tmx[e], __shfl_xor_sync(0xffffffffu, tmx[e], o));
+        }
+        float pr[2][2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float mn = fmaxf(mh[e], tmx[e]);
+          const float al = (mn == -CUDART_INF_F) ? 1.f : exp2f(mh[e] - mn);  // 0 when mh = -inf
+          pr[0][e] = (sc[0][e] == -CUDART_INF_F) ? 0.f : exp2f(sc[0][e] - mn);
+          pr[1][e] = (sc[1][e] == -CUDART_INF_F) ? 0.f : exp2f(sc[1][e] - mn);
+          lh[e] = lh[e] * al + (pr[0][e] + pr[1][e]);
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            oacc[mt][e] *= al;
+            oacc[mt][2 + e] *= al;
+          }
+          mh[e] = mn;
+        }
+        // B fragments of P (k = 16 rows, n = 8 columns = query heads): lane
+        // (g, t4) needs P[rows 2 t4, 2 t4 + 1, 2 t4 + 8, 2 t4 + 9][head g],
+        // held by lanes (2 t4) * 4 + g / 2 and (2 t4 + 1) * 4 + g / 2
+        const unsigned u0 = pack_bf16(pr[0][0], pr[0][1]);  // row g: heads 2 t4, 2 t4 + 1
+        const unsigned u1 = pack_bf16(pr[1][0], pr[1][1]);  // row g + 8
+        const int s0 = (2 * t4) * 4 + (gq >> 1), s1 = (2 * t4 + 1) * 4 + (gq >> 1);
+        const unsigned x0 = __shfl_sync(0xffffffffu, u0, s0), x1 = __shfl_sync(0xffffffffu, u0, s1);
+        const unsigned y0 = __shfl_sync(0xffffffffu, u1, s0), y1 = __shfl_sync(0xffffffffu, u1, s1);
+        const unsigned sel = (gq & 1) ? 0x7632u : 0x5410u;
+        const unsigned pb0 = gq < G ? __byte_perm(x0, x1, sel) : 0u;
+        const unsigned pb1 = gq < G ? __byte_perm(y0, y1, sel) : 0u;
+        // O^T += V^T P: V^T fragments by transposing loads of V rows
+        {
+          const int rr = r0 + (lane & 7) + ((lane >> 4) & 1) * 8;
+          const unsigned char* vrow = sv + (size_t)(rr < n ? rr : 0) * RB + ((lane >> 3) & 1) * 16;
+#pragma unroll
+          for (int mt = 0; mt < KS; ++mt) {
+            unsigned a0, a1, a2, a3;
+            ldsm_x4_t(a0, a1, a2, a3, vrow + mt * 32);
+            mma_bf16(oacc[mt], a0, a1, a2, a3, pb0, pb1);
+          }
+        }
+      }
+      __syncthreads();  // buffer st & 1 is free
+      if (tid == 0 && st + 2 < n_st) issue(st + 2);
+    }
+    // the warp's state: l summed over its lanes' rows; O^T fragments to shared memory
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) lh[e] += __shfl_xor_sync(0xffffffffu, lh[e], o);
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      if (!own[e]) continue;
+      const int hd = 2 * t4 + e;
+#pragma unroll
+      for (int mt = 0; mt < KS; ++mt) {
+        s_wo[warp][hd][mt * 16 + gq] = oacc[mt][e];
+        s_wo[warp][hd][mt * 16 + gq + 8] = oacc[mt][2 + e];
+      }
+      if (gq == 0) {
+        s_wml[warp][hd][0] = mh[e];
+        s_wml[warp][hd][1] = lh[e];
+      }
+    }
+  } else {
+  // this lane's dims of the G RoPE'd queries
+  float qr[G][EPL];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) qr[g][e] = s_q[g * D + c * EPL + e];
   float m[G], l[G], o[G][EPL];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -398,69 +649,76 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
 #pragma unroll
     for (int e = 0; e < EPL; ++e) o[g][e] = 0.f;
   }
-  int failed = -1;
+  // Per stage: every score of the warp's rows first, then one running-max
+  // update per head, then the weights and the weighted values.
+  constexpr int PPW = (SR / 2 + kWarps - 1) / kWarps;  // row pairs per warp per stage
   for (int st = 0; st < n_st; ++st) {
-    if (!mbar_wait_bounded(bar + (st & 1), (uint32_t)(st >> 1) & 1u, a.wait_ns, a.status)) {
+    const bool arrived = mbar_wait_bounded(bar + (st & 1), (uint32_t)(st >> 1) & 1u, a.wait_ns, a.status);
+    if (__syncthreads_or(!arrived)) {  // every thread takes the same branch
       failed = st;
       break;
     }
     const int n = min(e_hi, e_lo + (st + 1) * SR) - (e_lo + st * SR);
     const unsigned char* sk = dsm + (size_t)(st & 1) * (kStreamSmem / 2);
     const unsigned char* sv = sk + (size_t)SR * RB;
-    for (int p = warp; 2 * p < n; p += kWarps) {
-      const int i = 2 * p + half;
+    float sc[PPW][G];
+    float smax[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) smax[g] = -CUDART_INF_F;
+#pragma unroll
+    for (int k = 0; k < PPW; ++k) {
+      const int i = 2 * (warp + k * kWarps) + half;
       const bool ok = i < n;  // uniform over the half-warp
-      Lane kr, vr;
+      Lane kr;
       kr.load(sk + (size_t)(ok ? i : 0) * RB + c * Lane::VB);
-      vr.load(sv + (size_t)(ok ? i : 0) * RB + c * Lane::VB);
       float kf[EPL];
       kr.to_f32(kf);
-      float s[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float* qg = s_q + g * D + c * EPL;
         float acc = 0.f;
 #pragma unroll
-        for (int e4 = 0; e4 < EPL; e4 += 4) {
-          const float4 qq = *reinterpret_cast<const float4*>(qg + e4);
-          acc = fmaf(qq.x, kf[e4], acc);
-          acc = fmaf(qq.y, kf[e4 + 1], acc);
-          acc = fmaf(qq.z, kf[e4 + 2], acc);
-          acc = fmaf(qq.w, kf[e4 + 3], acc);
-        }
-        s[g] = acc;
+        for (int e = 0; e < EPL; ++e) acc = fmaf(qr[g][e], kf[e], acc);
+        sc[k][g] = acc;
       }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        s[g] += __shfl_xor_sync(0xffffffffu, s[g], 8);
-        s[g] += __shfl_xor_sync(0xffffffffu, s[g], 4);
-        s[g] += __shfl_xor_sync(0xffffffffu, s[g], 2);
-        s[g] += __shfl_xor_sync(0xffffffffu, s[g], 1);
+        float v = sc[k][g];
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        sc[k][g] = ok ? v : -CUDART_INF_F;
+        smax[g] = fmaxf(smax[g], sc[k][g]);
       }
-      if (ok) {
-        float vf[EPL];
-        vr.to_f32(vf);
+    }
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          const float mn = fmaxf(m[g], s[g]);
-          const float al = exp2f(m[g] - mn);  // 0 while nothing was attended (m = -inf)
-          const float pv = exp2f(s[g] - mn);
-          l[g] = fmaf(l[g], al, pv);
+    for (int g = 0; g < G; ++g) {
+      const float mn = fmaxf(m[g], smax[g]);
+      if (mn == -CUDART_INF_F) continue;  // nothing in this half-warp yet (uniform over it)
+      const float al = exp2f(m[g] - mn);   // 0 while nothing was attended (m = -inf)
+      l[g] *= al;
 #pragma unroll
-          for (int e = 0; e < EPL; ++e) o[g][e] = fmaf(o[g][e], al, pv * vf[e]);
-          m[g] = mn;
-        }
+      for (int e = 0; e < EPL; ++e) o[g][e] *= al;
+      m[g] = mn;
+    }
+#pragma unroll
+    for (int k = 0; k < PPW; ++k) {
+      const int i = 2 * (warp + k * kWarps) + half;
+      if (i >= n) continue;  // uniform over the half-warp
+      Lane vr;
+      vr.load(sv + (size_t)i * RB + c * Lane::VB);
+      float vf[EPL];
+      vr.to_f32(vf);
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float pv = exp2f(sc[k][g] - m[g]);
+        l[g] += pv;
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) o[g][e] = fmaf(pv, vf[e], o[g][e]);
       }
     }
     __syncthreads();  // buffer st & 1 is free
     if (tid == 0 && st + 2 < n_st) issue(st + 2);
-  }
-  if (failed >= 0) {
-    // a copy did not complete in time (RTP_DEV_TIMEOUT is set): wait, again
-    // with a limit, for the stages still in flight before leaving; the
-    // output is invalid
-    for (int st = failed; st < min(n_st, failed + 2); ++st)
-      mbar_wait_bounded(bar + (st & 1), (uint32_t)(st >> 1) & 1u, a.wait_ns, a.status);
   }
   // the two halves of the warp, then the warps of the CTA
 #pragma unroll
@@ -486,7 +744,17 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
       s_wml[warp][g][1] = l[g];
     }
   }
+  }
+  if (failed >= 0) {
+    // a copy did not complete in time (RTP_DEV_TIMEOUT is set): wait, again
+    // with a limit, for the stages still in flight before leaving; the
+    // output is invalid
+    for (int st = failed; st < min(n_st, failed + 2); ++st)
+      mbar_wait_bounded(bar + (st & 1), (uint32_t)(st >> 1) & 1u, a.wait_ns, a.status);
+  }
   __syncthreads();
+  // this CTA's partial (o[D], m, l) per query head -> the cluster's slot in L2
+  float* part = a.sw_scratch + ((size_t)bkv * kSwCluster + crank) * (G * (D + 2));
   for (int i = tid; i < G * D; i += kThreads) {
     const int g = i / D, d = i % D;
     float mn = -CUDART_INF_F;
@@ -503,16 +771,17 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
         den = fmaf(s_wml[w][g][1], sc, den);
       }
     }
-    s_part[g][d] = acc;
+    part[g * (D + 2) + d] = acc;
     if (d == 0) {
-      s_part[g][D] = mn;
-      s_part[g][D + 1] = den;
+      part[g * (D + 2) + D] = mn;
+      part[g * (D + 2) + D + 1] = den;
     }
   }
-  cl.sync();  // every rank's partial in its shared memory
+  cl.sync();  // every rank's partial written (the barrier orders global memory within the cluster)
   // The cluster's merge is spread over its ranks: element i of the G x D
   // outputs goes to rank i mod csw.  Each thread issues its loads of every
-  // rank's partial at once (distributed shared memory, one round trip).
+  // rank's partial at once (L2 hits, one round trip).
+  const float* parts = a.sw_scratch + (size_t)bkv * kSwCluster * (G * (D + 2));
   for (int i = crank + csw * tid; i < G * D; i += csw * kThreads) {
     const int g = i / D, d = i % D;
     float mq[kSwCluster], lq[kSwCluster], oq[kSwCluster];
@@ -522,10 +791,10 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
       lq[q] = 0.f;
       oq[q] = 0.f;
       if (q < csw) {
-        const float* pq = cl.map_shared_rank(&s_part[g][0], q);
-        mq[q] = pq[D];
-        lq[q] = pq[D + 1];
-        oq[q] = pq[d];
+        const float* pq = parts + (size_t)q * (G * (D + 2)) + g * (D + 2);
+        mq[q] = __ldcg(pq + D);
+        lq[q] = __ldcg(pq + D + 1);
+        oq[q] = __ldcg(pq + d);
       }
     }
     float mn = -CUDART_INF_F;
@@ -550,27 +819,32 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
       }
     }
   }
-  cl.sync();  // no rank reads another's shared memory after this
 }
 
 // ---------------------------------------------------------------------------
-// 1. stream kernel: [score CTAs, padded to whole clusters][sink/window clusters]
+// 1. the two stream kernels
 // ---------------------------------------------------------------------------
-// It lets the select kernel launch at once (its CTAs start with the work that
-// needs no scores); the select kernel waits for this whole grid to complete.
+// score_kernel (plain grid) waits for rtp_append_kv, then lets the sink/window
+// kernel launch; sw_kernel (clusters) lets the select kernel launch at once
+// and reads the cache without a wait of its own: it starts only after every
+// score CTA has passed its wait, so the appended rows are complete.  Its
+// closing wait makes its completion imply the score kernel's, which is what
+// the select kernel's wait relies on.
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads, 2) stream_kernel(const __grid_constant__ DecodeArgs a) {
+__global__ void __launch_bounds__(kThreads, kScoreCtasPerSm) score_kernel(const __grid_constant__ DecodeArgs a) {
+  extern __shared__ __align__(128) unsigned char dsm[];
+  __shared__ __align__(8) uint64_t s_bar[2];
+  score_ctas<T, D, G>(a, dsm, s_bar);
+}
+
+template <typename T, int D, int G>
+__global__ void __launch_bounds__(kThreads, 2) sw_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char dsm[];
   __shared__ __align__(8) uint64_t s_bar[2];
   griddep_launch();
-  const int blk = blockIdx.x;
-  if (blk < a.n_score_pad) {
-    if (blk < a.n_score_ctas) score_cta<T, D, G>(a, blk, dsm, s_bar);
-    return;
-  }
   const int csw = (int)cg::this_cluster().num_blocks();
-  const int sw = blk - a.n_score_pad;
-  sw_cta<T, D, G>(a, sw / csw, (int)cg::this_cluster().block_rank(), csw, dsm, s_bar);
+  sw_cta<T, D, G>(a, blockIdx.x / csw, (int)cg::this_cluster().block_rank(), csw, dsm, s_bar);
+  griddep_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -902,10 +1176,9 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   __shared__ uint2 s_top[kSelWarps][kTopPerWarp];  // this CTA's top-rung items per warp (key, index)
   __shared__ int s_wtop[kSelWarps];
   __shared__ __align__(16) float s_qh[D];
+  __shared__ __align__(8) uint64_t s_sbar;     // completion of the bulk copy of this CTA's scores
   __shared__ __align__(16) float s_wo[kSelWarps * D];
   __shared__ float s_wml[kSelWarps * 2];
-  __shared__ __align__(16) float s_cp[D + 2];  // this CTA's partial for query head g: (o[D], m, l)
-  __shared__ int s_ccnt;                       // and its kept-token count
   // retrieval heads keep the whole context: row pos of head h sits at row0 + pos
   const size_t row0 = a.kv.row(b, h, 0);
   const T* kb = static_cast<const T*>(a.k) + row0 * D;
@@ -945,6 +1218,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   }
   if (rank == 0 && tid == 0) sh->n_cand2 = 0u;
   if (lane < kSpec) s_spec_j[warp][lane] = -1;
+  if (tid == 0) mbar_init(&s_sbar, 1);
   griddep_launch();
   cluster_arrive();  // counter zeroed; every CTA of the cluster running
   griddep_wait();    // the stream kernel (scores, chunk maxima, sink/window partials) has completed
@@ -955,8 +1229,17 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   const int nch_h = (Lh + kChunk - 1) / kChunk;
   const float* cm = a.cmax + (size_t)bh * a.nch_score_max;
   const float cm0 = tid < nch_h ? __ldcg(cm + tid) : -CUDART_INF_F;
-  if (cached) stage(j0, jh);
+  // a share that fits is staged once, by one bulk copy (rounded up to whole
+  // 16-byte vectors; the score rows are padded to 32 floats)
+  const bool bulk = cached && jh > j0;
+  if (bulk && tid == 0) {
+    const uint32_t bytes = (uint32_t)(((jh - j0) + 3) & ~3) * 4u;
+    mbar_expect_tx(&s_sbar, bytes);
+    bulk_g2s(s_lg, lg_g + j0, bytes, &s_sbar, l2_evict_first());
+  }
   cluster_wait();
+  if (bulk && !mbar_wait_bounded(&s_sbar, 0, a.wait_ns, a.status))
+    mbar_wait_bounded(&s_sbar, 0, a.wait_ns, a.status);  // the copy, before going on (output invalid)
   const int j1 = min(L, jh);  // j1 <= j0: nothing of this sequence in this CTA's share
   uint32_t* mask = a.mask + (size_t)bh * a.words;
   const bool keep_all = a.top_p >= 1.0f;
@@ -1568,6 +1851,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
     sh->cnt[warp] = cnt;
   }
   __syncthreads();
+  float* sp_me = a.sel_scratch + ((size_t)bh * kMaxCS + rank) * (D + 3);
   for (int d = tid; d < D; d += kSelThreads) {
     float mn = -CUDART_INF_F;
 #pragma unroll
@@ -1583,33 +1867,34 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         den = fmaf(s_wml[w * 2 + 1], sc, den);
       }
     }
-    s_cp[d] = acc;
+    sp_me[d] = acc;
     if (d == 0) {
-      s_cp[D] = mn;
-      s_cp[D + 1] = den;
+      sp_me[D] = mn;
+      sp_me[D + 1] = den;
     }
   }
   if (tid == 0) {
     int c = 0;
 #pragma unroll
     for (int w = 0; w < kSelWarps; ++w) c += sh->cnt[w];
-    s_ccnt = c;
+    sp_me[D + 2] = __int_as_float(c);
   }
-  cl.sync();  // every rank's partial and count in its shared memory
+  cl.sync();  // every rank's partial and count written (the barrier orders global memory within the cluster)
   {
     // The head's sink/window partial plus every rank's kept-row partial, the
     // D output elements spread over the ranks (element d on rank d mod CS),
-    // each thread loading every rank's partial at once.
+    // each thread loading every rank's partial at once (L2 hits).
     const int bkv = b * a.Hkv + h;
     const float* sp = a.sw_part + ((size_t)bkv * a.G + g) * (D + 2);
+    const float* parts = a.sel_scratch + (size_t)bh * kMaxCS * (D + 3);
     for (int d = rank + CS * tid; d < D; d += CS * kSelThreads) {
       float mq[CS], lq[CS], oq[CS];
 #pragma unroll
       for (int q = 0; q < CS; ++q) {
-        const float* pq = cl.map_shared_rank(s_cp, q);
-        mq[q] = pq[D];
-        lq[q] = pq[D + 1];
-        oq[q] = pq[d];
+        const float* pq = parts + (size_t)q * (D + 3);
+        mq[q] = __ldcg(pq + D);
+        lq[q] = __ldcg(pq + D + 1);
+        oq[q] = __ldcg(pq + d);
       }
       const float m_sw = __ldcg(sp + D);
       const float l_sw = __ldcg(sp + D + 1);
@@ -1635,11 +1920,10 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
     if (rank == 0 && tid == 0 && a.sel_count) {
       int c = 0;
 #pragma unroll
-      for (int q = 0; q < CS; ++q) c += *cl.map_shared_rank(&s_ccnt, q);
+      for (int q = 0; q < CS; ++q) c += __float_as_int(__ldcg(parts + (size_t)q * (D + 3) + D + 2));
       a.sel_count[bh] = c;
     }
   }
-  cl.sync();  // no rank reads another's shared memory after this
 }
 
 // ---------------------------------------------------------------------------
@@ -1670,12 +1954,14 @@ cudaError_t launch_cluster_pdl(void (*k)(DecodeArgs), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, k, a);
 }
 
-// Stream kernel with 16-CTA sink/window clusters when the device can place
-// one (non-portable size), else 8.  Set up once per device under a mutex.
+// The two stream kernels: score CTAs (plain grid), then sink/window clusters of
+// 16 CTAs when the device can place one (non-portable size), else 8.  Set up
+// once per device under a mutex.
 template <typename T, int D, int G>
 cudaError_t launch_stream(DecodeArgs& a, int n_bkv, cudaStream_t st) {
   static std::mutex s_mu;
   static std::atomic<int> s_cs[64];  // chosen cluster size; 0 = not set up yet
+  static std::atomic<int> s_sms[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -1685,8 +1971,9 @@ cudaError_t launch_stream(DecodeArgs& a, int n_bkv, cudaStream_t st) {
     std::lock_guard<std::mutex> lock(s_mu);
     cs = s_cs[dev].load(std::memory_order_relaxed);
     if (cs == 0) {
-      cudaFuncSetAttribute(stream_kernel<T, D, G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      cudaFuncSetAttribute(stream_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
+      cudaFuncSetAttribute(score_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
+      cudaFuncSetAttribute(sw_kernel<T, D, G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      cudaFuncSetAttribute(sw_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(kSwCluster);
       cfg.blockDim = dim3(kThreads);
@@ -1699,15 +1986,28 @@ cudaError_t launch_stream(DecodeArgs& a, int n_bkv, cudaStream_t st) {
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, stream_kernel<T, D, G>, &cfg) != cudaSuccess) n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, sw_kernel<T, D, G>, &cfg) != cudaSuccess) n = 0;
       cudaGetLastError();  // clear a refused query
+      int sms = 0;
+      if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
+      cudaGetLastError();
+      s_sms[dev].store(sms, std::memory_order_relaxed);
       cs = n > 0 ? kSwCluster : 8;
       s_cs[dev].store(cs, std::memory_order_release);
     }
   }
-  a.n_score_pad = (a.n_score_ctas + cs - 1) / cs * cs;
-  const dim3 grid(a.n_score_pad + n_bkv * cs);
-  return launch_cluster_pdl(stream_kernel<T, D, G>, grid, dim3(kThreads), kStreamSmem, cs, st, a);
+  const int n_sms = s_sms[dev].load(std::memory_order_relaxed);
+  if (a.n_score_ctas > 0) {
+    trace_begin(RTP_STAGE_DECODE_SCORE, st);
+    e = launch_pdl(score_kernel<T, D, G>, dim3(std::min(a.n_score_ctas, kScoreCtasPerSm * n_sms)), dim3(kThreads),
+                   kScoreSmem, st, a);
+    trace_end(RTP_STAGE_DECODE_SCORE, st);
+    if (e != cudaSuccess) return e;
+  }
+  trace_begin(RTP_STAGE_DECODE_LOCAL, st);
+  e = launch_cluster_pdl(sw_kernel<T, D, G>, dim3(n_bkv * cs), dim3(kThreads), kStreamSmem, cs, st, a);
+  trace_end(RTP_STAGE_DECODE_LOCAL, st);
+  return e;
 }
 
 template <typename T, int D>
@@ -1803,6 +2103,8 @@ DecodeLayout decode_layout(const Shape& sh) {
   l.mask = off;       off = align256(off + NRt * words * sizeof(uint32_t));  // bitmask when the caller passes none
   l.cand = off;       off = align256(off + NRt * lstride * sizeof(uint2));
   l.sw_part = off;    off = align256(off + (size_t)sh.B * sh.Hkv * sh.G * (sh.D + 2) * sizeof(float));
+  l.sw_scratch = off; off = align256(off + (size_t)sh.B * sh.Hkv * kSwCluster * sh.G * (sh.D + 2) * sizeof(float));
+  l.sel_scratch = off; off = align256(off + NRt * kMaxCS * (sh.D + 3) * sizeof(float));
   l.total = off;
   return l;
 }
@@ -1827,6 +2129,8 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   a.want_mask = sel_bitmask != nullptr;
   a.cand = reinterpret_cast<uint2*>(w + lay.cand);
   a.sw_part = reinterpret_cast<float*>(w + lay.sw_part);
+  a.sw_scratch = reinterpret_cast<float*>(w + lay.sw_scratch);
+  a.sel_scratch = reinterpret_cast<float*>(w + lay.sel_scratch);
   a.nch_score_max = lay.nch_score_max;
   a.sel_cs = 0;
   a.tx_extra = 0u;
@@ -1844,9 +2148,7 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   const int chunk = score_chunk(sh.esize);
   a.n_score_ctas = sh.R > 0 ? sh.B * sh.R * ((Lh + chunk - 1) / chunk) : 0;
 
-  trace_begin(RTP_STAGE_DECODE_STREAM, st);
   cudaError_t e = launch_stream_any(sh, a, st);
-  trace_end(RTP_STAGE_DECODE_STREAM, st);
   if (e == cudaSuccess && sh.R > 0) {
     trace_begin(RTP_STAGE_DECODE_SELECT, st);
     e = launch_select_any(sh, a, sh.B * sh.NR, st);

@@ -263,11 +263,12 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
 /* Kernel stages, for rtp_trace_stage. */
 typedef enum rtp_stage {
   RTP_STAGE_APPEND = 0,         /* rtp_append_kv: RoPE + cache + indexer-key store */
-  RTP_STAGE_DECODE_STREAM = 1,  /* decode: indexer scores + sink/window attention (one grid) */
+  RTP_STAGE_DECODE_SCORE = 1,   /* decode: indexer scores over the 16-d key cache */
   RTP_STAGE_DECODE_SELECT = 2,  /* decode: exact top-p selection, bitmask, kept-row attention, merge */
-  RTP_STAGE_PREFILL_INDEX = 3,  /* prefill: per-row exact top-p selection */
-  RTP_STAGE_PREFILL_ATTN = 4,   /* prefill: masked causal attention */
-  RTP_STAGE_COUNT = 5
+  RTP_STAGE_DECODE_LOCAL = 3,   /* decode: sink/window attention of every KV head (overlaps the scores) */
+  RTP_STAGE_PREFILL_INDEX = 4,  /* prefill: per-row exact top-p selection */
+  RTP_STAGE_PREFILL_ATTN = 5,   /* prefill: masked causal attention */
+  RTP_STAGE_COUNT = 6
 } rtp_stage;
 
 /* Host.  Optional instrumentation (no work is skipped or added).  Arms a
