@@ -77,6 +77,9 @@ struct PrefillLayout {
   int block_rows;  // query rows per selection + attention pass
 };
 PrefillLayout prefill_layout(const Shape& sh, int T);
+int launch_attn_tc(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* start_pos, int T,
+                   void* out, const uint32_t* mask, int t_base, int t_end, int mask_t0, int mask_rows,
+                   unsigned long long wait_ns, cudaStream_t st);
 int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* start_pos,
                    int T, const float* w_q, void* out, uint32_t* sel_bitmask, float* sel_tau,
                    int* sel_jcut, int* sel_count, void* ws, const PrefillLayout& lay, cudaStream_t st);

@@ -54,6 +54,7 @@ struct PrefillArgs {
   uint32_t* mask;  // [B][NR][mask_rows][words] top-p bitmask of rows [mask_t0, mask_t0 + mask_rows)
   int t_base, t_end;         // this launch's query rows [t_base, t_end) of the chunk
   int mask_t0, mask_rows;
+  int ring_only;             // attention: only the heads that keep a window ring
   KvMap kv;
   int ret_head[kMaxRetrieval];
   int ret_rank[kMaxRetrieval];
@@ -718,6 +719,7 @@ __global__ void __launch_bounds__(128, 3) attn_rows_kernel(const __grid_constant
   const int b = bq / a.Hq, hq = bq % a.Hq;
   const int h = hq / a.G, g = hq % a.G;
   const int r = a.ret_rank[h];
+  if (a.ring_only && !((a.kv.ring_mask >> h) & 1ull)) return;  // the tensor-core kernel's head
   const int start = a.start_pos[b];
   if (start < 0 || start + a.T > a.Lmax) return;  // flagged by the selection kernel / host
   const int t0 = a.t_base + blockIdx.x * kBQ;
@@ -985,6 +987,7 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
   a.sel_tau = sel_tau; a.sel_jcut = sel_jcut; a.sel_count = sel_count;
   a.mask = sel_bitmask ? sel_bitmask : static_cast<uint32_t*>(ws);
   a.kv = sh.kv;
+  a.ring_only = 0;
   for (int i = 0; i < kMaxRetrieval; ++i) { a.ret_head[i] = sh.ret_head[i]; a.ret_rank[i] = sh.ret_rank[i]; }
   for (int i = 0; i < 64; ++i) a.inv_freq[i] = sh.inv_freq[i];
 
@@ -1015,10 +1018,18 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
       else select_rows_kernel<64><<<gs, kSelRows * 32, kSelDynSmem, st>>>(a);
       trace_end(RTP_STAGE_PREFILL_INDEX, st);
     }
-    const dim3 ga((n + kBQ - 1) / kBQ, sh.B * sh.Hq);
     trace_begin(RTP_STAGE_PREFILL_ATTN, st);
-    if (sh.D == 128) attn_rows_kernel<128><<<ga, 128, AttnSmem<128>::kBytes, st>>>(a);
-    else attn_rows_kernel<64><<<ga, 128, AttnSmem<64>::kBytes, st>>>(a);
+    // full-context heads on tcgen05 tensor cores; local heads that keep a
+    // window ring (rows not contiguous in positions) on the mma.sync kernel
+    int rc = launch_attn_tc(sh, cache, q_pre, start_pos, T, out, a.mask, a.t_base, a.t_end, a.mask_t0,
+                            a.mask_rows, 400ull * 1000 * 1000, st);
+    if (rc != RTP_OK) return rc;
+    if (sh.kv.ring_mask) {
+      a.ring_only = 1;
+      const dim3 ga((n + kBQ - 1) / kBQ, sh.B * sh.Hq);
+      if (sh.D == 128) attn_rows_kernel<128><<<ga, 128, AttnSmem<128>::kBytes, st>>>(a);
+      else attn_rows_kernel<64><<<ga, 128, AttnSmem<64>::kBytes, st>>>(a);
+    }
     trace_end(RTP_STAGE_PREFILL_ATTN, st);
   }
   cudaError_t e = cudaGetLastError();

@@ -156,7 +156,9 @@ int rtp_append_kv(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* 
  * Local KV heads: exact attention over sinks [0, S) and window
  * [seq_len-W, seq_len) (atlas.scime.ai summary, "Approach").
  * Retrieval KV heads, for each of their G query heads separately:
- *   q~ = W_q^(r) q_pre (fp32), s_j = q~ . kidx_j / 4 for every cached j,
+ *   q~ = W_q^(r) q_pre (fp32), s_j = q~ . kidx_j / 4 for every cached j
+ *   (fp32; for a bf16 layer on tensor cores from q~'s bf16 high and low parts,
+ *   the fp32 score to about 2^-17 of the score),
  *   P = softmax(s); keep the smallest set, ordered by (P desc, j asc), whose
  *   mass reaches top_p (abstract, observations (2)-(3)); attend exactly over
  *   that set united with the sinks and the window.
@@ -226,13 +228,12 @@ int rtp_decode_attn_noalloc(const rtp_layer_cfg* cfg, const rtp_cache* cache, co
  * query at position i (top-p over the indexer scores of [0, i] for retrieval
  * query heads; sinks and window [i-W+1, i] for every head).  The indexer
  * scores are computed on tensor cores from q~ split into a bf16 high part and
- * a bf16 low part, with fp32 accumulation: they equal the fp32 score of
- * rtp_decode_attn to about 2^-17 of the score, not bit for bit.  A row's
- * top-p set can therefore differ from the decode step's at that position, but
- * only in tokens at the cut (within the 1e-6 probability tolerance of the
- * parity tests).  The attention itself runs on tensor cores in bf16 with fp32
- * accumulation (atlas.scime.ai summary, "Approach"; abstract, observations
- * (2)-(3)).  cfg->dtype must be RTP_BF16.
+ * a bf16 low part accumulated in fp32 (the fp32 score to about 2^-17 of the
+ * score), with exactly the arithmetic rtp_decode_attn uses for a bf16 layer:
+ * a row's top-p set equals the decode step's at that position, bit for bit.
+ * The attention itself runs on tensor cores in bf16 with fp32 accumulation
+ * (atlas.scime.ai summary, "Approach"; abstract, observations (2)-(3)).
+ * cfg->dtype must be RTP_BF16.
  *
  *   q_pre        [B][T][Hq][D] bf16, device
  *   start_pos    [B] int32, device; 0 <= start_pos[b] and start_pos[b] + T <= max_ctx
