@@ -44,7 +44,7 @@ import torch  # noqa: E402
 
 METRIC = "sparse-attn layer decode µs/token & HBM GB/s at 128K–1M; prefill ms @32K"
 PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
-TRAFFIC_MD = os.path.join(ROOT, "profiles", "decode_128k_bf16_dram_bytes.md")
+TRAFFIC_MD = os.path.join(ROOT, "profiles", "decode_128k_bf16_dram_bytes.md")  # per-kernel DRAM bytes (ncu)
 STAGE_KERNEL = {"append": "append_kernel", "decode_score": "score_kernel", "decode_select": "select_kernel",
                 "decode_local": "sw_kernel"}
 FALLBACK_HBM_GBS = 6650.0
@@ -207,8 +207,48 @@ def measured_traffic(stage: str, workload: str):
         path = os.path.join(csrc, fname)
         if not os.path.exists(path) or hashlib.sha256(open(path, "rb").read()).hexdigest()[:16] != digest:
             return None
-    row = re.search(r"^\| %s \| (\d+) \| (\d+) \|" % STAGE_KERNEL[stage], text, re.M)
-    return int(row.group(1)) + int(row.group(2)) if row else None
+    names = list(STAGE_KERNEL.values()) if stage == "step" else [STAGE_KERNEL[stage]]
+    total = 0
+    for nm in names:
+        row = re.search(r"^\| %s \| (\d+) \| (\d+) \|" % nm, text, re.M)
+        if not row:
+            return None
+        total += int(row.group(1)) + int(row.group(2))
+    return total
+
+
+def append_context(rtp, lay, inp, w_k, dev):
+    """Append every sequence's whole context to `lay`'s cache.  With local heads
+    in ring mode each sequence goes on its own (a batch-1 view of its cache
+    slice), so rows past its own length never take slots of its window."""
+    sh = inp["shape"]
+    B = sh.batch
+    if not lay.ring:
+        lay.append(inp["k_pre"].to(dev), inp["v"].to(dev), torch.zeros(B, dtype=torch.int32, device=dev), w_k)
+        return
+    c = lay.cfg
+    cfg1 = rtp.rtp_layer_cfg.from_buffer_copy(c)
+    cfg1.batch = 1
+    zero = torch.zeros(1, dtype=torch.int32, device=dev)
+    for b in range(B):
+        L = int(inp["seq_len"][b])
+        cache1 = rtp.rtp_cache(lay.k[b].data_ptr(), lay.v[b].data_ptr(), lay.kidx[b].data_ptr(),
+                               lay.status.data_ptr())
+        rtp.rtp_append_kv(cfg1, cache1, inp["k_pre"][b:b + 1, :L].contiguous().to(dev),
+                          inp["v"][b:b + 1, :L].contiguous().to(dev), zero, L, w_k)
+        torch.cuda.synchronize()
+
+
+def cache_memory(rtp, cfg) -> dict:
+    """Bytes of the layer's cache with local heads in ring mode (sinks + a
+    window ring) against the full-context cache of every head."""
+    import ctypes
+    k, v, ki = rtp.rtp_cache_bytes(cfg)
+    full = rtp.rtp_layer_cfg.from_buffer_copy(cfg)
+    full.local_cap = 0
+    kf, vf, kif = rtp.rtp_cache_bytes(full)
+    used, whole = k + v + ki, kf + vf + kif
+    return {"cache_bytes": used, "full_cache_bytes": whole, "memory_sparsity": round(1.0 - used / whole, 4)}
 
 
 def l2_bytes() -> int:
@@ -236,8 +276,7 @@ def run_ours(args, dist: Dist) -> dict:
     seq_len = inp["seq_len"]
     Lh = int(seq_len.max())
     dt = sh.torch_dtype
-    cfg = rtp.make_cfg(B, Hq, Hkv, D, Lmax, sh.n_sink, sh.window, sh.top_p, sh.retrieval, sh.dtype,
-                       sh.rope_base)
+    ring = 0 if args.full_cache else sh.window
 
     # device inputs
     w_q = inp["w_q"].to(dev)
@@ -250,12 +289,10 @@ def run_ours(args, dist: Dist) -> dict:
     v_new = inp["v"][bidx, lastc][:, None].contiguous().to(dev)
     q = inp["q_pre"].to(dev)
 
-    # replica 0: the context (every sequence's first seq_len-1 tokens)
-    lay0 = rtp.Layer(sh, Lmax, device=dev)
-    kp = inp["k_pre"].to(dev)
-    vv = inp["v"].to(dev)
-    lay0.append(kp, vv, torch.zeros(B, dtype=torch.int32, device=dev), w_k)
-    del kp, vv
+    # replica 0: the context (local heads keep sinks + a window ring unless --full-cache)
+    lay0 = rtp.Layer(sh, Lmax, device=dev, local_cap=ring)
+    cfg = lay0.cfg
+    append_context(rtp, lay0, inp, w_k, dev)
     torch.cuda.synchronize()
 
     # selection + bytes per step (one decode with the optional selection outputs)
@@ -410,8 +447,12 @@ def run_ours(args, dist: Dist) -> dict:
     if not torch.equal(h_out, out0.cpu()):
         raise RuntimeError("end-to-end output differs from the device-resident output")
 
-    # roofline of the dominant kernel
-    dominant = max(kern_us, key=lambda s: kern_us[s])
+    # Roofline.  The step's four launches are chained by programmatic dependent
+    # launch and overlap, and a launch bracketed alone by events carries several
+    # microseconds of launch latency (an almost empty kernel measures ~9 us), so
+    # the HBM-bound unit whose duration the events resolve is the step: its
+    # algorithmic bytes over the device time of the timed steps.  The
+    # per-kernel figures (each launch alone, launch latency included) follow.
     kbytes = {"append": nbytes["append"], "decode_score": nbytes["score"], "decode_select": nbytes["kept"],
               "decode_local": nbytes["sw"] + nbytes["qo"]}
     peaks = {}
@@ -419,32 +460,37 @@ def run_ours(args, dist: Dist) -> dict:
         peaks = json.load(open(PEAKS_PATH))
     peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
     peak_src = "measured" if "hbm_gbs" in peaks else "fallback"
-    ach = kbytes[dominant] / (kern_us[dominant] * 1e-6) / 1e9
+    step_us = ms_max * 1e3 / K
+    ach = nbytes["total"] / (step_us * 1e-6) / 1e9
+    per_kernel = {k: {"us": round(kern_us[k], 3), "bytes": kbytes[k],
+                      "gbs": round(kbytes[k] / (kern_us[k] * 1e-6) / 1e9, 1)} for k in kern_us}
     tokens = K * B * dist.world
     us_per_token = ms_max * 1e3 / tokens
     return dict(
         us_per_token=us_per_token, ms_per_step=ms_max / K, shape=sh, n_rep=n_rep, nbytes=nbytes,
-        kept_out=kept_out, counts=cnt.cpu().numpy(), kern_us=kern_us, dominant=dominant,
-        roofline={"bound": "hbm", "kernel": dominant, "achieved": round(ach, 1), "peak": peak,
-                  "peak_source": peak_src, "unit": "GB/s", "frac": round(ach / peak, 4),
-                  "bytes_per_launch": kbytes[dominant],
-                  "traffic": measured_traffic(dominant, args.workload)},
+        kept_out=kept_out, counts=cnt.cpu().numpy(), kern_us=kern_us,
+        roofline={"bound": "hbm", "kernel": "decode step (append, score, sink/window, select kernels)",
+                  "achieved": round(ach, 1), "peak": peak, "peak_source": peak_src, "unit": "GB/s",
+                  "frac": round(ach / peak, 4), "bytes_per_launch": nbytes["total"],
+                  "traffic": measured_traffic("step", args.workload), "per_kernel": per_kernel},
         e2e={"value": e2e_s * 1e6 / (n_e * B * dist.world), "unit": "µs/token",
              "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e},
         clocks=(clocks.summary(t_wall0, t_wall1) if clocks else None),
-        gpu_launches=K * (4 if R else 2), l2=l2, inp=inp, Lh=Lh,
+        gpu_launches=K * (4 if R else 2), l2=l2, inp=inp, Lh=Lh, memory=cache_memory(rtp, cfg),
     )
 
 
 # ---------------------------------------------------------------------------
 # extra lines of the metric: 1M-token decode and the 32K prefill chunk
 # ---------------------------------------------------------------------------
-def decode_extra(name: str, dev, steps: int) -> dict:
-    """µs/token of (append + decode) on workload `name`: CUDA-graph replays over
-    replica caches whose bytes per step sum to more than twice the L2."""
+def decode_extra(name: str, dev, steps: int, top_p=None, ring: bool = True) -> dict:
+    """µs/token of (append + decode) on workload `name` (optionally another p):
+    CUDA-graph replays over replica caches whose bytes per step sum to more
+    than twice the L2.  Local heads keep a window ring unless ring=False."""
     import head_wise_sparse_local_b200 as rtp
     from synth import make_decode_inputs, workload
-    inp = make_decode_inputs(workload(name))
+    kw = {} if top_p is None else {"shape_top_p": top_p}
+    inp = make_decode_inputs(workload(name, **kw))
     sh = inp["shape"]
     B, Hq, D = sh.batch, sh.n_q_heads, sh.head_dim
     Lmax, seq_len = inp["max_ctx"], inp["seq_len"]
@@ -457,8 +503,8 @@ def decode_extra(name: str, dev, steps: int) -> dict:
     k_new = inp["k_pre"][bidx, lastc][:, None].contiguous().to(dev)
     v_new = inp["v"][bidx, lastc][:, None].contiguous().to(dev)
     q = inp["q_pre"].to(dev)
-    lay0 = rtp.Layer(sh, Lmax, device=dev)
-    lay0.append(inp["k_pre"].to(dev), inp["v"].to(dev), torch.zeros(B, dtype=torch.int32, device=dev), w_k)
+    lay0 = rtp.Layer(sh, Lmax, device=dev, local_cap=sh.window if ring else 0)
+    append_context(rtp, lay0, inp, w_k, dev)
     NR = max(sh.n_retrieval * sh.group, 1)
     bm = torch.zeros((B, NR, (Lmax + 31) // 32), dtype=torch.int32, device=dev)
     cnt = torch.zeros((B, NR), dtype=torch.int32, device=dev)
@@ -503,9 +549,18 @@ def decode_extra(name: str, dev, steps: int) -> dict:
     if sum(int(r["status"].item()) for r in reps):
         raise RuntimeError(f"device status set during the {name} steps")
     us = e0.elapsed_time(e1) * 1e3 / (n_graph * n_rep * B)
-    return {"us_per_token": round(us, 3), "hbm_gbs": round(nbytes["total"] / (us * B * 1e-6) / 1e9, 1),
-            "bytes_per_step": nbytes["total"], "steps": n_graph * n_rep, "replicas": n_rep,
-            "kept_per_head": cnt.cpu().numpy().tolist()}
+    peak = _peak_hbm()
+    gbs = nbytes["total"] / (us * B * 1e-6) / 1e9
+    return {"us_per_token": round(us, 3), "us_per_step": round(us * B, 3), "hbm_gbs": round(gbs, 1),
+            "frac": round(gbs / peak, 4), "batch": B, "top_p": sh.top_p,
+            "seq_len": [int(x) for x in seq_len], "bytes_per_step": nbytes["total"],
+            "steps": n_graph * n_rep, "replicas": n_rep, "kept_per_head": cnt.cpu().numpy().tolist(),
+            **cache_memory(rtp, lay0.cfg)}
+
+
+def _peak_hbm() -> float:
+    peaks = json.load(open(PEAKS_PATH)) if os.path.exists(PEAKS_PATH) else {}
+    return float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
 
 
 def _popcount_words(w: torch.Tensor, lut: torch.Tensor) -> torch.Tensor:
@@ -556,7 +611,19 @@ def prefill_extra(dev, reps: int, T: int = 0) -> dict:
     lay = rtp.Layer(sh, inp["max_ctx"], device=dev, prefill_T=T)
     w_q, w_k = inp["w_q"].to(dev), inp["w_k"].to(dev)
     start = torch.zeros(B, dtype=torch.int32, device=dev)
-    lay.append(inp["k_pre"][:, :T].contiguous().to(dev), inp["v"][:, :T].contiguous().to(dev), start, w_k)
+    k_chunk = inp["k_pre"][:, :T].contiguous().to(dev)
+    v_chunk = inp["v"][:, :T].contiguous().to(dev)
+    lay.append(k_chunk, v_chunk, start, w_k)
+    torch.cuda.synchronize()
+    ap = []  # the chunk's rtp_append_kv (RoPE'd K, V and indexer keys of T tokens), timed beside it
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lay.append(k_chunk, v_chunk, start, w_k)
+        e1.record()
+        torch.cuda.synchronize()
+        ap.append(e0.elapsed_time(e1))
+    del k_chunk, v_chunk
     q = inp["q_pre"].to(dev)
     out = torch.empty((B, T, Hq, D), dtype=sh.torch_dtype, device=dev)
     NR = sh.n_retrieval * sh.group
@@ -594,22 +661,33 @@ def prefill_extra(dev, reps: int, T: int = 0) -> dict:
     peaks = json.load(open(PEAKS_PATH)) if os.path.exists(PEAKS_PATH) else {}
     peak = float(peaks.get("bf16_tflops", 1590.0))
     att_tf = flops / (kern["prefill_attn"] * 1e-3) / 1e12
-    return {"ms": round(float(np.median(ts)), 4), "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
+    append_ms = float(np.median(ap))
+    return {"ms": round(float(np.median(ts)), 4), "append_ms": round(append_ms, 4),
+            "ms_with_append": round(float(np.median(ts)) + append_ms, 4),
+            "kernels_ms": {k: round(v, 4) for k, v in kern.items()},
             "attended_pairs": pairs, "attn_flop": flops,
             "roofline": {"bound": "tensor", "kernel": "prefill_attn", "achieved": round(att_tf, 1),
                          "peak": peak, "peak_source": "measured" if "bf16_tflops" in peaks else "fallback",
                          "unit": "TFLOP/s", "frac": round(att_tf / peak, 4),
-                         "note": "mma.sync m16n8k16 bf16 path (legacy tensor-core instructions)"},
+                         "note": "tcgen05.mma kind::f16 (bf16, fp32 accumulators in TMEM), TMA-staged K/V; "
+                                 "algorithmic FLOP = 4 D per attended (row, key) pair"},
             "data": f"T = {T}; q alone {B * T * Hq * D * 2 / 1e6:.0f} MB" + (" (larger than L2)" if B * T * Hq * D * 2 > l2_bytes() else "")}
 
 
 # ---------------------------------------------------------------------------
 # the oracle, timed on the host cores
 # ---------------------------------------------------------------------------
+def oracle_threads() -> int:
+    return max(1, os.cpu_count() or 1)
+
+
 def oracle_step_time(inp, budget_s: float, max_steps: int, warmup: int = 0, warm_budget_s: float = 0.0):
     """Time (append the decode token + decode) with the fp64 oracle after up to
     `warmup` untimed steps (at least one when asked for, then while
-    `warm_budget_s` lasts); returns (seconds per step, steps, threads, warm-up steps)."""
+    `warm_budget_s` lasts).  The decode's query heads run on a pool of host
+    threads (numpy releases the interpreter lock in its array work), one BLAS
+    thread each.  Returns (seconds per step, steps, threads, warm-up steps)."""
+    import concurrent.futures as cf
     import oracle
     from threadpoolctl import threadpool_limits
     sh = inp["shape"]
@@ -621,22 +699,70 @@ def oracle_step_time(inp, budget_s: float, max_steps: int, warmup: int = 0, warm
     bidx = torch.arange(B)
     k1 = inp["k_pre"][bidx, lastc][:, None]
     v1 = inp["v"][bidx, lastc][:, None]
-    with threadpool_limits(1):
+    n_thr = min(oracle_threads(), sh.n_q_heads)
+    chunks = [list(range(sh.n_q_heads))[i::n_thr] for i in range(n_thr)]
+
+    def one_step(pool):
+        oc.append(k1, v1, ctx, 1, inp["w_k"])
+        futs = [pool.submit(oracle.decode, oc, inp["q_pre"], inp["seq_len"], inp["w_q"], None, None, hs)
+                for hs in chunks]
+        for f in futs:
+            f.result()
+
+    with threadpool_limits(1), cf.ThreadPoolExecutor(n_thr) as pool:
         n_warm = 0
         t_start = time.perf_counter()
         while n_warm < warmup and (n_warm == 0 or (time.perf_counter() - t_start) < warm_budget_s):
-            oc.append(k1, v1, ctx, 1, inp["w_k"])
-            oracle.decode(oc, inp["q_pre"], inp["seq_len"], inp["w_q"])
+            one_step(pool)
             n_warm += 1
         times = []
         t_start = time.perf_counter()
         while len(times) < max_steps and (time.perf_counter() - t_start) < budget_s:
             t0 = time.perf_counter()
-            # per-sequence append at its own position (T = 1)
-            oc.append(k1, v1, ctx, 1, inp["w_k"])
-            oracle.decode(oc, inp["q_pre"], inp["seq_len"], inp["w_q"])
+            one_step(pool)
             times.append(time.perf_counter() - t0)
-    return float(np.mean(times)), len(times), 1, n_warm
+    return float(np.mean(times)), len(times), n_thr, n_warm
+
+
+def prefill_cpu_baseline(T: int, budget_s: float, n_rows: int = 512) -> dict:
+    """The fp64 oracle on a seeded subset of the 32K prefill chunk's query rows
+    (the last n_rows / 2 rows and n_rows / 2 drawn from the rest), rows spread
+    over host threads; the chunk's time is extrapolated by causal (row, key)
+    pairs, which the retrieval heads' work grows with."""
+    import concurrent.futures as cf
+    import oracle
+    from synth import make_prefill_inputs, workload
+    from threadpoolctl import threadpool_limits
+    inp = make_prefill_inputs(workload("prefill_32k_bf16"), T=T)
+    sh = inp["shape"]
+    oc = oracle.OracleCache(sh, inp["max_ctx"])
+    oc.append_in_place(inp["k_pre"], inp["v"], np.array([T]), inp["w_k"])  # setup, untimed
+    rng = np.random.default_rng(7)
+    last = np.arange(T - n_rows // 2, T)
+    rest = np.sort(rng.choice(T - n_rows // 2, size=n_rows // 2, replace=False))
+    rows = [int(t) for t in np.concatenate([rest, last])]
+    n_thr = oracle_threads()
+    done, t_used = [], 0.0
+    with threadpool_limits(1), cf.ThreadPoolExecutor(n_thr) as pool:
+        t0 = time.perf_counter()
+        # batches of rows until the budget is spent (later rows cost more: interleave)
+        order = rows[::2] + rows[1::2]
+        for i in range(0, len(order), n_thr):
+            batch = order[i:i + n_thr]
+            futs = [pool.submit(oracle.prefill, oc, inp["q_pre"], inp["start_pos"], inp["w_q"], [t]) for t in batch]
+            for f in futs:
+                f.result()
+            done += batch
+            t_used = time.perf_counter() - t0
+            if t_used > budget_s:
+                break
+    pairs_all = T * (T + 1) / 2.0
+    pairs_done = float(sum(t + 1 for t in done))
+    est_ms = t_used * pairs_all / pairs_done * 1e3
+    return {"value": round(est_ms, 1), "unit": "ms/chunk", "cores": n_thr, "kind": "oracle",
+            "sample": f"{len(done)} of the {T} query rows (the last {n_rows // 2} and a seeded draw of the "
+                      f"rest), all 32 query heads each, {t_used:.1f} s on {n_thr} host threads; the chunk's "
+                      f"time extrapolated by causal (row, key) pairs"}
 
 
 def run_reference(args, dist: Dist) -> dict:
@@ -667,6 +793,8 @@ def main():
     ap.add_argument("--prefill-only", action="store_true",
                     help="time only the prefill chunk (profiling); prints its JSON object")
     ap.add_argument("--prefill-T", type=int, default=0, help="prefill chunk length (default 32768)")
+    ap.add_argument("--full-cache", action="store_true",
+                    help="local heads keep the whole context (default: sinks + a window ring)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -715,13 +843,19 @@ def main():
     if dist.rank == 0 and dist.world == 1 and not args.no_extras:
         dev = torch.device("cuda", dist.local_rank)
         extras = {}
-        for name, fn in (("decode_1m_bf16", lambda: decode_extra("decode_1m_bf16", dev, args.extra_steps)),
-                         ("prefill_32k_bf16", lambda: prefill_extra(dev, 5))):
+        items = [("decode_1m_bf16", lambda: decode_extra("decode_1m_bf16", dev, args.extra_steps))]
+        for p in (0.8, 0.95, 0.99):
+            items.append((f"ragged_decode_b8_8k_32k_bf16_p{p}",
+                          lambda p=p: decode_extra("ragged_decode_b8_8k_32k_bf16", dev, args.extra_steps, top_p=p)))
+        items.append(("prefill_32k_bf16", lambda: prefill_extra(dev, 5)))
+        for name, fn in items:
             try:
                 extras[name] = fn()
             except torch.cuda.OutOfMemoryError as e:  # pragma: no cover - depends on the device
                 extras[name] = {"skipped": f"out of device memory: {e}"}
             torch.cuda.empty_cache()
+        if not args.no_cpu_baseline and "prefill_32k_bf16" in extras and "ms" in extras["prefill_32k_bf16"]:
+            extras["prefill_32k_bf16"]["cpu_baseline"] = prefill_cpu_baseline(32768, args.cpu_budget)
     if dist.rank == 0:
         tot_bytes = r["nbytes"]["total"]
         gbs = tot_bytes * args.steps * dist.world / (r["ms_per_step"] * args.steps * 1e-3) / 1e9
@@ -740,6 +874,7 @@ def main():
             "bytes_per_step": tot_bytes,
             "kernels_us": {k: round(v, 3) for k, v in r["kern_us"].items()},
             "kept_per_head": r["counts"].tolist(),
+            "memory": r["memory"],
             "roofline": r["roofline"],
             "cpu_baseline": cpu,
             "e2e": {k: (round(v, 3) if isinstance(v, float) else v) for k, v in r["e2e"].items()},

@@ -61,13 +61,13 @@ def _stream(stream) -> Optional[int]:
 def make_cfg(batch: int, n_q_heads: int, n_kv_heads: int, head_dim: int, max_ctx: int,
              n_sink: int, window: int, top_p: float, retrieval: Sequence[int],
              dtype: str = "bf16", rope_base: float = 10000.0, idx_dim: int = 16,
-             local_cap: int = 0) -> rtp_layer_cfg:
+             local_cap: int = 0, top_k: int = 0) -> rtp_layer_cfg:
     mask = 0
     for h in retrieval:
         mask |= 1 << int(h)
     return rtp_layer_cfg(batch, n_q_heads, n_kv_heads, head_dim, idx_dim, max_ctx, n_sink, window,
                          top_p, rope_base, mask, RTP_BF16 if dtype == "bf16" else RTP_FP32,
-                         int(local_cap))
+                         int(local_cap), int(top_k))
 
 
 def rtp_version() -> str:
@@ -157,7 +157,7 @@ class Layer:
         self.shape = shape
         self.cfg = make_cfg(shape.batch, shape.n_q_heads, shape.n_kv_heads, shape.head_dim, max_ctx,
                             shape.n_sink, shape.window, shape.top_p, shape.retrieval, shape.dtype,
-                            shape.rope_base, shape.idx_dim, local_cap)
+                            shape.rope_base, shape.idx_dim, local_cap, getattr(shape, "top_k", 0))
         self.max_ctx = max_ctx
         dt = torch.bfloat16 if shape.dtype == "bf16" else torch.float32
         B, Hkv, D, R = shape.batch, shape.n_kv_heads, shape.head_dim, shape.n_retrieval

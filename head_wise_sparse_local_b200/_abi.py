@@ -39,7 +39,7 @@ class rtp_layer_cfg(ctypes.Structure):
                 ("head_dim", ctypes.c_int), ("idx_dim", ctypes.c_int), ("max_ctx", ctypes.c_int),
                 ("n_sink", ctypes.c_int), ("window", ctypes.c_int), ("top_p", ctypes.c_float),
                 ("rope_base", ctypes.c_float), ("retrieval_mask", ctypes.c_uint64),
-                ("dtype", ctypes.c_int), ("local_cap", ctypes.c_int)]
+                ("dtype", ctypes.c_int), ("local_cap", ctypes.c_int), ("top_k", ctypes.c_int)]
 
 
 class rtp_cache(ctypes.Structure):

@@ -83,6 +83,7 @@ struct DecodeArgs {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W, max_seq_len, words;
   int lstride;      // row stride of the score scratch (Lmax rounded up to 32)
   float top_p, rope_base;
+  int top_k;        // > 0: static top-k instead of top-p
   const void* q_pre;
   const float* w_q;
   void* out;
@@ -864,6 +865,13 @@ __device__ __forceinline__ void mass_split36(float s, float m, unsigned& hi, uns
   lo = __float2uint_rn(fmaf(hf, -262144.0f, x));
 }
 
+// Weight of an item in the threshold search: its softmax mass in 2^-36 fixed
+// point (top-p), or 1 (static top-k: "the shortest prefix whose weight reaches
+// k" is then exactly the k highest scores, ties to the lower index).
+__device__ __forceinline__ unsigned long long item_w(float s, float m, bool cnt) {
+  return cnt ? 1ull : mass36(s, m);
+}
+
 struct DigitResult {
   int digit;
   unsigned long long above;
@@ -891,7 +899,7 @@ struct Items {
 // launch reaches for the first time costs an instruction fetch from L2).
 template <bool kMass>
 __device__ __noinline__ DigitResult radix_step(const Items& it, int n, uint32_t prefix, uint32_t mask,
-                                  uint32_t key_eq, int shift, float m, unsigned long long need,
+                                  uint32_t key_eq, int shift, float m, bool cntw, unsigned long long need,
                                   unsigned long long* h_m, unsigned* h_c, DigitResult* s_res) {
   const int tid = threadIdx.x;
   for (int i = tid; i < 256; i += blockDim.x) { h_m[i] = 0ull; h_c[i] = 0u; }
@@ -903,7 +911,7 @@ __device__ __noinline__ DigitResult radix_step(const Items& it, int n, uint32_t 
     if constexpr (kMass) {
       if ((e.x & mask) == prefix) {
         const int dg = (e.x >> shift) & 255;
-        atomicAdd(&h_m[dg], mass36(key_score(e.x), m));
+        atomicAdd(&h_m[dg], item_w(key_score(e.x), m, cntw));
         atomicAdd(&h_c[dg], 1u);
       }
     } else {
@@ -954,7 +962,7 @@ __device__ __noinline__ DigitResult radix_step(const Items& it, int n, uint32_t 
 // Exact tau / j_cut among n items whose mass must supply `need` (one CTA).
 // Order: key descending, index ascending.  The kept set is the shortest prefix
 // whose mass reaches `need`.
-__device__ __noinline__ void solve_radix(const Items& it, int n, float m, unsigned long long need,
+__device__ __noinline__ void solve_radix(const Items& it, int n, float m, bool cntw, unsigned long long need,
                             unsigned long long* h_m, unsigned* h_c, DigitResult* s_res,
                             uint32_t* s_kr, float& tau, int& jcut) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -994,7 +1002,7 @@ __device__ __noinline__ void solve_radix(const Items& it, int n, float m, unsign
     mask = (hb == 31) ? 0u : ~((2u << hb) - 1u);
     prefix = kmin & mask;
     for (int shift = (hb / 8) * 8; shift >= 0; shift -= 8) {
-      const DigitResult d = radix_step<true>(it, n, prefix, mask, 0u, shift, m, need, h_m, h_c, s_res);
+      const DigitResult d = radix_step<true>(it, n, prefix, mask, 0u, shift, m, cntw, need, h_m, h_c, s_res);
       need -= d.above;
       cnt_eq = d.cnt_digit;
       prefix |= (uint32_t)d.digit << shift;
@@ -1004,7 +1012,7 @@ __device__ __noinline__ void solve_radix(const Items& it, int n, float m, unsign
     cnt_eq = n_items;  // every item has the same key
   }
   const uint32_t tau_key = prefix;
-  const unsigned long long w_tau = mass36(key_score(tau_key), m);
+  const unsigned long long w_tau = item_w(key_score(tau_key), m, cntw);
   unsigned long long kk = (w_tau > 0ull) ? (need + w_tau - 1ull) / w_tau : (unsigned long long)cnt_eq;
   if (kk < 1ull) kk = 1ull;
   if (kk > cnt_eq) kk = cnt_eq;
@@ -1013,7 +1021,7 @@ __device__ __noinline__ void solve_radix(const Items& it, int n, float m, unsign
     uint32_t ip = 0u, im = 0u;
     unsigned long long want = kk;
     for (int shift = 16; shift >= 0; shift -= 8) {
-      const DigitResult d = radix_step<false>(it, n, ip, im, tau_key, shift, 0.f, want, h_m, h_c, s_res);
+      const DigitResult d = radix_step<false>(it, n, ip, im, tau_key, shift, 0.f, cntw, want, h_m, h_c, s_res);
       want -= d.above;
       ip |= (uint32_t)d.digit << shift;
       im |= 0xffu << shift;
@@ -1026,7 +1034,7 @@ __device__ __noinline__ void solve_radix(const Items& it, int n, float m, unsign
 
 // Exact tau / j_cut for n <= blockDim.x list items: item i is kept iff the
 // mass of the items ordered before it is below `need`.
-__device__ __noinline__ void solve_brute(const uint2* items, int n, float m, unsigned long long need,
+__device__ __noinline__ void solve_brute(const uint2* items, int n, float m, bool cntw, unsigned long long need,
                                          uint4* pack, uint32_t* s_min, int* s_jmax, float& tau, int& jcut) {
   // pack[i] = (key, index, mass lo, mass hi): one 16-byte broadcast load per
   // item in the pairwise loop (pack must not overlap items)
@@ -1034,7 +1042,7 @@ __device__ __noinline__ void solve_brute(const uint2* items, int n, float m, uns
   uint2 me = make_uint2(0u, 0u);
   if (tid < n) {
     me = items[tid];
-    const unsigned long long w = mass36(key_score(me.x), m);
+    const unsigned long long w = item_w(key_score(me.x), m, cntw);
     pack[tid] = make_uint4(me.x, me.y, (unsigned)w, (unsigned)(w >> 32));
   }
   if (tid == 0) { *s_min = 0xffffffffu; *s_jmax = -1; }
@@ -1088,11 +1096,11 @@ struct SelShared {
 
 // Exact tau / j_cut for n <= 32 items by one warp (lane i owns item i): an item
 // is kept iff the mass of the items ordered before it is below `need`.
-__device__ void solve_warp(const uint2* items, int n, float m, unsigned long long need, float& tau,
+__device__ void solve_warp(const uint2* items, int n, float m, bool cntw, unsigned long long need, float& tau,
                            int& jcut) {
   const int lane = threadIdx.x & 31;
   const uint2 me = lane < n ? items[lane] : make_uint2(0u, 0u);
-  const unsigned long long w = lane < n ? mass36(key_score(me.x), m) : 0ull;
+  const unsigned long long w = lane < n ? item_w(key_score(me.x), m, cntw) : 0ull;
   unsigned long long before = 0ull;
 #pragma unroll 4
   for (int j = 0; j < n; ++j) {
@@ -1242,7 +1250,8 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
     mbar_wait_bounded(&s_sbar, 0, a.wait_ns, a.status);  // the copy, before going on (output invalid)
   const int j1 = min(L, jh);  // j1 <= j0: nothing of this sequence in this CTA's share
   uint32_t* mask = a.mask + (size_t)bh * a.words;
-  const bool keep_all = a.top_p >= 1.0f;
+  const bool cntw = a.top_k > 0;  // static top-k: unit weights
+  const bool keep_all = !cntw && a.top_p >= 1.0f;
   float tau = -CUDART_INF_F;
   int jcut = INT_MAX;
   bool via_top = false;  // the tail reads only the top-rung items (tier 1, no bitmask)
@@ -1256,7 +1265,9 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
       for (int c = tid + kSelThreads; c < nch; c += kSelThreads) v = fmaxf(v, __ldcg(cm + c));
       m = block_max<kSelThreads>(v, sh->red);
     }
-    const float m_lo = m - 26.0f;  // exp(s - m) 2^36 rounds to 0 below m - 25.65
+    // exp(s - m) 2^36 rounds to 0 below m - 25.65: such scores weigh nothing
+    // (top-p); with unit weights every score counts
+    const float m_lo = cntw ? -CUDART_INF_F : m - 26.0f;
     SelShared<CS>* lead = cl.map_shared_rank(sh, 0);
     uint2* lead_cand = cl.map_shared_rank(s_cand, 0);
 
@@ -1287,7 +1298,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
           const int j = c0 + u * kSelThreads + tid;
           const float sv = j < c1 ? s_lg[j - c0] : -CUDART_INF_F;
           if (sv > m_lo) {
-            const float x = mass_x36(sv, m);
+            const float x = cntw ? 1.0f : mass_x36(sv, m);
             if (sv < top_lo) {  // x < 2^36 e^-8 < 2^25
               zs32 += __float2uint_rn(x);
             } else {
@@ -1394,7 +1405,8 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
     unsigned Ck[kRungs];
 #pragma unroll
     for (int k = 0; k < kRungs; ++k) { Mk[k] = sh->tot_m[1 + k]; Ck[k] = sh->tot_c[k]; }
-    unsigned long long target = (unsigned long long)ceil((double)a.top_p * (double)Z);
+    unsigned long long target = cntw ? (unsigned long long)a.top_k
+                                     : (unsigned long long)ceil((double)a.top_p * (double)Z);
     if (target > Z) target = Z;
     if (target < 1ull) target = 1ull;
     // lowest rung whose scores already hold the target mass: the kept set lies
@@ -1480,7 +1492,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
             for (int k = 0; k < RPL; ++k)
               for (unsigned i = 0; i < cr[k]; ++i) s_small[off++] = s_cand[(lane * RPL + k) * kTopPerWarp + i];
             __syncwarp();
-            solve_warp(s_small, n, m, target, t_tau, t_jcut);
+            solve_warp(s_small, n, m, cntw, target, t_tau, t_jcut);
           }
           done = true;
         } else if (tier1) {
@@ -1518,11 +1530,11 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
         }
         if (done) {
         } else if (n <= 32) {
-          if (warp == 0) solve_warp(s_cand, n, m, target, t_tau, t_jcut);
+          if (warp == 0) solve_warp(s_cand, n, m, cntw, target, t_tau, t_jcut);
         } else if (n <= kBruteMax) {
-          solve_brute(s_cand, n, m, target, reinterpret_cast<uint4*>(s_cand + kCandSmem / 2), &s_min, &s_jmax, t_tau, t_jcut);
+          solve_brute(s_cand, n, m, cntw, target, reinterpret_cast<uint4*>(s_cand + kCandSmem / 2), &s_min, &s_jmax, t_tau, t_jcut);
         } else {
-          solve_radix(Items{s_cand, false}, n, m, target, r_hm, r_hc, &s_dres, s_kr, t_tau, t_jcut);
+          solve_radix(Items{s_cand, false}, n, m, cntw, target, r_hm, r_hc, &s_dres, s_kr, t_tau, t_jcut);
         }
         if (warp == 0 && lane < CS) {
           SelShared<CS>* rem = cl.map_shared_rank(sh, lane);
@@ -1557,7 +1569,12 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
             for (int u = 0; u < 4; ++u) {
               if (!on[u]) continue;
               unsigned hi, lo;
-              mass_split36(sv[u], m, hi, lo);
+              if (cntw) {
+                hi = 0u;
+                lo = 1u;
+              } else {
+                mass_split36(sv[u], m, hi, lo);
+              }
               const int bk = score_bucket(sv[u]);
               if (hi) atomicAdd(&s_hi[bk], hi);
               if (lo) atomicAdd(&s_lo[bk], lo);
@@ -1659,7 +1676,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
               sv[u] = 0.f;
               if (j < c1) {
                 sv[u] = s_lg[j - c0];
-                in[u] = sv[u] > m_lo && score_bucket(sv[u]) == bucket && mass36(sv[u], m) != 0ull;
+                in[u] = sv[u] > m_lo && score_bucket(sv[u]) == bucket && (cntw || mass36(sv[u], m) != 0ull);
               }
             }
 #pragma unroll
@@ -1701,9 +1718,9 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
             items = Items{gcand, true};
           }
           if (n <= kBruteMax)
-            solve_brute(s_cand, n, m, need, reinterpret_cast<uint4*>(s_cand + kCandSmem / 2), &s_min, &s_jmax, t_tau, t_jcut);
+            solve_brute(s_cand, n, m, cntw, need, reinterpret_cast<uint4*>(s_cand + kCandSmem / 2), &s_min, &s_jmax, t_tau, t_jcut);
           else
-            solve_radix(items, n, m, need, r_hm, r_hc, &s_dres, s_kr, t_tau, t_jcut);
+            solve_radix(items, n, m, cntw, need, r_hm, r_hc, &s_dres, s_kr, t_tau, t_jcut);
         }
         if (tid < CS) {
           SelShared<CS>* rem = cl.map_shared_rank(sh, tid);
@@ -2118,7 +2135,7 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   a.max_seq_len = max_seq_len > 0 ? max_seq_len : sh.Lmax;
   a.words = (sh.Lmax + 31) / 32;
   a.lstride = (sh.Lmax + 31) & ~31;
-  a.top_p = sh.top_p; a.rope_base = sh.rope_base;
+  a.top_p = sh.top_p; a.rope_base = sh.rope_base; a.top_k = sh.top_k;
   a.q_pre = q_pre; a.w_q = w_q; a.out = out;
   a.k = cache->k; a.v = cache->v; a.kidx = cache->kidx; a.status = cache->status;
   a.seq_len = seq_len; a.sel_count = sel_count;

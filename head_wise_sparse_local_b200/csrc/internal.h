@@ -41,6 +41,7 @@ struct KvMap {
 struct Shape {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W;
   int ring;          // window rows a local head keeps in ring mode (0: whole context)
+  int top_k;         // > 0: retrieval heads keep a fixed k tokens (static top-k) instead of top-p
   KvMap kv;
   float top_p, rope_base;
   int dtype;  // rtp_dtype

@@ -90,6 +90,8 @@ int make_shape(const rtp_layer_cfg* cfg, Shape* sh) {
   sh->R = r;
   sh->NR = r * G;
   if (cfg->local_cap < 0) return fail(RTP_ERR_INVALID, "local_cap must be >= 0");
+  if (cfg->top_k < 0) return fail(RTP_ERR_INVALID, "top_k must be >= 0");
+  sh->top_k = cfg->top_k;
   if (cfg->local_cap > 0 && cfg->local_cap < cfg->window)
     return fail(RTP_ERR_SHAPE, "local_cap must be 0 or at least the window");
   // ring mode only when it actually saves rows
@@ -227,6 +229,8 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
   if (rc != RTP_OK) return rc;
   if ((rc = check_cache(sh, cache)) != RTP_OK) return rc;
   if (T < 1 || T > sh.Lmax) return fail(RTP_ERR_SHAPE, "T must be in [1, max_ctx]");
+  if (sh.top_k > 0)
+    return fail(RTP_ERR_SHAPE, "static top-k (cfg top_k > 0) is a decode-only variant; prefill selects by top-p");
   if (sh.ring > 0 && (long long)T + sh.W - 1 > sh.ring)
     return fail(RTP_ERR_SHAPE, "ring mode: a prefill chunk needs local_cap >= T + window - 1");
   if (!q_pre || !start_pos || !out) return fail(RTP_ERR_INVALID, "q_pre/start_pos/out is NULL");

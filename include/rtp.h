@@ -83,6 +83,12 @@ typedef enum rtp_dtype { RTP_BF16 = 0, RTP_FP32 = 1 } rtp_dtype;
  *                 the full KV cache is kept for retrieval heads only).  A
  *                 prefill chunk of T tokens then needs local_cap >= T + W - 1.
  *                 Ignored (whole context kept) when S + local_cap >= max_ctx.
+ *   top_k         0: top-p selection.  k > 0: static top-k, the pages' fixed-
+ *                 budget baseline (atlas.scime.ai summary, "Key results" and
+ *                 "Baselines": static top-k): retrieval query heads keep the k
+ *                 highest indexer scores (ties to the lower index; every token
+ *                 when k >= the context), united with sinks and window as for
+ *                 top-p.  Decode only: rtp_prefill_attn returns RTP_ERR_SHAPE.
  */
 typedef struct rtp_layer_cfg {
   int batch;
@@ -98,6 +104,7 @@ typedef struct rtp_layer_cfg {
   uint64_t retrieval_mask;
   int dtype;
   int local_cap;
+  int top_k;
 } rtp_layer_cfg;
 
 /* The layer's cache (device memory owned by the caller; sizes from

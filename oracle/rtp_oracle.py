@@ -26,6 +26,9 @@ arXiv 2605.16928):
   ordered by (P descending, index ascending) whose cumulative P reaches p
   (>= p); p >= 1 keeps everything.  Sinks and window are always added to the
   kept set (union after the top-p choice).
+* Static top-k (the pages' ablation baseline, atlas "Key results" and
+  "Baselines"): when the layer asks for a fixed k, the k highest scores (ties
+  to the lower index) replace the top-p set.
 * Attention itself is exact softmax attention with RoPE (rotate-half, angle
   pos * base^(-2k/D)) and scale 1/sqrt(D), over only the kept rows.
 
@@ -142,6 +145,16 @@ def top_p_set(scores, p: float) -> np.ndarray:
     return np.sort(order[:k]).astype(np.int64)
 
 
+def top_k_set(scores, k: int) -> np.ndarray:
+    """Static top-k, the pages' fixed-budget baseline (atlas.scime.ai summary,
+    "Baselines: static top-k"): the k highest scores, ties to the lower index;
+    every token when k >= n.  Returns the kept token indices, ascending."""
+    s = _as_f64(scores)
+    n = s.shape[0]
+    order = np.lexsort((np.arange(n), -s))  # score descending, then index ascending
+    return np.sort(order[:min(int(k), n)]).astype(np.int64)
+
+
 def sink_window_set(i: int, n_sink: int, window: int) -> np.ndarray:
     """Sinks [0, S) and the window of the last W positions ending at i, both within [0, i]."""
     sinks = np.arange(min(n_sink, i + 1), dtype=np.int64)
@@ -244,7 +257,8 @@ def _row(cache: OracleCache, b: int, hq: int, i: int, q_pre_row, w_q, p: float,
         r = sh.retrieval.index(h)
         q_idx = indexer_project(q_pre_row, w_q[r])
         s = indexer_scores(q_idx, cache.indexer_keys(b, r, i + 1))
-        topp = top_p_set(s, p)
+        k_fixed = int(getattr(sh, "top_k", 0) or 0)
+        topp = top_k_set(s, k_fixed) if k_fixed > 0 else top_p_set(s, p)
         rows = np.union1d(topp, sw)
     else:
         rows = sw
@@ -279,6 +293,30 @@ def decode(cache: OracleCache, q_pre, seq_len, w_q, top_p: Optional[float] = Non
             if t is not None:
                 topp[(b, hq)] = t
     return out, topp, final
+
+
+def recall_of_rows(cache: OracleCache, b: int, hq: int, i: int, q_pre_row, rows) -> float:
+    """Attention mass recall of an attended row set (atlas.scime.ai summary,
+    "Experimental setup", metrics): the share of the full causal attention's
+    softmax mass, over every position in [0, i], that `rows` carry."""
+    sh = cache.shape
+    h = hq // sh.group
+    q = rope(_as_f64(q_pre_row), i, sh.rope_base)
+    allr = np.arange(i + 1, dtype=np.int64)
+    z = (cache.keys(b, h, allr) @ q) / math.sqrt(q.shape[-1])
+    e = np.exp(z - z.max())
+    return float(e[np.asarray(rows, dtype=np.int64)].sum() / e.sum())
+
+
+def decode_recall(cache: OracleCache, q_pre, seq_len, final: Dict) -> Dict:
+    """Recall of each retrieval query head's attended rows of a decode step
+    (`final` as returned by decode: {(b, hq): rows})."""
+    sh = cache.shape
+    out = {}
+    for (b, hq), rows in final.items():
+        if hq // sh.group in sh.retrieval:
+            out[(b, hq)] = recall_of_rows(cache, b, hq, int(seq_len[b]) - 1, q_pre[b, hq], rows)
+    return out
 
 
 def prefill(cache: OracleCache, q_pre, start_pos, w_q, rows: Optional[Sequence[int]] = None,

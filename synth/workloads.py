@@ -36,6 +36,7 @@ class LayerShape:
     dtype: str = "bf16"          # storage / IO dtype: "bf16" or "fp32"
     rope_base: float = 10000.0
     idx_dim: int = IDX_DIM
+    top_k: int = 0               # > 0: static top-k selection instead of top-p
 
     @property
     def group(self) -> int:

@@ -81,8 +81,8 @@ def append_context(lay, inp, w_k, n_rows=None, dev="cuda"):
                    torch.zeros(sh.batch, dtype=torch.int32, device=dev), w_k)
         return
     c = lay.cfg
-    cfg1 = rtp.rtp_layer_cfg(1, c.n_q_heads, c.n_kv_heads, c.head_dim, c.idx_dim, c.max_ctx, c.n_sink,
-                             c.window, c.top_p, c.rope_base, c.retrieval_mask, c.dtype, c.local_cap)
+    cfg1 = rtp.rtp_layer_cfg.from_buffer_copy(c)
+    cfg1.batch = 1
     zero = torch.zeros(1, dtype=torch.int32, device=dev)
     for b in range(sh.batch):
         L = int(n_rows[b])

@@ -282,3 +282,43 @@ def test_bounded_wait_expiry_sets_timeout_and_returns():
     torch.cuda.synchronize()
     assert lay.device_status() == 0
     assert np.array_equal(out.double().cpu().numpy(), g["out"])
+
+
+@pytest.mark.parametrize("k", [1, 16, 300, 4999, 7000])
+def test_decode_static_topk(k):
+    """Static top-k (the pages' fixed-budget baseline): each retrieval q head
+    keeps exactly min(k, L) tokens, the highest scores, ties to the lower index
+    (k above the 16 needles of a head and above the context length included)."""
+    inp = _small(ctx=5000, needles=16, shape_top_k=k)
+    st = check_decode_parity(inp)
+    assert st["exact"] >= st["heads"] - 1
+    assert np.all(st["counts"] == min(k, 5000)), st["counts"]
+
+
+def test_decode_static_topk_tie_block():
+    """The k-th score sits inside a block of 300 identical keys: the lowest
+    indices of the block are kept, bit for bit."""
+    inp = _small(ctx=5000, needles=8, shape_top_k=150)
+    sh = inp["shape"]
+    h = sh.retrieval[0]
+    src = int(inp["needles"][0][0][0])
+    inp["k_pre"][0, 100:400, h] = inp["k_pre"][0, src, h]
+    g = run_gpu_decode(inp)
+    oc = oracle_cache_from_inputs(inp)
+    _, topk_o, _ = oracle.decode(oc, inp["q_pre"], inp["seq_len"], inp["w_q"], heads=[h * sh.group])
+    gset = bitmask_to_sets(g["bitmask"][0], [5000] * (sh.n_retrieval * sh.group))[0]
+    assert np.array_equal(gset, topk_o[(0, h * sh.group)]), (len(gset), len(topk_o[(0, h * sh.group)]))
+
+
+@pytest.mark.parametrize("k", [64, 4096])
+def test_decode_static_topk_128k(k):
+    inp = make_decode_inputs(workload("decode_128k_bf16", shape_top_k=k))
+    st = check_decode_parity(inp)
+    assert st["exact"] >= st["heads"] - 1
+    assert np.all(st["counts"] == k)
+
+
+def test_decode_static_topk_ragged():
+    inp = make_decode_inputs(workload("ragged_decode_b8_8k_32k_bf16", shape_top_k=1000))
+    st = check_decode_parity(inp)
+    assert np.all(st["counts"] == 1000)

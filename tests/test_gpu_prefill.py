@@ -135,3 +135,16 @@ def test_prefill_tied_block_keeps_lowest_indices():
                 assert np.array_equal(kept, np.arange(len(kept))), (t, gg, kept[:8])
     check_prefill_parity(inp, rows=list(range(600, 900, 37)), g=g)
     assert n_cut > 0
+
+
+def test_prefill_refuses_static_topk():
+    """Static top-k is a decode-only variant: the prefill entry point refuses it
+    on the host, before any device work."""
+    import head_wise_sparse_local_b200 as rtp
+    sh = workload("prefill_32k_bf16")["shape"].replace(top_k=100)
+    lay = rtp.Layer(sh, 1024, device="cuda")
+    q = torch.zeros((1, 64, sh.n_q_heads, sh.head_dim), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(rtp.RtpError) as e:
+        lay.prefill(q, torch.zeros(1, dtype=torch.int32, device="cuda"),
+                    torch.zeros((2, 16, sh.head_dim), device="cuda"), torch.empty_like(q))
+    assert e.value.code == 2 and "top-k" in str(e.value)

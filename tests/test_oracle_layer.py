@@ -279,3 +279,29 @@ def test_synth_is_deterministic_and_needles_outside_sink_window():
             assert np.all(pos >= sh.n_sink) and np.all(pos < L - sh.window)
     p = make_prefill_inputs(workload("prefill_32k_bf16", needles=4), T=64)
     assert p["q_pre"].shape == (1, 64, 32, 128)
+
+
+def test_recall_golden_three_keys():
+    d = json.load(open(os.path.join(GOLD, "recall_three_keys.json")))
+    D = d["head_dim"]
+    sh = LayerShape(batch=1, n_q_heads=1, n_kv_heads=1, head_dim=D, n_sink=0, window=1,
+                    top_p=0.5, retrieval=(0,), dtype="fp32")
+    k = torch.tensor(d["keys"], dtype=torch.float32)[None, :, None, :]
+    c = OracleCache(sh, 3)
+    c.append(k, torch.zeros_like(k), [0], 3, torch.zeros((1, 16, D)))
+    q = torch.tensor(d["q"], dtype=torch.float32)
+    for case in d["cases"]:
+        got = oracle.recall_of_rows(c, 0, 0, 2, q, case["rows"])
+        assert abs(got - case["recall"]) < 1e-6, (case, got)
+
+
+def test_recall_is_one_for_the_dense_reduction():
+    """p = 1 with a window covering the context attends every row: recall 1."""
+    L = 40
+    sh = _shape(batch=1, top_p=1.0, window=L, n_sink=2, retrieval=(0,), dtype="bf16")
+    q, k, v, wq, wk = _rand_layer(sh, L, 9)
+    c = OracleCache(sh, L)
+    c.append(k, v, [0], L, wk)
+    _, _, final = oracle.decode(c, q[:, L - 1], [L], wq)
+    rec = oracle.decode_recall(c, q[:, L - 1], [L], final)
+    assert rec and all(abs(x - 1.0) < 1e-12 for x in rec.values())
