@@ -24,7 +24,8 @@ _lib = _abi.load()
 
 __all__ = ["Layer", "RtpError", "rtp_layer_cfg", "rtp_cache", "rtp_cache_bytes",
            "rtp_decode_workspace_bytes", "rtp_prefill_workspace_bytes", "rtp_append_kv",
-           "rtp_decode_attn", "rtp_decode_attn_noalloc", "rtp_prefill_attn", "rtp_trace_stage",
+           "rtp_decode_attn", "rtp_decode_attn_noalloc", "rtp_decode_recall", "rtp_prefill_attn",
+           "rtp_trace_stage",
            "rtp_debug_wait_expiry",
            "rtp_last_error", "RTP_NOALLOC_SCRATCH_BYTES",
            "rtp_version", "make_cfg", "STAGES",
@@ -136,6 +137,13 @@ def rtp_decode_attn_noalloc(cfg, cache, q_pre, seq_len, max_seq_len, w_q, out, s
                                             _ptr(sel_bitmask), _ptr(sel_count), _stream(stream)))
 
 
+def rtp_decode_recall(cfg, cache, q_pre, seq_len, max_seq_len, sel_bitmask, recall, workspace=None,
+                      workspace_bytes=0, stream=None) -> None:
+    _abi.check(_lib.rtp_decode_recall(ctypes.byref(cfg), ctypes.byref(cache), _ptr(q_pre),
+                                      _ptr(seq_len), int(max_seq_len), _ptr(sel_bitmask), _ptr(recall),
+                                      _ptr(workspace), int(workspace_bytes), _stream(stream)))
+
+
 def rtp_prefill_attn(cfg, cache, q_pre, start_pos, T, w_q, out, sel_bitmask=None, sel_tau=None,
                      sel_jcut=None, sel_count=None, workspace=None, workspace_bytes=0,
                      stream=None) -> None:
@@ -170,9 +178,15 @@ class Layer:
         else:
             self.k = torch.empty((B, Hkv, max_ctx, D), dtype=dt, device=device)
         self.v = torch.empty_like(self.k)
-        self.kidx = torch.empty((B, max(R, 1), max_ctx, 16), dtype=dt, device=device)
+        # indexer keys [B, R, Lk, d] (Lk = max_ctx, or max_ctx rounded up to even
+        # for 8-byte bf16 d = 4 rows); kidx views the first max_ctx rows of each block
+        d = shape.idx_dim
+        _, _, ki_bytes = rtp_cache_bytes(self.cfg)
+        Lk = ki_bytes // (B * max(R, 1) * d * es) if R > 0 else max_ctx
+        self.kidx_full = torch.empty((B, max(R, 1), Lk, d), dtype=dt, device=device)
+        self.kidx = self.kidx_full[:, :, :max_ctx]
         self.status = torch.zeros(1, dtype=torch.int32, device=device)
-        self.cache = rtp_cache(self.k.data_ptr(), self.v.data_ptr(), self.kidx.data_ptr(),
+        self.cache = rtp_cache(self.k.data_ptr(), self.v.data_ptr(), self.kidx_full.data_ptr(),
                                self.status.data_ptr())
         self.ws_decode_bytes = rtp_decode_workspace_bytes(self.cfg)
         self.ws_decode = torch.empty(self.ws_decode_bytes, dtype=torch.uint8, device=device)
@@ -194,6 +208,10 @@ class Layer:
                sel_count=None, stream=None) -> None:
         rtp_decode_attn(self.cfg, self.cache, q_pre, seq_len, max_seq_len, w_q, out, sel_bitmask,
                         sel_count, self.ws_decode, self.ws_decode_bytes, stream)
+
+    def recall(self, q_pre, seq_len, sel_bitmask, recall, max_seq_len: int = 0, stream=None) -> None:
+        rtp_decode_recall(self.cfg, self.cache, q_pre, seq_len, max_seq_len, sel_bitmask, recall,
+                          self.ws_decode, self.ws_decode_bytes, stream)
 
     def prefill(self, q_pre, start_pos, w_q, out, sel_bitmask=None, sel_tau=None, sel_jcut=None,
                 sel_count=None, stream=None) -> None:

@@ -26,7 +26,8 @@ STATUS_NAMES = {0: "RTP_OK", 1: "RTP_ERR_INVALID", 2: "RTP_ERR_SHAPE", 3: "RTP_E
 
 # Every entry point declared in include/rtp.h.
 EXPORTS = ("rtp_cache_bytes", "rtp_decode_workspace_bytes", "rtp_prefill_workspace_bytes",
-           "rtp_append_kv", "rtp_decode_attn", "rtp_decode_attn_noalloc", "rtp_prefill_attn",
+           "rtp_append_kv", "rtp_decode_attn", "rtp_decode_attn_noalloc", "rtp_decode_recall",
+           "rtp_prefill_attn",
            "rtp_trace_stage", "rtp_debug_wait_expiry",
            "rtp_last_error", "rtp_version")
 
@@ -76,6 +77,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.rtp_trace_stage.argtypes = [i32, vp, vp]
     lib.rtp_debug_wait_expiry.argtypes = [i32]
     lib.rtp_decode_attn_noalloc.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, vp, vp]
+    lib.rtp_decode_recall.argtypes = [cfgp, cachep, vp, vp, i32, vp, vp, vp, sz, vp]
     for name in EXPORTS:
         getattr(lib, name).restype = ctypes.c_char_p if name in ("rtp_last_error", "rtp_version") \
             else ctypes.c_int

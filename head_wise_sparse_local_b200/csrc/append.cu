@@ -1,11 +1,11 @@
-// rtp_append_kv: RoPE'd key, value and 16-d pre-RoPE indexer key per token.
+// rtp_append_kv: RoPE'd key, value and d-dim pre-RoPE indexer key per token.
 //
 // One warp per (sequence, token, KV head) row.  Lane l owns the RoPE pairs
 // (k, k + D/2) for k in [l*PP, (l+1)*PP), PP = D/64, so the rotation needs no
 // shuffle.  Retrieval heads also project the pre-RoPE key through W_k^(r)
 // ("pre-RoPE low-dimensional projection", atlas.scime.ai summary, "Approach"):
 // each lane forms partial dot products over its dims and a butterfly reduction
-// gives every lane the same 16 sums.
+// gives every lane the same d sums (d = 4, 8, 16 or 32).
 #include "common.cuh"
 #include "internal.h"
 
@@ -13,7 +13,7 @@ namespace rtp {
 namespace {
 
 struct AppendArgs {
-  int B, T, Hkv, D, Lmax, R;
+  int B, T, Hkv, D, Lmax, Lk, R;
   float rope_base;
   const void* k_pre;
   const void* v_in;
@@ -28,7 +28,7 @@ struct AppendArgs {
   double inv_freq[64];
 };
 
-template <typename T, int D>
+template <typename T, int D, int IDX>
 __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ AppendArgs a) {
   // The inputs (k_pre, v, start_pos, W_k) are read and the rotated key and the
   // indexer key formed before waiting for the previous kernel on the stream;
@@ -76,11 +76,11 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     y2[i] = from_f32<T>(x2[i] * c + x1[i] * s);
   }
   const int r = a.ret_rank[h];
-  float acc[kIdxDim];
+  float acc[IDX];
   if (r >= 0) {  // warp-uniform
-    const float* w = a.w_k + (size_t)r * kIdxDim * D;
+    const float* w = a.w_k + (size_t)r * IDX * D;
 #pragma unroll
-    for (int i = 0; i < kIdxDim; ++i) {
+    for (int i = 0; i < IDX; ++i) {
       float sacc = 0.f;
 #pragma unroll
       for (int p = 0; p < PP; ++p) {
@@ -93,7 +93,7 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
 #pragma unroll
-      for (int i = 0; i < kIdxDim; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
+      for (int i = 0; i < IDX; ++i) acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], o);
     }
   }
   griddep_wait();
@@ -109,10 +109,20 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
     vo[k + H] = v2[i];
   }
   if (r >= 0) {
-    T* ki = static_cast<T*>(a.kidx) + (((size_t)b * a.R + r) * a.Lmax + pos) * kIdxDim;
+    T* ki = static_cast<T*>(a.kidx) + (((size_t)b * a.R + r) * a.Lk + pos) * IDX;
 #pragma unroll
-    for (int i = 0; i < kIdxDim; ++i)
+    for (int i = 0; i < IDX; ++i)
       if (lane == i) ki[i] = from_f32<T>(acc[i]);
+  }
+}
+
+template <typename T, int D>
+cudaError_t launch_append_idx(int idx, unsigned grid, cudaStream_t st, const AppendArgs& a) {
+  switch (idx) {
+    case 4: return launch_pdl(append_kernel<T, D, 4>, dim3(grid), dim3(256), 0, st, a);
+    case 8: return launch_pdl(append_kernel<T, D, 8>, dim3(grid), dim3(256), 0, st, a);
+    case 32: return launch_pdl(append_kernel<T, D, 32>, dim3(grid), dim3(256), 0, st, a);
+    default: return launch_pdl(append_kernel<T, D, 16>, dim3(grid), dim3(256), 0, st, a);
   }
 }
 
@@ -121,7 +131,7 @@ __global__ void __launch_bounds__(256) append_kernel(const __grid_constant__ App
 int launch_append(const Shape& sh, const rtp_cache* cache, const void* k_pre, const void* v_in,
                   const int* start_pos, int T, const float* w_k, cudaStream_t st) {
   AppendArgs a;
-  a.B = sh.B; a.T = T; a.Hkv = sh.Hkv; a.D = sh.D; a.Lmax = sh.Lmax; a.R = sh.R;
+  a.B = sh.B; a.T = T; a.Hkv = sh.Hkv; a.D = sh.D; a.Lmax = sh.Lmax; a.Lk = sh.Lk; a.R = sh.R;
   a.rope_base = sh.rope_base;
   a.k_pre = k_pre; a.v_in = v_in; a.start_pos = start_pos; a.w_k = w_k;
   a.k = cache->k; a.v = cache->v; a.kidx = cache->kidx; a.status = cache->status;
@@ -134,11 +144,11 @@ int launch_append(const Shape& sh, const rtp_cache* cache, const void* k_pre, co
   trace_begin(RTP_STAGE_APPEND, st);
   cudaError_t e;
   if (sh.dtype == RTP_BF16) {
-    if (sh.D == 128) e = launch_pdl(append_kernel<__nv_bfloat16, 128>, dim3(grid), dim3(256), 0, st, a);
-    else e = launch_pdl(append_kernel<__nv_bfloat16, 64>, dim3(grid), dim3(256), 0, st, a);
+    if (sh.D == 128) e = launch_append_idx<__nv_bfloat16, 128>(sh.idx, grid, st, a);
+    else e = launch_append_idx<__nv_bfloat16, 64>(sh.idx, grid, st, a);
   } else {
-    if (sh.D == 128) e = launch_pdl(append_kernel<float, 128>, dim3(grid), dim3(256), 0, st, a);
-    else e = launch_pdl(append_kernel<float, 64>, dim3(grid), dim3(256), 0, st, a);
+    if (sh.D == 128) e = launch_append_idx<float, 128>(sh.idx, grid, st, a);
+    else e = launch_append_idx<float, 64>(sh.idx, grid, st, a);
   }
   trace_end(RTP_STAGE_APPEND, st);
   if (e == cudaSuccess) e = cudaGetLastError();

@@ -11,7 +11,15 @@
 namespace rtp {
 
 constexpr int kIdxDim = 16;        // indexer width (abstract, observation (2))
-constexpr float kIdxScale = 0.25f; // 1/sqrt(16)
+// Score scale 1/sqrt(d) for the indexer widths the layer takes: d = 16 and the
+// pages' ablation widths 4, 8, 32 (atlas.scime.ai summary, "Surprising
+// findings"); exact for 4 and 16, rounded to fp32 for 8 and 32.
+template <int IDX>
+__host__ __device__ constexpr float idx_scale() {
+  static_assert(IDX == 4 || IDX == 8 || IDX == 16 || IDX == 32, "indexer width");
+  return IDX == 4 ? 0.5f : IDX == 8 ? 0.35355339059327376f : IDX == 16 ? 0.25f : 0.17677669529663688f;
+}
+constexpr float kIdxScale = idx_scale<16>();
 constexpr int kMaxRetrieval = 64;
 
 // ---------------------------------------------------------------------------
@@ -236,6 +244,7 @@ __device__ __forceinline__ void ldsm_x2_t(unsigned& r0, unsigned& r1, const void
   const unsigned a = (unsigned)__cvta_generic_to_shared(p);
   asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];\n" : "=r"(r0), "=r"(r1) : "r"(a));
 }
+
 __device__ __forceinline__ void mma_bf16(float (&c)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3,
                                          unsigned b0, unsigned b1) {
   asm volatile(
@@ -248,6 +257,69 @@ __device__ __forceinline__ unsigned pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const unsigned*>(&v);
 }
+
+// Indexer scores on tensor cores (decode and prefill share these, so a prefill
+// row and the decode step at its position compute bit-identical scores).
+// S = K~ Q~^T by m16n8k16 products: the M side is 16 keys, the K side the
+// indexer dims in steps of 16 (dims past d read as zero), the N side 8 query
+// columns; q~ enters as a bf16 high part and a bf16 low part, all high steps
+// accumulated before the low ones into one fp32 accumulator.
+template <int IDX>
+struct IdxMma {
+  static constexpr int KS = (IDX + 15) / 16;  // k-steps of 16 dims
+  static constexpr int KB = IDX * 2;          // bytes per bf16 key
+  unsigned bh[KS][2], bl[KS][2];
+
+  // B fragments from the fp32 q~ of this lane's column (lane / 4), `q`
+  // pointing at its IDX values, or nullptr for a column with no query.
+  __device__ __forceinline__ void set_q(const float* q, int lane) {
+    const int t4 = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      float hi[4], lo[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int d = ks * 16 + 2 * t4 + (e & 1) + (e >> 1) * 8;
+        const float v = (q != nullptr && d < IDX) ? q[d] : 0.f;
+        hi[e] = __bfloat162float(__float2bfloat16_rn(v));
+        lo[e] = v - hi[e];
+      }
+      bh[ks][0] = pack_bf16(hi[0], hi[1]);
+      bh[ks][1] = pack_bf16(hi[2], hi[3]);
+      bl[ks][0] = pack_bf16(lo[0], lo[1]);
+      bl[ks][1] = pack_bf16(lo[2], lo[3]);
+    }
+  }
+
+  // Accumulators c[4] of the 16 keys starting at `tile` (shared memory, KB
+  // bytes per key, 16-byte aligned): c[0], c[1] key lane/4, columns 2 (lane%4)
+  // and 2 (lane%4) + 1; c[2], c[3] key lane/4 + 8.
+  __device__ __forceinline__ void scores(const unsigned char* tile, int lane, float (&c)[4]) const {
+    unsigned a[KS][4];
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      if constexpr (IDX >= 16) {
+        ldsm_x4(a[ks][0], a[ks][1], a[ks][2], a[ks][3],
+                tile + (size_t)((lane & 7) + ((lane >> 3) & 1) * 8) * KB + ks * 32 + (lane >> 4) * 16);
+      } else if constexpr (IDX == 8) {
+        ldsm_x2(a[ks][0], a[ks][1], tile + (size_t)((lane & 7) + ((lane >> 3) & 1) * 8) * KB);
+        a[ks][2] = 0u;
+        a[ks][3] = 0u;
+      } else {  // 8-byte keys: dims 2 t4, 2 t4 + 1 for t4 < 2, by plain 4-byte loads
+        const int gq = lane >> 2, t4 = lane & 3;
+        a[ks][0] = t4 < 2 ? *reinterpret_cast<const unsigned*>(tile + gq * KB + t4 * 4) : 0u;
+        a[ks][1] = t4 < 2 ? *reinterpret_cast<const unsigned*>(tile + (gq + 8) * KB + t4 * 4) : 0u;
+        a[ks][2] = 0u;
+        a[ks][3] = 0u;
+      }
+    }
+    c[0] = c[1] = c[2] = c[3] = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) mma_bf16(c, a[ks][0], a[ks][1], a[ks][2], a[ks][3], bh[ks][0], bh[ks][1]);
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) mma_bf16(c, a[ks][0], a[ks][1], a[ks][2], a[ks][3], bl[ks][0], bl[ks][1]);
+  }
+};
 
 __device__ __forceinline__ void ldsm_x4_t(unsigned& r0, unsigned& r1, unsigned& r2, unsigned& r3, const void* p) {
   const unsigned a = (unsigned)__cvta_generic_to_shared(p);

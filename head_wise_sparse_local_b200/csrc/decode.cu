@@ -73,14 +73,15 @@ constexpr int kTopPerWarp = 16;     // top-rung items a warp hands the leader in
 static_assert(kTopPerWarp <= 32, "the tail gives each top-rung item of a warp its own lane");
 constexpr int kSpec = 2;            // of those, rows whose keys and values a warp stages early
 
-// Tokens per score chunk (32 KB of indexer keys): four (bf16) or two (fp32)
-// 16-d keys per thread.
+// Tokens per score chunk: four (bf16) or two (fp32) keys per thread, 2 KB of
+// indexer keys per indexer dim (32 KB at d = 16).
 __host__ __device__ constexpr int score_chunk(int esize) { return kThreads * (esize == 2 ? 4 : 2); }
-constexpr int kScoreSmem = 2 * 32 * 1024;  // two chunk buffers
-constexpr int kScoreCtasPerSm = 3;
+__host__ __device__ constexpr int score_smem(int idx) { return 2 * 2048 * idx; }  // two chunk buffers
+__host__ __device__ constexpr int score_ctas_per_sm(int idx) { return idx == 32 ? 1 : 3; }
 
 struct DecodeArgs {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W, max_seq_len, words;
+  int Lk;           // indexer-key rows per (sequence, retrieval head) block
   int lstride;      // row stride of the score scratch (Lmax rounded up to 32)
   float top_p, rope_base;
   int top_k;        // > 0: static top-k instead of top-p
@@ -165,21 +166,21 @@ __device__ void rope_query(const DecodeArgs& a, int b, int h, int pos, float* s_
 // ---------------------------------------------------------------------------
 // 1a. score CTAs: indexer scores + per-chunk maxima of the retrieval KV heads
 // ---------------------------------------------------------------------------
-// A persistent grid (at most kScoreCtasPerSm per SM) walks the chunks
+// A persistent grid (at most score_ctas_per_sm per SM) walks the chunks
 // (sequence, retrieval KV head, chunk of kChunk tokens) in order, a CTA taking
 // every gridDim.x-th.  A chunk's indexer keys (contiguous rows of the key
 // cache) arrive in shared memory with one bulk asynchronous copy, two chunks in
 // flight per CTA; the scores are formed there.
-template <typename T, int D, int G>
+template <typename T, int D, int G, int IDX>
 __device__ __forceinline__ void score_q(const DecodeArgs& a, int b, int r, float* s_q) {
   // q~ = W_q q_pre: four threads per output, a quarter of the dims each
   const int tid = threadIdx.x;
   const int h = a.ret_head[r];
-  for (int o4 = tid; o4 < G * kIdxDim * 4; o4 += kThreads) {
+  for (int o4 = tid; o4 < G * IDX * 4; o4 += kThreads) {
     const int o = o4 >> 2, qd = o4 & 3;
-    const int g = o / kIdxDim, i = o % kIdxDim;
+    const int g = o / IDX, i = o % IDX;
     constexpr int DQ = D / 4;
-    const float4* w = reinterpret_cast<const float4*>(a.w_q + ((size_t)r * kIdxDim + i) * D + qd * DQ);
+    const float4* w = reinterpret_cast<const float4*>(a.w_q + ((size_t)r * IDX + i) * D + qd * DQ);
     const T* q = static_cast<const T*>(a.q_pre) + ((size_t)b * a.Hq + h * G + g) * D + qd * DQ;
     float wv[DQ], qv[DQ];
 #pragma unroll
@@ -193,18 +194,19 @@ __device__ __forceinline__ void score_q(const DecodeArgs& a, int b, int r, float
     for (int k = 0; k < DQ; ++k) acc = fmaf(wv[k], qv[k], acc);
     acc += __shfl_xor_sync(0xffffffffu, acc, 1);
     acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-    if (qd == 0) s_q[g * kIdxDim + i] = acc;
+    if (qd == 0) s_q[g * IDX + i] = acc;
   }
 }
 
-template <typename T, int D, int G>
+template <typename T, int D, int G, int IDX>
 __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* dsm, uint64_t* bar) {
   constexpr int kChunk = score_chunk(sizeof(T));
   constexpr int TPT = kChunk / kThreads;        // keys per thread
-  constexpr int NV = kIdxDim * sizeof(T) / 16;  // 16-byte vectors per key
-  constexpr int KB = kIdxDim * sizeof(T);       // bytes per key
+  constexpr int KB = IDX * sizeof(T);           // bytes per key
   constexpr int kBuf = kChunk * KB;             // bytes of one chunk buffer
-  __shared__ __align__(16) float s_q[G * kIdxDim];
+  static_assert(2 * kBuf == score_smem(IDX), "chunk buffers");
+  constexpr float kScale = idx_scale<IDX>();
+  __shared__ __align__(16) float s_q[G * IDX];
   __shared__ float s_ml[kWarps * G];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nch = a.n_score_ctas / (a.B * a.R);  // chunks per (sequence, retrieval head)
@@ -220,7 +222,7 @@ __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* d
     mbar_init(bar + 1, 1);
   }
   int cur_br = blockIdx.x / nch;
-  score_q<T, D, G>(a, cur_br / a.R, cur_br % a.R, s_q);  // the caller's inputs: before the wait
+  score_q<T, D, G, IDX>(a, cur_br / a.R, cur_br % a.R, s_q);  // the caller's inputs: before the wait
   __syncthreads();  // barriers initialised, q~ visible
   griddep_wait();   // rtp_append_kv (and with it the previous decode step) has completed
   griddep_launch();
@@ -231,8 +233,10 @@ __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* d
     const int br = c / nch, chunk = c % nch;
     const int j0 = chunk * kChunk, jh = min(a.max_seq_len, j0 + kChunk);
     const unsigned char* src = static_cast<const unsigned char*>(a.kidx) +
-                               ((size_t)br * a.Lmax + j0) * KB;
-    const uint32_t bytes = (uint32_t)(jh - j0) * KB;
+                               ((size_t)br * a.Lk + j0) * KB;
+    // whole 16-byte units: an odd count of 8-byte keys takes the next key of
+    // the block too (Lk is even then, and jh < Lk), never past the block
+    const uint32_t bytes = ((uint32_t)(jh - j0) * KB + 15u) & ~15u;
     mbar_expect_tx(bar + (k & 1), bytes + a.tx_extra);
     bulk_g2s(dsm + (size_t)(k & 1) * kBuf, src, bytes, bar + (k & 1), pol);
   };
@@ -247,7 +251,7 @@ __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* d
     const int L = a.seq_len[b];
     if (br != cur_br) {  // another (sequence, retrieval head): its q~ (uniform over the CTA)
       __syncthreads();
-      score_q<T, D, G>(a, b, r, s_q);
+      score_q<T, D, G, IDX>(a, b, r, s_q);
       cur_br = br;
     }
     const bool arrived = mbar_wait_bounded(bar + (k & 1), (uint32_t)(k >> 1) & 1u, a.wait_ns, a.status);
@@ -273,22 +277,8 @@ __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* d
         // accumulator.  A prefill row and the decode step at its position then
         // see bit-identical scores.
         const int t4 = lane & 3, gq = lane >> 2;
-        unsigned bh0 = 0u, bh1 = 0u, bl0 = 0u, bl1 = 0u;
-        if (gq < G) {
-          const int k0 = t4 * 2;
-          const float v[4] = {s_q[gq * kIdxDim + k0], s_q[gq * kIdxDim + k0 + 1], s_q[gq * kIdxDim + k0 + 8],
-                              s_q[gq * kIdxDim + k0 + 9]};
-          float hi[4], lo[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            hi[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
-            lo[e] = v[e] - hi[e];
-          }
-          bh0 = pack_bf16(hi[0], hi[1]);
-          bh1 = pack_bf16(hi[2], hi[3]);
-          bl0 = pack_bf16(lo[0], lo[1]);
-          bl1 = pack_bf16(lo[2], lo[3]);
-        }
+        IdxMma<IDX> mm;
+        mm.set_q(gq < G ? s_q + gq * IDX : nullptr, lane);
         // this lane's columns 2 t4, 2 t4 + 1 (query heads when < G)
         float mxa = -CUDART_INF_F, mxb = -CUDART_INF_F;
         const bool ca = 2 * t4 < G, cb = 2 * t4 + 1 < G;
@@ -296,17 +286,14 @@ __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* d
         for (int tt = warp; tt < kTiles; tt += kWarps) {
           const int kb = tt * 16;  // first key of the tile (chunk-local)
           if (j0 + kb >= j1) break;  // warp-uniform
-          unsigned a0, a1, a2, a3;
-          ldsm_x4(a0, a1, a2, a3, kbuf + (size_t)(kb + (lane & 7) + ((lane >> 3) & 1) * 8) * KB + (lane >> 4) * 16);
-          float cc[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_bf16(cc, a0, a1, a2, a3, bh0, bh1);
-          mma_bf16(cc, a0, a1, a2, a3, bl0, bl1);
+          float cc[4];
+          mm.scores(kbuf + (size_t)kb * KB, lane, cc);
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             const int j = j0 + kb + gq + 8 * x;
             if (j >= j1) continue;
-            const float sa = cc[2 * x] * kIdxScale + 0.0f;  // +0 turns -0 into +0
-            const float sb = cc[2 * x + 1] * kIdxScale + 0.0f;
+            const float sa = cc[2 * x] * kScale + 0.0f;  // +0 turns -0 into +0
+            const float sb = cc[2 * x + 1] * kScale + 0.0f;
             if (ca) {
               lg[(size_t)(2 * t4) * a.lstride + j] = sa;
               mxa = fmaxf(mxa, sa);
@@ -335,10 +322,11 @@ __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* d
           const int jl = t * kThreads + tid;
           const int j = j0 + jl;
           if (j >= j1) continue;
+          constexpr int NV = KB / 16;  // 16-byte vectors per fp32 key
           uint4 kr[NV];
 #pragma unroll
           for (int v = 0; v < NV; ++v) kr[v] = reinterpret_cast<const uint4*>(kbuf + (size_t)jl * KB)[v];
-          float kv[kIdxDim];
+          float kv[IDX];
 #pragma unroll
           for (int v = 0; v < NV; ++v) {
             kv[v * 4 + 0] = __uint_as_float(kr[v].x); kv[v * 4 + 1] = __uint_as_float(kr[v].y);
@@ -346,17 +334,17 @@ __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* d
           }
 #pragma unroll
           for (int g = 0; g < G; ++g) {
-            const float4* q4 = reinterpret_cast<const float4*>(s_q + g * kIdxDim);
+            const float4* q4 = reinterpret_cast<const float4*>(s_q + g * IDX);
             float sco = 0.f;
 #pragma unroll
-            for (int i4 = 0; i4 < kIdxDim / 4; ++i4) {
+            for (int i4 = 0; i4 < IDX / 4; ++i4) {
               const float4 qq = q4[i4];
               sco = fmaf(qq.x, kv[4 * i4], sco);
               sco = fmaf(qq.y, kv[4 * i4 + 1], sco);
               sco = fmaf(qq.z, kv[4 * i4 + 2], sco);
               sco = fmaf(qq.w, kv[4 * i4 + 3], sco);
             }
-            sco = sco * kIdxScale + 0.0f;  // exact scaling; +0 turns -0 into +0
+            sco = sco * kScale + 0.0f;  // +0 turns -0 into +0
             lg[(size_t)g * a.lstride + j] = sco;
             mx[g] = fmaxf(mx[g], sco);
           }
@@ -831,11 +819,11 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
 // score CTA has passed its wait, so the appended rows are complete.  Its
 // closing wait makes its completion imply the score kernel's, which is what
 // the select kernel's wait relies on.
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(kThreads, kScoreCtasPerSm) score_kernel(const __grid_constant__ DecodeArgs a) {
+template <typename T, int D, int G, int IDX>
+__global__ void __launch_bounds__(kThreads, score_ctas_per_sm(IDX)) score_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char dsm[];
   __shared__ __align__(8) uint64_t s_bar[2];
-  score_ctas<T, D, G>(a, dsm, s_bar);
+  score_ctas<T, D, G, IDX>(a, dsm, s_bar);
 }
 
 template <typename T, int D, int G>
@@ -1974,8 +1962,14 @@ cudaError_t launch_cluster_pdl(void (*k)(DecodeArgs), dim3 grid, dim3 block, siz
 // The two stream kernels: score CTAs (plain grid), then sink/window clusters of
 // 16 CTAs when the device can place one (non-portable size), else 8.  Set up
 // once per device under a mutex.
+template <typename T, int D, int G, int IDX>
+cudaError_t launch_score(const DecodeArgs& a, int n_sms, cudaStream_t st) {
+  return launch_pdl(score_kernel<T, D, G, IDX>, dim3(std::min(a.n_score_ctas, score_ctas_per_sm(IDX) * n_sms)),
+                    dim3(kThreads), score_smem(IDX), st, a);
+}
+
 template <typename T, int D, int G>
-cudaError_t launch_stream(DecodeArgs& a, int n_bkv, cudaStream_t st) {
+cudaError_t launch_stream(DecodeArgs& a, int n_bkv, int idx, cudaStream_t st) {
   static std::mutex s_mu;
   static std::atomic<int> s_cs[64];  // chosen cluster size; 0 = not set up yet
   static std::atomic<int> s_sms[64];
@@ -1988,7 +1982,10 @@ cudaError_t launch_stream(DecodeArgs& a, int n_bkv, cudaStream_t st) {
     std::lock_guard<std::mutex> lock(s_mu);
     cs = s_cs[dev].load(std::memory_order_relaxed);
     if (cs == 0) {
-      cudaFuncSetAttribute(score_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kScoreSmem);
+      cudaFuncSetAttribute(score_kernel<T, D, G, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, score_smem(4));
+      cudaFuncSetAttribute(score_kernel<T, D, G, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, score_smem(8));
+      cudaFuncSetAttribute(score_kernel<T, D, G, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, score_smem(16));
+      cudaFuncSetAttribute(score_kernel<T, D, G, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, score_smem(32));
       cudaFuncSetAttribute(sw_kernel<T, D, G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       cudaFuncSetAttribute(sw_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
       cudaLaunchConfig_t cfg = {};
@@ -2016,8 +2013,12 @@ cudaError_t launch_stream(DecodeArgs& a, int n_bkv, cudaStream_t st) {
   const int n_sms = s_sms[dev].load(std::memory_order_relaxed);
   if (a.n_score_ctas > 0) {
     trace_begin(RTP_STAGE_DECODE_SCORE, st);
-    e = launch_pdl(score_kernel<T, D, G>, dim3(std::min(a.n_score_ctas, kScoreCtasPerSm * n_sms)), dim3(kThreads),
-                   kScoreSmem, st, a);
+    switch (idx) {
+      case 4: e = launch_score<T, D, G, 4>(a, n_sms, st); break;
+      case 8: e = launch_score<T, D, G, 8>(a, n_sms, st); break;
+      case 32: e = launch_score<T, D, G, 32>(a, n_sms, st); break;
+      default: e = launch_score<T, D, G, 16>(a, n_sms, st); break;
+    }
     trace_end(RTP_STAGE_DECODE_SCORE, st);
     if (e != cudaSuccess) return e;
   }
@@ -2028,21 +2029,22 @@ cudaError_t launch_stream(DecodeArgs& a, int n_bkv, cudaStream_t st) {
 }
 
 template <typename T, int D>
-cudaError_t launch_stream_d(DecodeArgs& a, int n_bkv, cudaStream_t st) {
+cudaError_t launch_stream_d(DecodeArgs& a, int n_bkv, int idx, cudaStream_t st) {
   switch (a.G) {
-    case 1: return launch_stream<T, D, 1>(a, n_bkv, st);
-    case 2: return launch_stream<T, D, 2>(a, n_bkv, st);
-    case 4: return launch_stream<T, D, 4>(a, n_bkv, st);
-    default: return launch_stream<T, D, 8>(a, n_bkv, st);
+    case 1: return launch_stream<T, D, 1>(a, n_bkv, idx, st);
+    case 2: return launch_stream<T, D, 2>(a, n_bkv, idx, st);
+    case 4: return launch_stream<T, D, 4>(a, n_bkv, idx, st);
+    default: return launch_stream<T, D, 8>(a, n_bkv, idx, st);
   }
 }
 
 cudaError_t launch_stream_any(const Shape& sh, DecodeArgs& a, cudaStream_t st) {
   const int n_bkv = sh.B * sh.Hkv;
   if (sh.dtype == RTP_BF16)
-    return sh.D == 128 ? launch_stream_d<__nv_bfloat16, 128>(a, n_bkv, st)
-                       : launch_stream_d<__nv_bfloat16, 64>(a, n_bkv, st);
-  return sh.D == 128 ? launch_stream_d<float, 128>(a, n_bkv, st) : launch_stream_d<float, 64>(a, n_bkv, st);
+    return sh.D == 128 ? launch_stream_d<__nv_bfloat16, 128>(a, n_bkv, sh.idx, st)
+                       : launch_stream_d<__nv_bfloat16, 64>(a, n_bkv, sh.idx, st);
+  return sh.D == 128 ? launch_stream_d<float, 128>(a, n_bkv, sh.idx, st)
+                     : launch_stream_d<float, 64>(a, n_bkv, sh.idx, st);
 }
 
 // Select kernel with 16-CTA clusters when the device can keep all of this
@@ -2131,7 +2133,7 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
                   int* sel_count, void* ws, const DecodeLayout& lay, cudaStream_t st) {
   DecodeArgs a;
   a.B = sh.B; a.Hq = sh.Hq; a.Hkv = sh.Hkv; a.G = sh.G; a.D = sh.D; a.R = sh.R; a.NR = sh.NR;
-  a.Lmax = sh.Lmax; a.S = sh.S; a.W = sh.W;
+  a.Lmax = sh.Lmax; a.S = sh.S; a.W = sh.W; a.Lk = sh.Lk;
   a.max_seq_len = max_seq_len > 0 ? max_seq_len : sh.Lmax;
   a.words = (sh.Lmax + 31) / 32;
   a.lstride = (sh.Lmax + 31) & ~31;

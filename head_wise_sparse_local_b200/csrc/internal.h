@@ -42,6 +42,8 @@ struct Shape {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W;
   int ring;          // window rows a local head keeps in ring mode (0: whole context)
   int top_k;         // > 0: retrieval heads keep a fixed k tokens (static top-k) instead of top-p
+  int idx;           // indexer width d (4, 8, 16 or 32)
+  int Lk;            // indexer-key rows per (sequence, retrieval head) block of the kidx cache
   KvMap kv;
   float top_p, rope_base;
   int dtype;  // rtp_dtype
@@ -72,6 +74,10 @@ int launch_append(const Shape& sh, const rtp_cache* cache, const void* k_pre, co
 int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* seq_len,
                   int max_seq_len, const float* w_q, void* out, uint32_t* sel_bitmask,
                   int* sel_count, void* ws, const DecodeLayout& lay, cudaStream_t st);
+
+size_t recall_workspace_bytes(const Shape& sh);
+int launch_recall(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* seq_len,
+                  int max_seq_len, const uint32_t* sel_bitmask, float* recall, void* ws, cudaStream_t st);
 
 struct PrefillLayout {
   size_t total;

@@ -53,7 +53,8 @@ int make_shape(const rtp_layer_cfg* cfg, Shape* sh) {
     return fail(RTP_ERR_SHAPE, "group size n_q_heads/n_kv_heads must be 1, 2, 4 or 8");
   if (cfg->head_dim != 64 && cfg->head_dim != 128)
     return fail(RTP_ERR_SHAPE, "head_dim must be 64 or 128");
-  if (cfg->idx_dim != 16) return fail(RTP_ERR_SHAPE, "idx_dim must be 16");
+  if (cfg->idx_dim != 4 && cfg->idx_dim != 8 && cfg->idx_dim != 16 && cfg->idx_dim != 32)
+    return fail(RTP_ERR_SHAPE, "idx_dim must be 4, 8, 16 or 32");
   if (cfg->max_ctx < 1 || cfg->max_ctx > (1 << 23))
     return fail(RTP_ERR_SHAPE, "max_ctx must be in [1, 2^23]");
   if (cfg->n_sink < 0) return fail(RTP_ERR_INVALID, "n_sink must be >= 0");
@@ -75,6 +76,10 @@ int make_shape(const rtp_layer_cfg* cfg, Shape* sh) {
   sh->rope_base = cfg->rope_base;
   sh->dtype = cfg->dtype;
   sh->esize = cfg->dtype == RTP_BF16 ? 2 : 4;
+  sh->idx = cfg->idx_dim;
+  // an indexer-key block of (sequence, retrieval head) starts on a 16-byte
+  // boundary: 8-byte rows (bf16, d = 4) take an even number of rows
+  sh->Lk = sh->idx * sh->esize < 16 ? (sh->Lmax + 1) & ~1 : sh->Lmax;
   int r = 0;
   for (int h = 0; h < 64; ++h) {
     sh->ret_rank[h] = -1;
@@ -159,7 +164,7 @@ int rtp_cache_bytes(const rtp_layer_cfg* cfg, size_t* k_bytes, size_t* v_bytes,
   const size_t kv = (size_t)sh.B * (size_t)sh.kv.rows_per_seq * sh.D * sh.esize;
   if (k_bytes) *k_bytes = kv;
   if (v_bytes) *v_bytes = kv;
-  if (kidx_bytes) *kidx_bytes = (size_t)sh.B * sh.R * sh.Lmax * 16 * sh.esize;
+  if (kidx_bytes) *kidx_bytes = (size_t)sh.B * sh.R * sh.Lk * sh.idx * sh.esize;
   return RTP_OK;
 }
 
@@ -220,6 +225,27 @@ int rtp_decode_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void
                        workspace, lay, (cudaStream_t)stream);
 }
 
+int rtp_decode_recall(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
+                      const int* seq_len, int max_seq_len, const uint32_t* sel_bitmask,
+                      float* recall, void* workspace, size_t workspace_bytes, void* stream) {
+  Shape sh;
+  int rc = make_shape(cfg, &sh);
+  if (rc != RTP_OK) return rc;
+  if ((rc = check_cache(sh, cache)) != RTP_OK) return rc;
+  if (max_seq_len < 0 || max_seq_len > sh.Lmax)
+    return fail(RTP_ERR_SHAPE, "max_seq_len must be in [0, max_ctx]");
+  if (sh.R == 0) return RTP_OK;
+  if (!q_pre || !seq_len || !sel_bitmask || !recall)
+    return fail(RTP_ERR_INVALID, "q_pre/seq_len/sel_bitmask/recall is NULL");
+  if (!workspace) return fail(RTP_ERR_WORKSPACE, "workspace is NULL");
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(RTP_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (workspace_bytes < recall_workspace_bytes(sh))
+    return fail(RTP_ERR_WORKSPACE, "workspace too small for rtp_decode_recall");
+  return launch_recall(sh, cache, q_pre, seq_len, max_seq_len, sel_bitmask, recall, workspace,
+                       (cudaStream_t)stream);
+}
+
 int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
                      const int* start_pos, int T, const float* w_q, void* out,
                      uint32_t* sel_bitmask, float* sel_tau, int* sel_jcut, int* sel_count,
@@ -231,6 +257,7 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
   if (T < 1 || T > sh.Lmax) return fail(RTP_ERR_SHAPE, "T must be in [1, max_ctx]");
   if (sh.top_k > 0)
     return fail(RTP_ERR_SHAPE, "static top-k (cfg top_k > 0) is a decode-only variant; prefill selects by top-p");
+  if (sh.idx != 16) return fail(RTP_ERR_SHAPE, "prefill takes idx_dim 16 only");
   if (sh.ring > 0 && (long long)T + sh.W - 1 > sh.ring)
     return fail(RTP_ERR_SHAPE, "ring mode: a prefill chunk needs local_cap >= T + window - 1");
   if (!q_pre || !start_pos || !out) return fail(RTP_ERR_INVALID, "q_pre/start_pos/out is NULL");

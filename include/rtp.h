@@ -63,7 +63,11 @@ typedef enum rtp_dtype { RTP_BF16 = 0, RTP_FP32 = 1 } rtp_dtype;
  *   n_q_heads     Hq;  n_kv_heads Hkv;  G = Hq / Hkv query heads share a KV head
  *                 (GQA; q head hq reads KV head hq / G).  Supported G: 1, 2, 4, 8.
  *   head_dim      D: 64 or 128
- *   idx_dim       indexer width; must be 16 (abstract, observation (2))
+ *   idx_dim       d, the indexer width: 16 (abstract, observation (2)), or 4, 8
+ *                 or 32 for the pages' indexer-dimension ablation
+ *                 (atlas.scime.ai summary, "Surprising findings": dimension 4).
+ *                 Scores are q~ . k~ / sqrt(d), with 1/sqrt(d) rounded to fp32.
+ *                 Prefill takes d = 16 only (RTP_ERR_SHAPE otherwise).
  *   max_ctx       Lmax, cache capacity per sequence (positions [0, Lmax));
  *                 at most 2^23
  *   n_sink        S >= 0: positions [0, S) are always attended (sinks)
@@ -116,8 +120,11 @@ typedef struct rtp_layer_cfg {
  *           a retrieval head taking Lmax rows (position j in row j) and a local
  *           head S + local_cap rows (position j < S in row j, position j >= S
  *           in row S + (j - S) mod local_cap).
- *   kidx    [B][R][Lmax][16]   16-d indexer keys k~ = W_k k_pre, one row per
- *                              token for each retrieval KV head (pre-RoPE)
+ *   kidx    [B][R][Lk][d]      d-dim indexer keys k~ = W_k k_pre, one row per
+ *                              token for each retrieval KV head (pre-RoPE);
+ *                              Lk = Lmax, except Lmax rounded up to even when a
+ *                              row is 8 bytes (bf16, d = 4), so that every
+ *                              (b, r) block starts on a 16-byte boundary
  *   status  one int of device-side error bits (see RTP_DEV_*), zeroed by the
  *           caller before first use
  */
@@ -150,7 +157,7 @@ int rtp_prefill_workspace_bytes(const rtp_layer_cfg* cfg, int T, size_t* bytes);
  *
  *   k_pre, v_in  [B][T][Hkv][D] dtype, device
  *   start_pos    [B] int32, device
- *   w_k          [R][16][D] fp32, device (may be NULL when R = 0)
+ *   w_k          [R][d][D] fp32, device (may be NULL when R = 0)
  * Rows with pos outside [0, max_ctx) are skipped and set RTP_DEV_POSITION.
  */
 int rtp_append_kv(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* k_pre,
@@ -163,7 +170,7 @@ int rtp_append_kv(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* 
  * Local KV heads: exact attention over sinks [0, S) and window
  * [seq_len-W, seq_len) (atlas.scime.ai summary, "Approach").
  * Retrieval KV heads, for each of their G query heads separately:
- *   q~ = W_q^(r) q_pre (fp32), s_j = q~ . kidx_j / 4 for every cached j
+ *   q~ = W_q^(r) q_pre (fp32), s_j = q~ . kidx_j / sqrt(d) for every cached j
  *   (fp32; for a bf16 layer on tensor cores from q~'s bf16 high and low parts,
  *   the fp32 score to about 2^-17 of the score),
  *   P = softmax(s); keep the smallest set, ordered by (P desc, j asc), whose
@@ -175,7 +182,7 @@ int rtp_append_kv(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* 
  *   seq_len      [B] int32, device, 1 <= seq_len[b] <= max_seq_len
  *   max_seq_len  host int, an upper bound on seq_len (sizes the grid);
  *                0 means cfg->max_ctx
- *   w_q          [R][16][D] fp32, device
+ *   w_q          [R][d][D] fp32, device
  *   out          [B][Hq][D] dtype, device
  *   sel_bitmask  optional (NULL to skip) [B][R*G][ceil(max_ctx/32)] uint32: bit
  *                j of head (b, r*G+g) is set iff token j is in that query head's
@@ -198,6 +205,29 @@ int rtp_decode_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void
                     const int* seq_len, int max_seq_len, const float* w_q, void* out,
                     uint32_t* sel_bitmask, int* sel_count, void* workspace,
                     size_t workspace_bytes, void* stream);
+
+/* Attention mass recall of a decode step's retrieval heads, a diagnostic the
+ * method is evaluated by (atlas.scime.ai summary, "Experimental setup",
+ * metrics): for each sequence b and retrieval query head r*G+g, the share of
+ * the full causal attention's softmax mass, softmax(RoPE(q, L-1) . k_j /
+ * sqrt(D)) over every j in [0, L), L = seq_len[b], that the rows the decode
+ * step attended carry: the top-p set of sel_bitmask united with the sinks
+ * [0, S) and the window [L-W, L).  fp32 arithmetic; a full-attention pass
+ * over the retrieval heads' keys, so it costs about a dense decode step.
+ *
+ *   q_pre, seq_len, max_seq_len  as for the rtp_decode_attn call that wrote
+ *                sel_bitmask (same cache contents)
+ *   sel_bitmask  [B][R*G][ceil(max_ctx/32)] uint32, device, as rtp_decode_attn
+ *                writes it
+ *   recall       [B][R*G] float, device, in [0, 1]
+ *   workspace    device, 256-byte aligned, contents clobbered; a workspace of
+ *                rtp_decode_workspace_bytes bytes is always large enough
+ * A sequence with an invalid seq_len is skipped (its recall entries untouched).
+ * With no retrieval heads the call does nothing.
+ */
+int rtp_decode_recall(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
+                      const int* seq_len, int max_seq_len, const uint32_t* sel_bitmask,
+                      float* recall, void* workspace, size_t workspace_bytes, void* stream);
 
 /* Size of the fixed device scratch array behind rtp_decode_attn_noalloc. */
 #define RTP_NOALLOC_SCRATCH_BYTES (32u << 20)
@@ -240,7 +270,7 @@ int rtp_decode_attn_noalloc(const rtp_layer_cfg* cfg, const rtp_cache* cache, co
  * a row's top-p set equals the decode step's at that position, bit for bit.
  * The attention itself runs on tensor cores in bf16 with fp32 accumulation
  * (atlas.scime.ai summary, "Approach"; abstract, observations (2)-(3)).
- * cfg->dtype must be RTP_BF16.
+ * cfg->dtype must be RTP_BF16 and cfg->idx_dim 16.
  *
  *   q_pre        [B][T][Hq][D] bf16, device
  *   start_pos    [B] int32, device; 0 <= start_pos[b] and start_pos[b] + T <= max_ctx
@@ -271,7 +301,7 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
 /* Kernel stages, for rtp_trace_stage. */
 typedef enum rtp_stage {
   RTP_STAGE_APPEND = 0,         /* rtp_append_kv: RoPE + cache + indexer-key store */
-  RTP_STAGE_DECODE_SCORE = 1,   /* decode: indexer scores over the 16-d key cache */
+  RTP_STAGE_DECODE_SCORE = 1,   /* decode: indexer scores over the d-dim key cache */
   RTP_STAGE_DECODE_SELECT = 2,  /* decode: exact top-p selection, bitmask, kept-row attention, merge */
   RTP_STAGE_DECODE_LOCAL = 3,   /* decode: sink/window attention of every KV head (overlaps the scores) */
   RTP_STAGE_PREFILL_INDEX = 4,  /* prefill: per-row exact top-p selection */

@@ -18,7 +18,9 @@ arXiv 2605.16928):
   observation (2)) built on a pre-RoPE low-dimensional projection
   (atlas.scime.ai summary, "Approach" and the one-line summary above
   "Problem"):  q~ = W_q q_pre,  k~ = W_k k_pre,  score = q~ . k~ / 4
-  (1/sqrt(16)).
+  (1/sqrt(16)).  The pages' dimension ablation also runs other widths
+  (atlas "Surprising findings": dimension 4); at width d the score is
+  q~ . k~ / sqrt(d) (the reading that keeps d = 16 as above).
 * The token budget is query-dependent: a top-p threshold rather than a fixed
   top-k (abstract, observation (3); atlas "Approach": "query-adaptive top-p
   threshold").  Reading used here: P = softmax of the scores over every
@@ -51,7 +53,7 @@ from typing import Dict, Iterable, Optional, Sequence
 import numpy as np
 
 IDX_DIM = 16
-INDEXER_SCALE = 0.25  # 1 / sqrt(16)
+INDEXER_SCALE = 0.25  # 1 / sqrt(16), the pages' width
 
 _BF16_DROP = 45  # fp64 has 52 explicit mantissa bits, bf16 keeps 7
 
@@ -117,13 +119,16 @@ def rope(x, pos, base: float) -> np.ndarray:
 
 
 def indexer_project(x_pre, w) -> np.ndarray:
-    """16-d pre-RoPE projection:  w [16, D] applied to x_pre [..., D]."""
+    """d-dim pre-RoPE projection:  w [d, D] applied to x_pre [..., D]."""
     return _as_f64(x_pre) @ _as_f64(w).T
 
 
 def indexer_scores(q_idx, k_idx) -> np.ndarray:
-    """score_j = q~ . k~_j / 4  for k_idx [n, 16], q_idx [16]."""
-    return (_as_f64(k_idx) @ _as_f64(q_idx)) * INDEXER_SCALE
+    """score_j = q~ . k~_j / sqrt(d)  for k_idx [n, d], q_idx [d] (d = 16: / 4)."""
+    q = _as_f64(q_idx)
+    d = q.shape[-1]
+    scale = INDEXER_SCALE if d == IDX_DIM else 1.0 / math.sqrt(d)
+    return (_as_f64(k_idx) @ q) * scale
 
 
 def top_p_set(scores, p: float) -> np.ndarray:
@@ -174,7 +179,7 @@ class OracleCache:
     """The layer's cache as the oracle sees it.
 
     Holds the pre-RoPE keys and the values as given (bf16 / fp32 containers,
-    converted to fp64 on read) and the stored 16-d indexer keys (fp64, rounded
+    converted to fp64 on read) and the stored d-dim indexer keys (fp64, rounded
     to the storage precision) for the retrieval KV heads.  A stored key row is
     round(RoPE(k_pre, pos)), produced when read.
     """
@@ -185,7 +190,8 @@ class OracleCache:
         B, Hkv, D = shape.batch, shape.n_kv_heads, shape.head_dim
         self.k_pre = k_store  # [B, Lmax, Hkv, D]
         self.v = v_store
-        self.kidx = np.full((B, shape.n_retrieval, self.max_ctx, IDX_DIM), np.nan)
+        d = int(getattr(shape, "idx_dim", IDX_DIM))
+        self.kidx = np.full((B, shape.n_retrieval, self.max_ctx, d), np.nan)
         self.length = np.zeros(B, dtype=np.int64)
 
     # -- append ---------------------------------------------------------

@@ -54,11 +54,33 @@ def test_cache_and_workspace_sizes(rtp):
     assert ws % 256 == 0
 
 
+@pytest.mark.parametrize("d,dtype,lmax,lk", [(4, "bf16", 1001, 1002), (4, "bf16", 1000, 1000),
+                                              (4, "fp32", 1001, 1001), (8, "bf16", 1001, 1001),
+                                              (32, "bf16", 777, 777)])
+def test_indexer_cache_rows_per_width(rtp, d, dtype, lmax, lk):
+    """kidx is [B][R][Lk][d]: Lk = Lmax except 8-byte rows (bf16, d = 4), which
+    take an even row count so every (sequence, head) block is 16-byte aligned."""
+    es = 2 if dtype == "bf16" else 4
+    _, _, ki = rtp.rtp_cache_bytes(_cfg(rtp, idx_dim=d, dtype=dtype, max_ctx=lmax, window=64, n_sink=4))
+    assert ki == 1 * 2 * lk * d * es
+    assert (lk * d * es) % 16 == 0
+
+
+def test_prefill_takes_width_16_only(rtp):
+    c = _cfg(rtp, idx_dim=8)
+    fake = 1 << 20  # never dereferenced: validation fails first
+    cache = rtp.rtp_cache(fake, fake, fake, fake)
+    with pytest.raises(rtp.RtpError) as e:
+        rtp.rtp_prefill_attn(c, cache, fake, fake, 8, fake, fake, workspace=fake, workspace_bytes=1 << 40,
+                             stream=0)
+    assert e.value.code == 2
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(head_dim=96), 2), (dict(n_q_heads=24), 2), (dict(n_q_heads=30), 2),
     (dict(top_p=0.0), 1), (dict(top_p=1.5), 1), (dict(window=0), 1), (dict(n_sink=-1), 1),
     (dict(max_ctx=0), 2), (dict(max_ctx=(1 << 23) + 1), 2), (dict(retrieval=(9,)), 2),
-    (dict(idx_dim=8), 2), (dict(rope_base=1.0), 1),
+    (dict(idx_dim=12), 2), (dict(rope_base=1.0), 1),
 ])
 def test_invalid_cfg_rejected(rtp, kw, code):
     with pytest.raises(rtp.RtpError) as e:

@@ -131,6 +131,35 @@ def test_indexer_scale_two_token_golden():
         assert list(topp[(0, 0)]) == case["kept"], case
 
 
+@pytest.mark.parametrize("width", [0, 1, 2, 3])
+def test_indexer_width_golden(width):
+    """Score scale 1/sqrt(d) at every width of the dimension ablation, with the
+    projection into the last of the d indexer dims (hand-derived, tests/golden)."""
+    d = json.load(open(os.path.join(GOLD, "indexer_widths.json")))
+    D, qc, kc = d["head_dim"], d["q_coord"], d["k_coord"]
+    w = d["widths"][width]
+    n = w["idx_dim"]
+    for case in d["cases"]:
+        sh = LayerShape(batch=1, n_q_heads=1, n_kv_heads=1, head_dim=D, n_sink=0, window=1,
+                        top_p=case["p"], retrieval=(0,), dtype="fp32", idx_dim=n)
+        wq = torch.zeros((1, n, D))
+        wq[0, n - 1, qc] = 1.0
+        wk = torch.zeros((1, n, D))
+        wk[0, n - 1, kc] = 1.0
+        k = torch.zeros((1, 2, 1, D), dtype=torch.float64)
+        for j in range(2):
+            k[0, j, 0, kc] = w["k_values"][j]
+            k[0, j, 0, qc] = d["k_junk"][j]
+        v = torch.randn((1, 2, 1, D))
+        q = torch.zeros((1, 1, D))
+        q[0, 0, qc] = d["q_value"]
+        q[0, 0, kc] = d["q_junk"]
+        c = OracleCache(sh, 2)
+        c.append(k, v, [0], 2, wk)
+        _, topp, _ = oracle.decode(c, q, [2], wq)
+        assert list(topp[(0, 0)]) == case["kept"], (n, case)
+
+
 @pytest.mark.parametrize("path", ["append", "append_in_place", "prefill"])
 def test_indexer_key_storage_rounding_golden(path):
     """The stored indexer key is rounded to the cache's storage type before it
