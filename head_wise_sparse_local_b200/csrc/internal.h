@@ -81,12 +81,14 @@ int launch_recall(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
 
 struct PrefillLayout {
   size_t total;
-  int block_rows;  // query rows per selection + attention pass
+  size_t tmap;     // offset of the attention's key-tile map
+  int block_rows;  // query rows per selection + attention pass (a multiple of 256 unless the whole chunk)
 };
+size_t tile_map_bytes(const Shape& sh, int T);
 PrefillLayout prefill_layout(const Shape& sh, int T);
 int launch_attn_tc(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* start_pos, int T,
                    void* out, const uint32_t* mask, int t_base, int t_end, int mask_t0, int mask_rows,
-                   unsigned long long wait_ns, cudaStream_t st);
+                   uint32_t* tmap, unsigned long long wait_ns, cudaStream_t st);
 int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* start_pos,
                    int T, const float* w_q, void* out, uint32_t* sel_bitmask, float* sel_tau,
                    int* sel_jcut, int* sel_count, void* ws, const PrefillLayout& lay, cudaStream_t st);

@@ -948,17 +948,19 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 }  // namespace
 
 // Rows whose top-p bitmask the workspace holds at once: the whole chunk when
-// that stays under kMaskBudget, else blocks of a multiple of the attention
-// tile (the chunk then runs block by block: selection, attention, next block).
+// that stays under kMaskBudget, else blocks of a multiple of the tcgen05
+// attention's 256-row groups (the chunk then runs block by block: selection,
+// attention, next block).
 constexpr size_t kMaskBudget = size_t(1) << 30;
+constexpr int kBlockAlign = 256;
 
 int prefill_block_rows(const Shape& sh, int T) {
   const size_t words = (size_t)(sh.Lmax + 31) / 32;
   const size_t per_row = (size_t)sh.B * (size_t)(sh.NR > 0 ? sh.NR : 1) * words * sizeof(uint32_t);
   size_t rows = kMaskBudget / per_row;
   if (rows >= (size_t)T) return T;
-  rows = rows / kBQ * kBQ;
-  return rows < (size_t)kBQ ? kBQ : (int)rows;
+  rows = rows / kBlockAlign * kBlockAlign;
+  return rows < (size_t)kBlockAlign ? kBlockAlign : (int)rows;
 }
 
 PrefillLayout prefill_layout(const Shape& sh, int T) {
@@ -966,7 +968,8 @@ PrefillLayout prefill_layout(const Shape& sh, int T) {
   const size_t words = (size_t)(sh.Lmax + 31) / 32;
   const int rows = prefill_block_rows(sh, T);
   l.block_rows = rows;
-  l.total = align256((size_t)sh.B * sh.NR * rows * words * sizeof(uint32_t)) + 256;
+  l.tmap = align256((size_t)sh.B * sh.NR * rows * words * sizeof(uint32_t));
+  l.total = l.tmap + align256(tile_map_bytes(sh, T)) + 256;
   return l;
 }
 
@@ -1022,7 +1025,8 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
     // full-context heads on tcgen05 tensor cores; local heads that keep a
     // window ring (rows not contiguous in positions) on the mma.sync kernel
     int rc = launch_attn_tc(sh, cache, q_pre, start_pos, T, out, a.mask, a.t_base, a.t_end, a.mask_t0,
-                            a.mask_rows, 400ull * 1000 * 1000, st);
+                            a.mask_rows, reinterpret_cast<uint32_t*>(static_cast<char*>(ws) + lay.tmap),
+                            400ull * 1000 * 1000, st);
     if (rc != RTP_OK) return rc;
     if (sh.kv.ring_mask) {
       a.ring_only = 1;

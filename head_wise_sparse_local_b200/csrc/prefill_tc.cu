@@ -1,31 +1,44 @@
 // Prefill attention on the fifth-generation tensor cores (tcgen05 + TMEM).
 //
-// One CTA per (sequence, query head, 128-row query tile).  Per key tile of 128
-// keys: S = Q K^T (128 x 128, fp32 in TMEM), a softmax over S by the thread
-// that owns the row (one TMEM lane per thread), then O += P V (128 x D, fp32
-// in TMEM).  The layer's masks (causality; sinks and window; for retrieval
-// heads the row's top-p bitmask from the selection kernel) are applied to S
-// (atlas.scime.ai summary, "Approach"; abstract, observations (2)-(3)).
+// One CTA per (sequence, query head, 256 query rows), the rows split into two
+// slots of 128 (one TMEM lane per row).  The CTA walks the key tiles (128 keys)
+// that any of its rows attends, and for each tile and slot: S = Q K^T (128 x
+// 128, fp32 in TMEM), a softmax over S by the thread that owns the row, P (bf16)
+// written back into S's TMEM columns, then O += P V with P taken from TMEM
+// (128 x D, fp32 in TMEM).  The layer's masks (causality; sinks and window;
+// for retrieval heads the row's top-p bitmask from the selection kernel) are
+// applied to S (atlas.scime.ai summary, "Approach"; abstract, observations
+// (2)-(3)).  Tiles in which every row of a slot sees every key need no mask.
 //
-// Roles (256 threads):
+// The key tiles: the sink tiles and the window tiles of the CTA's rows, and for
+// retrieval heads every tile in which some row keeps a token (a per-CTA tile
+// map that tile_map_kernel reduces from the selection bitmask); never a tile
+// past the last row's position.
+//
+// Roles (320 threads):
 //   warp 0, lane 0   stages K and V tiles with TMA (cp.async.bulk.tensor,
 //                    128-byte swizzle, boxes of 64 dims x 128 keys), two
 //                    stages in flight;
 //   warp 1           allocates TMEM; lane 0 issues every tcgen05.mma and
-//                    commits its completions to mbarriers;
-//   warps 4-7        one thread per query row: read S from TMEM, mask, keep
-//                    the running maximum and sum, write P (bf16) to shared
-//                    memory, rescale O in TMEM when the maximum grows by more
-//                    than 2^8, and finally read O and write the output.
-// S has two TMEM buffers, so S of tile j + 1 is computed while tile j's
-// softmax runs.  Every wait on an mbarrier is bounded: on expiry the CTA sets
+//                    commits its completions to mbarriers, in the order
+//                    S0(i), PV1(i-1), S1(i), PV0(i), so that each slot's
+//                    softmax overlaps the other slot's products;
+//   warps 2-5, 6-9   the softmax of slot 0 and slot 1 (thread = query row):
+//                    read S from TMEM, mask, keep the running maximum and
+//                    sum, write P to TMEM, rescale O in TMEM when the maximum
+//                    grows by more than 2^8, and finally write the output.
+// tcgen05.mma operations issued by one thread execute in issue order, so S of
+// the next tile may overwrite the TMEM columns that the previous PV read P
+// from; a commit after S(i) of a slot also tells that slot's softmax that
+// PV(i-1) has completed (its O may be rescaled, its P columns rewritten).
+// Every wait on an mbarrier is bounded: on expiry the CTA sets
 // RTP_DEV_TIMEOUT, stops issuing work, waits (bounded) for what it issued and
 // frees its TMEM.
 //
 // Shared-memory operands use the canonical 128-byte-swizzled layouts of the
-// tcgen05 matrix descriptors: K-major (Q, K, P: 8-row atoms of 128-byte rows,
-// 16-byte chunk c of row r at chunk c ^ (r mod 8)) and MN-major (V: 8-key
-// atoms of 64 dims, the next 64 dims one region further).
+// tcgen05 matrix descriptors: K-major (Q, K: 8-row atoms of 128-byte rows,
+// 16-byte chunk c of row r at chunk c ^ (r mod 8)) and MN-major (V: 8-key atoms
+// of 64 dims, the next 64 dims one region further).
 #include <cuda.h>  // CUtensorMap and its encoding enums (the encoder is fetched through the runtime)
 
 #include <mutex>
@@ -36,12 +49,15 @@
 namespace rtp {
 namespace {
 
-constexpr int kTcRows = 128;      // query rows per CTA = TMEM lanes
+constexpr int kTcRows = 128;      // query rows per slot = TMEM lanes
+constexpr int kSlots = 2;
+constexpr int kGroupRows = kSlots * kTcRows;  // query rows per CTA
 constexpr int kTcKeys = 128;      // keys per tile
-constexpr int kTcThreads = 256;
+constexpr int kTcThreads = 320;
 constexpr int kRegion = 128 * 128;  // bytes of a 128-row x 64-dim bf16 region (one TMA box)
 constexpr int kTmemCols = 512;
 constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
+constexpr int kMaxTileWords = ((1 << 23) / kTcKeys) / 32 + 1;  // tile bitmap words for the largest context
 
 struct __align__(64) TcArgs {
   CUtensorMap tm_k;  // K cache as [rows][D] bf16, boxes of 64 x 128, 128-byte swizzle
@@ -52,6 +68,9 @@ struct __align__(64) TcArgs {
   int* status;
   const int* start_pos;
   const uint32_t* mask;  // [B][NR][mask_rows][words] top-p bitmask of rows [mask_t0, mask_t0 + mask_rows)
+  const uint32_t* tmap;  // [B][NR][map_groups][map_words] key tiles some row of a 256-row group keeps
+  uint32_t* tmap_out;    // the same array, written by tile_map_kernel
+  int map_words, map_groups, map_g0;  // words per group; groups per head; group of this launch's first CTA
   int t_base, t_end, mask_t0, mask_rows;
   int n_heads;            // query heads this launch covers: head_list[0, n_heads)
   unsigned long long wait_ns;
@@ -63,15 +82,14 @@ struct __align__(64) TcArgs {
 
 template <int D>
 struct TcSmem {
-  static constexpr int kQ = (D / 64) * kRegion;        // Q: D/64 regions
+  static constexpr int kQ = (D / 64) * kRegion;        // Q of one slot: D/64 regions
   static constexpr int kK = (D / 64) * kRegion;        // one K stage
   static constexpr int kV = (D / 64) * kRegion;        // one V stage
-  static constexpr int kP = 2 * kRegion;               // P: keys 0-63, 64-127
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQ;             // two stages
+  static constexpr int kOffQ = 0;                      // two slots
+  static constexpr int kOffK = kOffQ + kSlots * kQ;    // two stages
   static constexpr int kOffV = kOffK + 2 * kK;         // two stages
-  static constexpr int kOffP = kOffV + 2 * kV;
-  static constexpr int kBytes = kOffP + kP + 1024;     // + alignment slack
+  static constexpr int kOffTiles = kOffV + 2 * kV;     // key-tile bitmap
+  static constexpr int kBytes = kOffTiles + kMaxTileWords * 4 + 1024;  // + alignment slack
 };
 
 // ---------------------------------------------------------------------------
@@ -177,26 +195,57 @@ __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, const Tc
   return true;
 }
 
-// Key tiles a (head, row tile) attends: all causal tiles for retrieval heads;
-// for local heads the tiles holding sinks, then those holding the window.
-struct TileSeq {
-  int n_a, b0, n;  // tiles [0, n_a), then tiles b0, b0 + 1, ... (n in total)
-  __device__ __forceinline__ int start(int j) const { return (j < n_a ? j : b0 + (j - n_a)) * kTcKeys; }
-};
-__device__ __forceinline__ TileSeq tile_seq(bool local, int S, int W, int i_min, int i_max) {
-  TileSeq q;
-  const int last = i_max / kTcKeys;
-  if (!local) {
-    q.n_a = last + 1;
-    q.b0 = last + 1;
-    q.n = last + 1;
-    return q;
-  }
-  q.n_a = min((S + kTcKeys - 1) / kTcKeys, last + 1);
-  q.b0 = max(q.n_a, max(0, i_min - W + 1) / kTcKeys);
-  q.n = q.n_a + max(0, last - q.b0 + 1);
-  return q;
+// tcgen05.mma of kind::f16 with A from TMEM (P) and B from shared memory (V).
+__device__ __forceinline__ void umma_f16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, {%5, %6, %7, %8}, p;\n\t}\n"
+      :: "r"(tmem_d), "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
+
+// 16 consecutive 32-bit columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+      :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+         "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]));
+}
+
+__device__ __forceinline__ float max3f(float x, float y, float z) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(x), "f"(y), "f"(z));
+  return m;
+}
+
+// 2^x by the hardware approximation (relative error about 2^-22; -inf -> +0).
+__device__ __forceinline__ float ex2f(float x) {
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x));
+  return e;
+}
+
+// Walks the set bits of a shared-memory tile bitmap in increasing order.
+struct TileCursor {
+  const uint32_t* bits;
+  int nw, w;
+  uint32_t cur;
+  __device__ __forceinline__ void init(const uint32_t* b, int n) {
+    bits = b;
+    nw = n;
+    w = 0;
+    cur = n > 0 ? b[0] : 0u;
+  }
+  __device__ __forceinline__ int next() {
+    while (cur == 0u) {
+      if (++w >= nw) return -1;
+      cur = bits[w];
+    }
+    const int t = w * 32 + (__ffs(cur) - 1);
+    cur &= cur - 1u;
+    return t;
+  }
+};
 
 // ---------------------------------------------------------------------------
 // the kernel
@@ -204,16 +253,17 @@ __device__ __forceinline__ TileSeq tile_seq(bool local, int S, int W, int i_min,
 template <int D>
 __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_constant__ TcArgs a) {
   using SM = TcSmem<D>;
-  constexpr int NR = D / 64;  // 64-dim regions
+  constexpr int NRG = D / 64;  // 64-dim regions
   extern __shared__ __align__(1024) unsigned char dsm_raw[];
-  __shared__ __align__(8) uint64_t bar_kv_full[2], bar_kv_empty[2], bar_s_full[2], bar_s_free[2];
-  __shared__ __align__(8) uint64_t bar_p_full, bar_o_done, bar_fin;
+  __shared__ __align__(8) uint64_t bar_kv_full[2], bar_kv_empty[2], bar_s_full[kSlots], bar_p_full[kSlots];
+  __shared__ __align__(8) uint64_t bar_o_done, bar_fin;
   __shared__ uint32_t s_tmem;
-  __shared__ int s_abort;
+  __shared__ int s_abort, s_ntiles;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned char* dsm = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);
   const uint32_t sQ = smem_u32(dsm + SM::kOffQ), sK = smem_u32(dsm + SM::kOffK);
-  const uint32_t sV = smem_u32(dsm + SM::kOffV), sP = smem_u32(dsm + SM::kOffP);
+  const uint32_t sV = smem_u32(dsm + SM::kOffV);
+  uint32_t* s_tiles = reinterpret_cast<uint32_t*>(dsm + SM::kOffTiles);
 
   const int bq = blockIdx.y;
   const int b = bq / a.n_heads, hq = a.head_list[bq % a.n_heads];
@@ -221,10 +271,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
   const int r = a.ret_rank[h];
   const int start = a.start_pos[b];
   if (start < 0 || start + a.T > a.Lmax) return;  // flagged by the selection kernel / host (uniform)
-  const int t0 = a.t_base + blockIdx.x * kTcRows;
-  const int t_last = min(a.t_end, t0 + kTcRows) - 1;
-  const int i_min = start + t0, i_max = start + t_last;
-  const TileSeq ts = tile_seq(r < 0, a.S, a.W, i_min, i_max);
+  const int t0 = a.t_base + blockIdx.x * kGroupRows;
+  const int t_last = min(a.t_end, t0 + kGroupRows) - 1;
+  const int i_lo = start + t0, i_hi = start + t_last;
+  const int last_tile = i_hi / kTcKeys;
+  const int n_words = last_tile / 32 + 1;
   const int hh = r >= 0 ? r * a.G + g : 0;
 
   if (tid == 0) {
@@ -232,25 +283,52 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       mbar_init(&bar_kv_full[s], 1);
       mbar_init(&bar_kv_empty[s], 1);
       mbar_init(&bar_s_full[s], 1);
-      mbar_init(&bar_s_free[s], 128);
+      mbar_init(&bar_p_full[s], kTcRows);
     }
-    mbar_init(&bar_p_full, 128);
     mbar_init(&bar_o_done, 1);
     mbar_init(&bar_fin, 1);
     s_abort = 0;
+    s_ntiles = 0;
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                  :: "r"(smem_u32(&s_tmem)), "r"(kTmemCols) : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  // ---- Q tile: RoPE at each row's position, scaled by log2(e)/sqrt(D), bf16,
-  // into the swizzled K-major layout (rows past the chunk are zero) ----
+  __syncthreads();
+  // ---- key tiles: sinks, the rows' windows and (retrieval heads) the tiles
+  // some row keeps, none past the last row's tile ----
+  {
+    const int ns = min((a.S + kTcKeys - 1) / kTcKeys, last_tile + 1);  // sink tiles [0, ns)
+    const int w0 = max(0, i_lo - a.W + 1) / kTcKeys;                   // window tiles [w0, last_tile]
+    const uint32_t* mp = r >= 0 ? a.tmap + (((size_t)b * a.NR + hh) * a.map_groups + a.map_g0 + blockIdx.x) *
+                                               (size_t)a.map_words
+                                : nullptr;
+    int cnt = 0;
+    for (int w = tid; w < n_words; w += kTcThreads) {
+      const int lo = w * 32, hi = lo + 31;
+      uint32_t v = 0u;
+      if (lo < ns) v |= ns - lo >= 32 ? 0xffffffffu : (1u << (ns - lo)) - 1u;
+      const int a0 = max(lo, w0), a1 = min(hi, last_tile);
+      if (a0 <= a1) v |= a1 - a0 == 31 ? 0xffffffffu : ((1u << (a1 - a0 + 1)) - 1u) << (a0 - lo);
+      if (mp) v |= __ldg(mp + w);
+      if (hi > last_tile) v &= (1u << (last_tile - lo + 1)) - 1u;  // lo <= last_tile < hi
+      s_tiles[w] = v;
+      cnt += __popc(v);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+    if (lane == 0 && cnt) atomicAdd(&s_ntiles, cnt);
+  }
+  // ---- Q of both slots: RoPE at each row's position, scaled by
+  // log2(e)/sqrt(D), bf16, into the swizzled K-major layout (rows past the
+  // chunk are zero) ----
   {
     const float qscale = 1.4426950408889634f * rsqrtf((float)D);
     constexpr int H = D / 2;
-    for (int task = tid; task < kTcRows * (H / 8); task += kTcThreads) {
-      const int rr = task / (H / 8), c8 = task % (H / 8);  // row, 8-dim chunk of the low half
+    for (int task = tid; task < kGroupRows * (H / 8); task += kTcThreads) {
+      const int rr = task / (H / 8), c8 = task % (H / 8);  // row of the CTA, 8-dim chunk of the low half
+      const int slot = rr / kTcRows, lr = rr % kTcRows;
       const int t = t0 + rr;
       float y1[8], y2[8];
       if (t <= t_last) {
@@ -274,10 +352,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       hi.x = pack_bf16(y2[0], y2[1]); hi.y = pack_bf16(y2[2], y2[3]); hi.z = pack_bf16(y2[4], y2[5]); hi.w = pack_bf16(y2[6], y2[7]);
       // dims d = c8*8.. (low half) and H + c8*8.. (high half): region d / 64, chunk (d % 64) / 8
       const int d_lo = c8 * 8, d_hi = H + c8 * 8;
-      const int reg_lo = d_lo / 64, ch_lo = (d_lo % 64) / 8;
-      const int reg_hi = d_hi / 64, ch_hi = (d_hi % 64) / 8;
-      *reinterpret_cast<uint4*>(dsm + SM::kOffQ + reg_lo * kRegion + rr * 128 + ((ch_lo ^ (rr & 7)) * 16)) = lo;
-      *reinterpret_cast<uint4*>(dsm + SM::kOffQ + reg_hi * kRegion + rr * 128 + ((ch_hi ^ (rr & 7)) * 16)) = hi;
+      unsigned char* qs = dsm + SM::kOffQ + slot * SM::kQ + lr * 128;
+      *reinterpret_cast<uint4*>(qs + (d_lo / 64) * kRegion + ((((d_lo % 64) / 8) ^ (lr & 7)) * 16)) = lo;
+      *reinterpret_cast<uint4*>(qs + (d_hi / 64) * kRegion + ((((d_hi % 64) / 8) ^ (lr & 7)) * 16)) = hi;
     }
   }
   fence_async_smem();
@@ -285,190 +362,219 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem;
-  const uint32_t tS[2] = {tmem, tmem + kTcKeys};
-  const uint32_t tO = tmem + 2 * kTcKeys;
-  const int n = ts.n;
+  const int n = s_ntiles;
 
   if (warp == 0) {
     if (lane == 0) {
       // ---- producer: K and V tiles by TMA ----
       const uint64_t pol = l2_evict_last();
       const size_t rowbase = a.kv.row(b, h, 0);  // full-cache head: position p at rowbase + p
-      for (int j = 0; j < n; ++j) {
-        const int s = j & 1, k = j >> 1;
-        if (!tc_wait(&bar_kv_empty[s], (uint32_t)(k & 1) ^ 1u, a, &s_abort)) break;
-        mbar_expect_tx(&bar_kv_full[s], (uint32_t)(2 * NR * kRegion));
-        const int y = (int)(rowbase + ts.start(j));
+      TileCursor cur;
+      cur.init(s_tiles, n_words);
+      for (int i = 0; i < n; ++i) {
+        const int kt = cur.next() * kTcKeys;
+        const int st = i & 1;
+        if (!tc_wait(&bar_kv_empty[st], ((uint32_t)(i >> 1) & 1u) ^ 1u, a, &s_abort)) break;
+        mbar_expect_tx(&bar_kv_full[st], (uint32_t)(2 * NRG * kRegion));
+        const int y = (int)(rowbase + kt);
 #pragma unroll
-        for (int rg = 0; rg < NR; ++rg) {
-          tma_load_2d(dsm + SM::kOffK + s * SM::kK + rg * kRegion, &a.tm_k, rg * 64, y, &bar_kv_full[s], pol);
-          tma_load_2d(dsm + SM::kOffV + s * SM::kV + rg * kRegion, &a.tm_v, rg * 64, y, &bar_kv_full[s], pol);
+        for (int rg = 0; rg < NRG; ++rg) {
+          tma_load_2d(dsm + SM::kOffK + st * SM::kK + rg * kRegion, &a.tm_k, rg * 64, y, &bar_kv_full[st], pol);
+          tma_load_2d(dsm + SM::kOffV + st * SM::kV + rg * kRegion, &a.tm_v, rg * 64, y, &bar_kv_full[st], pol);
         }
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---- MMA issuer ----
-      constexpr uint32_t idS = umma_idesc(kTcRows, kTcKeys, false);
-      constexpr uint32_t idO = umma_idesc(kTcRows, D, true);
-      auto issue_s = [&](int j) {  // S(j) = Q K(j)^T into buffer j & 1
-        const int s = j & 1;
+    // ---- MMA issuer: the warp walks the tiles together (it zeroes the value
+    // rows past the CTA's last position in the last tile); lane 0 issues ----
+    constexpr uint32_t idS = umma_idesc(kTcRows, kTcKeys, false);
+    constexpr uint32_t idO = umma_idesc(kTcRows, D, true);
+    const uint32_t tS[2] = {tmem, tmem + kTcKeys};
+    const uint32_t tO[2] = {tmem + 2 * kTcKeys, tmem + 3 * kTcKeys};
+    auto issue_s = [&](int slot, int st) {  // S(slot) = Q(slot) K(stage st)^T
+      if (lane == 0) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int rg = kk / 4, ko = (kk % 4) * 32;
-          const uint64_t ad = umma_desc(sQ + rg * kRegion + ko, 16, 1024);
-          const uint64_t bd = umma_desc(sK + s * SM::kK + rg * kRegion + ko, 16, 1024);
-          umma_f16(tS[s], ad, bd, idS, kk > 0 ? 1u : 0u);
+          const uint64_t ad = umma_desc(sQ + slot * SM::kQ + rg * kRegion + ko, 16, 1024);
+          const uint64_t bd = umma_desc(sK + st * SM::kK + rg * kRegion + ko, 16, 1024);
+          umma_f16(tS[slot], ad, bd, idS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&bar_s_full[s]);
-      };
-      bool ok = n > 0 && tc_wait(&bar_kv_full[0], 0u, a, &s_abort);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
+        umma_commit(&bar_s_full[slot]);
       }
-      for (int j = 0; ok && j < n; ++j) {
-        if (j + 1 < n) {
-          const int s1 = (j + 1) & 1, k1 = (j + 1) >> 1;
-          if (!tc_wait(&bar_kv_full[s1], (uint32_t)(k1 & 1), a, &s_abort)) break;
-          if (!tc_wait(&bar_s_free[s1], (uint32_t)(k1 & 1) ^ 1u, a, &s_abort)) break;
-          tc_fence_after();
-          issue_s(j + 1);
-        }
-        if (!tc_wait(&bar_p_full, (uint32_t)(j & 1), a, &s_abort)) break;
-        tc_fence_after();
-        const int s = j & 1;
+      __syncwarp();
+    };
+    auto issue_pv = [&](int slot, int st, bool acc) {  // O(slot) += P(slot) V(stage st), P in S's columns
+      if (lane == 0) {
 #pragma unroll
-        for (int kk = 0; kk < kTcKeys / 16; ++kk) {  // O += P V(j)
-          const int rg = kk / 4, ko = (kk % 4) * 32;
-          const uint64_t ad = umma_desc(sP + rg * kRegion + ko, 16, 1024);
-          const uint64_t bd = umma_desc(sV + s * SM::kV + kk * 2048, kRegion, 1024);
-          umma_f16(tO, ad, bd, idO, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kTcKeys / 16; ++kk) {
+          const uint64_t bd = umma_desc(sV + st * SM::kV + kk * 2048, kRegion, 1024);
+          umma_f16_ts(tO[slot], tS[slot] + kk * 8, bd, idO, (acc || kk > 0) ? 1u : 0u);
         }
-        umma_commit(&bar_o_done);
-        umma_commit(&bar_kv_empty[s]);
       }
+      __syncwarp();
+    };
+    TileCursor cur;
+    cur.init(s_tiles, n_words);
+    bool ok = true;
+    for (int i = 0; i < n; ++i) {
+      const int kt = cur.next() * kTcKeys;
+      const int st = i & 1;
+      if (!__all_sync(0xffffffffu, tc_wait(&bar_kv_full[st], (uint32_t)(i >> 1) & 1u, a, &s_abort))) { ok = false; break; }
+      if (kt + kTcKeys - 1 > i_hi) {
+        // value rows past the CTA's last position may be unwritten cache (their
+        // weights are 0, but 0 x NaN would not be)
+        for (int rr = i_hi - kt + 1 + lane; rr < kTcKeys; rr += 32) {
+#pragma unroll
+          for (int rg = 0; rg < NRG; ++rg) {
+            uint4* vr = reinterpret_cast<uint4*>(dsm + SM::kOffV + st * SM::kV + rg * kRegion + rr * 128);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) vr[c] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        fence_async_smem();
+        __syncwarp();
+      }
+      tc_fence_after();
+      issue_s(0, st);
+      if (i > 0) {
+        if (!__all_sync(0xffffffffu, tc_wait(&bar_p_full[1], (uint32_t)(i - 1) & 1u, a, &s_abort))) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, st ^ 1, i > 1);
+        if (lane == 0) umma_commit(&bar_kv_empty[st ^ 1]);
+      }
+      issue_s(1, st);
+      if (!__all_sync(0xffffffffu, tc_wait(&bar_p_full[0], (uint32_t)i & 1u, a, &s_abort))) { ok = false; break; }
+      tc_fence_after();
+      issue_pv(0, st, i > 0);
+    }
+    if (ok && n > 0 &&
+        __all_sync(0xffffffffu, tc_wait(&bar_p_full[1], (uint32_t)(n - 1) & 1u, a, &s_abort))) {
+      tc_fence_after();
+      issue_pv(1, (n - 1) & 1, n > 1);
+      if (lane == 0) umma_commit(&bar_kv_empty[(n - 1) & 1]);
+    }
+    if (lane == 0) {
+      umma_commit(&bar_o_done);
       // every MMA this thread issued has completed before TMEM is freed
       umma_commit(&bar_fin);
       mbar_wait_bounded(&bar_fin, 0u, a.wait_ns, a.status);
     }
-  } else if (warp >= 4) {
-    // ---- softmax: thread = query row ----
-    const int row = tid - 128;  // TMEM lane
-    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
-    const int t = t0 + row;
+    __syncwarp();
+  } else {
+    // ---- softmax: warps 2-5 slot 0, warps 6-9 slot 1; thread = query row ----
+    const int slot = (warp - 2) >> 2;
+    const int quad = warp & 3;  // the TMEM lane quarter this warp may access
+    const int row = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tSs = tmem + slot * kTcKeys, tOs = tmem + (2 + slot) * kTcKeys;
+    const int t = t0 + slot * kTcRows + row;
     const bool rv = t <= t_last;
     const int pi = start + t;
     const int wlo = pi - a.W + 1;
+    const int s_lo = i_lo + slot * kTcRows;          // the slot's first row position
+    const int s_hi = min(i_hi, s_lo + kTcRows - 1);  // its last valid row position (< s_lo: none)
     const uint32_t* mrow = a.mask + (((size_t)b * a.NR + hh) * a.mask_rows + (rv ? t - a.mask_t0 : 0)) * a.words;
+    TileCursor cur;
+    cur.init(s_tiles, n_words);
     float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n; ++j) {
-      const int kt = ts.start(j);
-      const int s = j & 1;
+      const int kt = cur.next() * kTcKeys;
       // every wait's outcome is made warp-uniform: TMEM loads and stores are warp-collective
-      if (!__all_sync(0xffffffffu, tc_wait(&bar_s_full[s], (uint32_t)(j >> 1) & 1u, a, &s_abort))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, tc_wait(&bar_s_full[slot], (uint32_t)j & 1u, a, &s_abort))) { ok = false; break; }
       tc_fence_after();
-      float sv[kTcKeys];
-#pragma unroll
-      for (int c = 0; c < kTcKeys / 32; ++c) {
-        float v[32];
-        tmem_ld32(tS[s] + lane_off + c * 32, v);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = v[e];
-      }
-      tmem_wait_ld();
-      tc_fence_before();
-      mbar_arrive(&bar_s_free[s]);
-      // mask: causal; sinks or window; retrieval heads also keep the top-p set
+      // S is read from TMEM twice (the row maximum, then the weights), 32
+      // columns at a time, which keeps the thread's registers to a few chunks
+      const bool whole = s_lo <= s_hi && kt + kTcKeys - 1 <= s_lo &&
+                         (kt + kTcKeys - 1 < a.S || kt >= s_hi - a.W + 1);
+      // a tile every row of the slot sees whole (causal, inside sinks or
+      // window) needs no mask (uniform over the slot); otherwise causality,
+      // sinks or window, and for retrieval heads the top-p set
       uint32_t mw[4] = {0u, 0u, 0u, 0u};
-      if (r >= 0 && rv) {
+      if (!whole && r >= 0 && rv) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const int wd = (kt >> 5) + q;
           mw[q] = (wd * 32 <= pi) ? __ldg(mrow + wd) : 0u;
         }
       }
+      auto apply_mask = [&](float (&v)[32], int c) {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const int jk = kt + c * 32 + e;
+          const bool keep = rv && jk <= pi && (jk < a.S || jk >= wlo || ((mw[c] >> e) & 1u));
+          v[e] = keep ? v[e] : -CUDART_INF_F;
+        }
+      };
       float tmax = -CUDART_INF_F;
 #pragma unroll
-      for (int c = 0; c < kTcKeys; ++c) {
-        const int jk = kt + c;
-        bool keep = rv && jk <= pi && (jk < a.S || jk >= wlo);
-        if (r >= 0) keep = keep || (rv && jk <= pi && ((mw[c >> 5] >> (c & 31)) & 1u));
-        sv[c] = keep ? sv[c] : -CUDART_INF_F;
-        tmax = fmaxf(tmax, sv[c]);
+      for (int c = 0; c < kTcKeys / 32; c += 2) {
+        float v0[32], v1[32];
+        tmem_ld32(tSs + lane_off + c * 32, v0);
+        tmem_ld32(tSs + lane_off + (c + 1) * 32, v1);
+        tmem_wait_ld();
+        if (!whole) {
+          apply_mask(v0, c);
+          apply_mask(v1, c + 1);
+        }
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) tmax = max3f(tmax, max3f(v0[e], v0[e + 1], v1[e]), v1[e + 1]);
       }
       // lazy rescale: the maximum used moves only when the tile's exceeds it by > 2^8
       float m_new = m_used, f = 1.f;
       if (tmax > m_used + kRescale || (m_used == -CUDART_INF_F && tmax != -CUDART_INF_F)) {
         m_new = tmax;
-        f = (m_used == -CUDART_INF_F) ? 0.f : exp2f(m_used - m_new);
+        f = (m_used == -CUDART_INF_F) ? 0.f : ex2f(m_used - m_new);
       }
-      float lsum = 0.f;
-      uint32_t pk[kTcKeys / 2];
-#pragma unroll
-      for (int c = 0; c < kTcKeys; c += 2) {
-        const float p0 = sv[c] == -CUDART_INF_F ? 0.f : exp2f(sv[c] - m_new);
-        const float p1 = sv[c + 1] == -CUDART_INF_F ? 0.f : exp2f(sv[c + 1] - m_new);
-        lsum += p0 + p1;
-        pk[c / 2] = pack_bf16(p0, p1);
-      }
-      l = l * f + lsum;
       m_used = m_new;
-      // P's buffer and O are free once PV(j - 1) has completed
-      if (j > 0 && !__all_sync(0xffffffffu, tc_wait(&bar_o_done, (uint32_t)((j - 1) & 1), a, &s_abort))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {  // rescale O rows (warp-uniform TMEM access)
+      // this slot's PV of the previous tile has completed (its commit precedes
+      // this tile's S): O may be rescaled and P's columns rewritten
+      if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           float o[32];
-          tmem_ld32(tO + lane_off + c * 32, o);
+          tmem_ld32(tOs + lane_off + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] *= f;
-          tmem_st32(tO + lane_off + c * 32, o);
-        }
-        tmem_wait_st();
-      }
-      // last tile: value rows past the query tile's last position may be
-      // unwritten cache (their weights are 0, but 0 x NaN would not be)
-      if (kt + kTcKeys - 1 > i_max) {
-        if (!__all_sync(0xffffffffu, tc_wait(&bar_kv_full[s], (uint32_t)(j >> 1) & 1u, a, &s_abort))) {
-          ok = false;
-          break;
-        }
-        if (kt + row > i_max) {
-#pragma unroll
-          for (int rg = 0; rg < NR; ++rg) {
-            uint4* vr = reinterpret_cast<uint4*>(dsm + SM::kOffV + s * SM::kV + rg * kRegion + row * 128);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) vr[c] = make_uint4(0u, 0u, 0u, 0u);
-          }
+          tmem_st32(tOs + lane_off + c * 32, o);
         }
       }
-      // P row -> swizzled K-major layout (keys 0-63 in region 0, 64-127 in region 1)
+      const float msub = m_new == -CUDART_INF_F ? 0.f : m_new;  // all masked so far: every weight is 0
+      float lsum0 = 0.f, lsum1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < kTcKeys / 8; ++c) {
-        const int rg = c / 8, ch = c % 8;
-        uint4 v = make_uint4(pk[c * 4], pk[c * 4 + 1], pk[c * 4 + 2], pk[c * 4 + 3]);
-        *reinterpret_cast<uint4*>(dsm + SM::kOffP + rg * kRegion + row * 128 + ((ch ^ (row & 7)) * 16)) = v;
+      for (int c = 0; c < kTcKeys / 32; ++c) {
+        // P chunk c goes to columns [16 c, 16 c + 16), inside S chunks already read
+        float v[32];
+        tmem_ld32(tSs + lane_off + c * 32, v);
+        tmem_wait_ld();
+        if (!whole) apply_mask(v, c);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2f(v[2 * e] - msub);
+          const float p1 = ex2f(v[2 * e + 1] - msub);
+          lsum0 += p0;
+          lsum1 += p1;
+          pk[e] = pack_bf16(p0, p1);
+        }
+        tmem_st16(tSs + lane_off + c * 16, pk);
       }
-      fence_async_smem();
+      l = l * f + (lsum0 + lsum1);
+      tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&bar_p_full);
+      mbar_arrive(&bar_p_full[slot]);
     }
     // ---- epilogue: O / l -> out ----
-    if (ok && n > 0 && __all_sync(0xffffffffu, tc_wait(&bar_o_done, (uint32_t)((n - 1) & 1), a, &s_abort))) {
+    if (ok && n > 0 && __all_sync(0xffffffffu, tc_wait(&bar_o_done, 0u, a, &s_abort))) {
       tc_fence_after();
       __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.T + (rv ? t : 0)) * a.Hq + hq) * D;
       const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
-        tmem_ld32(tO + lane_off + c * 32, o);
+        tmem_ld32(tOs + lane_off + c * 32, o);
         tmem_wait_ld();
         if (rv) {
 #pragma unroll
@@ -496,6 +602,43 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(kTmemCols) : "memory");
   }
+}
+
+// Key tiles (128 keys) in which some row of a 256-row group keeps a token: one
+// bit per tile, the OR of the rows' top-p bitmask words (of each row only the
+// words at or below its position hold bits).
+__global__ void __launch_bounds__(256) tile_map_kernel(const __grid_constant__ TcArgs a) {
+  __shared__ uint32_t s_map[kMaxTileWords];
+  const int bh = blockIdx.y, b = bh / a.NR;
+  const int start = a.start_pos[b];
+  if (start < 0 || start + a.T > a.Lmax) return;  // uniform
+  const int t0 = a.t_base + blockIdx.x * kGroupRows;
+  const int t1 = min(a.t_end, t0 + kGroupRows);  // rows [t0, t1)
+  const int nw = (start + t1 - 1) / 32 + 1;     // words that can hold bits
+  for (int w = threadIdx.x; w < a.map_words; w += 256) s_map[w] = 0u;
+  __syncthreads();
+  const uint32_t* rows = a.mask + ((size_t)bh * a.mask_rows) * a.words;
+  for (int wb = 0; wb < nw; wb += 256) {  // uniform trip count: the shuffles below see every lane
+    const int w = wb + threadIdx.x;
+    uint32_t acc = 0u;
+    if (w < nw) {
+      for (int t = max(t0, w * 32 - start); t < t1; ++t) acc |= __ldg(rows + (size_t)(t - a.mask_t0) * a.words + w);
+    }
+    // a tile is 4 words: lanes 4k .. 4k + 3
+    acc |= __shfl_xor_sync(0xffffffffu, acc, 1);
+    acc |= __shfl_xor_sync(0xffffffffu, acc, 2);
+    const unsigned bal = __ballot_sync(0xffffffffu, acc != 0u && (threadIdx.x & 3) == 0);
+    if ((threadIdx.x & 31) == 0 && bal != 0u) {
+      uint32_t bits8 = 0u;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) bits8 |= ((bal >> (4 * k)) & 1u) << k;
+      const int tile0 = (wb + (threadIdx.x & ~31)) / 4;  // a multiple of 8
+      atomicOr(&s_map[tile0 >> 5], bits8 << (tile0 & 31));
+    }
+  }
+  __syncthreads();
+  uint32_t* dst = a.tmap_out + ((size_t)bh * a.map_groups + a.map_g0 + blockIdx.x) * a.map_words;
+  for (int w = threadIdx.x; w < a.map_words; w += 256) dst[w] = s_map[w];
 }
 
 // ---------------------------------------------------------------------------
@@ -533,11 +676,18 @@ bool make_map(CUtensorMap* tm, const void* base, int D, unsigned long long rows)
 
 }  // namespace
 
+size_t tile_map_words(const Shape& sh) { return (size_t)((sh.Lmax + kTcKeys - 1) / kTcKeys + 31) / 32; }
+size_t tile_map_bytes(const Shape& sh, int T) {
+  return (size_t)sh.B * sh.NR * (size_t)((T + kGroupRows - 1) / kGroupRows) * tile_map_words(sh) * sizeof(uint32_t);
+}
+
 // Query heads whose keys and values sit in the full-context layout go to the
-// tcgen05 kernel (all of them unless local heads keep a ring).
+// tcgen05 kernel (all of them unless local heads keep a ring).  With retrieval
+// heads, tile_map_kernel first reduces the rows' bitmask to the key tiles each
+// 256-row group keeps (t_base must be a multiple of 256).
 int launch_attn_tc(const Shape& sh, const rtp_cache* cache, const void* q_pre, const int* start_pos, int T,
                    void* out, const uint32_t* mask, int t_base, int t_end, int mask_t0, int mask_rows,
-                   unsigned long long wait_ns, cudaStream_t st) {
+                   uint32_t* tmap, unsigned long long wait_ns, cudaStream_t st) {
   TcArgs a;
   const unsigned long long rows = (unsigned long long)sh.B * (unsigned long long)sh.kv.rows_per_seq;
   if (!make_map(&a.tm_k, cache->k, sh.D, rows) || !make_map(&a.tm_v, cache->v, sh.D, rows)) {
@@ -548,11 +698,15 @@ int launch_attn_tc(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
   a.Lmax = sh.Lmax; a.S = sh.S; a.W = sh.W; a.T = T; a.words = (sh.Lmax + 31) / 32;
   a.q_pre = q_pre; a.out = out; a.status = cache->status; a.start_pos = start_pos;
   a.mask = mask; a.t_base = t_base; a.t_end = t_end; a.mask_t0 = mask_t0; a.mask_rows = mask_rows;
+  a.tmap = tmap; a.tmap_out = tmap;
+  a.map_words = (int)tile_map_words(sh);
+  a.map_groups = (T + kGroupRows - 1) / kGroupRows;
+  a.map_g0 = t_base / kGroupRows;
   a.wait_ns = wait_ns;
   a.kv = sh.kv;
   for (int i = 0; i < kMaxRetrieval; ++i) a.ret_rank[i] = sh.ret_rank[i];
   for (int i = 0; i < 64; ++i) a.inv_freq[i] = sh.inv_freq[i];
-  // heavier heads first: retrieval heads attend every causal tile
+  // retrieval heads first: they attend the most tiles
   int n = 0;
   for (int pass = 0; pass < 2; ++pass)
     for (int hq = 0; hq < sh.Hq; ++hq) {
@@ -575,7 +729,9 @@ int launch_attn_tc(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
       done[dev] = true;
     }
   }
-  const dim3 grid((t_end - t_base + kTcRows - 1) / kTcRows, sh.B * n);
+  const int n_groups = (t_end - t_base + kGroupRows - 1) / kGroupRows;
+  if (sh.R > 0) tile_map_kernel<<<dim3(n_groups, sh.B * sh.NR), 256, 0, st>>>(a);
+  const dim3 grid(n_groups, sh.B * n);
   if (sh.D == 128) attn_tc_kernel<128><<<grid, kTcThreads, TcSmem<128>::kBytes, st>>>(a);
   else attn_tc_kernel<64><<<grid, kTcThreads, TcSmem<64>::kBytes, st>>>(a);
   cudaError_t e = cudaGetLastError();

@@ -60,6 +60,21 @@ def compare_selection(scores: np.ndarray, p: float, gpu_set: np.ndarray, oracle_
     return False, len(diff)
 
 
+def kidx_bound(inp, b: int, r: int, rows) -> np.ndarray:
+    """Allowed |GPU - oracle| of stored indexer keys [len(rows), d]: the kernel
+    accumulates W_k k_pre in fp32 (D products: error at most D 2^-24 sum|w k|)
+    and rounds to the storage type, the oracle rounds the exact value; one
+    storage rounding step (2^-7 relative for bf16, 2^-23 for fp32) on top."""
+    sh = inp["shape"]
+    h = sorted(sh.retrieval)[r]
+    kp = np.abs(inp["k_pre"][b, np.asarray(rows), h].double().numpy())
+    w = np.abs(inp["w_k"][r].double().numpy())
+    acc = kp @ w.T
+    exact = np.abs(inp["k_pre"][b, np.asarray(rows), h].double().numpy() @ inp["w_k"][r].double().numpy().T)
+    rel = 2.0 ** -7 if sh.dtype == "bf16" else 2.0 ** -23
+    return sh.head_dim * 2.0 ** -24 * acc * (1 + rel) + exact * rel + 1e-30
+
+
 def oracle_cache_from_inputs(inp) -> OracleCache:
     sh = inp["shape"]
     c = OracleCache(sh, inp["max_ctx"])

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import oracle
-from parity import (TOL, bitmask_to_sets, check_decode_parity, oracle_cache_from_inputs,
+from parity import (TOL, bitmask_to_sets, check_decode_parity, kidx_bound, oracle_cache_from_inputs,
                     run_gpu_decode)
 from synth import LayerShape, make_decode_inputs, workload
 
@@ -123,7 +123,7 @@ def test_append_matches_oracle_cache():
     for r in range(sh.n_retrieval):
         kig = lay.kidx[0, r, :3000].double().cpu().numpy()
         kio = oc.indexer_keys(0, r, 3000)
-        assert np.all(np.abs(kig - kio) <= np.abs(kio) * 2.0 ** -7 + 1e-30)
+        assert np.all(np.abs(kig - kio) <= kidx_bound(inp, 0, r, np.arange(3000)))
         assert np.mean(kig == kio) > 0.999
 
 

@@ -6,7 +6,7 @@ outputs against the fp64 oracle at the same width."""
 import numpy as np
 import pytest
 
-from parity import check_decode_parity, oracle_cache_from_inputs, run_gpu_decode
+from parity import check_decode_parity, kidx_bound, oracle_cache_from_inputs, run_gpu_decode
 from synth import LayerShape, make_decode_inputs, workload
 
 pytestmark = pytest.mark.gpu
@@ -44,7 +44,7 @@ def test_append_indexer_keys_widths(d):
         kig = lay.kidx[0, r, :3001].double().cpu().numpy()
         kio = oc.indexer_keys(0, r, 3001)
         assert kig.shape == kio.shape == (3001, d)
-        assert np.all(np.abs(kig - kio) <= np.abs(kio) * 2.0 ** -7 + 1e-30)
+        assert np.all(np.abs(kig - kio) <= kidx_bound(inp, 0, r, np.arange(3001)))
         assert np.mean(kig == kio) > 0.999
 
 
