@@ -481,31 +481,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     bool ok = true;
     for (int j = 0; j < n; ++j) {
       const int kt = cur.next() * kTcKeys;
+      // a tile every row of the slot sees whole (causal, inside sinks or
+      // window) needs no mask (uniform over the slot); otherwise each row
+      // keeps keys <= its position that lie in the sinks, its window or (for
+      // retrieval heads) its top-p set: four 32-key words of keep bits, formed
+      // before the wait for S (the bitmask loads overlap it)
+      const bool whole = s_lo <= s_hi && kt + kTcKeys - 1 <= s_lo &&
+                         (kt + kTcKeys - 1 < a.S || kt >= s_hi - a.W + 1);
+      uint32_t kw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      if (!whole) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int base = kt + 32 * q;
+          const uint32_t mw = (r >= 0 && rv && base <= pi) ? __ldg(mrow + (base >> 5)) : 0u;
+          const int nc = pi - base + 1;  // keys <= pi: bits [0, nc)
+          const uint32_t causal = !rv || nc <= 0 ? 0u : nc >= 32 ? 0xffffffffu : (1u << nc) - 1u;
+          const int nsk = a.S - base;    // sinks: bits [0, nsk)
+          const uint32_t sink = nsk <= 0 ? 0u : nsk >= 32 ? 0xffffffffu : (1u << nsk) - 1u;
+          const int nw0 = wlo - base;    // window: bits [nw0, 32)
+          const uint32_t win = nw0 <= 0 ? 0xffffffffu : nw0 >= 32 ? 0u : ~((1u << nw0) - 1u);
+          kw[q] = causal & (sink | win | mw);
+        }
+      }
       // every wait's outcome is made warp-uniform: TMEM loads and stores are warp-collective
       if (!__all_sync(0xffffffffu, tc_wait(&bar_s_full[slot], (uint32_t)j & 1u, a, &s_abort))) { ok = false; break; }
       tc_fence_after();
       // S is read from TMEM twice (the row maximum, then the weights), 32
       // columns at a time, which keeps the thread's registers to a few chunks
-      const bool whole = s_lo <= s_hi && kt + kTcKeys - 1 <= s_lo &&
-                         (kt + kTcKeys - 1 < a.S || kt >= s_hi - a.W + 1);
-      // a tile every row of the slot sees whole (causal, inside sinks or
-      // window) needs no mask (uniform over the slot); otherwise causality,
-      // sinks or window, and for retrieval heads the top-p set
-      uint32_t mw[4] = {0u, 0u, 0u, 0u};
-      if (!whole && r >= 0 && rv) {
+      auto apply_mask = [&](float (&v)[32], uint32_t bits) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int wd = (kt >> 5) + q;
-          mw[q] = (wd * 32 <= pi) ? __ldg(mrow + wd) : 0u;
-        }
-      }
-      auto apply_mask = [&](float (&v)[32], int c) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int jk = kt + c * 32 + e;
-          const bool keep = rv && jk <= pi && (jk < a.S || jk >= wlo || ((mw[c] >> e) & 1u));
-          v[e] = keep ? v[e] : -CUDART_INF_F;
-        }
+        for (int e = 0; e < 32; ++e) v[e] = (bits >> e) & 1u ? v[e] : -CUDART_INF_F;
       };
       float tmax = -CUDART_INF_F;
 #pragma unroll
@@ -515,8 +520,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         tmem_ld32(tSs + lane_off + (c + 1) * 32, v1);
         tmem_wait_ld();
         if (!whole) {
-          apply_mask(v0, c);
-          apply_mask(v1, c + 1);
+          apply_mask(v0, kw[c]);
+          apply_mask(v1, kw[c + 1]);
         }
 #pragma unroll
         for (int e = 0; e < 32; e += 2) tmax = max3f(tmax, max3f(v0[e], v0[e + 1], v1[e]), v1[e + 1]);
@@ -549,7 +554,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         float v[32];
         tmem_ld32(tSs + lane_off + c * 32, v);
         tmem_wait_ld();
-        if (!whole) apply_mask(v, c);
+        if (!whole) apply_mask(v, kw[c]);
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
