@@ -15,7 +15,7 @@
 // map that tile_map_kernel reduces from the selection bitmask); never a tile
 // past the last row's position.
 //
-// Roles (320 threads):
+// Roles (576 threads):
 //   warp 0, lane 0   stages K and V tiles with TMA (cp.async.bulk.tensor,
 //                    128-byte swizzle, boxes of 64 dims x 128 keys), two
 //                    stages in flight;
@@ -23,10 +23,11 @@
 //                    commits its completions to mbarriers, in the order
 //                    S0(i), PV1(i-1), S1(i), PV0(i), so that each slot's
 //                    softmax overlaps the other slot's products;
-//   warps 2-5, 6-9   the softmax of slot 0 and slot 1 (thread = query row):
-//                    read S from TMEM, mask, keep the running maximum and
-//                    sum, write P to TMEM, rescale O in TMEM when the maximum
-//                    grows by more than 2^8, and finally write the output.
+//   warps 2-9, 10-17 the softmax of slot 0 and slot 1, two threads per query
+//                    row (each half of the tile's keys): read S from TMEM,
+//                    mask, keep the running maximum and sum, write P to TMEM,
+//                    rescale O in TMEM when the maximum grows by more than 2^8,
+//                    and finally write the output.
 // tcgen05.mma operations issued by one thread execute in issue order, so S of
 // the next tile may overwrite the TMEM columns that the previous PV read P
 // from; a commit after S(i) of a slot also tells that slot's softmax that
@@ -53,7 +54,7 @@ constexpr int kTcRows = 128;      // query rows per slot = TMEM lanes
 constexpr int kSlots = 2;
 constexpr int kGroupRows = kSlots * kTcRows;  // query rows per CTA
 constexpr int kTcKeys = 128;      // keys per tile
-constexpr int kTcThreads = 320;
+constexpr int kTcThreads = 576;  // producer warp, MMA warp, 16 softmax warps
 constexpr int kRegion = 128 * 128;  // bytes of a 128-row x 64-dim bf16 region (one TMA box)
 constexpr int kTmemCols = 512;
 constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
@@ -225,6 +226,18 @@ __device__ __forceinline__ float ex2f(float x) {
   return e;
 }
 
+// Packed fp32 pairs (one instruction for two lanes of arithmetic).
+__device__ __forceinline__ void add2(float& x, float& y, float a, float b) {  // (x, y) += (a, b)
+  asm("{\n\t.reg .b64 p, q;\n\tmov.b64 p, {%0, %1};\n\tmov.b64 q, {%2, %3};\n\t"
+      "add.rn.f32x2 p, p, q;\n\tmov.b64 {%0, %1}, p;\n\t}"
+      : "+f"(x), "+f"(y) : "f"(a), "f"(b));
+}
+__device__ __forceinline__ void mul2(float& x, float& y, float f) {  // (x, y) *= f
+  asm("{\n\t.reg .b64 p, q;\n\tmov.b64 p, {%0, %1};\n\tmov.b64 q, {%2, %2};\n\t"
+      "mul.rn.f32x2 p, p, q;\n\tmov.b64 {%0, %1}, p;\n\t}"
+      : "+f"(x), "+f"(y) : "f"(f));
+}
+
 // Walks the set bits of a shared-memory tile bitmap in increasing order.
 struct TileCursor {
   const uint32_t* bits;
@@ -257,8 +270,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
   extern __shared__ __align__(1024) unsigned char dsm_raw[];
   __shared__ __align__(8) uint64_t bar_kv_full[2], bar_kv_empty[2], bar_s_full[kSlots], bar_p_full[kSlots];
   __shared__ __align__(8) uint64_t bar_o_done, bar_fin;
+  __shared__ __align__(8) uint64_t bar_pair[kSlots][4];  // the two softmax warps of a row quarter
   __shared__ uint32_t s_tmem;
   __shared__ int s_abort, s_ntiles;
+  // the two softmax halves of a row: tile maxima by tile parity, then the sums
+  __shared__ float s_xch[kSlots][4][3 * 64];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   unsigned char* dsm = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);
   const uint32_t sQ = smem_u32(dsm + SM::kOffQ), sK = smem_u32(dsm + SM::kOffK);
@@ -283,10 +299,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       mbar_init(&bar_kv_full[s], 1);
       mbar_init(&bar_kv_empty[s], 1);
       mbar_init(&bar_s_full[s], 1);
-      mbar_init(&bar_p_full[s], kTcRows);
+      mbar_init(&bar_p_full[s], 2 * kTcRows);
     }
     mbar_init(&bar_o_done, 1);
     mbar_init(&bar_fin, 1);
+    for (int s = 0; s < kSlots; ++s)
+      for (int q = 0; q < 4; ++q) mbar_init(&bar_pair[s][q], 64);
     s_abort = 0;
     s_ntiles = 0;
   }
@@ -404,12 +422,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       }
       __syncwarp();
     };
-    auto issue_pv = [&](int slot, int st, bool acc) {  // O(slot) += P(slot) V(stage st), P in S's columns
+    auto issue_pv = [&](int slot, int st, bool acc) {  // O(slot) += P(slot) V(stage st), P in S's TMEM
       if (lane == 0) {
 #pragma unroll
         for (int kk = 0; kk < kTcKeys / 16; ++kk) {
           const uint64_t bd = umma_desc(sV + st * SM::kV + kk * 2048, kRegion, 1024);
-          umma_f16_ts(tO[slot], tS[slot] + kk * 8, bd, idO, (acc || kk > 0) ? 1u : 0u);
+          // P of keys [64 h, 64 h + 64) sits in S columns [64 h, 64 h + 32)
+          const uint32_t pa = tS[slot] + (kk >> 2) * 64 + (kk & 3) * 8;
+          umma_f16_ts(tO[slot], pa, bd, idO, (acc || kk > 0) ? 1u : 0u);
         }
       }
       __syncwarp();
@@ -462,12 +482,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     }
     __syncwarp();
   } else {
-    // ---- softmax: warps 2-5 slot 0, warps 6-9 slot 1; thread = query row ----
-    const int slot = (warp - 2) >> 2;
+    // ---- softmax: warps 2-9 slot 0, warps 10-17 slot 1.  A query row has
+    // two threads, in two warps of the same TMEM lane quarter: half h takes the
+    // keys [64 h, 64 h + 64) of each tile, writes their P over the first 32 of
+    // those S columns and rescales O's columns [h D/2, (h+1) D/2); the halves
+    // exchange their tile maxima (and at the end their sums) through shared
+    // memory under the pair's mbarrier (a bounded wait, like every other) ----
+    const int sw = warp - 2;
+    const int slot = sw >> 3, hf = (sw >> 2) & 1;
     const int quad = warp & 3;  // the TMEM lane quarter this warp may access
     const int row = quad * 32 + lane;
+    uint64_t* pbar = &bar_pair[slot][quad];  // phase j: tile j's maxima; phase n: the sums
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const uint32_t tSs = tmem + slot * kTcKeys, tOs = tmem + (2 + slot) * kTcKeys;
+    const uint32_t tSs = tmem + slot * kTcKeys + hf * 64, tOs = tmem + (2 + slot) * kTcKeys + hf * (D / 2);
     const int t = t0 + slot * kTcRows + row;
     const bool rv = t <= t_last;
     const int pi = start + t;
@@ -475,24 +502,30 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     const int s_lo = i_lo + slot * kTcRows;          // the slot's first row position
     const int s_hi = min(i_hi, s_lo + kTcRows - 1);  // its last valid row position (< s_lo: none)
     const uint32_t* mrow = a.mask + (((size_t)b * a.NR + hh) * a.mask_rows + (rv ? t - a.mask_t0 : 0)) * a.words;
+    float* xch = s_xch[slot][quad];                  // [2 tile parities][2 halves][32 lanes]
     TileCursor cur;
     cur.init(s_tiles, n_words);
     float m_used = -CUDART_INF_F, l = 0.f;
     bool ok = true;
+    auto apply_mask = [&](float (&v)[32], uint32_t bits) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = (bits >> e) & 1u ? v[e] : -CUDART_INF_F;
+    };
     for (int j = 0; j < n; ++j) {
       const int kt = cur.next() * kTcKeys;
+      const int k0 = kt + hf * 64;  // this half's first key
       // a tile every row of the slot sees whole (causal, inside sinks or
       // window) needs no mask (uniform over the slot); otherwise each row
       // keeps keys <= its position that lie in the sinks, its window or (for
-      // retrieval heads) its top-p set: four 32-key words of keep bits, formed
+      // retrieval heads) its top-p set: 32-key words of keep bits, formed
       // before the wait for S (the bitmask loads overlap it)
       const bool whole = s_lo <= s_hi && kt + kTcKeys - 1 <= s_lo &&
                          (kt + kTcKeys - 1 < a.S || kt >= s_hi - a.W + 1);
-      uint32_t kw[4] = {0xffffffffu, 0xffffffffu, 0xffffffffu, 0xffffffffu};
+      uint32_t kw[2] = {0xffffffffu, 0xffffffffu};
       if (!whole) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int base = kt + 32 * q;
+        for (int q = 0; q < 2; ++q) {
+          const int base = k0 + 32 * q;
           const uint32_t mw = (r >= 0 && rv && base <= pi) ? __ldg(mrow + (base >> 5)) : 0u;
           const int nc = pi - base + 1;  // keys <= pi: bits [0, nc)
           const uint32_t causal = !rv || nc <= 0 ? 0u : nc >= 32 ? 0xffffffffu : (1u << nc) - 1u;
@@ -506,51 +539,50 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       // every wait's outcome is made warp-uniform: TMEM loads and stores are warp-collective
       if (!__all_sync(0xffffffffu, tc_wait(&bar_s_full[slot], (uint32_t)j & 1u, a, &s_abort))) { ok = false; break; }
       tc_fence_after();
-      // S is read from TMEM twice (the row maximum, then the weights), 32
-      // columns at a time, which keeps the thread's registers to a few chunks
-      auto apply_mask = [&](float (&v)[32], uint32_t bits) {
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = (bits >> e) & 1u ? v[e] : -CUDART_INF_F;
-      };
-      float tmax = -CUDART_INF_F;
-#pragma unroll
-      for (int c = 0; c < kTcKeys / 32; c += 2) {
+      // S is read from TMEM twice (the row maximum, then the weights)
+      float hmax = -CUDART_INF_F;
+      {
         float v0[32], v1[32];
-        tmem_ld32(tSs + lane_off + c * 32, v0);
-        tmem_ld32(tSs + lane_off + (c + 1) * 32, v1);
+        tmem_ld32(tSs + lane_off, v0);
+        tmem_ld32(tSs + lane_off + 32, v1);
         tmem_wait_ld();
         if (!whole) {
-          apply_mask(v0, kw[c]);
-          apply_mask(v1, kw[c + 1]);
+          apply_mask(v0, kw[0]);
+          apply_mask(v1, kw[1]);
         }
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) tmax = max3f(tmax, max3f(v0[e], v0[e + 1], v1[e]), v1[e + 1]);
+        for (int e = 0; e < 32; e += 2) hmax = max3f(hmax, max3f(v0[e], v0[e + 1], v1[e]), v1[e + 1]);
       }
+      float* xm = xch + (j & 1) * 64;
+      xm[hf * 32 + lane] = hmax;
+      mbar_arrive(pbar);  // release: the partner's wait makes xm visible
+      if (!__all_sync(0xffffffffu, tc_wait(pbar, (uint32_t)j & 1u, a, &s_abort))) { ok = false; break; }
+      const float tmax = fmaxf(hmax, xm[(hf ^ 1) * 32 + lane]);
       // lazy rescale: the maximum used moves only when the tile's exceeds it by > 2^8
       float m_new = m_used, f = 1.f;
       if (tmax > m_used + kRescale || (m_used == -CUDART_INF_F && tmax != -CUDART_INF_F)) {
         m_new = tmax;
         f = (m_used == -CUDART_INF_F) ? 0.f : ex2f(m_used - m_new);
       }
-      m_used = m_new;
       // this slot's PV of the previous tile has completed (its commit precedes
       // this tile's S): O may be rescaled and P's columns rewritten
       if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           float o[32];
           tmem_ld32(tOs + lane_off + c * 32, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] *= f;
+          for (int e = 0; e < 32; e += 2) mul2(o[e], o[e + 1], f);
           tmem_st32(tOs + lane_off + c * 32, o);
         }
       }
       const float msub = m_new == -CUDART_INF_F ? 0.f : m_new;  // all masked so far: every weight is 0
       float lsum0 = 0.f, lsum1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < kTcKeys / 32; ++c) {
-        // P chunk c goes to columns [16 c, 16 c + 16), inside S chunks already read
+      for (int c = 0; c < 2; ++c) {
+        // P of keys [k0 + 32 c, +32) goes to columns [16 c, 16 c + 16) of this
+        // half, inside its first S chunk, already read
         float v[32];
         tmem_ld32(tSs + lane_off + c * 32, v);
         tmem_wait_ld();
@@ -558,30 +590,37 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2f(v[2 * e] - msub);
-          const float p1 = ex2f(v[2 * e + 1] - msub);
-          lsum0 += p0;
-          lsum1 += p1;
+          float x0 = v[2 * e], x1 = v[2 * e + 1];
+          add2(x0, x1, -msub, -msub);
+          const float p0 = ex2f(x0), p1 = ex2f(x1);
+          add2(lsum0, lsum1, p0, p1);
           pk[e] = pack_bf16(p0, p1);
         }
         tmem_st16(tSs + lane_off + c * 16, pk);
       }
+      m_used = m_new;
       l = l * f + (lsum0 + lsum1);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&bar_p_full[slot]);
     }
-    // ---- epilogue: O / l -> out ----
+    // ---- epilogue: O / l -> out, each half its D/2 columns ----
     if (ok && n > 0 && __all_sync(0xffffffffu, tc_wait(&bar_o_done, 0u, a, &s_abort))) {
       tc_fence_after();
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.T + (rv ? t : 0)) * a.Hq + hq) * D;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      float* xl = xch + 128;
+      xl[hf * 32 + lane] = l;
+      mbar_arrive(pbar);
+      const bool got = __all_sync(0xffffffffu, tc_wait(pbar, (uint32_t)n & 1u, a, &s_abort));
+      const float lt = got ? l + xl[(hf ^ 1) * 32 + lane] : 0.f;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(a.out) + (((size_t)b * a.T + (rv ? t : 0)) * a.Hq + hq) * D +
+                            hf * (D / 2);
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / 64; ++c) {
         float o[32];
         tmem_ld32(tOs + lane_off + c * 32, o);
         tmem_wait_ld();
-        if (rv) {
+        if (rv && got) {
 #pragma unroll
           for (int e = 0; e < 32; e += 8) {
             uint4 v;
