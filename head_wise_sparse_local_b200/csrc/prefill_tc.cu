@@ -238,6 +238,23 @@ __device__ __forceinline__ void mul2(float& x, float& y, float f) {  // (x, y) *
       : "+f"(x), "+f"(y) : "f"(f));
 }
 
+// 2^x on the FMA pipe, for a share of the softmax weights, so that the MUFU
+// pipe (ex2f) does not bound the softmax.  Cody-Waite split x = j + f with
+// j = round(x) (by adding 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f by a cubic
+// fitted to it in relative error on that interval (Chebyshev-node least
+// squares reweighted toward equal ripple: maximum relative error 7.5e-5,
+// far below a bf16 weight's rounding); 2^j added to the exponent field.
+// Inputs below -125 are taken as -125 (a weight of about 2^-125).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -125.f);
+  const float t = x + 12582912.f;  // round(x) in the low mantissa bits of t
+  const float f = x - (t - 12582912.f);
+  float p = fmaf(0.05517161f, f, 0.24261111f);
+  p = fmaf(p, f, 0.69326097f);
+  p = fmaf(p, f, 0.99992806f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 // Walks the set bits of a shared-memory tile bitmap in increasing order.
 struct TileCursor {
   const uint32_t* bits;
@@ -511,47 +528,77 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
 #pragma unroll
       for (int e = 0; e < 32; ++e) v[e] = (bits >> e) & 1u ? v[e] : -CUDART_INF_F;
     };
+    // a tile every row of the slot sees whole (causal, inside sinks or window)
+    // needs no mask (uniform over the slot)
+    auto is_whole = [&](int kt) {
+      return s_lo <= s_hi && kt + kTcKeys - 1 <= s_lo && (kt + kTcKeys - 1 < a.S || kt >= s_hi - a.W + 1);
+    };
+    // this row's top-p bitmask words of a tile's half (retrieval heads), loaded
+    // one tile ahead of their use
+    auto load_mw = [&](int kt, uint32_t (&mw)[2]) {
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int base = kt + hf * 64 + 32 * q;
+        mw[q] = (r >= 0 && rv && kt >= 0 && base <= pi && !is_whole(kt)) ? __ldg(mrow + (base >> 5)) : 0u;
+      }
+    };
+    int kt_next = n > 0 ? cur.next() * kTcKeys : -1;
+    uint32_t mw_next[2];
+    load_mw(kt_next, mw_next);
     for (int j = 0; j < n; ++j) {
-      const int kt = cur.next() * kTcKeys;
+      const int kt = kt_next;
+      const uint32_t mw[2] = {mw_next[0], mw_next[1]};
+      kt_next = j + 1 < n ? cur.next() * kTcKeys : -1;
+      load_mw(kt_next, mw_next);
       const int k0 = kt + hf * 64;  // this half's first key
-      // a tile every row of the slot sees whole (causal, inside sinks or
-      // window) needs no mask (uniform over the slot); otherwise each row
-      // keeps keys <= its position that lie in the sinks, its window or (for
-      // retrieval heads) its top-p set: 32-key words of keep bits, formed
-      // before the wait for S (the bitmask loads overlap it)
-      const bool whole = s_lo <= s_hi && kt + kTcKeys - 1 <= s_lo &&
-                         (kt + kTcKeys - 1 < a.S || kt >= s_hi - a.W + 1);
+      // otherwise each row keeps keys <= its position that lie in the sinks,
+      // its window or (retrieval heads) its top-p set: 32-key words of keep bits
+      const bool whole = is_whole(kt);
       uint32_t kw[2] = {0xffffffffu, 0xffffffffu};
+      bool full[2] = {true, true};  // the chunk is kept whole by every row of the warp
       if (!whole) {
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
           const int base = k0 + 32 * q;
-          const uint32_t mw = (r >= 0 && rv && base <= pi) ? __ldg(mrow + (base >> 5)) : 0u;
           const int nc = pi - base + 1;  // keys <= pi: bits [0, nc)
           const uint32_t causal = !rv || nc <= 0 ? 0u : nc >= 32 ? 0xffffffffu : (1u << nc) - 1u;
           const int nsk = a.S - base;    // sinks: bits [0, nsk)
           const uint32_t sink = nsk <= 0 ? 0u : nsk >= 32 ? 0xffffffffu : (1u << nsk) - 1u;
           const int nw0 = wlo - base;    // window: bits [nw0, 32)
           const uint32_t win = nw0 <= 0 ? 0xffffffffu : nw0 >= 32 ? 0u : ~((1u << nw0) - 1u);
-          kw[q] = causal & (sink | win | mw);
+          kw[q] = causal & (sink | win | mw[q]);
+          full[q] = __all_sync(0xffffffffu, kw[q] == 0xffffffffu);
         }
       }
       // every wait's outcome is made warp-uniform: TMEM loads and stores are warp-collective
       if (!__all_sync(0xffffffffu, tc_wait(&bar_s_full[slot], (uint32_t)j & 1u, a, &s_abort))) { ok = false; break; }
       tc_fence_after();
-      // S is read from TMEM twice (the row maximum, then the weights)
-      float hmax = -CUDART_INF_F;
-      {
-        float v0[32], v1[32];
-        tmem_ld32(tSs + lane_off, v0);
-        tmem_ld32(tSs + lane_off + 32, v1);
-        tmem_wait_ld();
-        if (!whole) {
-          apply_mask(v0, kw[0]);
-          apply_mask(v1, kw[1]);
-        }
+      // One read of S: the half-row's maximum and, against the row's running
+      // maximum m_used, its weights (P held in registers).  The halves then
+      // exchange their maxima; a row with no maximum yet, or whose tile
+      // maximum exceeds m_used by more than 2^8 (the lazy rescale threshold),
+      // makes its warps (the same rows in both halves) recompute P against
+      // the new maximum from S, which is still intact.
+      const bool have_m = m_used != -CUDART_INF_F;
+      const float mspec = have_m ? m_used : 0.f;  // a row with no maximum yet keeps only 0 weights here
+      float hmax = -CUDART_INF_F, lsum0 = 0.f, lsum1 = 0.f;
+      uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) hmax = max3f(hmax, max3f(v0[e], v0[e + 1], v1[e]), v1[e + 1]);
+      for (int c = 0; c < 2; ++c) {
+        float v[32];
+        tmem_ld32(tSs + lane_off + c * 32, v);
+        tmem_wait_ld();
+        if (!full[c]) apply_mask(v, kw[c]);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          float x0 = v[2 * e], x1 = v[2 * e + 1];
+          hmax = max3f(hmax, x0, x1);
+          add2(x0, x1, -mspec, -mspec);
+          // one weight in four on the FMA pipe, the rest on MUFU
+          const float p0 = ex2f(x0), p1 = (e & 1) ? ex2_poly(x1) : ex2f(x1);
+          add2(lsum0, lsum1, p0, p1);
+          pk[c * 16 + e] = pack_bf16(p0, p1);
+        }
       }
       float* xm = xch + (j & 1) * 64;
       xm[hf * 32 + lane] = hmax;
@@ -560,43 +607,50 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       const float tmax = fmaxf(hmax, xm[(hf ^ 1) * 32 + lane]);
       // lazy rescale: the maximum used moves only when the tile's exceeds it by > 2^8
       float m_new = m_used, f = 1.f;
-      if (tmax > m_used + kRescale || (m_used == -CUDART_INF_F && tmax != -CUDART_INF_F)) {
+      if (tmax > m_used + kRescale || (!have_m && tmax != -CUDART_INF_F)) {
         m_new = tmax;
-        f = (m_used == -CUDART_INF_F) ? 0.f : ex2f(m_used - m_new);
+        f = have_m ? ex2f(m_used - m_new) : 0.f;
       }
-      // this slot's PV of the previous tile has completed (its commit precedes
-      // this tile's S): O may be rescaled and P's columns rewritten
-      if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
+      if (!__any_sync(0xffffffffu, m_new != m_used)) {
+        // P of keys [k0 + 32 c, +32) to columns [16 c, 16 c + 16)
+        tmem_st16(tSs + lane_off, *reinterpret_cast<const uint32_t(*)[16]>(&pk[0]));
+        tmem_st16(tSs + lane_off + 16, *reinterpret_cast<const uint32_t(*)[16]>(&pk[16]));
+      } else {
+        // this slot's PV of the previous tile has completed (its commit precedes
+        // this tile's S): O may be rescaled and P's columns written
+        if (j > 0 && __any_sync(0xffffffffu, f != 1.f)) {
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
-          float o[32];
-          tmem_ld32(tOs + lane_off + c * 32, o);
+          for (int c = 0; c < D / 64; ++c) {
+            float o[32];
+            tmem_ld32(tOs + lane_off + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) mul2(o[e], o[e + 1], f);
+            tmem_st32(tOs + lane_off + c * 32, o);
+          }
+        }
+        const float msub = m_new == -CUDART_INF_F ? 0.f : m_new;  // all masked so far: every weight is 0
+        lsum0 = 0.f;
+        lsum1 = 0.f;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          // P of keys [k0 + 32 c, +32) goes to columns [16 c, 16 c + 16) of this
+          // half, inside its first S chunk, already read
+          float v[32];
+          tmem_ld32(tSs + lane_off + c * 32, v);
           tmem_wait_ld();
+          if (!full[c]) apply_mask(v, kw[c]);
+          uint32_t q16[16];
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) mul2(o[e], o[e + 1], f);
-          tmem_st32(tOs + lane_off + c * 32, o);
+          for (int e = 0; e < 16; ++e) {
+            float x0 = v[2 * e], x1 = v[2 * e + 1];
+            add2(x0, x1, -msub, -msub);
+            const float p0 = ex2f(x0), p1 = (e & 1) ? ex2_poly(x1) : ex2f(x1);
+            add2(lsum0, lsum1, p0, p1);
+            q16[e] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tSs + lane_off + c * 16, q16);
         }
-      }
-      const float msub = m_new == -CUDART_INF_F ? 0.f : m_new;  // all masked so far: every weight is 0
-      float lsum0 = 0.f, lsum1 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        // P of keys [k0 + 32 c, +32) goes to columns [16 c, 16 c + 16) of this
-        // half, inside its first S chunk, already read
-        float v[32];
-        tmem_ld32(tSs + lane_off + c * 32, v);
-        tmem_wait_ld();
-        if (!whole) apply_mask(v, kw[c]);
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float x0 = v[2 * e], x1 = v[2 * e + 1];
-          add2(x0, x1, -msub, -msub);
-          const float p0 = ex2f(x0), p1 = ex2f(x1);
-          add2(lsum0, lsum1, p0, p1);
-          pk[e] = pack_bf16(p0, p1);
-        }
-        tmem_st16(tSs + lane_off + c * 16, pk);
       }
       m_used = m_new;
       l = l * f + (lsum0 + lsum1);
