@@ -285,7 +285,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
   using SM = TcSmem<D>;
   constexpr int NRG = D / 64;  // 64-dim regions
   extern __shared__ __align__(1024) unsigned char dsm_raw[];
-  __shared__ __align__(8) uint64_t bar_kv_full[2], bar_kv_empty[2], bar_s_full[kSlots], bar_p_full[kSlots];
+  __shared__ __align__(8) uint64_t bar_k_full[2], bar_k_empty[2], bar_v_full[2], bar_v_empty[2];
+  __shared__ __align__(8) uint64_t bar_s_full[kSlots], bar_p_full[kSlots];
   __shared__ __align__(8) uint64_t bar_o_done, bar_fin;
   __shared__ __align__(8) uint64_t bar_pair[kSlots][4];  // the two softmax warps of a row quarter
   __shared__ uint32_t s_tmem;
@@ -313,8 +314,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
 
   if (tid == 0) {
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bar_kv_full[s], 1);
-      mbar_init(&bar_kv_empty[s], 1);
+      mbar_init(&bar_k_full[s], 1);
+      mbar_init(&bar_k_empty[s], 1);
+      mbar_init(&bar_v_full[s], 1);
+      mbar_init(&bar_v_empty[s], 1);
       mbar_init(&bar_s_full[s], 1);
       mbar_init(&bar_p_full[s], 2 * kTcRows);
     }
@@ -401,7 +404,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---- producer: K and V tiles by TMA ----
+      // ---- producer: K and V tiles by TMA, each as soon as its stage is
+      // free (a K stage frees after the tile's two S products, a V stage after
+      // its two PV products) ----
       const uint64_t pol = l2_evict_last();
       const size_t rowbase = a.kv.row(b, h, 0);  // full-cache head: position p at rowbase + p
       TileCursor cur;
@@ -409,14 +414,18 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
       for (int i = 0; i < n; ++i) {
         const int kt = cur.next() * kTcKeys;
         const int st = i & 1;
-        if (!tc_wait(&bar_kv_empty[st], ((uint32_t)(i >> 1) & 1u) ^ 1u, a, &s_abort)) break;
-        mbar_expect_tx(&bar_kv_full[st], (uint32_t)(2 * NRG * kRegion));
+        const uint32_t par = ((uint32_t)(i >> 1) & 1u) ^ 1u;
         const int y = (int)(rowbase + kt);
+        if (!tc_wait(&bar_k_empty[st], par, a, &s_abort)) break;
+        mbar_expect_tx(&bar_k_full[st], (uint32_t)(NRG * kRegion));
 #pragma unroll
-        for (int rg = 0; rg < NRG; ++rg) {
-          tma_load_2d(dsm + SM::kOffK + st * SM::kK + rg * kRegion, &a.tm_k, rg * 64, y, &bar_kv_full[st], pol);
-          tma_load_2d(dsm + SM::kOffV + st * SM::kV + rg * kRegion, &a.tm_v, rg * 64, y, &bar_kv_full[st], pol);
-        }
+        for (int rg = 0; rg < NRG; ++rg)
+          tma_load_2d(dsm + SM::kOffK + st * SM::kK + rg * kRegion, &a.tm_k, rg * 64, y, &bar_k_full[st], pol);
+        if (!tc_wait(&bar_v_empty[st], par, a, &s_abort)) break;
+        mbar_expect_tx(&bar_v_full[st], (uint32_t)(NRG * kRegion));
+#pragma unroll
+        for (int rg = 0; rg < NRG; ++rg)
+          tma_load_2d(dsm + SM::kOffV + st * SM::kV + rg * kRegion, &a.tm_v, rg * 64, y, &bar_v_full[st], pol);
       }
     }
   } else if (warp == 1) {
@@ -426,14 +435,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     constexpr uint32_t idO = umma_idesc(kTcRows, D, true);
     const uint32_t tS[2] = {tmem, tmem + kTcKeys};
     const uint32_t tO[2] = {tmem + 2 * kTcKeys, tmem + 3 * kTcKeys};
+    // Descriptors: one base per operand, the k-step's offset added to the
+    // address field (start address / 16 in the low 14 bits; shared memory is
+    // below 256 KB, so the field never carries into the next)
+    const uint64_t dq0 = umma_desc(sQ, 16, 1024), dk0 = umma_desc(sK, 16, 1024);
+    const uint64_t dv0 = umma_desc(sV, kRegion, 1024);
     auto issue_s = [&](int slot, int st) {  // S(slot) = Q(slot) K(stage st)^T
       if (lane == 0) {
+        const uint64_t dq = dq0 + (uint64_t)((slot * SM::kQ) >> 4);
+        const uint64_t dk = dk0 + (uint64_t)((st * SM::kK) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const int rg = kk / 4, ko = (kk % 4) * 32;
-          const uint64_t ad = umma_desc(sQ + slot * SM::kQ + rg * kRegion + ko, 16, 1024);
-          const uint64_t bd = umma_desc(sK + st * SM::kK + rg * kRegion + ko, 16, 1024);
-          umma_f16(tS[slot], ad, bd, idS, kk > 0 ? 1u : 0u);
+          const uint32_t off = (uint32_t)(((kk / 4) * kRegion + (kk % 4) * 32) >> 4);
+          umma_f16(tS[slot], dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
         }
         umma_commit(&bar_s_full[slot]);
       }
@@ -441,12 +455,12 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     };
     auto issue_pv = [&](int slot, int st, bool acc) {  // O(slot) += P(slot) V(stage st), P in S's TMEM
       if (lane == 0) {
+        const uint64_t dv = dv0 + (uint64_t)((st * SM::kV) >> 4);
 #pragma unroll
         for (int kk = 0; kk < kTcKeys / 16; ++kk) {
-          const uint64_t bd = umma_desc(sV + st * SM::kV + kk * 2048, kRegion, 1024);
           // P of keys [64 h, 64 h + 64) sits in S columns [64 h, 64 h + 32)
           const uint32_t pa = tS[slot] + (kk >> 2) * 64 + (kk & 3) * 8;
-          umma_f16_ts(tO[slot], pa, bd, idO, (acc || kk > 0) ? 1u : 0u);
+          umma_f16_ts(tO[slot], pa, dv + (uint64_t)((kk * 2048) >> 4), idO, (acc || kk > 0) ? 1u : 0u);
         }
       }
       __syncwarp();
@@ -457,7 +471,19 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
     for (int i = 0; i < n; ++i) {
       const int kt = cur.next() * kTcKeys;
       const int st = i & 1;
-      if (!__all_sync(0xffffffffu, tc_wait(&bar_kv_full[st], (uint32_t)(i >> 1) & 1u, a, &s_abort))) { ok = false; break; }
+      const uint32_t par = (uint32_t)(i >> 1) & 1u;
+      if (!__all_sync(0xffffffffu, tc_wait(&bar_k_full[st], par, a, &s_abort))) { ok = false; break; }
+      tc_fence_after();
+      issue_s(0, st);
+      if (i > 0) {
+        if (!__all_sync(0xffffffffu, tc_wait(&bar_p_full[1], (uint32_t)(i - 1) & 1u, a, &s_abort))) { ok = false; break; }
+        tc_fence_after();
+        issue_pv(1, st ^ 1, i > 1);
+        if (lane == 0) umma_commit(&bar_v_empty[st ^ 1]);
+      }
+      issue_s(1, st);
+      if (lane == 0) umma_commit(&bar_k_empty[st]);
+      if (!__all_sync(0xffffffffu, tc_wait(&bar_v_full[st], par, a, &s_abort))) { ok = false; break; }
       if (kt + kTcKeys - 1 > i_hi) {
         // value rows past the CTA's last position may be unwritten cache (their
         // weights are 0, but 0 x NaN would not be)
@@ -472,15 +498,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         fence_async_smem();
         __syncwarp();
       }
-      tc_fence_after();
-      issue_s(0, st);
-      if (i > 0) {
-        if (!__all_sync(0xffffffffu, tc_wait(&bar_p_full[1], (uint32_t)(i - 1) & 1u, a, &s_abort))) { ok = false; break; }
-        tc_fence_after();
-        issue_pv(1, st ^ 1, i > 1);
-        if (lane == 0) umma_commit(&bar_kv_empty[st ^ 1]);
-      }
-      issue_s(1, st);
       if (!__all_sync(0xffffffffu, tc_wait(&bar_p_full[0], (uint32_t)i & 1u, a, &s_abort))) { ok = false; break; }
       tc_fence_after();
       issue_pv(0, st, i > 0);
@@ -489,7 +506,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
         __all_sync(0xffffffffu, tc_wait(&bar_p_full[1], (uint32_t)(n - 1) & 1u, a, &s_abort))) {
       tc_fence_after();
       issue_pv(1, (n - 1) & 1, n > 1);
-      if (lane == 0) umma_commit(&bar_kv_empty[(n - 1) & 1]);
+      if (lane == 0) umma_commit(&bar_v_empty[(n - 1) & 1]);
     }
     if (lane == 0) {
       umma_commit(&bar_o_done);
@@ -692,8 +709,10 @@ __global__ void __launch_bounds__(kTcThreads, 1) attn_tc_kernel(const __grid_con
   __syncthreads();
   if (s_abort && warp == 0 && lane == 0) {
     // copies still in flight after an abort: wait for them (bounded) before leaving
-    mbar_wait_bounded(&bar_kv_full[0], 0u, a.wait_ns, a.status);
-    mbar_wait_bounded(&bar_kv_full[1], 0u, a.wait_ns, a.status);
+    for (int s = 0; s < 2; ++s) {
+      mbar_wait_bounded(&bar_k_full[s], 0u, a.wait_ns, a.status);
+      mbar_wait_bounded(&bar_v_full[s], 0u, a.wait_ns, a.status);
+    }
   }
   __syncthreads();
   if (warp == 1) {
