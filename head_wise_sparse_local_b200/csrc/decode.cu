@@ -6,8 +6,9 @@
 // into shared memory with bulk asynchronous copies (TMA) that complete on an
 // mbarrier:
 //
-//   score_kernel   a chunk of the 16-d indexer-key cache (contiguous rows) per
-//                  CTA; the fp32 scores s_j = q~ . k~_j / 4 of the G query
+//   score_kernel   a chunk of the d-dim indexer-key cache (contiguous rows)
+//                  per CTA (d = 16, or 4, 8, 32 for the dimension ablation);
+//                  the fp32 scores s_j = q~ . k~_j / sqrt(d) of the G query
 //                  heads of a retrieval KV head are formed on tensor cores
 //                  (q~ as bf16 high and low parts, as in the prefill) and
 //                  written with a per-chunk maximum.
@@ -33,14 +34,18 @@
 //                  top-p bitmask and attends, for its query head, the kept
 //                  rows of its share that lie outside the sinks and the
 //                  window.  The cluster merges its partials with the head's
-//                  sink/window partial and writes the output.
+//                  sink/window partial and writes the output.  Static top-k
+//                  (the pages' fixed-budget baseline) runs the same solver
+//                  with every token weighing 1 and the target k.
 //
 // Every in-kernel wait is either a hardware barrier reached uniformly or a
 // bounded wait on a copy barrier (RTP_DEV_TIMEOUT when it gives up).
 //
 // Top-p follows the abstract's observation (3) and the atlas.scime.ai summary
 // ("query-adaptive top-p threshold"); sinks + window follow that summary's
-// "Approach"; the 16-d pre-RoPE indexer follows observation (2).
+// "Approach"; the 16-d pre-RoPE indexer follows observation (2), the other
+// widths the summary's "Surprising findings" (dimension 4); static top-k its
+// "Baselines".
 #include <algorithm>
 #include <atomic>
 #include <climits>

@@ -54,7 +54,7 @@ typedef enum rtp_status {
 /* Device-side status bits OR-ed into *cache->status. */
 #define RTP_DEV_SEQ_LEN  0x1  /* decode: seq_len[b] < 1 or > max_seq_len; sequence b skipped */
 #define RTP_DEV_POSITION 0x2  /* append/prefill: a position outside [0, max_ctx); rows skipped */
-#define RTP_DEV_TIMEOUT  0x4  /* decode: a bounded in-kernel wait gave up; that call's output is invalid */
+#define RTP_DEV_TIMEOUT  0x4  /* decode or prefill: a bounded in-kernel wait gave up; that call's output is invalid */
 
 typedef enum rtp_dtype { RTP_BF16 = 0, RTP_FP32 = 1 } rtp_dtype;
 
