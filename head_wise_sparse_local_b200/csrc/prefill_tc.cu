@@ -185,7 +185,7 @@ __device__ __forceinline__ uint64_t l2_evict_last() {
 __device__ __forceinline__ bool tc_wait(uint64_t* bar, uint32_t parity, const TcArgs& a, volatile int* s_abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_sleep(bar, parity, kWaitHintNs)) {
     if (*s_abort) return false;
     if (global_ns() - t0 > a.wait_ns) {
       *s_abort = 1;

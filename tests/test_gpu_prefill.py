@@ -148,3 +148,45 @@ def test_prefill_refuses_static_topk():
         lay.prefill(q, torch.zeros(1, dtype=torch.int32, device="cuda"),
                     torch.zeros((2, 16, sh.head_dim), device="cuda"), torch.empty_like(q))
     assert e.value.code == 2 and "top-k" in str(e.value)
+
+
+def test_prefill_row_blocks_equal_one_block():
+    """A chunk whose per-row bitmask would pass the workspace budget runs in
+    blocks of rows: at a 1M-token capacity a row's bitmask over 8 retrieval q
+    heads is 1 MiB, so a 2304-row chunk without a caller bitmask runs as blocks
+    of 1024, 1024 and 256 rows (selection, tile map and attention per block).
+    Its outputs, counts, thresholds and cut indices equal the one-block run's
+    (the caller's bitmask holds every row) bit for bit, and the one-block run
+    matches the oracle on rows at the block edges."""
+    from head_wise_sparse_local_b200 import Layer
+    inp = _inp(T=2304, n_sink=16, window=256, top_p=0.9, needles=16)
+    sh, T = inp["shape"], inp["T"]
+    Lmax = 1 << 20
+    dev = torch.device("cuda")
+    lay = Layer(sh, Lmax, device=dev, prefill_T=T)
+    zero = torch.zeros(sh.batch, dtype=torch.int32, device=dev)
+    lay.append(inp["k_pre"][:, :T].contiguous().to(dev), inp["v"][:, :T].contiguous().to(dev), zero,
+               inp["w_k"].to(dev))
+    q, w_q = inp["q_pre"].to(dev), inp["w_q"].to(dev)
+    NR = sh.n_retrieval * sh.group
+    runs = []
+    for with_bm in (True, False):
+        out = torch.empty((sh.batch, T, sh.n_q_heads, sh.head_dim), dtype=sh.torch_dtype, device=dev)
+        bm = torch.zeros((sh.batch, NR, T, Lmax // 32), dtype=torch.int32, device=dev) if with_bm else None
+        cnt = torch.full((sh.batch, NR, T), -1, dtype=torch.int32, device=dev)
+        tau = torch.zeros((sh.batch, NR, T), dtype=torch.float32, device=dev)
+        jcut = torch.zeros((sh.batch, NR, T), dtype=torch.int32, device=dev)
+        lay.prefill(q, zero, w_q, out, sel_bitmask=bm, sel_tau=tau, sel_jcut=jcut, sel_count=cnt)
+        torch.cuda.synchronize()
+        runs.append(dict(out=out, bitmask=bm, count=cnt.cpu().numpy(), tau=tau.cpu().numpy(),
+                         jcut=jcut.cpu().numpy()))
+        del bm
+    assert lay.device_status() == 0
+    one, blocks = runs
+    assert torch.equal(one["out"], blocks["out"])
+    assert np.array_equal(one["count"], blocks["count"])
+    assert np.array_equal(one["tau"], blocks["tau"])
+    assert np.array_equal(one["jcut"], blocks["jcut"])
+    g = dict(out=one["out"].double().cpu().numpy(), bitmask=one["bitmask"], count=one["count"], status=0)
+    st = check_prefill_parity(inp, rows=[0, 1, 1023, 1024, 1025, 2047, 2048, 2303], g=g)
+    assert st["exact"] >= st["heads"] - 2
