@@ -22,6 +22,7 @@
 //       causality, sinks, the window and (retrieval heads) the bitmask; key
 //       tiles holding nothing a row keeps are skipped.
 #include <climits>
+#include <mutex>
 
 #include "common.cuh"
 #include "internal.h"
@@ -994,9 +995,13 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
   for (int i = 0; i < kMaxRetrieval; ++i) { a.ret_head[i] = sh.ret_head[i]; a.ret_rank[i] = sh.ret_rank[i]; }
   for (int i = 0; i < 64; ++i) a.inv_freq[i] = sh.inv_freq[i];
 
+  // per-device kernel attributes, set once under a mutex (calls may come from
+  // several host threads)
+  static std::mutex s_mu;
   static bool s_attr[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(s_mu);
   if (dev >= 0 && dev < 64 && !s_attr[dev]) {
     cudaFuncSetAttribute(attn_rows_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)AttnSmem<128>::kBytes);
