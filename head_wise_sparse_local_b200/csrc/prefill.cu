@@ -33,13 +33,17 @@ namespace {
 constexpr int kSelRows = 8;       // query rows (warps) per selection CTA
 constexpr int kKeyTile = 512;     // indexer keys staged per step
 constexpr int kKeyStages = 2;     // key tiles in flight: the one in use and one ahead
-constexpr size_t kSelDynSmem = kKeyStages * kKeyTile * kIdxDim * sizeof(__nv_bfloat16) + kSelRows * (kKeyTile + 4) * sizeof(float);
+// dynamic shared memory of the selection at indexer width d: the key-tile ring and one tile's scores of the rows
+constexpr size_t sel_dyn_smem(int idx) {
+  return (size_t)kKeyStages * kKeyTile * idx * sizeof(__nv_bfloat16) + kSelRows * (kKeyTile + 4) * sizeof(float);
+}
 constexpr int kCand = 160;        // tokens the exact solve takes per row
 constexpr int kBQ = 64;           // attention: query rows per CTA (16 per warp)
 constexpr int kBK = 64;           // attention: keys per tile
 
 struct PrefillArgs {
   int B, Hq, Hkv, G, D, R, NR, Lmax, S, W, T, words;
+  int Lk;  // indexer-key rows per (sequence, retrieval head) block
   float top_p, rope_base;
   const void* q_pre;
   const float* w_q;
@@ -170,14 +174,15 @@ __device__ __forceinline__ void split_item(const SplitView& v, float sv, unsigne
   }
 }
 
-template <int D>
+template <int D, int IDX>
 __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __grid_constant__ PrefillArgs a) {
+  constexpr int KB = IDX * (int)sizeof(__nv_bfloat16);  // bytes per indexer key
   // dynamic shared memory: a ring of key tiles, then this tile's scores of
   // the CTA's rows
   extern __shared__ __align__(16) unsigned char sel_dsm[];
-  auto s_k = reinterpret_cast<__nv_bfloat16 (*)[kKeyTile * kIdxDim]>(sel_dsm);
-  auto s_sc = reinterpret_cast<float (*)[kKeyTile + 4]>(sel_dsm + kKeyStages * kKeyTile * kIdxDim * sizeof(__nv_bfloat16));
-  __shared__ float s_qi[kSelRows][kIdxDim];
+  auto s_k = reinterpret_cast<__nv_bfloat16 (*)[kKeyTile * IDX]>(sel_dsm);
+  auto s_sc = reinterpret_cast<float (*)[kKeyTile + 4]>(sel_dsm + kKeyStages * kKeyTile * IDX * sizeof(__nv_bfloat16));
+  __shared__ float s_qi[kSelRows][IDX];
   __shared__ uint2 s_cand[kSelRows][kCand];
   __shared__ unsigned long long s_cw[kSelRows][kCand];
   // Each row's selection state lives in shared memory: a pass loads only the
@@ -203,17 +208,18 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
 
   // q~ = W_q q_pre with the decode path's association: four quarter sums of
   // D/4 dims each, then butterfly adds.
-  float qi[kIdxDim];
+  float qi[IDX];
   {
     constexpr int DQ = D / 4;
-    float part[2];
+    constexpr int NIT = (IDX * 4 + 31) / 32;
+    float part[NIT];
 #pragma unroll
-    for (int it = 0; it < 2; ++it) {
-      const int task = it * 32 + lane;  // 16 outputs x 4 quarters
+    for (int it = 0; it < NIT; ++it) {
+      const int task = it * 32 + lane;  // IDX outputs x 4 quarters
       const int o = task >> 2, qd = task & 3;
       float acc = 0.f;
-      if (row_ok) {
-        const float4* w = reinterpret_cast<const float4*>(a.w_q + ((size_t)r * kIdxDim + o) * D + qd * DQ);
+      if (row_ok && o < IDX) {
+        const float4* w = reinterpret_cast<const float4*>(a.w_q + ((size_t)r * IDX + o) * D + qd * DQ);
         const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(a.q_pre) +
                                  (((size_t)b * a.T + t) * a.Hq + h * a.G + g) * D + qd * DQ;
         float wv[DQ], qv[DQ];
@@ -231,36 +237,25 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
       part[it] = acc;
     }
 #pragma unroll
-    for (int o = 0; o < kIdxDim; ++o) qi[o] = __shfl_sync(0xffffffffu, part[o >> 3], (o & 7) * 4);
+    for (int o = 0; o < IDX; ++o) qi[o] = __shfl_sync(0xffffffffu, part[o >> 3], (o & 7) * 4);
   }
   {
-    // lane l < 16 stores q~[l] (constant register indices only)
+    // lane l < IDX stores q~[l] (constant register indices only)
     float mine = 0.f;
 #pragma unroll
-    for (int o = 0; o < kIdxDim; ++o)
+    for (int o = 0; o < IDX; ++o)
       if (lane == o) mine = qi[o];
-    if (lane < kIdxDim) s_qi[warp][lane] = mine;
+    if (lane < IDX) s_qi[warp][lane] = mine;
   }
   __syncthreads();
-  // Scores on tensor cores: S = K~ Q~^T with K = 16, q~ split into bf16 hi and
-  // lo parts (the products are exact; fp32 accumulation), so the score is the
-  // fp32 q~ . k~ to about 2^-17 relative.  B fragments (16 dims x 8 rows): lane
-  // holds row lane/4, dims 2t, 2t+1 (b0) and 2t+8, 2t+9 (b1), t = lane % 4.
-  unsigned bh0, bh1, bl0, bl1;
-  {
-    const int n = lane >> 2, k0 = (lane & 3) * 2;
-    float v[4] = {s_qi[n][k0], s_qi[n][k0 + 1], s_qi[n][k0 + 8], s_qi[n][k0 + 9]};
-    float hi[4], lo[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      hi[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
-      lo[e] = v[e] - hi[e];
-    }
-    bh0 = pack_bf16(hi[0], hi[1]);
-    bh1 = pack_bf16(hi[2], hi[3]);
-    bl0 = pack_bf16(lo[0], lo[1]);
-    bl1 = pack_bf16(lo[2], lo[3]);
-  }
+  // Scores on tensor cores with the decode path's fragments (IdxMma): S =
+  // K~ Q~^T, q~ split into bf16 hi and lo parts (the products are exact; fp32
+  // accumulation), so the score is the fp32 q~ . k~ to about 2^-17 relative
+  // and equals the decode step's bit for bit.  Column n of the product is row
+  // n of this CTA.
+  IdxMma<IDX> mm;
+  mm.set_q(s_qi[lane >> 2], lane);
+  constexpr float kScale = idx_scale<IDX>();
 
   if (lane == 0) {
     s_rs[warp] = RowSel{};
@@ -270,7 +265,7 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
   }
   __syncwarp();
   const RowSel& R = s_rs[warp];
-  const __nv_bfloat16* kidx = static_cast<const __nv_bfloat16*>(a.kidx) + ((size_t)b * a.R + r) * a.Lmax * kIdxDim;
+  const __nv_bfloat16* kidx = static_cast<const __nv_bfloat16*>(a.kidx) + ((size_t)b * a.R + r) * a.Lk * IDX;
   uint32_t* mrow = a.mask + (((size_t)b * a.NR + hh) * a.mask_rows + (row_ok ? t - a.mask_t0 : 0)) * a.words;
 
   // pass accumulators
@@ -296,9 +291,12 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
     auto stage_async = [&](int kt_, int buf) {
       if (kt_ <= i_last) {
         const int n = min(kKeyTile, i_last + 1 - kt_);
-        const char* src = reinterpret_cast<const char*>(kidx + (size_t)kt_ * kIdxDim);
+        const char* src = reinterpret_cast<const char*>(kidx + (size_t)kt_ * IDX);
         const unsigned dst = (unsigned)__cvta_generic_to_shared(s_k[buf]);
-        for (int v = threadIdx.x; v < n * 2; v += kSelRows * 32)
+        // whole 16-byte vectors: an odd count of 8-byte keys takes the next key
+        // of the block too (the block then has an even row count past it)
+        const int nvec = (n * KB + 15) / 16;
+        for (int v = threadIdx.x; v < nvec; v += kSelRows * 32)
           asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst + 16u * v), "l"(src + 16 * (size_t)v));
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
@@ -315,16 +313,13 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
 #pragma unroll
       for (int half = 0; half < kKeyTile / kSelRows / 16; ++half) {
         const int kb = warp * (kKeyTile / kSelRows) + half * 16;  // first key (M row) of this 16 x 8 tile
-        unsigned a0, a1, a2, a3;
-        ldsm_x4(a0, a1, a2, a3, s_k[buf] + (size_t)(kb + (lane & 7) + ((lane >> 3) & 1) * 8) * kIdxDim + (lane >> 4) * 8);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-        mma_bf16(c, a0, a1, a2, a3, bh0, bh1);
-        mma_bf16(c, a0, a1, a2, a3, bl0, bl1);
+        float c[4];
+        mm.scores(reinterpret_cast<const unsigned char*>(s_k[buf]) + (size_t)kb * KB, lane, c);
         const int key0 = kb + (lane >> 2), row0 = (lane & 3) * 2;
-        s_sc[row0][key0] = c[0] * kIdxScale + 0.0f;  // +0 turns -0 into +0
-        s_sc[row0 + 1][key0] = c[1] * kIdxScale + 0.0f;
-        s_sc[row0][key0 + 8] = c[2] * kIdxScale + 0.0f;
-        s_sc[row0 + 1][key0 + 8] = c[3] * kIdxScale + 0.0f;
+        s_sc[row0][key0] = c[0] * kScale + 0.0f;  // +0 turns -0 into +0
+        s_sc[row0 + 1][key0] = c[1] * kScale + 0.0f;
+        s_sc[row0][key0 + 8] = c[2] * kScale + 0.0f;
+        s_sc[row0 + 1][key0 + 8] = c[3] * kScale + 0.0f;
       }
       __syncthreads();
       buf = buf + 1 == kKeyStages ? 0 : buf + 1;  // the next tile's buffer
@@ -944,6 +939,24 @@ __global__ void __launch_bounds__(128, 3) attn_rows_kernel(const __grid_constant
   }
 }
 
+template <int D>
+void set_select_attrs() {
+  cudaFuncSetAttribute(select_rows_kernel<D, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_dyn_smem(4));
+  cudaFuncSetAttribute(select_rows_kernel<D, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_dyn_smem(8));
+  cudaFuncSetAttribute(select_rows_kernel<D, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_dyn_smem(16));
+  cudaFuncSetAttribute(select_rows_kernel<D, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_dyn_smem(32));
+}
+
+template <int D>
+void launch_select_rows(int idx, dim3 gs, cudaStream_t st, const PrefillArgs& a) {
+  switch (idx) {
+    case 4: select_rows_kernel<D, 4><<<gs, kSelRows * 32, sel_dyn_smem(4), st>>>(a); break;
+    case 8: select_rows_kernel<D, 8><<<gs, kSelRows * 32, sel_dyn_smem(8), st>>>(a); break;
+    case 32: select_rows_kernel<D, 32><<<gs, kSelRows * 32, sel_dyn_smem(32), st>>>(a); break;
+    default: select_rows_kernel<D, 16><<<gs, kSelRows * 32, sel_dyn_smem(16), st>>>(a); break;
+  }
+}
+
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 }  // namespace
@@ -983,7 +996,7 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
   }
   PrefillArgs a;
   a.B = sh.B; a.Hq = sh.Hq; a.Hkv = sh.Hkv; a.G = sh.G; a.D = sh.D; a.R = sh.R; a.NR = sh.NR;
-  a.Lmax = sh.Lmax; a.S = sh.S; a.W = sh.W; a.T = T; a.words = (sh.Lmax + 31) / 32;
+  a.Lmax = sh.Lmax; a.S = sh.S; a.W = sh.W; a.T = T; a.words = (sh.Lmax + 31) / 32; a.Lk = sh.Lk;
   a.top_p = sh.top_p; a.rope_base = sh.rope_base;
   a.q_pre = q_pre; a.w_q = w_q; a.out = out;
   a.k = cache->k; a.v = cache->v; a.kidx = cache->kidx; a.status = cache->status;
@@ -1007,8 +1020,8 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
                          (int)AttnSmem<128>::kBytes);
     cudaFuncSetAttribute(attn_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)AttnSmem<64>::kBytes);
-    cudaFuncSetAttribute(select_rows_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDynSmem);
-    cudaFuncSetAttribute(select_rows_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSelDynSmem);
+    set_select_attrs<128>();
+    set_select_attrs<64>();
     s_attr[dev] = true;
   }
   // The caller's bitmask holds every row; the workspace one block of rows.
@@ -1022,8 +1035,8 @@ int launch_prefill(const Shape& sh, const rtp_cache* cache, const void* q_pre, c
     if (sh.R > 0) {
       const dim3 gs((n + kSelRows - 1) / kSelRows, sh.B * sh.NR);
       trace_begin(RTP_STAGE_PREFILL_INDEX, st);
-      if (sh.D == 128) select_rows_kernel<128><<<gs, kSelRows * 32, kSelDynSmem, st>>>(a);
-      else select_rows_kernel<64><<<gs, kSelRows * 32, kSelDynSmem, st>>>(a);
+      if (sh.D == 128) launch_select_rows<128>(sh.idx, gs, st, a);
+      else launch_select_rows<64>(sh.idx, gs, st, a);
       trace_end(RTP_STAGE_PREFILL_INDEX, st);
     }
     trace_begin(RTP_STAGE_PREFILL_ATTN, st);

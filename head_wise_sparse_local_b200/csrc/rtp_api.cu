@@ -257,7 +257,6 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
   if (T < 1 || T > sh.Lmax) return fail(RTP_ERR_SHAPE, "T must be in [1, max_ctx]");
   if (sh.top_k > 0)
     return fail(RTP_ERR_SHAPE, "static top-k (cfg top_k > 0) is a decode-only variant; prefill selects by top-p");
-  if (sh.idx != 16) return fail(RTP_ERR_SHAPE, "prefill takes idx_dim 16 only");
   if (sh.ring > 0 && (long long)T + sh.W - 1 > sh.ring)
     return fail(RTP_ERR_SHAPE, "ring mode: a prefill chunk needs local_cap >= T + window - 1");
   if (!q_pre || !start_pos || !out) return fail(RTP_ERR_INVALID, "q_pre/start_pos/out is NULL");

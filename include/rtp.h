@@ -67,7 +67,6 @@ typedef enum rtp_dtype { RTP_BF16 = 0, RTP_FP32 = 1 } rtp_dtype;
  *                 or 32 for the pages' indexer-dimension ablation
  *                 (atlas.scime.ai summary, "Surprising findings": dimension 4).
  *                 Scores are q~ . k~ / sqrt(d), with 1/sqrt(d) rounded to fp32.
- *                 Prefill takes d = 16 only (RTP_ERR_SHAPE otherwise).
  *   max_ctx       Lmax, cache capacity per sequence (positions [0, Lmax));
  *                 at most 2^23
  *   n_sink        S >= 0: positions [0, S) are always attended (sinks)
@@ -270,12 +269,12 @@ int rtp_decode_attn_noalloc(const rtp_layer_cfg* cfg, const rtp_cache* cache, co
  * a row's top-p set equals the decode step's at that position, bit for bit.
  * The attention itself runs on tensor cores in bf16 with fp32 accumulation
  * (atlas.scime.ai summary, "Approach"; abstract, observations (2)-(3)).
- * cfg->dtype must be RTP_BF16 and cfg->idx_dim 16.
+ * cfg->dtype must be RTP_BF16.
  *
  *   q_pre        [B][T][Hq][D] bf16, device
  *   start_pos    [B] int32, device; 0 <= start_pos[b] and start_pos[b] + T <= max_ctx
  *                (else the sequence is skipped and RTP_DEV_POSITION is set)
- *   w_q          [R][16][D] fp32, device
+ *   w_q          [R][d][D] fp32, device
  *   out          [B][T][Hq][D] bf16, device
  *   sel_bitmask  optional [B][R*G][T][ceil(max_ctx/32)] uint32: row (b, r*G+g, t)
  *                has bit j set iff token j is in that row's top-p set; words

@@ -66,16 +66,6 @@ def test_indexer_cache_rows_per_width(rtp, d, dtype, lmax, lk):
     assert (lk * d * es) % 16 == 0
 
 
-def test_prefill_takes_width_16_only(rtp):
-    c = _cfg(rtp, idx_dim=8)
-    fake = 1 << 20  # never dereferenced: validation fails first
-    cache = rtp.rtp_cache(fake, fake, fake, fake)
-    with pytest.raises(rtp.RtpError) as e:
-        rtp.rtp_prefill_attn(c, cache, fake, fake, 8, fake, fake, workspace=fake, workspace_bytes=1 << 40,
-                             stream=0)
-    assert e.value.code == 2
-
-
 @pytest.mark.parametrize("kw,code", [
     (dict(head_dim=96), 2), (dict(n_q_heads=24), 2), (dict(n_q_heads=30), 2),
     (dict(top_p=0.0), 1), (dict(top_p=1.5), 1), (dict(window=0), 1), (dict(n_sink=-1), 1),
