@@ -3,24 +3,25 @@
 // (atlas.scime.ai summary, "Approach"; abstract, observations (2)-(3)).
 //
 //   select_rows_kernel  retrieval query heads only.  One warp per query row,
-//       8 rows per CTA sharing the 16-d indexer-key tiles staged in shared
-//       memory.  Each pass computes a tile's scores for all 8 rows on tensor
-//       cores (q~ as bf16 hi + lo parts: the fp32 score to about 2^-17), so a
-//       row's selection equals the decode step's at that position except for
-//       tokens within that rounding of the threshold.
-//       The exact top-p threshold is found by splitting the score interval
-//       that contains the boundary 8 ways per pass, with the softmax mass
-//       exp(s - max) of every score in 2^-36 fixed point (mass36, shared with
-//       the decode path; exact integer sums in registers), until at most
-//       kCand tokens remain; a warp-level exact solve finishes (ties to the
-//       lower index).  The first pass also takes the scores' mean and spread,
-//       and the first split's edges go around the boundary a Gaussian score
-//       model predicts (a guess that only places them).  The pass that
-//       collects the last candidates also writes the row's top-p bitmask.
+//       8 rows per CTA sharing the indexer-key tiles staged in shared memory.
+//       Each pass computes a tile's scores for all 8 rows on tensor cores with
+//       the decode path's fragments (IdxMma: q~ as bf16 hi + lo parts, the
+//       fp32 score to about 2^-17), so a row's scores, and its selection,
+//       equal the decode step's at that position bit for bit.
+//       The softmax mass exp(s - max) of every score is taken in 2^-36 fixed
+//       point (mass36, shared with the decode path; exact integer sums).  The
+//       first pass takes the maximum and the scores' mean and spread; the
+//       first split sums every key's mass into 8 sub-intervals whose edges go
+//       around the boundary a Gaussian score model predicts (a guess that only
+//       places them); later (wide) splits bin the few keys inside the boundary
+//       interval into 32 sub-intervals in shared memory, until at most kCand
+//       tokens remain; a warp-level exact solve finishes (ties to the lower
+//       index), in the pass that also writes the row's top-p bitmask.
 //   attn_rows_kernel  tensor-core (mma.sync m16n8k16 bf16, fp32 accumulate)
 //       flash attention over 64-row query tiles and 64-key tiles, masked by
-//       causality, sinks, the window and (retrieval heads) the bitmask; key
-//       tiles holding nothing a row keeps are skipped.
+//       causality, sinks, the window and (retrieval heads) the bitmask; used
+//       for local heads that keep a ring of window rows (the tcgen05 kernel in
+//       prefill_tc.cu takes every other head).
 #include <climits>
 #include <mutex>
 
@@ -104,14 +105,16 @@ __device__ __forceinline__ unsigned wmaxu(unsigned v) {
 // What a row's warp does with each of its scores in one pass over its keys.
 enum : int {
   kOpMax = 0,    // row maximum
-  kOpSplit = 1,  // mass/count of the 8 sub-intervals of the current interval
+  kOpSplit = 1,  // first split: every key's mass into the 8 sub-intervals around the guessed boundary
   kOpRange = 2,  // min/max order key inside the current interval
   kOpCand = 3,   // collect the current interval's tokens for the exact solve; write the bitmask
   kOpTies = 4,   // count tied tokens with index <= probe (index bisection)
   kOpEmit = 5,   // write the top-p bitmask (after exact ties or p >= 1; the
                  // candidate pass writes it itself)
-  kOpDone = 6
+  kOpDone = 6,
+  kOpWide = 7    // later splits: the keys inside the current interval into 32 sub-intervals
 };
+constexpr int kWideBins = 32;
 
 // Per-row selection state (kept identical in every lane of the row's warp).
 struct RowSel {
@@ -154,24 +157,25 @@ __device__ __forceinline__ SplitView load_split(const RowSel& R) {
   for (int e = 0; e < 7; ++e) v.thr[e] = v.by_key ? __uint_as_float(R.kth[e]) : R.th[e];
   return v;
 }
-// One score inside the interval of a later split: its mass into the cumulative
-// sums (pm[e] / pc[e], e < 7: past edge e; [7]: everything inside).
-__device__ __forceinline__ void split_item(const SplitView& v, float sv, unsigned long long (&pm)[8],
-                                           unsigned (&pc)[8]) {
-  const float d = v.m - sv;
+// One score inside the interval of a wide split: its exact mass and a count
+// into the bin it falls in (the number of the interval's 31 edges it passes;
+// edges are d thresholds ascending, or order keys descending, so passing is
+// monotone in the edge index and a 5-step search finds the bin).
+__device__ __forceinline__ void wide_item(float m, bool by_key, const unsigned* edges, unsigned long long* bm,
+                                          unsigned* bc, float sv) {
+  const float d = m - sv;
   const unsigned key = score_key(sv);
-  const unsigned long long w = mass36(sv, v.m);
-  pm[7] += w;
-  pc[7] += 1u;
-  if (!v.by_key) {
+  int nb = 0;
 #pragma unroll
-    for (int e = 0; e < 7; ++e)
-      if (d >= v.thr[e]) { pm[e] += w; pc[e] += 1u; }
-  } else {
-#pragma unroll
-    for (int e = 0; e < 7; ++e)
-      if (key < __float_as_uint(v.thr[e])) { pm[e] += w; pc[e] += 1u; }
+  for (int step = 16; step >= 1; step >>= 1) {
+    const int e = nb + step - 1;
+    if (e < kWideBins - 1) {
+      const unsigned ed = edges[e];
+      if (by_key ? key < ed : d >= __uint_as_float(ed)) nb += step;
+    }
   }
+  atomicAdd(&bm[nb], mass36(sv, m));
+  atomicAdd(&bc[nb], 1u);
 }
 
 template <int D, int IDX>
@@ -267,6 +271,40 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
   const RowSel& R = s_rs[warp];
   const __nv_bfloat16* kidx = static_cast<const __nv_bfloat16*>(a.kidx) + ((size_t)b * a.R + r) * a.Lk * IDX;
   uint32_t* mrow = a.mask + (((size_t)b * a.NR + hh) * a.mask_rows + (row_ok ? t - a.mask_t0 : 0)) * a.words;
+  // The wide split's bins and edges use the warp's candidate arrays (a row is
+  // never in a split pass and a candidate pass at once): exact mass and count
+  // per sub-interval, and the 31 edges (d as float bits, or order keys).
+  unsigned long long* wd_m = s_cw[warp];
+  unsigned* wd_c = reinterpret_cast<unsigned*>(s_cand[warp]);
+  unsigned* wd_e = wd_c + kWideBins;
+  static_assert(kCand * sizeof(uint2) >= (2 * kWideBins) * sizeof(unsigned), "bins and edges fit");
+  static_assert(kCand >= kWideBins, "bin masses fit");
+  // After a split: the candidate pass once the boundary interval holds few
+  // enough tokens; else a wide split of a d interval while d still separates
+  // its tokens (edges written to the warp's edge array), else the range pass,
+  // which bounds the interval by the keys present (and finds exact ties)
+  // before a wide split on order keys.
+  auto next_step = [&](RowSel& rs, unsigned before) {
+    if (rs.cnt_in <= (unsigned)kCand) {
+      rs.op = kOpCand;
+      return;
+    }
+    if (rs.by_key || rs.dhi < 0.f || rs.cnt_in >= before) {
+      rs.op = kOpRange;
+      return;
+    }
+    const float step = (rs.dhi - rs.dlo) * (1.0f / kWideBins);
+    const float ed = fminf(rs.dlo + step * (float)(lane + 1), rs.dhi);  // edge `lane` (< 31)
+    const bool splits = __shfl_sync(0xffffffffu, ed, 0) > rs.dlo &&
+                        __shfl_sync(0xffffffffu, ed, kWideBins - 2) < rs.dhi;
+    if (!splits) {
+      rs.op = kOpRange;
+      return;
+    }
+    if (lane < kWideBins - 1) wd_e[lane] = __float_as_uint(ed);
+    __syncwarp();
+    rs.op = kOpWide;
+  };
 
   // pass accumulators
   unsigned long long pm[8];
@@ -285,6 +323,11 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
     x1 = 0u;  // also 0.f
     x2 = 0u;
     const bool first_split = (op == kOpSplit) && R.first;
+    if (op == kOpWide) {
+      wd_m[lane] = 0ull;
+      wd_c[lane] = 0u;
+      __syncwarp();
+    }
     unsigned q_head = 0u, q_tail = 0u;  // s_ring[warp] positions (warp-uniform)
     // key tiles [kt, kt + kKeyTile) up to i_last, copied asynchronously
     // kKeyStages - 1 tiles ahead of their use (an empty group past the end)
@@ -360,46 +403,49 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
           }
           break;
         }
-        case kOpSplit: {
+        case kOpSplit: {  // the first split: every key is inside; total mass and d-thresholds
           const SplitView v = load_split(R);
           const float m = v.m;
-          if (first_split) {  // every key is inside: total mass and d-thresholds
 #pragma unroll 4
-            for (int u = 0; u < kKeyTile / 32; ++u) {
-              const int j = kt + u * 32 + lane;
-              if (u >= ulim || j > i) continue;
-              const float sv = srow[u * 32 + lane];
-              const float d = m - sv;
-              const unsigned long long w = mass36(sv, m);
-              pm[7] += w;  // every key: the total mass
-              pc[7] += 1u;
+          for (int u = 0; u < kKeyTile / 32; ++u) {
+            const int j = kt + u * 32 + lane;
+            if (u >= ulim || j > i) continue;
+            const float sv = srow[u * 32 + lane];
+            const float d = m - sv;
+            const unsigned long long w = mass36(sv, m);
+            pm[7] += w;  // every key: the total mass
+            pc[7] += 1u;
 #pragma unroll
-              for (int e = 0; e < 7; ++e)
-                if (d >= v.thr[e]) { pm[e] += w; pc[e] += 1u; }
-            }
-          } else {
-            // a small share of the keys lies inside: gather those scores in
-            // the warp's ring and add them 32 at a time (no divergent lanes)
-            float* ring = s_ring[warp];
+            for (int e = 0; e < 7; ++e)
+              if (d >= v.thr[e]) { pm[e] += w; pc[e] += 1u; }
+          }
+          break;
+        }
+        case kOpWide: {
+          // a small share of the keys lies inside: gather those scores in the
+          // warp's ring and bin them 32 at a time (no divergent lanes)
+          const float m = R.m, dlo = R.dlo, dhi = R.dhi;
+          const unsigned klo = R.klo, khi = R.khi;
+          const bool by_key = R.by_key;
+          float* ring = s_ring[warp];
 #pragma unroll 4
-            for (int u = 0; u < kKeyTile / 32; ++u) {
-              if (u >= ulim) break;
-              const int j = kt + u * 32 + lane;
-              const float sv = srow[u * 32 + lane];
-              const float d = m - sv;
-              const unsigned key = score_key(sv);
-              const bool inside = j <= i && d >= v.dlo && (v.dhi < 0.f || d < v.dhi) && key >= v.klo && key <= v.khi;
-              const unsigned bal = __ballot_sync(0xffffffffu, inside);
-              if (bal == 0u) continue;
-              if (inside) ring[(q_tail + __popc(bal & ((1u << lane) - 1u))) & 63u] = sv;
-              q_tail += (unsigned)__popc(bal);
-              if (q_tail - q_head >= 32u) {
-                __syncwarp();
-                const float sq = ring[(q_head + lane) & 63u];
-                __syncwarp();
-                q_head += 32u;
-                split_item(v, sq, pm, pc);
-              }
+          for (int u = 0; u < kKeyTile / 32; ++u) {
+            if (u >= ulim) break;
+            const int j = kt + u * 32 + lane;
+            const float sv = srow[u * 32 + lane];
+            const float d = m - sv;
+            const unsigned key = score_key(sv);
+            const bool inside = j <= i && d >= dlo && (dhi < 0.f || d < dhi) && key >= klo && key <= khi;
+            const unsigned bal = __ballot_sync(0xffffffffu, inside);
+            if (bal == 0u) continue;
+            if (inside) ring[(q_tail + __popc(bal & ((1u << lane) - 1u))) & 63u] = sv;
+            q_tail += (unsigned)__popc(bal);
+            if (q_tail - q_head >= 32u) {
+              __syncwarp();
+              const float sq = ring[(q_head + lane) & 63u];
+              __syncwarp();
+              q_head += 32u;
+              wide_item(m, by_key, wd_e, wd_m, wd_c, sq);
             }
           }
           break;
@@ -462,9 +508,9 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
           break;
       }
     }
-    if (op == kOpSplit && !first_split && q_tail != q_head) {  // the ring's last (< 32) scores
+    if (op == kOpWide && q_tail != q_head) {  // the ring's last (< 32) scores
       __syncwarp();
-      if (lane < q_tail - q_head) split_item(load_split(R), s_ring[warp][(q_head + lane) & 63u], pm, pc);
+      if (lane < q_tail - q_head) wide_item(R.m, R.by_key, wd_e, wd_m, wd_c, s_ring[warp][(q_head + lane) & 63u]);
     }
     // ---- reduce this pass and choose the next step (warp-uniform) ----
     RowSel rs = R;
@@ -564,22 +610,45 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
         rs.klo = lo;
         rs.khi = hi;
       }
-      if (rs.cnt_in <= (unsigned)kCand) {
-        rs.op = kOpCand;
-      } else {
-        // next split: d thresholds while they still separate, else order keys
-        bool split_d = !rs.by_key && rs.dhi >= 0.f && rs.cnt_in < before;
-        if (!rs.by_key && rs.dhi < 0.f) {  // open interval: bound it first
-          rs.op = kOpRange;
-        } else if (split_d) {
-          const float step = (rs.dhi - rs.dlo) * 0.125f;
+      next_step(rs, before);
+    } else if (op == kOpWide) {
+      // bins from the highest scores (lane 0) down: the first whose cumulative
+      // mass reaches the mass still needed holds the boundary
+      __syncwarp();
+      const unsigned long long mb = wd_m[lane];
+      const unsigned cb = wd_c[lane];
+      unsigned long long cm = mb;
+      unsigned ck = cb;
 #pragma unroll
-          for (int e = 0; e < 7; ++e) rs.th[e] = fminf(rs.dlo + step * (float)(e + 1), rs.dhi);
-          rs.op = (rs.th[0] > rs.dlo && rs.th[6] < rs.dhi) ? kOpSplit : kOpRange;
-        } else {
-          rs.op = kOpRange;
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long tm = __shfl_up_sync(0xffffffffu, cm, o);
+        const unsigned tc = __shfl_up_sync(0xffffffffu, ck, o);
+        if (lane >= o) {
+          cm += tm;
+          ck += tc;
         }
       }
+      const unsigned ball = __ballot_sync(0xffffffffu, cm >= rs.need);
+      const int sel = ball ? __ffs(ball) - 1 : kWideBins - 1;
+      const unsigned long long ex_m = __shfl_sync(0xffffffffu, cm - mb, sel);
+      const unsigned ex_c = __shfl_sync(0xffffffffu, ck - cb, sel);
+      const unsigned in_c = __shfl_sync(0xffffffffu, cb, sel);
+      const unsigned my_e = lane < kWideBins - 1 ? wd_e[lane] : 0u;
+      const unsigned e_lo = __shfl_sync(0xffffffffu, my_e, sel > 0 ? sel - 1 : 0);
+      const unsigned e_hi = __shfl_sync(0xffffffffu, my_e, sel < kWideBins - 1 ? sel : 0);
+      rs.need -= ex_m;
+      rs.cnt_above += ex_c;
+      const unsigned before = rs.cnt_in;
+      rs.cnt_in = in_c;
+      if (!rs.by_key) {  // bin b: d in [edge b-1, edge b)
+        if (sel > 0) rs.dlo = __uint_as_float(e_lo);
+        if (sel < kWideBins - 1) rs.dhi = __uint_as_float(e_hi);
+      } else {           // bin b: keys in [edge b, edge b-1 - 1]
+        if (sel > 0) rs.khi = e_lo - 1u;
+        if (sel < kWideBins - 1) rs.klo = e_hi;
+      }
+      __syncwarp();  // every lane has read the edges before they are rewritten
+      next_step(rs, before);
     } else if (op == kOpRange) {
       rs.klo = max(rs.klo, wminu(x0));
       rs.khi = min(rs.khi, wmaxu(x1));
@@ -605,11 +674,13 @@ __global__ void __launch_bounds__(kSelRows * 32, 3) select_rows_kernel(const __g
           rs.kth[0] = (unsigned)i;  // upper end of the bisection range
         }
       } else {
+        // edge e (< 31): first key of the (e+1)-th of 32 key sub-intervals from the top
         const unsigned long long span = (unsigned long long)rs.khi - rs.klo + 1ull;
-#pragma unroll
-        for (int e = 0; e < 7; ++e)  // kth[e]: first key of the (e+1)-th interval from the top
-          rs.kth[e] = (unsigned)(rs.khi + 1ull - (span * (unsigned long long)(e + 1) + 7ull) / 8ull);
-        rs.op = kOpSplit;
+        if (lane < kWideBins - 1)
+          wd_e[lane] = (unsigned)(rs.khi + 1ull -
+                                  (span * (unsigned long long)(lane + 1) + (kWideBins - 1)) / kWideBins);
+        __syncwarp();
+        rs.op = kOpWide;
       }
     } else if (op == kOpTies) {
       // bisection on the index: smallest probe with count(ties <= probe) >= need_ties
