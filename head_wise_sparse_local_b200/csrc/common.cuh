@@ -10,7 +10,6 @@
 
 namespace rtp {
 
-constexpr int kIdxDim = 16;        // indexer width (abstract, observation (2))
 // Score scale 1/sqrt(d) for the indexer widths the layer takes: d = 16 and the
 // pages' ablation widths 4, 8, 32 (atlas.scime.ai summary, "Surprising
 // findings"); exact for 4 and 16, rounded to fp32 for 8 and 32.
@@ -19,7 +18,6 @@ __host__ __device__ constexpr float idx_scale() {
   static_assert(IDX == 4 || IDX == 8 || IDX == 16 || IDX == 32, "indexer width");
   return IDX == 4 ? 0.5f : IDX == 8 ? 0.35355339059327376f : IDX == 16 ? 0.25f : 0.17677669529663688f;
 }
-constexpr float kIdxScale = idx_scale<16>();
 constexpr int kMaxRetrieval = 64;
 
 // ---------------------------------------------------------------------------
