@@ -420,11 +420,18 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
   using Lane = SwLane<T, D>;
   constexpr int EPL = Lane::EPL;
   constexpr int RB = D * (int)sizeof(T);             // bytes per cache row
+  // Shared-memory row stride: a bf16 row is padded by 16 bytes, so the 8 rows
+  // that one ldmatrix phase reads start 4 banks apart (conflict-free) instead
+  // of all in the same 4 banks.
+  constexpr int RBS = sizeof(T) == 2 ? RB + 16 : RB;
+  constexpr int CPW = 2 * RB / 16;                   // 16-byte chunks of a row's K and V
+  static_assert((CPW & (CPW - 1)) == 0, "chunks per row: a power of two");
   // rows per stage (K and V of a stage take at most half the buffer; at most
   // 80 rows, 32 for G = 8, which keeps a warp's scores of a stage in registers)
   constexpr int kCapRows = G >= 8 ? 32 : 80;
-  constexpr int SR = (kStreamSmem / 4 / RB) < kCapRows ? (kStreamSmem / 4 / RB) : kCapRows;
+  constexpr int SR = ((kStreamSmem / 4 / RBS) < kCapRows ? (kStreamSmem / 4 / RBS) : kCapRows) & ~1;
   static_assert(SR >= 2 && SR % 2 == 0, "a stage holds whole row pairs");
+  static_assert(2 * SR * RBS <= kStreamSmem / 2, "a stage's K and V fit in half the buffer");
   __shared__ __align__(16) float s_q[G * D];
   __shared__ __align__(16) float s_wo[kWarps][G][D];
   __shared__ float s_wml[kWarps][G][2];
@@ -438,13 +445,21 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
     if (crank == 0 && h == 0 && tid == 0) atomicOr(a.status, RTP_DEV_SEQ_LEN);
     return;
   }
+  // A stage's barrier phase completes with one arrival per thread, made once
+  // that thread's copies have landed, plus one from thread 0 (which, when a
+  // test arms expiry, also expects bytes that never come).
   if (tid == 0) {
-    mbar_init(bar, 1);
-    mbar_init(bar + 1, 1);
+    mbar_init(bar, kThreads + 1);
+    mbar_init(bar + 1, kThreads + 1);
   }
-  rope_query<T, D, G>(a, b, h, L - 1, s_q);
-  __syncthreads();  // barriers initialised, s_q visible
-  if (a.n_score_ctas == 0) griddep_wait();  // no score kernel ahead: wait for rtp_append_kv here
+  // With a score kernel ahead the appended rows are complete already (this
+  // kernel starts after every score CTA has passed its wait): the copies go
+  // out first and the query is formed while they fly.  Without one, the query
+  // comes first, then the wait for rtp_append_kv.
+  const bool waits = a.n_score_ctas == 0;
+  if (waits) rope_query<T, D, G>(a, b, h, L - 1, s_q);
+  __syncthreads();  // barriers initialised
+  if (waits) griddep_wait();
 
   const int s_cnt = min(a.S, L);
   const int sw0 = max(s_cnt, L - a.W);
@@ -455,31 +470,47 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
   const int n_st = (e_hi - e_lo + SR - 1) / SR;
   const unsigned char* kbase = static_cast<const unsigned char*>(a.k);
   const unsigned char* vbase = static_cast<const unsigned char*>(a.v);
-  const bool ringed = (a.kv.ring_mask >> h) & 1ull;
+  // Cache row of stage row e.  A ring head's window positions (at or past the
+  // sinks whenever the window is not empty) sit in consecutive ring slots from
+  // the slot of sw0, wrapping at most once (the ring holds at least W rows).
+  const bool fast_ring = ((a.kv.ring_mask >> h) & 1ull) && sw0 >= a.kv.S;
+  const int ws0 = fast_ring ? a.kv.S + (sw0 - a.kv.S) % a.kv.ring : 0;
+  const size_t seq_row0 = (size_t)b * (size_t)a.kv.rows_per_seq + (size_t)a.kv.row0[h];
+  auto row_of = [&](int e) -> size_t {
+    if (e >= s_cnt && fast_ring) {
+      int sl = ws0 + (e - s_cnt);
+      if (sl >= a.kv.S + a.kv.ring) sl -= a.kv.ring;
+      return seq_row0 + (size_t)sl;
+    }
+    return a.kv.row(b, h, e < s_cnt ? e : sw0 + (e - s_cnt));
+  };
 
-  // stage st: rows [e_lo + st*SR, ...) into buffer st & 1 (K, then V)
+  // stage st: rows [e_lo + st*SR, ...) into buffer st & 1 (K rows, then V
+  // rows, RBS apart), 16 bytes per cp.async; every thread takes part
   auto issue = [&](int st) {
     const int e0 = e_lo + st * SR, e1 = min(e_hi, e0 + SR);
     uint64_t* bb = bar + (st & 1);
     unsigned char* dk = dsm + (size_t)(st & 1) * (kStreamSmem / 2);
-    unsigned char* dv = dk + (size_t)SR * RB;
-    mbar_expect_tx(bb, (uint32_t)(e1 - e0) * 2u * RB + a.tx_extra);
+    unsigned char* dv = dk + (size_t)SR * RBS;
     const uint64_t pol = l2_evict_first();
-    for (int e = e0; e < e1;) {
-      const int pos = e < s_cnt ? e : sw0 + (e - s_cnt);
-      int n = (e < s_cnt ? s_cnt : e1) - e;
-      if (e < s_cnt && n > e1 - e) n = e1 - e;
-      if (ringed && pos >= a.kv.S) n = min(n, a.kv.S + a.kv.ring - (a.kv.S + (pos - a.kv.S) % a.kv.ring));
-      const size_t row = a.kv.row(b, h, pos);
-      bulk_g2s(dk + (size_t)(e - e0) * RB, kbase + row * RB, (uint32_t)n * RB, bb, pol);
-      bulk_g2s(dv + (size_t)(e - e0) * RB, vbase + row * RB, (uint32_t)n * RB, bb, pol);
-      e += n;
+    const int nch = (e1 - e0) * CPW;
+    for (int i = tid; i < nch; i += kThreads) {
+      const int e = e0 + i / CPW, cc = i % CPW;
+      const bool isv = cc >= CPW / 2;
+      const int off = 16 * (isv ? cc - CPW / 2 : cc);
+      const size_t row = row_of(e);
+      cp_async16((isv ? dv : dk) + (size_t)(e - e0) * RBS + off, (isv ? vbase : kbase) + row * RB + off, pol);
+    }
+    cp_async_arrive_noinc(bb);
+    if (tid == 0) {
+      if (a.tx_extra) mbar_expect_tx(bb, a.tx_extra);
+      else mbar_arrive(bb);
     }
   };
-  if (tid == 0) {
-    if (n_st > 0) issue(0);
-    if (n_st > 1) issue(1);
-  }
+  if (n_st > 0) issue(0);
+  if (n_st > 1) issue(1);
+  if (!waits) rope_query<T, D, G>(a, b, h, L - 1, s_q);
+  __syncthreads();  // s_q visible
 
   int failed = -1;
   if constexpr (sizeof(T) == 2) {
@@ -527,7 +558,7 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
       }
       const int n = min(e_hi, e_lo + (st + 1) * SR) - (e_lo + st * SR);
       const unsigned char* sk = dsm + (size_t)(st & 1) * (kStreamSmem / 2);
-      const unsigned char* sv = sk + (size_t)SR * RB;
+      const unsigned char* sv = sk + (size_t)SR * RBS;
       for (int tt = warp; 16 * tt < n; tt += kWarps) {  // warp-uniform
         const int r0 = 16 * tt;
         // S = K Q^T; rows past n read row 0 (their weights are zeroed)
@@ -536,7 +567,7 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
         for (int nt = 0; nt < NT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.f;
         {
           const int rr = r0 + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const unsigned char* krow = sk + (size_t)(rr < n ? rr : 0) * RB + (lane >> 4) * 16;
+          const unsigned char* krow = sk + (size_t)(rr < n ? rr : 0) * RBS + (lane >> 4) * 16;
 #pragma unroll
           for (int ks = 0; ks < KS; ++ks) {
             unsigned a0, a1, a2, a3;
@@ -597,7 +628,7 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
         // O^T += V^T P: V^T fragments by transposing loads of V rows
         {
           const int rr = r0 + (lane & 7) + ((lane >> 4) & 1) * 8;
-          const unsigned char* vrow = sv + (size_t)(rr < n ? rr : 0) * RB + ((lane >> 3) & 1) * 16;
+          const unsigned char* vrow = sv + (size_t)(rr < n ? rr : 0) * RBS + ((lane >> 3) & 1) * 16;
 #pragma unroll
           for (int mt = 0; mt < KS; ++mt) {
             unsigned a0, a1, a2, a3;
@@ -607,7 +638,7 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
         }
       }
       __syncthreads();  // buffer st & 1 is free
-      if (tid == 0 && st + 2 < n_st) issue(st + 2);
+      if (st + 2 < n_st) issue(st + 2);
     }
     // the warp's state: l summed over its lanes' rows; O^T fragments to shared memory
 #pragma unroll
@@ -654,7 +685,7 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
     }
     const int n = min(e_hi, e_lo + (st + 1) * SR) - (e_lo + st * SR);
     const unsigned char* sk = dsm + (size_t)(st & 1) * (kStreamSmem / 2);
-    const unsigned char* sv = sk + (size_t)SR * RB;
+    const unsigned char* sv = sk + (size_t)SR * RBS;
     float sc[PPW][G];
     float smax[G];
 #pragma unroll
@@ -664,7 +695,7 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
       const int i = 2 * (warp + k * kWarps) + half;
       const bool ok = i < n;  // uniform over the half-warp
       Lane kr;
-      kr.load(sk + (size_t)(ok ? i : 0) * RB + c * Lane::VB);
+      kr.load(sk + (size_t)(ok ? i : 0) * RBS + c * Lane::VB);
       float kf[EPL];
       kr.to_f32(kf);
 #pragma unroll
@@ -700,7 +731,7 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
       const int i = 2 * (warp + k * kWarps) + half;
       if (i >= n) continue;  // uniform over the half-warp
       Lane vr;
-      vr.load(sv + (size_t)i * RB + c * Lane::VB);
+      vr.load(sv + (size_t)i * RBS + c * Lane::VB);
       float vf[EPL];
       vr.to_f32(vf);
 #pragma unroll
@@ -712,7 +743,7 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
       }
     }
     __syncthreads();  // buffer st & 1 is free
-    if (tid == 0 && st + 2 < n_st) issue(st + 2);
+    if (st + 2 < n_st) issue(st + 2);
   }
   // the two halves of the warp, then the warps of the CTA
 #pragma unroll
@@ -745,6 +776,7 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
     // output is invalid
     for (int st = failed; st < min(n_st, failed + 2); ++st)
       mbar_wait_bounded(bar + (st & 1), (uint32_t)(st >> 1) & 1u, a.wait_ns, a.status);
+    asm volatile("cp.async.wait_all;" ::: "memory");  // this thread's own copies, which always land
   }
   __syncthreads();
   // this CTA's partial (o[D], m, l) per query head -> the cluster's slot in L2
