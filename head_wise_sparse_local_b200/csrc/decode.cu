@@ -1,10 +1,10 @@
 // rtp_decode_attn: one decode step of the head-wise sparse attention layer.
 //
 // Three kernels on the caller's stream, chained with programmatic dependent
-// launch, scratch in the caller's workspace.  The first two are the step's
-// HBM streams and run side by side; each of their CTAs pulls its whole share
-// into shared memory with bulk asynchronous copies (TMA) that complete on an
-// mbarrier:
+// launch, scratch in the caller's workspace, launched in the order score,
+// select, sink/window.  The sink/window stream runs beside the select kernel;
+// the stream kernels' CTAs pull their whole share into shared memory with
+// asynchronous copies that complete on an mbarrier:
 //
 //   score_kernel   a chunk of the d-dim indexer-key cache (contiguous rows)
 //                  per CTA (d = 16, or 4, 8, 32 for the dimension ablation);
@@ -12,14 +12,10 @@
 //                  heads of a retrieval KV head are formed on tensor cores
 //                  (q~ as bf16 high and low parts, as in the prefill) and
 //                  written with a per-chunk maximum.
-//   sw_kernel      one cluster per (sequence, KV head) attends the sinks and
-//                  the window: S = K Q^T and O^T = V^T P on tensor cores per
-//                  16-row tile (bf16; fp32 layers on CUDA cores), log-sum-exp
-//                  merged across the cluster.  Local heads write their output
-//                  here; retrieval heads leave one partial per query head.
 //   select_kernel  one thread-block cluster per (sequence, retrieval q head).
-//                  It launches at once and prepares its query, then waits for
-//                  the stream kernel to complete.  The softmax mass
+//                  It launches once every score CTA has passed its wait and
+//                  prepares its query, then waits for the score kernel to
+//                  complete.  The softmax mass
 //                  exp(s - max) of every score is taken in 2^-36 fixed point
 //                  (integer sums: exact and order independent).  One pass sums
 //                  the total mass and the mass and count at or above rungs 1,
@@ -33,10 +29,16 @@
 //                  scores are solved.  Every CTA then writes its share of the
 //                  top-p bitmask and attends, for its query head, the kept
 //                  rows of its share that lie outside the sinks and the
-//                  window.  The cluster merges its partials with the head's
-//                  sink/window partial and writes the output.  Static top-k
-//                  (the pages' fixed-budget baseline) runs the same solver
-//                  with every token weighing 1 and the target k.
+//                  window, and leaves its partial (o, max, sum) in L2.  Static
+//                  top-k (the pages' fixed-budget baseline) runs the same
+//                  solver with every token weighing 1 and the target k.
+//   sw_kernel      one cluster per (sequence, KV head) attends the sinks and
+//                  the window: S = K Q^T and O^T = V^T P on tensor cores per
+//                  16-row tile (bf16; fp32 layers on CUDA cores), rows staged
+//                  by cp.async into a padded layout, log-sum-exp merged across
+//                  the cluster.  Local heads write their output here; a
+//                  retrieval head's clusters wait for the select kernel and
+//                  merge its partials into the output.
 //
 // Every in-kernel wait is either a hardware barrier reached uniformly or a
 // bounded wait on a copy barrier (RTP_DEV_TIMEOUT when it gives up).
@@ -64,7 +66,10 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
-constexpr int kSwCluster = 16;      // CTAs per sink/window cluster (one cluster per sequence and KV head)
+// CTAs per sink/window cluster (one cluster per sequence and KV head).  A
+// portable size: the clusters launch beside the select kernel's, and 8-CTA
+// clusters find room on SMs where 16-CTA ones would wait for it to finish.
+constexpr int kSwCluster = 8;
 constexpr int kStreamSmem = 80 * 1024;  // stream kernel: bytes of staged keys (score) or K/V rows (two stages)
 constexpr int kSelThreads = 512;
 constexpr int kSelWarps = kSelThreads / 32;
@@ -102,7 +107,6 @@ struct DecodeArgs {
   int* sel_count;   // optional [B][NR]
   float* logits;    // [B][NR][lstride]
   float* cmax;      // [B][NR][nch_score_max]
-  float* sw_part;   // [B][Hkv][G][D + 2]: sink/window partial per query head (o[D], m, l)
   float* sw_scratch;  // [B][Hkv][kSwCluster][G][D + 2]: partial of each CTA of a sink/window cluster
   float* sel_scratch; // [B][NR][kMaxCS][D + 3]: partial (o[D], m, l) and kept count of each select CTA
   uint2* cand;      // [B][NR][lstride] boundary-bucket candidates past kCandSmem
@@ -805,12 +809,18 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
   }
   cl.sync();  // every rank's partial written (the barrier orders global memory within the cluster)
   // The cluster's merge is spread over its ranks: element i of the G x D
-  // outputs goes to rank i mod csw.  Each thread issues its loads of every
-  // rank's partial at once (L2 hits, one round trip).
+  // outputs goes to rank i mod csw.  A retrieval head adds the kept-row
+  // partials of the select kernel's ranks: that kernel was launched ahead of
+  // this one and ran beside it; once the wait below returns it has completed.
+  // Each thread issues its loads of every partial at once (L2 hits, one round
+  // trip).
   const float* parts = a.sw_scratch + (size_t)bkv * kSwCluster * (G * (D + 2));
+  const int ncs = r >= 0 ? a.sel_cs : 0;  // select CTAs per retrieval query head (uniform over the cluster)
+  if (ncs > 0) griddep_wait();
   for (int i = crank + csw * tid; i < G * D; i += csw * kThreads) {
     const int g = i / D, d = i % D;
     float mq[kSwCluster], lq[kSwCluster], oq[kSwCluster];
+    float ms[kMaxCS], ls[kMaxCS], os[kMaxCS];
 #pragma unroll
     for (int q = 0; q < kSwCluster; ++q) {
       mq[q] = -CUDART_INF_F;
@@ -823,9 +833,24 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
         oq[q] = __ldcg(pq + d);
       }
     }
+    const float* sel = a.sel_scratch + ((size_t)(b * a.NR + (r < 0 ? 0 : r) * G + g) * kMaxCS) * (D + 3);
+#pragma unroll
+    for (int q = 0; q < kMaxCS; ++q) {
+      ms[q] = -CUDART_INF_F;
+      ls[q] = 0.f;
+      os[q] = 0.f;
+      if (q < ncs) {
+        const float* pq = sel + (size_t)q * (D + 3);
+        ms[q] = __ldcg(pq + D);
+        ls[q] = __ldcg(pq + D + 1);
+        os[q] = __ldcg(pq + d);
+      }
+    }
     float mn = -CUDART_INF_F;
 #pragma unroll
     for (int q = 0; q < kSwCluster; ++q) mn = fmaxf(mn, mq[q]);
+#pragma unroll
+    for (int q = 0; q < kMaxCS; ++q) mn = fmaxf(mn, ms[q]);
     float acc = 0.f, den = 0.f;
 #pragma unroll
     for (int q = 0; q < kSwCluster; ++q) {
@@ -833,29 +858,36 @@ __device__ __forceinline__ void sw_cta(const DecodeArgs& a, int bkv, int crank, 
       acc = fmaf(oq[q], sc, acc);
       den = fmaf(lq[q], sc, den);
     }
-    if (r < 0) {  // local head: this is the whole attention
-      T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + h * G + g) * D + d;
-      *out = from_f32<T>(acc / den);
-    } else {      // retrieval head: the select kernel adds its kept rows
-      float* sp = a.sw_part + ((size_t)bkv * G + g) * (D + 2);
-      sp[d] = acc;
-      if (d == 0) {
-        sp[D] = mn;
-        sp[D + 1] = den;
-      }
+#pragma unroll
+    for (int q = 0; q < kMaxCS; ++q) {
+      const float sc = ms[q] == -CUDART_INF_F ? 0.f : exp2f(ms[q] - mn);
+      acc = fmaf(os[q], sc, acc);
+      den = fmaf(ls[q], sc, den);
     }
+    T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + h * G + g) * D + d;
+    *out = from_f32<T>(acc / den);
+  }
+  // kept-token counts of the head's query heads: the sum over the select ranks
+  if (ncs > 0 && crank == 0 && tid < G && a.sel_count != nullptr) {
+    const float* sel = a.sel_scratch + ((size_t)(b * a.NR + r * G + tid) * kMaxCS) * (D + 3);
+    int cnt = 0;
+    for (int q = 0; q < ncs; ++q) cnt += __float_as_int(__ldcg(sel + (size_t)q * (D + 3) + D + 2));
+    a.sel_count[b * a.NR + r * G + tid] = cnt;
   }
 }
 
 // ---------------------------------------------------------------------------
 // 1. the two stream kernels
 // ---------------------------------------------------------------------------
-// score_kernel (plain grid) waits for rtp_append_kv, then lets the sink/window
-// kernel launch; sw_kernel (clusters) lets the select kernel launch at once
-// and reads the cache without a wait of its own: it starts only after every
-// score CTA has passed its wait, so the appended rows are complete.  Its
-// closing wait makes its completion imply the score kernel's, which is what
-// the select kernel's wait relies on.
+// Launch order score -> select -> sink/window.  score_kernel (plain grid)
+// waits for rtp_append_kv, then lets the select kernel launch; the select
+// kernel lets the sink/window kernel launch at once.  sw_kernel (clusters)
+// reads the cache without a wait of its own: it starts only after every score
+// CTA has passed its wait, so the appended rows are complete.  A retrieval
+// head's clusters wait for the select kernel before their merge; every CTA's
+// closing wait makes the kernel's completion imply the select kernel's (and
+// with it the score kernel's), which is what the next kernel on the stream
+// relies on.
 template <typename T, int D, int G, int IDX>
 __global__ void __launch_bounds__(kThreads, score_ctas_per_sm(IDX)) score_kernel(const __grid_constant__ DecodeArgs a) {
   extern __shared__ __align__(128) unsigned char dsm[];
@@ -1237,7 +1269,7 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   };
   // Before waiting for the scores: seq_len and this head's RoPE'd query
   // (scaled by log2(e)/sqrt(D)) from the caller's inputs.  This kernel starts
-  // only once every stream CTA has passed its wait for rtp_append_kv, so the
+  // only once every score CTA has passed its wait for rtp_append_kv, so the
   // cache rows it reads are complete.
   const int L = a.seq_len[b];
   if (tid < D / 2 && seq_ok(L, a)) {
@@ -1254,8 +1286,8 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
   if (tid == 0) mbar_init(&s_sbar, 1);
   griddep_launch();
   cluster_arrive();  // counter zeroed; every CTA of the cluster running
-  griddep_wait();    // the stream kernel (scores, chunk maxima, sink/window partials) has completed
-  if (!seq_ok(L, a)) {  // uniform over the cluster; the stream kernel flagged it
+  griddep_wait();    // the score kernel (scores, chunk maxima) has completed
+  if (!seq_ok(L, a)) {  // uniform over the cluster; the score kernel flagged it
     cluster_wait();
     return;
   }
@@ -1921,51 +1953,10 @@ __global__ void __cluster_dims__(CS, 1, 1) __launch_bounds__(kSelThreads, 2) sel
     for (int w = 0; w < kSelWarps; ++w) c += sh->cnt[w];
     sp_me[D + 2] = __int_as_float(c);
   }
-  cl.sync();  // every rank's partial and count written (the barrier orders global memory within the cluster)
-  {
-    // The head's sink/window partial plus every rank's kept-row partial, the
-    // D output elements spread over the ranks (element d on rank d mod CS),
-    // each thread loading every rank's partial at once (L2 hits).
-    const int bkv = b * a.Hkv + h;
-    const float* sp = a.sw_part + ((size_t)bkv * a.G + g) * (D + 2);
-    const float* parts = a.sel_scratch + (size_t)bh * kMaxCS * (D + 3);
-    for (int d = rank + CS * tid; d < D; d += CS * kSelThreads) {
-      float mq[CS], lq[CS], oq[CS];
-#pragma unroll
-      for (int q = 0; q < CS; ++q) {
-        const float* pq = parts + (size_t)q * (D + 3);
-        mq[q] = __ldcg(pq + D);
-        lq[q] = __ldcg(pq + D + 1);
-        oq[q] = __ldcg(pq + d);
-      }
-      const float m_sw = __ldcg(sp + D);
-      const float l_sw = __ldcg(sp + D + 1);
-      const float o_sw = __ldcg(sp + d);
-      float mn = m_sw;
-#pragma unroll
-      for (int q = 0; q < CS; ++q) mn = fmaxf(mn, mq[q]);
-      float acc = 0.f, den = 0.f;
-      if (m_sw != -CUDART_INF_F) {
-        const float sc = exp2f(m_sw - mn);
-        acc = o_sw * sc;
-        den = l_sw * sc;
-      }
-#pragma unroll
-      for (int q = 0; q < CS; ++q) {
-        const float sc = mq[q] == -CUDART_INF_F ? 0.f : exp2f(mq[q] - mn);
-        acc = fmaf(oq[q], sc, acc);
-        den = fmaf(lq[q], sc, den);
-      }
-      T* out = static_cast<T*>(a.out) + ((size_t)b * a.Hq + h * a.G + g) * D + d;
-      *out = from_f32<T>(acc / den);
-    }
-    if (rank == 0 && tid == 0 && a.sel_count) {
-      int c = 0;
-#pragma unroll
-      for (int q = 0; q < CS; ++q) c += __float_as_int(__ldcg(parts + (size_t)q * (D + 3) + D + 2));
-      a.sel_count[bh] = c;
-    }
-  }
+  // The sink/window kernel, launched after this one, merges every rank's
+  // partial with the head's sink/window partial once this grid has completed.
+  // No rank touches another's shared memory after the last cluster barrier,
+  // so the ranks leave independently.
 }
 
 // ---------------------------------------------------------------------------
@@ -1996,9 +1987,8 @@ cudaError_t launch_cluster_pdl(void (*k)(DecodeArgs), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, k, a);
 }
 
-// The two stream kernels: score CTAs (plain grid), then sink/window clusters of
-// 16 CTAs when the device can place one (non-portable size), else 8.  Set up
-// once per device under a mutex.
+// The two stream kernels: score CTAs (plain grid; part 0), and sink/window
+// clusters of kSwCluster CTAs (part 1).  Set up once per device under a mutex.
 template <typename T, int D, int G, int IDX>
 cudaError_t launch_score(const DecodeArgs& a, int n_sms, cudaStream_t st) {
   return launch_pdl(score_kernel<T, D, G, IDX>, dim3(std::min(a.n_score_ctas, score_ctas_per_sm(IDX) * n_sms)),
@@ -2006,7 +1996,7 @@ cudaError_t launch_score(const DecodeArgs& a, int n_sms, cudaStream_t st) {
 }
 
 template <typename T, int D, int G>
-cudaError_t launch_stream(DecodeArgs& a, int n_bkv, int idx, cudaStream_t st) {
+cudaError_t launch_stream(DecodeArgs& a, int n_bkv, int idx, int part, cudaStream_t st) {
   static std::mutex s_mu;
   static std::atomic<int> s_cs[64];  // chosen cluster size; 0 = not set up yet
   static std::atomic<int> s_sms[64];
@@ -2023,32 +2013,29 @@ cudaError_t launch_stream(DecodeArgs& a, int n_bkv, int idx, cudaStream_t st) {
       cudaFuncSetAttribute(score_kernel<T, D, G, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, score_smem(8));
       cudaFuncSetAttribute(score_kernel<T, D, G, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, score_smem(16));
       cudaFuncSetAttribute(score_kernel<T, D, G, 32>, cudaFuncAttributeMaxDynamicSharedMemorySize, score_smem(32));
-      cudaFuncSetAttribute(sw_kernel<T, D, G>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       cudaFuncSetAttribute(sw_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kStreamSmem);
-      cudaLaunchConfig_t cfg = {};
-      cfg.gridDim = dim3(kSwCluster);
-      cfg.blockDim = dim3(kThreads);
-      cfg.dynamicSmemBytes = kStreamSmem;
-      cudaLaunchAttribute attr[1];
-      attr[0].id = cudaLaunchAttributeClusterDimension;
-      attr[0].val.clusterDim.x = kSwCluster;
-      attr[0].val.clusterDim.y = 1;
-      attr[0].val.clusterDim.z = 1;
-      cfg.attrs = attr;
-      cfg.numAttrs = 1;
-      int n = 0;
-      if (cudaOccupancyMaxActiveClusters(&n, sw_kernel<T, D, G>, &cfg) != cudaSuccess) n = 0;
-      cudaGetLastError();  // clear a refused query
+      // every decode kernel asks for the largest shared-memory carveout, so
+      // their CTAs can share an SM
+      cudaFuncSetAttribute(sw_kernel<T, D, G>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+      cudaFuncSetAttribute(score_kernel<T, D, G, 4>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+      cudaFuncSetAttribute(score_kernel<T, D, G, 8>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+      cudaFuncSetAttribute(score_kernel<T, D, G, 16>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+      cudaFuncSetAttribute(score_kernel<T, D, G, 32>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
       int sms = 0;
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) sms = 148;
       cudaGetLastError();
       s_sms[dev].store(sms, std::memory_order_relaxed);
-      cs = n > 0 ? kSwCluster : 8;
+      cs = kSwCluster;
       s_cs[dev].store(cs, std::memory_order_release);
     }
   }
   const int n_sms = s_sms[dev].load(std::memory_order_relaxed);
-  if (a.n_score_ctas > 0) {
+  if (part == 0) {
     trace_begin(RTP_STAGE_DECODE_SCORE, st);
     switch (idx) {
       case 4: e = launch_score<T, D, G, 4>(a, n_sms, st); break;
@@ -2057,7 +2044,7 @@ cudaError_t launch_stream(DecodeArgs& a, int n_bkv, int idx, cudaStream_t st) {
       default: e = launch_score<T, D, G, 16>(a, n_sms, st); break;
     }
     trace_end(RTP_STAGE_DECODE_SCORE, st);
-    if (e != cudaSuccess) return e;
+    return e;
   }
   trace_begin(RTP_STAGE_DECODE_LOCAL, st);
   e = launch_cluster_pdl(sw_kernel<T, D, G>, dim3(n_bkv * cs), dim3(kThreads), kStreamSmem, cs, st, a);
@@ -2066,22 +2053,23 @@ cudaError_t launch_stream(DecodeArgs& a, int n_bkv, int idx, cudaStream_t st) {
 }
 
 template <typename T, int D>
-cudaError_t launch_stream_d(DecodeArgs& a, int n_bkv, int idx, cudaStream_t st) {
+cudaError_t launch_stream_d(DecodeArgs& a, int n_bkv, int idx, int part, cudaStream_t st) {
   switch (a.G) {
-    case 1: return launch_stream<T, D, 1>(a, n_bkv, idx, st);
-    case 2: return launch_stream<T, D, 2>(a, n_bkv, idx, st);
-    case 4: return launch_stream<T, D, 4>(a, n_bkv, idx, st);
-    default: return launch_stream<T, D, 8>(a, n_bkv, idx, st);
+    case 1: return launch_stream<T, D, 1>(a, n_bkv, idx, part, st);
+    case 2: return launch_stream<T, D, 2>(a, n_bkv, idx, part, st);
+    case 4: return launch_stream<T, D, 4>(a, n_bkv, idx, part, st);
+    default: return launch_stream<T, D, 8>(a, n_bkv, idx, part, st);
   }
 }
 
-cudaError_t launch_stream_any(const Shape& sh, DecodeArgs& a, cudaStream_t st) {
+// part 0: the score kernel; part 1: the sink/window clusters
+cudaError_t launch_stream_any(const Shape& sh, DecodeArgs& a, int part, cudaStream_t st) {
   const int n_bkv = sh.B * sh.Hkv;
   if (sh.dtype == RTP_BF16)
-    return sh.D == 128 ? launch_stream_d<__nv_bfloat16, 128>(a, n_bkv, sh.idx, st)
-                       : launch_stream_d<__nv_bfloat16, 64>(a, n_bkv, sh.idx, st);
-  return sh.D == 128 ? launch_stream_d<float, 128>(a, n_bkv, sh.idx, st)
-                     : launch_stream_d<float, 64>(a, n_bkv, sh.idx, st);
+    return sh.D == 128 ? launch_stream_d<__nv_bfloat16, 128>(a, n_bkv, sh.idx, part, st)
+                       : launch_stream_d<__nv_bfloat16, 64>(a, n_bkv, sh.idx, part, st);
+  return sh.D == 128 ? launch_stream_d<float, 128>(a, n_bkv, sh.idx, part, st)
+                     : launch_stream_d<float, 64>(a, n_bkv, sh.idx, part, st);
 }
 
 // Select kernel with 16-CTA clusters when the device can keep all of this
@@ -2107,6 +2095,10 @@ cudaError_t launch_select(DecodeArgs& a, int n_clusters, cudaStream_t st) {
       cudaFuncSetAttribute(select_kernel<T, D, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<8>::kSmem);
       cudaFuncSetAttribute(select_kernel<T, D, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SelCfg<16>::kSmem);
       cudaFuncSetAttribute(select_kernel<T, D, 16>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      cudaFuncSetAttribute(select_kernel<T, D, 8>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
+      cudaFuncSetAttribute(select_kernel<T, D, 16>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                           (int)cudaSharedmemCarveoutMaxShared);
       cudaLaunchConfig_t cfg = {};
       cfg.gridDim = dim3(16, 1);
       cfg.blockDim = dim3(kSelThreads);
@@ -2158,7 +2150,6 @@ DecodeLayout decode_layout(const Shape& sh) {
   l.cmax = off;       off = align256(off + NRt * l.nch_score_max * sizeof(float));
   l.mask = off;       off = align256(off + NRt * words * sizeof(uint32_t));  // bitmask when the caller passes none
   l.cand = off;       off = align256(off + NRt * lstride * sizeof(uint2));
-  l.sw_part = off;    off = align256(off + (size_t)sh.B * sh.Hkv * sh.G * (sh.D + 2) * sizeof(float));
   l.sw_scratch = off; off = align256(off + (size_t)sh.B * sh.Hkv * kSwCluster * sh.G * (sh.D + 2) * sizeof(float));
   l.sel_scratch = off; off = align256(off + NRt * kMaxCS * (sh.D + 3) * sizeof(float));
   l.total = off;
@@ -2184,7 +2175,6 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   a.mask = sel_bitmask ? sel_bitmask : reinterpret_cast<uint32_t*>(w + lay.mask);
   a.want_mask = sel_bitmask != nullptr;
   a.cand = reinterpret_cast<uint2*>(w + lay.cand);
-  a.sw_part = reinterpret_cast<float*>(w + lay.sw_part);
   a.sw_scratch = reinterpret_cast<float*>(w + lay.sw_scratch);
   a.sel_scratch = reinterpret_cast<float*>(w + lay.sel_scratch);
   a.nch_score_max = lay.nch_score_max;
@@ -2204,12 +2194,17 @@ int launch_decode(const Shape& sh, const rtp_cache* cache, const void* q_pre, co
   const int chunk = score_chunk(sh.esize);
   a.n_score_ctas = sh.R > 0 ? sh.B * sh.R * ((Lh + chunk - 1) / chunk) : 0;
 
-  cudaError_t e = launch_stream_any(sh, a, st);
+  // score -> select -> sink/window: the select clusters start as soon as the
+  // scores are complete, the sink/window clusters stream beside them and merge
+  // the select's partials at their end
+  cudaError_t e = cudaSuccess;
+  if (a.n_score_ctas > 0) e = launch_stream_any(sh, a, 0, st);
   if (e == cudaSuccess && sh.R > 0) {
     trace_begin(RTP_STAGE_DECODE_SELECT, st);
     e = launch_select_any(sh, a, sh.B * sh.NR, st);
     trace_end(RTP_STAGE_DECODE_SELECT, st);
   }
+  if (e == cudaSuccess) e = launch_stream_any(sh, a, 1, st);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) {
     set_error(std::string("decode launch: ") + cudaGetErrorString(e));

@@ -58,7 +58,7 @@ int make_shape(const rtp_layer_cfg* cfg, Shape* sh);
 
 // Decode scratch layout (byte offsets into the workspace).
 struct DecodeLayout {
-  size_t logits, cmax, mask, cand, sw_part, sw_scratch, sel_scratch, total;
+  size_t logits, cmax, mask, cand, sw_scratch, sel_scratch, total;
   int nch_score_max;
 };
 DecodeLayout decode_layout(const Shape& sh);
