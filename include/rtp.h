@@ -196,9 +196,9 @@ int rtp_append_kv(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* 
  * on the stream (only the cache reads wait): they must not be written by a
  * kernel that may still be running when this call's kernels start, such as an
  * earlier kernel launched with programmatic dependent launch.
- * Two bounded waits inside the call (for the step's indexer scores and for
- * each head's sink/window partial) give up after about 0.4 s; the call's output
- * is then invalid and RTP_DEV_TIMEOUT is set.
+ * The bounded waits inside the call (on the asynchronous copies of the
+ * indexer keys, of the scores and of the sink/window rows) give up after about
+ * 0.4 s; the call's output is then invalid and RTP_DEV_TIMEOUT is set.
  */
 int rtp_decode_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const void* q_pre,
                     const int* seq_len, int max_seq_len, const float* w_q, void* out,
@@ -301,8 +301,8 @@ int rtp_prefill_attn(const rtp_layer_cfg* cfg, const rtp_cache* cache, const voi
 typedef enum rtp_stage {
   RTP_STAGE_APPEND = 0,         /* rtp_append_kv: RoPE + cache + indexer-key store */
   RTP_STAGE_DECODE_SCORE = 1,   /* decode: indexer scores over the d-dim key cache */
-  RTP_STAGE_DECODE_SELECT = 2,  /* decode: exact top-p selection, bitmask, kept-row attention, merge */
-  RTP_STAGE_DECODE_LOCAL = 3,   /* decode: sink/window attention of every KV head (overlaps the scores) */
+  RTP_STAGE_DECODE_SELECT = 2,  /* decode: exact top-p selection, bitmask, kept-row attention */
+  RTP_STAGE_DECODE_LOCAL = 3,   /* decode: sink/window attention of every KV head (beside the selection), final merge */
   RTP_STAGE_PREFILL_INDEX = 4,  /* prefill: per-row exact top-p selection */
   RTP_STAGE_PREFILL_ATTN = 5,   /* prefill: masked causal attention */
   RTP_STAGE_COUNT = 6
