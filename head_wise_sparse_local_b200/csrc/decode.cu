@@ -381,12 +381,13 @@ __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* d
 // ---------------------------------------------------------------------------
 // 1b. sink/window CTA: rank `crank` of the cluster of (sequence b, KV head h)
 // ---------------------------------------------------------------------------
-// The CTA's rows arrive in shared memory by bulk asynchronous copies, one per
-// contiguous run of cache rows (the sinks, the window, and a second window run
-// where a ring wraps), in stages of kStreamSmem / 2 bytes (K and V), two stages
-// in flight.  A half-warp then owns a row: lane (half, c) reads dims
-// [c*EPL, c*EPL + EPL) of the row's key and value, so a warp covers two rows.
-// Scores of the G query heads are reduced over the half-warp by shuffles;
+// The CTA's rows (the sinks, then the window, which wraps once in a ring)
+// arrive in shared memory by cp.async, 16 bytes per thread, in stages of at
+// most kStreamSmem / 2 bytes (K and V), two stages in flight; a bf16 row is
+// padded by 16 bytes there.  bf16 layers run the tensor-core tiles below.
+// fp32 layers: a half-warp owns a row, lane (half, c) reading dims
+// [c*EPL, c*EPL + EPL) of the row's key and value, so a warp covers two rows;
+// scores of the G query heads are reduced over the half-warp by shuffles, and
 // every lane keeps the running (max, sum) of its half and the weighted value
 // sum of its own dims.
 template <typename T, int D>
