@@ -291,18 +291,25 @@ __device__ __forceinline__ void score_ctas(const DecodeArgs& a, unsigned char* d
         // this lane's columns 2 t4, 2 t4 + 1 (query heads when < G)
         float mxa = -CUDART_INF_F, mxb = -CUDART_INF_F;
         const bool ca = 2 * t4 < G, cb = 2 * t4 + 1 < G;
+        // The warp's tiles are warp, warp + kWarps, ...: all of their products
+        // are issued first (independent mma chains overlap their latency),
+        // then the scores are stored.  A tile past the chunk's keys reads
+        // stale shared memory (inside the buffer) whose scores are dropped.
         constexpr int kTiles = kChunk / 16;
-        for (int tt = warp; tt < kTiles; tt += kWarps) {
-          const int kb = tt * 16;  // first key of the tile (chunk-local)
-          if (j0 + kb >= j1) break;  // warp-uniform
-          float cc[4];
-          mm.scores(kbuf + (size_t)kb * KB, lane, cc);
+        constexpr int kTPW = kTiles / kWarps;  // tiles per warp
+        static_assert(kTiles % kWarps == 0, "whole tiles per warp");
+        float cc[kTPW][4];
+#pragma unroll
+        for (int u = 0; u < kTPW; ++u) mm.scores(kbuf + (size_t)(warp + u * kWarps) * 16 * KB, lane, cc[u]);
+#pragma unroll
+        for (int u = 0; u < kTPW; ++u) {
+          const int kb = (warp + u * kWarps) * 16;  // first key of the tile (chunk-local)
 #pragma unroll
           for (int x = 0; x < 2; ++x) {
             const int j = j0 + kb + gq + 8 * x;
             if (j >= j1) continue;
-            const float sa = cc[2 * x] * kScale + 0.0f;  // +0 turns -0 into +0
-            const float sb = cc[2 * x + 1] * kScale + 0.0f;
+            const float sa = cc[u][2 * x] * kScale + 0.0f;  // +0 turns -0 into +0
+            const float sb = cc[u][2 * x + 1] * kScale + 0.0f;
             if (ca) {
               lg[(size_t)(2 * t4) * a.lstride + j] = sa;
               mxa = fmaxf(mxa, sa);
